@@ -1,0 +1,69 @@
+// common.cuh -- types and small device helpers shared by the DFlash kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+typedef __nv_bfloat16 bf16;
+
+namespace dfl {
+
+// Per-row metadata of one forward pass.
+//  target / drafter block rows: seq = slot, pos = absolute position,
+//    nk = number of visible keys (causal: pos+1; drafter block: p+B),
+//    aux = destination row in the tap buffer (target rows).
+//  drafter context rows: seq, pos = context position, aux = 1 if the row is a
+//    committed position whose context K/V must be written, else 0.
+struct RowMeta {
+    int32_t seq, pos, nk, aux;
+};
+
+// Device-resident state of one sequence slot.
+struct SeqState {
+    int32_t len;        // valid target KV positions == position of the anchor
+    int32_t anchor;     // last committed token (input of the next block's row 0)
+    int32_t ctx_len;    // valid drafter context positions
+    int32_t pend_pos0;  // first position of context rows still to be injected
+    int32_t pend_n;     // number of such rows (their taps sit in the pending tap rows of the slot)
+    int32_t n_out;      // tokens emitted after the prompt (the first comes from prefill)
+    int32_t max_new;    // stop after this many tokens
+    int32_t done;
+};
+
+// Accumulated decode statistics (device side).
+struct DevStats {
+    unsigned long long iterations;          // sequence-iterations
+    unsigned long long tokens;              // tokens emitted by verify/commit
+    unsigned long long hist[16];
+    int32_t n_done;                         // sequences that reached max_new
+    int32_t status;                         // nonzero: non-finite logits seen
+};
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// (value, index) max with the lowest index winning exact ties.
+__device__ __forceinline__ void argmax_merge(float &v, int &i, float v2, int i2) {
+    if (v2 > v || (v2 == v && i2 < i)) { v = v2; i = i2; }
+}
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+
+}  // namespace dfl

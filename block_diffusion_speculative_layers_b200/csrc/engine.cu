@@ -1,0 +1,1060 @@
+// engine.cu -- the dflash C ABI: configuration checks, arena layout, weight
+// slots and the orchestration of prefill, draft, verify+commit and whole
+// generations.  Every step of the path runs in the kernels of this library;
+// the host only launches them and checks arguments.
+//
+// The decode iteration follows the DFlash pages (by title and section):
+//  * "DFlash: Decodificação Especulativa com Blocos em Paralelo ..." (iaemfoco):
+//    "O que o DFlash faz de diferente" -- one drafter pass proposes the whole
+//    block, one target pass verifies it; "O alvo sabe mais" -- hidden states
+//    of several target layers are fused into a context vector and injected
+//    into the Key/Value projections of every drafter layer (persisting in the
+//    drafter KV cache); "Decodificação especulativa tradicional" -- lossless.
+//  * "DFlash e Spec V2 revolucionam a speculative decoding" (ceviu): host-device
+//    synchronisation kept to the minimum -> the whole iteration is enqueued
+//    without host round trips; generate() polls a done counter once per
+//    iteration, one iteration behind.
+#include <algorithm>
+#include <chrono>
+#include <climits>
+#include <cstdio>
+#include <cstring>
+#include <thread>
+
+#include "engine.h"
+#include "gemm_tc.h"
+#include "attn_mma.h"
+
+namespace dfl {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static int elem_size(int dtype) { return dtype == DFLASH_BF16 ? 2 : 4; }
+
+static bool check_model(const dflash_model_cfg &m, std::string &why) {
+    if (m.n_layers < 1 || m.hidden < 32 || m.n_q_heads < 1 || m.n_kv_heads < 1 || m.vocab < 2) {
+        why = "model dimensions must be positive";
+        return false;
+    }
+    if (m.n_q_heads % m.n_kv_heads) { why = "n_q_heads must be a multiple of n_kv_heads"; return false; }
+    if (m.head_dim != 64 && m.head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
+    if (m.hidden % 64) { why = "hidden must be a multiple of 64"; return false; }
+    if (m.n_experts < 0 || m.n_experts > 256) { why = "n_experts must be in [0, 256]"; return false; }
+    if (m.n_experts > 0) {
+        if (m.top_k < 1 || m.top_k > m.n_experts || m.top_k > 32 || m.expert_ffn < 8 || m.expert_ffn % 8) {
+            why = "bad MoE dims (top_k in [1, min(E,32)], expert_ffn multiple of 8)";
+            return false;
+        }
+    } else if (m.ffn < 8 || m.ffn % 8) {
+        why = "ffn must be a positive multiple of 8";
+        return false;
+    }
+    if (!(m.rms_eps >= 0.0) || !(m.rope_theta > 1.0)) { why = "bad rms_eps / rope_theta"; return false; }
+    return true;
+}
+
+static bool check_config(const dflash_config &c, std::string &why) {
+    if (!check_model(c.target, why)) { why = "target: " + why; return false; }
+    if (!check_model(c.drafter, why)) { why = "drafter: " + why; return false; }
+    if (c.drafter.n_experts != 0) { why = "the drafter must be dense"; return false; }
+    if (c.drafter.hidden != c.target.hidden || c.drafter.vocab != c.target.vocab) {
+        why = "drafter hidden/vocab must equal the target's (shared embedding and head)";
+        return false;
+    }
+    if (c.block_size < 1 || c.block_size > DFLASH_MAX_BLOCK) { why = "block_size must be in [1, 16]"; return false; }
+    if (c.n_taps < 1 || c.n_taps > DFLASH_MAX_TAPS) { why = "n_taps must be in [1, 8]"; return false; }
+    for (int i = 0; i < c.n_taps; ++i)
+        if (c.tap_layers[i] < 0 || c.tap_layers[i] >= c.target.n_layers) { why = "tap layer out of range"; return false; }
+    if (c.mask_token_id < 0 || c.mask_token_id >= c.target.vocab) { why = "mask_token_id out of vocab"; return false; }
+    if (c.max_batch < 1 || c.max_batch > 64) { why = "max_batch must be in [1, 64]"; return false; }
+    if (c.max_len < c.block_size + 1 || c.max_len > (1 << 20)) { why = "max_len out of range"; return false; }
+    if (c.prefill_chunk < 0 || c.prefill_chunk > 8192) { why = "prefill_chunk must be in [0, 8192]"; return false; }
+    if (c.dtype != DFLASH_FP32 && c.dtype != DFLASH_BF16) { why = "dtype must be DFLASH_FP32 or DFLASH_BF16"; return false; }
+    return true;
+}
+
+static void add_slot(Layout &L, const std::string &name, int ndim, int64_t d0, int64_t d1, int64_t d2, int dtype) {
+    WeightSlot s;
+    s.name = name;
+    s.ndim = ndim;
+    s.shape[0] = d0;
+    s.shape[1] = d1;
+    s.shape[2] = d2;
+    s.numel = (size_t)d0 * (ndim > 1 ? d1 : 1) * (ndim > 2 ? d2 : 1);
+    s.dtype = dtype;
+    L.weight_bytes = align_up(L.weight_bytes, 256);
+    s.offset = L.weight_bytes;
+    L.weight_bytes += s.numel * elem_size(dtype);
+    L.slots.push_back(s);
+}
+
+static void add_model_slots(Layout &L, const char *prefix, const dflash_model_cfg &m, int dt) {
+    const int64_t H = m.hidden, qd = (int64_t)m.n_q_heads * m.head_dim, kd = (int64_t)m.n_kv_heads * m.head_dim;
+    for (int l = 0; l < m.n_layers; ++l) {
+        std::string p = std::string(prefix) + ".L" + std::to_string(l) + ".";
+        add_slot(L, p + "attn_norm", 1, H, 0, 0, DFLASH_FP32);
+        add_slot(L, p + "wqkv", 2, qd + 2 * kd, H, 0, dt);
+        add_slot(L, p + "wo", 2, H, qd, 0, dt);
+        add_slot(L, p + "ffn_norm", 1, H, 0, 0, DFLASH_FP32);
+        if (m.n_experts > 0) {
+            add_slot(L, p + "w_router", 2, m.n_experts, H, 0, dt);
+            add_slot(L, p + "we_gate_up", 3, m.n_experts, 2 * (int64_t)m.expert_ffn, H, dt);
+            add_slot(L, p + "we_down", 3, m.n_experts, H, m.expert_ffn, dt);
+        } else {
+            add_slot(L, p + "w_gate_up", 2, 2 * (int64_t)m.ffn, H, 0, dt);
+            add_slot(L, p + "w_down", 2, H, m.ffn, 0, dt);
+        }
+    }
+    add_slot(L, std::string(prefix) + ".final_norm", 1, H, 0, 0, DFLASH_FP32);
+}
+
+static Layout make_layout(const dflash_config &c) {
+    Layout L;
+    const int dt = c.dtype, es = elem_size(dt);
+    const dflash_model_cfg &t = c.target, &d = c.drafter;
+    add_slot(L, "embed", 2, t.vocab, t.hidden, 0, dt);
+    add_slot(L, "lm_head", 2, t.vocab, t.hidden, 0, dt);
+    add_model_slots(L, "target", t, dt);
+    add_model_slots(L, "drafter", d, dt);
+    add_slot(L, "fuse.w_fc", 2, d.hidden, (int64_t)c.n_taps * t.hidden, 0, dt);
+    add_slot(L, "fuse.norm", 1, d.hidden, 0, 0, DFLASH_FP32);
+    L.weight_bytes = align_up(L.weight_bytes, 256);
+
+    const int B = c.block_size, nb = c.max_batch, H = t.hidden;
+    L.R_dec = nb * B;
+    L.C = c.prefill_chunk > 0 ? c.prefill_chunk : 1024;
+    L.R_max = std::max(2 * L.R_dec, L.C);
+    const int qd_t = t.n_q_heads * t.head_dim, kd_t = t.n_kv_heads * t.head_dim;
+    const int qd_d = d.n_q_heads * d.head_dim, kd_d = d.n_kv_heads * d.head_dim;
+    const int F_t = t.n_experts > 0 ? t.expert_ffn : t.ffn;
+    int ycols = std::max({qd_t + 2 * kd_t, qd_d + 2 * kd_d, 2 * d.ffn, H});
+    if (t.n_experts == 0) ycols = std::max(ycols, 2 * t.ffn);
+    else ycols = std::max(ycols, t.n_experts);
+    L.Y_cols = ycols;
+    const int qmax = std::max(qd_t, qd_d);
+    const int fmax = std::max(F_t, d.ffn);
+    const int TK = c.n_taps * H;
+    const size_t R = L.R_max;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { o = align_up(o, 256); size_t r = o; o += std::max<size_t>(bytes, 16); return r; };
+    L.x = take(R * H * 4);
+    L.xn = take(R * H * es);
+    L.dq_in = take((size_t)2 * L.R_dec * H * es);
+    L.Y = take(R * (size_t)ycols * 4);
+    L.q = take(R * qmax * es);
+    L.ao = take(R * qmax * es);
+    const size_t hrows = t.n_experts > 0 ? R * (size_t)t.top_k : R;
+    L.h = take(hrows * fmax * es);
+    L.taps_dec = take((size_t)L.R_dec * TK * es);
+    L.taps_gather = take((size_t)L.R_dec * TK * es);
+    L.taps_pre = take((size_t)L.C * TK * es);
+    L.cbuf = take((size_t)L.C * H * es);
+    L.logits = take((size_t)L.R_dec * t.vocab * 4);
+    L.plogits = take((size_t)t.vocab * 4);
+    L.g = take((size_t)L.R_dec * 4);
+    L.drafts = take((size_t)nb * B * 4);
+    L.accept = take((size_t)nb * 4);
+    L.committed = take((size_t)nb * B * 4);
+    L.new_len = take((size_t)nb * 4);
+    L.st = take((size_t)nb * sizeof(SeqState));
+    L.active = take((size_t)nb * 4);
+    L.meta = take(R * sizeof(RowMeta));
+    L.ctx_meta = take((size_t)L.R_dec * sizeof(RowMeta));
+    L.ctx_meta_pre = take((size_t)L.C * sizeof(RowMeta));
+    L.rope_t = take((size_t)c.max_len * (t.head_dim / 2) * sizeof(float2));
+    L.rope_d = take((size_t)c.max_len * (d.head_dim / 2) * sizeof(float2));
+    const size_t kv_t = (size_t)t.n_layers * nb * t.n_kv_heads * c.max_len * t.head_dim * es;
+    const size_t kv_d = (size_t)d.n_layers * nb * d.n_kv_heads * c.max_len * d.head_dim * es;
+    L.tk = take(kv_t);
+    L.tv = take(kv_t);
+    L.dk = take(kv_d);
+    L.dv = take(kv_d);
+    L.script = take((size_t)nb * c.max_len * 4);
+    L.out_tok = take((size_t)nb * c.max_len * 4);
+    L.tokens = take((size_t)c.max_len * 4);
+    L.stats = take(sizeof(DevStats));
+    L.first_tok = take(16);
+    const size_t mrows = t.n_experts > 0 ? R * (size_t)t.top_k : 1;
+    L.moe_sel = take(mrows * 4);
+    L.moe_wt = take(mrows * 4);
+    L.moe_part = take(t.n_experts > 0 ? mrows * H * 4 : 16);
+    // split-K workspace and tile semaphores of the tensor-core GEMM
+    L.ws_floats = gemm_tc_workspace_floats(L.R_max, std::max(ycols, t.vocab > 0 ? H : H));
+    L.gemm_ws = take((size_t)L.ws_floats * 4);
+    L.n_sem = gemm_tc_semaphores();
+    L.gemm_sem = take((size_t)L.n_sem * 4);
+    (void)kd_t;
+    (void)kd_d;
+    L.state_bytes = align_up(o, 256);
+    return L;
+}
+
+// ------------------------------------------------------------------------
+// engine
+// ------------------------------------------------------------------------
+
+template <typename T>
+class Engine : public EngineBase {
+  public:
+    dflash_config c;
+    const Layout &L;
+    cudaStream_t s;
+    char *W, *S;
+    // weights
+    const T *embed, *lm_head, *w_fc;
+    const float *fc_norm, *t_final, *d_final;
+    std::vector<LayerW> tl, dl;
+    // state
+    float *x, *Y, *logits, *plogits, *moe_wt, *moe_part;
+    T *xn, *dq_in, *q, *ao, *h, *taps_dec, *taps_gather, *taps_pre, *cbuf, *tk, *tv, *dk, *dv;
+    int *g, *drafts, *accept, *committed, *new_len, *active, *script, *out_tok, *tokens, *first_tok, *moe_sel;
+    SeqState *st;
+    RowMeta *meta, *ctx_meta, *ctx_meta_pre;
+    float2 *rope_t, *rope_d;
+    DevStats *stats;
+    float *gemm_ws;
+    int *gemm_sem;
+    GemmTC<T> tc;
+    // host mirrors
+    std::vector<int> h_len, h_prefilled;
+    std::vector<int> last_draft;
+    int last_logits_rows[3] = {0, 0, 0};
+    int *pinned = nullptr;  // small pinned host buffer for the done counter
+    cudaEvent_t ev_a = nullptr, ev_b = nullptr;
+
+    Engine(const dflash_config &cfg, const Layout &lay, char *warena, char *sarena, cudaStream_t stream)
+        : c(cfg), L(lay), s(stream), W(warena), S(sarena) {}
+
+    template <typename P>
+    P *sp(size_t off) { return reinterpret_cast<P *>(S + off); }
+
+    const void *wslot(const std::unordered_map<std::string, int> &by, const std::string &n) {
+        return W + L.slots[by.at(n)].offset;
+    }
+
+    dflash_status init(const std::unordered_map<std::string, int> &by) {
+        embed = (const T *)wslot(by, "embed");
+        lm_head = (const T *)wslot(by, "lm_head");
+        w_fc = (const T *)wslot(by, "fuse.w_fc");
+        fc_norm = (const float *)wslot(by, "fuse.norm");
+        t_final = (const float *)wslot(by, "target.final_norm");
+        d_final = (const float *)wslot(by, "drafter.final_norm");
+        auto fill = [&](const char *pre, const dflash_model_cfg &m, std::vector<LayerW> &v) {
+            v.resize(m.n_layers);
+            for (int l = 0; l < m.n_layers; ++l) {
+                std::string p = std::string(pre) + ".L" + std::to_string(l) + ".";
+                LayerW &w = v[l];
+                w.attn_norm = (const float *)wslot(by, p + "attn_norm");
+                w.ffn_norm = (const float *)wslot(by, p + "ffn_norm");
+                w.wqkv = wslot(by, p + "wqkv");
+                w.wo = wslot(by, p + "wo");
+                if (m.n_experts > 0) {
+                    w.w_router = wslot(by, p + "w_router");
+                    w.we_gate_up = wslot(by, p + "we_gate_up");
+                    w.we_down = wslot(by, p + "we_down");
+                } else {
+                    w.w_gate_up = wslot(by, p + "w_gate_up");
+                    w.w_down = wslot(by, p + "w_down");
+                }
+            }
+        };
+        fill("target", c.target, tl);
+        fill("drafter", c.drafter, dl);
+        x = sp<float>(L.x);
+        Y = sp<float>(L.Y);
+        logits = sp<float>(L.logits);
+        plogits = sp<float>(L.plogits);
+        moe_wt = sp<float>(L.moe_wt);
+        moe_part = sp<float>(L.moe_part);
+        xn = sp<T>(L.xn);
+        dq_in = sp<T>(L.dq_in);
+        q = sp<T>(L.q);
+        ao = sp<T>(L.ao);
+        h = sp<T>(L.h);
+        taps_dec = sp<T>(L.taps_dec);
+        taps_gather = sp<T>(L.taps_gather);
+        taps_pre = sp<T>(L.taps_pre);
+        cbuf = sp<T>(L.cbuf);
+        tk = sp<T>(L.tk);
+        tv = sp<T>(L.tv);
+        dk = sp<T>(L.dk);
+        dv = sp<T>(L.dv);
+        g = sp<int>(L.g);
+        drafts = sp<int>(L.drafts);
+        accept = sp<int>(L.accept);
+        committed = sp<int>(L.committed);
+        new_len = sp<int>(L.new_len);
+        active = sp<int>(L.active);
+        script = sp<int>(L.script);
+        out_tok = sp<int>(L.out_tok);
+        tokens = sp<int>(L.tokens);
+        first_tok = sp<int>(L.first_tok);
+        moe_sel = sp<int>(L.moe_sel);
+        st = sp<SeqState>(L.st);
+        meta = sp<RowMeta>(L.meta);
+        ctx_meta = sp<RowMeta>(L.ctx_meta);
+        ctx_meta_pre = sp<RowMeta>(L.ctx_meta_pre);
+        rope_t = sp<float2>(L.rope_t);
+        rope_d = sp<float2>(L.rope_d);
+        stats = sp<DevStats>(L.stats);
+        gemm_ws = sp<float>(L.gemm_ws);
+        gemm_sem = sp<int>(L.gemm_sem);
+        h_len.assign(c.max_batch, 0);
+        h_prefilled.assign(c.max_batch, 0);
+        // zero the whole state arena once: stale taps / KV never hold NaN bit patterns
+        if (cudaMemsetAsync(S, 0, L.state_bytes, s) != cudaSuccess) return fail_cuda("memset state");
+        launch_rope_table(rope_t, c.max_len, c.target.head_dim, c.target.rope_theta, s);
+        launch_rope_table(rope_d, c.max_len, c.drafter.head_dim, c.drafter.rope_theta, s);
+        if (cudaMallocHost((void **)&pinned, 64) != cudaSuccess) return fail_cuda("pinned host buffer");
+        if (cudaEventCreateWithFlags(&ev_a, cudaEventDisableTiming) != cudaSuccess) return fail_cuda("event");
+        if (cudaEventCreateWithFlags(&ev_b, cudaEventDisableTiming) != cudaSuccess) return fail_cuda("event");
+        if (tc.init(gemm_ws, L.ws_floats, gemm_sem, L.n_sem) != 0) {
+            err = "tensor-core GEMM set-up failed: " + tc.err;
+            return DFLASH_ECUDA;
+        }
+        return check("create");
+    }
+
+    ~Engine() override {
+        if (pinned) cudaFreeHost(pinned);
+        if (ev_a) cudaEventDestroy(ev_a);
+        if (ev_b) cudaEventDestroy(ev_b);
+    }
+
+    dflash_status fail_cuda(const char *what) {
+        cudaError_t e = cudaGetLastError();
+        err = std::string(what) + ": " + cudaGetErrorString(e);
+        return DFLASH_ECUDA;
+    }
+
+    dflash_status check(const char *what) {
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) {
+            err = std::string(what) + ": " + cudaGetErrorString(e);
+            return DFLASH_ECUDA;
+        }
+        return DFLASH_OK;
+    }
+
+    dflash_status sync(const char *what) {
+        if (cudaEventRecord(ev_a, s) != cudaSuccess) return fail_cuda(what);
+        const int tmo = c.timeout_ms > 0 ? c.timeout_ms : 600000;
+        auto t0 = std::chrono::steady_clock::now();
+        while (true) {
+            cudaError_t e = cudaEventQuery(ev_a);
+            if (e == cudaSuccess) break;
+            if (e != cudaErrorNotReady) {
+                err = std::string(what) + ": " + cudaGetErrorString(e);
+                return DFLASH_ECUDA;
+            }
+            auto dt = std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0);
+            if (dt.count() > tmo) {
+                err = std::string(what) + ": stream did not finish within the timeout";
+                return DFLASH_ETIMEOUT;
+            }
+            std::this_thread::sleep_for(std::chrono::microseconds(20));
+        }
+        return check(what);
+    }
+
+    // ---- projections ----
+    size_t kv_layer_elems(const dflash_model_cfg &m) const {
+        return (size_t)c.max_batch * m.n_kv_heads * c.max_len * m.head_dim;
+    }
+
+    void gemm(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e) {
+        if (M <= 0) return;
+        if (tc.supports(M, N, K)) {
+            tc.run(X, ldx, M, (const T *)Wt, N, K, e, s);
+            return;
+        }
+        // CUDA-core path (fp32 models): GEMM into fp32 Y, then the epilogue.
+        float *Yo = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.Y : Y;
+        const int ldy = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.ldy : N;
+        launch_gemm_simt<T>(X, ldx, M, (const T *)Wt, K, N, K, Yo, ldy, s);
+        switch (e.kind) {
+            case EPI_QKV:
+                launch_qkv_epilogue<T>(Y, N, e.col0, e.R_blk, M, e.meta, e.ctx_meta, e.nq, e.nkv, e.hd, e.rope,
+                                       e.q_out, e.kc, e.vc, e.max_len, s);
+                break;
+            case EPI_RESID:
+                launch_residual<T>(e.x, Y, N, N, M, e.taps, e.meta, s);
+                break;
+            case EPI_SWIGLU:
+                launch_swiglu<T>(Y, N, e.F, M, e.h, e.F, s);
+                break;
+            default:
+                break;
+        }
+    }
+
+    void attention(const T *qq, const T *kc, const T *vc, const RowMeta *mt, int R, const dflash_model_cfg &m,
+                   T *out) {
+        const int qd = m.n_q_heads * m.head_dim;
+        if (attn_mma_supported<T>(m.head_dim)) {
+            launch_attention_mma<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out,
+                                    qd, s);
+            return;
+        }
+        launch_attention_simt<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out,
+                                 qd, s);
+    }
+
+    // one pre-norm decoder layer of the target over R rows in x (meta)
+    void target_layer(int l, int R, const RowMeta *mt, T *tap_base, int tap_ld) {
+        const dflash_model_cfg &m = c.target;
+        const LayerW &w = tl[l];
+        const int H = m.hidden, hd = m.head_dim, qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd;
+        launch_rmsnorm<T>(x, H, w.attn_norm, H, (float)m.rms_eps, xn, H, R, s);
+        Epi<T> e;
+        e.kind = EPI_QKV;
+        e.R_blk = R;
+        e.meta = mt;
+        e.nq = m.n_q_heads;
+        e.nkv = m.n_kv_heads;
+        e.hd = hd;
+        e.max_len = c.max_len;
+        e.rope = rope_t;
+        e.q_out = q;
+        e.kc = tk + (size_t)l * kv_layer_elems(m);
+        e.vc = tv + (size_t)l * kv_layer_elems(m);
+        gemm(xn, H, R, w.wqkv, qd + 2 * kd, H, e);
+        attention(q, e.kc, e.vc, mt, R, m, ao);
+        Epi<T> r;
+        r.kind = EPI_RESID;
+        r.x = x;
+        r.meta = mt;
+        gemm(ao, qd, R, w.wo, H, qd, r);
+        launch_rmsnorm<T>(x, H, w.ffn_norm, H, (float)m.rms_eps, xn, H, R, s);
+        TapDst<T> taps{};
+        taps.base = tap_base;
+        taps.ld = tap_ld;
+        taps.n = 0;
+        if (tap_base)
+            for (int i = 0; i < c.n_taps; ++i)
+                if (c.tap_layers[i] == l) taps.col[taps.n++] = i * H;
+        if (m.n_experts > 0) {
+            moe_ffn(l, R, mt, taps);
+        } else {
+            Epi<T> sw;
+            sw.kind = EPI_SWIGLU;
+            sw.h = h;
+            sw.F = m.ffn;
+            gemm(xn, H, R, w.w_gate_up, 2 * m.ffn, H, sw);
+            Epi<T> dn;
+            dn.kind = EPI_RESID;
+            dn.x = x;
+            dn.meta = mt;
+            dn.taps = taps;
+            gemm(h, m.ffn, R, w.w_down, H, m.ffn, dn);
+        }
+    }
+
+    void moe_ffn(int l, int R, const RowMeta *mt, const TapDst<T> &taps) {
+        const dflash_model_cfg &m = c.target;
+        const LayerW &w = tl[l];
+        const int H = m.hidden, E = m.n_experts, k = m.top_k, Fe = m.expert_ffn;
+        Epi<T> e;
+        e.kind = EPI_STORE;
+        e.Y = Y;
+        e.ldy = E;
+        gemm(xn, H, R, w.w_router, E, H, e);
+        launch_moe_topk(Y, E, R, k, moe_sel, moe_wt, s);
+        if (moe_tc_supported<T>()) {
+            run_moe_tc<T>(xn, H, R, k, moe_sel, (const T *)w.we_gate_up, (const T *)w.we_down, H, Fe, E, h, moe_part,
+                          tc, s);
+        } else {
+            launch_moe_experts_simt<T>(xn, H, R, k, moe_sel, (const T *)w.we_gate_up, (const T *)w.we_down, H, Fe,
+                                       moe_part, s);
+        }
+        launch_moe_combine<T>(x, moe_part, moe_wt, H, R, k, taps, mt, s);
+    }
+
+    void drafter_layer(int j, int R, bool with_ctx) {
+        const dflash_model_cfg &m = c.drafter;
+        const LayerW &w = dl[j];
+        const int H = m.hidden, hd = m.head_dim, qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd;
+        launch_rmsnorm<T>(x, H, w.attn_norm, H, (float)m.rms_eps, dq_in, H, R, s);
+        Epi<T> e;
+        e.kind = EPI_QKV;
+        e.R_blk = R;
+        e.meta = meta;
+        e.ctx_meta = ctx_meta;
+        e.nq = m.n_q_heads;
+        e.nkv = m.n_kv_heads;
+        e.hd = hd;
+        e.max_len = c.max_len;
+        e.rope = rope_d;
+        e.q_out = q;
+        e.kc = dk + (size_t)j * kv_layer_elems(m);
+        e.vc = dv + (size_t)j * kv_layer_elems(m);
+        // block rows and context rows share one pass over Wqkv (K/V injection)
+        gemm(dq_in, H, with_ctx ? 2 * R : R, w.wqkv, qd + 2 * kd, H, e);
+        attention(q, e.kc, e.vc, meta, R, m, ao);
+        Epi<T> r;
+        r.kind = EPI_RESID;
+        r.x = x;
+        r.meta = meta;
+        gemm(ao, qd, R, w.wo, H, qd, r);
+        launch_rmsnorm<T>(x, H, w.ffn_norm, H, (float)m.rms_eps, xn, H, R, s);
+        Epi<T> sw;
+        sw.kind = EPI_SWIGLU;
+        sw.h = h;
+        sw.F = m.ffn;
+        gemm(xn, H, R, w.w_gate_up, 2 * m.ffn, H, sw);
+        Epi<T> dn;
+        dn.kind = EPI_RESID;
+        dn.x = x;
+        dn.meta = meta;
+        gemm(h, m.ffn, R, w.w_down, H, m.ffn, dn);
+    }
+
+    void lm_head_rows(const float *final_norm, float eps, int R, float *lg, int64_t ldl) {
+        const int H = c.target.hidden;
+        launch_rmsnorm<T>(x, H, final_norm, H, eps, xn, H, R, s);
+        Epi<T> e;
+        e.kind = EPI_LOGITS;
+        e.Y = lg;
+        e.ldy = (int)ldl;
+        gemm(xn, H, R, lm_head, c.target.vocab, H, e);
+    }
+
+    // ---- steps ----
+    void enqueue_prefill(int seq, int n, int max_new) {
+        const dflash_model_cfg &t = c.target, &d = c.drafter;
+        const int H = t.hidden, TK = c.n_taps * H;
+        const int qd = d.n_q_heads * d.head_dim, kd = d.n_kv_heads * d.head_dim;
+        for (int c0 = 0; c0 < n; c0 += L.C) {
+            const int R = std::min(L.C, n - c0);
+            launch_embed_tokens<T>(embed, H, tokens + c0, R, seq, c0, x, meta, s);
+            for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, meta, taps_pre, TK);
+            if (c0 + R == n) {
+                // greedy first token from the last prompt row
+                launch_rmsnorm<T>(x + (size_t)(R - 1) * H, H, t_final, H, (float)t.rms_eps, xn, H, 1, s);
+                Epi<T> e;
+                e.kind = EPI_LOGITS;
+                e.Y = plogits;
+                e.ldy = t.vocab;
+                gemm(xn, H, 1, lm_head, t.vocab, H, e);
+                launch_argmax_rows(plogits, t.vocab, t.vocab, 1, 0, 1, first_tok, stats, s);
+            }
+            // context vectors of the prompt rows -> drafter context K/V
+            Epi<T> f;
+            f.kind = EPI_STORE;
+            f.Y = Y;
+            f.ldy = H;
+            gemm(taps_pre, TK, R, w_fc, H, TK, f);
+            launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, cbuf, H, R, s);
+            launch_ctx_meta_prefill(ctx_meta_pre, R, seq, c0, s);
+            for (int j = 0; j < d.n_layers; ++j) {
+                Epi<T> e;
+                e.kind = EPI_QKV;
+                e.col0 = qd;
+                e.R_blk = 0;
+                e.ctx_meta = ctx_meta_pre;
+                e.nq = d.n_q_heads;
+                e.nkv = d.n_kv_heads;
+                e.hd = d.head_dim;
+                e.max_len = c.max_len;
+                e.rope = rope_d;
+                e.kc = dk + (size_t)j * kv_layer_elems(d);
+                e.vc = dv + (size_t)j * kv_layer_elems(d);
+                const T *wkv = (const T *)dl[j].wqkv + (size_t)qd * H;
+                gemm(cbuf, H, R, wkv, 2 * kd, H, e);
+            }
+        }
+        launch_prefill_finish(st, seq, n, first_tok, out_tok, c.max_len, max_new, s);
+    }
+
+    void enqueue_draft(int nseq, bool contiguous) {
+        const dflash_model_cfg &t = c.target, &d = c.drafter;
+        const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
+        launch_embed_block<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, s);
+        // fuse pending taps -> context vectors (rows R..2R-1 of the drafter QKV input)
+        const T *tin = taps_dec;
+        if (!contiguous) {
+            launch_gather_rows(taps_dec, taps_gather, (size_t)TK * sizeof(T), active, nseq, B, s);
+            tin = taps_gather;
+        }
+        Epi<T> f;
+        f.kind = EPI_STORE;
+        f.Y = Y;
+        f.ldy = H;
+        gemm(tin, TK, R, w_fc, H, TK, f);
+        launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, dq_in + (size_t)R * H, H, R, s);
+        for (int j = 0; j < d.n_layers; ++j) drafter_layer(j, R, true);
+        lm_head_rows(d_final, (float)d.rms_eps, R, logits, t.vocab);
+        if (B > 1) launch_argmax_rows(logits, t.vocab, t.vocab, R, 1, B, drafts, stats, s);
+        if (draft_mode == DFLASH_DRAFT_SCRIPT)
+            launch_script_drafts(st, active, nseq, B, tau, t.vocab, script, c.max_len, drafts, s);
+    }
+
+    void enqueue_verify(int nseq) {
+        const dflash_model_cfg &t = c.target;
+        const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
+        launch_embed_block<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
+        for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, meta, taps_dec, TK);
+        lm_head_rows(t_final, (float)t.rms_eps, R, logits, t.vocab);
+        launch_argmax_rows(logits, t.vocab, t.vocab, R, 0, B, g, stats, s);
+        launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
+    }
+
+    void enqueue_ar_step(int nseq) {
+        const dflash_model_cfg &t = c.target;
+        const int H = t.hidden;
+        launch_embed_block<T>(embed, H, st, active, nseq, 1, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
+        for (int l = 0; l < t.n_layers; ++l) target_layer(l, nseq, meta, nullptr, 0);
+        lm_head_rows(t_final, (float)t.rms_eps, nseq, logits, t.vocab);
+        launch_argmax_rows(logits, t.vocab, t.vocab, nseq, 0, 1, g, stats, s);
+        launch_ar_step(st, active, nseq, g, out_tok, c.max_len, stats, s);
+    }
+
+    // ---- API ----
+    dflash_status check_seqs(const int32_t *seqs, int n) {
+        if (!seqs || n < 1 || n > c.max_batch) { err = "seqs must hold 1..max_batch slots"; return DFLASH_EINVAL; }
+        std::vector<char> seen(c.max_batch, 0);
+        for (int i = 0; i < n; ++i) {
+            if (seqs[i] < 0 || seqs[i] >= c.max_batch || seen[seqs[i]]) { err = "bad or repeated slot"; return DFLASH_EINVAL; }
+            seen[seqs[i]] = 1;
+            if (!h_prefilled[seqs[i]]) { err = "slot not prefilled"; return DFLASH_ESTATE; }
+            if (h_len[seqs[i]] + c.block_size > c.max_len) { err = "sequence would exceed max_len"; return DFLASH_ECAPACITY; }
+        }
+        return DFLASH_OK;
+    }
+
+    dflash_status prefill(int seq, const int32_t *prompt, int n, int max_new, int32_t *first) override {
+        if (seq < 0 || seq >= c.max_batch || !prompt || n < 1) { err = "bad prefill arguments"; return DFLASH_EINVAL; }
+        if (n + c.block_size > c.max_len) { err = "prompt + block exceeds max_len"; return DFLASH_ECAPACITY; }
+        for (int i = 0; i < n; ++i)
+            if (prompt[i] < 0 || prompt[i] >= c.target.vocab) { err = "prompt id out of vocab"; return DFLASH_EINVAL; }
+        if (cudaMemcpyAsync(tokens, prompt, sizeof(int32_t) * n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return fail_cuda("prompt copy");
+        enqueue_prefill(seq, n, max_new);
+        dflash_status r = check("prefill launch");
+        if (r) return r;
+        h_len[seq] = n;
+        h_prefilled[seq] = 1;
+        last_draft.clear();
+        last_logits_rows[2] = 1;
+        if (first) {
+            if ((r = sync("prefill"))) return r;
+            if (cudaMemcpy(first, first_tok, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return fail_cuda("first token");
+        }
+        return DFLASH_OK;
+    }
+
+    dflash_status set_active(const int32_t *seqs, int n) {
+        if (cudaMemcpyAsync(active, seqs, sizeof(int32_t) * n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return fail_cuda("active copy");
+        return DFLASH_OK;
+    }
+
+    static bool is_iota(const int32_t *seqs, int n) {
+        for (int i = 0; i < n; ++i) if (seqs[i] != i) return false;
+        return true;
+    }
+
+    dflash_status draft(const int32_t *seqs, int n, int32_t *out, bool) override {
+        dflash_status r = check_seqs(seqs, n);
+        if (r) return r;
+        if ((r = set_active(seqs, n))) return r;
+        enqueue_draft(n, is_iota(seqs, n));
+        if ((r = check("draft launch"))) return r;
+        last_draft.assign(seqs, seqs + n);
+        last_logits_rows[0] = n * c.block_size;
+        if (out && c.block_size > 1) {
+            if ((r = sync("draft"))) return r;
+            if (cudaMemcpy(out, drafts, sizeof(int32_t) * n * (c.block_size - 1), cudaMemcpyDeviceToHost) != cudaSuccess)
+                return fail_cuda("drafts copy");
+        }
+        return DFLASH_OK;
+    }
+
+    dflash_status verify(const int32_t *seqs, int n, const int32_t *dr, int32_t *acc, int32_t *com,
+                         int32_t *nl) override {
+        dflash_status r = check_seqs(seqs, n);
+        if (r) return r;
+        if ((int)last_draft.size() != n || !std::equal(last_draft.begin(), last_draft.end(), seqs)) {
+            err = "verify_commit must follow dflash_draft_block on the same sequences";
+            return DFLASH_ESTATE;
+        }
+        const int B = c.block_size;
+        if (dr) {
+            for (int i = 0; i < n * (B - 1); ++i)
+                if (dr[i] < 0 || dr[i] >= c.target.vocab) { err = "draft id out of vocab"; return DFLASH_EINVAL; }
+            if (B > 1 && cudaMemcpyAsync(drafts, dr, sizeof(int32_t) * n * (B - 1), cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return fail_cuda("drafts copy");
+        }
+        enqueue_verify(n);
+        if ((r = check("verify launch"))) return r;
+        last_draft.clear();
+        last_logits_rows[1] = n * B;
+        if ((r = sync("verify"))) return r;
+        std::vector<int32_t> lens(n);
+        if (cudaMemcpy(lens.data(), new_len, sizeof(int32_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return fail_cuda("new_len copy");
+        for (int i = 0; i < n; ++i) h_len[seqs[i]] = lens[i];
+        if (nl) std::copy(lens.begin(), lens.end(), nl);
+        if (acc && cudaMemcpy(acc, accept, sizeof(int32_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return fail_cuda("accept copy");
+        if (com && cudaMemcpy(com, committed, sizeof(int32_t) * n * B, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return fail_cuda("committed copy");
+        return DFLASH_OK;
+    }
+
+    dflash_status numeric_status() {
+        DevStats hs;
+        if (cudaMemcpy(&hs, stats, sizeof hs, cudaMemcpyDeviceToHost) != cudaSuccess) return fail_cuda("stats copy");
+        if (hs.status) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
+        return DFLASH_OK;
+    }
+
+    dflash_status start_run(const int32_t *const *prompts, const int32_t *lens, int n, int max_new) {
+        if (!prompts || !lens || n < 1 || n > c.max_batch || max_new < 1) { err = "bad generate arguments"; return DFLASH_EINVAL; }
+        for (int i = 0; i < n; ++i) {
+            if (!prompts[i] || lens[i] < 1) { err = "empty prompt"; return DFLASH_EINVAL; }
+            if ((int64_t)lens[i] + max_new + c.block_size > c.max_len) { err = "prompt + max_new + block exceeds max_len"; return DFLASH_ECAPACITY; }
+        }
+        if (cudaMemsetAsync(stats, 0, sizeof(DevStats), s) != cudaSuccess) return fail_cuda("stats reset");
+        for (int i = 0; i < n; ++i) {
+            dflash_status r = prefill(i, prompts[i], lens[i], max_new, nullptr);
+            if (r) return r;
+        }
+        std::vector<int32_t> iota(n);
+        for (int i = 0; i < n; ++i) iota[i] = i;
+        return set_active(iota.data(), n);
+    }
+
+    // Run iterations until every sequence is done; the done counter of
+    // iteration k is read while iteration k+1 is already queued.
+    template <typename F>
+    dflash_status run_loop(int n, int max_iters, F &&step, int64_t *iters_out) {
+        int64_t it = 0;
+        bool pending = false;
+        while (it < max_iters) {
+            step();
+            ++it;
+            if (cudaMemcpyAsync(pinned + (it & 1), &stats->n_done, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+                return fail_cuda("done counter");
+            cudaEvent_t ev = (it & 1) ? ev_a : ev_b;
+            if (cudaEventRecord(ev, s) != cudaSuccess) return fail_cuda("event");
+            if (pending) {
+                cudaEvent_t prev = (it & 1) ? ev_b : ev_a;
+                const int tmo = c.timeout_ms > 0 ? c.timeout_ms : 600000;
+                auto t0 = std::chrono::steady_clock::now();
+                while (true) {
+                    cudaError_t e = cudaEventQuery(prev);
+                    if (e == cudaSuccess) break;
+                    if (e != cudaErrorNotReady) { err = cudaGetErrorString(e); return DFLASH_ECUDA; }
+                    if (std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0).count() > tmo) {
+                        err = "decode iteration did not finish within the timeout";
+                        return DFLASH_ETIMEOUT;
+                    }
+                    std::this_thread::yield();
+                }
+                if (pinned[(it - 1) & 1] >= n) break;
+            }
+            pending = true;
+        }
+        dflash_status r = sync("decode");
+        if (r) return r;
+        if (iters_out) *iters_out = it;
+        return check("decode loop");
+    }
+
+    dflash_status generate(const int32_t *const *prompts, const int32_t *lens, int n, int max_new, int32_t *out,
+                           dflash_stats *ost) override {
+        cudaEvent_t t0, t1, t2;
+        cudaEventCreate(&t0);
+        cudaEventCreate(&t1);
+        cudaEventCreate(&t2);
+        cudaEventRecord(t0, s);
+        dflash_status r = start_run(prompts, lens, n, max_new);
+        if (r) return r;
+        cudaEventRecord(t1, s);
+        const bool contiguous = true;
+        if (max_new > 1) {
+            r = run_loop(n, max_new + 2, [&] { enqueue_draft(n, contiguous); enqueue_verify(n); }, nullptr);
+            if (r) return r;
+        }
+        cudaEventRecord(t2, s);
+        if ((r = sync("generate"))) return r;
+        for (int i = 0; i < n; ++i)
+            if (cudaMemcpy(out + (size_t)i * max_new, out_tok + (size_t)i * c.max_len, sizeof(int32_t) * max_new,
+                           cudaMemcpyDeviceToHost) != cudaSuccess)
+                return fail_cuda("output copy");
+        DevStats hs;
+        if (cudaMemcpy(&hs, stats, sizeof hs, cudaMemcpyDeviceToHost) != cudaSuccess) return fail_cuda("stats");
+        for (int i = 0; i < n; ++i) h_len[i] = 0;
+        if (ost) {
+            memset(ost, 0, sizeof *ost);
+            ost->iterations = (int64_t)hs.iterations;
+            ost->tokens = (int64_t)hs.tokens;
+            for (int i = 0; i < DFLASH_MAX_BLOCK; ++i) ost->accept_hist[i] = (int64_t)hs.hist[i];
+            ost->mean_tau = hs.iterations ? (double)hs.tokens / (double)hs.iterations : 0.0;
+            float a = 0, b = 0;
+            cudaEventElapsedTime(&a, t0, t1);
+            cudaEventElapsedTime(&b, t1, t2);
+            ost->ms_prefill = a;
+            ost->ms_decode = b;
+        }
+        cudaEventDestroy(t0);
+        cudaEventDestroy(t1);
+        cudaEventDestroy(t2);
+        // generation leaves the slots in a finished state: refuse draft/verify on them
+        for (int i = 0; i < n; ++i) h_prefilled[i] = 0;
+        if (hs.status) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
+        return check("generate");
+    }
+
+    dflash_status generate_ar(const int32_t *const *prompts, const int32_t *lens, int n, int max_new, int32_t *out,
+                              double *ms) override {
+        cudaEvent_t t1, t2;
+        cudaEventCreate(&t1);
+        cudaEventCreate(&t2);
+        dflash_status r = start_run(prompts, lens, n, max_new);
+        if (r) return r;
+        cudaEventRecord(t1, s);
+        if (max_new > 1) {
+            r = run_loop(n, max_new + 1, [&] { enqueue_ar_step(n); }, nullptr);
+            if (r) return r;
+        }
+        cudaEventRecord(t2, s);
+        if ((r = sync("generate_ar"))) return r;
+        for (int i = 0; i < n; ++i)
+            if (cudaMemcpy(out + (size_t)i * max_new, out_tok + (size_t)i * c.max_len, sizeof(int32_t) * max_new,
+                           cudaMemcpyDeviceToHost) != cudaSuccess)
+                return fail_cuda("output copy");
+        if (ms) {
+            float b = 0;
+            cudaEventElapsedTime(&b, t1, t2);
+            *ms = b;
+        }
+        cudaEventDestroy(t1);
+        cudaEventDestroy(t2);
+        for (int i = 0; i < n; ++i) h_prefilled[i] = 0;
+        return numeric_status();
+    }
+
+    dflash_status debug_logits(int which, float *out, int64_t cap, int64_t *rows) override {
+        if (!c.keep_logits) { err = "context created without keep_logits"; return DFLASH_ESTATE; }
+        if (which < 0 || which > 2 || !out) { err = "bad debug_logits arguments"; return DFLASH_EINVAL; }
+        const int64_t V = c.target.vocab;
+        const int64_t nr = last_logits_rows[which];
+        if (nr * V > cap) { err = "output buffer too small"; return DFLASH_EINVAL; }
+        dflash_status r = sync("debug_logits");
+        if (r) return r;
+        const float *src = which == 2 ? plogits : logits;
+        if (cudaMemcpy(out, src, sizeof(float) * nr * V, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return fail_cuda("logits copy");
+        if (rows) *rows = nr;
+        return DFLASH_OK;
+    }
+
+    dflash_status seq_state(int seq, int32_t *len, int32_t *anchor, int32_t *n_out) override {
+        if (seq < 0 || seq >= c.max_batch) { err = "bad slot"; return DFLASH_EINVAL; }
+        dflash_status r = sync("seq_state");
+        if (r) return r;
+        SeqState hs;
+        if (cudaMemcpy(&hs, st + seq, sizeof hs, cudaMemcpyDeviceToHost) != cudaSuccess) return fail_cuda("state copy");
+        if (len) *len = hs.len;
+        if (anchor) *anchor = hs.anchor;
+        if (n_out) *n_out = hs.n_out;
+        return DFLASH_OK;
+    }
+
+    dflash_status debug_kv(int which, int layer, int seq, int p0, int n, float *ko, float *vo) override {
+        const dflash_model_cfg &m = which == 0 ? c.target : c.drafter;
+        if (which < 0 || which > 1 || layer < 0 || layer >= m.n_layers || seq < 0 || seq >= c.max_batch || p0 < 0 ||
+            n < 1 || p0 + n > c.max_len || !ko || !vo) {
+            err = "bad debug_kv arguments";
+            return DFLASH_EINVAL;
+        }
+        dflash_status r = sync("debug_kv");
+        if (r) return r;
+        const T *kc = (which == 0 ? tk : dk) + (size_t)layer * kv_layer_elems(m);
+        const T *vc = (which == 0 ? tv : dv) + (size_t)layer * kv_layer_elems(m);
+        const int hd = m.head_dim, nkv = m.n_kv_heads;
+        std::vector<T> buf((size_t)n * hd);
+        for (int pass = 0; pass < 2; ++pass) {
+            const T *src = pass ? vc : kc;
+            float *dst = pass ? vo : ko;
+            for (int hh = 0; hh < nkv; ++hh) {
+                const T *p = src + (((size_t)seq * nkv + hh) * c.max_len + p0) * hd;
+                if (cudaMemcpy(buf.data(), p, sizeof(T) * n * hd, cudaMemcpyDeviceToHost) != cudaSuccess)
+                    return fail_cuda("kv copy");
+                for (int t = 0; t < n; ++t)
+                    for (int e = 0; e < hd; ++e) dst[(size_t)t * nkv * hd + hh * hd + e] = host_to_f(buf[(size_t)t * hd + e]);
+            }
+        }
+        return DFLASH_OK;
+    }
+
+    static float host_to_f(float v) { return v; }
+    static float host_to_f(bf16 v) {
+        uint16_t b;
+        memcpy(&b, &v, 2);
+        uint32_t u = (uint32_t)b << 16;
+        float f;
+        memcpy(&f, &u, 4);
+        return f;
+    }
+
+    dflash_status set_script(int seq, const int32_t *sc, int n) override {
+        if (seq < 0 || seq >= c.max_batch || !sc || n < 1 || n > c.max_len) { err = "bad script arguments"; return DFLASH_EINVAL; }
+        for (int i = 0; i < n; ++i)
+            if (sc[i] < 0 || sc[i] >= c.target.vocab) { err = "script id out of vocab"; return DFLASH_EINVAL; }
+        if (cudaMemcpyAsync(script + (size_t)seq * c.max_len, sc, sizeof(int32_t) * n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return fail_cuda("script copy");
+        return sync("script");
+    }
+};
+
+}  // namespace dfl
+
+using namespace dfl;
+
+// ------------------------------------------------------------------------
+// C ABI
+// ------------------------------------------------------------------------
+
+extern "C" {
+
+dflash_status dflash_workspace_size(const dflash_config *cfg, size_t *wb, size_t *sb) {
+    if (!cfg || !wb || !sb) return DFLASH_EINVAL;
+    std::string why;
+    if (!check_config(*cfg, why)) return DFLASH_EINVAL;
+    Layout L = make_layout(*cfg);
+    *wb = L.weight_bytes;
+    *sb = L.state_bytes;
+    return DFLASH_OK;
+}
+
+dflash_status dflash_create(const dflash_config *cfg, void *warena, size_t wbytes, void *sarena, size_t sbytes,
+                            void *stream, dflash_ctx **out) {
+    if (!cfg || !out) return DFLASH_EINVAL;
+    *out = nullptr;
+    std::string why;
+    if (!check_config(*cfg, why)) return DFLASH_EINVAL;
+    dflash_ctx *ctx = new dflash_ctx();
+    ctx->cfg = *cfg;
+    ctx->lay = make_layout(*cfg);
+    if (!warena || !sarena || wbytes < ctx->lay.weight_bytes || sbytes < ctx->lay.state_bytes ||
+        ((uintptr_t)warena & 255) || ((uintptr_t)sarena & 255)) {
+        delete ctx;
+        return DFLASH_EINVAL;
+    }
+    for (size_t i = 0; i < ctx->lay.slots.size(); ++i) ctx->by_name[ctx->lay.slots[i].name] = (int)i;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cfg->dtype == DFLASH_BF16)
+        ctx->eng.reset(new Engine<bf16>(*cfg, ctx->lay, (char *)warena, (char *)sarena, s));
+    else
+        ctx->eng.reset(new Engine<float>(*cfg, ctx->lay, (char *)warena, (char *)sarena, s));
+    dflash_status r;
+    if (cfg->dtype == DFLASH_BF16) r = static_cast<Engine<bf16> *>(ctx->eng.get())->init(ctx->by_name);
+    else r = static_cast<Engine<float> *>(ctx->eng.get())->init(ctx->by_name);
+    if (r != DFLASH_OK) {
+        fprintf(stderr, "dflash_create: %s\n", ctx->eng->err.c_str());
+        delete ctx;
+        return r;
+    }
+    *out = ctx;
+    return DFLASH_OK;
+}
+
+void dflash_destroy(dflash_ctx *ctx) { delete ctx; }
+
+const char *dflash_last_error(const dflash_ctx *ctx) {
+    if (!ctx) return "null context";
+    return ctx->err.c_str();
+}
+
+int32_t dflash_weight_count(const dflash_ctx *ctx) { return ctx ? (int32_t)ctx->lay.slots.size() : 0; }
+
+dflash_status dflash_weight_info(const dflash_ctx *ctx, int32_t i, const char **name, size_t *offset, size_t *numel,
+                                 int32_t *dtype, int32_t *ndim, int64_t *shape) {
+    if (!ctx || i < 0 || i >= (int32_t)ctx->lay.slots.size()) return DFLASH_EINVAL;
+    const WeightSlot &w = ctx->lay.slots[i];
+    if (name) *name = w.name.c_str();
+    if (offset) *offset = w.offset;
+    if (numel) *numel = w.numel;
+    if (dtype) *dtype = w.dtype;
+    if (ndim) *ndim = w.ndim;
+    if (shape) for (int k = 0; k < 3; ++k) shape[k] = w.shape[k];
+    return DFLASH_OK;
+}
+
+dflash_status dflash_weight_slot(const dflash_ctx *ctx, const char *name, size_t *offset, size_t *numel,
+                                 int32_t *dtype) {
+    if (!ctx || !name) return DFLASH_EINVAL;
+    auto it = ctx->by_name.find(name);
+    if (it == ctx->by_name.end()) return DFLASH_EINVAL;
+    const WeightSlot &w = ctx->lay.slots[it->second];
+    if (offset) *offset = w.offset;
+    if (numel) *numel = w.numel;
+    if (dtype) *dtype = w.dtype;
+    return DFLASH_OK;
+}
+
+#define DFL_CALL(ctx, expr)                                                   \
+    do {                                                                      \
+        if (!(ctx)) return DFLASH_EINVAL;                                     \
+        if ((ctx)->broken) { (ctx)->err = "context unusable after a CUDA error"; return DFLASH_ECUDA; } \
+        dflash_status _r = (expr);                                            \
+        (ctx)->err = _r ? (ctx)->eng->err : std::string();                    \
+        if (_r == DFLASH_ECUDA) (ctx)->broken = true;                         \
+        return _r;                                                            \
+    } while (0)
+
+dflash_status dflash_prefill(dflash_ctx *ctx, int32_t seq, const int32_t *prompt, int32_t n, int32_t *first) {
+    DFL_CALL(ctx, ctx->eng->prefill(seq, prompt, n, INT_MAX, first));
+}
+
+dflash_status dflash_draft_block(dflash_ctx *ctx, const int32_t *seqs, int32_t n, int32_t *drafts) {
+    DFL_CALL(ctx, ctx->eng->draft(seqs, n, drafts, drafts != nullptr));
+}
+
+dflash_status dflash_verify_commit(dflash_ctx *ctx, const int32_t *seqs, int32_t n, const int32_t *drafts,
+                                   int32_t *accept, int32_t *committed, int32_t *new_len) {
+    DFL_CALL(ctx, ctx->eng->verify(seqs, n, drafts, accept, committed, new_len));
+}
+
+dflash_status dflash_generate(dflash_ctx *ctx, const int32_t *const *prompts, const int32_t *lens, int32_t n,
+                              int32_t max_new, int32_t *out, dflash_stats *stats) {
+    if (!out) return DFLASH_EINVAL;
+    DFL_CALL(ctx, ctx->eng->generate(prompts, lens, n, max_new, out, stats));
+}
+
+dflash_status dflash_generate_ar(dflash_ctx *ctx, const int32_t *const *prompts, const int32_t *lens, int32_t n,
+                                 int32_t max_new, int32_t *out, double *ms) {
+    if (!out) return DFLASH_EINVAL;
+    DFL_CALL(ctx, ctx->eng->generate_ar(prompts, lens, n, max_new, out, ms));
+}
+
+dflash_status dflash_set_draft_mode(dflash_ctx *ctx, int32_t mode, int32_t tau) {
+    if (!ctx) return DFLASH_EINVAL;
+    if ((mode != DFLASH_DRAFT_MODEL && mode != DFLASH_DRAFT_SCRIPT) || tau < 1 || tau > ctx->cfg.block_size)
+        return DFLASH_EINVAL;
+    ctx->eng->draft_mode = mode;
+    ctx->eng->tau = tau;
+    return DFLASH_OK;
+}
+
+dflash_status dflash_set_script(dflash_ctx *ctx, int32_t seq, const int32_t *script, int32_t n) {
+    DFL_CALL(ctx, ctx->eng->set_script(seq, script, n));
+}
+
+dflash_status dflash_debug_logits(dflash_ctx *ctx, int32_t which, float *out, int64_t cap, int64_t *rows) {
+    DFL_CALL(ctx, ctx->eng->debug_logits(which, out, cap, rows));
+}
+
+dflash_status dflash_seq_state(dflash_ctx *ctx, int32_t seq, int32_t *len, int32_t *anchor, int32_t *n_out) {
+    DFL_CALL(ctx, ctx->eng->seq_state(seq, len, anchor, n_out));
+}
+
+dflash_status dflash_debug_kv(dflash_ctx *ctx, int32_t which, int32_t layer, int32_t seq, int32_t p0, int32_t n,
+                              float *k, float *v) {
+    DFL_CALL(ctx, ctx->eng->debug_kv(which, layer, seq, p0, n, k, v));
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// engine.h -- internal structures of a dflash context.
+#pragma once
+
+#include <memory>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/dflash.h"
+#include "kernels.h"
+
+namespace dfl {
+
+struct WeightSlot {
+    std::string name;
+    size_t offset = 0, numel = 0;
+    int dtype = 0;  // DFLASH_FP32 / DFLASH_BF16
+    int ndim = 0;
+    int64_t shape[3] = {0, 0, 0};
+};
+
+struct LayerW {
+    const float *attn_norm = nullptr, *ffn_norm = nullptr;
+    const void *wqkv = nullptr, *wo = nullptr, *w_gate_up = nullptr, *w_down = nullptr;
+    const void *w_router = nullptr, *we_gate_up = nullptr, *we_down = nullptr;
+};
+
+// Byte layout of the two arenas, computed identically by workspace_size and create.
+struct Layout {
+    std::vector<WeightSlot> slots;
+    size_t weight_bytes = 0;
+    // state arena offsets
+    size_t x, xn, dq_in, Y, q, ao, h, taps_dec, taps_gather, taps_pre, cbuf, logits, plogits;
+    size_t g, drafts, accept, committed, new_len, st, active, meta, ctx_meta, ctx_meta_pre;
+    size_t rope_t, rope_d, tk, tv, dk, dv, script, out_tok, tokens, stats, first_tok;
+    size_t moe_sel, moe_wt, moe_part;
+    size_t gemm_ws, gemm_sem;
+    size_t state_bytes = 0;
+    // dims
+    int R_dec = 0, C = 0, R_max = 0, Y_cols = 0, ws_floats = 0, n_sem = 0;
+};
+
+struct Status {
+    dflash_status code;
+    std::string msg;
+};
+
+class EngineBase {
+  public:
+    virtual ~EngineBase() {}
+    virtual dflash_status prefill(int seq, const int32_t *prompt, int n, int max_new, int32_t *first) = 0;
+    virtual dflash_status draft(const int32_t *seqs, int n, int32_t *drafts, bool sync) = 0;
+    virtual dflash_status verify(const int32_t *seqs, int n, const int32_t *drafts, int32_t *accept,
+                                 int32_t *committed, int32_t *new_len) = 0;
+    virtual dflash_status generate(const int32_t *const *prompts, const int32_t *lens, int n, int max_new,
+                                   int32_t *out, dflash_stats *stats) = 0;
+    virtual dflash_status generate_ar(const int32_t *const *prompts, const int32_t *lens, int n,
+                                      int max_new, int32_t *out, double *ms) = 0;
+    virtual dflash_status debug_logits(int which, float *out, int64_t cap, int64_t *rows) = 0;
+    virtual dflash_status seq_state(int seq, int32_t *len, int32_t *anchor, int32_t *n_out) = 0;
+    virtual dflash_status debug_kv(int which, int layer, int seq, int p0, int n, float *k, float *v) = 0;
+    virtual dflash_status set_script(int seq, const int32_t *script, int n) = 0;
+    std::string err;
+    int draft_mode = DFLASH_DRAFT_MODEL, tau = 1;
+};
+
+}  // namespace dfl
+
+struct dflash_ctx {
+    dflash_config cfg;
+    dfl::Layout lay;
+    std::unordered_map<std::string, int> by_name;
+    std::unique_ptr<dfl::EngineBase> eng;
+    std::string err;
+    bool broken = false;
+};

@@ -1,0 +1,117 @@
+// kernels.h -- host launchers of the DFlash kernels (internal interface).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace dfl {
+
+// Tap destinations of one target layer: the residual after the layer is
+// copied (rounded to T) to columns col[i] .. col[i]+H of row meta[r].aux of
+// `base` (leading dimension ld), for i < n.
+template <typename T>
+struct TapDst {
+    T *base;
+    int ld;
+    int n;
+    int col[8];
+};
+
+// ---- rows: embedding + metadata ----
+template <typename T>
+void launch_embed_block(const T *emb, int H, SeqState *st, const int *active, int nseq, int B,
+                        int is_draft, const int *drafts, int mask_id, float *x, RowMeta *meta,
+                        RowMeta *ctx_meta, cudaStream_t s);
+template <typename T>
+void launch_embed_tokens(const T *emb, int H, const int *tokens, int R, int seq, int pos0,
+                         float *x, RowMeta *meta, cudaStream_t s);
+void launch_ctx_meta_prefill(RowMeta *meta, int R, int seq, int pos0, cudaStream_t s);
+
+// ---- normalisation / elementwise ----
+template <typename TO>
+void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, TO *out, int ldo,
+                    int R, cudaStream_t s);
+template <typename T>
+void launch_residual(float *x, const float *Y, int ldy, int H, int R, const TapDst<T> &taps,
+                     const RowMeta *meta, cudaStream_t s);
+template <typename T>
+void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, cudaStream_t s);
+template <typename T>
+void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot,
+                         const RowMeta *meta, const RowMeta *ctx_meta, int nq, int nkv, int hd,
+                         const float2 *rope, T *q_out, T *kc, T *vc, int max_len, cudaStream_t s);
+
+// ---- GEMM (CUDA-core, fp32 accumulate): Y[M][N] = X[M][K] . W[N][K]^T ----
+template <typename T>
+void launch_gemm_simt(const T *X, int ldx, int M, const T *W, int ldw, int N, int K, float *Y,
+                      int ldy, cudaStream_t s);
+
+// ---- attention (CUDA-core reference path, used for fp32 models) ----
+template <typename T>
+void launch_attention_simt(const T *q, int ldq, const T *kc, const T *vc, const RowMeta *meta,
+                           int R, int nq, int nkv, int hd, int max_len, T *out, int ldo,
+                           cudaStream_t s);
+
+// ---- heads, acceptance, scripts ----
+// mode 0: idx[r] = argmax of row r.  mode 1 (drafter): rows r = i*B + j with
+// j >= 1 go to idx[i*(B-1) + j-1]; rows with j == 0 are skipped.
+void launch_argmax_rows(const float *logits, int64_t ldl, int V, int R, int mode, int B, int *idx,
+                        DevStats *stats, cudaStream_t s);
+void launch_accept(SeqState *st, const int *active, int nseq, int B, const int *drafts,
+                   const int *g, int *accept, int *committed, int *new_len, int *out_tok,
+                   int out_ld, DevStats *stats, cudaStream_t s);
+void launch_script_drafts(const SeqState *st, const int *active, int nseq, int B, int tau, int V,
+                          const int *script, int script_ld, int *drafts, cudaStream_t s);
+void launch_prefill_finish(SeqState *st, int seq, int n, const int *first_tok, int *out_tok,
+                           int out_ld, int max_new, cudaStream_t s);
+void launch_ar_step(SeqState *st, const int *active, int nseq, const int *g, int *out_tok,
+                    int out_ld, DevStats *stats, cudaStream_t s);
+
+// ---- MoE (routing + CUDA-core expert FFN reference path) ----
+void launch_moe_topk(const float *router_logits, int E, int R, int k, int *sel, float *wt,
+                     cudaStream_t s);
+template <typename T>
+void launch_moe_experts_simt(const T *m, int ldm, int R, int k, const int *sel, const T *w_gate_up,
+                             const T *w_down, int H, int Fe, float *part, cudaStream_t s);
+template <typename T>
+void launch_moe_combine(float *x, const float *part, const float *wt, int H, int R, int k,
+                        const TapDst<T> &taps, const RowMeta *meta, cudaStream_t s);
+
+// ---- tables ----
+void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStream_t s);
+
+}  // namespace dfl
+
+namespace dfl {
+
+// Epilogue of a projection Y[M][N] = X[M][K] . W[N][K]^T.
+enum EpiKind { EPI_STORE = 0, EPI_QKV = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_LOGITS = 4 };
+
+template <typename T>
+struct Epi {
+    EpiKind kind = EPI_STORE;
+    // EPI_STORE / EPI_LOGITS: fp32 output Y[M][ldy]
+    float *Y = nullptr;
+    int ldy = 0;
+    // EPI_QKV: columns are rows col0.. of [Wq; Wk; Wv]; rows < R_blk are block rows
+    // (q, k, v at meta.pos), rows >= R_blk context rows (k, v at ctx_meta.pos if aux)
+    int col0 = 0, R_blk = 0;
+    const RowMeta *meta = nullptr, *ctx_meta = nullptr;
+    int nq = 0, nkv = 0, hd = 0, max_len = 0;
+    const float2 *rope = nullptr;
+    T *q_out = nullptr, *kc = nullptr, *vc = nullptr;
+    // EPI_RESID: x[M][N] += Y, then tap copies of the new x
+    float *x = nullptr;
+    TapDst<T> taps{};
+    // EPI_SWIGLU: N = 2F, columns [gate; up]; h[M][F] = SiLU(gate) * up
+    T *h = nullptr;
+    int F = 0;
+};
+
+void launch_gather_rows(const void *src, void *dst, size_t row_bytes, const int *active, int nseq, int B,
+                        cudaStream_t s);
+
+}  // namespace dfl

@@ -1,0 +1,460 @@
+// kernels_rows.cu -- row bookkeeping, normalisation, elementwise epilogues,
+// greedy heads and the accept/commit step of the DFlash decode iteration.
+//
+// Method passages (DFlash pages, by title and section):
+//  * "DFlash: Decodificação Especulativa com Blocos em Paralelo ..." (iaemfoco),
+//    "O que o DFlash faz de diferente": the drafter fills a whole block in one
+//    pass; the target verifies the block in parallel.  Block rows are
+//    [anchor, mask x (B-1)] for the drafter and [anchor, d_1..d_{B-1}] for
+//    the target.
+//  * same page, "Decodificação especulativa tradicional": accepted tokens are
+//    kept and the output equals target-only decoding -> greedy acceptance of
+//    the longest prefix with d_i == g_{i-1}, plus the target's bonus token.
+//  * "Nova técnica faz modelo Qwen rodar ..." (forbuilders), "Como funciona a
+//    decodificação especulativa": only the wrong entries are discarded -> the
+//    KV cache is rolled back by length only.
+#include <math.h>
+
+#include "kernels.h"
+
+namespace dfl {
+
+// ------------------------------------------------------------------------
+// embeddings + row metadata
+// ------------------------------------------------------------------------
+
+template <typename T>
+__global__ void embed_block_kernel(const T *__restrict__ emb, int H, SeqState *st,
+                                   const int *__restrict__ active, int B, int is_draft,
+                                   const int *__restrict__ drafts, int mask_id, float *__restrict__ x,
+                                   RowMeta *meta, RowMeta *ctx_meta) {
+    const int r = blockIdx.x;
+    const int i = r / B, j = r % B;
+    const int s = active[i];
+    const SeqState S = st[s];
+    const int p = S.len;
+    int tok;
+    if (j == 0) tok = S.anchor;
+    else tok = is_draft ? mask_id : drafts[i * (B - 1) + (j - 1)];
+    const T *e = emb + (size_t)tok * H;
+    float *xr = x + (size_t)r * H;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) xr[c] = to_f(e[c]);
+    if (threadIdx.x == 0) {
+        RowMeta m;
+        m.seq = s;
+        m.pos = p + j;
+        m.nk = is_draft ? p + B : p + j + 1;
+        m.aux = s * B + j;  // pending tap row of the slot
+        meta[r] = m;
+        if (is_draft && ctx_meta) {
+            RowMeta c;
+            c.seq = s;
+            c.pos = S.pend_pos0 + j;
+            c.nk = 0;
+            c.aux = (j < S.pend_n) ? 1 : 0;
+            ctx_meta[r] = c;
+        }
+    }
+}
+
+template <typename T>
+void launch_embed_block(const T *emb, int H, SeqState *st, const int *active, int nseq, int B,
+                        int is_draft, const int *drafts, int mask_id, float *x, RowMeta *meta,
+                        RowMeta *ctx_meta, cudaStream_t s) {
+    embed_block_kernel<T><<<nseq * B, 256, 0, s>>>(emb, H, st, active, B, is_draft, drafts, mask_id,
+                                                   x, meta, ctx_meta);
+}
+
+template <typename T>
+__global__ void embed_tokens_kernel(const T *__restrict__ emb, int H, const int *__restrict__ tokens,
+                                    int seq, int pos0, float *__restrict__ x, RowMeta *meta) {
+    const int r = blockIdx.x;
+    const int tok = tokens[r];
+    const T *e = emb + (size_t)tok * H;
+    float *xr = x + (size_t)r * H;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) xr[c] = to_f(e[c]);
+    if (threadIdx.x == 0) {
+        RowMeta m;
+        m.seq = seq;
+        m.pos = pos0 + r;
+        m.nk = pos0 + r + 1;  // causal
+        m.aux = r;            // prefill tap rows are chunk rows
+        meta[r] = m;
+    }
+}
+
+template <typename T>
+void launch_embed_tokens(const T *emb, int H, const int *tokens, int R, int seq, int pos0, float *x,
+                         RowMeta *meta, cudaStream_t s) {
+    embed_tokens_kernel<T><<<R, 256, 0, s>>>(emb, H, tokens, seq, pos0, x, meta);
+}
+
+__global__ void ctx_meta_prefill_kernel(RowMeta *meta, int R, int seq, int pos0) {
+    int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= R) return;
+    RowMeta m;
+    m.seq = seq;
+    m.pos = pos0 + r;
+    m.nk = 0;
+    m.aux = 1;
+    meta[r] = m;
+}
+
+void launch_ctx_meta_prefill(RowMeta *meta, int R, int seq, int pos0, cudaStream_t s) {
+    ctx_meta_prefill_kernel<<<(R + 127) / 128, 128, 0, s>>>(meta, R, seq, pos0);
+}
+
+// ------------------------------------------------------------------------
+// RMSNorm: out = x / sqrt(mean(x^2) + eps) * g   (fp32 statistics)
+// ------------------------------------------------------------------------
+
+template <typename TO>
+__global__ void rmsnorm_kernel(const float *__restrict__ x, int ldx, const float *__restrict__ g,
+                               int H, float eps, TO *__restrict__ out, int ldo) {
+    const int r = blockIdx.x;
+    const float *xr = x + (size_t)r * ldx;
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) ss += xr[c] * xr[c];
+    __shared__ float red[32];
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+        v = warp_sum(v);
+        if (threadIdx.x == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
+    TO *o = out + (size_t)r * ldo;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) o[c] = from_f<TO>(xr[c] * inv * g[c]);
+}
+
+template <typename TO>
+void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, TO *out, int ldo, int R,
+                    cudaStream_t s) {
+    if (R <= 0) return;
+    rmsnorm_kernel<TO><<<R, 256, 0, s>>>(x, ldx, g, H, eps, out, ldo);
+}
+
+// ------------------------------------------------------------------------
+// residual add (+ tap copies), SwiGLU, QKV RoPE + KV write
+// ------------------------------------------------------------------------
+
+template <typename T>
+__global__ void residual_kernel(float *__restrict__ x, const float *__restrict__ Y, int ldy, int H,
+                                TapDst<T> taps, const RowMeta *__restrict__ meta) {
+    const int r = blockIdx.x;
+    float *xr = x + (size_t)r * H;
+    const float *yr = Y + (size_t)r * ldy;
+    const int trow = taps.n ? meta[r].aux : 0;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) {
+        float v = xr[c] + yr[c];
+        xr[c] = v;
+        for (int t = 0; t < taps.n; ++t)
+            taps.base[(size_t)trow * taps.ld + taps.col[t] + c] = from_f<T>(v);
+    }
+}
+
+template <typename T>
+void launch_residual(float *x, const float *Y, int ldy, int H, int R, const TapDst<T> &taps,
+                     const RowMeta *meta, cudaStream_t s) {
+    if (R <= 0) return;
+    residual_kernel<T><<<R, 256, 0, s>>>(x, Y, ldy, H, taps, meta);
+}
+
+template <typename T>
+__global__ void swiglu_kernel(const float *__restrict__ Y, int ldy, int F, T *__restrict__ h, int ldh) {
+    const int r = blockIdx.y;
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= F) return;
+    const float gt = Y[(size_t)r * ldy + c], up = Y[(size_t)r * ldy + F + c];
+    h[(size_t)r * ldh + c] = from_f<T>(silu_f(gt) * up);
+}
+
+template <typename T>
+void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, cudaStream_t s) {
+    if (R <= 0) return;
+    dim3 grid((F + 255) / 256, R);
+    swiglu_kernel<T><<<grid, 256, 0, s>>>(Y, ldy, F, h, ldh);
+}
+
+// Y columns c correspond to rows col0 + c of the layer's Wqkv = [Wq; Wk; Wv].
+// Block rows (r < R_blk): q -> RoPE -> q_out; k -> RoPE -> kc; v -> vc at meta.pos.
+// Context rows (r >= R_blk): k -> RoPE -> kc; v -> vc at ctx_meta.pos when ctx_meta.aux.
+template <typename T>
+__global__ void qkv_epilogue_kernel(const float *__restrict__ Y, int ldy, int col0, int R_blk,
+                                    const RowMeta *__restrict__ meta, const RowMeta *__restrict__ ctx_meta,
+                                    int nq, int nkv, int hd, const float2 *__restrict__ rope,
+                                    T *__restrict__ q_out, T *__restrict__ kc, T *__restrict__ vc,
+                                    int max_len) {
+    const int r = blockIdx.x;
+    const bool is_ctx = r >= R_blk;
+    RowMeta m = is_ctx ? ctx_meta[r - R_blk] : meta[r];
+    if (is_ctx && !m.aux) return;
+    const int qd = nq * hd, kd = nkv * hd, half = hd / 2;
+    const float *y = Y + (size_t)r * ldy - col0;   // y[c] for global Wqkv row c
+    const float2 *tab = rope + (size_t)m.pos * half;
+    const int c_begin = is_ctx ? qd : 0;
+    // RoPE pairs over q and k heads
+    for (int e = threadIdx.x; e < (nq + nkv) * half; e += blockDim.x) {
+        const int head = e / half, i = e % half;
+        if (head < nq && is_ctx) continue;
+        const int base = head * hd;  // q heads then k heads (k starts at qd)
+        const float x1 = y[base + i], x2 = y[base + i + half];
+        const float2 cs = tab[i];
+        const float o1 = x1 * cs.x - x2 * cs.y, o2 = x2 * cs.x + x1 * cs.y;
+        if (head < nq) {
+            q_out[(size_t)r * qd + base + i] = from_f<T>(o1);
+            q_out[(size_t)r * qd + base + i + half] = from_f<T>(o2);
+        } else {
+            const int kh = head - nq;
+            T *dst = kc + (((size_t)m.seq * nkv + kh) * max_len + m.pos) * hd;
+            dst[i] = from_f<T>(o1);
+            dst[i + half] = from_f<T>(o2);
+        }
+    }
+    (void)c_begin;
+    for (int e = threadIdx.x; e < kd; e += blockDim.x) {
+        const int kh = e / hd, d = e % hd;
+        T *dst = vc + (((size_t)m.seq * nkv + kh) * max_len + m.pos) * hd;
+        dst[d] = from_f<T>(y[qd + kd + e]);
+    }
+}
+
+template <typename T>
+void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot, const RowMeta *meta,
+                         const RowMeta *ctx_meta, int nq, int nkv, int hd, const float2 *rope, T *q_out,
+                         T *kc, T *vc, int max_len, cudaStream_t s) {
+    if (R_tot <= 0) return;
+    qkv_epilogue_kernel<T><<<R_tot, 128, 0, s>>>(Y, ldy, col0, R_blk, meta, ctx_meta, nq, nkv, hd, rope,
+                                                 q_out, kc, vc, max_len);
+}
+
+// ------------------------------------------------------------------------
+// greedy heads
+// ------------------------------------------------------------------------
+
+__global__ void argmax_rows_kernel(const float *__restrict__ logits, int64_t ldl, int V, int mode, int B,
+                                   int *__restrict__ idx, DevStats *stats) {
+    const int r = blockIdx.x;
+    if (mode == 1 && (r % B) == 0) return;
+    const float *l = logits + (size_t)r * ldl;
+    float best = -INFINITY;
+    int bi = 0x7fffffff;
+    bool bad = false;
+    for (int c = threadIdx.x; c < V; c += blockDim.x) {
+        float v = l[c];
+        if (!isfinite(v)) bad = true;
+        argmax_merge(best, bi, v, c);
+    }
+    __shared__ float sv[32];
+    __shared__ int si[32];
+    for (int o = 16; o > 0; o >>= 1) {
+        float v2 = __shfl_xor_sync(0xffffffffu, best, o);
+        int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+        argmax_merge(best, bi, v2, i2);
+    }
+    if ((threadIdx.x & 31) == 0) { sv[threadIdx.x >> 5] = best; si[threadIdx.x >> 5] = bi; }
+    if (bad && stats) atomicOr(&stats->status, 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        best = sv[0];
+        bi = si[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) argmax_merge(best, bi, sv[w], si[w]);
+        if (bi >= V) bi = 0;
+        if (mode == 0) idx[r] = bi;
+        else idx[(r / B) * (B - 1) + (r % B) - 1] = bi;
+    }
+}
+
+void launch_argmax_rows(const float *logits, int64_t ldl, int V, int R, int mode, int B, int *idx,
+                        DevStats *stats, cudaStream_t s) {
+    if (R <= 0) return;
+    argmax_rows_kernel<<<R, 512, 0, s>>>(logits, ldl, V, mode, B, idx, stats);
+}
+
+// ------------------------------------------------------------------------
+// accept + commit (greedy, lossless) and token scripts
+// ------------------------------------------------------------------------
+
+__global__ void accept_kernel(SeqState *st, const int *__restrict__ active, int nseq, int B,
+                              const int *__restrict__ drafts, const int *__restrict__ g, int *accept,
+                              int *committed, int *new_len, int *out_tok, int out_ld, DevStats *stats) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nseq) return;
+    const int s = active[i];
+    SeqState S = st[s];
+    const int *d = drafts + i * (B - 1);
+    const int *gi = g + i * B;
+    int a = 0;
+    if (!S.done)
+        while (a < B - 1 && d[a] == gi[a]) ++a;
+    if (committed)
+        for (int k = 0; k < B; ++k) committed[i * B + k] = (k < a) ? d[k] : (k == a ? gi[a] : -1);
+    if (!S.done) {
+        int emitted = 0;
+        for (int k = 0; k <= a; ++k) {
+            const int tok = (k < a) ? d[k] : gi[a];
+            if (S.n_out < S.max_new) {
+                out_tok[(size_t)s * out_ld + S.n_out] = tok;
+                S.n_out++;
+                emitted++;
+            }
+        }
+        S.anchor = gi[a];
+        if (S.n_out >= S.max_new) {
+            S.done = 1;
+            S.pend_n = 0;
+            if (stats) atomicAdd(&stats->n_done, 1);
+        } else {
+            S.pend_pos0 = S.len;
+            S.pend_n = a + 1;
+            S.len += a + 1;
+        }
+        if (stats) {
+            atomicAdd(&stats->iterations, 1ull);
+            atomicAdd(&stats->tokens, (unsigned long long)emitted);
+            atomicAdd(&stats->hist[a], 1ull);
+        }
+        st[s] = S;
+    }
+    if (accept) accept[i] = a;
+    if (new_len) new_len[i] = S.len;
+}
+
+void launch_accept(SeqState *st, const int *active, int nseq, int B, const int *drafts, const int *g,
+                   int *accept, int *committed, int *new_len, int *out_tok, int out_ld, DevStats *stats,
+                   cudaStream_t s) {
+    accept_kernel<<<(nseq + 127) / 128, 128, 0, s>>>(st, active, nseq, B, drafts, g, accept, committed,
+                                                     new_len, out_tok, out_ld, stats);
+}
+
+__global__ void script_drafts_kernel(const SeqState *st, const int *__restrict__ active, int nseq, int B,
+                                     int tau, int V, const int *__restrict__ script, int script_ld,
+                                     int *drafts) {
+    const int i = blockIdx.x;
+    const int k = threadIdx.x;
+    if (i >= nseq || k >= B - 1) return;
+    const int s = active[i];
+    int idx = st[s].n_out + k;
+    if (idx >= script_ld) idx = script_ld - 1;
+    int tok = script[(size_t)s * script_ld + idx];
+    if (k == tau - 1) tok = (tok + 1) % V;
+    drafts[i * (B - 1) + k] = tok;
+}
+
+void launch_script_drafts(const SeqState *st, const int *active, int nseq, int B, int tau, int V,
+                          const int *script, int script_ld, int *drafts, cudaStream_t s) {
+    if (B <= 1 || nseq <= 0) return;
+    script_drafts_kernel<<<nseq, 32 * ((B + 30) / 32), 0, s>>>(st, active, nseq, B, tau, V, script,
+                                                               script_ld, drafts);
+}
+
+__global__ void prefill_finish_kernel(SeqState *st, int seq, int n, const int *first_tok, int *out_tok,
+                                      int out_ld, int max_new) {
+    SeqState S;
+    S.len = n;
+    S.anchor = *first_tok;
+    S.ctx_len = n;
+    S.pend_pos0 = n;
+    S.pend_n = 0;
+    S.n_out = max_new > 0 ? 1 : 0;
+    S.max_new = max_new;
+    S.done = max_new <= 1 ? 1 : 0;
+    if (max_new > 0) out_tok[(size_t)seq * out_ld] = S.anchor;
+    st[seq] = S;
+}
+
+void launch_prefill_finish(SeqState *st, int seq, int n, const int *first_tok, int *out_tok, int out_ld,
+                           int max_new, cudaStream_t s) {
+    prefill_finish_kernel<<<1, 1, 0, s>>>(st, seq, n, first_tok, out_tok, out_ld, max_new);
+}
+
+// target-only greedy step: g is the argmax of the single row of each sequence
+__global__ void ar_step_kernel(SeqState *st, const int *__restrict__ active, int nseq, const int *g,
+                               int *out_tok, int out_ld, DevStats *stats) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nseq) return;
+    const int s = active[i];
+    SeqState S = st[s];
+    if (S.done) return;
+    const int tok = g[i];
+    out_tok[(size_t)s * out_ld + S.n_out] = tok;
+    S.n_out++;
+    S.anchor = tok;
+    if (S.n_out >= S.max_new) {
+        S.done = 1;
+        if (stats) atomicAdd(&stats->n_done, 1);
+    } else {
+        S.len += 1;
+    }
+    st[s] = S;
+}
+
+void launch_ar_step(SeqState *st, const int *active, int nseq, const int *g, int *out_tok, int out_ld,
+                    DevStats *stats, cudaStream_t s) {
+    ar_step_kernel<<<(nseq + 127) / 128, 128, 0, s>>>(st, active, nseq, g, out_tok, out_ld, stats);
+}
+
+// ------------------------------------------------------------------------
+// RoPE table: (cos, sin)(pos * theta^(-2i/hd)), angles in double precision
+// ------------------------------------------------------------------------
+
+__global__ void rope_table_kernel(float2 *tab, int max_len, int hd, double theta) {
+    const int half = hd / 2;
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= (int64_t)max_len * half) return;
+    const int pos = (int)(e / half), i = (int)(e % half);
+    const double freq = pow(theta, -2.0 * (double)i / (double)hd);
+    double sn, cs;
+    sincos((double)pos * freq, &sn, &cs);
+    tab[e] = make_float2((float)cs, (float)sn);
+}
+
+void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStream_t s) {
+    const int64_t n = (int64_t)max_len * (hd / 2);
+    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(tab, max_len, hd, theta);
+}
+
+// ------------------------------------------------------------------------
+// explicit instantiations
+// ------------------------------------------------------------------------
+#define DFL_INST(T)                                                                                         \
+    template void launch_embed_block<T>(const T *, int, SeqState *, const int *, int, int, int, const int *, \
+                                        int, float *, RowMeta *, RowMeta *, cudaStream_t);                  \
+    template void launch_embed_tokens<T>(const T *, int, const int *, int, int, int, float *, RowMeta *,    \
+                                         cudaStream_t);                                                     \
+    template void launch_rmsnorm<T>(const float *, int, const float *, int, float, T *, int, int,           \
+                                    cudaStream_t);                                                          \
+    template void launch_residual<T>(float *, const float *, int, int, int, const TapDst<T> &,              \
+                                     const RowMeta *, cudaStream_t);                                        \
+    template void launch_swiglu<T>(const float *, int, int, int, T *, int, cudaStream_t);                   \
+    template void launch_qkv_epilogue<T>(const float *, int, int, int, int, const RowMeta *,                \
+                                         const RowMeta *, int, int, int, const float2 *, T *, T *, T *,     \
+                                         int, cudaStream_t);
+DFL_INST(float)
+DFL_INST(bf16)
+#undef DFL_INST
+
+}  // namespace dfl
+
+namespace dfl {
+
+// dst rows i*B + j  <-  src rows active[i]*B + j  (16-byte words)
+__global__ void gather_rows_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, size_t row_words,
+                                   const int *__restrict__ active, int B) {
+    const int r = blockIdx.x;
+    const int i = r / B, j = r % B;
+    const uint4 *s = src + ((size_t)active[i] * B + j) * row_words;
+    uint4 *d = dst + (size_t)r * row_words;
+    for (size_t w = threadIdx.x; w < row_words; w += blockDim.x) d[w] = s[w];
+}
+
+void launch_gather_rows(const void *src, void *dst, size_t row_bytes, const int *active, int nseq, int B,
+                        cudaStream_t s) {
+    if (nseq <= 0) return;
+    gather_rows_kernel<<<nseq * B, 256, 0, s>>>((const uint4 *)src, (uint4 *)dst, row_bytes / 16, active, B);
+}
+
+}  // namespace dfl

@@ -1,0 +1,198 @@
+/*
+ * dflash.h -- C ABI of the DFlash block-diffusion draft-and-verify decode
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages about DFlash, cited by title and section):
+ *  - "DFlash: Decodificação Especulativa com Blocos em Paralelo Alcança Até 15x
+ *    Mais Throughput em GPUs Blackwell" (iaemfoco.com), sections "O que o DFlash
+ *    faz de diferente" (a light block-diffusion drafter proposes a whole block
+ *    in one forward pass; the target verifies the whole block in parallel),
+ *    "O alvo sabe mais" (hidden states of several target layers are fused into
+ *    a compact context vector injected into the Key and Value projections of
+ *    every drafter layer, where it persists in the KV cache),
+ *    "Decodificação especulativa tradicional" (accepted tokens are kept; output
+ *    identical to target-only decoding) and "Como usar" (15 speculative tokens).
+ *  - "NVIDIA acelera LLMs autorregressivos em até 15 vezes" (imasters.com.br),
+ *    sections "Como o DFlash troca o drafter por difusão de blocos" and "Os três
+ *    mecanismos por trás do DFlash".
+ *  - "DFlash e Spec V2 revolucionam a speculative decoding" (ceviu.com.br): 16
+ *    tokens per drafter pass, K/V injection into every drafter layer, minimal
+ *    host-device synchronisation.
+ *
+ * Conventions for every entry point:
+ *  - Status codes are returned; no exception crosses the ABI.  Out-parameters
+ *    are written only when DFLASH_OK is returned.  After DFLASH_ECUDA the
+ *    context is unusable and must be destroyed.
+ *  - Host pointers (const int32_t *prompt, int32_t *drafts ...) are ordinary
+ *    host memory owned by the caller.  Calls that return results through host
+ *    pointers synchronise the context's stream, bounded by a host-side timeout
+ *    (DFLASH_ETIMEOUT).
+ *  - Device memory: the caller allocates two device arenas (weights, state) of
+ *    the sizes dflash_workspace_size reports and keeps them alive until
+ *    dflash_destroy.  The library allocates no device memory of its own.
+ *  - All GPU work is enqueued on the CUDA stream given to dflash_create.
+ *  - A context is not thread-safe; use one context per host thread.
+ */
+#ifndef DFLASH_H
+#define DFLASH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dflash_ctx dflash_ctx;
+
+typedef enum {
+    DFLASH_OK = 0,
+    DFLASH_EINVAL = 1,     /* bad argument (null pointer, size out of range, unknown name) */
+    DFLASH_ESTATE = 2,     /* call out of order (verify without draft, sequence not prefilled) */
+    DFLASH_ECAPACITY = 3,  /* a sequence would exceed max_len / a batch exceeds max_batch */
+    DFLASH_ECUDA = 4,      /* a CUDA call failed; the context must be destroyed */
+    DFLASH_ENUMERIC = 5,   /* a non-finite value reached an argmax (device status word) */
+    DFLASH_ETIMEOUT = 6,   /* the stream did not finish within the host-side timeout */
+    DFLASH_EUNSUPPORTED = 7/* shape the kernels do not support (e.g. head_dim not 64/128) */
+} dflash_status;
+
+enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1 };
+
+/* Draft modes.  MODEL: drafts are the drafter's argmax.  SCRIPT: the drafter
+ * still runs in full, then its drafts are replaced from a per-sequence token
+ * script (dflash_set_script): drafts d_1..d_{tau-1} are taken from the script
+ * and d_tau is made wrong ((script+1) mod vocab), so each iteration commits
+ * exactly tau tokens when the script is the target's own greedy continuation.
+ * tau = block_size makes every draft come from the script. */
+enum { DFLASH_DRAFT_MODEL = 0, DFLASH_DRAFT_SCRIPT = 1 };
+
+#define DFLASH_MAX_TAPS 8
+#define DFLASH_MAX_BLOCK 16
+
+typedef struct {
+    int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+    int32_t n_experts, top_k, expert_ffn;   /* n_experts == 0: dense SwiGLU FFN */
+    double rms_eps, rope_theta;
+} dflash_model_cfg;
+
+typedef struct {
+    dflash_model_cfg target;      /* the model whose greedy output is reproduced */
+    dflash_model_cfg drafter;     /* dense; drafter.vocab == target.vocab, same hidden */
+    int32_t block_size;           /* B in [1, 16]: anchor + (B-1) drafted tokens */
+    int32_t n_taps;               /* target layers whose outputs feed the context vector */
+    int32_t tap_layers[DFLASH_MAX_TAPS];
+    int32_t mask_token_id;        /* id embedded at block positions 1..B-1 */
+    int32_t max_batch;            /* sequences held at once */
+    int32_t max_len;              /* positions per sequence (prompt + generated + B) */
+    int32_t prefill_chunk;        /* prompt rows per prefill pass (0: default 1024) */
+    int32_t dtype;                /* DFLASH_FP32 or DFLASH_BF16 (weights, KV, GEMM inputs) */
+    int32_t keep_logits;          /* 1: keep fp32 logits of the last draft/verify for dflash_debug_logits */
+    int32_t timeout_ms;           /* host wait bound for synchronising calls (0: 600000) */
+} dflash_config;
+
+typedef struct {
+    int64_t iterations;           /* draft+verify iterations run */
+    int64_t tokens;               /* tokens emitted after the prompt, all sequences */
+    int64_t accept_hist[DFLASH_MAX_BLOCK];  /* histogram of a (tokens committed - 1) */
+    double mean_tau;              /* tokens committed per sequence-iteration */
+    double ms_prefill, ms_decode; /* device time of the prefill and decode phases */
+} dflash_stats;
+
+/* Bytes of the weight and state arenas for this configuration.
+ * Errors: DFLASH_EINVAL on inconsistent configuration, DFLASH_EUNSUPPORTED on
+ * shapes the kernels do not implement. */
+dflash_status dflash_workspace_size(const dflash_config *cfg, size_t *weight_bytes, size_t *state_bytes);
+
+/* Create a context on the current CUDA device.  weight_arena/state_arena are
+ * device pointers (256-byte aligned) of at least the sizes reported above;
+ * cuda_stream is a cudaStream_t (NULL = legacy default stream).  Builds the
+ * RoPE tables and tensor descriptors; weights may be loaded afterwards. */
+dflash_status dflash_create(const dflash_config *cfg, void *weight_arena, size_t weight_bytes,
+                            void *state_arena, size_t state_bytes, void *cuda_stream,
+                            dflash_ctx **out);
+
+void dflash_destroy(dflash_ctx *ctx);
+
+/* Last error message of the context (owned by ctx, valid until the next call). */
+const char *dflash_last_error(const dflash_ctx *ctx);
+
+/* Weight tensors: names, shapes, storage.  Tensors are row-major and live at
+ * byte `offset` of the weight arena.  Matrices use cfg.dtype storage, RMSNorm
+ * gains are always fp32.  Names:
+ *   embed [V,H], lm_head [V,H] (both shared by the drafter),
+ *   {target|drafter}.L{l}.attn_norm [H], .wqkv [(nq+2nkv)*hd, H] (rows Wq;Wk;Wv),
+ *   .wo [H, nq*hd], .ffn_norm [H], .w_gate_up [2F, H] (rows W_gate;W_up),
+ *   .w_down [H, F]; MoE layers: .w_router [E,H], .we_gate_up [E,2Fe,H],
+ *   .we_down [E,H,Fe]; {target|drafter}.final_norm [H];
+ *   fuse.w_fc [H, n_taps*H], fuse.norm [H]. */
+int32_t dflash_weight_count(const dflash_ctx *ctx);
+dflash_status dflash_weight_info(const dflash_ctx *ctx, int32_t index, const char **name,
+                                 size_t *offset, size_t *numel, int32_t *dtype,
+                                 int32_t *ndim, int64_t *shape /* [3] */);
+dflash_status dflash_weight_slot(const dflash_ctx *ctx, const char *name, size_t *offset,
+                                 size_t *numel, int32_t *dtype);
+
+/* Prefill sequence slot `seq` with prompt[0..n): target causal forward over
+ * the prompt (KV cache positions 0..n-1), taps fused into the drafter's
+ * context K/V for the same positions, first greedy token returned (it is the
+ * anchor of the first block).  Resets the slot.
+ * Errors: EINVAL (seq out of range, n < 1, ids out of vocab), ECAPACITY
+ * (n + block_size > max_len). */
+dflash_status dflash_prefill(dflash_ctx *ctx, int32_t seq, const int32_t *prompt, int32_t n,
+                             int32_t *first_token);
+
+/* One drafter forward for the listed sequences (seqs[0..n), distinct, each
+ * prefilled): block [anchor, mask x (B-1)] at positions p..p+B-1 attends
+ * bidirectionally over the context K/V [0, p) and the block itself.
+ * drafts: host [n*(B-1)] or NULL (then nothing is copied and the call does not
+ * synchronise).  Errors: EINVAL, ESTATE, ECAPACITY. */
+dflash_status dflash_draft_block(dflash_ctx *ctx, const int32_t *seqs, int32_t n, int32_t *drafts);
+
+/* Target verify of [anchor, d_1..d_{B-1}] for the same sequences as the last
+ * dflash_draft_block (drafts == NULL: use the drafter's; else host [n*(B-1)]
+ * supplied by the caller), greedy acceptance a = longest prefix with
+ * d_i == g_{i-1}, commit of d_1..d_a and the bonus g_a, KV rollback by length.
+ * accept [n], committed [n*B] (first a+1 valid), new_len [n]: host or NULL.
+ * Errors: EINVAL, ESTATE (no preceding draft for these sequences). */
+dflash_status dflash_verify_commit(dflash_ctx *ctx, const int32_t *seqs, int32_t n,
+                                   const int32_t *drafts, int32_t *accept, int32_t *committed,
+                                   int32_t *new_len);
+
+/* Whole generation: prefill each of n prompts into slots 0..n-1, then
+ * draft/verify iterations until every sequence holds exactly max_new tokens
+ * after its prompt (no EOS).  out: host [n*max_new].  stats: nullable. */
+dflash_status dflash_generate(dflash_ctx *ctx, const int32_t *const *prompts, const int32_t *prompt_lens,
+                              int32_t n, int32_t max_new, int32_t *out, dflash_stats *stats);
+
+/* Target-only greedy decoding on the same context (slots 0..n-1): prefill,
+ * then one target row per step.  Used for speedup baselines and scripts. */
+dflash_status dflash_generate_ar(dflash_ctx *ctx, const int32_t *const *prompts, const int32_t *prompt_lens,
+                                 int32_t n, int32_t max_new, int32_t *out, double *ms_decode);
+
+/* Draft mode and token scripts (see DFLASH_DRAFT_SCRIPT). tau in [1, B]. */
+dflash_status dflash_set_draft_mode(dflash_ctx *ctx, int32_t mode, int32_t tau);
+/* script[i] is the token expected at output index i of slot `seq` (index 0 =
+ * first token after the prompt); n <= max_len. */
+dflash_status dflash_set_script(dflash_ctx *ctx, int32_t seq, const int32_t *script, int32_t n);
+
+/* fp32 logits of the last pass (needs keep_logits): which = 0 drafter rows
+ * [n_seqs][B][V] (row 0 of each block is the anchor row), 1 verify rows
+ * [n_seqs][B][V], 2 last prefill row [V].  host_out sized accordingly;
+ * rows_out receives the number of rows copied. */
+dflash_status dflash_debug_logits(dflash_ctx *ctx, int32_t which, float *host_out, int64_t capacity,
+                                  int64_t *rows_out);
+
+/* Sequence state of slot seq: length (valid target KV positions = position of
+ * the anchor), anchor token, tokens emitted after the prompt. */
+dflash_status dflash_seq_state(dflash_ctx *ctx, int32_t seq, int32_t *len, int32_t *anchor,
+                               int32_t *n_out);
+
+/* Copy the target (which=0) or drafter (which=1) K and V of one layer, sequence
+ * and position range [p0, p0+n) to host fp32 buffers [n][n_kv*hd] each. */
+dflash_status dflash_debug_kv(dflash_ctx *ctx, int32_t which, int32_t layer, int32_t seq,
+                              int32_t p0, int32_t n, float *k_out, float *v_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

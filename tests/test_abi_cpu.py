@@ -1,0 +1,83 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad configurations before touching the device."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+import subprocess
+from dataclasses import replace
+
+import pytest
+
+import block_diffusion_speculative_layers_b200 as dfl
+from block_diffusion_speculative_layers_b200.build import build, lib_path
+from synthetic import get_config
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return dfl.load_library()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dflash.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dflash_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_binding_exports():
+    assert _declared() == sorted(dfl.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path()], capture_output=True, text=True, check=True).stdout
+    syms = set(l.split()[-1] for l in out.splitlines() if l.strip())
+    for name in _declared():
+        assert name in syms, name
+        assert getattr(lib, name) is not None
+
+
+def _sizes(cfg, **kw):
+    c = dfl.make_config(cfg, **kw)
+    wb, sb = C.c_size_t(), C.c_size_t()
+    st = dfl.load_library().dflash_workspace_size(C.byref(c), C.byref(wb), C.byref(sb))
+    return st, wb.value, sb.value
+
+
+def test_workspace_size_matches_weight_count(lib):
+    from synthetic.weights import weight_shapes
+    cfg = get_config("tiny")
+    st, wb, sb = _sizes(cfg, max_batch=2, max_len=256)
+    assert st == 0 and sb > 0
+    n = sum(int(__import__("numpy").prod(s)) * (4 if k == "norm" or cfg.dtype == "fp32" else 2)
+            for s, k in weight_shapes(cfg).values())
+    assert n <= wb <= n + 256 * len(weight_shapes(cfg))
+    cfg2 = get_config("qwen3_8b")
+    st, wb2, _ = _sizes(cfg2, max_batch=1, max_len=3000)
+    assert st == 0 and 18.0e9 < wb2 < 19.0e9  # embed + head + 36 + 5 layers + fuse
+
+
+@pytest.mark.parametrize("mutate", [
+    lambda c: c.with_(block_size=0),
+    lambda c: c.with_(block_size=17),
+    lambda c: c.with_(tap_layers=(0, 5)),
+    lambda c: c.with_(mask_token_id=5000),
+    lambda c: c.with_(target=replace(c.target, head_dim=96)),
+    lambda c: c.with_(target=replace(c.target, n_q_heads=3)),
+    lambda c: c.with_(drafter=replace(c.drafter, hidden=128)),
+])
+def test_bad_configs_rejected(lib, mutate):
+    st, _, _ = _sizes(mutate(get_config("tiny")), max_batch=1, max_len=128)
+    assert st == dfl.DFLASH_EINVAL if hasattr(dfl, "DFLASH_EINVAL") else st == 1
+
+
+def test_create_rejects_missing_arenas(lib):
+    c = dfl.make_config(get_config("tiny"), max_batch=1, max_len=128)
+    h = C.c_void_p()
+    assert lib.dflash_create(C.byref(c), None, 0, None, 0, None, C.byref(h)) == 1
+    assert lib.dflash_create(C.byref(c), 256, 1 << 40, 256, 1, None, C.byref(h)) == 1  # too small state arena
+    assert not h.value
