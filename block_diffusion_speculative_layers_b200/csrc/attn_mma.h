@@ -1,18 +1,35 @@
-// attn_mma.h -- tensor-core attention for bf16 models.
+// attn_mma.h -- tensor-core block attention for bf16 models (split-KV).
 #pragma once
+
+#include <algorithm>
 
 #include "kernels.h"
 
 namespace dfl {
 
-template <typename T>
-bool attn_mma_supported(int hd) { (void)hd; return false; }
+// Split-KV scratch: unnormalised partial outputs [parts][hd], (max, sum) [parts][2]
+// with parts = (query tile, q head, split, row), and one arrival counter per
+// (query tile, kv head).
+struct AttnScratch {
+    float *o_part = nullptr;
+    float *ml_part = nullptr;
+    int *sem = nullptr;
+    size_t max_parts = 0;
+    int n_sem = 0;
+};
+
+struct AttnWorkspace {
+    size_t max_parts = 0;
+};
+AttnWorkspace attn_workspace_plan(int max_rows, int nq, int nkv, int max_len, int num_sms);
 
 template <typename T>
-void launch_attention_mma(const T *q, int ldq, const T *kc, const T *vc, const RowMeta *meta, int R, int nq, int nkv,
-                          int hd, int max_len, T *out, int ldo, cudaStream_t s) {
-    (void)q; (void)ldq; (void)kc; (void)vc; (void)meta; (void)R; (void)nq; (void)nkv; (void)hd; (void)max_len;
-    (void)out; (void)ldo; (void)s;
-}
+bool attn_mma_supported(int hd);
+
+// rows_per_tile: rows of one sequence that share a query tile (block size for
+// draft/verify, 16 for prompt rows, 1 for single-row target steps).
+template <typename T>
+void launch_attention_mma(const T *q, int ldq, const T *kc, const T *vc, const RowMeta *meta, int R, int rows_per_tile,
+                          int nq, int nkv, int hd, int max_len, T *out, int ldo, const AttnScratch &ws, cudaStream_t s);
 
 }  // namespace dfl

@@ -178,6 +178,19 @@ static Layout make_layout(const dflash_config &c) {
     L.moe_sel = take(mrows * 4);
     L.moe_wt = take(mrows * 4);
     L.moe_part = take(t.n_experts > 0 ? mrows * H * 4 : 16);
+    // per-(vocab tile, row) best logit of the LM-head GEMM
+    L.lm_part = take((size_t)((t.vocab + 127) / 128) * std::max(L.R_dec, 1) * sizeof(float2));
+    // split-KV attention partials (sized for 148 SMs; launches cap their splits to fit)
+    {
+        const int nq_max = std::max(t.n_q_heads, d.n_q_heads), nkv_min = std::min(t.n_kv_heads, d.n_kv_heads);
+        const int hd_max = std::max(t.head_dim, d.head_dim);
+        const int tiles = std::max(L.R_dec, (L.C + 15) / 16);
+        AttnWorkspace aw = attn_workspace_plan(tiles, nq_max, nkv_min, c.max_len, 148);
+        L.att_parts = aw.max_parts;
+        L.att_o = take(L.att_parts * hd_max * 4);
+        L.att_ml = take(L.att_parts * 2 * 4);
+        L.att_sem = take((size_t)tiles * std::max(t.n_kv_heads, d.n_kv_heads) * 4);
+    }
     // split-K workspace and tile semaphores of the tensor-core GEMM
     L.ws_floats = gemm_tc_workspace_floats(L.R_max, std::max(ycols, t.vocab > 0 ? H : H));
     L.gemm_ws = take((size_t)L.ws_floats * 4);
@@ -214,6 +227,8 @@ class Engine : public EngineBase {
     DevStats *stats;
     float *gemm_ws;
     int *gemm_sem;
+    float2 *lm_part;
+    AttnScratch att;
     GemmTC<T> tc;
     // host mirrors
     std::vector<int> h_len, h_prefilled;
@@ -299,6 +314,12 @@ class Engine : public EngineBase {
         stats = sp<DevStats>(L.stats);
         gemm_ws = sp<float>(L.gemm_ws);
         gemm_sem = sp<int>(L.gemm_sem);
+        lm_part = sp<float2>(L.lm_part);
+        att.o_part = sp<float>(L.att_o);
+        att.ml_part = sp<float>(L.att_ml);
+        att.sem = sp<int>(L.att_sem);
+        att.max_parts = L.att_parts;
+        att.n_sem = std::max(L.R_dec, (L.C + 15) / 16) * std::max(c.target.n_kv_heads, c.drafter.n_kv_heads);
         h_len.assign(c.max_batch, 0);
         h_prefilled.assign(c.max_batch, 0);
         // zero the whole state arena once: stale taps / KV never hold NaN bit patterns
@@ -312,6 +333,9 @@ class Engine : public EngineBase {
             err = "tensor-core GEMM set-up failed: " + tc.err;
             return DFLASH_ECUDA;
         }
+        tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
+        tc.set_err(&stats->status);
+        tc.keep_logits = c.keep_logits;
         return check("create");
     }
 
@@ -388,20 +412,19 @@ class Engine : public EngineBase {
         }
     }
 
-    void attention(const T *qq, const T *kc, const T *vc, const RowMeta *mt, int R, const dflash_model_cfg &m,
-                   T *out) {
+    void attention(const T *qq, const T *kc, const T *vc, const RowMeta *mt, int R, int rows_per_tile,
+                   const dflash_model_cfg &m, T *out) {
         const int qd = m.n_q_heads * m.head_dim;
         if (attn_mma_supported<T>(m.head_dim)) {
-            launch_attention_mma<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out,
-                                    qd, s);
+            launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads, m.head_dim,
+                                    c.max_len, out, qd, att, s);
             return;
         }
-        launch_attention_simt<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out,
-                                 qd, s);
+        launch_attention_simt<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out, qd, s);
     }
 
     // one pre-norm decoder layer of the target over R rows in x (meta)
-    void target_layer(int l, int R, const RowMeta *mt, T *tap_base, int tap_ld) {
+    void target_layer(int l, int R, int rpt, const RowMeta *mt, T *tap_base, int tap_ld) {
         const dflash_model_cfg &m = c.target;
         const LayerW &w = tl[l];
         const int H = m.hidden, hd = m.head_dim, qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd;
@@ -419,7 +442,7 @@ class Engine : public EngineBase {
         e.kc = tk + (size_t)l * kv_layer_elems(m);
         e.vc = tv + (size_t)l * kv_layer_elems(m);
         gemm(xn, H, R, w.wqkv, qd + 2 * kd, H, e);
-        attention(q, e.kc, e.vc, mt, R, m, ao);
+        attention(q, e.kc, e.vc, mt, R, rpt, m, ao);
         Epi<T> r;
         r.kind = EPI_RESID;
         r.x = x;
@@ -490,7 +513,7 @@ class Engine : public EngineBase {
         e.vc = dv + (size_t)j * kv_layer_elems(m);
         // block rows and context rows share one pass over Wqkv (K/V injection)
         gemm(dq_in, H, with_ctx ? 2 * R : R, w.wqkv, qd + 2 * kd, H, e);
-        attention(q, e.kc, e.vc, meta, R, m, ao);
+        attention(q, e.kc, e.vc, meta, R, c.block_size, m, ao);
         Epi<T> r;
         r.kind = EPI_RESID;
         r.x = x;
@@ -509,14 +532,23 @@ class Engine : public EngineBase {
         gemm(h, m.ffn, R, w.w_down, H, m.ffn, dn);
     }
 
-    void lm_head_rows(const float *final_norm, float eps, int R, float *lg, int64_t ldl) {
-        const int H = c.target.hidden;
-        launch_rmsnorm<T>(x, H, final_norm, H, eps, xn, H, R, s);
+    // LM head on normalised rows xin[R][H] -> greedy ids (mode 0: idx[r];
+    // mode 1: drafter rows j >= 1 of each block -> idx[i*(B-1)+j-1]).
+    void head_argmax(const T *xin, int R, float *lg, int mode, int B, int *idx) {
+        const int H = c.target.hidden, V = c.target.vocab;
         Epi<T> e;
         e.kind = EPI_LOGITS;
         e.Y = lg;
-        e.ldy = (int)ldl;
-        gemm(xn, H, R, lm_head, c.target.vocab, H, e);
+        e.ldy = V;
+        gemm(xin, H, R, lm_head, V, H, e);
+        if (tc.supports(R, V, H)) launch_lm_argmax(lm_part, (V + 127) / 128, R, mode, B, idx, stats, s);
+        else launch_argmax_rows(lg, V, V, R, mode, B, idx, stats, s);
+    }
+
+    void lm_head_rows(const float *final_norm, float eps, int R, float *lg, int mode, int B, int *idx) {
+        const int H = c.target.hidden;
+        launch_rmsnorm<T>(x, H, final_norm, H, eps, xn, H, R, s);
+        head_argmax(xn, R, lg, mode, B, idx);
     }
 
     // ---- steps ----
@@ -527,16 +559,11 @@ class Engine : public EngineBase {
         for (int c0 = 0; c0 < n; c0 += L.C) {
             const int R = std::min(L.C, n - c0);
             launch_embed_tokens<T>(embed, H, tokens + c0, R, seq, c0, x, meta, s);
-            for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, meta, taps_pre, TK);
+            for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, 16, meta, taps_pre, TK);
             if (c0 + R == n) {
                 // greedy first token from the last prompt row
                 launch_rmsnorm<T>(x + (size_t)(R - 1) * H, H, t_final, H, (float)t.rms_eps, xn, H, 1, s);
-                Epi<T> e;
-                e.kind = EPI_LOGITS;
-                e.Y = plogits;
-                e.ldy = t.vocab;
-                gemm(xn, H, 1, lm_head, t.vocab, H, e);
-                launch_argmax_rows(plogits, t.vocab, t.vocab, 1, 0, 1, first_tok, stats, s);
+                head_argmax(xn, 1, plogits, 0, 1, first_tok);
             }
             // context vectors of the prompt rows -> drafter context K/V
             Epi<T> f;
@@ -583,8 +610,7 @@ class Engine : public EngineBase {
         gemm(tin, TK, R, w_fc, H, TK, f);
         launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, dq_in + (size_t)R * H, H, R, s);
         for (int j = 0; j < d.n_layers; ++j) drafter_layer(j, R, true);
-        lm_head_rows(d_final, (float)d.rms_eps, R, logits, t.vocab);
-        if (B > 1) launch_argmax_rows(logits, t.vocab, t.vocab, R, 1, B, drafts, stats, s);
+        if (B > 1) lm_head_rows(d_final, (float)d.rms_eps, R, logits, 1, B, drafts);
         if (draft_mode == DFLASH_DRAFT_SCRIPT)
             launch_script_drafts(st, active, nseq, B, tau, t.vocab, script, c.max_len, drafts, s);
     }
@@ -593,9 +619,8 @@ class Engine : public EngineBase {
         const dflash_model_cfg &t = c.target;
         const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
         launch_embed_block<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
-        for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, meta, taps_dec, TK);
-        lm_head_rows(t_final, (float)t.rms_eps, R, logits, t.vocab);
-        launch_argmax_rows(logits, t.vocab, t.vocab, R, 0, B, g, stats, s);
+        for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, B, meta, taps_dec, TK);
+        lm_head_rows(t_final, (float)t.rms_eps, R, logits, 0, B, g);
         launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
     }
 
@@ -603,9 +628,8 @@ class Engine : public EngineBase {
         const dflash_model_cfg &t = c.target;
         const int H = t.hidden;
         launch_embed_block<T>(embed, H, st, active, nseq, 1, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
-        for (int l = 0; l < t.n_layers; ++l) target_layer(l, nseq, meta, nullptr, 0);
-        lm_head_rows(t_final, (float)t.rms_eps, nseq, logits, t.vocab);
-        launch_argmax_rows(logits, t.vocab, t.vocab, nseq, 0, 1, g, stats, s);
+        for (int l = 0; l < t.n_layers; ++l) target_layer(l, nseq, 1, meta, nullptr, 0);
+        lm_head_rows(t_final, (float)t.rms_eps, nseq, logits, 0, 1, g);
         launch_ar_step(st, active, nseq, g, out_tok, c.max_len, stats, s);
     }
 

@@ -33,7 +33,8 @@ struct Layout {
     size_t x, xn, dq_in, Y, q, ao, h, taps_dec, taps_gather, taps_pre, cbuf, logits, plogits;
     size_t g, drafts, accept, committed, new_len, st, active, meta, ctx_meta, ctx_meta_pre;
     size_t rope_t, rope_d, tk, tv, dk, dv, script, out_tok, tokens, stats, first_tok;
-    size_t moe_sel, moe_wt, moe_part;
+    size_t moe_sel, moe_wt, moe_part, lm_part, att_o, att_ml, att_sem;
+    size_t att_parts = 0;
     size_t gemm_ws, gemm_sem;
     size_t state_bytes = 0;
     // dims

@@ -1,7 +1,16 @@
-// gemm_tc.h -- tensor-core (tcgen05) weight-streaming projection for bf16 models.
+// gemm_tc.h -- tensor-core (tcgen05 + TMEM + TMA) weight-streaming projection
+// for bf16 models.
+//
+// Y[M][N] = X[M][K] . W[N][K]^T is computed "swap-AB": the weight tile is the
+// 128-row A operand and the few activation rows (M = batch x block) are the
+// N operand of tcgen05.mma, so a 16-row decode step still runs on the tensor
+// cores while W streams through shared memory exactly once.
 #pragma once
 
+#include <cuda.h>
+
 #include <string>
+#include <unordered_map>
 
 #include "kernels.h"
 
@@ -10,27 +19,50 @@ namespace dfl {
 int gemm_tc_workspace_floats(int max_rows, int max_n);
 int gemm_tc_semaphores();
 
-template <typename T>
-struct GemmTC {
-    std::string err;
-    int init(float *ws, int ws_floats, int *sem, int n_sem) {
-        (void)ws; (void)ws_floats; (void)sem; (void)n_sem;
-        return 0;
-    }
-    bool supports(int M, int N, int K) const { (void)M; (void)N; (void)K; return false; }
-    void run(const T *X, int ldx, int M, const T *W, int N, int K, const Epi<T> &e, cudaStream_t s) {
-        (void)X; (void)ldx; (void)M; (void)W; (void)N; (void)K; (void)e; (void)s;
-    }
+// Launch parameters shared by host and device.
+struct TcParams {
+    int M, N, K;            // logical sizes (N = 2F for SwiGLU)
+    int n_tiles, m_tiles;   // tiles of 128 weight rows (64 output columns for SwiGLU) x TM rows
+    int k_steps, splits;    // 64-wide K steps in total; K splits
+    int swiglu_F;           // SwiGLU: rows [0,F) gate, [F,2F) up; else 0
+    float *ws;              // split-K partials
+    int *sem;               // per-tile arrival counters (self-resetting)
+    int *err;               // device error word (bounded waits)
+    float2 *lm_part;        // EPI_LOGITS: per (n_tile, row) best (value, index)
+    int keep_logits;        // EPI_LOGITS: also store fp32 logits in Y
 };
 
 template <typename T>
-bool moe_tc_supported() { return false; }
+struct GemmTC {
+    std::string err;
+    bool supports(int M, int N, int K) const;
+    int init(float *ws, int ws_floats, int *sem, int n_sem);
+    void run(const T *X, int ldx, int M, const T *W, int N, int K, const Epi<T> &e, cudaStream_t s);
+    // LM-head partial argmax buffer (value, index as float bits), [n_tiles][rows]
+    void set_lm_part(float2 *p, int cap) { lm_part = p; lm_cap = cap; }
+    void set_err(int *e) { err_word = e; }
+    float2 *lm_part = nullptr;
+    int lm_cap = 0;
+    int keep_logits = 0;
+    float *ws = nullptr;
+    int ws_floats = 0;
+    int *sem = nullptr;
+    int n_sem = 0;
+    int *err_word = nullptr;
+    int num_sms = 148;
+    std::unordered_map<std::string, CUtensorMap> maps;
+    const CUtensorMap *tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows);
+};
+
+// Row-wise argmax over the LM-head partials: mode 0 idx[r]; mode 1 drafter rows.
+void launch_lm_argmax(const float2 *part, int n_tiles, int R, int mode, int B, int *idx, DevStats *stats,
+                      cudaStream_t s);
+
+template <typename T>
+bool moe_tc_supported();
 
 template <typename T>
 void run_moe_tc(const T *m, int ldm, int R, int k, const int *sel, const T *w_gate_up, const T *w_down, int H,
-                int Fe, int E, T *h, float *part, GemmTC<T> &tc, cudaStream_t s) {
-    (void)m; (void)ldm; (void)R; (void)k; (void)sel; (void)w_gate_up; (void)w_down; (void)H; (void)Fe; (void)E;
-    (void)h; (void)part; (void)tc; (void)s;
-}
+                int Fe, int E, T *h, float *part, GemmTC<T> &tc, cudaStream_t s);
 
 }  // namespace dfl
