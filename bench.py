@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""DFlash draft-and-verify decode benchmark on one or more B200s.
+
+One step = one decode iteration of the whole hot path for every sequence of
+the batch: context fuse + K/V injection, the 5-layer block-bidirectional
+drafter pass and its LM-head argmax, the 36-layer causal verify pass, the
+target LM-head argmax and the accept/commit step.  Workload: Qwen3-8B-shaped
+target with a 5-layer block-16 drafter, bf16 random-init weights N(0, 0.02),
+batch 1 per GPU, 512-token Zipf(1.1) prompt.  Weights (18.5 GB) exceed the
+126 MB L2, so every step streams them from HBM.
+
+--gpus N runs N independent replicas (one process per GPU; the decode step has
+no collective), and `value` sums their tokens over the slowest replica's time.
+
+Prints one JSON line on stdout.  Progress goes to stderr.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synthetic import get_config, make_prompt, make_weight  # noqa: E402
+from synthetic.weights import weight_shapes  # noqa: E402
+
+METRIC = "generated tokens/s @1×B200 batch 1 (Qwen3-8B shape); µs/iter vs HBM roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={uuid}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception as e:  # no nvidia-smi: report nothing rather than fail the run
+            log("clock sampler unavailable:", e)
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r[0] > 500] or rows
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for nm, flag in zip(names, r[2][1:]):
+                if flag.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ bytes
+def iteration_bytes(cfg, batch: int, mean_ctx: float) -> float:
+    """Algorithmic HBM bytes of one draft+verify iteration: every projection
+    matrix once (the LM head twice: drafter and target), plus K/V reads of both
+    models at the mean context length."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    shapes = weight_shapes(cfg)
+    w = 0
+    for name, (shape, kind) in shapes.items():
+        if kind != "matrix" or name == "embed":
+            continue
+        n = int(np.prod(shape))
+        if name.endswith("we_gate_up") or name.endswith("we_down"):
+            continue  # MoE experts are counted by touched experts elsewhere
+        w += n * es * (2 if name == "lm_head" else 1)
+    t, d = cfg.target, cfg.drafter
+    kv = batch * (mean_ctx + cfg.block_size) * 2 * es * (t.n_layers * t.n_kv_heads * t.head_dim
+                                                          + d.n_layers * d.n_kv_heads * d.head_dim)
+    return float(w * (1 if batch else 0) + kv)
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def cpu_oracle_sample(cfg, prompt_len: int = 16, iters: int = 1, seed: int = 0):
+    """Time the fp64 CPU oracle on a bounded sample of the workload: one
+    draft + verify iteration of the full-size model after a short prompt."""
+    import oracle
+    from synthetic.fast import make_weights_host
+    t0 = time.time()
+    w = make_weights_host(cfg)
+    gen_s = time.time() - t0
+    spec = oracle.OracleSpec(cfg, w)
+    prompt = make_prompt(cfg.prompt_kind, prompt_len, cfg.target.vocab, cfg.seed + seed)
+    ss = spec.session(prompt_len + (iters + 2) * cfg.block_size)
+    t0 = time.time()
+    anchor, _, _ = ss.prefill(prompt)
+    pre_s = time.time() - t0
+    tokens = 0
+    t0 = time.time()
+    for _ in range(iters):
+        d, _, _ = ss.draft(anchor)
+        g, _, _ = ss.verify([anchor] + list(d))
+        a = 0
+        while a < cfg.block_size - 1 and d[a] == g[a]:
+            a += 1
+        ss.commit(a)
+        anchor = int(g[a])
+        tokens += a + 1
+    it_s = time.time() - t0
+    return {"tokens": tokens, "seconds": it_s, "iters": iters, "weight_gen_s": gen_s, "prefill_s": pre_s}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="qwen3_8b")
+    ap.add_argument("--batch", type=int, default=None, help="sequences per GPU (default: the config's)")
+    ap.add_argument("--prompt-len", type=int, default=None)
+    ap.add_argument("--forced", default="1,4,8,16", help="forced accept lengths to time ('' = none)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-tokens", type=int, default=128)
+    ap.add_argument("--target-layers", type=int, default=None, help="layer-reduced copy (profiling small cases)")
+    ap.add_argument("--drafter-layers", type=int, default=None)
+    ap.add_argument("--ref-budget-s", type=float, default=150.0, help="reference arm: cap on timed CPU seconds")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = get_config(args.config)
+    if args.batch:
+        cfg = cfg.with_(batch=args.batch)
+    if args.prompt_len:
+        cfg = cfg.with_(prompt_len=args.prompt_len)
+    if args.target_layers or args.drafter_layers:
+        from synthetic.configs import shrink
+        cfg = shrink(cfg, target_layers=args.target_layers or cfg.target.n_layers,
+                     drafter_layers=args.drafter_layers or cfg.drafter.n_layers)
+
+    if args.impl == "reference":
+        return run_reference(args, cfg, world, rank)
+
+    import block_diffusion_speculative_layers_b200 as dfl
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+        pg = dist
+
+    b, B = cfg.batch, cfg.block_size
+    max_new_cap = (args.warmup + args.steps + 8) * B
+    max_len = cfg.prompt_len + max(max_new_cap, args.e2e_tokens + 2 * B, 2048) + 2 * B
+    log(f"[rank {rank}] building context: {cfg.name} batch {b} max_len {max_len}")
+    ctx = dfl.DFlash(cfg, max_batch=b, max_len=max_len, device=dev)
+    t0 = time.time()
+    ctx.load_weights_from(lambda n: make_weight(cfg, n, device=dev))
+    log(f"[rank {rank}] weights generated + loaded in {time.time() - t0:.1f}s ({ctx.weight_bytes / 1e9:.2f} GB)")
+    prompts = [make_prompt(cfg.prompt_kind, cfg.prompt_len, cfg.target.vocab, cfg.seed + 1000 * rank + i)
+               for i in range(b)]
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill_all():
+        for i, p in enumerate(prompts):
+            ctx.prefill(i, p)
+
+    def timed_iters(k):
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        ctx.reset_stats()
+        l0 = ctx.stats().kernel_launches
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ctx.decode_iters(b, k)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        st = ctx.stats()
+        return e0.elapsed_time(e1), st, st.kernel_launches - l0
+
+    # ---- natural acceptance (the drafter's own argmax) ----
+    t0 = time.time()
+    prefill_all()
+    torch.cuda.synchronize(dev)
+    prefill_s = time.time() - t0
+    ctx.decode_iters(b, args.warmup)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms, st, launches = timed_iters(args.steps)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    tokens = st.tokens
+    ms_max, tok_sum = ms, tokens
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_max = float(t.item())
+        n = torch.tensor([tokens], device=dev, dtype=torch.float64)
+        pg.all_reduce(n)
+        tok_sum = int(n.item())
+    value = tok_sum / (ms_max / 1000.0)
+    mean_tau = st.mean_tau
+    ctx_len_mean = cfg.prompt_len + args.warmup * mean_tau + 0.5 * args.steps * mean_tau
+    it_bytes = iteration_bytes(cfg, b, ctx_len_mean)
+    us_iter = ms_max * 1000.0 / args.steps
+    log(f"[rank {rank}] {args.steps} iters in {ms:.2f} ms: {us_iter:.1f} us/iter, tau {mean_tau:.3f}, "
+        f"{value:.1f} tok/s, launches {launches}")
+
+    # ---- per-kernel roofline: CUDA events around each projection / attention launch ----
+    ctx.profile(True)
+    ctx.decode_iters(b, min(args.steps, 50))
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    pl, pms, pbytes = prof["projection"]
+    al, ams, _ = prof["attention"]
+    peak, peak_kind = hbm_peak()
+    achieved = pbytes / (pms / 1000.0) / 1e9 if pms > 0 else 0.0
+    log(f"[rank {rank}] projections: {pl} launches, {pms:.2f} ms, {pbytes / 1e9:.2f} GB -> {achieved:.0f} GB/s; "
+        f"attention {al} launches {ams:.2f} ms")
+
+    # ---- forced acceptance lengths via a script = the GPU's own target-only continuation ----
+    forced = {}
+    taus = [int(x) for x in args.forced.split(",") if x.strip()] if args.forced else []
+    ar_tps = None
+    if taus:
+        need = (args.warmup + args.steps) * B + 2 * B
+        need = min(need, max_len - cfg.prompt_len - B)
+        ar_out, ar_ms = ctx.generate_ar(prompts, need)
+        ar_tps = b * (need - 1) / (ar_ms / 1000.0) if ar_ms > 0 else None
+        for tau in taus:
+            if tau < 1 or tau > B:
+                continue
+            for i in range(b):
+                ctx.set_script(i, ar_out[i])
+            ctx.set_draft_mode(dfl.DFLASH_DRAFT_SCRIPT, tau)
+            prefill_all()
+            ctx.decode_iters(b, args.warmup)
+            k = max(1, min(args.steps, (need - args.warmup * tau) // max(tau, 1) - 2))
+            fms, fst, _ = timed_iters(k)
+            forced[str(tau)] = {"tokens_per_s": b * 0 + fst.tokens / (fms / 1000.0), "mean_tau": fst.mean_tau,
+                                "us_per_iter": fms * 1000.0 / k, "iters": k}
+            log(f"[rank {rank}] forced tau={tau}: {forced[str(tau)]}")
+        ctx.set_draft_mode(dfl.DFLASH_DRAFT_MODEL, 1)
+
+    # ---- end to end through the public call, host buffers in and out ----
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    host_prompts = [np.ascontiguousarray(p) for p in prompts]
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    out, gst = ctx.generate(host_prompts, args.e2e_tokens)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    e2e_tokens = b * args.e2e_tokens
+    iters_e2e = max(1, gst.iterations // max(1, b))
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * e2e_tokens / (e2e_ms / 1000.0)
+    h2d = sum(p.nbytes for p in host_prompts) + 4 * b
+    d2h = out.nbytes + 4 * (iters_e2e + 2)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        log("[rank 0] timing the CPU oracle on a bounded sample ...")
+        try:
+            s = cpu_oracle_sample(cfg)
+            cpu = {"value": s["tokens"] / s["seconds"], "unit": "tokens/s", "cores": os.cpu_count(),
+                   "kind": "oracle",
+                   "sample": (f"{s['iters']} full-size fp64 draft+verify iteration(s) after a 16-token prompt "
+                              f"({s['seconds']:.1f} s; weight generation {s['weight_gen_s']:.1f} s and prefill "
+                              f"{s['prefill_s']:.1f} s not counted)")}
+        except Exception as e:  # report, do not fail the GPU measurement
+            cpu = {"value": None, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+                   "sample": f"failed: {e}"}
+
+    if rank != 0:
+        if pg:
+            pg.destroy_process_group()
+        return
+    result = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.dtype,
+        "data": "synthetic (counter-based N(0,0.02)-like weights, Zipf(1.1) prompts)",
+        "config": {"workload": f"{cfg.name}: {cfg.target.n_layers}-layer target (hidden {cfg.target.hidden}, "
+                               f"vocab {cfg.target.vocab}) + {cfg.drafter.n_layers}-layer block-{B} drafter, "
+                               f"batch {b} per GPU, {cfg.prompt_len}-token prompt",
+                   "global_batch": b * world, "seq_len": cfg.prompt_len, "block_size": B,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (18.5 GB of weights streamed per step)"},
+        "us_per_iter": round(us_iter, 2),
+        "mean_tau": round(mean_tau, 4),
+        "iter_bytes": it_bytes,
+        "iter_hbm_frac_8tbps": round(it_bytes / (us_iter * 1e-6) / 8e12, 4),
+        "iter_hbm_frac_measured": round(it_bytes / (us_iter * 1e-6) / (peak * 1e9), 4),
+        "forced_tau": forced,
+        "ar_tokens_per_s": round(ar_tps, 2) if ar_tps else None,
+        "prefill_s": round(prefill_s, 3),
+        "gpu_launches": int(launches),
+        "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s", "h2d_bytes_per_step": h2d / iters_e2e,
+                "d2h_bytes_per_step": d2h / iters_e2e,
+                "note": f"dflash_generate: prefill + {args.e2e_tokens} tokens, host prompt in, host tokens out"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "gemm_tc (tcgen05 projections, all launches of one step)",
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6.65 TB/s",
+                     "launches": pl, "ms": round(pms, 3), "bytes": pbytes},
+        "attention_ms_per_step": round(ams / max(1, min(args.steps, 50)), 4),
+        "cpu_baseline": cpu,
+        "clocks": clk,
+    }
+    print(json.dumps(result), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+def run_reference(args, cfg, world, rank):
+    """The reference arm: the fp64 CPU oracle, timed as it stands on the host
+    cores, each step one full-size draft+verify iteration after a short prompt."""
+    if rank != 0:
+        return
+    import oracle
+    from synthetic.fast import make_weights_host
+    t0 = time.time()
+    w = make_weights_host(cfg)
+    log(f"reference: host weights in {time.time() - t0:.1f}s")
+    spec = oracle.OracleSpec(cfg, w)
+    B = cfg.block_size
+    plen = 16
+    prompt = make_prompt(cfg.prompt_kind, plen, cfg.target.vocab, cfg.seed)
+    ss = spec.session(plen + (args.warmup + args.steps + 2) * B)
+    anchor, _, _ = ss.prefill(prompt)
+
+    def step():
+        nonlocal anchor
+        d, _, _ = ss.draft(anchor)
+        g, _, _ = ss.verify([anchor] + list(d))
+        a = 0
+        while a < B - 1 and d[a] == g[a]:
+            a += 1
+        ss.commit(a)
+        anchor = int(g[a])
+        return a + 1
+
+    # the oracle needs no warm-up; one untimed step sizes the time budget
+    t0 = time.time()
+    step()
+    first = time.time() - t0
+    n_steps = max(1, min(args.steps, int(args.ref_budget_s / max(first, 1e-3))))
+    log(f"reference: one step {first:.1f}s -> timing {n_steps} of {args.steps} steps")
+    t0 = time.time()
+    tokens = sum(step() for _ in range(n_steps))
+    sec = time.time() - t0
+    v = tokens / sec
+    res = {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "tokens/s", "n_gpus": world,
+           "steps": n_steps, "warmup": 1, "ms_per_step": round(1000 * sec / n_steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": f"{cfg.name} batch 1, fp64 CPU oracle, 16-token prompt"},
+           "cpu_baseline": {"value": round(v, 5), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+                            "sample": f"{n_steps} full-size draft+verify iterations after a 16-token prompt "
+                                      f"(capped at {args.ref_budget_s:.0f} s of CPU time; {args.steps} requested)"},
+           "e2e": {"value": round(v, 5), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -32,7 +32,8 @@ EXPORTS = [
     "dflash_weight_count", "dflash_weight_info", "dflash_weight_slot", "dflash_prefill",
     "dflash_draft_block", "dflash_verify_commit", "dflash_generate", "dflash_generate_ar",
     "dflash_set_draft_mode", "dflash_set_script", "dflash_debug_logits", "dflash_seq_state",
-    "dflash_debug_kv",
+    "dflash_debug_kv", "dflash_decode_iters", "dflash_get_stats", "dflash_reset_stats",
+    "dflash_profile", "dflash_profile_read",
 ]
 
 
@@ -60,7 +61,12 @@ class Config(C.Structure):
 class Stats(C.Structure):
     _fields_ = [("iterations", C.c_int64), ("tokens", C.c_int64),
                 ("accept_hist", C.c_int64 * MAX_BLOCK), ("mean_tau", C.c_double),
-                ("ms_prefill", C.c_double), ("ms_decode", C.c_double)]
+                ("ms_prefill", C.c_double), ("ms_decode", C.c_double),
+                ("kernel_launches", C.c_int64)]
+
+
+class KernelProf(C.Structure):
+    _fields_ = [("launches", C.c_int64), ("ms", C.c_double), ("bytes", C.c_double)]
 
 
 _lib = None
@@ -98,6 +104,11 @@ def load_library(path: Optional[str] = None):
         "dflash_seq_state": (_i32, [_vp, _i32, _ip, _ip, _ip]),
         "dflash_debug_kv": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, C.POINTER(C.c_float),
                                    C.POINTER(C.c_float)]),
+        "dflash_decode_iters": (_i32, [_vp, _i32, _i32]),
+        "dflash_get_stats": (_i32, [_vp, C.POINTER(Stats)]),
+        "dflash_reset_stats": (_i32, [_vp]),
+        "dflash_profile": (_i32, [_vp, _i32]),
+        "dflash_profile_read": (_i32, [_vp, C.POINTER(KernelProf)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -273,6 +284,42 @@ class DFlash:
         self._check(self.lib.dflash_generate_ar(self.h, ptrs, _iptr(lens), n, max_new, _iptr(out), C.byref(ms)),
                     "dflash_generate_ar")
         return out.reshape(n, max_new), ms.value
+
+    def decode_iters(self, n_seqs: int, iters: int):
+        """Enqueue draft+verify iterations on slots 0..n_seqs-1 (asynchronous)."""
+        self._check(self.lib.dflash_decode_iters(self.h, n_seqs, iters), "dflash_decode_iters")
+
+    def stats(self) -> Stats:
+        st = Stats()
+        self._check(self.lib.dflash_get_stats(self.h, C.byref(st)), "dflash_get_stats")
+        return st
+
+    def reset_stats(self):
+        self._check(self.lib.dflash_reset_stats(self.h), "dflash_reset_stats")
+
+    def profile(self, enable: bool):
+        self._check(self.lib.dflash_profile(self.h, 1 if enable else 0), "dflash_profile")
+
+    def profile_read(self):
+        out = (KernelProf * 2)()
+        self._check(self.lib.dflash_profile_read(self.h, out), "dflash_profile_read")
+        return {"projection": (out[0].launches, out[0].ms, out[0].bytes),
+                "attention": (out[1].launches, out[1].ms, out[1].bytes)}
+
+    def load_weights_from(self, make_one, names=None):
+        """Fill each weight slot from make_one(name) (one tensor alive at a time)."""
+        slots = self.weight_slots()
+        for name in (names or slots):
+            off, numel, dt, shape = slots[name]
+            t = make_one(name)
+            tdt = torch.bfloat16 if dt == DFLASH_BF16 else torch.float32
+            if tuple(t.shape) != shape or t.dtype != tdt:
+                raise ValueError(f"{name}: expected {shape} {tdt}, got {tuple(t.shape)} {t.dtype}")
+            es = 2 if dt == DFLASH_BF16 else 4
+            base = self._woff + off
+            self.warena[base:base + numel * es].view(tdt).view(shape).copy_(t)
+            del t
+        torch.cuda.synchronize(self.device)
 
     def set_draft_mode(self, mode: int, tau: int = 1):
         self._check(self.lib.dflash_set_draft_mode(self.h, mode, tau), "dflash_set_draft_mode")

@@ -18,6 +18,7 @@
 #include <math.h>
 
 #include "attn_mma.h"
+#include "launch.h"
 
 namespace dfl {
 namespace at {
@@ -58,18 +59,42 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ const float *peer_ptr(const float *p, uint32_t rank) {
+    uint64_t out;
+    asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+    return reinterpret_cast<const float *>(out);
+}
+
+// The n_splits CTAs of one (query tile, kv head) form a cluster along z.  Each
+// takes an equal share of the visible keys (chunk sized on the device from the
+// tile's key count), keeps an unnormalised partial (o, running max, running
+// sum) in shared memory, and after a cluster barrier combines a slice of the
+// (head, row) pairs over all CTAs of the cluster in rank order.
 template <int HD>
 __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ q, int ldq, const bf16 *__restrict__ kc,
                                                        const bf16 *__restrict__ vc, const RowMeta *__restrict__ meta,
-                                                       int R, int rows_per_tile, int nq, int nkv, int max_len, int chunk,
-                                                       int n_splits, float scale_log2, bf16 *__restrict__ out, int ldo,
-                                                       float *o_part, float *ml_part, int *sem) {
+                                                       int R, int rows_per_tile, int nq, int nkv, int max_len,
+                                                       int n_splits, float scale_log2, bf16 *__restrict__ out, int ldo) {
     constexpr int LDS = HD + 8;  // padded smem row (bf16 elements)
+    constexpr int OLD = HD + 4;  // partial-output row stride (floats)
     extern __shared__ __align__(16) uint8_t smem_raw[];
     bf16 *Ks = reinterpret_cast<bf16 *>(smem_raw);  // [2][KB][LDS]
     bf16 *Vs = Ks + 2 * KB * LDS;                    // [2][KB][LDS]
-    __shared__ int s_last;
+    float *Op = reinterpret_cast<float *>(smem_raw); // [grp][16][OLD], reuses K/V tiles after the loop
+    __shared__ float MLs[8 * 16 * 2];                // [grp][16][(max, sum)]
 
+    pdl_trigger();
+    pdl_wait();
     const int tile = blockIdx.x, kvh = blockIdx.y, split = blockIdx.z;
     const int grp = nq / nkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,6 +110,8 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
     const int nk_b = rb < nrows ? meta[r0 + rb].nk : 0;
     int nk_max = 0;
     for (int i = 0; i < nrows; ++i) nk_max = max(nk_max, meta[r0 + i].nk);
+    // equal share of the visible keys for each split, in whole 64-key tiles
+    const int chunk = ((nk_max + n_splits - 1) / n_splits + KB - 1) / KB * KB;
     const int kb = split * chunk;
     const int ke = min(kb + chunk, nk_max);
 
@@ -236,47 +263,77 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
         }
         return;
     }
-    // partials
-    const size_t pbase = ((size_t)(tile * nq + h) * n_splits + split) * 16;
+    // ---- cluster combine of the splits ----
+    __syncthreads();  // K/V tiles are no longer read: reuse them for the partial outputs
+    {
+        float *ow = Op + (size_t)warp * 16 * OLD;
 #pragma unroll
-    for (int j = 0; j < HD / 8; ++j) {
-        const int d = j * 8 + (lane & 3) * 2;
-        *reinterpret_cast<float2 *>(o_part + (pbase + ra) * HD + d) = make_float2(o[j][0], o[j][1]);
-        *reinterpret_cast<float2 *>(o_part + (pbase + rb) * HD + d) = make_float2(o[j][2], o[j][3]);
-    }
-    if ((lane & 3) == 0) {
-        *reinterpret_cast<float2 *>(ml_part + (pbase + ra) * 2) = make_float2(m_a, l_a);
-        *reinterpret_cast<float2 *>(ml_part + (pbase + rb) * 2) = make_float2(m_b, l_b);
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int old = atomicAdd(&sem[tile * nkv + kvh], 1);
-        s_last = (old == n_splits - 1) ? 1 : 0;
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    // combine all splits for the group's heads and the tile's rows, in split order
-    for (int e = threadIdx.x; e < grp * 16 * HD; e += nthr) {
-        const int hh = e / (16 * HD), rem = e % (16 * HD), row = rem / HD, d = rem % HD;
-        if (row >= nrows) continue;
-        const int hq = kvh * grp + hh;
-        const size_t b0 = ((size_t)(tile * nq + hq) * n_splits) * 16 + row;
-        float mstar = -INFINITY;
-        for (int s2 = 0; s2 < n_splits; ++s2) mstar = fmaxf(mstar, __ldcg(ml_part + (b0 + (size_t)s2 * 16) * 2));
-        const float mu = mstar == -INFINITY ? 0.f : mstar;
-        float lsum = 0.f, acc = 0.f;
-        for (int s2 = 0; s2 < n_splits; ++s2) {
-            const size_t bb = b0 + (size_t)s2 * 16;
-            const float ms = __ldcg(ml_part + bb * 2), ls = __ldcg(ml_part + bb * 2 + 1);
-            const float w = exp2f(ms - mu);
-            lsum += ls * w;
-            acc += __ldcg(o_part + bb * HD + d) * w;
+        for (int j = 0; j < HD / 8; ++j) {
+            const int d = j * 8 + (lane & 3) * 2;
+            ow[ra * OLD + d] = o[j][0];
+            ow[ra * OLD + d + 1] = o[j][1];
+            ow[rb * OLD + d] = o[j][2];
+            ow[rb * OLD + d + 1] = o[j][3];
         }
-        out[(size_t)(r0 + row) * ldo + hq * HD + d] = __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
+        if ((lane & 3) == 0) {
+            MLs[(warp * 16 + ra) * 2] = m_a;
+            MLs[(warp * 16 + ra) * 2 + 1] = l_a;
+            MLs[(warp * 16 + rb) * 2] = m_b;
+            MLs[(warp * 16 + rb) * 2 + 1] = l_b;
+        }
     }
-    if (threadIdx.x == 0) sem[tile * nkv + kvh] = 0;
+    __syncwarp();
+    cluster_sync_all();
+    {
+        const int rank = (int)cluster_rank();
+        const int pairs = grp * 16;                       // (head, row) pairs of the tile
+        const int per = (pairs + n_splits - 1) / n_splits;
+        const int p0 = rank * per, p1 = min(pairs, p0 + per);
+        constexpr int DPT = 8;                             // output elements per thread
+        const int tpp = HD / DPT;                          // threads per pair
+        for (int e = threadIdx.x; e < (p1 - p0) * tpp; e += nthr) {
+            const int pr = p0 + e / tpp, d0 = (e % tpp) * DPT;
+            const int hh = pr / 16, row = pr % 16;
+            if (row >= nrows) continue;
+            float ms[8], ls[8];
+            float mstar = -INFINITY;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                if (s2 < n_splits) {
+                    const float *ml = peer_ptr(MLs, (uint32_t)s2);
+                    ms[s2] = ml[(hh * 16 + row) * 2];
+                    ls[s2] = ml[(hh * 16 + row) * 2 + 1];
+                    mstar = fmaxf(mstar, ms[s2]);
+                } else {
+                    ms[s2] = -INFINITY;
+                    ls[s2] = 0.f;
+                }
+            }
+            const float mu = mstar == -INFINITY ? 0.f : mstar;
+            float acc[DPT];
+#pragma unroll
+            for (int t = 0; t < DPT; ++t) acc[t] = 0.f;
+            float lsum = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                if (s2 >= n_splits) break;
+                const float w = exp2f(ms[s2] - mu);
+                lsum += ls[s2] * w;
+                const float *src = peer_ptr(Op, (uint32_t)s2) + ((size_t)hh * 16 + row) * OLD + d0;
+                const float4 a = *reinterpret_cast<const float4 *>(src);
+                const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+                acc[0] += a.x * w; acc[1] += a.y * w; acc[2] += a.z * w; acc[3] += a.w * w;
+                acc[4] += b.x * w; acc[5] += b.y * w; acc[6] += b.z * w; acc[7] += b.w * w;
+            }
+            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+            const int hq = kvh * grp + hh;
+            bf16 *dst = out + (size_t)(r0 + row) * ldo + hq * HD + d0;
+#pragma unroll
+            for (int t = 0; t < DPT; t += 2)
+                *reinterpret_cast<__nv_bfloat162 *>(dst + t) = __floats2bfloat162_rn(acc[t] * inv, acc[t + 1] * inv);
+        }
+    }
+    cluster_sync_all();
 }
 
 }  // namespace at
@@ -302,10 +359,28 @@ bool attn_mma_supported<float>(int) {
 
 static int g_num_sms = 0;
 
+template <int HD>
+static void launch_hd(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
+                      int rows_per_tile, int nq, int nkv, int max_len, bf16 *out, int ldo, int n_tiles, int n_splits,
+                      cudaStream_t s) {
+    const int grp = nq / nkv;
+    size_t smem = 2 * 2 * at::KB * (HD + 8) * sizeof(bf16);
+    smem = std::max(smem, (size_t)grp * 16 * (HD + 4) * sizeof(float));
+    static bool set = false;
+    if (!set) {
+        cudaFuncSetAttribute(at::attn_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+        set = true;
+    }
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+    launch_k(at::attn_mma_kernel<HD>, dim3(n_tiles, nkv, n_splits), dim3(32 * grp), smem, s, n_splits, q, ldq, kc, vc,
+             meta, R, rows_per_tile, nq, nkv, max_len, n_splits, scale_log2, out, ldo);
+}
+
 template <>
 void launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
                                 int rows_per_tile, int nq, int nkv, int hd, int max_len, bf16 *out, int ldo,
                                 const AttnScratch &ws, cudaStream_t s) {
+    (void)ws;
     if (R <= 0) return;
     if (!g_num_sms) {
         int dev = 0;
@@ -313,39 +388,14 @@ void launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf
         cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
     }
     const int n_tiles = (R + rows_per_tile - 1) / rows_per_tile;
-    const int grp = nq / nkv;
     const int ctas = n_tiles * nkv;
-    int n_splits = std::max(1, std::min((max_len + 255) / 256, (2 * g_num_sms + ctas - 1) / ctas));
-    // partial buffers bound the split count
-    while (n_splits > 1 && (size_t)n_tiles * nq * n_splits * 16 > ws.max_parts) --n_splits;
-    if ((size_t)n_tiles * nkv > (size_t)ws.n_sem) n_splits = 1;
-    int chunk = (max_len + n_splits - 1) / n_splits;
-    chunk = (chunk + at::KB - 1) / at::KB * at::KB;
-    n_splits = (max_len + chunk - 1) / chunk;
-    const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
-    dim3 grid(n_tiles, nkv, n_splits);
-    const int threads = 32 * grp;
-    if (hd == 128) {
-        const size_t smem = 2 * 2 * at::KB * (128 + 8) * sizeof(bf16);
-        static bool set = false;
-        if (!set) {
-            cudaFuncSetAttribute(at::attn_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            set = true;
-        }
-        at::attn_mma_kernel<128><<<grid, threads, smem, s>>>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len,
-                                                             chunk, n_splits, scale_log2, out, ldo, ws.o_part,
-                                                             ws.ml_part, ws.sem);
-    } else {
-        const size_t smem = 2 * 2 * at::KB * (64 + 8) * sizeof(bf16);
-        static bool set = false;
-        if (!set) {
-            cudaFuncSetAttribute(at::attn_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            set = true;
-        }
-        at::attn_mma_kernel<64><<<grid, threads, smem, s>>>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len,
-                                                            chunk, n_splits, scale_log2, out, ldo, ws.o_part,
-                                                            ws.ml_part, ws.sem);
-    }
+    // splits of one (tile, kv head) form a cluster of at most 8 CTAs; no more
+    // splits than 64-key tiles the longest possible context has
+    const int n_splits = std::max(1, std::min({8, (2 * g_num_sms + ctas - 1) / ctas, (max_len + 63) / 64}));
+    if (hd == 128)
+        launch_hd<128>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, n_tiles, n_splits, s);
+    else
+        launch_hd<64>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, n_tiles, n_splits, s);
 }
 
 template <>

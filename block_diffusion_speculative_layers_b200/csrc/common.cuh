@@ -67,3 +67,13 @@ __device__ __forceinline__ void argmax_merge(float &v, int &i, float v2, int i2)
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
 
 }  // namespace dfl
+
+namespace dfl {
+
+// Programmatic dependent launch: let the next kernel in the stream begin its
+// prologue now, and wait here until the previous kernel's writes are visible.
+// Both are no-ops for kernels launched without the programmatic attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+}  // namespace dfl

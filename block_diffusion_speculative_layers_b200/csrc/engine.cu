@@ -235,6 +235,13 @@ class Engine : public EngineBase {
     std::vector<int> last_draft;
     int last_logits_rows[3] = {0, 0, 0};
     int *pinned = nullptr;  // small pinned host buffer for the done counter
+    bool lens_stale = false;
+    // per-launch timing (dflash_profile)
+    struct ProfRec { int cls; double bytes; cudaEvent_t a, b; };
+    bool profiling = false;
+    std::vector<ProfRec> prof;
+    std::vector<cudaEvent_t> ev_pool;
+    size_t ev_used = 0;
     cudaEvent_t ev_a = nullptr, ev_b = nullptr;
 
     Engine(const dflash_config &cfg, const Layout &lay, char *warena, char *sarena, cudaStream_t stream)
@@ -340,6 +347,7 @@ class Engine : public EngineBase {
     }
 
     ~Engine() override {
+        for (cudaEvent_t e : ev_pool) cudaEventDestroy(e);
         if (pinned) cudaFreeHost(pinned);
         if (ev_a) cudaEventDestroy(ev_a);
         if (ev_b) cudaEventDestroy(ev_b);
@@ -386,8 +394,47 @@ class Engine : public EngineBase {
         return (size_t)c.max_batch * m.n_kv_heads * c.max_len * m.head_dim;
     }
 
+    cudaEvent_t next_event() {
+        if (ev_used == ev_pool.size()) {
+            cudaEvent_t e;
+            cudaEventCreate(&e);
+            ev_pool.push_back(e);
+        }
+        return ev_pool[ev_used++];
+    }
+
+    template <typename F>
+    void timed(int cls, double bytes, F &&launch) {
+        if (!profiling) {
+            launch();
+            return;
+        }
+        ProfRec r{cls, bytes, next_event(), next_event()};
+        cudaEventRecord(r.a, s);
+        launch();
+        cudaEventRecord(r.b, s);
+        prof.push_back(r);
+    }
+
+    static double gemm_bytes(int M, int N, int K, const Epi<T> &e) {
+        const double es = sizeof(T);
+        double b = (double)N * K * es + (double)M * K * es;
+        switch (e.kind) {
+            case EPI_QKV: b += (double)M * N * es; break;
+            case EPI_RESID: b += (double)M * N * 8 + (double)M * N * es * e.taps.n; break;
+            case EPI_SWIGLU: b += (double)M * e.F * es; break;
+            case EPI_LOGITS: b += (double)((N + 127) / 128) * M * 8; break;
+            default: b += (double)M * N * 4; break;
+        }
+        return b;
+    }
+
     void gemm(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e) {
         if (M <= 0) return;
+        timed(0, gemm_bytes(M, N, K, e), [&] { gemm_launch(X, ldx, M, Wt, N, K, e); });
+    }
+
+    void gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e) {
         if (tc.supports(M, N, K)) {
             tc.run(X, ldx, M, (const T *)Wt, N, K, e, s);
             return;
@@ -415,12 +462,14 @@ class Engine : public EngineBase {
     void attention(const T *qq, const T *kc, const T *vc, const RowMeta *mt, int R, int rows_per_tile,
                    const dflash_model_cfg &m, T *out) {
         const int qd = m.n_q_heads * m.head_dim;
-        if (attn_mma_supported<T>(m.head_dim)) {
-            launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads, m.head_dim,
-                                    c.max_len, out, qd, att, s);
-            return;
-        }
-        launch_attention_simt<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out, qd, s);
+        timed(1, 0.0, [&] {
+            if (attn_mma_supported<T>(m.head_dim))
+                launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads, m.head_dim,
+                                        c.max_len, out, qd, att, s);
+            else
+                launch_attention_simt<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out,
+                                         qd, s);
+        });
     }
 
     // one pre-norm decoder layer of the target over R rows in x (meta)
@@ -634,8 +683,23 @@ class Engine : public EngineBase {
     }
 
     // ---- API ----
+    dflash_status refresh_lens() {
+        if (!lens_stale) return DFLASH_OK;
+        dflash_status r = sync("lengths");
+        if (r) return r;
+        std::vector<SeqState> hs(c.max_batch);
+        if (cudaMemcpy(hs.data(), st, sizeof(SeqState) * c.max_batch, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return fail_cuda("state copy");
+        for (int i = 0; i < c.max_batch; ++i)
+            if (h_prefilled[i]) h_len[i] = hs[i].len;
+        lens_stale = false;
+        return DFLASH_OK;
+    }
+
     dflash_status check_seqs(const int32_t *seqs, int n) {
         if (!seqs || n < 1 || n > c.max_batch) { err = "seqs must hold 1..max_batch slots"; return DFLASH_EINVAL; }
+        dflash_status rr = refresh_lens();
+        if (rr) return rr;
         std::vector<char> seen(c.max_batch, 0);
         for (int i = 0; i < n; ++i) {
             if (seqs[i] < 0 || seqs[i] >= c.max_batch || seen[seqs[i]]) { err = "bad or repeated slot"; return DFLASH_EINVAL; }
@@ -821,6 +885,7 @@ class Engine : public EngineBase {
             cudaEventElapsedTime(&b, t1, t2);
             ost->ms_prefill = a;
             ost->ms_decode = b;
+            ost->kernel_launches = launch_count();
         }
         cudaEventDestroy(t0);
         cudaEventDestroy(t1);
@@ -922,6 +987,76 @@ class Engine : public EngineBase {
         float f;
         memcpy(&f, &u, 4);
         return f;
+    }
+
+    dflash_status decode_iters(int n, int iters) override {
+        if (n < 1 || n > c.max_batch || iters < 0) { err = "bad decode_iters arguments"; return DFLASH_EINVAL; }
+        dflash_status r = refresh_lens();
+        if (r) return r;
+        for (int i = 0; i < n; ++i) {
+            if (!h_prefilled[i]) { err = "slot not prefilled"; return DFLASH_ESTATE; }
+            if ((int64_t)h_len[i] + (int64_t)(iters + 1) * c.block_size > c.max_len) {
+                err = "decode_iters could exceed max_len";
+                return DFLASH_ECAPACITY;
+            }
+        }
+        std::vector<int32_t> iota(n);
+        for (int i = 0; i < n; ++i) iota[i] = i;
+        if ((r = set_active(iota.data(), n))) return r;
+        for (int it = 0; it < iters; ++it) {
+            enqueue_draft(n, true);
+            enqueue_verify(n);
+        }
+        last_draft.clear();
+        lens_stale = true;
+        return check("decode_iters launch");
+    }
+
+    dflash_status get_stats(dflash_stats *o) override {
+        if (!o) { err = "null stats"; return DFLASH_EINVAL; }
+        dflash_status r = sync("stats");
+        if (r) return r;
+        DevStats hs;
+        if (cudaMemcpy(&hs, stats, sizeof hs, cudaMemcpyDeviceToHost) != cudaSuccess) return fail_cuda("stats copy");
+        memset(o, 0, sizeof *o);
+        o->iterations = (int64_t)hs.iterations;
+        o->tokens = (int64_t)hs.tokens;
+        for (int i = 0; i < DFLASH_MAX_BLOCK; ++i) o->accept_hist[i] = (int64_t)hs.hist[i];
+        o->mean_tau = hs.iterations ? (double)hs.tokens / (double)hs.iterations : 0.0;
+        o->kernel_launches = launch_count();
+        if (hs.status & 4) { err = "a bounded device wait expired"; return DFLASH_ETIMEOUT; }
+        return DFLASH_OK;
+    }
+
+    dflash_status reset_stats() override {
+        if (cudaMemsetAsync(stats, 0, sizeof(DevStats), s) != cudaSuccess) return fail_cuda("stats reset");
+        return DFLASH_OK;
+    }
+
+    dflash_status profile(int enable) override {
+        dflash_status r = sync("profile");
+        if (r) return r;
+        profiling = enable != 0;
+        if (profiling) {
+            prof.clear();
+            ev_used = 0;
+        }
+        return DFLASH_OK;
+    }
+
+    dflash_status profile_read(dflash_kernel_prof *o) override {
+        if (!o) { err = "null profile output"; return DFLASH_EINVAL; }
+        dflash_status r = sync("profile_read");
+        if (r) return r;
+        for (int k = 0; k < DFLASH_PROF_CLASSES; ++k) o[k] = dflash_kernel_prof{0, 0.0, 0.0};
+        for (const ProfRec &p : prof) {
+            float ms = 0.f;
+            if (cudaEventElapsedTime(&ms, p.a, p.b) != cudaSuccess) return fail_cuda("event time");
+            o[p.cls].launches += 1;
+            o[p.cls].ms += ms;
+            o[p.cls].bytes += p.bytes;
+        }
+        return DFLASH_OK;
     }
 
     dflash_status set_script(int seq, const int32_t *sc, int n) override {
@@ -1053,6 +1188,20 @@ dflash_status dflash_generate_ar(dflash_ctx *ctx, const int32_t *const *prompts,
                                  int32_t max_new, int32_t *out, double *ms) {
     if (!out) return DFLASH_EINVAL;
     DFL_CALL(ctx, ctx->eng->generate_ar(prompts, lens, n, max_new, out, ms));
+}
+
+dflash_status dflash_decode_iters(dflash_ctx *ctx, int32_t n, int32_t iters) {
+    DFL_CALL(ctx, ctx->eng->decode_iters(n, iters));
+}
+
+dflash_status dflash_get_stats(dflash_ctx *ctx, dflash_stats *out) { DFL_CALL(ctx, ctx->eng->get_stats(out)); }
+
+dflash_status dflash_reset_stats(dflash_ctx *ctx) { DFL_CALL(ctx, ctx->eng->reset_stats()); }
+
+dflash_status dflash_profile(dflash_ctx *ctx, int32_t enable) { DFL_CALL(ctx, ctx->eng->profile(enable)); }
+
+dflash_status dflash_profile_read(dflash_ctx *ctx, dflash_kernel_prof *out) {
+    DFL_CALL(ctx, ctx->eng->profile_read(out));
 }
 
 dflash_status dflash_set_draft_mode(dflash_ctx *ctx, int32_t mode, int32_t tau) {

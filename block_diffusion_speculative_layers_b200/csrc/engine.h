@@ -61,6 +61,11 @@ class EngineBase {
     virtual dflash_status seq_state(int seq, int32_t *len, int32_t *anchor, int32_t *n_out) = 0;
     virtual dflash_status debug_kv(int which, int layer, int seq, int p0, int n, float *k, float *v) = 0;
     virtual dflash_status set_script(int seq, const int32_t *script, int n) = 0;
+    virtual dflash_status decode_iters(int n, int iters) = 0;
+    virtual dflash_status get_stats(dflash_stats *out) = 0;
+    virtual dflash_status reset_stats() = 0;
+    virtual dflash_status profile(int enable) = 0;
+    virtual dflash_status profile_read(dflash_kernel_prof *out) = 0;
     std::string err;
     int draft_mode = DFLASH_DRAFT_MODEL, tau = 1;
 };

@@ -21,6 +21,7 @@
 #include <cstring>
 
 #include "gemm_tc.h"
+#include "launch.h"
 
 namespace dfl {
 namespace tc {
@@ -46,6 +47,10 @@ __device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
@@ -128,33 +133,40 @@ __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: 
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 // ---------------------------------------------------------------------------
-// fused epilogue on one chunk of CH accumulator columns (activation rows
-// m0c .. m0c+CH-1) for weight row n_local of the tile
+// fused epilogue on one chunk of up to CH accumulator columns (activation rows
+// m0c .. m0c+nc-1) for weight row n_local of the tile.  Global loads of a
+// chunk are issued together before any use.
 // ---------------------------------------------------------------------------
 template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16> &e, int nt, int n_local, int q,
-                                               int lane, int m0c, const float *v, float *stg, float2 *red) {
+                                               int lane, int m0c, int nc, const float *v, float *stg, float2 *red,
+                                               RowMeta *smeta) {
     const int M = p.M;
-    if (KIND == EPI_STORE || KIND == EPI_RESID) {
+    if (KIND == EPI_STORE) {
         const int n = nt * 128 + n_local;
         if (n < p.N) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) {
-                const int m = m0c + j;
-                if (m >= M) break;
-                if (KIND == EPI_STORE) {
-                    e.Y[(size_t)m * e.ldy + n] = v[j];
-                } else {
-                    float *xp = e.x + (size_t)m * p.N + n;
-                    const float nx = *xp + v[j];
-                    *xp = nx;
-                    if (e.taps.n) {
-                        const int trow = e.meta[m].aux;
-                        for (int t = 0; t < e.taps.n; ++t)
-                            e.taps.base[(size_t)trow * e.taps.ld + e.taps.col[t] + n] = __float2bfloat16_rn(nx);
-                    }
-                }
-            }
+            for (int j = 0; j < CH; ++j)
+                if (j < nc && m0c + j < M) e.Y[(size_t)(m0c + j) * e.ldy + n] = v[j];
+        }
+    } else if (KIND == EPI_RESID) {
+        const int n = nt * 128 + n_local;
+        const bool nok = n < p.N;
+        float xo[CH];
+        int trow[CH];
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            const bool ok = nok && j < nc && m0c + j < M;
+            xo[j] = ok ? e.x[(size_t)(m0c + j) * p.N + n] : 0.f;
+            trow[j] = (ok && e.taps.n) ? e.meta[m0c + j].aux : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            if (!(nok && j < nc && m0c + j < M)) continue;
+            const float nx = xo[j] + v[j];
+            e.x[(size_t)(m0c + j) * p.N + n] = nx;
+            for (int t = 0; t < e.taps.n; ++t)
+                e.taps.base[(size_t)trow[j] * e.taps.ld + e.taps.col[t] + n] = __float2bfloat16_rn(nx);
         }
     } else if (KIND == EPI_LOGITS) {
         const int n = nt * 128 + n_local;
@@ -162,9 +174,10 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
             const int m = m0c + j;
-            if (p.keep_logits && ok && m < M) e.Y[(size_t)m * e.ldy + n] = v[j];
-            float bv = ok ? v[j] : -INFINITY;
-            int bi = ok ? n : 0x7fffffff;
+            const bool col = j < nc && m < M;
+            if (p.keep_logits && ok && col) e.Y[(size_t)m * e.ldy + n] = v[j];
+            float bv = (ok && col) ? v[j] : -INFINITY;
+            int bi = (ok && col) ? n : 0x7fffffff;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -180,7 +193,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             float bv = red[j].x;
             int bi = __float_as_int(red[j].y);
             for (int qq = 1; qq < 4; ++qq) argmax_merge(bv, bi, red[qq * CH + j].x, __float_as_int(red[qq * CH + j].y));
-            if (m < M) p.lm_part[(size_t)nt * p.M + m] = make_float2(bv, __int_as_float(bi));
+            if (j < nc && m < M) p.lm_part[(size_t)nt * p.M + m] = make_float2(bv, __int_as_float(bi));
         }
         epi_bar();
     } else if (KIND == EPI_SWIGLU) {
@@ -193,8 +206,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
 #pragma unroll
                 for (int j = 0; j < CH; ++j) {
                     const int m = m0c + j;
-                    if (m >= M) break;
-                    // gate and up are bf16-rounded like any projection output feeding a GEMM
+                    if (j >= nc || m >= M) break;
                     const float up = stg[(n_local + 64) * STG_LD + j];
                     e.h[(size_t)m * p.swiglu_F + f] = __float2bfloat16_rn(silu_f(v[j]) * up);
                 }
@@ -204,32 +216,49 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
     } else if (KIND == EPI_QKV) {
 #pragma unroll
         for (int j = 0; j < CH; ++j) stg[n_local * STG_LD + j] = v[j];
+        if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+            const int j = threadIdx.x - 64, m = m0c + j;
+            RowMeta mt;
+            mt.seq = mt.pos = mt.nk = 0;
+            mt.aux = -1;  // -1: skip this column
+            if (j < nc && m < M) {
+                if (m >= e.R_blk) {
+                    mt = e.ctx_meta[m - e.R_blk];
+                    mt.aux = mt.aux ? 1 : -1;
+                } else {
+                    mt = e.meta[m];
+                    mt.aux = 0;
+                }
+            }
+            smeta[j] = mt;
+        }
         epi_bar();
         const int hd = e.hd, half = hd >> 1;
         const int qd = e.nq * hd, kd = e.nkv * hd;
         const int cg = e.col0 + nt * 128 + n_local;  // row of [Wq; Wk; Wv]
-        const int nloc_ok = (nt * 128 + n_local) < p.N;
-        if (nloc_ok) {
+        if (nt * 128 + n_local < p.N) {
             const int head_base = (cg / hd) * hd;
             const int d = cg - head_base;
             const int partner = n_local + (d < half ? half : -half);
             const int i = d < half ? d : d - half;
             const bool is_q = cg < qd, is_k = !is_q && cg < qd + kd;
-#pragma unroll 4
+            float2 cs[CH];
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+                cs[j] = (is_q || is_k) && smeta[j].aux >= 0 ? e.rope[(size_t)smeta[j].pos * half + i] : make_float2(1.f, 0.f);
+#pragma unroll
             for (int j = 0; j < CH; ++j) {
-                const int m = m0c + j;
-                if (m >= M) break;
-                const bool ctx = m >= e.R_blk;
-                const RowMeta mt = ctx ? e.ctx_meta[m - e.R_blk] : e.meta[m];
-                if (ctx && (is_q || !mt.aux)) continue;
+                const RowMeta mt = smeta[j];
+                if (mt.aux < 0) continue;          // padding column or uncommitted context row
+                const bool ctx = mt.aux == 1;
+                if (ctx && is_q) continue;         // context rows only feed K/V
                 float out = v[j];
                 if (is_q || is_k) {
-                    const float2 cs = e.rope[(size_t)mt.pos * half + i];
                     const float other = stg[partner * STG_LD + j];
-                    out = d < half ? v[j] * cs.x - other * cs.y : v[j] * cs.x + other * cs.y;
+                    out = d < half ? v[j] * cs[j].x - other * cs[j].y : v[j] * cs[j].x + other * cs[j].y;
                 }
                 if (is_q) {
-                    e.q_out[(size_t)m * qd + cg] = __float2bfloat16_rn(out);
+                    e.q_out[(size_t)(m0c + j) * qd + cg] = __float2bfloat16_rn(out);
                 } else {
                     const int hh = is_k ? (cg - qd) / hd : (cg - qd - kd) / hd;
                     bf16 *dst = (is_k ? e.kc : e.vc) + (((size_t)mt.seq * e.nkv + hh) * e.max_len + mt.pos) * hd;
@@ -241,6 +270,36 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
     }
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// generic address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ const float *peer_ptr(const float *p, uint32_t rank) {
+    uint64_t out;
+    asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+    return reinterpret_cast<const float *>(out);
+}
+
+// Work split.  Small projections (fewer tiles than SMs) run one tile per CTA
+// with the K range split over a thread-block cluster of p.splits CTAs along z:
+// each CTA accumulates its K range in TMEM, parks it in its shared memory, and
+// after a cluster barrier reduces a slice of the tile's columns over all CTAs
+// of the cluster (in rank order, so results are identical run to run) through
+// distributed shared memory, then runs the fused epilogue on that slice.
+// Large projections (p.splits == 1) are persistent: CTA b handles tiles
+// b, b + gridDim.x, ... with two TMEM accumulators, so the epilogue of one tile
+// overlaps the MMAs of the next while the TMA ring streams weights without a
+// break.  Grids never exceed one CTA per SM, which leaves room on every SM for
+// the next kernel's CTA to start streaming its weights early (programmatic
+// dependent launch: weights are loaded before griddepcontrol.wait,
+// activations after it).
 template <int TM, int KIND>
 __global__ void __launch_bounds__(NT, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcParams p,
@@ -248,147 +307,215 @@ __global__ void __launch_bounds__(NT, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     constexpr int B_BYTES = TM * 128;
-    constexpr int NCOLS = TM < 32 ? 32 : TM;
+    constexpr int NC1 = TM < 32 ? 32 : TM;  // TMEM columns of one accumulator
+    constexpr int PLD = TM + 1;             // parked partial tile row stride (floats)
     uint8_t *sA = smem;
     uint8_t *sB = smem + (size_t)stages * A_BYTES;
     float *stg = (float *)(sB + (size_t)stages * B_BYTES);
     float2 *red = (float2 *)(stg + 128 * STG_LD);
-    uint64_t *full = (uint64_t *)(red + 4 * CH);
+    RowMeta *smeta = (RowMeta *)(red + 4 * CH);
+    uint64_t *full = (uint64_t *)(smeta + CH);
     uint64_t *empty = full + stages;
-    uint64_t *done = empty + stages;
-    uint32_t *tmem_slot = (uint32_t *)(done + 1);
-    int *flag = (int *)(tmem_slot + 1);
+    uint64_t *acc_full = empty + stages;   // [2]
+    uint64_t *acc_empty = acc_full + 2;    // [2]
+    uint32_t *tmem_slot = (uint32_t *)(acc_empty + 2);
+    float *part = (float *)sA;  // [128][PLD] after the last MMA (split-K only)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nt = blockIdx.x, mt = blockIdx.y, sp = blockIdx.z;
-    const int k_per = (p.k_steps + p.splits - 1) / p.splits;
-    const int kb = sp * k_per, ke = min(p.k_steps, kb + k_per);
-    const int nk = ke - kb;
+    const int S = p.splits;
+    const bool split = S > 1;
+    const int n_tiles_total = p.n_tiles * p.m_tiles;
+    // one tile per CTA: (blockIdx.x, blockIdx.y); a persistent launch would pass
+    // a 1-D grid smaller than the tile count and stride over the tiles
+    const bool persistent = !split && gridDim.y == 1 && (int)gridDim.x < n_tiles_total;
+    const int tile0 = persistent ? blockIdx.x : blockIdx.y * p.n_tiles + blockIdx.x;
+    const int tstride = persistent ? gridDim.x : n_tiles_total;
+    const int k_per = (p.k_steps + S - 1) / S;
+    const int kb = split ? blockIdx.z * k_per : 0;
+    const int ke = split ? min(p.k_steps, kb + k_per) : p.k_steps;
+    const int nk = max(0, ke - kb);
+    const int ncols = persistent ? 2 * NC1 : NC1;  // persistent CTAs double-buffer the accumulator
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(done, 1);
-        flag[0] = 0;
-        flag[1] = 0;
+        mbar_init(&acc_full[0], 1);
+        mbar_init(&acc_full[1], 1);
+        mbar_init(&acc_empty[0], 4);
+        mbar_init(&acc_empty[1], 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(NCOLS));
+                     "r"(ncols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer ----------------
-            const int rowA0 = p.swiglu_F ? nt * 64 : nt * 128;
-            const int rowA1 = p.swiglu_F ? p.swiglu_F + nt * 64 : nt * 128 + 64;
-            const int m0 = mt * TM;
-            for (int it = 0; it < nk; ++it) {
-                const int s = it % stages;
-                if (it >= stages && !mbar_wait(&empty[s], ((it / stages) & 1) ^ 1, p.err)) {
-                    flag[1] = 1;
-                    break;
+            // ---------------- TMA producer: one continuous ring over all tiles of this CTA ----------------
+            int it = 0;     // global stage counter
+            bool first = true, abort = false;
+            for (int t = tile0; t < n_tiles_total && !abort; t += tstride) {
+                const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+                const int rowA0 = p.swiglu_F ? nt * 64 : nt * 128;
+                const int rowA1 = p.swiglu_F ? p.swiglu_F + nt * 64 : nt * 128 + 64;
+                const int m0 = mt * TM;
+                int kk0 = 0;
+                if (first) {
+                    // weights do not depend on the previous kernel: start streaming them first
+                    const int pre = min(nk, stages);
+                    for (int i = 0; i < pre; ++i) {
+                        uint8_t *a = sA + (size_t)i * A_BYTES;
+                        mbar_expect_tx(&full[i], A_BYTES + B_BYTES);
+                        tma_load_2d(a, &tmW, (kb + i) * BK, rowA0, &full[i]);
+                        tma_load_2d(a + A_BYTES / 2, &tmW, (kb + i) * BK, rowA1, &full[i]);
+                    }
+                    pdl_wait();
+                    for (int i = 0; i < pre; ++i)
+                        tma_load_2d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, &full[i]);
+                    kk0 = pre;
+                    it = pre;
+                    first = false;
                 }
-                if (flag[1]) break;
-                const int k = (kb + it) * BK;
-                uint8_t *a = sA + (size_t)s * A_BYTES;
-                mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
-                tma_load_2d(a, &tmW, k, rowA0, &full[s]);
-                tma_load_2d(a + A_BYTES / 2, &tmW, k, rowA1, &full[s]);
-                tma_load_2d(sB + (size_t)s * B_BYTES, &tmX, k, m0, &full[s]);
+                for (int kk = kk0; kk < nk; ++kk, ++it) {
+                    const int s = it % stages;
+                    if (it >= stages && !mbar_wait(&empty[s], ((it / stages) & 1) ^ 1, p.err)) {
+                        abort = true;
+                        break;
+                    }
+                    const int k = (kb + kk) * BK;
+                    uint8_t *a = sA + (size_t)s * A_BYTES;
+                    mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
+                    tma_load_2d(a, &tmW, k, rowA0, &full[s]);
+                    tma_load_2d(a + A_BYTES / 2, &tmW, k, rowA1, &full[s]);
+                    tma_load_2d(sB + (size_t)s * B_BYTES, &tmX, k, m0, &full[s]);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
             const uint32_t idesc = idesc_bf16(TM);
-            for (int it = 0; it < nk; ++it) {
-                const int s = it % stages;
-                if (!mbar_wait(&full[s], (it / stages) & 1, p.err)) {
-                    flag[1] = 1;
-                    break;
-                }
+            int it = 0, lt = 0;  // global stage counter, local tile counter
+            bool ok = true;
+            for (int t = tile0; t < n_tiles_total && ok; t += tstride, ++lt) {
+                const int b = lt & 1;
+                if (lt >= 2 && !mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1, p.err)) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_BYTES));
-                const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_BYTES));
+                const uint32_t acc = tmem + (uint32_t)(b * NC1);
+                for (int kk = 0; kk < nk; ++kk, ++it) {
+                    const int s = it % stages;
+                    if (!mbar_wait(&full[s], (it / stages) & 1, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_BYTES));
+                    const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_BYTES));
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes per K=16 step inside the swizzle row
-                    mma_bf16(tmem, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), idesc, (it > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&empty[s]);
+                    for (int k4 = 0; k4 < BK / 16; ++k4)  // +32 bytes per K=16 step inside the swizzle row
+                        mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)(k4 * 2), idesc,
+                                 (kk > 0 || k4 > 0) ? 1u : 0u);
+                    mma_commit(&empty[s]);
+                }
+                mma_commit(&acc_full[b]);
             }
-            mma_commit(done);
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue warps 2..5 ----------------
+        pdl_wait();
         const int q = warp & 3;
         const int n_local = q * 32 + lane;
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-        const bool ok = mbar_wait(done, 0, p.err);
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const int tile = mt * p.n_tiles + nt;
-        float v[CH];
-        bool last = true;
-        if (p.splits > 1) {
-            float *mine = p.ws + ((size_t)tile * p.splits + sp) * (size_t)TM * 128;
-            for (int c = 0; c < TM; c += CH) {
-                if (ok) tmem_ld16(trow + c, v);
-                else
-                    for (int j = 0; j < CH; ++j) v[j] = 0.f;
+        int lt = 0;
+        for (int t = tile0; t < n_tiles_total; t += tstride, ++lt) {
+            const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+            const int b = lt & 1;
+            const uint32_t trow = tmem + (uint32_t)(b * NC1) + ((uint32_t)(q * 32) << 16);
+            const bool ok = mbar_wait(&acc_full[b], (lt >> 1) & 1, p.err) && nk > 0;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            float v[CH];
+            if (!split) {
+                for (int c = 0; c < TM; c += CH) {
+                    if (ok) tmem_ld16(trow + c, v);
+                    else
 #pragma unroll
-                for (int j = 0; j < CH; ++j) mine[(size_t)(c + j) * 128 + n_local] = v[j];
-            }
-            __threadfence();
-            epi_bar();
-            if (threadIdx.x == 64) {
-                const int old = atomicAdd(&p.sem[tile], 1);
-                flag[0] = (old == p.splits - 1) ? 1 : 0;
-            }
-            epi_bar();
-            last = flag[0] != 0;
-            if (last) __threadfence();
-        }
-        if (last) {
-            for (int c = 0; c < TM; c += CH) {
-                if (p.splits > 1) {
-#pragma unroll
-                    for (int j = 0; j < CH; ++j) v[j] = 0.f;
-                    for (int s2 = 0; s2 < p.splits; ++s2) {
-                        const float *src = p.ws + ((size_t)tile * p.splits + s2) * (size_t)TM * 128;
-#pragma unroll
-                        for (int j = 0; j < CH; ++j) v[j] += __ldcg(src + (size_t)(c + j) * 128 + n_local);
+                        for (int j = 0; j < CH; ++j) v[j] = 0.f;
+                    if (c == TM - CH || TM == CH) {
+                        // accumulator fully read: hand it back to the MMA warp
+                        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[b]);
                     }
-                } else if (ok) {
-                    tmem_ld16(trow + c, v);
-                } else {
-                    for (int j = 0; j < CH; ++j) v[j] = 0.f;
+                    if (mt * TM + c < p.M || KIND != EPI_STORE)
+                        epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, mt * TM + c, CH, v, stg, red, smeta);
                 }
-                const int m0c = mt * TM + c;
-                if (m0c < p.M || KIND == EPI_LOGITS || KIND == EPI_SWIGLU || KIND == EPI_QKV)
-                    epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, m0c, v, stg, red);
+            } else {
+                // park this CTA's partial tile in shared memory (the stage ring is idle now)
+                for (int c = 0; c < TM; c += CH) {
+                    if (ok) tmem_ld16(trow + c, v);
+                    else
+#pragma unroll
+                        for (int j = 0; j < CH; ++j) v[j] = 0.f;
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) part[n_local * PLD + c + j] = v[j];
+                }
             }
-            if (p.splits > 1 && threadIdx.x == 64) p.sem[tile] = 0;
         }
+    }
+    if (split) {
+        __syncwarp();
+        cluster_sync_all();
+        if (warp >= 2) {
+            const int q = warp & 3;
+            const int n_local = q * 32 + lane;
+            const int nt = blockIdx.x, mt = blockIdx.y;
+            const int rank = (int)cluster_rank();
+            const int cpr = (TM + S - 1) / S;  // columns reduced by this CTA
+            const int c_begin = rank * cpr, c_end = min(TM, c_begin + cpr);
+            const float *peers[8];
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) peers[s2] = s2 < S ? peer_ptr(part, (uint32_t)s2) : part;
+            for (int c = c_begin; c < c_end; c += CH) {
+                const int nc = min(CH, c_end - c);
+                float v[CH];
+#pragma unroll
+                for (int j = 0; j < CH; ++j) v[j] = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 8; ++s2) {
+                    if (s2 >= S) break;
+                    float tv[CH];
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) tv[j] = j < nc ? peers[s2][n_local * PLD + c + j] : 0.f;
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) v[j] += tv[j];
+                }
+                epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, mt * TM + c, nc, v, stg, red, smeta);
+            }
+        }
+        cluster_sync_all();
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
     }
 }
 
 // final argmax over the per-tile partials of each row
 __global__ void lm_argmax_kernel(const float2 *__restrict__ part, int n_tiles, int R, int mode, int B, int *idx,
                                  DevStats *stats) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     if (mode == 1 && (r % B) == 0) return;
     float bv = -INFINITY;
@@ -425,7 +552,7 @@ __global__ void lm_argmax_kernel(const float2 *__restrict__ part, int n_tiles, i
 void launch_lm_argmax(const float2 *part, int n_tiles, int R, int mode, int B, int *idx, DevStats *stats,
                       cudaStream_t s) {
     if (R <= 0) return;
-    tc::lm_argmax_kernel<<<R, 256, 0, s>>>(part, n_tiles, R, mode, B, idx, stats);
+    launch_k(tc::lm_argmax_kernel, dim3(R), dim3(256), 0, s, 1, part, n_tiles, R, mode, B, idx, stats);
 }
 
 int gemm_tc_workspace_floats(int max_rows, int max_n) {
@@ -435,6 +562,11 @@ int gemm_tc_workspace_floats(int max_rows, int max_n) {
 }
 
 int gemm_tc_semaphores() { return 1 << 16; }
+
+bool &pdl_enabled() {
+    static bool on = true;
+    return on;
+}
 
 // ---------------------------------------------------------------------------
 // host side
@@ -502,26 +634,27 @@ const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, in
 
 template <int TM, int KIND>
 static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p, const Epi<bf16> &e,
-                      int stages, size_t smem, cudaStream_t s) {
+                      int stages, size_t smem, cudaStream_t s, int grid_x) {
     auto kern = tc::gemm_tc_kernel<TM, KIND>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         attr_set = true;
     }
+    (void)grid_x;
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-    kern<<<grid, tc::NT, smem, s>>>(*mw, *mx, p, e, stages);
+    launch_k(kern, grid, dim3(tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
 }
 
 template <int TM>
 static void launch_kind(int kind, const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p,
-                        const Epi<bf16> &e, int stages, size_t smem, cudaStream_t s) {
+                        const Epi<bf16> &e, int stages, size_t smem, cudaStream_t s, int gx) {
     switch (kind) {
-        case EPI_STORE: launch_tm<TM, EPI_STORE>(mw, mx, p, e, stages, smem, s); break;
-        case EPI_QKV: launch_tm<TM, EPI_QKV>(mw, mx, p, e, stages, smem, s); break;
-        case EPI_RESID: launch_tm<TM, EPI_RESID>(mw, mx, p, e, stages, smem, s); break;
-        case EPI_SWIGLU: launch_tm<TM, EPI_SWIGLU>(mw, mx, p, e, stages, smem, s); break;
-        default: launch_tm<TM, EPI_LOGITS>(mw, mx, p, e, stages, smem, s); break;
+        case EPI_STORE: launch_tm<TM, EPI_STORE>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_QKV: launch_tm<TM, EPI_QKV>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_RESID: launch_tm<TM, EPI_RESID>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_SWIGLU: launch_tm<TM, EPI_SWIGLU>(mw, mx, p, e, stages, smem, s, gx); break;
+        default: launch_tm<TM, EPI_LOGITS>(mw, mx, p, e, stages, smem, s, gx); break;
     }
 }
 
@@ -540,34 +673,38 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
     p.m_tiles = (M + TM - 1) / TM;
     p.k_steps = (K + tc::BK - 1) / tc::BK;
     const int tiles = p.n_tiles * p.m_tiles;
+    const int stage_bytes = tc::A_BYTES + TM * 128;
+    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + 64 * 8 + 64;
+    // Measured on B200 (decode shapes, M = 16): projections with at least as
+    // many tiles as SMs stream fastest with one tile per CTA and two ~100 KB
+    // CTAs per SM; projections with fewer tiles split K over a cluster so that
+    // about one CTA per SM runs, each with a deeper (~150 KB) ring.
     int splits = 1;
-    if (e.kind != EPI_LOGITS) {
-        const int target = 2 * num_sms;
-        splits = std::max(1, std::min(p.k_steps / 4, target / std::max(1, tiles)));
-        while (splits > 1 && ((size_t)tiles * splits * TM * 128 > (size_t)ws_floats || tiles > n_sem)) --splits;
+    if (e.kind != EPI_LOGITS && tiles < num_sms && p.k_steps >= 4) {
+        splits = std::max(1, std::min({8, p.k_steps / 2, num_sms / std::max(1, tiles)}));
+        if (tune_splits > 0) splits = std::min(8, tune_splits);
         const int k_per = (p.k_steps + splits - 1) / splits;
         splits = (p.k_steps + k_per - 1) / k_per;
     }
+    int budget = splits > 1 ? 150 * 1024 : (TM <= 64 ? 112 * 1024 : 200 * 1024);
+    if (tune_smem_kb > 0) budget = tune_smem_kb * 1024;
+    const int stages = std::max(2, std::min(16, (budget - fixed) / stage_bytes));
+    const size_t smem = (size_t)fixed + (size_t)stages * stage_bytes;
+    if (splits > 1 && (size_t)stages * stage_bytes < (size_t)128 * (TM + 1) * 4) splits = 1;  // no room to park
     p.splits = splits;
-    p.ws = ws;
-    p.sem = sem;
     p.err = err_word;
     p.lm_part = lm_part;
     p.keep_logits = keep_logits;
+    const int grid_x = p.n_tiles;  // one tile per CTA
     const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
     const CUtensorMap *mx = tensor_map(X, M, K, ldx, TM);
     if (!mw || !mx) return;
-    const int stage_bytes = tc::A_BYTES + TM * 128;
-    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + 64 * 8 + 64;
-    const int budget = TM <= 64 ? 112 * 1024 : 200 * 1024;
-    const int stages = std::max(2, std::min(8, (budget - fixed) / stage_bytes));
-    const size_t smem = (size_t)fixed + (size_t)stages * stage_bytes;
     switch (TM) {
-        case 16: launch_kind<16>(e.kind, mw, mx, p, e, stages, smem, s); break;
-        case 32: launch_kind<32>(e.kind, mw, mx, p, e, stages, smem, s); break;
-        case 64: launch_kind<64>(e.kind, mw, mx, p, e, stages, smem, s); break;
-        case 128: launch_kind<128>(e.kind, mw, mx, p, e, stages, smem, s); break;
-        default: launch_kind<256>(e.kind, mw, mx, p, e, stages, smem, s); break;
+        case 16: launch_kind<16>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+        case 32: launch_kind<32>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+        case 64: launch_kind<64>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+        case 128: launch_kind<128>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+        default: launch_kind<256>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
     }
 }
 

@@ -50,6 +50,8 @@ struct GemmTC {
     int n_sem = 0;
     int *err_word = nullptr;
     int num_sms = 148;
+    // tuning overrides (0 = automatic): K splits per tile, shared-memory budget in KB
+    int tune_splits = 0, tune_smem_kb = 0;
     std::unordered_map<std::string, CUtensorMap> maps;
     const CUtensorMap *tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows);
 };

@@ -9,6 +9,10 @@
 
 namespace dfl {
 
+// Host-side count of kernels launched by this library (all contexts).
+void note_launch();
+long long launch_count();
+
 // Tap destinations of one target layer: the residual after the layer is
 // copied (rounded to T) to columns col[i] .. col[i]+H of row meta[r].aux of
 // `base` (leading dimension ld), for i < n.

@@ -15,9 +15,16 @@
 //    KV cache is rolled back by length only.
 #include <math.h>
 
+#include <atomic>
+
 #include "kernels.h"
+#include "launch.h"
 
 namespace dfl {
+
+static std::atomic<long long> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+long long launch_count() { return g_launches.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------------
 // embeddings + row metadata
@@ -28,6 +35,8 @@ __global__ void embed_block_kernel(const T *__restrict__ emb, int H, SeqState *s
                                    const int *__restrict__ active, int B, int is_draft,
                                    const int *__restrict__ drafts, int mask_id, float *__restrict__ x,
                                    RowMeta *meta, RowMeta *ctx_meta) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const int i = r / B, j = r % B;
     const int s = active[i];
@@ -61,13 +70,15 @@ template <typename T>
 void launch_embed_block(const T *emb, int H, SeqState *st, const int *active, int nseq, int B,
                         int is_draft, const int *drafts, int mask_id, float *x, RowMeta *meta,
                         RowMeta *ctx_meta, cudaStream_t s) {
-    embed_block_kernel<T><<<nseq * B, 256, 0, s>>>(emb, H, st, active, B, is_draft, drafts, mask_id,
+    launch_k(embed_block_kernel<T>, dim3(nseq * B), dim3(256), 0, s, 1, emb, H, st, active, B, is_draft, drafts, mask_id,
                                                    x, meta, ctx_meta);
 }
 
 template <typename T>
 __global__ void embed_tokens_kernel(const T *__restrict__ emb, int H, const int *__restrict__ tokens,
                                     int seq, int pos0, float *__restrict__ x, RowMeta *meta) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const int tok = tokens[r];
     const T *e = emb + (size_t)tok * H;
@@ -86,10 +97,12 @@ __global__ void embed_tokens_kernel(const T *__restrict__ emb, int H, const int 
 template <typename T>
 void launch_embed_tokens(const T *emb, int H, const int *tokens, int R, int seq, int pos0, float *x,
                          RowMeta *meta, cudaStream_t s) {
-    embed_tokens_kernel<T><<<R, 256, 0, s>>>(emb, H, tokens, seq, pos0, x, meta);
+    launch_k(embed_tokens_kernel<T>, dim3(R), dim3(256), 0, s, 1, emb, H, tokens, seq, pos0, x, meta);
 }
 
 __global__ void ctx_meta_prefill_kernel(RowMeta *meta, int R, int seq, int pos0) {
+    pdl_trigger();
+    pdl_wait();
     int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= R) return;
     RowMeta m;
@@ -101,7 +114,7 @@ __global__ void ctx_meta_prefill_kernel(RowMeta *meta, int R, int seq, int pos0)
 }
 
 void launch_ctx_meta_prefill(RowMeta *meta, int R, int seq, int pos0, cudaStream_t s) {
-    ctx_meta_prefill_kernel<<<(R + 127) / 128, 128, 0, s>>>(meta, R, seq, pos0);
+    launch_k(ctx_meta_prefill_kernel, dim3((R + 127) / 128), dim3(128), 0, s, 1, meta, R, seq, pos0);
 }
 
 // ------------------------------------------------------------------------
@@ -111,6 +124,8 @@ void launch_ctx_meta_prefill(RowMeta *meta, int R, int seq, int pos0, cudaStream
 template <typename TO>
 __global__ void rmsnorm_kernel(const float *__restrict__ x, int ldx, const float *__restrict__ g,
                                int H, float eps, TO *__restrict__ out, int ldo) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const float *xr = x + (size_t)r * ldx;
     float ss = 0.f;
@@ -134,7 +149,7 @@ template <typename TO>
 void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, TO *out, int ldo, int R,
                     cudaStream_t s) {
     if (R <= 0) return;
-    rmsnorm_kernel<TO><<<R, 256, 0, s>>>(x, ldx, g, H, eps, out, ldo);
+    launch_k(rmsnorm_kernel<TO>, dim3(R), dim3(256), 0, s, 1, x, ldx, g, H, eps, out, ldo);
 }
 
 // ------------------------------------------------------------------------
@@ -144,6 +159,8 @@ void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, T
 template <typename T>
 __global__ void residual_kernel(float *__restrict__ x, const float *__restrict__ Y, int ldy, int H,
                                 TapDst<T> taps, const RowMeta *__restrict__ meta) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     float *xr = x + (size_t)r * H;
     const float *yr = Y + (size_t)r * ldy;
@@ -160,11 +177,13 @@ template <typename T>
 void launch_residual(float *x, const float *Y, int ldy, int H, int R, const TapDst<T> &taps,
                      const RowMeta *meta, cudaStream_t s) {
     if (R <= 0) return;
-    residual_kernel<T><<<R, 256, 0, s>>>(x, Y, ldy, H, taps, meta);
+    launch_k(residual_kernel<T>, dim3(R), dim3(256), 0, s, 1, x, Y, ldy, H, taps, meta);
 }
 
 template <typename T>
 __global__ void swiglu_kernel(const float *__restrict__ Y, int ldy, int F, T *__restrict__ h, int ldh) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.y;
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= F) return;
@@ -176,7 +195,7 @@ template <typename T>
 void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, cudaStream_t s) {
     if (R <= 0) return;
     dim3 grid((F + 255) / 256, R);
-    swiglu_kernel<T><<<grid, 256, 0, s>>>(Y, ldy, F, h, ldh);
+    launch_k(swiglu_kernel<T>, dim3(grid), dim3(256), 0, s, 1, Y, ldy, F, h, ldh);
 }
 
 // Y columns c correspond to rows col0 + c of the layer's Wqkv = [Wq; Wk; Wv].
@@ -188,6 +207,8 @@ __global__ void qkv_epilogue_kernel(const float *__restrict__ Y, int ldy, int co
                                     int nq, int nkv, int hd, const float2 *__restrict__ rope,
                                     T *__restrict__ q_out, T *__restrict__ kc, T *__restrict__ vc,
                                     int max_len) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const bool is_ctx = r >= R_blk;
     RowMeta m = is_ctx ? ctx_meta[r - R_blk] : meta[r];
@@ -227,7 +248,7 @@ void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot
                          const RowMeta *ctx_meta, int nq, int nkv, int hd, const float2 *rope, T *q_out,
                          T *kc, T *vc, int max_len, cudaStream_t s) {
     if (R_tot <= 0) return;
-    qkv_epilogue_kernel<T><<<R_tot, 128, 0, s>>>(Y, ldy, col0, R_blk, meta, ctx_meta, nq, nkv, hd, rope,
+    launch_k(qkv_epilogue_kernel<T>, dim3(R_tot), dim3(128), 0, s, 1, Y, ldy, col0, R_blk, meta, ctx_meta, nq, nkv, hd, rope,
                                                  q_out, kc, vc, max_len);
 }
 
@@ -237,6 +258,8 @@ void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot
 
 __global__ void argmax_rows_kernel(const float *__restrict__ logits, int64_t ldl, int V, int mode, int B,
                                    int *__restrict__ idx, DevStats *stats) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     if (mode == 1 && (r % B) == 0) return;
     const float *l = logits + (size_t)r * ldl;
@@ -271,7 +294,7 @@ __global__ void argmax_rows_kernel(const float *__restrict__ logits, int64_t ldl
 void launch_argmax_rows(const float *logits, int64_t ldl, int V, int R, int mode, int B, int *idx,
                         DevStats *stats, cudaStream_t s) {
     if (R <= 0) return;
-    argmax_rows_kernel<<<R, 512, 0, s>>>(logits, ldl, V, mode, B, idx, stats);
+    launch_k(argmax_rows_kernel, dim3(R), dim3(512), 0, s, 1, logits, ldl, V, mode, B, idx, stats);
 }
 
 // ------------------------------------------------------------------------
@@ -281,6 +304,8 @@ void launch_argmax_rows(const float *logits, int64_t ldl, int V, int R, int mode
 __global__ void accept_kernel(SeqState *st, const int *__restrict__ active, int nseq, int B,
                               const int *__restrict__ drafts, const int *__restrict__ g, int *accept,
                               int *committed, int *new_len, int *out_tok, int out_ld, DevStats *stats) {
+    pdl_trigger();
+    pdl_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= nseq) return;
     const int s = active[i];
@@ -326,13 +351,15 @@ __global__ void accept_kernel(SeqState *st, const int *__restrict__ active, int 
 void launch_accept(SeqState *st, const int *active, int nseq, int B, const int *drafts, const int *g,
                    int *accept, int *committed, int *new_len, int *out_tok, int out_ld, DevStats *stats,
                    cudaStream_t s) {
-    accept_kernel<<<(nseq + 127) / 128, 128, 0, s>>>(st, active, nseq, B, drafts, g, accept, committed,
+    launch_k(accept_kernel, dim3((nseq + 127) / 128), dim3(128), 0, s, 1, st, active, nseq, B, drafts, g, accept, committed,
                                                      new_len, out_tok, out_ld, stats);
 }
 
 __global__ void script_drafts_kernel(const SeqState *st, const int *__restrict__ active, int nseq, int B,
                                      int tau, int V, const int *__restrict__ script, int script_ld,
                                      int *drafts) {
+    pdl_trigger();
+    pdl_wait();
     const int i = blockIdx.x;
     const int k = threadIdx.x;
     if (i >= nseq || k >= B - 1) return;
@@ -347,12 +374,14 @@ __global__ void script_drafts_kernel(const SeqState *st, const int *__restrict__
 void launch_script_drafts(const SeqState *st, const int *active, int nseq, int B, int tau, int V,
                           const int *script, int script_ld, int *drafts, cudaStream_t s) {
     if (B <= 1 || nseq <= 0) return;
-    script_drafts_kernel<<<nseq, 32 * ((B + 30) / 32), 0, s>>>(st, active, nseq, B, tau, V, script,
+    launch_k(script_drafts_kernel, dim3(nseq), dim3(32 * ((B + 30) / 32)), 0, s, 1, st, active, nseq, B, tau, V, script,
                                                                script_ld, drafts);
 }
 
 __global__ void prefill_finish_kernel(SeqState *st, int seq, int n, const int *first_tok, int *out_tok,
                                       int out_ld, int max_new) {
+    pdl_trigger();
+    pdl_wait();
     SeqState S;
     S.len = n;
     S.anchor = *first_tok;
@@ -368,12 +397,14 @@ __global__ void prefill_finish_kernel(SeqState *st, int seq, int n, const int *f
 
 void launch_prefill_finish(SeqState *st, int seq, int n, const int *first_tok, int *out_tok, int out_ld,
                            int max_new, cudaStream_t s) {
-    prefill_finish_kernel<<<1, 1, 0, s>>>(st, seq, n, first_tok, out_tok, out_ld, max_new);
+    launch_k(prefill_finish_kernel, dim3(1), dim3(1), 0, s, 1, st, seq, n, first_tok, out_tok, out_ld, max_new);
 }
 
 // target-only greedy step: g is the argmax of the single row of each sequence
 __global__ void ar_step_kernel(SeqState *st, const int *__restrict__ active, int nseq, const int *g,
                                int *out_tok, int out_ld, DevStats *stats) {
+    pdl_trigger();
+    pdl_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= nseq) return;
     const int s = active[i];
@@ -394,7 +425,7 @@ __global__ void ar_step_kernel(SeqState *st, const int *__restrict__ active, int
 
 void launch_ar_step(SeqState *st, const int *active, int nseq, const int *g, int *out_tok, int out_ld,
                     DevStats *stats, cudaStream_t s) {
-    ar_step_kernel<<<(nseq + 127) / 128, 128, 0, s>>>(st, active, nseq, g, out_tok, out_ld, stats);
+    launch_k(ar_step_kernel, dim3((nseq + 127) / 128), dim3(128), 0, s, 1, st, active, nseq, g, out_tok, out_ld, stats);
 }
 
 // ------------------------------------------------------------------------
@@ -402,6 +433,8 @@ void launch_ar_step(SeqState *st, const int *active, int nseq, const int *g, int
 // ------------------------------------------------------------------------
 
 __global__ void rope_table_kernel(float2 *tab, int max_len, int hd, double theta) {
+    pdl_trigger();
+    pdl_wait();
     const int half = hd / 2;
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= (int64_t)max_len * half) return;
@@ -414,7 +447,7 @@ __global__ void rope_table_kernel(float2 *tab, int max_len, int hd, double theta
 
 void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStream_t s) {
     const int64_t n = (int64_t)max_len * (hd / 2);
-    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(tab, max_len, hd, theta);
+    launch_k(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, 1, tab, max_len, hd, theta);
 }
 
 // ------------------------------------------------------------------------
@@ -444,6 +477,8 @@ namespace dfl {
 // dst rows i*B + j  <-  src rows active[i]*B + j  (16-byte words)
 __global__ void gather_rows_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, size_t row_words,
                                    const int *__restrict__ active, int B) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const int i = r / B, j = r % B;
     const uint4 *s = src + ((size_t)active[i] * B + j) * row_words;
@@ -454,7 +489,7 @@ __global__ void gather_rows_kernel(const uint4 *__restrict__ src, uint4 *__restr
 void launch_gather_rows(const void *src, void *dst, size_t row_bytes, const int *active, int nseq, int B,
                         cudaStream_t s) {
     if (nseq <= 0) return;
-    gather_rows_kernel<<<nseq * B, 256, 0, s>>>((const uint4 *)src, (uint4 *)dst, row_bytes / 16, active, B);
+    launch_k(gather_rows_kernel, dim3(nseq * B), dim3(256), 0, s, 1, (const uint4 *)src, (uint4 *)dst, row_bytes / 16, active, B);
 }
 
 }  // namespace dfl

@@ -5,6 +5,7 @@
 #include <math.h>
 
 #include "kernels.h"
+#include "launch.h"
 
 namespace dfl {
 
@@ -15,6 +16,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const T *__restrict__ X, int ldx, int M,
                                                         const T *__restrict__ W, int ldw, int N, int K,
                                                         float *__restrict__ Y, int ldy) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ float Ws[64][33];
     __shared__ float Xs[32][33];
     const int n0 = blockIdx.x * 64, m0 = blockIdx.y * 32;
@@ -56,7 +59,7 @@ void launch_gemm_simt(const T *X, int ldx, int M, const T *W, int ldw, int N, in
                       cudaStream_t s) {
     if (M <= 0 || N <= 0) return;
     dim3 grid((N + 63) / 64, (M + 31) / 32);
-    gemm_simt_kernel<T><<<grid, 256, 0, s>>>(X, ldx, M, W, ldw, N, K, Y, ldy);
+    launch_k(gemm_simt_kernel<T>, dim3(grid), dim3(256), 0, s, 1, X, ldx, M, W, ldw, N, K, Y, ldy);
 }
 
 // ------------------------------------------------------------------------
@@ -68,6 +71,8 @@ __global__ void attention_simt_kernel(const T *__restrict__ q, int ldq, const T 
                                       const T *__restrict__ vc, const RowMeta *__restrict__ meta, int nq,
                                       int nkv, int hd, int max_len, float scale, T *__restrict__ out,
                                       int ldo) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
     const RowMeta m = meta[r];
     const int kvh = h / (nq / nkv);
@@ -107,7 +112,7 @@ void launch_attention_simt(const T *q, int ldq, const T *kc, const T *vc, const 
                            int nkv, int hd, int max_len, T *out, int ldo, cudaStream_t s) {
     if (R <= 0) return;
     dim3 grid(R, nq);
-    attention_simt_kernel<T><<<grid, 32, 0, s>>>(q, ldq, kc, vc, meta, nq, nkv, hd, max_len,
+    launch_k(attention_simt_kernel<T>, dim3(grid), dim3(32), 0, s, 1, q, ldq, kc, vc, meta, nq, nkv, hd, max_len,
                                                  1.0f / sqrtf((float)hd), out, ldo);
 }
 
@@ -116,6 +121,8 @@ void launch_attention_simt(const T *q, int ldq, const T *kc, const T *vc, const 
 // weights renormalised over the chosen k.  One warp per row.
 // ------------------------------------------------------------------------
 __global__ void moe_topk_kernel(const float *__restrict__ lg, int E, int R, int k, int *sel, float *wt) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= R) return;
@@ -154,7 +161,7 @@ __global__ void moe_topk_kernel(const float *__restrict__ lg, int E, int R, int 
 
 void launch_moe_topk(const float *router_logits, int E, int R, int k, int *sel, float *wt, cudaStream_t s) {
     if (R <= 0) return;
-    moe_topk_kernel<<<(R + 3) / 4, 128, 0, s>>>(router_logits, E, R, k, sel, wt);
+    launch_k(moe_topk_kernel, dim3((R + 3) / 4), dim3(128), 0, s, 1, router_logits, E, R, k, sel, wt);
 }
 
 // Expert FFN per (row, choice): part[rk] = W_down_e (SiLU(W_gate_e m) * W_up_e m)
@@ -162,6 +169,8 @@ template <typename T>
 __global__ void moe_experts_simt_kernel(const T *__restrict__ m, int ldm, int k, const int *__restrict__ sel,
                                         const T *__restrict__ w_gate_up, const T *__restrict__ w_down, int H,
                                         int Fe, float *__restrict__ part) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ float sm[];
     float *xs = sm;          // [H]
     float *gu = sm + H;      // [2Fe]
@@ -193,13 +202,15 @@ void launch_moe_experts_simt(const T *m, int ldm, int R, int k, const int *sel, 
                              const T *w_down, int H, int Fe, float *part, cudaStream_t s) {
     if (R <= 0) return;
     const size_t smem = sizeof(float) * (size_t)(H + 2 * Fe);
-    moe_experts_simt_kernel<T><<<R * k, 256, smem, s>>>(m, ldm, k, sel, w_gate_up, w_down, H, Fe, part);
+    launch_k(moe_experts_simt_kernel<T>, dim3(R * k), dim3(256), smem, s, 1, m, ldm, k, sel, w_gate_up, w_down, H, Fe, part);
 }
 
 template <typename T>
 __global__ void moe_combine_kernel(float *__restrict__ x, const float *__restrict__ part,
                                    const float *__restrict__ wt, int H, int k, TapDst<T> taps,
                                    const RowMeta *__restrict__ meta) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const int trow = taps.n ? meta[r].aux : 0;
     for (int c = threadIdx.x; c < H; c += blockDim.x) {
@@ -215,7 +226,7 @@ template <typename T>
 void launch_moe_combine(float *x, const float *part, const float *wt, int H, int R, int k,
                         const TapDst<T> &taps, const RowMeta *meta, cudaStream_t s) {
     if (R <= 0) return;
-    moe_combine_kernel<T><<<R, 256, 0, s>>>(x, part, wt, H, k, taps, meta);
+    launch_k(moe_combine_kernel<T>, dim3(R), dim3(256), 0, s, 1, x, part, wt, H, k, taps, meta);
 }
 
 #define DFL_INST(T)                                                                                          \

@@ -96,7 +96,20 @@ typedef struct {
     int64_t accept_hist[DFLASH_MAX_BLOCK];  /* histogram of a (tokens committed - 1) */
     double mean_tau;              /* tokens committed per sequence-iteration */
     double ms_prefill, ms_decode; /* device time of the prefill and decode phases */
+    int64_t kernel_launches;      /* kernels this library launched (process-wide counter) */
 } dflash_stats;
+
+/* Per-class kernel timing (dflash_profile): launches, summed device time of
+ * the launches (CUDA events around each launch on the context's stream) and
+ * the algorithmic bytes they move (weights + activations read + outputs
+ * written; attention K/V bytes are not counted here). */
+typedef struct {
+    int64_t launches;
+    double ms;
+    double bytes;
+} dflash_kernel_prof;
+
+enum { DFLASH_PROF_PROJECTION = 0, DFLASH_PROF_ATTENTION = 1, DFLASH_PROF_CLASSES = 2 };
 
 /* Bytes of the weight and state arenas for this configuration.
  * Errors: DFLASH_EINVAL on inconsistent configuration, DFLASH_EUNSUPPORTED on
@@ -169,7 +182,24 @@ dflash_status dflash_generate(dflash_ctx *ctx, const int32_t *const *prompts, co
 dflash_status dflash_generate_ar(dflash_ctx *ctx, const int32_t *const *prompts, const int32_t *prompt_lens,
                                  int32_t n, int32_t max_new, int32_t *out, double *ms_decode);
 
-/* Draft mode and token scripts (see DFLASH_DRAFT_SCRIPT). tau in [1, B]. */
+/* Enqueue `iters` draft+verify iterations for slots 0..n_seqs-1 (all
+ * prefilled) without synchronising: the decode hot loop.  Capacity is checked
+ * for the worst case (every iteration commits block_size tokens).
+ * Errors: EINVAL, ESTATE, ECAPACITY. */
+dflash_status dflash_decode_iters(dflash_ctx *ctx, int32_t n_seqs, int32_t iters);
+
+/* Decode statistics accumulated on the device since the last reset (or the
+ * last dflash_generate), plus the process-wide kernel launch counter. */
+dflash_status dflash_get_stats(dflash_ctx *ctx, dflash_stats *out);
+dflash_status dflash_reset_stats(dflash_ctx *ctx);
+
+/* Per-launch CUDA-event timing of the projection and attention kernels
+ * (enable = 1 starts a fresh record, 0 stops).  Adds two event records per
+ * timed launch.  dflash_profile_read fills out[DFLASH_PROF_CLASSES]. */
+dflash_status dflash_profile(dflash_ctx *ctx, int32_t enable);
+dflash_status dflash_profile_read(dflash_ctx *ctx, dflash_kernel_prof *out);
+
+/* Draft mode (see DFLASH_DRAFT_SCRIPT); tau in [1, B]. */
 dflash_status dflash_set_draft_mode(dflash_ctx *ctx, int32_t mode, int32_t tau);
 /* script[i] is the token expected at output index i of slot `seq` (index 0 =
  * first token after the prompt); n <= max_len. */
