@@ -33,7 +33,7 @@ EXPORTS = [
     "dflash_draft_block", "dflash_verify_commit", "dflash_generate", "dflash_generate_ar",
     "dflash_set_draft_mode", "dflash_set_script", "dflash_debug_logits", "dflash_seq_state",
     "dflash_debug_kv", "dflash_decode_iters", "dflash_get_stats", "dflash_reset_stats",
-    "dflash_profile", "dflash_profile_read",
+    "dflash_profile", "dflash_profile_read", "dflash_head_argmax_noalloc",
 ]
 
 
@@ -109,6 +109,7 @@ def load_library(path: Optional[str] = None):
         "dflash_reset_stats": (_i32, [_vp]),
         "dflash_profile": (_i32, [_vp, _i32]),
         "dflash_profile_read": (_i32, [_vp, C.POINTER(KernelProf)]),
+        "dflash_head_argmax_noalloc": (_i32, [_vp, _i32, _ip, _ip]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -320,6 +321,16 @@ class DFlash:
             self.warena[base:base + numel * es].view(tdt).view(shape).copy_(t)
             del t
         torch.cuda.synchronize(self.device)
+
+    def head_argmax_noalloc(self, which: int) -> np.ndarray:
+        """Greedy ids of the rows of the last pass (0 draft, 1 verify, 2 prefill),
+        computed without any caller-provided scratch (see dflash.h)."""
+        cap = max(64, self.cfg.max_batch * self.block_size)
+        out = np.zeros(cap, np.int32)
+        n = C.c_int32()
+        self._check(self.lib.dflash_head_argmax_noalloc(self.h, which, _iptr(out), C.byref(n)),
+                    "dflash_head_argmax_noalloc")
+        return out[:n.value].copy()
 
     def set_draft_mode(self, mode: int, tau: int = 1):
         self._check(self.lib.dflash_set_draft_mode(self.h, mode, tau), "dflash_set_draft_mode")

@@ -20,12 +20,41 @@
 #include <cstdio>
 #include <cstring>
 #include <thread>
+#include <type_traits>
 
 #include "engine.h"
 #include "gemm_tc.h"
 #include "attn_mma.h"
 
 namespace dfl {
+
+// Scratch of dflash_head_argmax_noalloc: per-(vocab tile, row) partial maxima
+// for up to 64 rows and 2048 vocab tiles (vocab <= 262144), then the output ids.
+constexpr int kNoallocRows = 64;
+constexpr int kNoallocTiles = 2048;
+constexpr size_t kNoallocPartBytes = (size_t)kNoallocRows * kNoallocTiles * sizeof(float2);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocPartBytes + kNoallocRows * sizeof(int)];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side symbol is not a device address).
+static void *noalloc_scratch_ptr(std::string &err) {
+    static void *ptrs[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        err = "no current CUDA device";
+        return nullptr;
+    }
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            err = std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e);
+            return nullptr;
+        }
+        ptrs[dev] = p;
+    }
+    return ptrs[dev];
+}
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -1059,6 +1088,43 @@ class Engine : public EngineBase {
         return DFLASH_OK;
     }
 
+    // LM-head argmax of the rows of the last pass, with the per-tile partials
+    // and the output ids in caller-free static scratch (see dflash.h).
+    dflash_status head_argmax_noalloc(int which, int32_t *host_out, int32_t *rows_out, void *scratch) override {
+        if (!std::is_same<T, bf16>::value) { err = "dflash_head_argmax_noalloc needs a bf16 context"; return DFLASH_EUNSUPPORTED; }
+        if (which < 0 || which > 2 || !host_out || !rows_out) { err = "bad dflash_head_argmax_noalloc arguments"; return DFLASH_EINVAL; }
+        const int V = c.target.vocab, H = c.target.hidden, B = c.block_size;
+        const int rows = last_logits_rows[which];
+        const int n_tiles = (V + 127) / 128;
+        if (rows < 1) { err = "no pass of that kind has run on this context"; return DFLASH_ESTATE; }
+        if (rows > kNoallocRows || n_tiles > kNoallocTiles) {
+            err = "dflash_head_argmax_noalloc: more than 64 rows or a vocabulary above 262144";
+            return DFLASH_ECAPACITY;
+        }
+        float2 *part = reinterpret_cast<float2 *>(scratch);
+        int *idx = reinterpret_cast<int *>(reinterpret_cast<char *>(scratch) + kNoallocPartBytes);
+        Epi<T> e;
+        e.kind = EPI_LOGITS;
+        e.Y = nullptr;
+        e.ldy = V;
+        float2 *saved_part = tc.lm_part;
+        const int saved_keep = tc.keep_logits;
+        tc.lm_part = part;
+        tc.keep_logits = 0;
+        gemm_launch(xn, H, rows, lm_head, V, H, e);
+        tc.lm_part = saved_part;
+        tc.keep_logits = saved_keep;
+        const int mode = which == 0 ? 1 : 0;
+        launch_lm_argmax(part, n_tiles, rows, mode, B, idx, nullptr, s);
+        const int n_out = which == 0 ? (rows / B) * (B - 1) : rows;
+        dflash_status r = sync("head_argmax_noalloc");
+        if (r) return r;
+        if (n_out > 0 && cudaMemcpy(host_out, idx, sizeof(int32_t) * n_out, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return fail_cuda("head_argmax_noalloc copy");
+        *rows_out = n_out;
+        return DFLASH_OK;
+    }
+
     dflash_status set_script(int seq, const int32_t *sc, int n) override {
         if (seq < 0 || seq >= c.max_batch || !sc || n < 1 || n > c.max_len) { err = "bad script arguments"; return DFLASH_EINVAL; }
         for (int i = 0; i < n; ++i)
@@ -1202,6 +1268,17 @@ dflash_status dflash_profile(dflash_ctx *ctx, int32_t enable) { DFL_CALL(ctx, ct
 
 dflash_status dflash_profile_read(dflash_ctx *ctx, dflash_kernel_prof *out) {
     DFL_CALL(ctx, ctx->eng->profile_read(out));
+}
+
+dflash_status dflash_head_argmax_noalloc(dflash_ctx *ctx, int32_t which, int32_t *host_out, int32_t *rows_out) {
+    if (!ctx) return DFLASH_EINVAL;
+    std::string e;
+    void *scratch = noalloc_scratch_ptr(e);
+    if (!scratch) {
+        ctx->err = e;
+        return DFLASH_ECUDA;
+    }
+    DFL_CALL(ctx, ctx->eng->head_argmax_noalloc(which, host_out, rows_out, scratch));
 }
 
 dflash_status dflash_set_draft_mode(dflash_ctx *ctx, int32_t mode, int32_t tau) {

@@ -66,6 +66,7 @@ class EngineBase {
     virtual dflash_status reset_stats() = 0;
     virtual dflash_status profile(int enable) = 0;
     virtual dflash_status profile_read(dflash_kernel_prof *out) = 0;
+    virtual dflash_status head_argmax_noalloc(int which, int32_t *host_out, int32_t *rows_out, void *scratch) = 0;
     std::string err;
     int draft_mode = DFLASH_DRAFT_MODEL, tau = 1;
 };

@@ -222,6 +222,34 @@ dflash_status dflash_seq_state(dflash_ctx *ctx, int32_t seq, int32_t *len, int32
 dflash_status dflash_debug_kv(dflash_ctx *ctx, int32_t which, int32_t layer, int32_t seq,
                               int32_t p0, int32_t n, float *k_out, float *v_out);
 
+/* Greedy LM-head argmax that uses no caller-provided or allocated scratch.
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot hand the library more device memory at this point -- a serving
+ * process that reserved its whole device memory pool up front, or a runtime
+ * that forbids cudaMalloc on its decode thread (cudaMalloc can synchronise
+ * the device and may fail once the pool is carved up).
+ * It recomputes the argmax over the vocabulary of the rows that the last
+ * pass on this context fed to the LM head -- which = 0: the drafter rows of
+ * the last dflash_draft_block (outputs: n*(B-1) draft ids, as that call
+ * returns them); 1: the rows of the last dflash_verify_commit (n*B ids);
+ * 2: the last row of the last dflash_prefill (1 id) -- and must be called
+ * right after that pass, before any other call on the context.  The per-tile
+ * partial maxima and the output ids live in one file-scope device array of
+ * the library (about 1 MiB; every GPU that loads the library holds it until
+ * exit) instead of in the state arena, so the call allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ * Limits: bf16 contexts only (DFLASH_EUNSUPPORTED otherwise); at most 64 rows
+ * and a vocabulary of at most 262144 (DFLASH_ECAPACITY beyond).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array: calls whose GPU work
+ * overlaps (several contexts or streams at once) race on it.  The array keeps
+ * the last call's contents; every element a call reads is written by the
+ * same call first, so nothing needs clearing.
+ * host_out: host buffer of at least *rows_out ids (n*(B-1), n*B or 1);
+ * rows_out: receives the number of ids written.  Synchronises the stream. */
+dflash_status dflash_head_argmax_noalloc(dflash_ctx *ctx, int32_t which, int32_t *host_out, int32_t *rows_out);
+
 #ifdef __cplusplus
 }
 #endif
