@@ -18,6 +18,7 @@
 #include <chrono>
 #include <climits>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <thread>
 #include <type_traits>
@@ -25,6 +26,7 @@
 #include "engine.h"
 #include "gemm_tc.h"
 #include "attn_mma.h"
+#include "chain_tc.h"
 
 namespace dfl {
 
@@ -220,6 +222,33 @@ static Layout make_layout(const dflash_config &c) {
         L.att_ml = take(L.att_parts * 2 * 4);
         L.att_sem = take((size_t)tiles * std::max(t.n_kv_heads, d.n_kv_heads) * 4);
     }
+    // persistent projection chains (bf16 decode): folded-norm activations,
+    // per-tile sums of squares, two programs (verify, draft) and split-K partials
+    {
+        L.xg_t = take((size_t)L.R_dec * H * es);
+        L.xg2 = take((size_t)L.R_dec * H * es);
+        L.ssq_ld = 2 * L.R_dec;
+        L.ssq = take((size_t)(H / 128 + 1) * L.ssq_ld * 4);
+        const int F_d = d.ffn;
+        const int F_tmax = t.n_experts > 0 ? t.expert_ffn : t.ffn;
+        L.max_tiles = std::max({(t.vocab + 127) / 128, (qd_t + 2 * kd_t + 127) / 128, (qd_d + 2 * kd_d + 127) / 128,
+                                (F_tmax + 63) / 64, (F_d + 63) / 64, (H + 127) / 128});
+        L.n_ops_v = 1 + 4 * t.n_layers;
+        L.n_ops_d = 2 + 4 * d.n_layers;
+        auto prog_bytes = [&](int n_ops) {
+            return align_up((size_t)n_ops * sizeof(ChainOp), 256) + align_up((size_t)2 * n_ops * sizeof(CUtensorMap), 256) +
+                   align_up((size_t)n_ops * 4, 256) + align_up((size_t)n_ops * L.max_tiles * 4, 256) +
+                   align_up((size_t)n_ops * L.max_tiles * sizeof(int4), 256);
+        };
+        L.chain_v_bytes = prog_bytes(L.n_ops_v);
+        L.chain_d_bytes = prog_bytes(L.n_ops_d);
+        L.chain_v = take(L.chain_v_bytes);
+        L.chain_d = take(L.chain_d_bytes);
+        int tm_max = 16;
+        while (tm_max < 2 * L.R_dec && tm_max < 256) tm_max *= 2;
+        L.chain_ws_floats = (size_t)2 * 160 * tm_max * 128;  // units per op stay near the SM count
+        L.chain_ws = take(2 * L.chain_ws_floats * 4);
+    }
     // split-K workspace and tile semaphores of the tensor-core GEMM
     L.ws_floats = gemm_tc_workspace_floats(L.R_max, std::max(ycols, t.vocab > 0 ? H : H));
     L.gemm_ws = take((size_t)L.ws_floats * 4);
@@ -258,6 +287,13 @@ class Engine : public EngineBase {
     int *gemm_sem;
     float2 *lm_part;
     AttnScratch att;
+    // persistent projection chains (bf16 decode)
+    T *xg_t = nullptr, *xg2 = nullptr;
+    float *ssq = nullptr;
+    ChainProgram pv, pd;
+    bool chain_verify_ok = false, chain_draft_ok = false;
+    bool chain_used[3] = {false, false, false};
+    int num_sms = 148;
     GemmTC<T> tc;
     // host mirrors
     std::vector<int> h_len, h_prefilled;
@@ -351,6 +387,39 @@ class Engine : public EngineBase {
         gemm_ws = sp<float>(L.gemm_ws);
         gemm_sem = sp<int>(L.gemm_sem);
         lm_part = sp<float2>(L.lm_part);
+        xg_t = sp<T>(L.xg_t);
+        xg2 = sp<T>(L.xg2);
+        ssq = sp<float>(L.ssq);
+        {
+            int dev = 0;
+            cudaGetDevice(&dev);
+            cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+            const bool bf = std::is_same<T, bf16>::value;
+            const int H = c.target.hidden;
+            const bool shapes = H % 128 == 0 && num_sms <= 160 && 2 * L.R_dec <= 256;
+            // DFLASH_PROJECTION_CHAIN=1 runs the dependent projections of a pass as
+            // persistent chains instead of one kernel per projection (same arithmetic)
+            const char *ev = getenv("DFLASH_PROJECTION_CHAIN");
+            const bool allow = ev && ev[0] == '1';
+            chain_draft_ok = allow && bf && shapes;
+            chain_verify_ok = allow && bf && shapes && c.target.n_experts == 0;
+            auto carve = [&](ChainProgram &pg, size_t off, int n_ops) {
+                char *b = S + off;
+                pg.d_ops = reinterpret_cast<ChainOp *>(b);
+                b += align_up((size_t)n_ops * sizeof(ChainOp), 256);
+                pg.d_maps = reinterpret_cast<CUtensorMap *>(b);
+                b += align_up((size_t)2 * n_ops * sizeof(CUtensorMap), 256);
+                pg.d_op_done = reinterpret_cast<int *>(b);
+                b += align_up((size_t)n_ops * 4, 256);
+                pg.d_tile_cnt = reinterpret_cast<int *>(b);
+                b += align_up((size_t)n_ops * L.max_tiles * 4, 256);
+                pg.d_tinfo = reinterpret_cast<int4 *>(b);
+                pg.d_ws = sp<float>(L.chain_ws);
+                pg.ws_floats = L.chain_ws_floats;
+            };
+            carve(pv, L.chain_v, L.n_ops_v);
+            carve(pd, L.chain_d, L.n_ops_d);
+        }
         att.o_part = sp<float>(L.att_o);
         att.ml_part = sp<float>(L.att_ml);
         att.sem = sp<int>(L.att_sem);
@@ -629,6 +698,261 @@ class Engine : public EngineBase {
         head_argmax(xn, R, lg, mode, B, idx);
     }
 
+    // ---- persistent projection chains (bf16 decode) ----
+    static int pow2_at_least(int x, int lo) {
+        int t = lo;
+        while (t < x) t *= 2;
+        return t;
+    }
+
+    // Append one projection to a chain program (host side; uploaded by finish_program).
+    void chain_add(ChainProgram &pg, int &tile_off, int kind, const void *W, int N, int K, const T *X, int ldx, int M,
+                   const Epi<T> &e) {
+        if constexpr (std::is_same<T, bf16>::value) {
+            ChainOp op{};
+            op.kind = kind;
+            TcParams &p = op.p;
+            const bool swiglu = kind == EPI_SWIGLU;
+            p.M = M;
+            p.N = N;
+            p.K = K;
+            p.swiglu_F = swiglu ? e.F : 0;
+            p.n_tiles = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
+            p.m_tiles = 1;
+            p.k_steps = (K + 63) / 64;
+            // stream-K: CTA b streams tile-k-steps [total*b/G, total*(b+1)/G); a tile
+            // covered by several CTAs gets consecutive partial slots in the workspace
+            p.splits = 1;
+            p.err = &stats->status;
+            p.lm_part = lm_part;
+            p.keep_logits = c.keep_logits;
+            const long long total = (long long)p.n_tiles * p.k_steps;
+            // ops with fewer tile-k-steps than SMs use only the first `total` CTAs, so
+            // the CTAs covering a tile are always consecutive (slot = CTA - first CTA)
+            const int G = (int)std::min<long long>(num_sms, total);
+            std::vector<int4> ti(p.n_tiles, make_int4(-1, 0, 0, 0));
+            for (int b = 0; b < G; ++b) {
+                const long long g0 = total * b / G, g1 = total * (b + 1) / G;
+                for (long long g = g0; g < g1;) {
+                    const int nt = (int)(g / p.k_steps);
+                    if (ti[nt].x < 0) ti[nt].x = b;
+                    ti[nt].y += 1;
+                    g = std::min(g1, (long long)(nt + 1) * p.k_steps);
+                }
+            }
+            int slots = 0;
+            for (int t = 0; t < p.n_tiles; ++t) {
+                ti[t].z = slots;
+                if (ti[t].y > 1) slots += ti[t].y;
+            }
+            if ((size_t)slots * pg.tm * 128 > pg.ws_floats) pg.valid = false;  // use the per-kernel path
+            const int idx = (int)pg.ops.size();
+            CUtensorMap mw = *tc.tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
+            CUtensorMap mx = *tc.tensor_map(X, M, K, ldx, pg.tm);
+            pg.maps.push_back(mw);
+            pg.maps.push_back(mx);
+            op.wmap = pg.d_maps + 2 * idx;
+            op.xmap = pg.d_maps + 2 * idx + 1;
+            op.e = e;
+            op.ws = pg.d_ws + (size_t)(idx & 1) * pg.ws_floats;
+            op.tile_cnt = pg.d_tile_cnt + tile_off;
+            op.tinfo = pg.d_tinfo + tile_off;
+            pg.tinfo.insert(pg.tinfo.end(), ti.begin(), ti.end());
+            tile_off += p.n_tiles;
+            pg.ops.push_back(op);
+        }
+    }
+
+    void finish_program(ChainProgram &pg) {
+        cudaMemcpyAsync(pg.d_ops, pg.ops.data(), sizeof(ChainOp) * pg.ops.size(), cudaMemcpyHostToDevice, s);
+        cudaMemcpyAsync(pg.d_tinfo, pg.tinfo.data(), sizeof(int4) * pg.tinfo.size(), cudaMemcpyHostToDevice, s);
+        cudaMemcpyAsync(pg.d_maps, pg.maps.data(), sizeof(CUtensorMap) * pg.maps.size(), cudaMemcpyHostToDevice, s);
+        cudaMemsetAsync(pg.d_op_done, 0, sizeof(int) * pg.ops.size(), s);
+        cudaMemsetAsync(pg.d_tile_cnt, 0, sizeof(int) * (size_t)pg.ops.size() * L.max_tiles, s);
+        pg.epoch = 0;
+    }
+
+    Epi<T> epi_norm_in(Epi<T> e, float eps, int H) {
+        e.rs_ssq = ssq;
+        e.rs_tiles = H / 128;
+        e.rs_ld = L.ssq_ld;
+        e.rs_inv_n = 1.0f / (float)H;
+        e.rs_eps = eps;
+        return e;
+    }
+
+    Epi<T> epi_norm_out(Epi<T> e, T *xg, const float *g, float *ssq_out) {
+        e.xg = xg;
+        e.xg_ld = c.target.hidden;
+        e.g_next = g;
+        e.ssq_out = ssq_out;
+        e.ssq_ld = L.ssq_ld;
+        return e;
+    }
+
+    // verify: QKV(0) | per layer O, gate/up, down, QKV(l+1) or LM head
+    void build_verify_program(int nseq) {
+        const dflash_model_cfg &m = c.target;
+        const int B = c.block_size, R = nseq * B, H = m.hidden, hd = m.head_dim;
+        const int qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd, TK = c.n_taps * H;
+        ChainProgram &pg = pv;
+        pg.ops.clear();
+        pg.maps.clear();
+        pg.tinfo.clear();
+        pg.valid = true;
+        pg.tm = pow2_at_least(R, 16);
+        pg.key = nseq;
+        int toff = 0;
+        auto qkv = [&](int l) {
+            Epi<T> e;
+            e.kind = EPI_QKV;
+            e.R_blk = R;
+            e.meta = meta;
+            e.nq = m.n_q_heads;
+            e.nkv = m.n_kv_heads;
+            e.hd = hd;
+            e.max_len = c.max_len;
+            e.rope = rope_t;
+            e.q_out = q;
+            e.kc = tk + (size_t)l * kv_layer_elems(m);
+            e.vc = tv + (size_t)l * kv_layer_elems(m);
+            chain_add(pg, toff, EPI_QKV, tl[l].wqkv, qd + 2 * kd, H, xg_t, H, R, epi_norm_in(e, (float)m.rms_eps, H));
+        };
+        qkv(0);
+        for (int l = 0; l < m.n_layers; ++l) {
+            Epi<T> o;
+            o.kind = EPI_RESID;
+            o.x = x;
+            o.meta = meta;
+            chain_add(pg, toff, EPI_RESID, tl[l].wo, H, qd, ao, qd, R, epi_norm_out(o, xg2, tl[l].ffn_norm, ssq));
+            Epi<T> gu;
+            gu.kind = EPI_SWIGLU;
+            gu.h = h;
+            gu.F = m.ffn;
+            chain_add(pg, toff, EPI_SWIGLU, tl[l].w_gate_up, 2 * m.ffn, H, xg2, H, R, epi_norm_in(gu, (float)m.rms_eps, H));
+            Epi<T> dn;
+            dn.kind = EPI_RESID;
+            dn.x = x;
+            dn.meta = meta;
+            TapDst<T> taps{};
+            taps.base = taps_dec;
+            taps.ld = TK;
+            for (int i = 0; i < c.n_taps; ++i)
+                if (c.tap_layers[i] == l) taps.col[taps.n++] = i * H;
+            dn.taps = taps;
+            const float *gn = l + 1 < m.n_layers ? tl[l + 1].attn_norm : t_final;
+            chain_add(pg, toff, EPI_RESID, tl[l].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, xg_t, gn, ssq));
+            if (l + 1 < m.n_layers) {
+                qkv(l + 1);
+            } else {
+                Epi<T> lg;
+                lg.kind = EPI_LOGITS;
+                lg.Y = logits;
+                lg.ldy = m.vocab;
+                chain_add(pg, toff, EPI_LOGITS, lm_head, m.vocab, H, xg_t, H, R, epi_norm_in(lg, (float)m.rms_eps, H));
+            }
+        }
+        finish_program(pg);
+    }
+
+    // draft: fuse (context rows) + QKV(0) | per layer O, gate/up, down, QKV(j+1) or LM head
+    void build_draft_program(int nseq) {
+        const dflash_model_cfg &m = c.drafter;
+        const int B = c.block_size, R = nseq * B, H = m.hidden, hd = m.head_dim;
+        const int qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd, TK = c.n_taps * c.target.hidden;
+        ChainProgram &pg = pd;
+        pg.ops.clear();
+        pg.maps.clear();
+        pg.tinfo.clear();
+        pg.valid = true;
+        pg.tm = pow2_at_least(2 * R, 16);
+        pg.key = nseq;
+        int toff = 0;
+        Epi<T> f;
+        f.kind = EPI_NORMOUT;
+        chain_add(pg, toff, EPI_NORMOUT, w_fc, H, TK, taps_dec, TK, R, epi_norm_out(f, dq_in + (size_t)R * H, fc_norm, ssq + R));
+        auto qkv = [&](int j) {
+            Epi<T> e;
+            e.kind = EPI_QKV;
+            e.R_blk = R;
+            e.meta = meta;
+            e.ctx_meta = ctx_meta;
+            e.nq = m.n_q_heads;
+            e.nkv = m.n_kv_heads;
+            e.hd = hd;
+            e.max_len = c.max_len;
+            e.rope = rope_d;
+            e.q_out = q;
+            e.kc = dk + (size_t)j * kv_layer_elems(m);
+            e.vc = dv + (size_t)j * kv_layer_elems(m);
+            chain_add(pg, toff, EPI_QKV, dl[j].wqkv, qd + 2 * kd, H, dq_in, H, 2 * R, epi_norm_in(e, (float)m.rms_eps, H));
+        };
+        qkv(0);
+        for (int j = 0; j < m.n_layers; ++j) {
+            Epi<T> o;
+            o.kind = EPI_RESID;
+            o.x = x;
+            o.meta = meta;
+            chain_add(pg, toff, EPI_RESID, dl[j].wo, H, qd, ao, qd, R, epi_norm_out(o, xg2, dl[j].ffn_norm, ssq));
+            Epi<T> gu;
+            gu.kind = EPI_SWIGLU;
+            gu.h = h;
+            gu.F = m.ffn;
+            chain_add(pg, toff, EPI_SWIGLU, dl[j].w_gate_up, 2 * m.ffn, H, xg2, H, R, epi_norm_in(gu, (float)m.rms_eps, H));
+            Epi<T> dn;
+            dn.kind = EPI_RESID;
+            dn.x = x;
+            dn.meta = meta;
+            if (j + 1 < m.n_layers) {
+                chain_add(pg, toff, EPI_RESID, dl[j].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, dq_in, dl[j + 1].attn_norm, ssq));
+                qkv(j + 1);
+            } else {
+                chain_add(pg, toff, EPI_RESID, dl[j].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, xg_t, d_final, ssq));
+                Epi<T> lg;
+                lg.kind = EPI_LOGITS;
+                lg.Y = logits;
+                lg.ldy = c.target.vocab;
+                chain_add(pg, toff, EPI_LOGITS, lm_head, c.target.vocab, H, xg_t, H, R, epi_norm_in(lg, (float)m.rms_eps, H));
+            }
+        }
+        finish_program(pg);
+    }
+
+    void enqueue_verify_chain(int nseq) {
+        const dflash_model_cfg &t = c.target;
+        const int B = c.block_size, R = nseq * B, H = t.hidden;
+        if (pv.key != nseq) build_verify_program(nseq);
+        pv.epoch++;
+        launch_embed_norm<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, tl[0].attn_norm,
+                             xg_t, H, ssq, L.ssq_ld, s);
+        launch_chain(pv, 0, 1, num_sms, &stats->status, s);
+        for (int l = 0; l < t.n_layers; ++l) {
+            attention(q, tk + (size_t)l * kv_layer_elems(t), tv + (size_t)l * kv_layer_elems(t), meta, R, B, t, ao);
+            launch_chain(pv, 1 + 4 * l, 5 + 4 * l, num_sms, &stats->status, s);
+        }
+        launch_lm_argmax(lm_part, (t.vocab + 127) / 128, R, 0, B, g, stats, s);
+        launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
+        chain_used[1] = true;
+    }
+
+    void enqueue_draft_chain(int nseq) {
+        const dflash_model_cfg &d = c.drafter;
+        const int B = c.block_size, R = nseq * B, H = d.hidden;
+        if (pd.key != nseq) build_draft_program(nseq);
+        pd.epoch++;
+        launch_embed_norm<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, dl[0].attn_norm,
+                             dq_in, H, ssq, L.ssq_ld, s);
+        launch_chain(pd, 0, 2, num_sms, &stats->status, s);
+        for (int j = 0; j < d.n_layers; ++j) {
+            attention(q, dk + (size_t)j * kv_layer_elems(d), dv + (size_t)j * kv_layer_elems(d), meta, R, B, d, ao);
+            launch_chain(pd, 2 + 4 * j, 6 + 4 * j, num_sms, &stats->status, s);
+        }
+        if (B > 1) launch_lm_argmax(lm_part, (c.target.vocab + 127) / 128, R, 1, B, drafts, stats, s);
+        if (draft_mode == DFLASH_DRAFT_SCRIPT)
+            launch_script_drafts(st, active, nseq, B, tau, c.target.vocab, script, c.max_len, drafts, s);
+        chain_used[0] = true;
+    }
+
     // ---- steps ----
     void enqueue_prefill(int seq, int n, int max_new) {
         const dflash_model_cfg &t = c.target, &d = c.drafter;
@@ -672,6 +996,14 @@ class Engine : public EngineBase {
     }
 
     void enqueue_draft(int nseq, bool contiguous) {
+        if (chain_draft_ok && contiguous) {
+            if (pd.key != nseq) build_draft_program(nseq);
+            if (pd.valid) {
+                enqueue_draft_chain(nseq);
+                return;
+            }
+        }
+        chain_used[0] = false;
         const dflash_model_cfg &t = c.target, &d = c.drafter;
         const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
         launch_embed_block<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, s);
@@ -694,6 +1026,14 @@ class Engine : public EngineBase {
     }
 
     void enqueue_verify(int nseq) {
+        if (chain_verify_ok) {
+            if (pv.key != nseq) build_verify_program(nseq);
+            if (pv.valid) {
+                enqueue_verify_chain(nseq);
+                return;
+            }
+        }
+        chain_used[1] = false;
         const dflash_model_cfg &t = c.target;
         const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
         launch_embed_block<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
@@ -1111,7 +1451,13 @@ class Engine : public EngineBase {
         const int saved_keep = tc.keep_logits;
         tc.lm_part = part;
         tc.keep_logits = 0;
-        gemm_launch(xn, H, rows, lm_head, V, H, e);
+        if (which < 2 && chain_used[which]) {
+            // chain passes feed the head bf16(x * g_final) and scale each row by its RMSNorm factor
+            const float eps = (float)(which == 0 ? c.drafter.rms_eps : c.target.rms_eps);
+            gemm_launch(xg_t, H, rows, lm_head, V, H, epi_norm_in(e, eps, H));
+        } else {
+            gemm_launch(xn, H, rows, lm_head, V, H, e);
+        }
         tc.lm_part = saved_part;
         tc.keep_logits = saved_keep;
         const int mode = which == 0 ? 1 : 0;

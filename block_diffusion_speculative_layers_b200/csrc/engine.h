@@ -35,6 +35,9 @@ struct Layout {
     size_t rope_t, rope_d, tk, tv, dk, dv, script, out_tok, tokens, stats, first_tok;
     size_t moe_sel, moe_wt, moe_part, lm_part, att_o, att_ml, att_sem;
     size_t att_parts = 0;
+    size_t xg_t, xg2, ssq, chain_v, chain_d, chain_ws;
+    size_t chain_v_bytes = 0, chain_d_bytes = 0, chain_ws_floats = 0;
+    int ssq_ld = 0, n_ops_v = 0, n_ops_d = 0, max_tiles = 0;
     size_t gemm_ws, gemm_sem;
     size_t state_bytes = 0;
     // dims

@@ -30,6 +30,10 @@ void launch_embed_block(const T *emb, int H, SeqState *st, const int *active, in
                         int is_draft, const int *drafts, int mask_id, float *x, RowMeta *meta,
                         RowMeta *ctx_meta, cudaStream_t s);
 template <typename T>
+void launch_embed_norm(const T *emb, int H, SeqState *st, const int *active, int nseq, int B, int is_draft,
+                       const int *drafts, int mask_id, float *x, RowMeta *meta, RowMeta *ctx_meta, const float *g, T *xg,
+                       int xg_ld, float *ssq, int ssq_ld, cudaStream_t s);
+template <typename T>
 void launch_embed_tokens(const T *emb, int H, const int *tokens, int R, int seq, int pos0,
                          float *x, RowMeta *meta, cudaStream_t s);
 void launch_ctx_meta_prefill(RowMeta *meta, int R, int seq, int pos0, cudaStream_t s);
@@ -92,7 +96,7 @@ void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStrea
 namespace dfl {
 
 // Epilogue of a projection Y[M][N] = X[M][K] . W[N][K]^T.
-enum EpiKind { EPI_STORE = 0, EPI_QKV = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_LOGITS = 4 };
+enum EpiKind { EPI_STORE = 0, EPI_QKV = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_LOGITS = 4, EPI_NORMOUT = 5 };
 
 template <typename T>
 struct Epi {
@@ -113,6 +117,20 @@ struct Epi {
     // EPI_SWIGLU: N = 2F, columns [gate; up]; h[M][F] = SiLU(gate) * up
     T *h = nullptr;
     int F = 0;
+    // RMSNorm folded into the projection.  Consumer side (QKV, SwiGLU, logits,
+    // store): the input rows are bf16(x * g) and the result of row m is scaled
+    // by 1/sqrt(sum_t rs_ssq[t*rs_ld + m] * rs_inv_n + rs_eps).
+    const float *rs_ssq = nullptr;
+    int rs_tiles = 0, rs_ld = 0;
+    float rs_inv_n = 0.f, rs_eps = 0.f;
+    // Producer side (EPI_RESID after the add, EPI_NORMOUT on the raw result y):
+    // xg[m][n] = bf16(y[m][n] * g_next[n]) and ssq_out[tile*ssq_ld + m] =
+    // sum of y^2 over the tile's 128 columns (for the next projection's norm).
+    T *xg = nullptr;
+    int xg_ld = 0;
+    const float *g_next = nullptr;
+    float *ssq_out = nullptr;
+    int ssq_ld = 0;
 };
 
 void launch_gather_rows(const void *src, void *dst, size_t row_bytes, const int *active, int nseq, int B,

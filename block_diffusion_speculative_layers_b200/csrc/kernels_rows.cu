@@ -74,6 +74,69 @@ void launch_embed_block(const T *emb, int H, SeqState *st, const int *active, in
                                                    x, meta, ctx_meta);
 }
 
+// Block rows as embed_block_kernel, plus the folded RMSNorm inputs of the first
+// projection: xg = bf16(x * g) and per-128-column-tile sums of squares.
+template <typename T>
+__global__ void embed_norm_kernel(const T *__restrict__ emb, int H, SeqState *st, const int *__restrict__ active, int B,
+                                  int is_draft, const int *__restrict__ drafts, int mask_id, float *__restrict__ x,
+                                  RowMeta *meta, RowMeta *ctx_meta, const float *__restrict__ g, T *__restrict__ xg,
+                                  int xg_ld, float *__restrict__ ssq, int ssq_ld) {
+    pdl_trigger();
+    pdl_wait();
+    __shared__ float red[8];
+    const int r = blockIdx.x;
+    const int i = r / B, j = r % B;
+    const int s = active[i];
+    const SeqState S = st[s];
+    const int p = S.len;
+    const int tok = j == 0 ? S.anchor : (is_draft ? mask_id : drafts[i * (B - 1) + (j - 1)]);
+    const T *e = emb + (size_t)tok * H;
+    for (int t0 = 0; t0 < H; t0 += 256) {
+        const int c = t0 + threadIdx.x;
+        float v = 0.f;
+        if (c < H) {
+            v = to_f(e[c]);
+            x[(size_t)r * H + c] = v;
+            xg[(size_t)r * xg_ld + c] = from_f<T>(v * g[c]);
+        }
+        float sq = warp_sum(v * v);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
+        __syncthreads();
+        if (threadIdx.x < 2) {  // two 128-column tiles per pass
+            const int tile = t0 / 128 + threadIdx.x;
+            if (tile * 128 < H) {
+                const float* rr = red + 4 * threadIdx.x;
+                ssq[(size_t)tile * ssq_ld + r] = (rr[0] + rr[1]) + (rr[2] + rr[3]);
+            }
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        RowMeta m;
+        m.seq = s;
+        m.pos = p + j;
+        m.nk = is_draft ? p + B : p + j + 1;
+        m.aux = s * B + j;
+        meta[r] = m;
+        if (is_draft && ctx_meta) {
+            RowMeta c;
+            c.seq = s;
+            c.pos = S.pend_pos0 + j;
+            c.nk = 0;
+            c.aux = (j < S.pend_n) ? 1 : 0;
+            ctx_meta[r] = c;
+        }
+    }
+}
+
+template <typename T>
+void launch_embed_norm(const T *emb, int H, SeqState *st, const int *active, int nseq, int B, int is_draft,
+                       const int *drafts, int mask_id, float *x, RowMeta *meta, RowMeta *ctx_meta, const float *g, T *xg,
+                       int xg_ld, float *ssq, int ssq_ld, cudaStream_t s) {
+    launch_k(embed_norm_kernel<T>, dim3(nseq * B), dim3(256), 0, s, 1, emb, H, st, active, B, is_draft, drafts, mask_id, x,
+             meta, ctx_meta, g, xg, xg_ld, ssq, ssq_ld);
+}
+
 template <typename T>
 __global__ void embed_tokens_kernel(const T *__restrict__ emb, int H, const int *__restrict__ tokens,
                                     int seq, int pos0, float *__restrict__ x, RowMeta *meta) {
@@ -454,6 +517,9 @@ void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStrea
 // explicit instantiations
 // ------------------------------------------------------------------------
 #define DFL_INST(T)                                                                                         \
+    template void launch_embed_norm<T>(const T *, int, SeqState *, const int *, int, int, int, const int *, int, \
+                                       float *, RowMeta *, RowMeta *, const float *, T *, int, float *, int,     \
+                                       cudaStream_t);                                                           \
     template void launch_embed_block<T>(const T *, int, SeqState *, const int *, int, int, int, const int *, \
                                         int, float *, RowMeta *, RowMeta *, cudaStream_t);                  \
     template void launch_embed_tokens<T>(const T *, int, const int *, int, int, int, float *, RowMeta *,    \

@@ -1,0 +1,333 @@
+// tc_device.cuh -- device helpers shared by the tensor-core projection kernels:
+// mbarriers, TMA tile loads, tcgen05 descriptors/MMA/TMEM loads, cluster
+// helpers and the fused projection epilogues.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include "gemm_tc.h"
+
+namespace dfl {
+namespace tc {
+
+constexpr int BK = 64;                 // bf16 K elements per stage = one 128-byte swizzle row
+constexpr int A_BYTES = 128 * BK * 2;  // 16 KB weight tile per stage
+constexpr int NT = 192;
+constexpr int CH = 16;                 // accumulator columns per epilogue chunk
+constexpr int STG_LD = CH + 1;
+constexpr unsigned long long WAIT_NS = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: false (and error bit 4) after WAIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, int *err) {
+    if (mbar_try(b, parity)) return true;
+    const unsigned long long t0 = gtimer();
+    while (true) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try(b, parity)) return true;
+        if (gtimer() - t0 > WAIT_NS) {
+            if (err) atomicOr(err, 4);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// K-major operand, 128-byte swizzle: 8-row groups 1024 B apart (SBO), sm100 descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;               // leading byte offset (16 B; unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset
+    d |= (uint64_t)1 << 46;               // descriptor version
+    d |= (uint64_t)2 << 61;               // SWIZZLE_128B
+    return d;
+}
+
+// bf16 x bf16 -> fp32, A and B K-major, M = 128, N = tm.
+__host__ __device__ constexpr uint32_t idesc_bf16(int tm) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(tm >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// ---------------------------------------------------------------------------
+// fused epilogue on one chunk of up to CH accumulator columns (activation rows
+// m0c .. m0c+nc-1) for weight row n_local of the tile.  Global loads of a
+// chunk are issued together before any use.
+// ---------------------------------------------------------------------------
+// Per-row RMSNorm scale of the chunk's rows (folded norm), computed by 16
+// threads into rsc[] and published with a named barrier.
+__device__ __forceinline__ void row_scales(const Epi<bf16> &e, int m0c, int nc, int M, float *rsc) {
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+        const int j = threadIdx.x - 64, m = m0c + j;
+        float sc = 1.f;
+        if (e.rs_ssq && j < nc && m < M) {
+            float ss = 0.f;
+            for (int t = 0; t < e.rs_tiles; ++t) ss += e.rs_ssq[(size_t)t * e.rs_ld + m];
+            sc = 1.0f / sqrtf(ss * e.rs_inv_n + e.rs_eps);
+        }
+        rsc[j] = sc;
+    }
+    epi_bar();
+}
+
+// y -> bf16(y * g_next) and the tile's per-row sum of squares (fixed reduction order).
+__device__ __forceinline__ void norm_outputs(const TcParams &p, const Epi<bf16> &e, int nt, int n, int q, int lane,
+                                             int m0c, int nc, const float *y, float2 *red) {
+    const int M = p.M;
+    const bool nok = n < p.N;
+    const float gn = (nok && e.g_next) ? e.g_next[n] : 0.f;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+        const bool ok = nok && j < nc && m0c + j < M;
+        if (ok && e.xg) e.xg[(size_t)(m0c + j) * e.xg_ld + n] = __float2bfloat16_rn(y[j] * gn);
+        float sq = ok ? y[j] * y[j] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) red[q * CH + j].x = sq;
+    }
+    epi_bar();
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+        const int j = threadIdx.x - 64, m = m0c + j;
+        if (j < nc && m < M && e.ssq_out)
+            e.ssq_out[(size_t)nt * e.ssq_ld + m] = (red[j].x + red[CH + j].x) + (red[2 * CH + j].x + red[3 * CH + j].x);
+    }
+    epi_bar();
+}
+
+template <int KIND>
+__device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16> &e, int nt, int n_local, int q,
+                                               int lane, int m0c, int nc, const float *vin, float *stg, float2 *red,
+                                               RowMeta *smeta, float *rsc) {
+    const int M = p.M;
+    float v[CH];
+    if (KIND == EPI_QKV || KIND == EPI_SWIGLU || KIND == EPI_LOGITS || KIND == EPI_STORE) {
+        if (e.rs_ssq) {
+            row_scales(e, m0c, nc, M, rsc);
+#pragma unroll
+            for (int j = 0; j < CH; ++j) v[j] = vin[j] * rsc[j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) v[j] = vin[j];
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) v[j] = vin[j];
+    }
+    if (KIND == EPI_STORE) {
+        const int n = nt * 128 + n_local;
+        if (n < p.N) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+                if (j < nc && m0c + j < M) e.Y[(size_t)(m0c + j) * e.ldy + n] = v[j];
+        }
+    } else if (KIND == EPI_RESID) {
+        const int n = nt * 128 + n_local;
+        const bool nok = n < p.N;
+        float xo[CH];
+        int trow[CH];
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            const bool ok = nok && j < nc && m0c + j < M;
+            xo[j] = ok ? e.x[(size_t)(m0c + j) * p.N + n] : 0.f;
+            trow[j] = (ok && e.taps.n) ? e.meta[m0c + j].aux : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            if (!(nok && j < nc && m0c + j < M)) continue;
+            const float nx = xo[j] + v[j];
+            xo[j] = nx;
+            e.x[(size_t)(m0c + j) * p.N + n] = nx;
+            for (int t = 0; t < e.taps.n; ++t)
+                e.taps.base[(size_t)trow[j] * e.taps.ld + e.taps.col[t] + n] = __float2bfloat16_rn(nx);
+        }
+        if (e.ssq_out) norm_outputs(p, e, nt, n, q, lane, m0c, nc, xo, red);
+    } else if (KIND == EPI_NORMOUT) {
+        norm_outputs(p, e, nt, nt * 128 + n_local, q, lane, m0c, nc, v, red);
+    } else if (KIND == EPI_LOGITS) {
+        const int n = nt * 128 + n_local;
+        const bool ok = n < p.N;
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            const int m = m0c + j;
+            const bool col = j < nc && m < M;
+            if (p.keep_logits && ok && col) e.Y[(size_t)m * e.ldy + n] = v[j];
+            float bv = (ok && col) ? v[j] : -INFINITY;
+            int bi = (ok && col) ? n : 0x7fffffff;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+                argmax_merge(bv, bi, v2, i2);
+            }
+            if (lane == 0) red[q * CH + j] = make_float2(bv, __int_as_float(bi));
+        }
+        epi_bar();
+        if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+            const int j = threadIdx.x - 64;
+            const int m = m0c + j;
+            float bv = red[j].x;
+            int bi = __float_as_int(red[j].y);
+            for (int qq = 1; qq < 4; ++qq) argmax_merge(bv, bi, red[qq * CH + j].x, __float_as_int(red[qq * CH + j].y));
+            if (j < nc && m < M) p.lm_part[(size_t)nt * p.M + m] = make_float2(bv, __int_as_float(bi));
+        }
+        epi_bar();
+    } else if (KIND == EPI_SWIGLU) {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) stg[n_local * STG_LD + j] = v[j];
+        epi_bar();
+        if (n_local < 64) {
+            const int f = nt * 64 + n_local;
+            if (f < p.swiglu_F) {
+#pragma unroll
+                for (int j = 0; j < CH; ++j) {
+                    const int m = m0c + j;
+                    if (j >= nc || m >= M) break;
+                    const float up = stg[(n_local + 64) * STG_LD + j];
+                    e.h[(size_t)m * p.swiglu_F + f] = __float2bfloat16_rn(silu_f(v[j]) * up);
+                }
+            }
+        }
+        epi_bar();
+    } else if (KIND == EPI_QKV) {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) stg[n_local * STG_LD + j] = v[j];
+        if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+            const int j = threadIdx.x - 64, m = m0c + j;
+            RowMeta mt;
+            mt.seq = mt.pos = mt.nk = 0;
+            mt.aux = -1;  // -1: skip this column
+            if (j < nc && m < M) {
+                if (m >= e.R_blk) {
+                    mt = e.ctx_meta[m - e.R_blk];
+                    mt.aux = mt.aux ? 1 : -1;
+                } else {
+                    mt = e.meta[m];
+                    mt.aux = 0;
+                }
+            }
+            smeta[j] = mt;
+        }
+        epi_bar();
+        const int hd = e.hd, half = hd >> 1;
+        const int qd = e.nq * hd, kd = e.nkv * hd;
+        const int cg = e.col0 + nt * 128 + n_local;  // row of [Wq; Wk; Wv]
+        if (nt * 128 + n_local < p.N) {
+            const int head_base = (cg / hd) * hd;
+            const int d = cg - head_base;
+            const int partner = n_local + (d < half ? half : -half);
+            const int i = d < half ? d : d - half;
+            const bool is_q = cg < qd, is_k = !is_q && cg < qd + kd;
+            float2 cs[CH];
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+                cs[j] = (is_q || is_k) && smeta[j].aux >= 0 ? e.rope[(size_t)smeta[j].pos * half + i] : make_float2(1.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+                const RowMeta mt = smeta[j];
+                if (mt.aux < 0) continue;          // padding column or uncommitted context row
+                const bool ctx = mt.aux == 1;
+                if (ctx && is_q) continue;         // context rows only feed K/V
+                float out = v[j];
+                if (is_q || is_k) {
+                    const float other = stg[partner * STG_LD + j];
+                    out = d < half ? v[j] * cs[j].x - other * cs[j].y : v[j] * cs[j].x + other * cs[j].y;
+                }
+                if (is_q) {
+                    e.q_out[(size_t)(m0c + j) * qd + cg] = __float2bfloat16_rn(out);
+                } else {
+                    const int hh = is_k ? (cg - qd) / hd : (cg - qd - kd) / hd;
+                    bf16 *dst = (is_k ? e.kc : e.vc) + (((size_t)mt.seq * e.nkv + hh) * e.max_len + mt.pos) * hd;
+                    dst[d] = __float2bfloat16_rn(out);
+                }
+            }
+        }
+        epi_bar();
+    }
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// generic address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ const float *peer_ptr(const float *p, uint32_t rank) {
+    uint64_t out;
+    asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+    return reinterpret_cast<const float *>(out);
+}
+
+}  // namespace tc
+}  // namespace dfl

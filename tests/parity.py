@@ -22,6 +22,7 @@ import block_diffusion_speculative_layers_b200 as dfl
 import oracle
 from oracle import api as orc
 from synthetic import make_weights
+from synthetic.fast import make_weights_host
 
 
 @dataclass
@@ -42,7 +43,7 @@ def accept_rule(drafts, g) -> int:
 
 
 def build_pair(cfg, max_batch=1, max_len=256, random_gains=True, prefill_chunk=0, seed=None):
-    w_cpu = make_weights(cfg, random_gains=random_gains, seed=seed)
+    w_cpu = make_weights_host(cfg, random_gains=random_gains, seed=seed)
     gpu = dfl.DFlash(cfg, max_batch=max_batch, max_len=max_len, prefill_chunk=prefill_chunk, keep_logits=True)
     w_gpu = make_weights(cfg, device="cuda", random_gains=random_gains, seed=seed)
     gpu.load_weights(w_gpu)

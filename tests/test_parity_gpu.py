@@ -27,12 +27,13 @@ TOL = {"fp32": (1e-4, 1e-3), "bf16": (3e-2, 0.05)}
 def tiny_cfg(dtype="fp32", block=4, moe=False, t_layers=2, d_layers=1, nq=4, nkv=2, hd=64, hidden=256,
              vocab=1024, taps=(0, 1)):
     base = get_config("tiny")
+    ffn = 3 * hidden
     t = replace(base.target, n_layers=t_layers, n_q_heads=nq, n_kv_heads=nkv, head_dim=hd, hidden=hidden,
-                vocab=vocab)
+                vocab=vocab, ffn=ffn)
     if moe:
         t = replace(t, n_experts=8, top_k=2, expert_ffn=64)
     d = replace(base.drafter, n_layers=d_layers, n_q_heads=nq, n_kv_heads=nkv, head_dim=hd, hidden=hidden,
-                vocab=vocab)
+                vocab=vocab, ffn=ffn)
     return base.with_(target=t, drafter=d, block_size=block, tap_layers=taps, dtype=dtype)
 
 
@@ -62,7 +63,7 @@ def test_config1_generate_is_lossless(cuda_device):
     assert 1.0 <= st.mean_tau <= cfg.block_size
 
 
-@pytest.mark.parametrize("case", ["block16", "moe", "mha_hd128", "chunked_prefill", "batch3"])
+@pytest.mark.parametrize("case", ["block16", "moe", "mha_hd128", "chunked_prefill", "batch3", "wide", "wide_batch2"])
 def test_bf16_variants_replay(cuda_device, case):
     kw = dict(dtype="bf16")
     prompts_n, lens, chunk = 1, [40], 0
@@ -78,6 +79,11 @@ def test_bf16_variants_replay(cuda_device, case):
     if case == "batch3":
         kw.update(block=8)
         lens = [17, 40, 33]
+    if case in ("wide", "wide_batch2"):
+        # wide enough that projections split K across CTAs (16-48 tiles per projection)
+        kw.update(block=16, hidden=2048, nq=16, nkv=4, hd=128, vocab=8192)
+        if case == "wide_batch2":
+            lens = [30, 21]
     cfg = tiny_cfg(**kw)
     tol, tie = TOL["bf16"]
     gpu, spec, _ = build_pair(cfg, max_batch=len(lens), max_len=256, prefill_chunk=chunk)
