@@ -110,10 +110,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ bytes
-def iteration_bytes(cfg, batch: int, mean_ctx: float) -> float:
+def iteration_bytes(cfg, batch: int, mean_ctx: float, kv_planes: int = 1) -> float:
     """Algorithmic HBM bytes of one draft+verify iteration: every projection
     matrix once (the LM head twice: drafter and target), plus K/V reads of both
-    models at the mean context length."""
+    models at the mean context length (kv_planes bf16 planes per element)."""
     es = 2 if cfg.dtype == "bf16" else 4
     shapes = weight_shapes(cfg)
     w = 0
@@ -125,7 +125,7 @@ def iteration_bytes(cfg, batch: int, mean_ctx: float) -> float:
             continue  # MoE experts are counted by touched experts elsewhere
         w += n * es * (2 if name == "lm_head" else 1)
     t, d = cfg.target, cfg.drafter
-    kv = batch * (mean_ctx + cfg.block_size) * 2 * es * (t.n_layers * t.n_kv_heads * t.head_dim
+    kv = batch * (mean_ctx + cfg.block_size) * 2 * es * kv_planes * (t.n_layers * t.n_kv_heads * t.head_dim
                                                           + d.n_layers * d.n_kv_heads * d.head_dim)
     return float(w * (1 if batch else 0) + kv)
 
@@ -172,6 +172,8 @@ def main():
     ap.add_argument("--prompt-len", type=int, default=None)
     ap.add_argument("--forced", default="1,4,8,16", help="forced accept lengths to time ('' = none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bf16-act", choices=["split", "fast"], default="split",
+                    help="bf16 activations as two planes (parity-grade) or one plane")
     ap.add_argument("--e2e-tokens", type=int, default=128)
     ap.add_argument("--target-layers", type=int, default=None, help="layer-reduced copy (profiling small cases)")
     ap.add_argument("--drafter-layers", type=int, default=None)
@@ -210,7 +212,7 @@ def main():
     max_new_cap = (args.warmup + args.steps + 8) * B
     max_len = cfg.prompt_len + max(max_new_cap, args.e2e_tokens + 2 * B, 2048) + 2 * B
     log(f"[rank {rank}] building context: {cfg.name} batch {b} max_len {max_len}")
-    ctx = dfl.DFlash(cfg, max_batch=b, max_len=max_len, device=dev)
+    ctx = dfl.DFlash(cfg, max_batch=b, max_len=max_len, device=dev, bf16_act=args.bf16_act)
     t0 = time.time()
     ctx.load_weights_from(lambda n: make_weight(cfg, n, device=dev))
     log(f"[rank {rank}] weights generated + loaded in {time.time() - t0:.1f}s ({ctx.weight_bytes / 1e9:.2f} GB)")
@@ -263,7 +265,7 @@ def main():
     value = tok_sum / (ms_max / 1000.0)
     mean_tau = st.mean_tau
     ctx_len_mean = cfg.prompt_len + args.warmup * mean_tau + 0.5 * args.steps * mean_tau
-    it_bytes = iteration_bytes(cfg, b, ctx_len_mean)
+    it_bytes = iteration_bytes(cfg, b, ctx_len_mean, 2 if (cfg.dtype == "bf16" and args.bf16_act == "split") else 1)
     us_iter = ms_max * 1000.0 / args.steps
     log(f"[rank {rank}] {args.steps} iters in {ms:.2f} ms: {us_iter:.1f} us/iter, tau {mean_tau:.3f}, "
         f"{value:.1f} tok/s, launches {launches}")
@@ -359,6 +361,8 @@ def main():
                                f"batch {b} per GPU, {cfg.prompt_len}-token prompt",
                    "global_batch": b * world, "seq_len": cfg.prompt_len, "block_size": B,
                    "parallelism": f"replicas x{world}",
+                   "activations": ("bf16 hi+lo planes, fp32 accumulate" if args.bf16_act == "split"
+                                   else "bf16 single plane, fp32 accumulate") if cfg.dtype == "bf16" else "fp32",
                    "l2": "inputs larger than L2 (18.5 GB of weights streamed per step)"},
         "us_per_iter": round(us_iter, 2),
         "mean_tau": round(mean_tau, 4),

@@ -19,7 +19,7 @@ from .build import lib_path
 
 DFLASH_OK, DFLASH_EINVAL, DFLASH_ESTATE, DFLASH_ECAPACITY = 0, 1, 2, 3
 DFLASH_ECUDA, DFLASH_ENUMERIC, DFLASH_ETIMEOUT, DFLASH_EUNSUPPORTED = 4, 5, 6, 7
-DFLASH_FP32, DFLASH_BF16 = 0, 1
+DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST = 0, 1, 2
 DFLASH_DRAFT_MODEL, DFLASH_DRAFT_SCRIPT = 0, 1
 MAX_TAPS, MAX_BLOCK = 8, 16
 
@@ -125,9 +125,13 @@ def _model_cfg(d) -> ModelCfg:
 
 
 def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: int = 0,
-                keep_logits: bool = False, timeout_ms: int = 0) -> Config:
+                keep_logits: bool = False, timeout_ms: int = 0, bf16_act: str = "split") -> Config:
     """dflash_config from any object with target/drafter dims, block_size, tap_layers,
-    mask_id and dtype ("bf16" / "fp32") attributes."""
+    mask_id and dtype ("bf16" / "fp32") attributes.  bf16_act selects how a bf16
+    model carries its activations: "split" (two bf16 planes, DFLASH_BF16) or
+    "fast" (one plane, DFLASH_BF16_FAST)."""
+    if bf16_act not in ("split", "fast"):
+        raise ValueError("bf16_act must be 'split' or 'fast'")
     c = Config()
     c.target = _model_cfg(spec.target)
     c.drafter = _model_cfg(spec.drafter)
@@ -142,7 +146,10 @@ def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: in
     c.max_batch = max_batch
     c.max_len = max_len
     c.prefill_chunk = prefill_chunk
-    c.dtype = DFLASH_BF16 if spec.dtype == "bf16" else DFLASH_FP32
+    if spec.dtype == "bf16":
+        c.dtype = DFLASH_BF16 if bf16_act == "split" else DFLASH_BF16_FAST
+    else:
+        c.dtype = DFLASH_FP32
     c.keep_logits = 1 if keep_logits else 0
     c.timeout_ms = timeout_ms
     return c
@@ -161,10 +168,10 @@ class DFlash:
 
     def __init__(self, spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: int = 0,
                  keep_logits: bool = False, device: Optional[torch.device] = None,
-                 stream: Optional[torch.cuda.Stream] = None, timeout_ms: int = 0):
+                 stream: Optional[torch.cuda.Stream] = None, timeout_ms: int = 0, bf16_act: str = "split"):
         self.lib = load_library()
         self.spec = spec
-        self.cfg = make_config(spec, max_batch, max_len, prefill_chunk, keep_logits, timeout_ms)
+        self.cfg = make_config(spec, max_batch, max_len, prefill_chunk, keep_logits, timeout_ms, bf16_act)
         self.device = torch.device(device or "cuda")
         wb, sb = _sz(), _sz()
         self._check(self.lib.dflash_workspace_size(C.byref(self.cfg), C.byref(wb), C.byref(sb)),
@@ -364,4 +371,4 @@ class DFlash:
 
 
 __all__ = ["DFlash", "DFlashError", "load_library", "make_config", "Config", "Stats", "EXPORTS",
-           "DFLASH_DRAFT_MODEL", "DFLASH_DRAFT_SCRIPT", "DFLASH_FP32", "DFLASH_BF16"]
+           "DFLASH_DRAFT_MODEL", "DFLASH_DRAFT_SCRIPT", "DFLASH_FP32", "DFLASH_BF16", "DFLASH_BF16_FAST"]

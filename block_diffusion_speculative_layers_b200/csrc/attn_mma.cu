@@ -59,6 +59,21 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// (a, b) as a bf16 pair of high parts and a bf16 pair of the rounding remainders
+__device__ __forceinline__ void split_pack(float a, float b, uint32_t &hi, uint32_t &rem) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    const __nv_bfloat162 r = __floats2bfloat162_rn(a - __low2float(h), b - __high2float(h));
+    rem = *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// two consecutive outputs, with their low plane `lo` elements further on when lo != 0
+__device__ __forceinline__ void store_pair(bf16 *dst, size_t lo, float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    *reinterpret_cast<__nv_bfloat162 *>(dst) = h;
+    if (lo) *reinterpret_cast<__nv_bfloat162 *>(dst + lo) = __floats2bfloat162_rn(a - __low2float(h), b - __high2float(h));
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -80,16 +95,24 @@ __device__ __forceinline__ const float *peer_ptr(const float *p, uint32_t rank) 
 // tile's key count), keeps an unnormalised partial (o, running max, running
 // sum) in shared memory, and after a cluster barrier combines a slice of the
 // (head, row) pairs over all CTAs of the cluster in rank order.
-template <int HD>
+//
+// SPLIT: q, K, V (and the output) are two-plane activations (hi at p, lo at
+// p + lo).  Each product then takes three bf16 MMAs, hi*hi + lo*hi + hi*lo
+// (the lo*lo term is below the fp32 accumulator's resolution), and the
+// probabilities P are split the same way in registers before P V.
+template <int HD, bool SPLIT>
 __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ q, int ldq, const bf16 *__restrict__ kc,
                                                        const bf16 *__restrict__ vc, const RowMeta *__restrict__ meta,
                                                        int R, int rows_per_tile, int nq, int nkv, int max_len,
-                                                       int n_splits, float scale_log2, bf16 *__restrict__ out, int ldo) {
+                                                       int n_splits, float scale_log2, bf16 *__restrict__ out, int ldo,
+                                                       size_t lo) {
     constexpr int LDS = HD + 8;  // padded smem row (bf16 elements)
     constexpr int OLD = HD + 4;  // partial-output row stride (floats)
     extern __shared__ __align__(16) uint8_t smem_raw[];
     bf16 *Ks = reinterpret_cast<bf16 *>(smem_raw);  // [2][KB][LDS]
     bf16 *Vs = Ks + 2 * KB * LDS;                    // [2][KB][LDS]
+    bf16 *Kl = Vs + 2 * KB * LDS;                    // SPLIT: lo planes [2][KB][LDS] each
+    bf16 *Vl = Kl + 2 * KB * LDS;
     float *Op = reinterpret_cast<float *>(smem_raw); // [grp][16][OLD], reuses K/V tiles after the loop
     __shared__ float MLs[8 * 16 * 2];                // [grp][16][(max, sum)]
 
@@ -119,8 +142,8 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
     const bf16 *Kg = kc + head_off;
     const bf16 *Vg = vc + head_off;
 
-    // Q fragments (A operand, 16 rows x HD)
-    uint32_t qa[HD / 16][4];
+    // Q fragments (A operand, 16 rows x HD); ql: lo plane
+    uint32_t qa[HD / 16][4], ql[SPLIT ? HD / 16 : 1][4];
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
         const int c0 = kk * 16 + (lane & 3) * 2;
@@ -130,6 +153,12 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
         qa[kk][1] = rb < nrows ? *reinterpret_cast<const uint32_t *>(qb_row + c0) : 0u;
         qa[kk][2] = ra < nrows ? *reinterpret_cast<const uint32_t *>(qa_row + c0 + 8) : 0u;
         qa[kk][3] = rb < nrows ? *reinterpret_cast<const uint32_t *>(qb_row + c0 + 8) : 0u;
+        if constexpr (SPLIT) {
+            ql[kk][0] = ra < nrows ? *reinterpret_cast<const uint32_t *>(qa_row + lo + c0) : 0u;
+            ql[kk][1] = rb < nrows ? *reinterpret_cast<const uint32_t *>(qb_row + lo + c0) : 0u;
+            ql[kk][2] = ra < nrows ? *reinterpret_cast<const uint32_t *>(qa_row + lo + c0 + 8) : 0u;
+            ql[kk][3] = rb < nrows ? *reinterpret_cast<const uint32_t *>(qb_row + lo + c0 + 8) : 0u;
+        }
     }
 
     float o[HD / 8][4];
@@ -146,6 +175,10 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
             const size_t off = (size_t)(valid ? key : 0) * HD + c;
             cp_async16(Ks + ((size_t)buf * KB + r) * LDS + c, Kg + off, valid);
             cp_async16(Vs + ((size_t)buf * KB + r) * LDS + c, Vg + off, valid);
+            if constexpr (SPLIT) {
+                cp_async16(Kl + ((size_t)buf * KB + r) * LDS + c, Kg + lo + off, valid);
+                cp_async16(Vl + ((size_t)buf * KB + r) * LDS + c, Vg + lo + off, valid);
+            }
         }
         cp_commit();
     };
@@ -164,6 +197,8 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
         __syncthreads();
         const bf16 *Kt = Ks + (size_t)buf * KB * LDS;
         const bf16 *Vt = Vs + (size_t)buf * KB * LDS;
+        const bf16 *Klt = Kl + (size_t)buf * KB * LDS;
+        const bf16 *Vlt = Vl + (size_t)buf * KB * LDS;
         // S = Q K^T over 64 keys: 8 n-tiles of 8 keys
         float sc[KB / 8][4];
 #pragma unroll
@@ -180,6 +215,13 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
                 ldm_x4(b0, b1, b2, b3, Kt + (size_t)key * LDS + dim);
                 mma16816(sc[2 * np], qa[kk], b0, b1);
                 mma16816(sc[2 * np + 1], qa[kk], b2, b3);
+                if constexpr (SPLIT) {
+                    mma16816(sc[2 * np], ql[kk], b0, b1);
+                    mma16816(sc[2 * np + 1], ql[kk], b2, b3);
+                    ldm_x4(b0, b1, b2, b3, Klt + (size_t)key * LDS + dim);
+                    mma16816(sc[2 * np], qa[kk], b0, b1);
+                    mma16816(sc[2 * np + 1], qa[kk], b2, b3);
+                }
             }
         }
         // mask + online softmax (log2 domain)
@@ -225,11 +267,18 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
         // O += P V : P as A operand (4 k-steps of 16 keys), V via transposed ldmatrix
 #pragma unroll
         for (int kk = 0; kk < KB / 16; ++kk) {
-            uint32_t pa[4];
-            pa[0] = pack_bf16(sc[2 * kk][0], sc[2 * kk][1]);
-            pa[1] = pack_bf16(sc[2 * kk][2], sc[2 * kk][3]);
-            pa[2] = pack_bf16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-            pa[3] = pack_bf16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+            uint32_t pa[4], pl[4];
+            if constexpr (SPLIT) {
+                split_pack(sc[2 * kk][0], sc[2 * kk][1], pa[0], pl[0]);
+                split_pack(sc[2 * kk][2], sc[2 * kk][3], pa[1], pl[1]);
+                split_pack(sc[2 * kk + 1][0], sc[2 * kk + 1][1], pa[2], pl[2]);
+                split_pack(sc[2 * kk + 1][2], sc[2 * kk + 1][3], pa[3], pl[3]);
+            } else {
+                pa[0] = pack_bf16(sc[2 * kk][0], sc[2 * kk][1]);
+                pa[1] = pack_bf16(sc[2 * kk][2], sc[2 * kk][3]);
+                pa[2] = pack_bf16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+                pa[3] = pack_bf16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+            }
 #pragma unroll
             for (int dp = 0; dp < HD / 16; ++dp) {
                 // matrices (keys 0-7, d 0-7), (keys 8-15, d 0-7), (keys 0-7, d 8-15), (keys 8-15, d 8-15)
@@ -239,6 +288,13 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
                 ldm_x4_t(b0, b1, b2, b3, Vt + (size_t)key * LDS + dim);
                 mma16816(o[2 * dp], pa, b0, b1);
                 mma16816(o[2 * dp + 1], pa, b2, b3);
+                if constexpr (SPLIT) {
+                    mma16816(o[2 * dp], pl, b0, b1);
+                    mma16816(o[2 * dp + 1], pl, b2, b3);
+                    ldm_x4_t(b0, b1, b2, b3, Vlt + (size_t)key * LDS + dim);
+                    mma16816(o[2 * dp], pa, b0, b1);
+                    mma16816(o[2 * dp + 1], pa, b2, b3);
+                }
             }
         }
         __syncthreads();
@@ -254,12 +310,8 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
 #pragma unroll
         for (int j = 0; j < HD / 8; ++j) {
             const int d = j * 8 + (lane & 3) * 2;
-            if (ra < nrows)
-                *reinterpret_cast<__nv_bfloat162 *>(out + (size_t)(r0 + ra) * ldo + h * HD + d) =
-                    __floats2bfloat162_rn(o[j][0] * ia, o[j][1] * ia);
-            if (rb < nrows)
-                *reinterpret_cast<__nv_bfloat162 *>(out + (size_t)(r0 + rb) * ldo + h * HD + d) =
-                    __floats2bfloat162_rn(o[j][2] * ib, o[j][3] * ib);
+            if (ra < nrows) store_pair(out + (size_t)(r0 + ra) * ldo + h * HD + d, lo, o[j][0] * ia, o[j][1] * ia);
+            if (rb < nrows) store_pair(out + (size_t)(r0 + rb) * ldo + h * HD + d, lo, o[j][2] * ib, o[j][3] * ib);
         }
         return;
     }
@@ -329,8 +381,7 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
             const int hq = kvh * grp + hh;
             bf16 *dst = out + (size_t)(r0 + row) * ldo + hq * HD + d0;
 #pragma unroll
-            for (int t = 0; t < DPT; t += 2)
-                *reinterpret_cast<__nv_bfloat162 *>(dst + t) = __floats2bfloat162_rn(acc[t] * inv, acc[t + 1] * inv);
+            for (int t = 0; t < DPT; t += 2) store_pair(dst + t, lo, acc[t] * inv, acc[t + 1] * inv);
         }
     }
     cluster_sync_all();
@@ -359,26 +410,26 @@ bool attn_mma_supported<float>(int) {
 
 static int g_num_sms = 0;
 
-template <int HD>
+template <int HD, bool SPLIT>
 static void launch_hd(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
-                      int rows_per_tile, int nq, int nkv, int max_len, bf16 *out, int ldo, int n_tiles, int n_splits,
-                      cudaStream_t s) {
+                      int rows_per_tile, int nq, int nkv, int max_len, bf16 *out, int ldo, size_t lo, int n_tiles,
+                      int n_splits, cudaStream_t s) {
     const int grp = nq / nkv;
-    size_t smem = 2 * 2 * at::KB * (HD + 8) * sizeof(bf16);
+    size_t smem = (SPLIT ? 4 : 2) * 2 * at::KB * (HD + 8) * sizeof(bf16);
     smem = std::max(smem, (size_t)grp * 16 * (HD + 4) * sizeof(float));
     static bool set = false;
     if (!set) {
-        cudaFuncSetAttribute(at::attn_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+        cudaFuncSetAttribute(at::attn_mma_kernel<HD, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         set = true;
     }
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-    launch_k(at::attn_mma_kernel<HD>, dim3(n_tiles, nkv, n_splits), dim3(32 * grp), smem, s, n_splits, q, ldq, kc, vc,
-             meta, R, rows_per_tile, nq, nkv, max_len, n_splits, scale_log2, out, ldo);
+    launch_k(at::attn_mma_kernel<HD, SPLIT>, dim3(n_tiles, nkv, n_splits), dim3(32 * grp), smem, s, n_splits, q, ldq, kc,
+             vc, meta, R, rows_per_tile, nq, nkv, max_len, n_splits, scale_log2, out, ldo, lo);
 }
 
 template <>
 void launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
-                                int rows_per_tile, int nq, int nkv, int hd, int max_len, bf16 *out, int ldo,
+                                int rows_per_tile, int nq, int nkv, int hd, int max_len, bf16 *out, int ldo, size_t lo,
                                 const AttnScratch &ws, cudaStream_t s) {
     (void)ws;
     if (R <= 0) return;
@@ -392,14 +443,17 @@ void launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf
     // splits of one (tile, kv head) form a cluster of at most 8 CTAs; no more
     // splits than 64-key tiles the longest possible context has
     const int n_splits = std::max(1, std::min({8, (2 * g_num_sms + ctas - 1) / ctas, (max_len + 63) / 64}));
-    if (hd == 128)
-        launch_hd<128>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, n_tiles, n_splits, s);
-    else
-        launch_hd<64>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, n_tiles, n_splits, s);
+    if (hd == 128) {
+        if (lo) launch_hd<128, true>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, lo, n_tiles, n_splits, s);
+        else launch_hd<128, false>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, 0, n_tiles, n_splits, s);
+    } else {
+        if (lo) launch_hd<64, true>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, lo, n_tiles, n_splits, s);
+        else launch_hd<64, false>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, 0, n_tiles, n_splits, s);
+    }
 }
 
 template <>
 void launch_attention_mma<float>(const float *, int, const float *, const float *, const RowMeta *, int, int, int, int,
-                                 int, int, float *, int, const AttnScratch &, cudaStream_t) {}
+                                 int, int, float *, int, size_t, const AttnScratch &, cudaStream_t) {}
 
 }  // namespace dfl

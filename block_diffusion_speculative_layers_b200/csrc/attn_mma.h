@@ -28,8 +28,10 @@ bool attn_mma_supported(int hd);
 
 // rows_per_tile: rows of one sequence that share a query tile (block size for
 // draft/verify, 16 for prompt rows, 1 for single-row target steps).
+// lo != 0: q, K/V and out are two-plane activations (low plane lo elements on).
 template <typename T>
 void launch_attention_mma(const T *q, int ldq, const T *kc, const T *vc, const RowMeta *meta, int R, int rows_per_tile,
-                          int nq, int nkv, int hd, int max_len, T *out, int ldo, const AttnScratch &ws, cudaStream_t s);
+                          int nq, int nkv, int hd, int max_len, T *out, int ldo, size_t lo, const AttnScratch &ws,
+                          cudaStream_t s);
 
 }  // namespace dfl

@@ -74,8 +74,10 @@ template <int TM>
 __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    constexpr int B_BYTES = TM * 128;
-    constexpr int NC1 = TM < 32 ? 32 : TM;
+    const int B_BYTES = TM * 128 * L.planes;
+    const bool wide = L.planes == 2 && TM <= 128;  // one N = 2*TM MMA over both planes
+    const int lo_col = wide ? TM : 0;
+    const int NC1 = max(32, wide ? 2 * TM : TM);
     const int stages = L.stages;
     uint8_t *sA = smem;
     uint8_t *sB = smem + (size_t)stages * A_BYTES;
@@ -146,7 +148,8 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                 return true;
             };
             auto issue_x = [&](const PendingX &px) {
-                tma_load_2d(sB + (size_t)px.s * B_BYTES, L.ops[px.j].xmap, px.k, 0, &full[px.s]);
+                if (L.planes == 2) tma_load_3d(sB + (size_t)px.s * B_BYTES, L.ops[px.j].xmap, px.k, 0, 0, &full[px.s]);
+                else tma_load_2d(sB + (size_t)px.s * B_BYTES, L.ops[px.j].xmap, px.k, 0, &full[px.s]);
             };
             auto flush = [&](bool block) -> bool {
                 int i = 0;
@@ -206,7 +209,7 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            const uint32_t idesc = idesc_bf16(TM);
+            const uint32_t idesc = idesc_bf16(wide ? 2 * TM : TM);
             int it = 0, lt = 0;
             bool ok = true;
             for (int j = L.op_begin; j < L.op_end && ok; ++j) {
@@ -236,9 +239,13 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                         const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_BYTES));
                         const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_BYTES));
 #pragma unroll
-                        for (int k4 = 0; k4 < BK / 16; ++k4)
+                        for (int k4 = 0; k4 < BK / 16; ++k4) {
                             mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)(k4 * 2), idesc,
                                      (kk > kb || k4 > 0) ? 1u : 0u);
+                            if (L.planes == 2 && !wide)  // lo plane, TM rows further on
+                                mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)((TM * 128) >> 4) + (uint64_t)(k4 * 2),
+                                         idesc, 1u);
+                        }
                         mma_commit(&empty[s]);
                     }
                     mma_commit(&acc_full[b]);
@@ -275,7 +282,7 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                 float v[CH];
                 if (S == 1) {
                     for (int c = 0; c < TM; c += CH) {
-                        if (ok) tmem_ld16(trow + c, v);
+                        if (ok) acc_ld16(trow, c, lo_col, v);
                         else
 #pragma unroll
                             for (int jj = 0; jj < CH; ++jj) v[jj] = 0.f;
@@ -296,7 +303,7 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                 } else {
                     float *mine = op.ws + ((size_t)ti.z + sp) * (size_t)TM * 128;
                     for (int c = 0; c < TM; c += CH) {
-                        if (ok) tmem_ld16(trow + c, v);
+                        if (ok) acc_ld16(trow, c, lo_col, v);
                         else
 #pragma unroll
                             for (int jj = 0; jj < CH; ++jj) v[jj] = 0.f;
@@ -367,15 +374,15 @@ static size_t chain_fixed_bytes() {
     return 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::CH * 4 + 64 * 8 + 64;
 }
 
-int chain_stages(int tm) {
+int chain_stages(int tm, int planes) {
     // ~150 KB keeps room on each SM for an attention CTA (~70 KB) of the next kernel
     const size_t budget = tm <= 32 ? 150 * 1024 : 200 * 1024;
-    const size_t stage = tc::A_BYTES + (size_t)tm * 128;
+    const size_t stage = tc::A_BYTES + (size_t)tm * 128 * planes;
     return (int)std::max<size_t>(2, std::min<size_t>(16, (budget - chain_fixed_bytes()) / stage));
 }
 
-size_t chain_smem_bytes(int tm, int stages) {
-    return chain_fixed_bytes() + (size_t)stages * (tc::A_BYTES + (size_t)tm * 128);
+size_t chain_smem_bytes(int tm, int planes, int stages) {
+    return chain_fixed_bytes() + (size_t)stages * (tc::A_BYTES + (size_t)tm * 128 * planes);
 }
 
 template <int TM>
@@ -396,8 +403,9 @@ void launch_chain(const ChainProgram &prog, int b, int e, int num_sms, int *err,
     L.epoch = prog.epoch;
     L.op_done = prog.d_op_done;
     L.err = err;
-    L.stages = chain_stages(prog.tm);
-    const size_t smem = chain_smem_bytes(prog.tm, L.stages);
+    L.planes = prog.planes;
+    L.stages = chain_stages(prog.tm, prog.planes);
+    const size_t smem = chain_smem_bytes(prog.tm, prog.planes, L.stages);
     switch (prog.tm) {
         case 16: launch_tm<16>(L, num_sms, smem, s); break;
         case 32: launch_tm<32>(L, num_sms, smem, s); break;

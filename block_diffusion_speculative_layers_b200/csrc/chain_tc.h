@@ -34,6 +34,7 @@ struct ChainLaunch {
     int *op_done;              // [n_ops] completion counters (monotonic)
     int *err;
     int stages;
+    int planes;                // activation planes of every op (2: hi + lo)
 };
 
 // Host-side program: a list of projections uploaded once, launched in runs.
@@ -49,6 +50,7 @@ struct ChainProgram {
     float *d_ws = nullptr;           // two split-K partial buffers (op parity)
     size_t ws_floats = 0;            // floats per buffer
     int tm = 16;
+    int planes = 1;
     unsigned epoch = 0;
     int key = -1;                    // program identity (pass, batch) it was built for
     bool valid = true;               // false: the shapes do not fit the reserved workspace
@@ -56,7 +58,7 @@ struct ChainProgram {
 
 // Launch ops [b, e) of a program (epoch must already be advanced for this run).
 void launch_chain(const ChainProgram &prog, int b, int e, int num_sms, int *err, cudaStream_t s);
-int chain_stages(int tm);
-size_t chain_smem_bytes(int tm, int stages);
+int chain_stages(int tm, int planes);
+size_t chain_smem_bytes(int tm, int planes, int stages);
 
 }  // namespace dfl

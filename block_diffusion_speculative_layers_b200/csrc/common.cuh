@@ -47,6 +47,23 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
 
+// Two-plane activations (bf16 models).  A value v of a GEMM input, q or the
+// K/V cache is kept as hi = bf16(v) at p[i] and lo = bf16(v - hi) at p[i + lo],
+// so hi + lo carries ~16 significant bits while each plane stays a bf16
+// tensor-core operand; lo == 0 means a single plane.
+template <typename T>
+__device__ __forceinline__ void st_act(T *p, size_t i, size_t lo, float v) {
+    const T h = from_f<T>(v);
+    p[i] = h;
+    if (lo) p[i + lo] = from_f<T>(v - to_f(h));
+}
+template <typename T>
+__device__ __forceinline__ float ld_act(const T *p, size_t i, size_t lo) {
+    float v = to_f(p[i]);
+    if (lo) v += to_f(p[i + lo]);
+    return v;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -60,7 +60,7 @@ static void *noalloc_scratch_ptr(std::string &err) {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-static int elem_size(int dtype) { return dtype == DFLASH_BF16 ? 2 : 4; }
+static int elem_size(int dtype) { return dtype == DFLASH_FP32 ? 4 : 2; }
 
 static bool check_model(const dflash_model_cfg &m, std::string &why) {
     if (m.n_layers < 1 || m.hidden < 32 || m.n_q_heads < 1 || m.n_kv_heads < 1 || m.vocab < 2) {
@@ -100,7 +100,10 @@ static bool check_config(const dflash_config &c, std::string &why) {
     if (c.max_batch < 1 || c.max_batch > 64) { why = "max_batch must be in [1, 64]"; return false; }
     if (c.max_len < c.block_size + 1 || c.max_len > (1 << 20)) { why = "max_len out of range"; return false; }
     if (c.prefill_chunk < 0 || c.prefill_chunk > 8192) { why = "prefill_chunk must be in [0, 8192]"; return false; }
-    if (c.dtype != DFLASH_FP32 && c.dtype != DFLASH_BF16) { why = "dtype must be DFLASH_FP32 or DFLASH_BF16"; return false; }
+    if (c.dtype != DFLASH_FP32 && c.dtype != DFLASH_BF16 && c.dtype != DFLASH_BF16_FAST) {
+        why = "dtype must be DFLASH_FP32, DFLASH_BF16 or DFLASH_BF16_FAST";
+        return false;
+    }
     return true;
 }
 
@@ -141,7 +144,8 @@ static void add_model_slots(Layout &L, const char *prefix, const dflash_model_cf
 
 static Layout make_layout(const dflash_config &c) {
     Layout L;
-    const int dt = c.dtype, es = elem_size(dt);
+    // weight storage: fp32 or bf16 (both bf16 activation modes store bf16 weights)
+    const int dt = c.dtype == DFLASH_FP32 ? DFLASH_FP32 : DFLASH_BF16, es = elem_size(dt);
     const dflash_model_cfg &t = c.target, &d = c.drafter;
     add_slot(L, "embed", 2, t.vocab, t.hidden, 0, dt);
     add_slot(L, "lm_head", 2, t.vocab, t.hidden, 0, dt);
@@ -168,10 +172,13 @@ static Layout make_layout(const dflash_config &c) {
     const size_t R = L.R_max;
     size_t o = 0;
     auto take = [&](size_t bytes) { o = align_up(o, 256); size_t r = o; o += std::max<size_t>(bytes, 16); return r; };
-    L.x = take(R * H * 4);
+    // Activations in the model dtype (GEMM inputs, q, the K/V caches) form one
+    // contiguous span; with two-plane bf16 activations (DFLASH_BF16) the span is
+    // repeated right after itself for the low planes, so every such buffer p has
+    // its low plane at p + act_lo elements.
+    const size_t act0 = o;
     L.xn = take(R * H * es);
     L.dq_in = take((size_t)2 * L.R_dec * H * es);
-    L.Y = take(R * (size_t)ycols * 4);
     L.q = take(R * qmax * es);
     L.ao = take(R * qmax * es);
     const size_t hrows = t.n_experts > 0 ? R * (size_t)t.top_k : R;
@@ -180,6 +187,21 @@ static Layout make_layout(const dflash_config &c) {
     L.taps_gather = take((size_t)L.R_dec * TK * es);
     L.taps_pre = take((size_t)L.C * TK * es);
     L.cbuf = take((size_t)L.C * H * es);
+    const size_t kv_t = (size_t)t.n_layers * nb * t.n_kv_heads * c.max_len * t.head_dim * es;
+    const size_t kv_d = (size_t)d.n_layers * nb * d.n_kv_heads * c.max_len * d.head_dim * es;
+    L.tk = take(kv_t);
+    L.tv = take(kv_t);
+    L.dk = take(kv_d);
+    L.dv = take(kv_d);
+    L.xg_t = take((size_t)L.R_dec * H * es);
+    L.xg2 = take((size_t)L.R_dec * H * es);
+    const size_t act_bytes = align_up(o, 256) - act0;
+    if (c.dtype == DFLASH_BF16) {
+        take(act_bytes);
+        L.act_lo = act_bytes / es;
+    }
+    L.x = take(R * H * 4);
+    L.Y = take(R * (size_t)ycols * 4);
     L.logits = take((size_t)L.R_dec * t.vocab * 4);
     L.plogits = take((size_t)t.vocab * 4);
     L.g = take((size_t)L.R_dec * 4);
@@ -194,12 +216,6 @@ static Layout make_layout(const dflash_config &c) {
     L.ctx_meta_pre = take((size_t)L.C * sizeof(RowMeta));
     L.rope_t = take((size_t)c.max_len * (t.head_dim / 2) * sizeof(float2));
     L.rope_d = take((size_t)c.max_len * (d.head_dim / 2) * sizeof(float2));
-    const size_t kv_t = (size_t)t.n_layers * nb * t.n_kv_heads * c.max_len * t.head_dim * es;
-    const size_t kv_d = (size_t)d.n_layers * nb * d.n_kv_heads * c.max_len * d.head_dim * es;
-    L.tk = take(kv_t);
-    L.tv = take(kv_t);
-    L.dk = take(kv_d);
-    L.dv = take(kv_d);
     L.script = take((size_t)nb * c.max_len * 4);
     L.out_tok = take((size_t)nb * c.max_len * 4);
     L.tokens = take((size_t)c.max_len * 4);
@@ -225,8 +241,6 @@ static Layout make_layout(const dflash_config &c) {
     // persistent projection chains (bf16 decode): folded-norm activations,
     // per-tile sums of squares, two programs (verify, draft) and split-K partials
     {
-        L.xg_t = take((size_t)L.R_dec * H * es);
-        L.xg2 = take((size_t)L.R_dec * H * es);
         L.ssq_ld = 2 * L.R_dec;
         L.ssq = take((size_t)(H / 128 + 1) * L.ssq_ld * 4);
         const int F_d = d.ffn;
@@ -289,6 +303,7 @@ class Engine : public EngineBase {
     AttnScratch att;
     // persistent projection chains (bf16 decode)
     T *xg_t = nullptr, *xg2 = nullptr;
+    size_t lo_ = 0;  // low plane offset of two-plane activations (elements), 0: one plane
     float *ssq = nullptr;
     ChainProgram pv, pd;
     bool chain_verify_ok = false, chain_draft_ok = false;
@@ -388,6 +403,7 @@ class Engine : public EngineBase {
         gemm_sem = sp<int>(L.gemm_sem);
         lm_part = sp<float2>(L.lm_part);
         xg_t = sp<T>(L.xg_t);
+        lo_ = L.act_lo;
         xg2 = sp<T>(L.xg2);
         ssq = sp<float>(L.ssq);
         {
@@ -532,7 +548,9 @@ class Engine : public EngineBase {
         timed(0, gemm_bytes(M, N, K, e), [&] { gemm_launch(X, ldx, M, Wt, N, K, e); });
     }
 
-    void gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e) {
+    void gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e_in) {
+        Epi<T> e = e_in;
+        e.lo = lo_;  // every input and output of the engine's projections lives in the activation span
         if (tc.supports(M, N, K)) {
             tc.run(X, ldx, M, (const T *)Wt, N, K, e, s);
             return;
@@ -540,17 +558,17 @@ class Engine : public EngineBase {
         // CUDA-core path (fp32 models): GEMM into fp32 Y, then the epilogue.
         float *Yo = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.Y : Y;
         const int ldy = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.ldy : N;
-        launch_gemm_simt<T>(X, ldx, M, (const T *)Wt, K, N, K, Yo, ldy, s);
+        launch_gemm_simt<T>(X, ldx, M, (const T *)Wt, K, N, K, Yo, ldy, lo_, s);
         switch (e.kind) {
             case EPI_QKV:
                 launch_qkv_epilogue<T>(Y, N, e.col0, e.R_blk, M, e.meta, e.ctx_meta, e.nq, e.nkv, e.hd, e.rope,
-                                       e.q_out, e.kc, e.vc, e.max_len, s);
+                                       e.q_out, e.kc, e.vc, e.max_len, lo_, s);
                 break;
             case EPI_RESID:
-                launch_residual<T>(e.x, Y, N, N, M, e.taps, e.meta, s);
+                launch_residual<T>(e.x, Y, N, N, M, e.taps, lo_, e.meta, s);
                 break;
             case EPI_SWIGLU:
-                launch_swiglu<T>(Y, N, e.F, M, e.h, e.F, s);
+                launch_swiglu<T>(Y, N, e.F, M, e.h, e.F, lo_, s);
                 break;
             default:
                 break;
@@ -563,7 +581,7 @@ class Engine : public EngineBase {
         timed(1, 0.0, [&] {
             if (attn_mma_supported<T>(m.head_dim))
                 launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads, m.head_dim,
-                                        c.max_len, out, qd, att, s);
+                                        c.max_len, out, qd, lo_, att, s);
             else
                 launch_attention_simt<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out,
                                          qd, s);
@@ -575,7 +593,7 @@ class Engine : public EngineBase {
         const dflash_model_cfg &m = c.target;
         const LayerW &w = tl[l];
         const int H = m.hidden, hd = m.head_dim, qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd;
-        launch_rmsnorm<T>(x, H, w.attn_norm, H, (float)m.rms_eps, xn, H, R, s);
+        launch_rmsnorm<T>(x, H, w.attn_norm, H, (float)m.rms_eps, xn, H, lo_, R, s);
         Epi<T> e;
         e.kind = EPI_QKV;
         e.R_blk = R;
@@ -595,7 +613,7 @@ class Engine : public EngineBase {
         r.x = x;
         r.meta = mt;
         gemm(ao, qd, R, w.wo, H, qd, r);
-        launch_rmsnorm<T>(x, H, w.ffn_norm, H, (float)m.rms_eps, xn, H, R, s);
+        launch_rmsnorm<T>(x, H, w.ffn_norm, H, (float)m.rms_eps, xn, H, lo_, R, s);
         TapDst<T> taps{};
         taps.base = tap_base;
         taps.ld = tap_ld;
@@ -634,17 +652,17 @@ class Engine : public EngineBase {
             run_moe_tc<T>(xn, H, R, k, moe_sel, (const T *)w.we_gate_up, (const T *)w.we_down, H, Fe, E, h, moe_part,
                           tc, s);
         } else {
-            launch_moe_experts_simt<T>(xn, H, R, k, moe_sel, (const T *)w.we_gate_up, (const T *)w.we_down, H, Fe,
+            launch_moe_experts_simt<T>(xn, H, lo_, R, k, moe_sel, (const T *)w.we_gate_up, (const T *)w.we_down, H, Fe,
                                        moe_part, s);
         }
-        launch_moe_combine<T>(x, moe_part, moe_wt, H, R, k, taps, mt, s);
+        launch_moe_combine<T>(x, moe_part, moe_wt, H, R, k, taps, lo_, mt, s);
     }
 
     void drafter_layer(int j, int R, bool with_ctx) {
         const dflash_model_cfg &m = c.drafter;
         const LayerW &w = dl[j];
         const int H = m.hidden, hd = m.head_dim, qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd;
-        launch_rmsnorm<T>(x, H, w.attn_norm, H, (float)m.rms_eps, dq_in, H, R, s);
+        launch_rmsnorm<T>(x, H, w.attn_norm, H, (float)m.rms_eps, dq_in, H, lo_, R, s);
         Epi<T> e;
         e.kind = EPI_QKV;
         e.R_blk = R;
@@ -666,7 +684,7 @@ class Engine : public EngineBase {
         r.x = x;
         r.meta = meta;
         gemm(ao, qd, R, w.wo, H, qd, r);
-        launch_rmsnorm<T>(x, H, w.ffn_norm, H, (float)m.rms_eps, xn, H, R, s);
+        launch_rmsnorm<T>(x, H, w.ffn_norm, H, (float)m.rms_eps, xn, H, lo_, R, s);
         Epi<T> sw;
         sw.kind = EPI_SWIGLU;
         sw.h = h;
@@ -694,7 +712,7 @@ class Engine : public EngineBase {
 
     void lm_head_rows(const float *final_norm, float eps, int R, float *lg, int mode, int B, int *idx) {
         const int H = c.target.hidden;
-        launch_rmsnorm<T>(x, H, final_norm, H, eps, xn, H, R, s);
+        launch_rmsnorm<T>(x, H, final_norm, H, eps, xn, H, lo_, R, s);
         head_argmax(xn, R, lg, mode, B, idx);
     }
 
@@ -748,12 +766,13 @@ class Engine : public EngineBase {
             if ((size_t)slots * pg.tm * 128 > pg.ws_floats) pg.valid = false;  // use the per-kernel path
             const int idx = (int)pg.ops.size();
             CUtensorMap mw = *tc.tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
-            CUtensorMap mx = *tc.tensor_map(X, M, K, ldx, pg.tm);
+            CUtensorMap mx = *tc.tensor_map(X, M, K, ldx, pg.tm, lo_);
             pg.maps.push_back(mw);
             pg.maps.push_back(mx);
             op.wmap = pg.d_maps + 2 * idx;
             op.xmap = pg.d_maps + 2 * idx + 1;
             op.e = e;
+            op.e.lo = lo_;
             op.ws = pg.d_ws + (size_t)(idx & 1) * pg.ws_floats;
             op.tile_cnt = pg.d_tile_cnt + tile_off;
             op.tinfo = pg.d_tinfo + tile_off;
@@ -801,6 +820,7 @@ class Engine : public EngineBase {
         pg.tinfo.clear();
         pg.valid = true;
         pg.tm = pow2_at_least(R, 16);
+        pg.planes = lo_ ? 2 : 1;
         pg.key = nseq;
         int toff = 0;
         auto qkv = [&](int l) {
@@ -866,6 +886,7 @@ class Engine : public EngineBase {
         pg.tinfo.clear();
         pg.valid = true;
         pg.tm = pow2_at_least(2 * R, 16);
+        pg.planes = lo_ ? 2 : 1;
         pg.key = nseq;
         int toff = 0;
         Epi<T> f;
@@ -924,7 +945,7 @@ class Engine : public EngineBase {
         if (pv.key != nseq) build_verify_program(nseq);
         pv.epoch++;
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, tl[0].attn_norm,
-                             xg_t, H, ssq, L.ssq_ld, s);
+                             xg_t, H, lo_, ssq, L.ssq_ld, s);
         launch_chain(pv, 0, 1, num_sms, &stats->status, s);
         for (int l = 0; l < t.n_layers; ++l) {
             attention(q, tk + (size_t)l * kv_layer_elems(t), tv + (size_t)l * kv_layer_elems(t), meta, R, B, t, ao);
@@ -941,7 +962,7 @@ class Engine : public EngineBase {
         if (pd.key != nseq) build_draft_program(nseq);
         pd.epoch++;
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, dl[0].attn_norm,
-                             dq_in, H, ssq, L.ssq_ld, s);
+                             dq_in, H, lo_, ssq, L.ssq_ld, s);
         launch_chain(pd, 0, 2, num_sms, &stats->status, s);
         for (int j = 0; j < d.n_layers; ++j) {
             attention(q, dk + (size_t)j * kv_layer_elems(d), dv + (size_t)j * kv_layer_elems(d), meta, R, B, d, ao);
@@ -964,7 +985,7 @@ class Engine : public EngineBase {
             for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, 16, meta, taps_pre, TK);
             if (c0 + R == n) {
                 // greedy first token from the last prompt row
-                launch_rmsnorm<T>(x + (size_t)(R - 1) * H, H, t_final, H, (float)t.rms_eps, xn, H, 1, s);
+                launch_rmsnorm<T>(x + (size_t)(R - 1) * H, H, t_final, H, (float)t.rms_eps, xn, H, lo_, 1, s);
                 head_argmax(xn, 1, plogits, 0, 1, first_tok);
             }
             // context vectors of the prompt rows -> drafter context K/V
@@ -973,7 +994,7 @@ class Engine : public EngineBase {
             f.Y = Y;
             f.ldy = H;
             gemm(taps_pre, TK, R, w_fc, H, TK, f);
-            launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, cbuf, H, R, s);
+            launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, cbuf, H, lo_, R, s);
             launch_ctx_meta_prefill(ctx_meta_pre, R, seq, c0, s);
             for (int j = 0; j < d.n_layers; ++j) {
                 Epi<T> e;
@@ -1011,6 +1032,7 @@ class Engine : public EngineBase {
         const T *tin = taps_dec;
         if (!contiguous) {
             launch_gather_rows(taps_dec, taps_gather, (size_t)TK * sizeof(T), active, nseq, B, s);
+            if (lo_) launch_gather_rows(taps_dec + lo_, taps_gather + lo_, (size_t)TK * sizeof(T), active, nseq, B, s);
             tin = taps_gather;
         }
         Epi<T> f;
@@ -1018,7 +1040,7 @@ class Engine : public EngineBase {
         f.Y = Y;
         f.ldy = H;
         gemm(tin, TK, R, w_fc, H, TK, f);
-        launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, dq_in + (size_t)R * H, H, R, s);
+        launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, dq_in + (size_t)R * H, H, lo_, R, s);
         for (int j = 0; j < d.n_layers; ++j) drafter_layer(j, R, true);
         if (B > 1) lm_head_rows(d_final, (float)d.rms_eps, R, logits, 1, B, drafts);
         if (draft_mode == DFLASH_DRAFT_SCRIPT)
@@ -1333,7 +1355,7 @@ class Engine : public EngineBase {
         const T *kc = (which == 0 ? tk : dk) + (size_t)layer * kv_layer_elems(m);
         const T *vc = (which == 0 ? tv : dv) + (size_t)layer * kv_layer_elems(m);
         const int hd = m.head_dim, nkv = m.n_kv_heads;
-        std::vector<T> buf((size_t)n * hd);
+        std::vector<T> buf((size_t)n * hd), bl((size_t)n * hd);
         for (int pass = 0; pass < 2; ++pass) {
             const T *src = pass ? vc : kc;
             float *dst = pass ? vo : ko;
@@ -1341,8 +1363,13 @@ class Engine : public EngineBase {
                 const T *p = src + (((size_t)seq * nkv + hh) * c.max_len + p0) * hd;
                 if (cudaMemcpy(buf.data(), p, sizeof(T) * n * hd, cudaMemcpyDeviceToHost) != cudaSuccess)
                     return fail_cuda("kv copy");
+                if (lo_ && cudaMemcpy(bl.data(), p + lo_, sizeof(T) * n * hd, cudaMemcpyDeviceToHost) != cudaSuccess)
+                    return fail_cuda("kv copy");
                 for (int t = 0; t < n; ++t)
-                    for (int e = 0; e < hd; ++e) dst[(size_t)t * nkv * hd + hh * hd + e] = host_to_f(buf[(size_t)t * hd + e]);
+                    for (int e = 0; e < hd; ++e) {
+                        const size_t i = (size_t)t * hd + e;
+                        dst[(size_t)t * nkv * hd + hh * hd + e] = host_to_f(buf[i]) + (lo_ ? host_to_f(bl[i]) : 0.f);
+                    }
             }
         }
         return DFLASH_OK;
@@ -1517,12 +1544,12 @@ dflash_status dflash_create(const dflash_config *cfg, void *warena, size_t wbyte
     }
     for (size_t i = 0; i < ctx->lay.slots.size(); ++i) ctx->by_name[ctx->lay.slots[i].name] = (int)i;
     cudaStream_t s = (cudaStream_t)stream;
-    if (cfg->dtype == DFLASH_BF16)
+    if (cfg->dtype != DFLASH_FP32)
         ctx->eng.reset(new Engine<bf16>(*cfg, ctx->lay, (char *)warena, (char *)sarena, s));
     else
         ctx->eng.reset(new Engine<float>(*cfg, ctx->lay, (char *)warena, (char *)sarena, s));
     dflash_status r;
-    if (cfg->dtype == DFLASH_BF16) r = static_cast<Engine<bf16> *>(ctx->eng.get())->init(ctx->by_name);
+    if (cfg->dtype != DFLASH_FP32) r = static_cast<Engine<bf16> *>(ctx->eng.get())->init(ctx->by_name);
     else r = static_cast<Engine<float> *>(ctx->eng.get())->init(ctx->by_name);
     if (r != DFLASH_OK) {
         fprintf(stderr, "dflash_create: %s\n", ctx->eng->err.c_str());

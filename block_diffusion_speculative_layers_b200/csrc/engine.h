@@ -36,6 +36,7 @@ struct Layout {
     size_t moe_sel, moe_wt, moe_part, lm_part, att_o, att_ml, att_sem;
     size_t att_parts = 0;
     size_t xg_t, xg2, ssq, chain_v, chain_d, chain_ws;
+    size_t act_lo = 0;  // two-plane activations: low plane offset in elements (0: one plane)
     size_t chain_v_bytes = 0, chain_d_bytes = 0, chain_ws_floats = 0;
     int ssq_ld = 0, n_ops_v = 0, n_ops_d = 0, max_tiles = 0;
     size_t gemm_ws, gemm_sem;

@@ -47,8 +47,12 @@ __global__ void __launch_bounds__(NT, 1)
                    Epi<bf16> e, int stages) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    constexpr int B_BYTES = TM * 128;
-    constexpr int NC1 = TM < 32 ? 32 : TM;  // TMEM columns of one accumulator
+    const int B_BYTES = TM * 128 * p.planes;  // activation tile(s) of one stage
+    // two planes and TM <= 128: one MMA with N = 2*TM covers the hi and lo rows
+    // (they are contiguous in the stage), accumulating into 2*TM columns
+    const bool wide = p.planes == 2 && TM <= 128;
+    const int lo_col = wide ? TM : 0;
+    const int NC1 = max(32, wide ? 2 * TM : TM);  // TMEM columns of one accumulator
     constexpr int PLD = TM + 1;             // parked partial tile row stride (floats)
     uint8_t *sA = smem;
     uint8_t *sB = smem + (size_t)stages * A_BYTES;
@@ -122,8 +126,10 @@ __global__ void __launch_bounds__(NT, 1)
                         tma_load_2d(a + A_BYTES / 2, &tmW, (kb + i) * BK, rowA1, &full[i]);
                     }
                     pdl_wait();
-                    for (int i = 0; i < pre; ++i)
-                        tma_load_2d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, &full[i]);
+                    for (int i = 0; i < pre; ++i) {
+                        if (p.planes == 2) tma_load_3d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, 0, &full[i]);
+                        else tma_load_2d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, &full[i]);
+                    }
                     kk0 = pre;
                     it = pre;
                     first = false;
@@ -139,14 +145,15 @@ __global__ void __launch_bounds__(NT, 1)
                     mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
                     tma_load_2d(a, &tmW, k, rowA0, &full[s]);
                     tma_load_2d(a + A_BYTES / 2, &tmW, k, rowA1, &full[s]);
-                    tma_load_2d(sB + (size_t)s * B_BYTES, &tmX, k, m0, &full[s]);
+                    if (p.planes == 2) tma_load_3d(sB + (size_t)s * B_BYTES, &tmX, k, m0, 0, &full[s]);
+                    else tma_load_2d(sB + (size_t)s * B_BYTES, &tmX, k, m0, &full[s]);
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            const uint32_t idesc = idesc_bf16(TM);
+            const uint32_t idesc = idesc_bf16(wide ? 2 * TM : TM);
             int it = 0, lt = 0;  // global stage counter, local tile counter
             bool ok = true;
             for (int t = tile0; t < n_tiles_total && ok; t += tstride, ++lt) {
@@ -164,9 +171,13 @@ __global__ void __launch_bounds__(NT, 1)
                     const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_BYTES));
                     const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_BYTES));
 #pragma unroll
-                    for (int k4 = 0; k4 < BK / 16; ++k4)  // +32 bytes per K=16 step inside the swizzle row
+                    for (int k4 = 0; k4 < BK / 16; ++k4) {  // +32 bytes per K=16 step inside the swizzle row
                         mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)(k4 * 2), idesc,
                                  (kk > 0 || k4 > 0) ? 1u : 0u);
+                        if (p.planes == 2 && !wide)  // lo plane: TM rows (TM*128 bytes, a multiple of 1024) further on
+                            mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)((TM * 128) >> 4) + (uint64_t)(k4 * 2),
+                                     idesc, 1u);
+                    }
                     mma_commit(&empty[s]);
                 }
                 mma_commit(&acc_full[b]);
@@ -187,7 +198,7 @@ __global__ void __launch_bounds__(NT, 1)
             float v[CH];
             if (!split) {
                 for (int c = 0; c < TM; c += CH) {
-                    if (ok) tmem_ld16(trow + c, v);
+                    if (ok) acc_ld16(trow, c, lo_col, v);
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(NT, 1)
             } else {
                 // park this CTA's partial tile in shared memory (the stage ring is idle now)
                 for (int c = 0; c < TM; c += CH) {
-                    if (ok) tmem_ld16(trow + c, v);
+                    if (ok) acc_ld16(trow, c, lo_col, v);
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
@@ -352,19 +363,25 @@ int GemmTC<T>::init(float *w, int wf, int *sm, int ns) {
 }
 
 template <typename T>
-const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows) {
-    char key[96];
-    snprintf(key, sizeof key, "%p/%d/%d/%d/%d", ptr, rows, cols, ld, box_rows);
+const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows,
+                                         size_t plane_stride) {
+    char key[128];
+    snprintf(key, sizeof key, "%p/%d/%d/%d/%d/%zu", ptr, rows, cols, ld, box_rows, plane_stride);
     auto it = maps.find(key);
     if (it != maps.end()) return &it->second;
     if (maps.size() > 4096) maps.clear();
     CUtensorMap m;
     memset(&m, 0, sizeof m);
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)ld * sizeof(bf16)};
-    cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = get_encode()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box,
+    const cuuint32_t rank = plane_stride ? 3 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, 2};
+    cuuint64_t strides[2] = {(cuuint64_t)ld * sizeof(bf16), (cuuint64_t)plane_stride * sizeof(bf16)};
+    cuuint32_t box[3] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (plane_stride && (plane_stride * sizeof(bf16)) % 16) {
+        err = "lo-plane offset is not a multiple of 16 bytes";
+        return nullptr;
+    }
+    CUresult r = get_encode()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -416,7 +433,8 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
     p.m_tiles = (M + TM - 1) / TM;
     p.k_steps = (K + tc::BK - 1) / tc::BK;
     const int tiles = p.n_tiles * p.m_tiles;
-    const int stage_bytes = tc::A_BYTES + TM * 128;
+    p.planes = e.lo ? 2 : 1;
+    const int stage_bytes = tc::A_BYTES + TM * 128 * p.planes;
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::CH * 4 + 64 * 8 + 64;
     // Measured on B200 (decode shapes, M = 16): projections with at least as
     // many tiles as SMs stream fastest with one tile per CTA and two ~100 KB
@@ -440,7 +458,7 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
     p.keep_logits = keep_logits;
     const int grid_x = p.n_tiles;  // one tile per CTA
     const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
-    const CUtensorMap *mx = tensor_map(X, M, K, ldx, TM);
+    const CUtensorMap *mx = tensor_map(X, M, K, ldx, TM, e.lo);
     if (!mw || !mx) return;
     switch (TM) {
         case 16: launch_kind<16>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;

@@ -30,6 +30,7 @@ struct TcParams {
     int *err;               // device error word (bounded waits)
     float2 *lm_part;        // EPI_LOGITS: per (n_tile, row) best (value, index)
     int keep_logits;        // EPI_LOGITS: also store fp32 logits in Y
+    int planes;             // activation planes (2: hi + lo, two MMAs per K step)
 };
 
 template <typename T>
@@ -53,7 +54,10 @@ struct GemmTC {
     // tuning overrides (0 = automatic): K splits per tile, shared-memory budget in KB
     int tune_splits = 0, tune_smem_kb = 0;
     std::unordered_map<std::string, CUtensorMap> maps;
-    const CUtensorMap *tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows);
+    // 2-D map of a [rows][cols] bf16 matrix (leading dimension ld), box {64, box_rows};
+    // plane_stride > 0: 3-D map over the hi plane and the lo plane plane_stride
+    // elements after it, box {64, box_rows, 2}
+    const CUtensorMap *tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows, size_t plane_stride = 0);
 };
 
 // Row-wise argmax over the LM-head partials: mode 0 idx[r]; mode 1 drafter rows.

@@ -32,30 +32,32 @@ void launch_embed_block(const T *emb, int H, SeqState *st, const int *active, in
 template <typename T>
 void launch_embed_norm(const T *emb, int H, SeqState *st, const int *active, int nseq, int B, int is_draft,
                        const int *drafts, int mask_id, float *x, RowMeta *meta, RowMeta *ctx_meta, const float *g, T *xg,
-                       int xg_ld, float *ssq, int ssq_ld, cudaStream_t s);
+                       int xg_ld, size_t lo, float *ssq, int ssq_ld, cudaStream_t s);
 template <typename T>
 void launch_embed_tokens(const T *emb, int H, const int *tokens, int R, int seq, int pos0,
                          float *x, RowMeta *meta, cudaStream_t s);
 void launch_ctx_meta_prefill(RowMeta *meta, int R, int seq, int pos0, cudaStream_t s);
 
 // ---- normalisation / elementwise ----
+// `lo` (elements) is the offset of the low plane of two-plane bf16 activations
+// (see st_act in common.cuh); 0 for single-plane outputs.
 template <typename TO>
-void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, TO *out, int ldo,
+void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, TO *out, int ldo, size_t lo,
                     int R, cudaStream_t s);
 template <typename T>
-void launch_residual(float *x, const float *Y, int ldy, int H, int R, const TapDst<T> &taps,
+void launch_residual(float *x, const float *Y, int ldy, int H, int R, const TapDst<T> &taps, size_t lo,
                      const RowMeta *meta, cudaStream_t s);
 template <typename T>
-void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, cudaStream_t s);
+void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, size_t lo, cudaStream_t s);
 template <typename T>
 void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot,
                          const RowMeta *meta, const RowMeta *ctx_meta, int nq, int nkv, int hd,
-                         const float2 *rope, T *q_out, T *kc, T *vc, int max_len, cudaStream_t s);
+                         const float2 *rope, T *q_out, T *kc, T *vc, int max_len, size_t lo, cudaStream_t s);
 
 // ---- GEMM (CUDA-core, fp32 accumulate): Y[M][N] = X[M][K] . W[N][K]^T ----
 template <typename T>
 void launch_gemm_simt(const T *X, int ldx, int M, const T *W, int ldw, int N, int K, float *Y,
-                      int ldy, cudaStream_t s);
+                      int ldy, size_t lo, cudaStream_t s);
 
 // ---- attention (CUDA-core reference path, used for fp32 models) ----
 template <typename T>
@@ -82,11 +84,11 @@ void launch_ar_step(SeqState *st, const int *active, int nseq, const int *g, int
 void launch_moe_topk(const float *router_logits, int E, int R, int k, int *sel, float *wt,
                      cudaStream_t s);
 template <typename T>
-void launch_moe_experts_simt(const T *m, int ldm, int R, int k, const int *sel, const T *w_gate_up,
+void launch_moe_experts_simt(const T *m, int ldm, size_t lo, int R, int k, const int *sel, const T *w_gate_up,
                              const T *w_down, int H, int Fe, float *part, cudaStream_t s);
 template <typename T>
 void launch_moe_combine(float *x, const float *part, const float *wt, int H, int R, int k,
-                        const TapDst<T> &taps, const RowMeta *meta, cudaStream_t s);
+                        const TapDst<T> &taps, size_t lo, const RowMeta *meta, cudaStream_t s);
 
 // ---- tables ----
 void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStream_t s);
@@ -131,6 +133,9 @@ struct Epi {
     const float *g_next = nullptr;
     float *ssq_out = nullptr;
     int ssq_ld = 0;
+    // two-plane bf16 activations: offset (elements) of the low plane of the
+    // input X and of every T output above (q_out, kc, vc, taps, h, xg); 0 = one plane
+    size_t lo = 0;
 };
 
 void launch_gather_rows(const void *src, void *dst, size_t row_bytes, const int *active, int nseq, int B,

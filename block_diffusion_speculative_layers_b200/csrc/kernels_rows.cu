@@ -80,7 +80,7 @@ template <typename T>
 __global__ void embed_norm_kernel(const T *__restrict__ emb, int H, SeqState *st, const int *__restrict__ active, int B,
                                   int is_draft, const int *__restrict__ drafts, int mask_id, float *__restrict__ x,
                                   RowMeta *meta, RowMeta *ctx_meta, const float *__restrict__ g, T *__restrict__ xg,
-                                  int xg_ld, float *__restrict__ ssq, int ssq_ld) {
+                                  int xg_ld, size_t lo, float *__restrict__ ssq, int ssq_ld) {
     pdl_trigger();
     pdl_wait();
     __shared__ float red[8];
@@ -97,7 +97,7 @@ __global__ void embed_norm_kernel(const T *__restrict__ emb, int H, SeqState *st
         if (c < H) {
             v = to_f(e[c]);
             x[(size_t)r * H + c] = v;
-            xg[(size_t)r * xg_ld + c] = from_f<T>(v * g[c]);
+            st_act(xg, (size_t)r * xg_ld + c, lo, v * g[c]);
         }
         float sq = warp_sum(v * v);
         if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
@@ -132,9 +132,9 @@ __global__ void embed_norm_kernel(const T *__restrict__ emb, int H, SeqState *st
 template <typename T>
 void launch_embed_norm(const T *emb, int H, SeqState *st, const int *active, int nseq, int B, int is_draft,
                        const int *drafts, int mask_id, float *x, RowMeta *meta, RowMeta *ctx_meta, const float *g, T *xg,
-                       int xg_ld, float *ssq, int ssq_ld, cudaStream_t s) {
+                       int xg_ld, size_t lo, float *ssq, int ssq_ld, cudaStream_t s) {
     launch_k(embed_norm_kernel<T>, dim3(nseq * B), dim3(256), 0, s, 1, emb, H, st, active, B, is_draft, drafts, mask_id, x,
-             meta, ctx_meta, g, xg, xg_ld, ssq, ssq_ld);
+             meta, ctx_meta, g, xg, xg_ld, lo, ssq, ssq_ld);
 }
 
 template <typename T>
@@ -186,7 +186,7 @@ void launch_ctx_meta_prefill(RowMeta *meta, int R, int seq, int pos0, cudaStream
 
 template <typename TO>
 __global__ void rmsnorm_kernel(const float *__restrict__ x, int ldx, const float *__restrict__ g,
-                               int H, float eps, TO *__restrict__ out, int ldo) {
+                               int H, float eps, TO *__restrict__ out, int ldo, size_t lo) {
     pdl_trigger();
     pdl_wait();
     const int r = blockIdx.x;
@@ -204,15 +204,14 @@ __global__ void rmsnorm_kernel(const float *__restrict__ x, int ldx, const float
     }
     __syncthreads();
     const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
-    TO *o = out + (size_t)r * ldo;
-    for (int c = threadIdx.x; c < H; c += blockDim.x) o[c] = from_f<TO>(xr[c] * inv * g[c]);
+    for (int c = threadIdx.x; c < H; c += blockDim.x) st_act(out, (size_t)r * ldo + c, lo, xr[c] * inv * g[c]);
 }
 
 template <typename TO>
-void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, TO *out, int ldo, int R,
+void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, TO *out, int ldo, size_t lo, int R,
                     cudaStream_t s) {
     if (R <= 0) return;
-    launch_k(rmsnorm_kernel<TO>, dim3(R), dim3(256), 0, s, 1, x, ldx, g, H, eps, out, ldo);
+    launch_k(rmsnorm_kernel<TO>, dim3(R), dim3(256), 0, s, 1, x, ldx, g, H, eps, out, ldo, lo);
 }
 
 // ------------------------------------------------------------------------
@@ -221,7 +220,7 @@ void launch_rmsnorm(const float *x, int ldx, const float *g, int H, float eps, T
 
 template <typename T>
 __global__ void residual_kernel(float *__restrict__ x, const float *__restrict__ Y, int ldy, int H,
-                                TapDst<T> taps, const RowMeta *__restrict__ meta) {
+                                TapDst<T> taps, size_t lo, const RowMeta *__restrict__ meta) {
     pdl_trigger();
     pdl_wait();
     const int r = blockIdx.x;
@@ -232,33 +231,33 @@ __global__ void residual_kernel(float *__restrict__ x, const float *__restrict__
         float v = xr[c] + yr[c];
         xr[c] = v;
         for (int t = 0; t < taps.n; ++t)
-            taps.base[(size_t)trow * taps.ld + taps.col[t] + c] = from_f<T>(v);
+            st_act(taps.base, (size_t)trow * taps.ld + taps.col[t] + c, lo, v);
     }
 }
 
 template <typename T>
-void launch_residual(float *x, const float *Y, int ldy, int H, int R, const TapDst<T> &taps,
+void launch_residual(float *x, const float *Y, int ldy, int H, int R, const TapDst<T> &taps, size_t lo,
                      const RowMeta *meta, cudaStream_t s) {
     if (R <= 0) return;
-    launch_k(residual_kernel<T>, dim3(R), dim3(256), 0, s, 1, x, Y, ldy, H, taps, meta);
+    launch_k(residual_kernel<T>, dim3(R), dim3(256), 0, s, 1, x, Y, ldy, H, taps, lo, meta);
 }
 
 template <typename T>
-__global__ void swiglu_kernel(const float *__restrict__ Y, int ldy, int F, T *__restrict__ h, int ldh) {
+__global__ void swiglu_kernel(const float *__restrict__ Y, int ldy, int F, T *__restrict__ h, int ldh, size_t lo) {
     pdl_trigger();
     pdl_wait();
     const int r = blockIdx.y;
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= F) return;
     const float gt = Y[(size_t)r * ldy + c], up = Y[(size_t)r * ldy + F + c];
-    h[(size_t)r * ldh + c] = from_f<T>(silu_f(gt) * up);
+    st_act(h, (size_t)r * ldh + c, lo, silu_f(gt) * up);
 }
 
 template <typename T>
-void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, cudaStream_t s) {
+void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, size_t lo, cudaStream_t s) {
     if (R <= 0) return;
     dim3 grid((F + 255) / 256, R);
-    launch_k(swiglu_kernel<T>, dim3(grid), dim3(256), 0, s, 1, Y, ldy, F, h, ldh);
+    launch_k(swiglu_kernel<T>, dim3(grid), dim3(256), 0, s, 1, Y, ldy, F, h, ldh, lo);
 }
 
 // Y columns c correspond to rows col0 + c of the layer's Wqkv = [Wq; Wk; Wv].
@@ -269,7 +268,7 @@ __global__ void qkv_epilogue_kernel(const float *__restrict__ Y, int ldy, int co
                                     const RowMeta *__restrict__ meta, const RowMeta *__restrict__ ctx_meta,
                                     int nq, int nkv, int hd, const float2 *__restrict__ rope,
                                     T *__restrict__ q_out, T *__restrict__ kc, T *__restrict__ vc,
-                                    int max_len) {
+                                    int max_len, size_t lo) {
     pdl_trigger();
     pdl_wait();
     const int r = blockIdx.x;
@@ -289,30 +288,30 @@ __global__ void qkv_epilogue_kernel(const float *__restrict__ Y, int ldy, int co
         const float2 cs = tab[i];
         const float o1 = x1 * cs.x - x2 * cs.y, o2 = x2 * cs.x + x1 * cs.y;
         if (head < nq) {
-            q_out[(size_t)r * qd + base + i] = from_f<T>(o1);
-            q_out[(size_t)r * qd + base + i + half] = from_f<T>(o2);
+            st_act(q_out, (size_t)r * qd + base + i, lo, o1);
+            st_act(q_out, (size_t)r * qd + base + i + half, lo, o2);
         } else {
             const int kh = head - nq;
             T *dst = kc + (((size_t)m.seq * nkv + kh) * max_len + m.pos) * hd;
-            dst[i] = from_f<T>(o1);
-            dst[i + half] = from_f<T>(o2);
+            st_act(dst, i, lo, o1);
+            st_act(dst, i + half, lo, o2);
         }
     }
     (void)c_begin;
     for (int e = threadIdx.x; e < kd; e += blockDim.x) {
         const int kh = e / hd, d = e % hd;
         T *dst = vc + (((size_t)m.seq * nkv + kh) * max_len + m.pos) * hd;
-        dst[d] = from_f<T>(y[qd + kd + e]);
+        st_act(dst, d, lo, y[qd + kd + e]);
     }
 }
 
 template <typename T>
 void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot, const RowMeta *meta,
                          const RowMeta *ctx_meta, int nq, int nkv, int hd, const float2 *rope, T *q_out,
-                         T *kc, T *vc, int max_len, cudaStream_t s) {
+                         T *kc, T *vc, int max_len, size_t lo, cudaStream_t s) {
     if (R_tot <= 0) return;
     launch_k(qkv_epilogue_kernel<T>, dim3(R_tot), dim3(128), 0, s, 1, Y, ldy, col0, R_blk, meta, ctx_meta, nq, nkv, hd, rope,
-                                                 q_out, kc, vc, max_len);
+                                                 q_out, kc, vc, max_len, lo);
 }
 
 // ------------------------------------------------------------------------
@@ -518,20 +517,20 @@ void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStrea
 // ------------------------------------------------------------------------
 #define DFL_INST(T)                                                                                         \
     template void launch_embed_norm<T>(const T *, int, SeqState *, const int *, int, int, int, const int *, int, \
-                                       float *, RowMeta *, RowMeta *, const float *, T *, int, float *, int,     \
+                                       float *, RowMeta *, RowMeta *, const float *, T *, int, size_t, float *, int, \
                                        cudaStream_t);                                                           \
     template void launch_embed_block<T>(const T *, int, SeqState *, const int *, int, int, int, const int *, \
                                         int, float *, RowMeta *, RowMeta *, cudaStream_t);                  \
     template void launch_embed_tokens<T>(const T *, int, const int *, int, int, int, float *, RowMeta *,    \
                                          cudaStream_t);                                                     \
-    template void launch_rmsnorm<T>(const float *, int, const float *, int, float, T *, int, int,           \
+    template void launch_rmsnorm<T>(const float *, int, const float *, int, float, T *, int, size_t, int,   \
                                     cudaStream_t);                                                          \
-    template void launch_residual<T>(float *, const float *, int, int, int, const TapDst<T> &,              \
+    template void launch_residual<T>(float *, const float *, int, int, int, const TapDst<T> &, size_t,      \
                                      const RowMeta *, cudaStream_t);                                        \
-    template void launch_swiglu<T>(const float *, int, int, int, T *, int, cudaStream_t);                   \
+    template void launch_swiglu<T>(const float *, int, int, int, T *, int, size_t, cudaStream_t);           \
     template void launch_qkv_epilogue<T>(const float *, int, int, int, int, const RowMeta *,                \
                                          const RowMeta *, int, int, int, const float2 *, T *, T *, T *,     \
-                                         int, cudaStream_t);
+                                         int, size_t, cudaStream_t);
 DFL_INST(float)
 DFL_INST(bf16)
 #undef DFL_INST

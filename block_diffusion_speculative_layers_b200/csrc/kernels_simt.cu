@@ -15,7 +15,7 @@ namespace dfl {
 template <typename T>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const T *__restrict__ X, int ldx, int M,
                                                         const T *__restrict__ W, int ldw, int N, int K,
-                                                        float *__restrict__ Y, int ldy) {
+                                                        float *__restrict__ Y, int ldy, size_t lo) {
     pdl_trigger();
     pdl_wait();
     __shared__ float Ws[64][33];
@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const T *__restrict__ X,
         for (int e = tid; e < 32 * 32; e += 256) {
             const int rr = e >> 5, kk = e & 31;
             const int m = m0 + rr, k = k0 + kk;
-            Xs[rr][kk] = (m < M && k < K) ? to_f(X[(size_t)m * ldx + k]) : 0.f;
+            Xs[rr][kk] = (m < M && k < K) ? ld_act(X, (size_t)m * ldx + k, lo) : 0.f;
         }
         __syncthreads();
 #pragma unroll 8
@@ -56,10 +56,10 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const T *__restrict__ X,
 
 template <typename T>
 void launch_gemm_simt(const T *X, int ldx, int M, const T *W, int ldw, int N, int K, float *Y, int ldy,
-                      cudaStream_t s) {
+                      size_t lo, cudaStream_t s) {
     if (M <= 0 || N <= 0) return;
     dim3 grid((N + 63) / 64, (M + 31) / 32);
-    launch_k(gemm_simt_kernel<T>, dim3(grid), dim3(256), 0, s, 1, X, ldx, M, W, ldw, N, K, Y, ldy);
+    launch_k(gemm_simt_kernel<T>, dim3(grid), dim3(256), 0, s, 1, X, ldx, M, W, ldw, N, K, Y, ldy, lo);
 }
 
 // ------------------------------------------------------------------------
@@ -166,7 +166,7 @@ void launch_moe_topk(const float *router_logits, int E, int R, int k, int *sel, 
 
 // Expert FFN per (row, choice): part[rk] = W_down_e (SiLU(W_gate_e m) * W_up_e m)
 template <typename T>
-__global__ void moe_experts_simt_kernel(const T *__restrict__ m, int ldm, int k, const int *__restrict__ sel,
+__global__ void moe_experts_simt_kernel(const T *__restrict__ m, int ldm, size_t lo, int k, const int *__restrict__ sel,
                                         const T *__restrict__ w_gate_up, const T *__restrict__ w_down, int H,
                                         int Fe, float *__restrict__ part) {
     pdl_trigger();
@@ -176,7 +176,7 @@ __global__ void moe_experts_simt_kernel(const T *__restrict__ m, int ldm, int k,
     float *gu = sm + H;      // [2Fe]
     const int rk = blockIdx.x, r = rk / k;
     const int e = sel[rk];
-    for (int c = threadIdx.x; c < H; c += blockDim.x) xs[c] = to_f(m[(size_t)r * ldm + c]);
+    for (int c = threadIdx.x; c < H; c += blockDim.x) xs[c] = ld_act(m, (size_t)r * ldm + c, lo);
     __syncthreads();
     const T *Wgu = w_gate_up + (size_t)e * 2 * Fe * H;
     for (int o = threadIdx.x; o < 2 * Fe; o += blockDim.x) {
@@ -186,7 +186,12 @@ __global__ void moe_experts_simt_kernel(const T *__restrict__ m, int ldm, int k,
         gu[o] = a;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < Fe; i += blockDim.x) gu[i] = to_f(from_f<T>(silu_f(gu[i]) * gu[Fe + i]));
+    // the expert's hidden activation is a GEMM input: rounded like a stored one
+    // (single bf16 plane), or kept at fp32 where two planes would carry it
+    for (int i = threadIdx.x; i < Fe; i += blockDim.x) {
+        const float hv = silu_f(gu[i]) * gu[Fe + i];
+        gu[i] = lo ? hv : to_f(from_f<T>(hv));
+    }
     __syncthreads();
     const T *Wd = w_down + (size_t)e * H * Fe;
     for (int o = threadIdx.x; o < H; o += blockDim.x) {
@@ -198,16 +203,17 @@ __global__ void moe_experts_simt_kernel(const T *__restrict__ m, int ldm, int k,
 }
 
 template <typename T>
-void launch_moe_experts_simt(const T *m, int ldm, int R, int k, const int *sel, const T *w_gate_up,
+void launch_moe_experts_simt(const T *m, int ldm, size_t lo, int R, int k, const int *sel, const T *w_gate_up,
                              const T *w_down, int H, int Fe, float *part, cudaStream_t s) {
     if (R <= 0) return;
     const size_t smem = sizeof(float) * (size_t)(H + 2 * Fe);
-    launch_k(moe_experts_simt_kernel<T>, dim3(R * k), dim3(256), smem, s, 1, m, ldm, k, sel, w_gate_up, w_down, H, Fe, part);
+    launch_k(moe_experts_simt_kernel<T>, dim3(R * k), dim3(256), smem, s, 1, m, ldm, lo, k, sel, w_gate_up, w_down, H, Fe,
+             part);
 }
 
 template <typename T>
 __global__ void moe_combine_kernel(float *__restrict__ x, const float *__restrict__ part,
-                                   const float *__restrict__ wt, int H, int k, TapDst<T> taps,
+                                   const float *__restrict__ wt, int H, int k, TapDst<T> taps, size_t lo,
                                    const RowMeta *__restrict__ meta) {
     pdl_trigger();
     pdl_wait();
@@ -218,26 +224,26 @@ __global__ void moe_combine_kernel(float *__restrict__ x, const float *__restric
         for (int t = 0; t < k; ++t) acc = fmaf(wt[r * k + t], part[((size_t)r * k + t) * H + c], acc);
         const float v = x[(size_t)r * H + c] + acc;
         x[(size_t)r * H + c] = v;
-        for (int i = 0; i < taps.n; ++i) taps.base[(size_t)trow * taps.ld + taps.col[i] + c] = from_f<T>(v);
+        for (int i = 0; i < taps.n; ++i) st_act(taps.base, (size_t)trow * taps.ld + taps.col[i] + c, lo, v);
     }
 }
 
 template <typename T>
 void launch_moe_combine(float *x, const float *part, const float *wt, int H, int R, int k,
-                        const TapDst<T> &taps, const RowMeta *meta, cudaStream_t s) {
+                        const TapDst<T> &taps, size_t lo, const RowMeta *meta, cudaStream_t s) {
     if (R <= 0) return;
-    launch_k(moe_combine_kernel<T>, dim3(R), dim3(256), 0, s, 1, x, part, wt, H, k, taps, meta);
+    launch_k(moe_combine_kernel<T>, dim3(R), dim3(256), 0, s, 1, x, part, wt, H, k, taps, lo, meta);
 }
 
 #define DFL_INST(T)                                                                                          \
-    template void launch_gemm_simt<T>(const T *, int, int, const T *, int, int, int, float *, int,           \
+    template void launch_gemm_simt<T>(const T *, int, int, const T *, int, int, int, float *, int, size_t,   \
                                       cudaStream_t);                                                         \
     template void launch_attention_simt<T>(const T *, int, const T *, const T *, const RowMeta *, int, int,  \
                                            int, int, int, T *, int, cudaStream_t);                           \
-    template void launch_moe_experts_simt<T>(const T *, int, int, int, const int *, const T *, const T *,    \
+    template void launch_moe_experts_simt<T>(const T *, int, size_t, int, int, const int *, const T *, const T *, \
                                              int, int, float *, cudaStream_t);                               \
     template void launch_moe_combine<T>(float *, const float *, const float *, int, int, int,                \
-                                        const TapDst<T> &, const RowMeta *, cudaStream_t);
+                                        const TapDst<T> &, size_t, const RowMeta *, cudaStream_t);
 DFL_INST(float)
 DFL_INST(bf16)
 #undef DFL_INST

@@ -71,6 +71,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Two-plane activation tile: box {BK, rows, 2} of a 3-D map whose third
+// dimension steps from the hi plane to the lo plane; lands as [2][rows][BK].
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // K-major operand, 128-byte swizzle: 8-row groups 1024 B apart (SBO), sm100 descriptor version 1.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     uint64_t d = 0;
@@ -112,6 +122,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
     for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Columns c..c+15 of a tile accumulator.  With a wide two-plane MMA (one
+// N = 2*TM product over the hi and lo activation rows) the lo-plane partial
+// sums sit lo_col = TM columns further on and are added here; lo_col = 0 otherwise.
+__device__ __forceinline__ void acc_ld16(uint32_t taddr, int c, int lo_col, float *v) {
+    tmem_ld16(taddr + (uint32_t)c, v);
+    if (lo_col) {
+        float t[16];
+        tmem_ld16(taddr + (uint32_t)(lo_col + c), t);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] += t[j];
+    }
+}
+
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
@@ -146,7 +169,7 @@ __device__ __forceinline__ void norm_outputs(const TcParams &p, const Epi<bf16> 
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
         const bool ok = nok && j < nc && m0c + j < M;
-        if (ok && e.xg) e.xg[(size_t)(m0c + j) * e.xg_ld + n] = __float2bfloat16_rn(y[j] * gn);
+        if (ok && e.xg) st_act(e.xg, (size_t)(m0c + j) * e.xg_ld + n, e.lo, y[j] * gn);
         float sq = ok ? y[j] * y[j] : 0.f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -205,7 +228,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             xo[j] = nx;
             e.x[(size_t)(m0c + j) * p.N + n] = nx;
             for (int t = 0; t < e.taps.n; ++t)
-                e.taps.base[(size_t)trow[j] * e.taps.ld + e.taps.col[t] + n] = __float2bfloat16_rn(nx);
+                st_act(e.taps.base, (size_t)trow[j] * e.taps.ld + e.taps.col[t] + n, e.lo, nx);
         }
         if (e.ssq_out) norm_outputs(p, e, nt, n, q, lane, m0c, nc, xo, red);
     } else if (KIND == EPI_NORMOUT) {
@@ -250,7 +273,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
                     const int m = m0c + j;
                     if (j >= nc || m >= M) break;
                     const float up = stg[(n_local + 64) * STG_LD + j];
-                    e.h[(size_t)m * p.swiglu_F + f] = __float2bfloat16_rn(silu_f(v[j]) * up);
+                    st_act(e.h, (size_t)m * p.swiglu_F + f, e.lo, silu_f(v[j]) * up);
                 }
             }
         }
@@ -300,11 +323,11 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
                     out = d < half ? v[j] * cs[j].x - other * cs[j].y : v[j] * cs[j].x + other * cs[j].y;
                 }
                 if (is_q) {
-                    e.q_out[(size_t)(m0c + j) * qd + cg] = __float2bfloat16_rn(out);
+                    st_act(e.q_out, (size_t)(m0c + j) * qd + cg, e.lo, out);
                 } else {
                     const int hh = is_k ? (cg - qd) / hd : (cg - qd - kd) / hd;
                     bf16 *dst = (is_k ? e.kc : e.vc) + (((size_t)mt.seq * e.nkv + hh) * e.max_len + mt.pos) * hd;
-                    dst[d] = __float2bfloat16_rn(out);
+                    st_act(dst, (size_t)d, e.lo, out);
                 }
             }
         }

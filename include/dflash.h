@@ -56,7 +56,14 @@ typedef enum {
     DFLASH_EUNSUPPORTED = 7/* shape the kernels do not support (e.g. head_dim not 64/128) */
 } dflash_status;
 
-enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1 };
+/* Model dtypes.  FP32: fp32 weights and activations.  BF16: bf16 weights;
+ * activations (GEMM inputs, q, the K/V caches) carried as two bf16 planes,
+ * hi = bf16(v) and lo = bf16(v - hi), so each bf16 tensor-core product takes
+ * two (attention: three) MMAs and the result keeps ~16 significant bits --
+ * weight bytes are unchanged, activation and K/V bytes double.  BF16_FAST:
+ * bf16 weights and single-plane bf16 activations (half the K/V bytes and MMAs,
+ * with the rounding error of plain bf16 inference). */
+enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1, DFLASH_BF16_FAST = 2 };
 
 /* Draft modes.  MODEL: drafts are the drafter's argmax.  SCRIPT: the drafter
  * still runs in full, then its drafts are replaced from a per-sequence token
@@ -85,7 +92,7 @@ typedef struct {
     int32_t max_batch;            /* sequences held at once */
     int32_t max_len;              /* positions per sequence (prompt + generated + B) */
     int32_t prefill_chunk;        /* prompt rows per prefill pass (0: default 1024) */
-    int32_t dtype;                /* DFLASH_FP32 or DFLASH_BF16 (weights, KV, GEMM inputs) */
+    int32_t dtype;                /* DFLASH_FP32, DFLASH_BF16 or DFLASH_BF16_FAST (see above) */
     int32_t keep_logits;          /* 1: keep fp32 logits of the last draft/verify for dflash_debug_logits */
     int32_t timeout_ms;           /* host wait bound for synchronising calls (0: 600000) */
 } dflash_config;
