@@ -84,8 +84,8 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
     float *stg = (float *)(sB + (size_t)stages * B_BYTES);
     float2 *red = (float2 *)(stg + 128 * STG_LD);
     RowMeta *smeta = (RowMeta *)(red + 4 * CH);
-    float *rsc = (float *)(smeta + CH);
-    uint64_t *full = (uint64_t *)(rsc + CH);
+    float *rsc = (float *)(smeta + CH);       // [RS_MAX] row scales of the folded norm
+    uint64_t *full = (uint64_t *)(rsc + RS_MAX);
     uint64_t *empty = full + stages;
     uint64_t *acc_full = empty + stages;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
+            const uint64_t wpol = l2_evict_first_policy();
             PendingX pend[16];
             int np = 0, ready_upto = L.op_begin - 1, it = 0;
             bool abort = false;
@@ -195,8 +196,8 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                         }
                         uint8_t *a = sA + (size_t)s * A_BYTES;
                         mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
-                        tma_load_2d(a, op.wmap, kk * BK, rowA0, &full[s]);
-                        tma_load_2d(a + A_BYTES / 2, op.wmap, kk * BK, rowA1, &full[s]);
+                        tma_load_2d_hint(a, op.wmap, kk * BK, rowA0, &full[s], wpol);
+                        tma_load_2d_hint(a + A_BYTES / 2, op.wmap, kk * BK, rowA1, &full[s], wpol);
                         const PendingX px{s, j, kk * BK};
                         if (np == 0 && x_ready(j)) issue_x(px);
                         else pend[np++] = px;
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                 if (threadIdx.x == 64) wait_counter(&L.op_done[j - 1], target, L.err);
                 epi_bar();
             }
+            if (op.e.rs_ssq) all_row_scales(op.e, 0, TM, op.p.M, rsc);
             const int ks = op.p.k_steps;
             long long g0, g1;
             cta_range(op, blockIdx.x, G, g0, g1);
@@ -292,12 +294,12 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                             if (lane == 0) mbar_arrive(&acc_empty[b]);
                         }
                         switch (op.kind) {
-                            case EPI_QKV: epilogue_chunk<EPI_QKV>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                            case EPI_RESID: epilogue_chunk<EPI_RESID>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                            case EPI_SWIGLU: epilogue_chunk<EPI_SWIGLU>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                            case EPI_LOGITS: epilogue_chunk<EPI_LOGITS>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                            case EPI_NORMOUT: epilogue_chunk<EPI_NORMOUT>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                            default: epilogue_chunk<EPI_STORE>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
+                            case EPI_QKV: epilogue_chunk<EPI_QKV>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                            case EPI_RESID: epilogue_chunk<EPI_RESID>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                            case EPI_SWIGLU: epilogue_chunk<EPI_SWIGLU>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                            case EPI_LOGITS: epilogue_chunk<EPI_LOGITS>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                            case EPI_NORMOUT: epilogue_chunk<EPI_NORMOUT>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                            default: epilogue_chunk<EPI_STORE>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
                         }
                     }
                 } else {
@@ -337,12 +339,12 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
                                 for (int jj = 0; jj < CH; ++jj) v[jj] += t[jj];
                             }
                             switch (op.kind) {
-                                case EPI_QKV: epilogue_chunk<EPI_QKV>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                                case EPI_RESID: epilogue_chunk<EPI_RESID>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                                case EPI_SWIGLU: epilogue_chunk<EPI_SWIGLU>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                                case EPI_LOGITS: epilogue_chunk<EPI_LOGITS>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                                case EPI_NORMOUT: epilogue_chunk<EPI_NORMOUT>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
-                                default: epilogue_chunk<EPI_STORE>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc); break;
+                                case EPI_QKV: epilogue_chunk<EPI_QKV>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                                case EPI_RESID: epilogue_chunk<EPI_RESID>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                                case EPI_SWIGLU: epilogue_chunk<EPI_SWIGLU>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                                case EPI_LOGITS: epilogue_chunk<EPI_LOGITS>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                                case EPI_NORMOUT: epilogue_chunk<EPI_NORMOUT>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
+                                default: epilogue_chunk<EPI_STORE>(op.p, op.e, nt, n_local, q, lane, c, CH, v, stg, red, smeta, rsc + c); break;
                             }
                         }
                     }
@@ -371,7 +373,7 @@ __global__ void __launch_bounds__(NT, 1) chain_kernel(ChainLaunch L) {
 }  // namespace tc
 
 static size_t chain_fixed_bytes() {
-    return 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::CH * 4 + 64 * 8 + 64;
+    return 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64;
 }
 
 int chain_stages(int tm, int planes) {

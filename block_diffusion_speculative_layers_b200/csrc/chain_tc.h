@@ -37,9 +37,19 @@ struct ChainLaunch {
     int planes;                // activation planes of every op (2: hi + lo)
 };
 
-// Host-side program: a list of projections uploaded once, launched in runs.
+// Raw operands of one op, for running a program one kernel per projection.
+struct HostOp {
+    const void *W;
+    int N, K;
+    const void *X;
+    int ldx, M;
+};
+
+// Host-side program: a list of projections uploaded once, launched in runs
+// (persistent chains) or one kernel per projection (same epilogues).
 struct ChainProgram {
     std::vector<ChainOp> ops;
+    std::vector<HostOp> hops;        // raw operands of ops[i]
     std::vector<CUtensorMap> maps;   // uploaded next to the ops
     ChainOp *d_ops = nullptr;        // device copies (state arena)
     CUtensorMap *d_maps = nullptr;

@@ -306,7 +306,9 @@ class Engine : public EngineBase {
     size_t lo_ = 0;  // low plane offset of two-plane activations (elements), 0: one plane
     float *ssq = nullptr;
     ChainProgram pv, pd;
-    bool chain_verify_ok = false, chain_draft_ok = false;
+    // bf16 decode passes run as projection programs with folded RMSNorms
+    // (fold_*_ok), one kernel per projection or, with chain_on, as persistent chains
+    bool chain_verify_ok = false, chain_draft_ok = false, chain_on = false;
     bool chain_used[3] = {false, false, false};
     int num_sms = 148;
     GemmTC<T> tc;
@@ -414,9 +416,12 @@ class Engine : public EngineBase {
             const int H = c.target.hidden;
             const bool shapes = H % 128 == 0 && num_sms <= 160 && 2 * L.R_dec <= 256;
             // DFLASH_PROJECTION_CHAIN=1 runs the dependent projections of a pass as
-            // persistent chains instead of one kernel per projection (same arithmetic)
+            // persistent chains instead of one kernel per projection (same arithmetic);
+            // DFLASH_FOLDED_NORM=0 goes back to separate RMSNorm kernels
             const char *ev = getenv("DFLASH_PROJECTION_CHAIN");
-            const bool allow = ev && ev[0] == '1';
+            chain_on = ev && ev[0] == '1';
+            const char *fv = getenv("DFLASH_FOLDED_NORM");
+            const bool allow = !(fv && fv[0] == '0');
             chain_draft_ok = allow && bf && shapes;
             chain_verify_ok = allow && bf && shapes && c.target.n_experts == 0;
             auto carve = [&](ChainProgram &pg, size_t off, int n_ops) {
@@ -454,6 +459,15 @@ class Engine : public EngineBase {
             err = "tensor-core GEMM set-up failed: " + tc.err;
             return DFLASH_ECUDA;
         }
+        // projection tiling overrides (measurement sweeps); unset = the built-in policy
+        auto env_int = [](const char *name) {
+            const char *v = getenv(name);
+            return v ? atoi(v) : 0;
+        };
+        tc.tune_splits = env_int("DFLASH_TC_SPLITS");
+        tc.tune_smem_kb = env_int("DFLASH_TC_SMEM_KB");
+        tc.tune_split_smem_kb = env_int("DFLASH_TC_SPLIT_SMEM_KB");
+        tc.tune_ctas_per_sm = env_int("DFLASH_TC_CTAS_PER_SM");
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);
         tc.keep_logits = c.keep_logits;
@@ -779,6 +793,7 @@ class Engine : public EngineBase {
             pg.tinfo.insert(pg.tinfo.end(), ti.begin(), ti.end());
             tile_off += p.n_tiles;
             pg.ops.push_back(op);
+            pg.hops.push_back(HostOp{W, N, K, X, ldx, M});
         }
     }
 
@@ -816,6 +831,7 @@ class Engine : public EngineBase {
         const int qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd, TK = c.n_taps * H;
         ChainProgram &pg = pv;
         pg.ops.clear();
+        pg.hops.clear();
         pg.maps.clear();
         pg.tinfo.clear();
         pg.valid = true;
@@ -882,6 +898,7 @@ class Engine : public EngineBase {
         const int qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd, TK = c.n_taps * c.target.hidden;
         ChainProgram &pg = pd;
         pg.ops.clear();
+        pg.hops.clear();
         pg.maps.clear();
         pg.tinfo.clear();
         pg.valid = true;
@@ -939,17 +956,34 @@ class Engine : public EngineBase {
         finish_program(pg);
     }
 
+    // ops [b, e) of a program: one persistent chain launch, or one projection kernel each
+    void run_ops(ChainProgram &pg, int b, int e) {
+        if constexpr (std::is_same<T, bf16>::value) {
+            if (chain_on && pg.valid) {
+                double bytes = 0.0;
+                for (int i = b; i < e; ++i)
+                    bytes += gemm_bytes(pg.hops[i].M, pg.hops[i].N, pg.hops[i].K, pg.ops[i].e);
+                timed(0, bytes, [&] { launch_chain(pg, b, e, num_sms, &stats->status, s); });
+                return;
+            }
+            for (int i = b; i < e; ++i) {
+                const HostOp &h = pg.hops[i];
+                gemm((const T *)h.X, h.ldx, h.M, h.W, h.N, h.K, pg.ops[i].e);
+            }
+        }
+    }
+
     void enqueue_verify_chain(int nseq) {
         const dflash_model_cfg &t = c.target;
         const int B = c.block_size, R = nseq * B, H = t.hidden;
         if (pv.key != nseq) build_verify_program(nseq);
-        pv.epoch++;
+        if (chain_on && pv.valid) pv.epoch++;
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, tl[0].attn_norm,
                              xg_t, H, lo_, ssq, L.ssq_ld, s);
-        launch_chain(pv, 0, 1, num_sms, &stats->status, s);
+        run_ops(pv, 0, 1);
         for (int l = 0; l < t.n_layers; ++l) {
             attention(q, tk + (size_t)l * kv_layer_elems(t), tv + (size_t)l * kv_layer_elems(t), meta, R, B, t, ao);
-            launch_chain(pv, 1 + 4 * l, 5 + 4 * l, num_sms, &stats->status, s);
+            run_ops(pv, 1 + 4 * l, 5 + 4 * l);
         }
         launch_lm_argmax(lm_part, (t.vocab + 127) / 128, R, 0, B, g, stats, s);
         launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
@@ -960,13 +994,13 @@ class Engine : public EngineBase {
         const dflash_model_cfg &d = c.drafter;
         const int B = c.block_size, R = nseq * B, H = d.hidden;
         if (pd.key != nseq) build_draft_program(nseq);
-        pd.epoch++;
+        if (chain_on && pd.valid) pd.epoch++;
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, dl[0].attn_norm,
                              dq_in, H, lo_, ssq, L.ssq_ld, s);
-        launch_chain(pd, 0, 2, num_sms, &stats->status, s);
+        run_ops(pd, 0, 2);
         for (int j = 0; j < d.n_layers; ++j) {
             attention(q, dk + (size_t)j * kv_layer_elems(d), dv + (size_t)j * kv_layer_elems(d), meta, R, B, d, ao);
-            launch_chain(pd, 2 + 4 * j, 6 + 4 * j, num_sms, &stats->status, s);
+            run_ops(pd, 2 + 4 * j, 6 + 4 * j);
         }
         if (B > 1) launch_lm_argmax(lm_part, (c.target.vocab + 127) / 128, R, 1, B, drafts, stats, s);
         if (draft_mode == DFLASH_DRAFT_SCRIPT)
@@ -1019,10 +1053,8 @@ class Engine : public EngineBase {
     void enqueue_draft(int nseq, bool contiguous) {
         if (chain_draft_ok && contiguous) {
             if (pd.key != nseq) build_draft_program(nseq);
-            if (pd.valid) {
-                enqueue_draft_chain(nseq);
-                return;
-            }
+            enqueue_draft_chain(nseq);
+            return;
         }
         chain_used[0] = false;
         const dflash_model_cfg &t = c.target, &d = c.drafter;
@@ -1050,10 +1082,8 @@ class Engine : public EngineBase {
     void enqueue_verify(int nseq) {
         if (chain_verify_ok) {
             if (pv.key != nseq) build_verify_program(nseq);
-            if (pv.valid) {
-                enqueue_verify_chain(nseq);
-                return;
-            }
+            enqueue_verify_chain(nseq);
+            return;
         }
         chain_used[1] = false;
         const dflash_model_cfg &t = c.target;

@@ -53,19 +53,20 @@ __global__ void __launch_bounds__(NT, 1)
     const bool wide = p.planes == 2 && TM <= 128;
     const int lo_col = wide ? TM : 0;
     const int NC1 = max(32, wide ? 2 * TM : TM);  // TMEM columns of one accumulator
-    constexpr int PLD = TM + 1;             // parked partial tile row stride (floats)
     uint8_t *sA = smem;
     uint8_t *sB = smem + (size_t)stages * A_BYTES;
     float *stg = (float *)(sB + (size_t)stages * B_BYTES);
     float2 *red = (float2 *)(stg + 128 * STG_LD);
     RowMeta *smeta = (RowMeta *)(red + 4 * CH);
-    float *rsc = (float *)(smeta + CH);
-    uint64_t *full = (uint64_t *)(rsc + CH);
+    float *rsc = (float *)(smeta + CH);       // [RS_MAX] row scales of the folded norm
+    uint64_t *full = (uint64_t *)(rsc + RS_MAX);
     uint64_t *empty = full + stages;
     uint64_t *acc_full = empty + stages;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
     uint32_t *tmem_slot = (uint32_t *)(acc_empty + 2);
-    float *part = (float *)sA;  // [128][PLD] after the last MMA (split-K only)
+    // split-K receive buffer [S][128][cpr] (16-byte aligned, after the fixed area)
+    float *recv = (float *)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
+    EpiIn pre;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.splits;
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer: one continuous ring over all tiles of this CTA ----------------
+            const uint64_t wpol = l2_evict_first_policy();
             int it = 0;     // global stage counter
             bool first = true, abort = false;
             for (int t = tile0; t < n_tiles_total && !abort; t += tstride) {
@@ -122,8 +124,8 @@ __global__ void __launch_bounds__(NT, 1)
                     for (int i = 0; i < pre; ++i) {
                         uint8_t *a = sA + (size_t)i * A_BYTES;
                         mbar_expect_tx(&full[i], A_BYTES + B_BYTES);
-                        tma_load_2d(a, &tmW, (kb + i) * BK, rowA0, &full[i]);
-                        tma_load_2d(a + A_BYTES / 2, &tmW, (kb + i) * BK, rowA1, &full[i]);
+                        tma_load_2d_hint(a, &tmW, (kb + i) * BK, rowA0, &full[i], wpol);
+                        tma_load_2d_hint(a + A_BYTES / 2, &tmW, (kb + i) * BK, rowA1, &full[i], wpol);
                     }
                     pdl_wait();
                     for (int i = 0; i < pre; ++i) {
@@ -143,8 +145,8 @@ __global__ void __launch_bounds__(NT, 1)
                     const int k = (kb + kk) * BK;
                     uint8_t *a = sA + (size_t)s * A_BYTES;
                     mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
-                    tma_load_2d(a, &tmW, k, rowA0, &full[s]);
-                    tma_load_2d(a + A_BYTES / 2, &tmW, k, rowA1, &full[s]);
+                    tma_load_2d_hint(a, &tmW, k, rowA0, &full[s], wpol);
+                    tma_load_2d_hint(a + A_BYTES / 2, &tmW, k, rowA1, &full[s], wpol);
                     if (p.planes == 2) tma_load_3d(sB + (size_t)s * B_BYTES, &tmX, k, m0, 0, &full[s]);
                     else tma_load_2d(sB + (size_t)s * B_BYTES, &tmX, k, m0, &full[s]);
                 }
@@ -188,10 +190,21 @@ __global__ void __launch_bounds__(NT, 1)
         pdl_wait();
         const int q = warp & 3;
         const int n_local = q * 32 + lane;
-        int lt = 0;
+        // K split: CTA `rank` of the cluster reduces and finishes columns [c_begin, c_end)
+        const int rank = split ? (int)cluster_rank() : 0;
+        const int cpr = split ? (TM + S - 1) / S : TM;
+        const int c_begin = split ? min(TM, rank * cpr) : 0;
+        const int c_end = split ? min(TM, c_begin + cpr) : TM;
+        int lt = 0, rs_mt = -1;
         for (int t = tile0; t < n_tiles_total; t += tstride, ++lt) {
             const int nt = t % p.n_tiles, mt = t / p.n_tiles;
             const int b = lt & 1;
+            if (e.rs_ssq && mt != rs_mt) {  // before the accumulator is ready
+                all_row_scales(e, mt * TM, TM, p.M, rsc);
+                rs_mt = mt;
+            }
+            // inputs of this CTA's first epilogue chunk, while the mainloop streams
+            if (c_end > c_begin) epi_prefetch<KIND>(p, e, nt, n_local, mt * TM + c_begin, min(CH, c_end - c_begin), pre, smeta);
             const uint32_t trow = tmem + (uint32_t)(b * NC1) + ((uint32_t)(q * 32) << 16);
             const bool ok = mbar_wait(&acc_full[b], (lt >> 1) & 1, p.err) && nk > 0;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -209,22 +222,32 @@ __global__ void __launch_bounds__(NT, 1)
                         if (lane == 0) mbar_arrive(&acc_empty[b]);
                     }
                     if (mt * TM + c < p.M || KIND != EPI_STORE)
-                        epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, mt * TM + c, CH, v, stg, red, smeta, rsc);
+                        epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, mt * TM + c, CH, v, stg, red, smeta, rsc + c,
+                                             c == 0 ? &pre : nullptr);
                 }
             } else {
-                // park this CTA's partial tile in shared memory (the stage ring is idle now)
+                // push this CTA's partial columns into the receive buffer of the CTA that
+                // finishes them: recv[source rank][weight row][column - owner's c_begin]
                 for (int c = 0; c < TM; c += CH) {
                     if (ok) acc_ld16(trow, c, lo_col, v);
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) part[n_local * PLD + c + j] = v[j];
+                    for (int j = 0; j < CH; ++j) {
+                        const int col = c + j, owner = col / cpr;
+                        if (col < TM) {
+                            float *dst = recv + ((size_t)rank * 128 + n_local) * cpr + (col - owner * cpr);
+                            st_cluster_f32(dst, (uint32_t)owner, v[j]);
+                        }
+                    }
                 }
             }
         }
     }
     if (split) {
+        // the pushes of every CTA are visible after the barrier (release / acquire);
+        // afterwards no CTA touches another's shared memory, so one barrier suffices
         __syncwarp();
         cluster_sync_all();
         if (warp >= 2) {
@@ -232,29 +255,23 @@ __global__ void __launch_bounds__(NT, 1)
             const int n_local = q * 32 + lane;
             const int nt = blockIdx.x, mt = blockIdx.y;
             const int rank = (int)cluster_rank();
-            const int cpr = (TM + S - 1) / S;  // columns reduced by this CTA
-            const int c_begin = rank * cpr, c_end = min(TM, c_begin + cpr);
-            const float *peers[8];
-#pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) peers[s2] = s2 < S ? peer_ptr(part, (uint32_t)s2) : part;
+            const int cpr = (TM + S - 1) / S;
+            const int c_begin = min(TM, rank * cpr), c_end = min(TM, c_begin + cpr);
             for (int c = c_begin; c < c_end; c += CH) {
                 const int nc = min(CH, c_end - c);
                 float v[CH];
 #pragma unroll
                 for (int j = 0; j < CH; ++j) v[j] = 0.f;
+                for (int s2 = 0; s2 < S; ++s2) {  // in rank order: identical results run to run
+                    const float *src = recv + ((size_t)s2 * 128 + n_local) * cpr + (c - c_begin);
 #pragma unroll
-                for (int s2 = 0; s2 < 8; ++s2) {
-                    if (s2 >= S) break;
-                    float tv[CH];
-#pragma unroll
-                    for (int j = 0; j < CH; ++j) tv[j] = j < nc ? peers[s2][n_local * PLD + c + j] : 0.f;
-#pragma unroll
-                    for (int j = 0; j < CH; ++j) v[j] += tv[j];
+                    for (int j = 0; j < CH; ++j)
+                        if (j < nc) v[j] += src[j];
                 }
-                epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, mt * TM + c, nc, v, stg, red, smeta, rsc);
+                epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, mt * TM + c, nc, v, stg, red, smeta, rsc + c,
+                                     c == c_begin ? &pre : nullptr);
             }
         }
-        cluster_sync_all();
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -317,7 +334,11 @@ int gemm_tc_workspace_floats(int max_rows, int max_n) {
 int gemm_tc_semaphores() { return 1 << 16; }
 
 bool &pdl_enabled() {
-    static bool on = true;
+    // DFLASH_PDL=0 launches every kernel without programmatic dependent launch
+    static bool on = [] {
+        const char *v = getenv("DFLASH_PDL");
+        return !(v && v[0] == '0');
+    }();
     return on;
 }
 
@@ -435,23 +456,30 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
     const int tiles = p.n_tiles * p.m_tiles;
     p.planes = e.lo ? 2 : 1;
     const int stage_bytes = tc::A_BYTES + TM * 128 * p.planes;
-    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::CH * 4 + 64 * 8 + 64;
-    // Measured on B200 (decode shapes, M = 16): projections with at least as
-    // many tiles as SMs stream fastest with one tile per CTA and two ~100 KB
-    // CTAs per SM; projections with fewer tiles split K over a cluster so that
-    // about one CTA per SM runs, each with a deeper (~150 KB) ring.
+    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64;
+    // Measured on B200 (decode shapes, M = 16, whole decode iteration): every
+    // projection streams best with ~110 KB CTAs, two of which fit on an SM --
+    // projections with fewer tiles than SMs split K over a cluster so that about
+    // one CTA per SM runs, and the other slot lets the next projection's CTAs
+    // start (programmatic dependent launch) and prefetch their weights while
+    // this one drains.  Larger (150 KB, one CTA per SM) rings were faster for
+    // a projection timed alone but 0.5 ms per iteration slower in the pipeline.
     int splits = 1;
-    if (e.kind != EPI_LOGITS && tiles < num_sms && p.k_steps >= 4) {
-        splits = std::max(1, std::min({8, p.k_steps / 2, num_sms / std::max(1, tiles)}));
+    const int slots = num_sms * std::max(1, tune_ctas_per_sm);  // CTAs the K-split aims to fill
+    if (e.kind != EPI_LOGITS && tiles < slots && p.k_steps >= 4) {
+        splits = std::max(1, std::min({8, p.k_steps / 2, slots / std::max(1, tiles)}));
         if (tune_splits > 0) splits = std::min(8, tune_splits);
         const int k_per = (p.k_steps + splits - 1) / splits;
         splits = (p.k_steps + k_per - 1) / k_per;
     }
-    int budget = splits > 1 ? 150 * 1024 : (TM <= 64 ? 112 * 1024 : 200 * 1024);
-    if (tune_smem_kb > 0) budget = tune_smem_kb * 1024;
-    const int stages = std::max(2, std::min(16, (budget - fixed) / stage_bytes));
-    const size_t smem = (size_t)fixed + (size_t)stages * stage_bytes;
-    if (splits > 1 && (size_t)stages * stage_bytes < (size_t)128 * (TM + 1) * 4) splits = 1;  // no room to park
+    if (TM > 64) splits = 1;  // keeps the split-K receive buffer (S x 128 x TM/S floats) small
+    // split-K receive buffer [S][128][ceil(TM/S)] floats, placed after the fixed area
+    const int recv_bytes = splits > 1 ? splits * 128 * ((TM + splits - 1) / splits) * 4 + 64 : 0;
+    int budget = splits > 1 ? 110 * 1024 : (TM <= 64 ? 112 * 1024 : 200 * 1024);
+    if (splits > 1 && tune_split_smem_kb > 0) budget = tune_split_smem_kb * 1024;
+    if (splits == 1 && tune_smem_kb > 0) budget = tune_smem_kb * 1024;
+    const int stages = std::max(2, std::min(16, (budget - fixed - recv_bytes) / stage_bytes));
+    const size_t smem = (size_t)fixed + (size_t)recv_bytes + (size_t)stages * stage_bytes;
     p.splits = splits;
     p.err = err_word;
     p.lm_part = lm_part;

@@ -52,7 +52,8 @@ struct GemmTC {
     int *err_word = nullptr;
     int num_sms = 148;
     // tuning overrides (0 = automatic): K splits per tile, shared-memory budget in KB
-    int tune_splits = 0, tune_smem_kb = 0;
+    // of unsplit / K-split launches, CTAs per SM the K split aims to fill
+    int tune_splits = 0, tune_smem_kb = 0, tune_split_smem_kb = 0, tune_ctas_per_sm = 0;
     std::unordered_map<std::string, CUtensorMap> maps;
     // 2-D map of a [rows][cols] bf16 matrix (leading dimension ld), box {64, box_rows};
     // plane_stride > 0: 3-D map over the hi plane and the lo plane plane_stride

@@ -30,6 +30,32 @@ long long launch_count() { return g_launches.load(std::memory_order_relaxed); }
 // embeddings + row metadata
 // ------------------------------------------------------------------------
 
+// x[0..H) = float(e[0..H)) with 16-byte loads, all issued before any store
+// (H a multiple of 64, rows 16-byte aligned).
+template <typename T>
+__device__ __forceinline__ void copy_embedding_row(const T *__restrict__ e, float *__restrict__ xr, int H) {
+    constexpr int EPC = 16 / (int)sizeof(T);
+    constexpr int NV = 4;
+    const uint4 *e4 = reinterpret_cast<const uint4 *>(e);
+    const int nch = H / EPC;
+    for (int base = 0; base < nch; base += NV * blockDim.x) {
+        uint4 raw[NV];
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int ch = base + threadIdx.x + u * blockDim.x;
+            raw[u] = ch < nch ? e4[ch] : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int ch = base + threadIdx.x + u * blockDim.x;
+            if (ch >= nch) continue;
+            const T *vals = reinterpret_cast<const T *>(&raw[u]);
+#pragma unroll
+            for (int k = 0; k < EPC; ++k) xr[ch * EPC + k] = to_f(vals[k]);
+        }
+    }
+}
+
 template <typename T>
 __global__ void embed_block_kernel(const T *__restrict__ emb, int H, SeqState *st,
                                    const int *__restrict__ active, int B, int is_draft,
@@ -45,9 +71,7 @@ __global__ void embed_block_kernel(const T *__restrict__ emb, int H, SeqState *s
     int tok;
     if (j == 0) tok = S.anchor;
     else tok = is_draft ? mask_id : drafts[i * (B - 1) + (j - 1)];
-    const T *e = emb + (size_t)tok * H;
-    float *xr = x + (size_t)r * H;
-    for (int c = threadIdx.x; c < H; c += blockDim.x) xr[c] = to_f(e[c]);
+    copy_embedding_row(emb + (size_t)tok * H, x + (size_t)r * H, H);
     if (threadIdx.x == 0) {
         RowMeta m;
         m.seq = s;
@@ -75,7 +99,9 @@ void launch_embed_block(const T *emb, int H, SeqState *st, const int *active, in
 }
 
 // Block rows as embed_block_kernel, plus the folded RMSNorm inputs of the first
-// projection: xg = bf16(x * g) and per-128-column-tile sums of squares.
+// projection: xg = x * g (two planes when lo != 0) and per-128-column-tile sums
+// of squares.  Each thread loads its 16-byte chunks of the embedding row
+// before using any of them, so a row costs one memory latency, not one per column.
 template <typename T>
 __global__ void embed_norm_kernel(const T *__restrict__ emb, int H, SeqState *st, const int *__restrict__ active, int B,
                                   int is_draft, const int *__restrict__ drafts, int mask_id, float *__restrict__ x,
@@ -83,33 +109,43 @@ __global__ void embed_norm_kernel(const T *__restrict__ emb, int H, SeqState *st
                                   int xg_ld, size_t lo, float *__restrict__ ssq, int ssq_ld) {
     pdl_trigger();
     pdl_wait();
-    __shared__ float red[8];
+    constexpr int EPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+    constexpr int CPT = 128 / EPC;            // chunks per 128-column tile (divides 32)
+    constexpr int NV = 4;                     // chunks in flight per thread
     const int r = blockIdx.x;
     const int i = r / B, j = r % B;
     const int s = active[i];
     const SeqState S = st[s];
     const int p = S.len;
     const int tok = j == 0 ? S.anchor : (is_draft ? mask_id : drafts[i * (B - 1) + (j - 1)]);
-    const T *e = emb + (size_t)tok * H;
-    for (int t0 = 0; t0 < H; t0 += 256) {
-        const int c = t0 + threadIdx.x;
-        float v = 0.f;
-        if (c < H) {
-            v = to_f(e[c]);
-            x[(size_t)r * H + c] = v;
-            st_act(xg, (size_t)r * xg_ld + c, lo, v * g[c]);
+    const uint4 *e4 = reinterpret_cast<const uint4 *>(emb + (size_t)tok * H);
+    const int nch = H / EPC;
+    for (int base = 0; base < nch; base += NV * blockDim.x) {
+        uint4 raw[NV];
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int ch = base + threadIdx.x + u * blockDim.x;
+            raw[u] = ch < nch ? e4[ch] : make_uint4(0, 0, 0, 0);
         }
-        float sq = warp_sum(v * v);
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
-        __syncthreads();
-        if (threadIdx.x < 2) {  // two 128-column tiles per pass
-            const int tile = t0 / 128 + threadIdx.x;
-            if (tile * 128 < H) {
-                const float* rr = red + 4 * threadIdx.x;
-                ssq[(size_t)tile * ssq_ld + r] = (rr[0] + rr[1]) + (rr[2] + rr[3]);
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int ch = base + threadIdx.x + u * blockDim.x;
+            const T *vals = reinterpret_cast<const T *>(&raw[u]);
+            float sq = 0.f;
+            if (ch < nch) {
+#pragma unroll
+                for (int k = 0; k < EPC; ++k) {
+                    const int col = ch * EPC + k;
+                    const float v = to_f(vals[k]);
+                    x[(size_t)r * H + col] = v;
+                    st_act(xg, (size_t)r * xg_ld + col, lo, v * g[col]);
+                    sq += v * v;
+                }
             }
+#pragma unroll
+            for (int o = CPT / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if (ch < nch && (threadIdx.x % CPT) == 0) ssq[(size_t)(ch / CPT) * ssq_ld + r] = sq;
         }
-        __syncthreads();
     }
     if (threadIdx.x == 0) {
         RowMeta m;
@@ -144,9 +180,7 @@ __global__ void embed_tokens_kernel(const T *__restrict__ emb, int H, const int 
     pdl_wait();
     const int r = blockIdx.x;
     const int tok = tokens[r];
-    const T *e = emb + (size_t)tok * H;
-    float *xr = x + (size_t)r * H;
-    for (int c = threadIdx.x; c < H; c += blockDim.x) xr[c] = to_f(e[c]);
+    copy_embedding_row(emb + (size_t)tok * H, x + (size_t)r * H, H);
     if (threadIdx.x == 0) {
         RowMeta m;
         m.seq = seq;
@@ -189,22 +223,56 @@ __global__ void rmsnorm_kernel(const float *__restrict__ x, int ldx, const float
                                int H, float eps, TO *__restrict__ out, int ldo, size_t lo) {
     pdl_trigger();
     pdl_wait();
+    // the row is held in registers (float4 chunks, all loads issued before any
+    // use); rows longer than NV * 4 * blockDim columns are re-read in a tail loop
+    constexpr int NV = 8;
     const int r = blockIdx.x;
-    const float *xr = x + (size_t)r * ldx;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x + (size_t)r * ldx);
+    const float4 *g4 = reinterpret_cast<const float4 *>(g);
+    const int H4 = H >> 2;
+    float4 v[NV];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int c = threadIdx.x + u * blockDim.x;
+        v[u] = c < H4 ? x4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float ss = 0.f;
-    for (int c = threadIdx.x; c < H; c += blockDim.x) ss += xr[c] * xr[c];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) ss += (v[u].x * v[u].x + v[u].y * v[u].y) + (v[u].z * v[u].z + v[u].w * v[u].w);
+    for (int c = threadIdx.x + NV * blockDim.x; c < H4; c += blockDim.x) {
+        const float4 t = x4[c];
+        ss += (t.x * t.x + t.y * t.y) + (t.z * t.z + t.w * t.w);
+    }
     __shared__ float red[32];
     ss = warp_sum(ss);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
     __syncthreads();
     if (threadIdx.x < 32) {
-        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-        v = warp_sum(v);
-        if (threadIdx.x == 0) red[0] = v;
+        float w = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+        w = warp_sum(w);
+        if (threadIdx.x == 0) red[0] = w;
     }
     __syncthreads();
     const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
-    for (int c = threadIdx.x; c < H; c += blockDim.x) st_act(out, (size_t)r * ldo + c, lo, xr[c] * inv * g[c]);
+    const size_t o0 = (size_t)r * ldo;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int c = threadIdx.x + u * blockDim.x;
+        if (c < H4) {
+            const float4 gg = g4[c];
+            st_act(out, o0 + 4 * c + 0, lo, v[u].x * inv * gg.x);
+            st_act(out, o0 + 4 * c + 1, lo, v[u].y * inv * gg.y);
+            st_act(out, o0 + 4 * c + 2, lo, v[u].z * inv * gg.z);
+            st_act(out, o0 + 4 * c + 3, lo, v[u].w * inv * gg.w);
+        }
+    }
+    for (int c = threadIdx.x + NV * blockDim.x; c < H4; c += blockDim.x) {
+        const float4 t = x4[c], gg = g4[c];
+        st_act(out, o0 + 4 * c + 0, lo, t.x * inv * gg.x);
+        st_act(out, o0 + 4 * c + 1, lo, t.y * inv * gg.y);
+        st_act(out, o0 + 4 * c + 2, lo, t.z * inv * gg.z);
+        st_act(out, o0 + 4 * c + 3, lo, t.w * inv * gg.w);
+    }
 }
 
 template <typename TO>

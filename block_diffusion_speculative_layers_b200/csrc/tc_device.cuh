@@ -71,6 +71,25 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// L2 policy for streamed weights: each weight byte is read once per decode
+// pass, so it is marked evict-first and does not push activations, K/V, the
+// per-row norm statistics or the kernels' own code out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// weight tile load with an L2 cache-policy hint
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+        "%4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
 // Two-plane activation tile: box {BK, rows, 2} of a 3-D map whose third
 // dimension steps from the hi plane to the lo plane; lands as [2][rows][BK].
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
@@ -144,28 +163,44 @@ __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(_
 // m0c .. m0c+nc-1) for weight row n_local of the tile.  Global loads of a
 // chunk are issued together before any use.
 // ---------------------------------------------------------------------------
-// Per-row RMSNorm scale of the chunk's rows (folded norm), computed by 16
-// threads into rsc[] and published with a named barrier.
-__device__ __forceinline__ void row_scales(const Epi<bf16> &e, int m0c, int nc, int M, float *rsc) {
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
-        const int j = threadIdx.x - 64, m = m0c + j;
-        float sc = 1.f;
-        if (e.rs_ssq && j < nc && m < M) {
-            float ss = 0.f;
-            for (int t = 0; t < e.rs_tiles; ++t) ss += e.rs_ssq[(size_t)t * e.rs_ld + m];
-            sc = 1.0f / sqrtf(ss * e.rs_inv_n + e.rs_eps);
+// Per-row RMSNorm scales of a tile's rows m_base .. m_base+rows-1 (folded
+// norm): 8 epilogue threads per row each sum every 8th per-tile sum of squares
+// (all loads issued together), combined by shuffles in a fixed order.  Runs
+// once per tile, before the accumulator is ready; the 128 epilogue threads
+// (64..191) all take part.
+constexpr int RS_MAX = 256;  // rows of one tile (TM <= 256)
+__device__ __forceinline__ void all_row_scales(const Epi<bf16> &e, int m_base, int rows, int M, float *rs) {
+    epi_bar();  // the previous tile's epilogue may still read rs
+    const int t = (int)threadIdx.x - 64;
+    const int part = t & 7, rr = t >> 3;
+    for (int r0 = 0; r0 < rows; r0 += 16) {
+        const int r = r0 + rr, m = m_base + r;
+        float a = 0.f;
+        if (r < rows && m < M) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int tile = part + 8 * u;
+                v[u] = tile < e.rs_tiles ? e.rs_ssq[(size_t)tile * e.rs_ld + m] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) a += v[u];
+            for (int tile = part + 64; tile < e.rs_tiles; tile += 8) a += e.rs_ssq[(size_t)tile * e.rs_ld + m];
         }
-        rsc[j] = sc;
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        a += __shfl_xor_sync(0xffffffffu, a, 2);
+        a += __shfl_xor_sync(0xffffffffu, a, 4);
+        if (part == 0 && r < rows) rs[r] = 1.0f / sqrtf(a * e.rs_inv_n + e.rs_eps);
     }
     epi_bar();
 }
 
 // y -> bf16(y * g_next) and the tile's per-row sum of squares (fixed reduction order).
 __device__ __forceinline__ void norm_outputs(const TcParams &p, const Epi<bf16> &e, int nt, int n, int q, int lane,
-                                             int m0c, int nc, const float *y, float2 *red) {
+                                             int m0c, int nc, const float *y, float2 *red, const float *gn_pre) {
     const int M = p.M;
     const bool nok = n < p.N;
-    const float gn = (nok && e.g_next) ? e.g_next[n] : 0.f;
+    const float gn = gn_pre ? *gn_pre : ((nok && e.g_next) ? e.g_next[n] : 0.f);
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
         const bool ok = nok && j < nc && m0c + j < M;
@@ -184,17 +219,86 @@ __device__ __forceinline__ void norm_outputs(const TcParams &p, const Epi<bf16> 
     epi_bar();
 }
 
+// Row metadata of a QKV chunk's columns (activation rows m0c..m0c+nc-1) into
+// smeta[]: aux = 0 block row, 1 context row whose K/V is written, -1 skip.
+__device__ __forceinline__ void qkv_fill_meta(const Epi<bf16> &e, int m0c, int nc, int M, RowMeta *smeta) {
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+        const int j = threadIdx.x - 64, m = m0c + j;
+        RowMeta mt;
+        mt.seq = mt.pos = mt.nk = 0;
+        mt.aux = -1;  // -1: skip this column
+        if (j < nc && m < M) {
+            if (m >= e.R_blk) {
+                mt = e.ctx_meta[m - e.R_blk];
+                mt.aux = mt.aux ? 1 : -1;
+            } else {
+                mt = e.meta[m];
+                mt.aux = 0;
+            }
+        }
+        smeta[j] = mt;
+    }
+    epi_bar();
+}
+
+// RoPE (cos, sin) of this thread's weight row for each column of the chunk.
+__device__ __forceinline__ void qkv_rope_factors(const Epi<bf16> &e, int cg, int N_ok, const RowMeta *smeta,
+                                                 float2 *cs) {
+    const int hd = e.hd, half = hd >> 1, qd = e.nq * hd, kd = e.nkv * hd;
+    const int d = cg % hd;
+    const int i = d < half ? d : d - half;
+    const bool rot = N_ok && cg < qd + kd;  // q and k rows are rotated
+#pragma unroll
+    for (int j = 0; j < CH; ++j)
+        cs[j] = rot && smeta[j].aux >= 0 ? e.rope[(size_t)smeta[j].pos * half + i] : make_float2(1.f, 0.f);
+}
+
+// Inputs of a chunk's fused epilogue that do not depend on the accumulator
+// (residual rows, tap rows, the next norm's gain; QKV row metadata and RoPE
+// factors).  They are loaded while the mainloop still streams, so that after
+// the last MMA the epilogue only computes and stores -- loads issued then would
+// queue behind the next projection's weight prefetch.
+struct EpiIn {
+    float xo[CH];
+    int trow[CH];
+    float gn;
+    float2 cs[CH];
+};
+
+template <int KIND>
+__device__ __forceinline__ void epi_prefetch(const TcParams &p, const Epi<bf16> &e, int nt, int n_local, int m0c,
+                                             int nc, EpiIn &in, RowMeta *smeta) {
+    const int M = p.M;
+    const int n = nt * 128 + n_local;
+    const bool nok = n < p.N;
+    if (KIND == EPI_RESID || KIND == EPI_NORMOUT) {
+        in.gn = (nok && e.g_next) ? e.g_next[n] : 0.f;
+        if (KIND == EPI_RESID) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+                const bool ok = nok && j < nc && m0c + j < M;
+                in.xo[j] = ok ? e.x[(size_t)(m0c + j) * p.N + n] : 0.f;
+                in.trow[j] = (ok && e.taps.n) ? e.meta[m0c + j].aux : 0;
+            }
+        }
+    } else if (KIND == EPI_QKV) {
+        qkv_fill_meta(e, m0c, nc, M, smeta);
+        qkv_rope_factors(e, e.col0 + n, nok, smeta, in.cs);
+    }
+}
+
 template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16> &e, int nt, int n_local, int q,
                                                int lane, int m0c, int nc, const float *vin, float *stg, float2 *red,
-                                               RowMeta *smeta, float *rsc) {
+                                               RowMeta *smeta, const float *rs, const EpiIn *pre = nullptr) {
+    // rs[j]: RMSNorm scale of row m0c + j (folded norm; see all_row_scales);
+    // pre: this chunk's inputs loaded by epi_prefetch (nullptr: load them here)
     const int M = p.M;
     float v[CH];
     if (KIND == EPI_QKV || KIND == EPI_SWIGLU || KIND == EPI_LOGITS || KIND == EPI_STORE) {
         if (e.rs_ssq) {
-            row_scales(e, m0c, nc, M, rsc);
 #pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = vin[j] * rsc[j];
+            for (int j = 0; j < CH; ++j) v[j] = vin[j] * rs[j];
         } else {
 #pragma unroll
             for (int j = 0; j < CH; ++j) v[j] = vin[j];
@@ -215,11 +319,19 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
         const bool nok = n < p.N;
         float xo[CH];
         int trow[CH];
+        if (pre) {
 #pragma unroll
-        for (int j = 0; j < CH; ++j) {
-            const bool ok = nok && j < nc && m0c + j < M;
-            xo[j] = ok ? e.x[(size_t)(m0c + j) * p.N + n] : 0.f;
-            trow[j] = (ok && e.taps.n) ? e.meta[m0c + j].aux : 0;
+            for (int j = 0; j < CH; ++j) {
+                xo[j] = pre->xo[j];
+                trow[j] = pre->trow[j];
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+                const bool ok = nok && j < nc && m0c + j < M;
+                xo[j] = ok ? e.x[(size_t)(m0c + j) * p.N + n] : 0.f;
+                trow[j] = (ok && e.taps.n) ? e.meta[m0c + j].aux : 0;
+            }
         }
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
@@ -230,9 +342,9 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             for (int t = 0; t < e.taps.n; ++t)
                 st_act(e.taps.base, (size_t)trow[j] * e.taps.ld + e.taps.col[t] + n, e.lo, nx);
         }
-        if (e.ssq_out) norm_outputs(p, e, nt, n, q, lane, m0c, nc, xo, red);
+        if (e.ssq_out) norm_outputs(p, e, nt, n, q, lane, m0c, nc, xo, red, pre ? &pre->gn : nullptr);
     } else if (KIND == EPI_NORMOUT) {
-        norm_outputs(p, e, nt, nt * 128 + n_local, q, lane, m0c, nc, v, red);
+        norm_outputs(p, e, nt, nt * 128 + n_local, q, lane, m0c, nc, v, red, pre ? &pre->gn : nullptr);
     } else if (KIND == EPI_LOGITS) {
         const int n = nt * 128 + n_local;
         const bool ok = n < p.N;
@@ -281,23 +393,8 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
     } else if (KIND == EPI_QKV) {
 #pragma unroll
         for (int j = 0; j < CH; ++j) stg[n_local * STG_LD + j] = v[j];
-        if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
-            const int j = threadIdx.x - 64, m = m0c + j;
-            RowMeta mt;
-            mt.seq = mt.pos = mt.nk = 0;
-            mt.aux = -1;  // -1: skip this column
-            if (j < nc && m < M) {
-                if (m >= e.R_blk) {
-                    mt = e.ctx_meta[m - e.R_blk];
-                    mt.aux = mt.aux ? 1 : -1;
-                } else {
-                    mt = e.meta[m];
-                    mt.aux = 0;
-                }
-            }
-            smeta[j] = mt;
-        }
-        epi_bar();
+        if (pre) epi_bar();  // smeta is already filled; stg must be complete before partners are read
+        else qkv_fill_meta(e, m0c, nc, M, smeta);
         const int hd = e.hd, half = hd >> 1;
         const int qd = e.nq * hd, kd = e.nkv * hd;
         const int cg = e.col0 + nt * 128 + n_local;  // row of [Wq; Wk; Wv]
@@ -305,12 +402,14 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             const int head_base = (cg / hd) * hd;
             const int d = cg - head_base;
             const int partner = n_local + (d < half ? half : -half);
-            const int i = d < half ? d : d - half;
             const bool is_q = cg < qd, is_k = !is_q && cg < qd + kd;
             float2 cs[CH];
+            if (pre) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j)
-                cs[j] = (is_q || is_k) && smeta[j].aux >= 0 ? e.rope[(size_t)smeta[j].pos * half + i] : make_float2(1.f, 0.f);
+                for (int j = 0; j < CH; ++j) cs[j] = pre->cs[j];
+            } else {
+                qkv_rope_factors(e, cg, true, smeta, cs);
+            }
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
                 const RowMeta mt = smeta[j];
@@ -343,6 +442,13 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// store v to the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ void st_cluster_f32(float *local, uint32_t rank, float v) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 // generic address of the same shared-memory location in CTA `rank` of the cluster
