@@ -17,6 +17,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cstdio>
 #include <cstring>
 
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int n_local = q * 32 + lane;
         // K split: CTA `rank` of the cluster reduces and finishes columns [c_begin, c_end)
         const int rank = split ? (int)cluster_rank() : 0;
-        const int cpr = split ? (TM + S - 1) / S : TM;
+        const int cpr = split ? split_cols(TM, S) : TM;
         const int c_begin = split ? min(TM, rank * cpr) : 0;
         const int c_end = split ? min(TM, c_begin + cpr) : TM;
         int lt = 0, rs_mt = -1;
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(NT, 1)
                 rs_mt = mt;
             }
             // inputs of this CTA's first epilogue chunk, while the mainloop streams
-            if (c_end > c_begin) epi_prefetch<KIND>(p, e, nt, n_local, mt * TM + c_begin, min(CH, c_end - c_begin), pre, smeta);
+            if (c_end > c_begin) epi_prefetch<KIND, CH>(p, e, nt, n_local, mt * TM + c_begin, min(CH, c_end - c_begin), pre, smeta);
             const uint32_t trow = tmem + (uint32_t)(b * NC1) + ((uint32_t)(q * 32) << 16);
             const bool ok = mbar_wait(&acc_full[b], (lt >> 1) & 1, p.err) && nk > 0;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -227,19 +228,18 @@ __global__ void __launch_bounds__(NT, 1)
                 }
             } else {
                 // push this CTA's partial columns into the receive buffer of the CTA that
-                // finishes them: recv[source rank][weight row][column - owner's c_begin]
+                // finishes them: recv[source rank][weight row][column - owner's c_begin],
+                // four columns (one owner, cpr being a multiple of 4) per store
                 for (int c = 0; c < TM; c += CH) {
                     if (ok) acc_ld16(trow, c, lo_col, v);
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) {
-                        const int col = c + j, owner = col / cpr;
-                        if (col < TM) {
-                            float *dst = recv + ((size_t)rank * 128 + n_local) * cpr + (col - owner * cpr);
-                            st_cluster_f32(dst, (uint32_t)owner, v[j]);
-                        }
+                    for (int g = 0; g < CH / 4; ++g) {
+                        const int col = c + 4 * g, owner = col / cpr;
+                        float *dst = recv + ((size_t)rank * 128 + n_local) * cpr + (col - owner * cpr);
+                        st_cluster_v4(dst, (uint32_t)owner, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
                     }
                 }
             }
@@ -255,22 +255,29 @@ __global__ void __launch_bounds__(NT, 1)
             const int n_local = q * 32 + lane;
             const int nt = blockIdx.x, mt = blockIdx.y;
             const int rank = (int)cluster_rank();
-            const int cpr = (TM + S - 1) / S;
+            const int cpr = split_cols(TM, S);
             const int c_begin = min(TM, rank * cpr), c_end = min(TM, c_begin + cpr);
-            for (int c = c_begin; c < c_end; c += CH) {
-                const int nc = min(CH, c_end - c);
-                float v[CH];
+            // finish the owned columns with an epilogue no wider than needed
+            auto finish = [&](auto width) {
+                constexpr int W = decltype(width)::value;
+                for (int c = c_begin; c < c_end; c += W) {
+                    const int nc = min(W, c_end - c);
+                    float v[CH];
 #pragma unroll
-                for (int j = 0; j < CH; ++j) v[j] = 0.f;
-                for (int s2 = 0; s2 < S; ++s2) {  // in rank order: identical results run to run
-                    const float *src = recv + ((size_t)s2 * 128 + n_local) * cpr + (c - c_begin);
+                    for (int j = 0; j < CH; ++j) v[j] = 0.f;
+                    for (int s2 = 0; s2 < S; ++s2) {  // in rank order: identical results run to run
+                        const float *src = recv + ((size_t)s2 * 128 + n_local) * cpr + (c - c_begin);
 #pragma unroll
-                    for (int j = 0; j < CH; ++j)
-                        if (j < nc) v[j] += src[j];
+                        for (int j = 0; j < W; ++j)
+                            if (j < nc) v[j] += src[j];
+                    }
+                    epilogue_chunk<KIND, W>(p, e, nt, n_local, q, lane, mt * TM + c, nc, v, stg, red, smeta, rsc + c,
+                                            c == c_begin ? &pre : nullptr);
                 }
-                epilogue_chunk<KIND>(p, e, nt, n_local, q, lane, mt * TM + c, nc, v, stg, red, smeta, rsc + c,
-                                     c == c_begin ? &pre : nullptr);
-            }
+            };
+            if (cpr <= 4) finish(std::integral_constant<int, 4>{});
+            else if (cpr <= 8) finish(std::integral_constant<int, 8>{});
+            else finish(std::integral_constant<int, CH>{});
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -474,7 +481,7 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
     }
     if (TM > 64) splits = 1;  // keeps the split-K receive buffer (S x 128 x TM/S floats) small
     // split-K receive buffer [S][128][ceil(TM/S)] floats, placed after the fixed area
-    const int recv_bytes = splits > 1 ? splits * 128 * ((TM + splits - 1) / splits) * 4 + 64 : 0;
+    const int recv_bytes = splits > 1 ? splits * 128 * tc::split_cols(TM, splits) * 4 + 64 : 0;
     int budget = splits > 1 ? 110 * 1024 : (TM <= 64 ? 112 * 1024 : 200 * 1024);
     if (splits > 1 && tune_split_smem_kb > 0) budget = tune_split_smem_kb * 1024;
     if (splits == 1 && tune_smem_kb > 0) budget = tune_smem_kb * 1024;

@@ -196,13 +196,14 @@ __device__ __forceinline__ void all_row_scales(const Epi<bf16> &e, int m_base, i
 }
 
 // y -> bf16(y * g_next) and the tile's per-row sum of squares (fixed reduction order).
+template <int W>
 __device__ __forceinline__ void norm_outputs(const TcParams &p, const Epi<bf16> &e, int nt, int n, int q, int lane,
                                              int m0c, int nc, const float *y, float2 *red, const float *gn_pre) {
     const int M = p.M;
     const bool nok = n < p.N;
     const float gn = gn_pre ? *gn_pre : ((nok && e.g_next) ? e.g_next[n] : 0.f);
 #pragma unroll
-    for (int j = 0; j < CH; ++j) {
+    for (int j = 0; j < W; ++j) {
         const bool ok = nok && j < nc && m0c + j < M;
         if (ok && e.xg) st_act(e.xg, (size_t)(m0c + j) * e.xg_ld + n, e.lo, y[j] * gn);
         float sq = ok ? y[j] * y[j] : 0.f;
@@ -211,7 +212,7 @@ __device__ __forceinline__ void norm_outputs(const TcParams &p, const Epi<bf16> 
         if (lane == 0) red[q * CH + j].x = sq;
     }
     epi_bar();
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + W) {
         const int j = threadIdx.x - 64, m = m0c + j;
         if (j < nc && m < M && e.ssq_out)
             e.ssq_out[(size_t)nt * e.ssq_ld + m] = (red[j].x + red[CH + j].x) + (red[2 * CH + j].x + red[3 * CH + j].x);
@@ -242,6 +243,7 @@ __device__ __forceinline__ void qkv_fill_meta(const Epi<bf16> &e, int m0c, int n
 }
 
 // RoPE (cos, sin) of this thread's weight row for each column of the chunk.
+template <int W>
 __device__ __forceinline__ void qkv_rope_factors(const Epi<bf16> &e, int cg, int N_ok, const RowMeta *smeta,
                                                  float2 *cs) {
     const int hd = e.hd, half = hd >> 1, qd = e.nq * hd, kd = e.nkv * hd;
@@ -249,7 +251,7 @@ __device__ __forceinline__ void qkv_rope_factors(const Epi<bf16> &e, int cg, int
     const int i = d < half ? d : d - half;
     const bool rot = N_ok && cg < qd + kd;  // q and k rows are rotated
 #pragma unroll
-    for (int j = 0; j < CH; ++j)
+    for (int j = 0; j < W; ++j)
         cs[j] = rot && smeta[j].aux >= 0 ? e.rope[(size_t)smeta[j].pos * half + i] : make_float2(1.f, 0.f);
 }
 
@@ -265,7 +267,7 @@ struct EpiIn {
     float2 cs[CH];
 };
 
-template <int KIND>
+template <int KIND, int W>
 __device__ __forceinline__ void epi_prefetch(const TcParams &p, const Epi<bf16> &e, int nt, int n_local, int m0c,
                                              int nc, EpiIn &in, RowMeta *smeta) {
     const int M = p.M;
@@ -275,7 +277,7 @@ __device__ __forceinline__ void epi_prefetch(const TcParams &p, const Epi<bf16> 
         in.gn = (nok && e.g_next) ? e.g_next[n] : 0.f;
         if (KIND == EPI_RESID) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) {
+            for (int j = 0; j < W; ++j) {
                 const bool ok = nok && j < nc && m0c + j < M;
                 in.xo[j] = ok ? e.x[(size_t)(m0c + j) * p.N + n] : 0.f;
                 in.trow[j] = (ok && e.taps.n) ? e.meta[m0c + j].aux : 0;
@@ -283,11 +285,14 @@ __device__ __forceinline__ void epi_prefetch(const TcParams &p, const Epi<bf16> 
         }
     } else if (KIND == EPI_QKV) {
         qkv_fill_meta(e, m0c, nc, M, smeta);
-        qkv_rope_factors(e, e.col0 + n, nok, smeta, in.cs);
+        qkv_rope_factors<W>(e, e.col0 + n, nok, smeta, in.cs);
     }
 }
 
-template <int KIND>
+// W: columns the chunk can hold (4, 8 or 16).  The epilogue runs once per CTA
+// and launch, so its code is fetched cold each time; K-split CTAs finishing only
+// a few columns use a narrow instantiation to keep that code short.
+template <int KIND, int W = CH>
 __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16> &e, int nt, int n_local, int q,
                                                int lane, int m0c, int nc, const float *vin, float *stg, float2 *red,
                                                RowMeta *smeta, const float *rs, const EpiIn *pre = nullptr) {
@@ -298,20 +303,20 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
     if (KIND == EPI_QKV || KIND == EPI_SWIGLU || KIND == EPI_LOGITS || KIND == EPI_STORE) {
         if (e.rs_ssq) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = vin[j] * rs[j];
+            for (int j = 0; j < W; ++j) v[j] = vin[j] * rs[j];
         } else {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = vin[j];
+            for (int j = 0; j < W; ++j) v[j] = vin[j];
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < CH; ++j) v[j] = vin[j];
+        for (int j = 0; j < W; ++j) v[j] = vin[j];
     }
     if (KIND == EPI_STORE) {
         const int n = nt * 128 + n_local;
         if (n < p.N) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j)
+            for (int j = 0; j < W; ++j)
                 if (j < nc && m0c + j < M) e.Y[(size_t)(m0c + j) * e.ldy + n] = v[j];
         }
     } else if (KIND == EPI_RESID) {
@@ -321,20 +326,20 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
         int trow[CH];
         if (pre) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) {
+            for (int j = 0; j < W; ++j) {
                 xo[j] = pre->xo[j];
                 trow[j] = pre->trow[j];
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) {
+            for (int j = 0; j < W; ++j) {
                 const bool ok = nok && j < nc && m0c + j < M;
                 xo[j] = ok ? e.x[(size_t)(m0c + j) * p.N + n] : 0.f;
                 trow[j] = (ok && e.taps.n) ? e.meta[m0c + j].aux : 0;
             }
         }
 #pragma unroll
-        for (int j = 0; j < CH; ++j) {
+        for (int j = 0; j < W; ++j) {
             if (!(nok && j < nc && m0c + j < M)) continue;
             const float nx = xo[j] + v[j];
             xo[j] = nx;
@@ -342,14 +347,14 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             for (int t = 0; t < e.taps.n; ++t)
                 st_act(e.taps.base, (size_t)trow[j] * e.taps.ld + e.taps.col[t] + n, e.lo, nx);
         }
-        if (e.ssq_out) norm_outputs(p, e, nt, n, q, lane, m0c, nc, xo, red, pre ? &pre->gn : nullptr);
+        if (e.ssq_out) norm_outputs<W>(p, e, nt, n, q, lane, m0c, nc, xo, red, pre ? &pre->gn : nullptr);
     } else if (KIND == EPI_NORMOUT) {
-        norm_outputs(p, e, nt, nt * 128 + n_local, q, lane, m0c, nc, v, red, pre ? &pre->gn : nullptr);
+        norm_outputs<W>(p, e, nt, nt * 128 + n_local, q, lane, m0c, nc, v, red, pre ? &pre->gn : nullptr);
     } else if (KIND == EPI_LOGITS) {
         const int n = nt * 128 + n_local;
         const bool ok = n < p.N;
 #pragma unroll
-        for (int j = 0; j < CH; ++j) {
+        for (int j = 0; j < W; ++j) {
             const int m = m0c + j;
             const bool col = j < nc && m < M;
             if (p.keep_logits && ok && col) e.Y[(size_t)m * e.ldy + n] = v[j];
@@ -364,7 +369,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             if (lane == 0) red[q * CH + j] = make_float2(bv, __int_as_float(bi));
         }
         epi_bar();
-        if (threadIdx.x >= 64 && threadIdx.x < 64 + CH) {
+        if (threadIdx.x >= 64 && threadIdx.x < 64 + W) {
             const int j = threadIdx.x - 64;
             const int m = m0c + j;
             float bv = red[j].x;
@@ -375,13 +380,13 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
         epi_bar();
     } else if (KIND == EPI_SWIGLU) {
 #pragma unroll
-        for (int j = 0; j < CH; ++j) stg[n_local * STG_LD + j] = v[j];
+        for (int j = 0; j < W; ++j) stg[n_local * STG_LD + j] = v[j];
         epi_bar();
         if (n_local < 64) {
             const int f = nt * 64 + n_local;
             if (f < p.swiglu_F) {
 #pragma unroll
-                for (int j = 0; j < CH; ++j) {
+                for (int j = 0; j < W; ++j) {
                     const int m = m0c + j;
                     if (j >= nc || m >= M) break;
                     const float up = stg[(n_local + 64) * STG_LD + j];
@@ -392,7 +397,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
         epi_bar();
     } else if (KIND == EPI_QKV) {
 #pragma unroll
-        for (int j = 0; j < CH; ++j) stg[n_local * STG_LD + j] = v[j];
+        for (int j = 0; j < W; ++j) stg[n_local * STG_LD + j] = v[j];
         if (pre) epi_bar();  // smeta is already filled; stg must be complete before partners are read
         else qkv_fill_meta(e, m0c, nc, M, smeta);
         const int hd = e.hd, half = hd >> 1;
@@ -406,12 +411,12 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             float2 cs[CH];
             if (pre) {
 #pragma unroll
-                for (int j = 0; j < CH; ++j) cs[j] = pre->cs[j];
+                for (int j = 0; j < W; ++j) cs[j] = pre->cs[j];
             } else {
-                qkv_rope_factors(e, cg, true, smeta, cs);
+                qkv_rope_factors<W>(e, cg, true, smeta, cs);
             }
 #pragma unroll
-            for (int j = 0; j < CH; ++j) {
+            for (int j = 0; j < W; ++j) {
                 const RowMeta mt = smeta[j];
                 if (mt.aux < 0) continue;          // padding column or uncommitted context row
                 const bool ctx = mt.aux == 1;
@@ -450,6 +455,17 @@ __device__ __forceinline__ void st_cluster_f32(float *local, uint32_t rank, floa
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
+
+// store 4 floats (16-byte aligned) to the same shared-memory location in CTA `rank`
+__device__ __forceinline__ void st_cluster_v4(float *local, uint32_t rank, float a, float b, float c, float d) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// columns of a K-split tile finished by each CTA of the cluster (a multiple of 4)
+__host__ __device__ constexpr int split_cols(int tm, int s) { return ((tm + s - 1) / s + 3) / 4 * 4; }
 
 // generic address of the same shared-memory location in CTA `rank` of the cluster
 __device__ __forceinline__ const float *peer_ptr(const float *p, uint32_t rank) {
