@@ -291,17 +291,32 @@ def main():
         need = min(need, max_len - cfg.prompt_len - B)
         ar_out, ar_ms = ctx.generate_ar(prompts, need)
         ar_tps = b * (need - 1) / (ar_ms / 1000.0) if ar_ms > 0 else None
+        # The one-row greedy decode and the block verify round differently; at a
+        # near-tie they can pick different tokens, after which the script no
+        # longer matches the verify's own continuation.  Re-derive the script
+        # from what a scripted full-block run commits until it is self-consistent.
+        script = ar_out
+        ctx.set_draft_mode(dfl.DFLASH_DRAFT_SCRIPT, B)
+        for _ in range(5):
+            for i in range(b):
+                ctx.set_script(i, script[i])
+            got, _st = ctx.generate(prompts, need)
+            same = bool((got == script[:, :got.shape[1]]).all())
+            script = got
+            if same:
+                break
         for tau in taus:
             if tau < 1 or tau > B:
                 continue
             for i in range(b):
-                ctx.set_script(i, ar_out[i])
+                ctx.set_script(i, script[i])
             ctx.set_draft_mode(dfl.DFLASH_DRAFT_SCRIPT, tau)
             prefill_all()
             ctx.decode_iters(b, args.warmup)
             k = max(1, min(args.steps, (need - args.warmup * tau) // max(tau, 1) - 2))
             fms, fst, _ = timed_iters(k)
-            forced[str(tau)] = {"tokens_per_s": b * 0 + fst.tokens / (fms / 1000.0), "mean_tau": fst.mean_tau,
+            forced[str(tau)] = {"tokens_per_s": fst.tokens / (fms / 1000.0), "mean_tau": fst.mean_tau,
+                                "tokens_per_s_at_tau": b * tau * k / (fms / 1000.0),
                                 "us_per_iter": fms * 1000.0 / k, "iters": k}
             log(f"[rank {rank}] forced tau={tau}: {forced[str(tau)]}")
         ctx.set_draft_mode(dfl.DFLASH_DRAFT_MODEL, 1)

@@ -80,6 +80,11 @@ __device__ __forceinline__ uint32_t cluster_rank() {
     return r;
 }
 
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -90,11 +95,27 @@ __device__ __forceinline__ const float *peer_ptr(const float *p, uint32_t rank) 
     return reinterpret_cast<const float *>(out);
 }
 
-// The n_splits CTAs of one (query tile, kv head) form a cluster along z.  Each
-// takes an equal share of the visible keys (chunk sized on the device from the
-// tile's key count), keeps an unnormalised partial (o, running max, running
-// sum) in shared memory, and after a cluster barrier combines a slice of the
-// (head, row) pairs over all CTAs of the cluster in rank order.
+// store 2 floats (8-byte aligned) to the same shared-memory location in CTA `rank`
+__device__ __forceinline__ void st_cluster_v2(float *local, uint32_t rank, float a, float b) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(ra), "f"(a), "f"(b) : "memory");
+}
+
+__device__ __forceinline__ void group_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// One CTA serves one (query tile, kv head, KV split); the n_splits CTAs of a
+// (tile, kv head) form a cluster along z.  A CTA's warps are G key groups of
+// `grp` warps, one warp per q head of the kv head (GQA): key group g takes key
+// tiles g, g+G, ... of the split's share, each tile loaded once into the
+// group's own buffer and read by all its heads.  Every warp ends with an
+// unnormalised partial (o, running max, running sum) for its head and rows;
+// it pushes that partial into the shared memory of the CTA that finishes the
+// (head, row) pair ("owner"), so after one cluster barrier each CTA combines
+// its pairs from local memory over all n_splits * G partials in a fixed order
+// (identical results run to run).
 //
 // SPLIT: q, K, V (and the output) are two-plane activations (hi at p, lo at
 // p + lo).  Each product then takes three bf16 MMAs, hi*hi + lo*hi + hi*lo
@@ -104,39 +125,46 @@ template <int HD, bool SPLIT>
 __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ q, int ldq, const bf16 *__restrict__ kc,
                                                        const bf16 *__restrict__ vc, const RowMeta *__restrict__ meta,
                                                        int R, int rows_per_tile, int nq, int nkv, int max_len,
-                                                       int n_splits, float scale_log2, bf16 *__restrict__ out, int ldo,
-                                                       size_t lo) {
-    constexpr int LDS = HD + 8;  // padded smem row (bf16 elements)
-    constexpr int OLD = HD + 4;  // partial-output row stride (floats)
+                                                       int n_splits, int G, float scale_log2, bf16 *__restrict__ out,
+                                                       int ldo, size_t lo) {
+    constexpr int LDS = HD + 8;                 // padded smem row (bf16 elements)
+    constexpr int NPL = SPLIT ? 4 : 2;          // planes per tile buffer: K, V (+ K lo, V lo)
+    constexpr int PLANE = KB * LDS;             // elements of one plane of a tile buffer
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    bf16 *Ks = reinterpret_cast<bf16 *>(smem_raw);  // [2][KB][LDS]
-    bf16 *Vs = Ks + 2 * KB * LDS;                    // [2][KB][LDS]
-    bf16 *Kl = Vs + 2 * KB * LDS;                    // SPLIT: lo planes [2][KB][LDS] each
-    bf16 *Vl = Kl + 2 * KB * LDS;
-    float *Op = reinterpret_cast<float *>(smem_raw); // [grp][16][OLD], reuses K/V tiles after the loop
-    __shared__ float MLs[8 * 16 * 2];                // [grp][16][(max, sum)]
 
+    // every CTA of the cluster has started before any CTA stores into another's
+    // shared memory: arrive now, wait before the first push
+    cluster_arrive_relaxed();
     pdl_trigger();
     pdl_wait();
     const int tile = blockIdx.x, kvh = blockIdx.y, split = blockIdx.z;
     const int grp = nq / nkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nthr = blockDim.x;
+    const int hw = warp % grp, g = warp / grp;  // head within the kv group, key group
+    const int gthr = 32 * grp;                  // threads of one key group
+    const int gt = threadIdx.x - g * gthr;
     const int r0 = tile * rows_per_tile;
     const int nrows = min(rows_per_tile, R - r0);
     const int seq = meta[r0].seq;
-    const int h = kvh * grp + warp;
+    const int h = kvh * grp + hw;
+    const int pairs = grp * 16, ppc = (pairs + n_splits - 1) / n_splits;  // (head, row) pairs per owner
+    const int nsrc = n_splits * G;                                       // partials per pair
+    bf16 *tb = reinterpret_cast<bf16 *>(smem_raw) + (size_t)g * NPL * PLANE;
+    float *recv_o = reinterpret_cast<float *>(smem_raw + (size_t)G * NPL * PLANE * sizeof(bf16));  // [nsrc][ppc][HD]
+    float *recv_ml = recv_o + (size_t)nsrc * ppc * HD;                                               // [nsrc][ppc][2]
 
     // visible keys of the two rows this thread's accumulators cover
     const int ra = lane >> 2, rb = ra + 8;
     const int nk_a = ra < nrows ? meta[r0 + ra].nk : 0;
     const int nk_b = rb < nrows ? meta[r0 + rb].nk : 0;
-    int nk_max = 0;
-    for (int i = 0; i < nrows; ++i) nk_max = max(nk_max, meta[r0 + i].nk);
-    // equal share of the visible keys for each split, in whole 64-key tiles
-    const int chunk = ((nk_max + n_splits - 1) / n_splits + KB - 1) / KB * KB;
-    const int kb = split * chunk;
-    const int ke = min(kb + chunk, nk_max);
+    // longest visible key range of the tile's rows (nrows <= 16), the same in every lane
+    int nk_max = lane < nrows ? meta[r0 + lane].nk : 0;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) nk_max = max(nk_max, __shfl_xor_sync(0xffffffffu, nk_max, o2));
+    // this split's key tiles [t0, t1); key group g takes t0 + g, t0 + g + G, ...
+    const int ntk = (nk_max + KB - 1) / KB;
+    const int per = (ntk + n_splits - 1) / n_splits;
+    const int t0 = min(ntk, split * per), t1 = min(ntk, t0 + per);
 
     const size_t head_off = ((size_t)seq * nkv + kvh) * (size_t)max_len * HD;
     const bf16 *Kg = kc + head_off;
@@ -166,39 +194,30 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
     for (int j = 0; j < HD / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
 
-    auto load_tile = [&](int buf, int j0) {
-        constexpr int CPR = HD / 8;  // 16-byte chunks per row
-        for (int e = threadIdx.x; e < KB * CPR; e += nthr) {
-            const int r = e / CPR, c = (e % CPR) * 8;
-            const int key = j0 + r;
-            const bool valid = key < ke;
-            const size_t off = (size_t)(valid ? key : 0) * HD + c;
-            cp_async16(Ks + ((size_t)buf * KB + r) * LDS + c, Kg + off, valid);
-            cp_async16(Vs + ((size_t)buf * KB + r) * LDS + c, Vg + off, valid);
-            if constexpr (SPLIT) {
-                cp_async16(Kl + ((size_t)buf * KB + r) * LDS + c, Kg + lo + off, valid);
-                cp_async16(Vl + ((size_t)buf * KB + r) * LDS + c, Vg + lo + off, valid);
+    const bf16 *Kt = tb, *Vt = tb + PLANE, *Klt = tb + 2 * PLANE, *Vlt = tb + 3 * PLANE;
+#pragma unroll 1
+    for (int tt = t0 + g; tt < t1; tt += G) {
+        const int j0 = tt * KB;
+        {
+            constexpr int CPR = HD / 8;  // 16-byte chunks per row
+            bf16 *Kw = tb, *Vw = tb + PLANE;
+#pragma unroll 1
+            for (int e = gt; e < KB * CPR; e += gthr) {
+                const int r = e / CPR, c = (e % CPR) * 8;
+                const int key = j0 + r;
+                const bool valid = key < nk_max;
+                const size_t off = (size_t)(valid ? key : 0) * HD + c;
+                cp_async16(Kw + r * LDS + c, Kg + off, valid);
+                cp_async16(Vw + r * LDS + c, Vg + off, valid);
+                if constexpr (SPLIT) {
+                    cp_async16(Kw + 2 * PLANE + r * LDS + c, Kg + lo + off, valid);
+                    cp_async16(Vw + 2 * PLANE + r * LDS + c, Vg + lo + off, valid);
+                }
             }
-        }
-        cp_commit();
-    };
-
-    const int n_blocks = ke > kb ? (ke - kb + KB - 1) / KB : 0;
-    if (n_blocks > 0) load_tile(0, kb);
-    for (int bi = 0; bi < n_blocks; ++bi) {
-        const int buf = bi & 1;
-        const int j0 = kb + bi * KB;
-        if (bi + 1 < n_blocks) {
-            load_tile(buf ^ 1, j0 + KB);
-            cp_wait<1>();
-        } else {
+            cp_commit();
             cp_wait<0>();
         }
-        __syncthreads();
-        const bf16 *Kt = Ks + (size_t)buf * KB * LDS;
-        const bf16 *Vt = Vs + (size_t)buf * KB * LDS;
-        const bf16 *Klt = Kl + (size_t)buf * KB * LDS;
-        const bf16 *Vlt = Vl + (size_t)buf * KB * LDS;
+        group_bar(1 + g, gthr);
         // S = Q K^T over 64 keys: 8 n-tiles of 8 keys
         float sc[KB / 8][4];
 #pragma unroll
@@ -297,7 +316,7 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
                 }
             }
         }
-        __syncthreads();
+        group_bar(1 + g, gthr);  // the buffer is reloaded by the next tile
     }
     // row sums across the quad
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
@@ -305,86 +324,54 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
 
-    if (n_splits == 1) {
-        const float ia = l_a > 0.f ? 1.f / l_a : 0.f, ib = l_b > 0.f ? 1.f / l_b : 0.f;
+    // ---- push this warp's partial to the owners of its (head, row) pairs ----
+    cluster_wait();
+    const int src = split * G + g;
 #pragma unroll
-        for (int j = 0; j < HD / 8; ++j) {
-            const int d = j * 8 + (lane & 3) * 2;
-            if (ra < nrows) store_pair(out + (size_t)(r0 + ra) * ldo + h * HD + d, lo, o[j][0] * ia, o[j][1] * ia);
-            if (rb < nrows) store_pair(out + (size_t)(r0 + rb) * ldo + h * HD + d, lo, o[j][2] * ib, o[j][3] * ib);
-        }
-        return;
-    }
-    // ---- cluster combine of the splits ----
-    __syncthreads();  // K/V tiles are no longer read: reuse them for the partial outputs
-    {
-        float *ow = Op + (size_t)warp * 16 * OLD;
+    for (int half = 0; half < 2; ++half) {
+        const int row = half ? rb : ra;
+        if (row >= nrows) continue;
+        const int pair = hw * 16 + row, owner = pair / ppc, pl = pair - owner * ppc;
+        float *dst = recv_o + ((size_t)src * ppc + pl) * HD + (lane & 3) * 2;
 #pragma unroll
-        for (int j = 0; j < HD / 8; ++j) {
-            const int d = j * 8 + (lane & 3) * 2;
-            ow[ra * OLD + d] = o[j][0];
-            ow[ra * OLD + d + 1] = o[j][1];
-            ow[rb * OLD + d] = o[j][2];
-            ow[rb * OLD + d + 1] = o[j][3];
-        }
-        if ((lane & 3) == 0) {
-            MLs[(warp * 16 + ra) * 2] = m_a;
-            MLs[(warp * 16 + ra) * 2 + 1] = l_a;
-            MLs[(warp * 16 + rb) * 2] = m_b;
-            MLs[(warp * 16 + rb) * 2 + 1] = l_b;
-        }
+        for (int j = 0; j < HD / 8; ++j)
+            st_cluster_v2(dst + j * 8, (uint32_t)owner, o[j][2 * half], o[j][2 * half + 1]);
+        if ((lane & 3) == 0)
+            st_cluster_v2(recv_ml + ((size_t)src * ppc + pl) * 2, (uint32_t)owner, half ? m_b : m_a, half ? l_b : l_a);
     }
     __syncwarp();
-    cluster_sync_all();
-    {
-        const int rank = (int)cluster_rank();
-        const int pairs = grp * 16;                       // (head, row) pairs of the tile
-        const int per = (pairs + n_splits - 1) / n_splits;
-        const int p0 = rank * per, p1 = min(pairs, p0 + per);
-        constexpr int DPT = 8;                             // output elements per thread
-        const int tpp = HD / DPT;                          // threads per pair
-        for (int e = threadIdx.x; e < (p1 - p0) * tpp; e += nthr) {
-            const int pr = p0 + e / tpp, d0 = (e % tpp) * DPT;
-            const int hh = pr / 16, row = pr % 16;
-            if (row >= nrows) continue;
-            float ms[8], ls[8];
-            float mstar = -INFINITY;
-#pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) {
-                if (s2 < n_splits) {
-                    const float *ml = peer_ptr(MLs, (uint32_t)s2);
-                    ms[s2] = ml[(hh * 16 + row) * 2];
-                    ls[s2] = ml[(hh * 16 + row) * 2 + 1];
-                    mstar = fmaxf(mstar, ms[s2]);
-                } else {
-                    ms[s2] = -INFINITY;
-                    ls[s2] = 0.f;
-                }
-            }
-            const float mu = mstar == -INFINITY ? 0.f : mstar;
-            float acc[DPT];
-#pragma unroll
-            for (int t = 0; t < DPT; ++t) acc[t] = 0.f;
-            float lsum = 0.f;
-#pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) {
-                if (s2 >= n_splits) break;
-                const float w = exp2f(ms[s2] - mu);
-                lsum += ls[s2] * w;
-                const float *src = peer_ptr(Op, (uint32_t)s2) + ((size_t)hh * 16 + row) * OLD + d0;
-                const float4 a = *reinterpret_cast<const float4 *>(src);
-                const float4 b = *reinterpret_cast<const float4 *>(src + 4);
-                acc[0] += a.x * w; acc[1] += a.y * w; acc[2] += a.z * w; acc[3] += a.w * w;
-                acc[4] += b.x * w; acc[5] += b.y * w; acc[6] += b.z * w; acc[7] += b.w * w;
-            }
-            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-            const int hq = kvh * grp + hh;
-            bf16 *dst = out + (size_t)(r0 + row) * ldo + hq * HD + d0;
-#pragma unroll
-            for (int t = 0; t < DPT; t += 2) store_pair(dst + t, lo, acc[t] * inv, acc[t + 1] * inv);
+    cluster_sync_all();  // (a 1-CTA cluster when n_splits == 1)
+
+    // ---- combine the owned pairs over all partials, in source order ----
+    const int p0 = split * ppc, p1 = min(pairs, p0 + ppc);
+    constexpr int D4 = HD / 4;
+#pragma unroll 1
+    for (int e = threadIdx.x; e < (p1 - p0) * D4; e += blockDim.x) {
+        const int pl = e / D4, d0 = (e % D4) * 4;
+        const int pair = p0 + pl, hh = pair / 16, row = pair % 16;
+        if (row >= nrows) continue;
+        float mstar = -INFINITY;
+#pragma unroll 1
+        for (int s2 = 0; s2 < nsrc; ++s2) mstar = fmaxf(mstar, recv_ml[((size_t)s2 * ppc + pl) * 2]);
+        const float mu = mstar == -INFINITY ? 0.f : mstar;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float lsum = 0.f;
+#pragma unroll 1
+        for (int s2 = 0; s2 < nsrc; ++s2) {
+            const float2 ml = *reinterpret_cast<const float2 *>(recv_ml + ((size_t)s2 * ppc + pl) * 2);
+            const float w = exp2f(ml.x - mu);
+            const float4 v = *reinterpret_cast<const float4 *>(recv_o + ((size_t)s2 * ppc + pl) * HD + d0);
+            lsum += ml.y * w;
+            acc.x += v.x * w;
+            acc.y += v.y * w;
+            acc.z += v.z * w;
+            acc.w += v.w * w;
         }
+        const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+        bf16 *dst = out + (size_t)(r0 + row) * ldo + (kvh * grp + hh) * HD + d0;
+        store_pair(dst, lo, acc.x * inv, acc.y * inv);
+        store_pair(dst + 2, lo, acc.z * inv, acc.w * inv);
     }
-    cluster_sync_all();
 }
 
 }  // namespace at
@@ -410,21 +397,32 @@ bool attn_mma_supported<float>(int) {
 
 static int g_num_sms = 0;
 
+// key groups per CTA: two when the kv group has at most 4 q heads (8 warps)
+static int attn_groups(int grp) { return grp <= 4 ? 2 : 1; }
+
+static size_t attn_smem(int hd, bool split, int grp, int n_splits) {
+    const int G = attn_groups(grp);
+    const size_t tiles = (size_t)G * (split ? 4 : 2) * at::KB * (hd + 8) * sizeof(bf16);
+    const int pairs = grp * 16, ppc = (pairs + n_splits - 1) / n_splits;
+    const size_t recv = (size_t)n_splits * G * ppc * (hd + 2) * sizeof(float);
+    return tiles + recv;
+}
+
 template <int HD, bool SPLIT>
 static void launch_hd(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
                       int rows_per_tile, int nq, int nkv, int max_len, bf16 *out, int ldo, size_t lo, int n_tiles,
                       int n_splits, cudaStream_t s) {
     const int grp = nq / nkv;
-    size_t smem = (SPLIT ? 4 : 2) * 2 * at::KB * (HD + 8) * sizeof(bf16);
-    smem = std::max(smem, (size_t)grp * 16 * (HD + 4) * sizeof(float));
+    const int G = attn_groups(grp);
+    const size_t smem = attn_smem(HD, SPLIT, grp, n_splits);
     static bool set = false;
     if (!set) {
-        cudaFuncSetAttribute(at::attn_mma_kernel<HD, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(at::attn_mma_kernel<HD, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         set = true;
     }
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-    launch_k(at::attn_mma_kernel<HD, SPLIT>, dim3(n_tiles, nkv, n_splits), dim3(32 * grp), smem, s, n_splits, q, ldq, kc,
-             vc, meta, R, rows_per_tile, nq, nkv, max_len, n_splits, scale_log2, out, ldo, lo);
+    launch_k(at::attn_mma_kernel<HD, SPLIT>, dim3(n_tiles, nkv, n_splits), dim3(32 * grp * G), smem, s, n_splits, q, ldq,
+             kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, n_splits, G, scale_log2, out, ldo, lo);
 }
 
 template <>

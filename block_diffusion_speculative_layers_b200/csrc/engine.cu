@@ -68,6 +68,7 @@ static bool check_model(const dflash_model_cfg &m, std::string &why) {
         return false;
     }
     if (m.n_q_heads % m.n_kv_heads) { why = "n_q_heads must be a multiple of n_kv_heads"; return false; }
+    if (m.n_q_heads / m.n_kv_heads > 8) { why = "at most 8 q heads per kv head"; return false; }
     if (m.head_dim != 64 && m.head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
     if (m.hidden % 64) { why = "hidden must be a multiple of 64"; return false; }
     if (m.n_experts < 0 || m.n_experts > 256) { why = "n_experts must be in [0, 256]"; return false; }

@@ -105,6 +105,9 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    // K split: every CTA of the cluster has started before any pushes into another's
+    // shared memory (arrive now; the epilogue warps wait before their first push)
+    if (split) cluster_arrive_relaxed();
     pdl_trigger();
 
     if (warp == 0) {
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(NT, 1)
                 // push this CTA's partial columns into the receive buffer of the CTA that
                 // finishes them: recv[source rank][weight row][column - owner's c_begin],
                 // four columns (one owner, cpr being a multiple of 4) per store
+                cluster_wait();
                 for (int c = 0; c < TM; c += CH) {
                     if (ok) acc_ld16(trow, c, lo_col, v);
                     else
@@ -249,6 +253,7 @@ __global__ void __launch_bounds__(NT, 1)
         // the pushes of every CTA are visible after the barrier (release / acquire);
         // afterwards no CTA touches another's shared memory, so one barrier suffices
         __syncwarp();
+        if (warp < 2) cluster_wait();  // the epilogue warps waited before pushing
         cluster_sync_all();
         if (warp >= 2) {
             const int q = warp & 3;
