@@ -309,10 +309,11 @@ class DFlash:
         self._check(self.lib.dflash_profile(self.h, 1 if enable else 0), "dflash_profile")
 
     def profile_read(self):
-        out = (KernelProf * 2)()
+        out = (KernelProf * 3)()
         self._check(self.lib.dflash_profile_read(self.h, out), "dflash_profile_read")
         return {"projection": (out[0].launches, out[0].ms, out[0].bytes),
-                "attention": (out[1].launches, out[1].ms, out[1].bytes)}
+                "attention": (out[1].launches, out[1].ms, out[1].bytes),
+                "gate_up": (out[2].launches, out[2].ms, out[2].bytes)}
 
     def load_weights_from(self, make_one, names=None):
         """Fill each weight slot from make_one(name) (one tensor alive at a time)."""

@@ -320,7 +320,7 @@ class Engine : public EngineBase {
     int *pinned = nullptr;  // small pinned host buffer for the done counter
     bool lens_stale = false;
     // per-launch timing (dflash_profile)
-    struct ProfRec { int cls; double bytes; cudaEvent_t a, b; };
+    struct ProfRec { int cls, sub; double bytes; cudaEvent_t a, b; };  // sub: second class or -1
     bool profiling = false;
     std::vector<ProfRec> prof;
     std::vector<cudaEvent_t> ev_pool;
@@ -533,25 +533,29 @@ class Engine : public EngineBase {
     }
 
     template <typename F>
-    void timed(int cls, double bytes, F &&launch) {
+    void timed(int cls, double bytes, F &&launch, int sub = -1) {
         if (!profiling) {
             launch();
             return;
         }
-        ProfRec r{cls, bytes, next_event(), next_event()};
+        ProfRec r{cls, sub, bytes, next_event(), next_event()};
         cudaEventRecord(r.a, s);
         launch();
         cudaEventRecord(r.b, s);
         prof.push_back(r);
     }
 
-    static double gemm_bytes(int M, int N, int K, const Epi<T> &e) {
-        const double es = sizeof(T);
-        double b = (double)N * K * es + (double)M * K * es;
+    // algorithmic HBM bytes of one projection: the weight matrix once, the
+    // activation input (both planes of two-plane activations) and the outputs
+    double gemm_bytes(int M, int N, int K, const Epi<T> &e) const {
+        const double es = sizeof(T), ea = es * (lo_ ? 2 : 1);
+        double b = (double)N * K * es + (double)M * K * ea;
         switch (e.kind) {
-            case EPI_QKV: b += (double)M * N * es; break;
-            case EPI_RESID: b += (double)M * N * 8 + (double)M * N * es * e.taps.n; break;
-            case EPI_SWIGLU: b += (double)M * e.F * es; break;
+            case EPI_QKV: b += (double)M * N * ea; break;
+            case EPI_RESID:
+                b += (double)M * N * 8 + (double)M * N * ea * e.taps.n + (e.xg ? (double)M * N * ea : 0.0);
+                break;
+            case EPI_SWIGLU: b += (double)M * e.F * ea; break;
             case EPI_LOGITS: b += (double)((N + 127) / 128) * M * 8; break;
             default: b += (double)M * N * 4; break;
         }
@@ -560,7 +564,8 @@ class Engine : public EngineBase {
 
     void gemm(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e) {
         if (M <= 0) return;
-        timed(0, gemm_bytes(M, N, K, e), [&] { gemm_launch(X, ldx, M, Wt, N, K, e); });
+        timed(DFLASH_PROF_PROJECTION, gemm_bytes(M, N, K, e), [&] { gemm_launch(X, ldx, M, Wt, N, K, e); },
+              e.kind == EPI_SWIGLU ? DFLASH_PROF_GATE_UP : -1);
     }
 
     void gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e_in) {
@@ -1479,9 +1484,13 @@ class Engine : public EngineBase {
         for (const ProfRec &p : prof) {
             float ms = 0.f;
             if (cudaEventElapsedTime(&ms, p.a, p.b) != cudaSuccess) return fail_cuda("event time");
-            o[p.cls].launches += 1;
-            o[p.cls].ms += ms;
-            o[p.cls].bytes += p.bytes;
+            const int cls2[2] = {p.cls, p.sub};
+            for (int k : cls2) {
+                if (k < 0) continue;
+                o[k].launches += 1;
+                o[k].ms += ms;
+                o[k].bytes += p.bytes;
+            }
         }
         return DFLASH_OK;
     }

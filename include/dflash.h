@@ -116,7 +116,9 @@ typedef struct {
     double bytes;
 } dflash_kernel_prof;
 
-enum { DFLASH_PROF_PROJECTION = 0, DFLASH_PROF_ATTENTION = 1, DFLASH_PROF_CLASSES = 2 };
+/* PROJECTION: every projection launch; ATTENTION: every attention launch;
+ * GATE_UP: the gate/up (SwiGLU) projections alone (also counted in PROJECTION). */
+enum { DFLASH_PROF_PROJECTION = 0, DFLASH_PROF_ATTENTION = 1, DFLASH_PROF_GATE_UP = 2, DFLASH_PROF_CLASSES = 3 };
 
 /* Bytes of the weight and state arenas for this configuration.
  * Errors: DFLASH_EINVAL on inconsistent configuration, DFLASH_EUNSUPPORTED on
