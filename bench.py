@@ -34,6 +34,7 @@ if ROOT not in sys.path:
 
 from synthetic import get_config, make_prompt, make_weight  # noqa: E402
 from synthetic.weights import weight_shapes  # noqa: E402
+from block_diffusion_speculative_layers_b200.replicas import rank_prompt_seeds, reduce_max, reduce_step  # noqa: E402
 
 METRIC = "generated tokens/s @1×B200 batch 1 (Qwen3-8B shape); µs/iter vs HBM roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -221,8 +222,8 @@ def main():
     t0 = time.time()
     ctx.load_weights_from(lambda n: make_weight(cfg, n, device=dev))
     log(f"[rank {rank}] weights generated + loaded in {time.time() - t0:.1f}s ({ctx.weight_bytes / 1e9:.2f} GB)")
-    prompts = [make_prompt(cfg.prompt_kind, cfg.prompt_len, cfg.target.vocab, cfg.seed + 1000 * rank + i)
-               for i in range(b)]
+    prompts = [make_prompt(cfg.prompt_kind, cfg.prompt_len, cfg.target.vocab, sd)
+               for sd in rank_prompt_seeds(cfg.seed, rank, b)]
     stream = torch.cuda.current_stream(dev)
 
     def prefill_all():
@@ -259,14 +260,7 @@ def main():
     time.sleep(0.2)
     clk = clocks.stop()
     tokens = st.tokens
-    ms_max, tok_sum = ms, tokens
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_max = float(t.item())
-        n = torch.tensor([tokens], device=dev, dtype=torch.float64)
-        pg.all_reduce(n)
-        tok_sum = int(n.item())
+    ms_max, tok_sum = reduce_step(pg, ms, tokens, dev)
     value = tok_sum / (ms_max / 1000.0)
     mean_tau = st.mean_tau
     ctx_len_mean = cfg.prompt_len + args.warmup * mean_tau + 0.5 * args.steps * mean_tau
@@ -341,10 +335,7 @@ def main():
     e2e_ms = e0.elapsed_time(e1)
     e2e_tokens = b * args.e2e_tokens
     iters_e2e = max(1, gst.iterations // max(1, b))
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(pg, e2e_ms, dev)
     e2e_value = world * e2e_tokens / (e2e_ms / 1000.0)
     h2d = sum(p.nbytes for p in host_prompts) + 4 * b
     d2h = out.nbytes + 4 * (iters_e2e + 2)
