@@ -470,14 +470,14 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
     const int stage_bytes = tc::A_BYTES + TM * 128 * p.planes;
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64;
     // Measured on B200 (decode shapes, M = 16, whole decode iteration): every
-    // projection streams best with ~110 KB CTAs, two of which fit on an SM --
-    // projections with fewer tiles than SMs split K over a cluster so that about
-    // one CTA per SM runs, and the other slot lets the next projection's CTAs
-    // start (programmatic dependent launch) and prefetch their weights while
-    // this one drains.  Larger (150 KB, one CTA per SM) rings were faster for
-    // a projection timed alone but 0.5 ms per iteration slower in the pipeline.
+    // projection streams best with ~110 KB CTAs, two of which fit on an SM;
+    // projections with fewer tiles than that split K over a cluster (up to 8
+    // CTAs) to fill both slots of every SM.  Larger (150 KB, one CTA per SM)
+    // rings were faster for a projection timed alone but 0.5 ms per iteration
+    // slower in the pipeline; filling one slot per SM was 0.2 ms slower.
     int splits = 1;
-    const int slots = num_sms * std::max(1, tune_ctas_per_sm);  // CTAs the K-split aims to fill
+    // the K split aims to fill two ~110 KB CTAs per SM (measured best in the decode pipeline)
+    const int slots = num_sms * (tune_ctas_per_sm > 0 ? tune_ctas_per_sm : 2);
     if (e.kind != EPI_LOGITS && tiles < slots && p.k_steps >= 4) {
         splits = std::max(1, std::min({8, p.k_steps / 2, slots / std::max(1, tiles)}));
         if (tune_splits > 0) splits = std::min(8, tune_splits);
