@@ -102,6 +102,28 @@ __device__ __forceinline__ void st_cluster_v2(float *local, uint32_t rank, float
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(ra), "f"(a), "f"(b) : "memory");
 }
 
+// bounded wait until *p >= target (acquire); error bit 16 after 2 s
+__device__ __forceinline__ void wait_ctr(const int *p, int target, int *err) {
+    auto ld = [&] {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        return v;
+    };
+    if (ld() >= target) return;
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    while (true) {
+        for (int i = 0; i < 32; ++i)
+            if (ld() >= target) return;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > 2000000000ull) {
+            if (err) atomicOr(err, 16);
+            return;
+        }
+        __nanosleep(32);
+    }
+}
+
 __device__ __forceinline__ void group_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -126,7 +148,8 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
                                                        const bf16 *__restrict__ vc, const RowMeta *__restrict__ meta,
                                                        int R, int rows_per_tile, int nq, int nkv, int max_len,
                                                        int n_splits, int G, float scale_log2, bf16 *__restrict__ out,
-                                                       int ldo, size_t lo) {
+                                                       int ldo, size_t lo, const int *dep_ctr, int dep_target,
+                                                       int *done_ctr, int *err) {
     constexpr int LDS = HD + 8;                 // padded smem row (bf16 elements)
     constexpr int NPL = SPLIT ? 4 : 2;          // planes per tile buffer: K, V (+ K lo, V lo)
     constexpr int PLANE = KB * LDS;             // elements of one plane of a tile buffer
@@ -136,7 +159,12 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
     // shared memory: arrive now, wait before the first push
     cluster_arrive_relaxed();
     pdl_trigger();
-    pdl_wait();
+    if (dep_ctr) {  // completion counter of the projection that wrote q and K/V
+        if (threadIdx.x == 0) wait_ctr(dep_ctr, dep_target, err);
+        __syncthreads();
+    } else {
+        pdl_wait();
+    }
     const int tile = blockIdx.x, kvh = blockIdx.y, split = blockIdx.z;
     const int grp = nq / nkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -372,6 +400,15 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const bf16 *__restrict__ 
         store_pair(dst, lo, acc.x * inv, acc.y * inv);
         store_pair(dst + 2, lo, acc.z * inv, acc.w * inv);
     }
+    if (done_ctr) {  // every writer fences (generic and async proxy), then one signal per CTA
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(done_ctr, 1);
+        }
+    }
 }
 
 }  // namespace at
@@ -411,7 +448,7 @@ static size_t attn_smem(int hd, bool split, int grp, int n_splits) {
 template <int HD, bool SPLIT>
 static void launch_hd(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
                       int rows_per_tile, int nq, int nkv, int max_len, bf16 *out, int ldo, size_t lo, int n_tiles,
-                      int n_splits, cudaStream_t s) {
+                      int n_splits, const AttnSync &sy, cudaStream_t s) {
     const int grp = nq / nkv;
     const int G = attn_groups(grp);
     const size_t smem = attn_smem(HD, SPLIT, grp, n_splits);
@@ -422,15 +459,16 @@ static void launch_hd(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, co
     }
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
     launch_k(at::attn_mma_kernel<HD, SPLIT>, dim3(n_tiles, nkv, n_splits), dim3(32 * grp * G), smem, s, n_splits, q, ldq,
-             kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, n_splits, G, scale_log2, out, ldo, lo);
+             kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, n_splits, G, scale_log2, out, ldo, lo, sy.dep_ctr,
+             sy.dep_target, sy.done_ctr, sy.err);
 }
 
 template <>
-void launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
-                                int rows_per_tile, int nq, int nkv, int hd, int max_len, bf16 *out, int ldo, size_t lo,
-                                const AttnScratch &ws, cudaStream_t s) {
+int launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
+                               int rows_per_tile, int nq, int nkv, int hd, int max_len, bf16 *out, int ldo, size_t lo,
+                               const AttnScratch &ws, cudaStream_t s, const AttnSync &sy) {
     (void)ws;
-    if (R <= 0) return;
+    if (R <= 0) return 0;
     if (!g_num_sms) {
         int dev = 0;
         cudaGetDevice(&dev);
@@ -442,16 +480,19 @@ void launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf
     // splits than 64-key tiles the longest possible context has
     const int n_splits = std::max(1, std::min({8, (2 * g_num_sms + ctas - 1) / ctas, (max_len + 63) / 64}));
     if (hd == 128) {
-        if (lo) launch_hd<128, true>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, lo, n_tiles, n_splits, s);
-        else launch_hd<128, false>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, 0, n_tiles, n_splits, s);
+        if (lo) launch_hd<128, true>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, lo, n_tiles, n_splits, sy, s);
+        else launch_hd<128, false>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, 0, n_tiles, n_splits, sy, s);
     } else {
-        if (lo) launch_hd<64, true>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, lo, n_tiles, n_splits, s);
-        else launch_hd<64, false>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, 0, n_tiles, n_splits, s);
+        if (lo) launch_hd<64, true>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, lo, n_tiles, n_splits, sy, s);
+        else launch_hd<64, false>(q, ldq, kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, out, ldo, 0, n_tiles, n_splits, sy, s);
     }
+    return n_tiles * nkv * n_splits;
 }
 
 template <>
-void launch_attention_mma<float>(const float *, int, const float *, const float *, const RowMeta *, int, int, int, int,
-                                 int, int, float *, int, size_t, const AttnScratch &, cudaStream_t) {}
+int launch_attention_mma<float>(const float *, int, const float *, const float *, const RowMeta *, int, int, int, int,
+                                int, int, float *, int, size_t, const AttnScratch &, cudaStream_t, const AttnSync &) {
+    return 0;
+}
 
 }  // namespace dfl

@@ -26,12 +26,21 @@ AttnWorkspace attn_workspace_plan(int max_rows, int nq, int nkv, int max_len, in
 template <typename T>
 bool attn_mma_supported(int hd);
 
+// Completion counters of a decode pass (all null: griddepcontrol.wait and no signal).
+struct AttnSync {
+    const int *dep_ctr = nullptr;  // wait until *dep_ctr >= dep_target
+    int dep_target = 0;
+    int *done_ctr = nullptr;       // each CTA adds 1 after its last store
+    int *err = nullptr;            // device error word (bit 16: a wait timed out)
+};
+
 // rows_per_tile: rows of one sequence that share a query tile (block size for
 // draft/verify, 16 for prompt rows, 1 for single-row target steps).
 // lo != 0: q, K/V and out are two-plane activations (low plane lo elements on).
+// Returns the number of CTAs launched.
 template <typename T>
-void launch_attention_mma(const T *q, int ldq, const T *kc, const T *vc, const RowMeta *meta, int R, int rows_per_tile,
-                          int nq, int nkv, int hd, int max_len, T *out, int ldo, size_t lo, const AttnScratch &ws,
-                          cudaStream_t s);
+int launch_attention_mma(const T *q, int ldq, const T *kc, const T *vc, const RowMeta *meta, int R, int rows_per_tile,
+                         int nq, int nkv, int hd, int max_len, T *out, int ldo, size_t lo, const AttnScratch &ws,
+                         cudaStream_t s, const AttnSync &sy = AttnSync());
 
 }  // namespace dfl

@@ -28,31 +28,6 @@
 namespace dfl {
 namespace tc {
 
-__device__ __forceinline__ int ld_acquire(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Bounded wait until *p >= target.  false (error bit 8) after WAIT_NS.
-__device__ bool wait_counter(const int *p, int target, int *err) {
-    if (ld_acquire(p) >= target) return true;
-    const unsigned long long t0 = gtimer();
-    while (true) {
-        for (int i = 0; i < 32; ++i)
-            if (ld_acquire(p) >= target) return true;
-        if (gtimer() - t0 > WAIT_NS) {
-            if (err) atomicOr(err, 8);
-            return false;
-        }
-        __nanosleep(32);
-    }
-}
-
 struct PendingX {
     int s, j, k;
 };

@@ -64,6 +64,13 @@ struct ChainProgram {
     unsigned epoch = 0;
     int key = -1;                    // program identity (pass, batch) it was built for
     bool valid = true;               // false: the shapes do not fit the reserved workspace
+    // per-kernel execution: completion counters [2 * n_ops] (projection i: i;
+    // attention of layer l: n_ops + l), runs of the program since its counters
+    // were cleared, CTAs each counter receives per run, last counter of the pass
+    int *d_dep = nullptr;
+    unsigned dep_run = 0;
+    std::vector<int> dep_ctas;
+    int dep_prev = -1;
 };
 
 // Launch ops [b, e) of a program (epoch must already be advanced for this run).

@@ -253,7 +253,7 @@ static Layout make_layout(const dflash_config &c) {
         auto prog_bytes = [&](int n_ops) {
             return align_up((size_t)n_ops * sizeof(ChainOp), 256) + align_up((size_t)2 * n_ops * sizeof(CUtensorMap), 256) +
                    align_up((size_t)n_ops * 4, 256) + align_up((size_t)n_ops * L.max_tiles * 4, 256) +
-                   align_up((size_t)n_ops * L.max_tiles * sizeof(int4), 256);
+                   align_up((size_t)n_ops * L.max_tiles * sizeof(int4), 256) + align_up((size_t)2 * n_ops * 4, 256);
         };
         L.chain_v_bytes = prog_bytes(L.n_ops_v);
         L.chain_d_bytes = prog_bytes(L.n_ops_d);
@@ -310,6 +310,7 @@ class Engine : public EngineBase {
     // bf16 decode passes run as projection programs with folded RMSNorms
     // (fold_*_ok), one kernel per projection or, with chain_on, as persistent chains
     bool chain_verify_ok = false, chain_draft_ok = false, chain_on = false;
+    bool dep_on = false;  // completion counters between the kernels of a pass (per-kernel mode)
     bool chain_used[3] = {false, false, false};
     int num_sms = 148;
     GemmTC<T> tc;
@@ -421,6 +422,11 @@ class Engine : public EngineBase {
             // DFLASH_FOLDED_NORM=0 goes back to separate RMSNorm kernels
             const char *ev = getenv("DFLASH_PROJECTION_CHAIN");
             chain_on = ev && ev[0] == '1';
+            // DFLASH_DEP_COUNTERS=1: device completion counters between the kernels of a
+            // pass instead of griddepcontrol.wait (same results; measured 0.2 ms per step
+            // slower on B200: the fences of every writer cost more than the grid release)
+            const char *dv_env = getenv("DFLASH_DEP_COUNTERS");
+            dep_on = !chain_on && dv_env && dv_env[0] == '1';
             const char *fv = getenv("DFLASH_FOLDED_NORM");
             const bool allow = !(fv && fv[0] == '0');
             chain_draft_ok = allow && bf && shapes;
@@ -436,6 +442,8 @@ class Engine : public EngineBase {
                 pg.d_tile_cnt = reinterpret_cast<int *>(b);
                 b += align_up((size_t)n_ops * L.max_tiles * 4, 256);
                 pg.d_tinfo = reinterpret_cast<int4 *>(b);
+                b += align_up((size_t)n_ops * L.max_tiles * sizeof(int4), 256);
+                pg.d_dep = reinterpret_cast<int *>(b);
                 pg.d_ws = sp<float>(L.chain_ws);
                 pg.ws_floats = L.chain_ws_floats;
             };
@@ -562,19 +570,23 @@ class Engine : public EngineBase {
         return b;
     }
 
-    void gemm(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e) {
-        if (M <= 0) return;
-        timed(DFLASH_PROF_PROJECTION, gemm_bytes(M, N, K, e), [&] { gemm_launch(X, ldx, M, Wt, N, K, e); },
+    // One projection; returns the CTAs launched (tensor-core path).  dep/done:
+    // completion counters of a decode pass (see PassSync), else griddepcontrol.wait.
+    int gemm(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e, const int *dep = nullptr,
+             int dep_target = 0, int *done = nullptr) {
+        if (M <= 0) return 0;
+        int ctas = 0;
+        timed(DFLASH_PROF_PROJECTION, gemm_bytes(M, N, K, e),
+              [&] { ctas = gemm_launch(X, ldx, M, Wt, N, K, e, dep, dep_target, done); },
               e.kind == EPI_SWIGLU ? DFLASH_PROF_GATE_UP : -1);
+        return ctas;
     }
 
-    void gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e_in) {
+    int gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e_in,
+                    const int *dep = nullptr, int dep_target = 0, int *done = nullptr) {
         Epi<T> e = e_in;
         e.lo = lo_;  // every input and output of the engine's projections lives in the activation span
-        if (tc.supports(M, N, K)) {
-            tc.run(X, ldx, M, (const T *)Wt, N, K, e, s);
-            return;
-        }
+        if (tc.supports(M, N, K)) return tc.run(X, ldx, M, (const T *)Wt, N, K, e, s, dep, dep_target, done);
         // CUDA-core path (fp32 models): GEMM into fp32 Y, then the epilogue.
         float *Yo = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.Y : Y;
         const int ldy = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.ldy : N;
@@ -593,19 +605,23 @@ class Engine : public EngineBase {
             default:
                 break;
         }
+        return 0;
     }
 
-    void attention(const T *qq, const T *kc, const T *vc, const RowMeta *mt, int R, int rows_per_tile,
-                   const dflash_model_cfg &m, T *out) {
+    // returns the CTAs launched by the tensor-core attention (0 on the CUDA-core path)
+    int attention(const T *qq, const T *kc, const T *vc, const RowMeta *mt, int R, int rows_per_tile,
+                  const dflash_model_cfg &m, T *out, const AttnSync &sy = AttnSync()) {
         const int qd = m.n_q_heads * m.head_dim;
+        int ctas = 0;
         timed(1, 0.0, [&] {
             if (attn_mma_supported<T>(m.head_dim))
-                launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads, m.head_dim,
-                                        c.max_len, out, qd, lo_, att, s);
+                ctas = launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads,
+                                               m.head_dim, c.max_len, out, qd, lo_, att, s, sy);
             else
                 launch_attention_simt<T>(qq, qd, kc, vc, mt, R, m.n_q_heads, m.n_kv_heads, m.head_dim, c.max_len, out,
                                          qd, s);
         });
+        return ctas;
     }
 
     // one pre-norm decoder layer of the target over R rows in x (meta)
@@ -810,6 +826,10 @@ class Engine : public EngineBase {
         cudaMemsetAsync(pg.d_op_done, 0, sizeof(int) * pg.ops.size(), s);
         cudaMemsetAsync(pg.d_tile_cnt, 0, sizeof(int) * (size_t)pg.ops.size() * L.max_tiles, s);
         pg.epoch = 0;
+        cudaMemsetAsync(pg.d_dep, 0, sizeof(int) * 2 * pg.ops.size(), s);
+        pg.dep_run = 0;
+        pg.dep_ctas.assign(2 * pg.ops.size(), 0);
+        pg.dep_prev = -1;
     }
 
     Epi<T> epi_norm_in(Epi<T> e, float eps, int H) {
@@ -974,9 +994,44 @@ class Engine : public EngineBase {
             }
             for (int i = b; i < e; ++i) {
                 const HostOp &h = pg.hops[i];
-                gemm((const T *)h.X, h.ldx, h.M, h.W, h.N, h.K, pg.ops[i].e);
+                int tgt = 0;
+                const int *dep = pass_dep(pg, tgt);
+                const int k = gemm((const T *)h.X, h.ldx, h.M, h.W, h.N, h.K, pg.ops[i].e, dep, tgt,
+                                   dep_on ? pg.d_dep + i : nullptr);
+                pass_done(pg, i, k);
             }
         }
+    }
+
+    // Completion counters of a decode pass run one kernel per projection: each
+    // projection and attention launch waits until every CTA of the launch before
+    // it has signalled (instead of waiting for that grid to exit and flush), which
+    // lets it start about as soon as the last epilogue store is visible.
+    void pass_begin(ChainProgram &pg) {
+        pg.dep_run += 1;
+        pg.dep_prev = -1;  // the first launch of a pass waits with griddepcontrol.wait
+    }
+    const int *pass_dep(ChainProgram &pg, int &target) {
+        if (!dep_on || pg.dep_prev < 0) {
+            target = 0;
+            return nullptr;
+        }
+        target = (int)pg.dep_run * pg.dep_ctas[pg.dep_prev];
+        return pg.d_dep + pg.dep_prev;
+    }
+    void pass_done(ChainProgram &pg, int idx, int ctas) {
+        if (!dep_on) return;
+        pg.dep_ctas[idx] = ctas;
+        pg.dep_prev = ctas > 0 ? idx : -1;  // a launch that signals nothing cannot be waited on
+    }
+    AttnSync pass_attn_sync(ChainProgram &pg, int layer, int &idx) {
+        AttnSync sy;
+        idx = (int)pg.ops.size() + layer;
+        if (!dep_on) return sy;
+        sy.dep_ctr = pass_dep(pg, sy.dep_target);
+        sy.done_ctr = pg.d_dep + idx;
+        sy.err = &stats->status;
+        return sy;
     }
 
     void enqueue_verify_chain(int nseq) {
@@ -984,11 +1039,16 @@ class Engine : public EngineBase {
         const int B = c.block_size, R = nseq * B, H = t.hidden;
         if (pv.key != nseq) build_verify_program(nseq);
         if (chain_on && pv.valid) pv.epoch++;
+        pass_begin(pv);
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, tl[0].attn_norm,
                              xg_t, H, lo_, ssq, L.ssq_ld, s);
         run_ops(pv, 0, 1);
         for (int l = 0; l < t.n_layers; ++l) {
-            attention(q, tk + (size_t)l * kv_layer_elems(t), tv + (size_t)l * kv_layer_elems(t), meta, R, B, t, ao);
+            int ai;
+            const AttnSync sy = pass_attn_sync(pv, l, ai);
+            const int k = attention(q, tk + (size_t)l * kv_layer_elems(t), tv + (size_t)l * kv_layer_elems(t), meta, R,
+                                    B, t, ao, sy);
+            pass_done(pv, ai, k);
             run_ops(pv, 1 + 4 * l, 5 + 4 * l);
         }
         launch_lm_argmax(lm_part, (t.vocab + 127) / 128, R, 0, B, g, stats, s);
@@ -1001,11 +1061,16 @@ class Engine : public EngineBase {
         const int B = c.block_size, R = nseq * B, H = d.hidden;
         if (pd.key != nseq) build_draft_program(nseq);
         if (chain_on && pd.valid) pd.epoch++;
+        pass_begin(pd);
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, dl[0].attn_norm,
                              dq_in, H, lo_, ssq, L.ssq_ld, s);
         run_ops(pd, 0, 2);
         for (int j = 0; j < d.n_layers; ++j) {
-            attention(q, dk + (size_t)j * kv_layer_elems(d), dv + (size_t)j * kv_layer_elems(d), meta, R, B, d, ao);
+            int ai;
+            const AttnSync sy = pass_attn_sync(pd, j, ai);
+            const int k = attention(q, dk + (size_t)j * kv_layer_elems(d), dv + (size_t)j * kv_layer_elems(d), meta, R,
+                                    B, d, ao, sy);
+            pass_done(pd, ai, k);
             run_ops(pd, 2 + 4 * j, 6 + 4 * j);
         }
         if (B > 1) launch_lm_argmax(lm_part, (c.target.vocab + 127) / 128, R, 1, B, drafts, stats, s);

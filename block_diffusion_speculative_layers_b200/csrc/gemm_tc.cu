@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(NT, 1)
                         tma_load_2d_hint(a, &tmW, (kb + i) * BK, rowA0, &full[i], wpol);
                         tma_load_2d_hint(a + A_BYTES / 2, &tmW, (kb + i) * BK, rowA1, &full[i], wpol);
                     }
-                    pdl_wait();
+                    dep_wait(p.dep_ctr, p.dep_target, p.err);
                     for (int i = 0; i < pre; ++i) {
                         if (p.planes == 2) tma_load_3d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, 0, &full[i]);
                         else tma_load_2d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, &full[i]);
@@ -191,7 +191,12 @@ __global__ void __launch_bounds__(NT, 1)
         }
     } else {
         // ---------------- epilogue warps 2..5 ----------------
-        pdl_wait();
+        if (p.dep_ctr) {
+            if (threadIdx.x == 64) dep_wait(p.dep_ctr, p.dep_target, p.err);
+            epi_bar();
+        } else {
+            pdl_wait();
+        }
         const int q = warp & 3;
         const int n_local = q * 32 + lane;
         // K split: CTA `rank` of the cluster reduces and finishes columns [c_begin, c_end)
@@ -285,8 +290,16 @@ __global__ void __launch_bounds__(NT, 1)
             else finish(std::integral_constant<int, CH>{});
         }
     }
+    if (p.done_ctr) {  // every writer fences (generic and async proxy) before the signal
+        __threadfence();
+        fence_proxy_async_global();
+    }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
+    if (p.done_ctr && threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(p.done_ctr, 1);
+    }
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
@@ -452,8 +465,8 @@ static void launch_kind(int kind, const CUtensorMap *mw, const CUtensorMap *mx, 
 }
 
 template <>
-void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int K, const Epi<bf16> &e,
-                       cudaStream_t s) {
+int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int K, const Epi<bf16> &e,
+                      cudaStream_t s, const int *dep_ctr, int dep_target, int *done_ctr) {
     const bool swiglu = e.kind == EPI_SWIGLU;
     int TM = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
     TcParams p;
@@ -496,10 +509,13 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
     p.err = err_word;
     p.lm_part = lm_part;
     p.keep_logits = keep_logits;
+    p.dep_ctr = dep_ctr;
+    p.dep_target = dep_target;
+    p.done_ctr = done_ctr;
     const int grid_x = p.n_tiles;  // one tile per CTA
     const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
     const CUtensorMap *mx = tensor_map(X, M, K, ldx, TM, e.lo);
-    if (!mw || !mx) return;
+    if (!mw || !mx) return 0;
     switch (TM) {
         case 16: launch_kind<16>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
         case 32: launch_kind<32>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
@@ -507,10 +523,14 @@ void GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int 
         case 128: launch_kind<128>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
         default: launch_kind<256>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
     }
+    return p.n_tiles * p.m_tiles * p.splits;
 }
 
 template <>
-void GemmTC<float>::run(const float *, int, int, const float *, int, int, const Epi<float> &, cudaStream_t) {}
+int GemmTC<float>::run(const float *, int, int, const float *, int, int, const Epi<float> &, cudaStream_t,
+                       const int *, int, int *) {
+    return 0;
+}
 
 template struct GemmTC<bf16>;
 template struct GemmTC<float>;

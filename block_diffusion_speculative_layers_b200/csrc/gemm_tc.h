@@ -31,6 +31,12 @@ struct TcParams {
     float2 *lm_part;        // EPI_LOGITS: per (n_tile, row) best (value, index)
     int keep_logits;        // EPI_LOGITS: also store fp32 logits in Y
     int planes;             // activation planes (2: hi + lo, two MMAs per K step)
+    // completion counters (decode passes): wait until *dep_ctr >= dep_target instead
+    // of griddepcontrol.wait (dep_ctr == nullptr: griddepcontrol.wait); each CTA adds
+    // 1 to *done_ctr after its last store (done_ctr == nullptr: no signal)
+    const int *dep_ctr;
+    int dep_target;
+    int *done_ctr;
 };
 
 template <typename T>
@@ -38,7 +44,9 @@ struct GemmTC {
     std::string err;
     bool supports(int M, int N, int K) const;
     int init(float *ws, int ws_floats, int *sem, int n_sem);
-    void run(const T *X, int ldx, int M, const T *W, int N, int K, const Epi<T> &e, cudaStream_t s);
+    // returns the number of CTAs launched (the count a completion counter reaches per run)
+    int run(const T *X, int ldx, int M, const T *W, int N, int K, const Epi<T> &e, cudaStream_t s,
+            const int *dep_ctr = nullptr, int dep_target = 0, int *done_ctr = nullptr);
     // LM-head partial argmax buffer (value, index as float bits), [n_tiles][rows]
     void set_lm_part(float2 *p, int cap) { lm_part = p; lm_cap = cap; }
     void set_err(int *e) { err_word = e; }

@@ -154,6 +154,43 @@ __device__ __forceinline__ void acc_ld16(uint32_t taddr, int c, int lo_col, floa
     }
 }
 
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *p >= target.  false (error bit 8) after WAIT_NS.
+__device__ __forceinline__ bool wait_counter(const int *p, int target, int *err) {
+    if (ld_acquire(p) >= target) return true;
+    const unsigned long long t0 = gtimer();
+    while (true) {
+        for (int i = 0; i < 32; ++i)
+            if (ld_acquire(p) >= target) return true;
+        if (gtimer() - t0 > WAIT_NS) {
+            if (err) atomicOr(err, 8);
+            return false;
+        }
+        __nanosleep(32);
+    }
+}
+
+// Wait for the producer of this kernel's inputs: with a completion counter
+// (dep != nullptr), until every CTA of the previous kernel has signalled
+// (acquire; then TMA reads see its writes); otherwise griddepcontrol.wait.
+__device__ __forceinline__ void dep_wait(const int *dep, int target, int *err) {
+    if (dep) {
+        wait_counter(dep, target, err);
+        fence_proxy_async_global();
+    } else {
+        pdl_wait();
+    }
+}
+
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
