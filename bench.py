@@ -345,13 +345,13 @@ def main():
         log("[rank 0] timing the CPU oracle on a bounded sample ...")
         try:
             s = cpu_oracle_sample(cfg)
-            cpu = {"value": s["tokens"] / s["seconds"], "unit": "tokens/s", "cores": os.cpu_count(),
+            cpu = {"value": s["tokens"] / s["seconds"], "unit": "tokens/s", "cores": omp_threads(),
                    "kind": "oracle",
                    "sample": (f"{s['iters']} full-size fp64 draft+verify iteration(s) after a 16-token prompt "
                               f"({s['seconds']:.1f} s; weight generation {s['weight_gen_s']:.1f} s and prefill "
                               f"{s['prefill_s']:.1f} s not counted)")}
         except Exception as e:  # report, do not fail the GPU measurement
-            cpu = {"value": None, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            cpu = {"value": None, "unit": "tokens/s", "cores": omp_threads(), "kind": "oracle",
                    "sample": f"failed: {e}"}
 
     if rank != 0:
@@ -371,14 +371,7 @@ def main():
         "vs_baseline": None,
         "dtype": cfg.dtype,
         "data": "synthetic (counter-based N(0,0.02)-like weights, Zipf(1.1) prompts)",
-        "config": {"workload": f"{cfg.name}: {cfg.target.n_layers}-layer target (hidden {cfg.target.hidden}, "
-                               f"vocab {cfg.target.vocab}) + {cfg.drafter.n_layers}-layer block-{B} drafter, "
-                               f"batch {b} per GPU, {cfg.prompt_len}-token prompt",
-                   "global_batch": b * world, "seq_len": cfg.prompt_len, "block_size": B,
-                   "parallelism": f"replicas x{world}",
-                   "activations": ("bf16 hi+lo planes, fp32 accumulate" if args.bf16_act == "split"
-                                   else "bf16 single plane, fp32 accumulate") if cfg.dtype == "bf16" else "fp32",
-                   "l2": "inputs larger than L2 (18.5 GB of weights streamed per step)"},
+        "config": workload_config(cfg, args, world),
         "us_per_iter": round(us_iter, 2),
         "mean_tau": round(mean_tau, 4),
         "iter_bytes": it_bytes,
@@ -406,6 +399,25 @@ def main():
     print(json.dumps(result), flush=True)
     if pg:
         pg.destroy_process_group()
+
+
+def omp_threads() -> int:
+    """Threads the oracle's OpenMP loops use on this host."""
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
+
+
+def workload_config(cfg, args, world):
+    """The `config` object of both arms' JSON lines."""
+    b, B = cfg.batch, cfg.block_size
+    return {"workload": f"{cfg.name}: {cfg.target.n_layers}-layer target (hidden {cfg.target.hidden}, "
+                        f"vocab {cfg.target.vocab}) + {cfg.drafter.n_layers}-layer block-{B} drafter, "
+                        f"batch {b} per GPU, {cfg.prompt_len}-token prompt",
+            "global_batch": b * world, "seq_len": cfg.prompt_len, "block_size": B,
+            "parallelism": f"replicas x{world}",
+            "activations": ("bf16 hi+lo planes, fp32 accumulate" if args.bf16_act == "split"
+                            else "bf16 single plane, fp32 accumulate") if cfg.dtype == "bf16" else "fp32",
+            "l2": "inputs larger than L2 (18.5 GB of weights streamed per step)"}
 
 
 def run_reference(args, cfg, world, rank):
@@ -436,10 +448,12 @@ def run_reference(args, cfg, world, rank):
         anchor = int(g[a])
         return a + 1
 
-    # the oracle needs no warm-up; one untimed step sizes the time budget
+    # untimed warm-up steps (the first one sizes the time budget)
     t0 = time.time()
     step()
     first = time.time() - t0
+    for _ in range(args.warmup - 1):
+        step()
     n_steps = max(1, min(args.steps, int(args.ref_budget_s / max(first, 1e-3))))
     log(f"reference: one step {first:.1f}s -> timing {n_steps} of {args.steps} steps")
     t0 = time.time()
@@ -447,10 +461,10 @@ def run_reference(args, cfg, world, rank):
     sec = time.time() - t0
     v = tokens / sec
     res = {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "tokens/s", "n_gpus": world,
-           "steps": n_steps, "warmup": 1, "ms_per_step": round(1000 * sec / n_steps, 3),
+           "steps": n_steps, "warmup": args.warmup, "ms_per_step": round(1000 * sec / n_steps, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": {"workload": f"{cfg.name} batch 1, fp64 CPU oracle, 16-token prompt"},
-           "cpu_baseline": {"value": round(v, 5), "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+           "data": "synthetic", "config": dict(workload_config(cfg, args, world), activations="fp64 (oracle)"),
+           "cpu_baseline": {"value": round(v, 5), "unit": "tokens/s", "cores": omp_threads(), "kind": "oracle",
                             "sample": f"{n_steps} full-size draft+verify iterations after a 16-token prompt "
                                       f"(capped at {args.ref_budget_s:.0f} s of CPU time; {args.steps} requested)"},
            "e2e": {"value": round(v, 5), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
