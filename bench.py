@@ -47,7 +47,7 @@ def log(*a):
 
 # DRAM bytes (read + write) of one gate/up projection launch, from an ncu
 # capture of the same kernel shape (see profiles/); None until measured
-GATE_UP_TRAFFIC = {"qwen3_8b": 205.2e6}
+GATE_UP_TRAFFIC = {"qwen3_8b": 205.26e6}
 
 
 def hbm_peak():

@@ -17,6 +17,9 @@ import block_diffusion_speculative_layers_b200 as dfl
 from synthetic import get_config, make_prompt
 from synthetic.configs import ModelDims
 
+import oracle
+from synthetic import make_weights
+from synthetic.fast import make_weights_host
 from parity import build_pair, replay, check_lossless_generate, accept_rule
 
 pytestmark = pytest.mark.gpu
@@ -180,3 +183,28 @@ def test_kv_rollback_matches_oracle(cuda_device):
             ko, vo = ss.ctx_kv(j, t)
             np.testing.assert_allclose(k[t], ko, rtol=0, atol=1e-4)
             np.testing.assert_allclose(v[t], vo, rtol=0, atol=1e-4)
+
+
+@pytest.mark.parametrize("mode", ["fast", "chain", "counters"])
+def test_alternative_execution_modes(cuda_device, mode, monkeypatch):
+    """The opt-in execution modes compute the same decode step: single-plane bf16
+    activations (DFLASH_BF16_FAST, looser logits), the persistent projection chain,
+    and device completion counters between the kernels of a pass."""
+    cfg = tiny_cfg(dtype="bf16", block=16, hidden=2048, nq=16, nkv=4, hd=128, vocab=8192)
+    tol, tie = TOL["bf16"]
+    act = "split"
+    if mode == "fast":
+        act, tol = "fast", 0.15   # one plane: plain bf16 rounding of GEMM inputs, q and K/V
+    if mode == "chain":
+        monkeypatch.setenv("DFLASH_PROJECTION_CHAIN", "1")
+    if mode == "counters":
+        monkeypatch.setenv("DFLASH_DEP_COUNTERS", "1")
+    w_cpu = make_weights_host(cfg, random_gains=True)
+    gpu = dfl.DFlash(cfg, max_batch=1, max_len=256, keep_logits=True, bf16_act=act)
+    gpu.load_weights(make_weights(cfg, device="cuda", random_gains=True))
+    spec = oracle.OracleSpec(cfg, w_cpu)
+    prompt = make_prompt("uniform", 30, cfg.target.vocab, 12)
+    rep = replay(gpu, spec, cfg, [prompt], 4, tol, tie)
+    print(f"{mode}: max |dlogit| {rep.max_dlogit:.4f}, near ties {rep.near_ties}/{rep.checked_tokens}")
+    _finish(rep, tol, strict=(mode != "fast"))
+    gpu.close()
