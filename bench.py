@@ -128,9 +128,15 @@ def iteration_bytes(cfg, batch: int, mean_ctx: float, kv_planes: int = 1) -> flo
             continue
         n = int(np.prod(shape))
         if name.endswith("we_gate_up") or name.endswith("we_down"):
-            continue  # MoE experts are counted by touched experts elsewhere
+            continue  # MoE experts: only the touched ones are read (below)
         w += n * es * (2 if name == "lm_head" else 1)
     t, d = cfg.target, cfg.drafter
+    if t.is_moe:
+        # expected experts a verify pass touches per layer when its batch*block rows
+        # each pick top_k of n_experts (near-uniform routing of random-init weights)
+        rows = batch * cfg.block_size
+        touched = t.n_experts * (1.0 - (1.0 - t.top_k / t.n_experts) ** rows)
+        w += t.n_layers * touched * 3 * t.hidden * t.expert_ffn * es
     kv = batch * (mean_ctx + cfg.block_size) * 2 * es * kv_planes * (t.n_layers * t.n_kv_heads * t.head_dim
                                                           + d.n_layers * d.n_kv_heads * d.head_dim)
     return float(w * (1 if batch else 0) + kv)

@@ -226,6 +226,8 @@ static Layout make_layout(const dflash_config &c) {
     L.moe_sel = take(mrows * 4);
     L.moe_wt = take(mrows * 4);
     L.moe_part = take(t.n_experts > 0 ? mrows * H * 4 : 16);
+    L.moe_off = take(t.n_experts > 0 ? (size_t)(t.n_experts + 1) * 4 : 16);
+    L.moe_list = take(mrows * 4);
     // per-(vocab tile, row) best logit of the LM-head GEMM
     L.lm_part = take((size_t)((t.vocab + 127) / 128) * std::max(L.R_dec, 1) * sizeof(float2));
     // split-KV attention partials (sized for 148 SMs; launches cap their splits to fit)
@@ -294,6 +296,7 @@ class Engine : public EngineBase {
     float *x, *Y, *logits, *plogits, *moe_wt, *moe_part;
     T *xn, *dq_in, *q, *ao, *h, *taps_dec, *taps_gather, *taps_pre, *cbuf, *tk, *tv, *dk, *dv;
     int *g, *drafts, *accept, *committed, *new_len, *active, *script, *out_tok, *tokens, *first_tok, *moe_sel;
+    int *moe_off = nullptr, *moe_list = nullptr;
     SeqState *st;
     RowMeta *meta, *ctx_meta, *ctx_meta_pre;
     float2 *rope_t, *rope_d;
@@ -396,6 +399,8 @@ class Engine : public EngineBase {
         tokens = sp<int>(L.tokens);
         first_tok = sp<int>(L.first_tok);
         moe_sel = sp<int>(L.moe_sel);
+        moe_off = sp<int>(L.moe_off);
+        moe_list = sp<int>(L.moe_list);
         st = sp<SeqState>(L.st);
         meta = sp<RowMeta>(L.meta);
         ctx_meta = sp<RowMeta>(L.ctx_meta);
@@ -684,6 +689,15 @@ class Engine : public EngineBase {
         e.ldy = E;
         gemm(xn, H, R, w.w_router, E, H, e);
         launch_moe_topk(Y, E, R, k, moe_sel, moe_wt, s);
+        if constexpr (std::is_same<T, bf16>::value) {
+            if (moe_bucketed_supported(H, Fe, E)) {
+                // touched experts only, each expert's weights streamed once per layer
+                launch_moe_experts_bucketed(xn, H, lo_, R, k, moe_sel, E, (const bf16 *)w.we_gate_up,
+                                            (const bf16 *)w.we_down, H, Fe, moe_off, moe_list, h, lo_, moe_part, s);
+                launch_moe_combine<T>(x, moe_part, moe_wt, H, R, k, taps, lo_, mt, s);
+                return;
+            }
+        }
         if (moe_tc_supported<T>()) {
             run_moe_tc<T>(xn, H, R, k, moe_sel, (const T *)w.we_gate_up, (const T *)w.we_down, H, Fe, E, h, moe_part,
                           tc, s);

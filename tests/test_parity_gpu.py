@@ -28,13 +28,13 @@ TOL = {"fp32": (1e-4, 1e-3), "bf16": (3e-2, 0.05)}
 
 
 def tiny_cfg(dtype="fp32", block=4, moe=False, t_layers=2, d_layers=1, nq=4, nkv=2, hd=64, hidden=256,
-             vocab=1024, taps=(0, 1)):
+             vocab=1024, taps=(0, 1), expert_ffn=64):
     base = get_config("tiny")
     ffn = 3 * hidden
     t = replace(base.target, n_layers=t_layers, n_q_heads=nq, n_kv_heads=nkv, head_dim=hd, hidden=hidden,
                 vocab=vocab, ffn=ffn)
     if moe:
-        t = replace(t, n_experts=8, top_k=2, expert_ffn=64)
+        t = replace(t, n_experts=8, top_k=2, expert_ffn=expert_ffn)
     d = replace(base.drafter, n_layers=d_layers, n_q_heads=nq, n_kv_heads=nkv, head_dim=hd, hidden=hidden,
                 vocab=vocab, ffn=ffn)
     return base.with_(target=t, drafter=d, block_size=block, tap_layers=taps, dtype=dtype)
@@ -66,14 +66,17 @@ def test_config1_generate_is_lossless(cuda_device):
     assert 1.0 <= st.mean_tau <= cfg.block_size
 
 
-@pytest.mark.parametrize("case", ["block16", "moe", "mha_hd128", "chunked_prefill", "batch3", "wide", "wide_batch2"])
+@pytest.mark.parametrize("case", ["block16", "moe", "moe_bucketed", "mha_hd128", "chunked_prefill", "batch3", "wide",
+                                  "wide_batch2"])
 def test_bf16_variants_replay(cuda_device, case):
     kw = dict(dtype="bf16")
     prompts_n, lens, chunk = 1, [40], 0
     if case == "block16":
         kw.update(block=16)
     if case == "moe":
-        kw.update(moe=True)
+        kw.update(moe=True)                   # expert FFN 64: CUDA-core expert kernel
+    if case == "moe_bucketed":
+        kw.update(moe=True, expert_ffn=256)   # bucketed experts (hidden and expert FFN multiples of 256)
     if case == "mha_hd128":
         kw.update(nq=2, nkv=2, hd=128)
     if case == "chunked_prefill":
