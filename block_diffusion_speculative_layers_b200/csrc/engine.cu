@@ -1356,12 +1356,22 @@ class Engine : public EngineBase {
         return check("decode loop");
     }
 
+    // CUDA events destroyed on every return path
+    struct ScopedEvents {
+        cudaEvent_t e[3] = {nullptr, nullptr, nullptr};
+        ScopedEvents() {
+            for (auto &x : e) cudaEventCreate(&x);
+        }
+        ~ScopedEvents() {
+            for (auto &x : e)
+                if (x) cudaEventDestroy(x);
+        }
+    };
+
     dflash_status generate(const int32_t *const *prompts, const int32_t *lens, int n, int max_new, int32_t *out,
                            dflash_stats *ost) override {
-        cudaEvent_t t0, t1, t2;
-        cudaEventCreate(&t0);
-        cudaEventCreate(&t1);
-        cudaEventCreate(&t2);
+        ScopedEvents ev;
+        cudaEvent_t t0 = ev.e[0], t1 = ev.e[1], t2 = ev.e[2];
         cudaEventRecord(t0, s);
         dflash_status r = start_run(prompts, lens, n, max_new);
         if (r) return r;
@@ -1393,9 +1403,6 @@ class Engine : public EngineBase {
             ost->ms_decode = b;
             ost->kernel_launches = launch_count();
         }
-        cudaEventDestroy(t0);
-        cudaEventDestroy(t1);
-        cudaEventDestroy(t2);
         // generation leaves the slots in a finished state: refuse draft/verify on them
         for (int i = 0; i < n; ++i) h_prefilled[i] = 0;
         if (hs.status) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
@@ -1404,9 +1411,8 @@ class Engine : public EngineBase {
 
     dflash_status generate_ar(const int32_t *const *prompts, const int32_t *lens, int n, int max_new, int32_t *out,
                               double *ms) override {
-        cudaEvent_t t1, t2;
-        cudaEventCreate(&t1);
-        cudaEventCreate(&t2);
+        ScopedEvents ev;
+        cudaEvent_t t1 = ev.e[0], t2 = ev.e[1];
         dflash_status r = start_run(prompts, lens, n, max_new);
         if (r) return r;
         cudaEventRecord(t1, s);
@@ -1425,8 +1431,6 @@ class Engine : public EngineBase {
             cudaEventElapsedTime(&b, t1, t2);
             *ms = b;
         }
-        cudaEventDestroy(t1);
-        cudaEventDestroy(t2);
         for (int i = 0; i < n; ++i) h_prefilled[i] = 0;
         return numeric_status();
     }

@@ -211,3 +211,44 @@ def test_alternative_execution_modes(cuda_device, mode, monkeypatch):
     print(f"{mode}: max |dlogit| {rep.max_dlogit:.4f}, near ties {rep.near_ties}/{rep.checked_tokens}")
     _finish(rep, tol, strict=(mode != "fast"))
     gpu.close()
+
+
+@pytest.mark.parametrize("block", [1, 2])
+def test_degenerate_block_sizes(cuda_device, block):
+    """B = 1: no drafts, every iteration commits the target's own token; B = 2:
+    a single draft per block.  Both stay lossless."""
+    cfg = tiny_cfg("bf16", block=block)
+    tol, tie = TOL["bf16"]
+    gpu, spec, _ = build_pair(cfg, max_len=128)
+    prompt = make_prompt("uniform", 24, cfg.target.vocab, 5)
+    rep = replay(gpu, spec, cfg, [prompt], 6, tol, tie)
+    _finish(rep, tol)
+    if block == 1:
+        assert all(a == 0 for a in rep.accepts)
+    k, st = check_lossless_generate(gpu, spec, cfg, prompt, 20, tie)
+    assert st.tokens == 19
+
+
+def test_one_token_prompt_and_short_generations(cuda_device):
+    """A one-token prompt, max_new = 1 (the prefill's token only) and max_new = 2."""
+    cfg = tiny_cfg("bf16", block=4)
+    tol, tie = TOL["bf16"]
+    gpu, spec, _ = build_pair(cfg, max_len=64)
+    prompt = make_prompt("uniform", 1, cfg.target.vocab, 8)
+    rep = replay(gpu, spec, cfg, [prompt], 3, tol, tie)
+    _finish(rep, tol)
+    for max_new in (1, 2):
+        k, st = check_lossless_generate(gpu, spec, cfg, prompt, max_new, tie)
+        assert st.tokens == max_new - 1  # the first token comes from the prefill
+
+
+def test_batch16_block16_uses_wide_row_tiles(cuda_device):
+    """16 sequences x 16 rows = 256 verify rows: the large-row-tile decode path of
+    the batch sweep, with ragged prompts."""
+    cfg = tiny_cfg("bf16", block=16)
+    tol, tie = TOL["bf16"]
+    gpu, spec, _ = build_pair(cfg, max_batch=16, max_len=128)
+    lens = [5 + 3 * i for i in range(16)]
+    prompts = [make_prompt("uniform", L, cfg.target.vocab, 40 + i) for i, L in enumerate(lens)]
+    rep = replay(gpu, spec, cfg, prompts, 2, tol, tie)
+    _finish(rep, tol)
