@@ -5,15 +5,18 @@
 // Roles per CTA (192 threads):
 //   warp 0      one thread issues TMA loads of the weight tile (two 64-row
 //               boxes) and the activation tile into a ring of stages;
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=TM,
-//               K=16) and commits each consumed stage back to the producer;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31 = weight rows), split-K reduction when the
-//               K range is split, then the fused epilogue (store / RoPE + KV
-//               write / residual + taps / SwiGLU / per-tile argmax).
-// Split-K partials are summed by the last-arriving CTA of a tile in split
-// order, so results are identical run to run.  Every mbarrier wait is bounded
-// (2 s of %globaltimer); on expiry the CTA records an error bit and drains.
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128 weight
+//               rows, N=TM activation rows, or N=2*TM over both planes of
+//               two-plane activations; K=16) and commits each consumed stage
+//               back to the producer;
+//   warps 2..5  epilogue: row scales of the folded RMSNorm and the inputs of
+//               the fused epilogue are loaded while the main loop runs; then
+//               tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31 = weight rows), the split-K exchange when the K
+//               range is split, and the fused epilogue (store / RoPE + KV write
+//               / residual + taps + next-norm inputs / SwiGLU / per-tile argmax).
+// Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
+// records an error bit and drains.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -29,19 +32,18 @@
 namespace dfl {
 namespace tc {
 
-// Work split.  Small projections (fewer tiles than SMs) run one tile per CTA
-// with the K range split over a thread-block cluster of p.splits CTAs along z:
-// each CTA accumulates its K range in TMEM, parks it in its shared memory, and
-// after a cluster barrier reduces a slice of the tile's columns over all CTAs
-// of the cluster (in rank order, so results are identical run to run) through
-// distributed shared memory, then runs the fused epilogue on that slice.
-// Large projections (p.splits == 1) are persistent: CTA b handles tiles
-// b, b + gridDim.x, ... with two TMEM accumulators, so the epilogue of one tile
-// overlaps the MMAs of the next while the TMA ring streams weights without a
-// break.  Grids never exceed one CTA per SM, which leaves room on every SM for
-// the next kernel's CTA to start streaming its weights early (programmatic
-// dependent launch: weights are loaded before griddepcontrol.wait,
-// activations after it).
+// Work split.  The host launches one CTA per (weight tile, activation-row
+// tile).  Projections with fewer tiles than two per SM split the K range over
+// a thread-block cluster of p.splits CTAs along z: each CTA accumulates its K
+// range in TMEM and pushes the columns other CTAs finish into their shared
+// memory; after one cluster barrier each CTA sums its columns over the cluster
+// in rank order (identical results run to run) and runs the fused epilogue on
+// them.  CTAs of ~110 KB leave room for the next kernel's CTA on the same SM,
+// which starts streaming its weights early (programmatic dependent launch:
+// weights are loaded before griddepcontrol.wait, activations after it).
+// A 1-D grid smaller than the tile count makes CTAs loop over tiles with two
+// TMEM accumulators (the epilogue of one tile overlapping the MMAs of the
+// next); the host policy does not use that form at present.
 template <int TM, int KIND>
 __global__ void __launch_bounds__(NT, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcParams p,
