@@ -2,19 +2,21 @@
 // m16n8k16, fp32 accumulate, online softmax), with split-KV across CTAs.
 //
 // One CTA serves one query tile (up to 16 consecutive rows of one sequence:
-// a draft/verify block, or 16 prompt rows) for one KV head; its warps are the
-// q heads that share that KV head (GQA), so each K/V tile is read from HBM once
-// for the whole group.  Row r sees keys [0, meta[r].nk): the target's verify
-// rows are causal (nk = pos + 1), the drafter's block rows are
-// block-bidirectional (nk = p + B: every committed context key and every key
-// of the block) -- "O que o DFlash faz de diferente" on the iaemfoco DFlash
-// page (the drafter fills the whole block in one parallel pass).
+// a draft/verify block, or 16 prompt rows) for one KV head and one share of
+// its keys; its warps are the q heads that share that KV head (GQA), in one or
+// two key groups, so each K/V tile is read from HBM once for the whole group.
+// Row r sees keys [0, meta[r].nk): the target's verify rows are causal
+// (nk = pos + 1), the drafter's block rows are block-bidirectional (nk = p + B:
+// every committed context key and every key of the block) -- "O que o DFlash
+// faz de diferente" on the iaemfoco DFlash page (the drafter fills the whole
+// block in one parallel pass).
 //
-// The KV range [0, max_len) is cut into n_splits chunks; each CTA writes an
-// unnormalised partial (o, running max, running sum) and the last CTA of the
-// (tile, kv head) combines the partials in split order (deterministic).
-// Attention reads K/V once per group and is bound by HBM traffic, which the
-// legacy tensor-core path covers; the projections use tcgen05 (gemm_tc.cu).
+// The visible keys are cut into n_splits shares (CTAs of one cluster); every
+// warp keeps an unnormalised partial (o, running max, running sum), pushes it
+// into the shared memory of the CTA that finishes its (head, row) pair, and
+// after one cluster barrier each CTA combines its pairs over all partials in a
+// fixed order (deterministic).  At 16 query rows the products are small; the
+// legacy tensor-core path (mma.sync) covers them, the projections use tcgen05.
 #include <math.h>
 
 #include "attn_mma.h"
