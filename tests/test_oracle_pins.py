@@ -388,3 +388,27 @@ def test_trained_like_drafter_partial_acceptance():
             n_out += a + 1
             anchor = int(g[a])
             assert anchor == ar[n_out - 1]
+
+
+# ---------------------------------------------------------------- property: lossless for any shape
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=12, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(block=st.integers(1, 8), kv=st.sampled_from([(4, 1), (4, 2), (4, 4), (2, 2)]), moe=st.booleans(),
+       taps=st.sampled_from([(0,), (1,), (0, 1), (1, 1, 0)]), t_layers=st.integers(1, 2),
+       prompt_len=st.integers(1, 12), seed=st.integers(0, 10_000))
+def test_spec_equals_target_only_for_random_shapes(block, kv, moe, taps, t_layers, prompt_len, seed):
+    """Draft-and-verify output equals target-only greedy output bit for bit for any
+    block size, GQA grouping, MoE routing, tap set and prompt; accept lengths stay
+    in [0, block-1].  (Taps beyond the last layer are clamped to it.)"""
+    nq, nkv = kv
+    taps = tuple(min(t, t_layers - 1) for t in taps)
+    cfg = tiny(block=block, nq=nq, nkv=nkv, moe=moe, taps=taps, t_layers=t_layers, vocab=256)
+    spec = oracle.OracleSpec(cfg, make_weights(cfg, seed=seed))
+    prompt = make_prompt("uniform", prompt_len, cfg.target.vocab, seed)
+    ar = spec.generate_ar(prompt, 24)
+    out, acc = spec.generate_spec(prompt, 24)
+    np.testing.assert_array_equal(out, ar)
+    assert ((acc >= 0) & (acc <= block - 1)).all()
