@@ -226,7 +226,7 @@ static Layout make_layout(const dflash_config &c) {
     L.moe_sel = take(mrows * 4);
     L.moe_wt = take(mrows * 4);
     L.moe_part = take(t.n_experts > 0 ? mrows * H * 4 : 16);
-    L.moe_off = take(t.n_experts > 0 ? (size_t)(t.n_experts + 1) * 4 : 16);
+    L.moe_off = take(t.n_experts > 0 ? (size_t)(2 * t.n_experts + 2) * 4 : 16);
     L.moe_list = take(mrows * 4);
     // per-(vocab tile, row) best logit of the LM-head GEMM
     L.lm_part = take((size_t)((t.vocab + 127) / 128) * std::max(L.R_dec, 1) * sizeof(float2));
@@ -693,7 +693,8 @@ class Engine : public EngineBase {
             if (moe_bucketed_supported(H, Fe, E)) {
                 // touched experts only, each expert's weights streamed once per layer
                 launch_moe_experts_bucketed(xn, H, lo_, R, k, moe_sel, E, (const bf16 *)w.we_gate_up,
-                                            (const bf16 *)w.we_down, H, Fe, moe_off, moe_list, h, lo_, moe_part, s);
+                                            (const bf16 *)w.we_down, H, Fe, moe_off, moe_list, h, lo_, moe_part,
+                                            num_sms, &stats->status, s);
                 launch_moe_combine<T>(x, moe_part, moe_wt, H, R, k, taps, lo_, mt, s);
                 return;
             }

@@ -86,12 +86,14 @@ void launch_moe_topk(const float *router_logits, int E, int R, int k, int *sel, 
 template <typename T>
 void launch_moe_experts_simt(const T *m, int ldm, size_t lo, int R, int k, const int *sel, const T *w_gate_up,
                              const T *w_down, int H, int Fe, float *part, cudaStream_t s);
-// Bucketed experts (bf16): pairs grouped by expert (off[E+1], list[R*k] scratch),
-// then gate/up -> h[pair][Fe] (two planes when hlo != 0) and down -> part[pair][H].
+// Bucketed experts (bf16, moe_experts.cu): pairs grouped by expert (off[2E+2]:
+// pair ranges then the touched-expert list; list[R*k] scratch), then gate/up ->
+// h[pair][Fe] (two planes when hlo != 0) and down -> part[pair][H], each a
+// persistent weight-streaming kernel of num_sms CTAs; timed-out waits set bit 4 of *err.
 bool moe_bucketed_supported(int H, int Fe, int E);
 void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k, const int *sel, int E,
                                  const bf16 *w_gate_up, const bf16 *w_down, int H, int Fe, int *off, int *list,
-                                 bf16 *h, size_t hlo, float *part, cudaStream_t s);
+                                 bf16 *h, size_t hlo, float *part, int num_sms, int *err, cudaStream_t s);
 template <typename T>
 void launch_moe_combine(float *x, const float *part, const float *wt, int H, int R, int k,
                         const TapDst<T> &taps, size_t lo, const RowMeta *meta, cudaStream_t s);

@@ -211,203 +211,6 @@ void launch_moe_experts_simt(const T *m, int ldm, size_t lo, int R, int k, const
              part);
 }
 
-// ------------------------------------------------------------------------
-// MoE experts, bucketed: every (row, choice) pair is listed under its expert,
-// then one CTA group per touched expert streams that expert's weights exactly
-// once (warp per weight row, 16-byte coalesced loads) and applies them to all
-// of the expert's rows staged in shared memory.  Experts no row routes to are
-// not read at all.
-// ------------------------------------------------------------------------
-constexpr int MOE_PC = 4;  // expert rows staged per pass
-
-// pairs rk = r*k + t grouped by expert: off[e] .. off[e+1]-1 index list[]
-__global__ void moe_bucket_kernel(const int *__restrict__ sel, int n_pairs, int E, int *off, int *list) {
-    pdl_trigger();
-    pdl_wait();
-    __shared__ int cnt[257], cur[256];
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) cnt[e] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) atomicAdd(&cnt[sel[i]], 1);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int e = 0; e < E; ++e) {
-            const int c = cnt[e];
-            cnt[e] = acc;
-            cur[e] = acc;
-            acc += c;
-        }
-        cnt[E] = acc;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) off[e] = cnt[e];
-    // the order of pairs within an expert does not matter: each pair has its own output row
-    for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) list[atomicAdd(&cur[sel[i]], 1)] = i;
-}
-
-__device__ __forceinline__ void bf16x8_to_f(const uint4 &u, float *f) {
-    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 t = __bfloat1622float2(b[i]);
-        f[2 * i] = t.x;
-        f[2 * i + 1] = t.y;
-    }
-}
-
-constexpr int MOE_CPL = 12;  // 16-byte weight chunks per lane and row (rows of up to 3072 bf16)
-
-// x rows of pairs c0 .. c0+nc-1 of the expert into xs[j][0..n) (fp32, both planes summed):
-// 16-byte loads of every staged row issued before any is used (n % 8 == 0, rows 16-byte aligned)
-template <typename T>
-__device__ __forceinline__ void moe_stage(const T *__restrict__ src, int ld, size_t lo, const int *__restrict__ list,
-                                          int p0, int c0, int nc, int div, int n, float *xs) {
-    int row[MOE_PC];
-#pragma unroll
-    for (int j = 0; j < MOE_PC; ++j) row[j] = j < nc ? list[p0 + c0 + j] / div : 0;
-    for (int c = threadIdx.x; c < n / 8; c += blockDim.x) {
-        uint4 hi[MOE_PC], lw[MOE_PC];
-#pragma unroll
-        for (int j = 0; j < MOE_PC; ++j) {
-            if (j >= nc) break;
-            const size_t at = (size_t)row[j] * ld + (size_t)c * 8;
-            hi[j] = *reinterpret_cast<const uint4 *>(src + at);
-            if (lo) lw[j] = *reinterpret_cast<const uint4 *>(src + lo + at);
-        }
-#pragma unroll
-        for (int j = 0; j < MOE_PC; ++j) {
-            if (j >= nc) break;
-            float a[8], b[8];
-            bf16x8_to_f(hi[j], a);
-            if (lo) bf16x8_to_f(lw[j], b);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) xs[j * n + c * 8 + t] = lo ? a[t] + b[t] : a[t];
-        }
-    }
-}
-
-// dot products of one weight row (in registers: lane's chunks q*32 + lane) with nc staged rows
-__device__ __forceinline__ void moe_dots(const uint4 *wr, int cpl, const float *xs, int n, int nc, float *acc) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int q = 0; q < MOE_CPL; ++q) {
-        if (q >= cpl) break;
-        float a[8];
-        bf16x8_to_f(wr[q], a);
-        const int col = (q * 32 + lane) * 8;
-#pragma unroll
-        for (int j = 0; j < MOE_PC; ++j) {
-            if (j >= nc) break;
-            const float4 x0 = *reinterpret_cast<const float4 *>(xs + j * n + col);
-            const float4 x1 = *reinterpret_cast<const float4 *>(xs + j * n + col + 4);
-            acc[j] += a[0] * x0.x + a[1] * x0.y + a[2] * x0.z + a[3] * x0.w + a[4] * x1.x + a[5] * x1.y + a[6] * x1.z +
-                      a[7] * x1.w;
-        }
-    }
-}
-
-// gate/up of expert blockIdx.x, one warp per column f = blockIdx.y * 8 + warp:
-// h[pair][f] = SiLU(W_gate[f] . m[row]) * (W_up[f] . m[row]) for every pair of the expert.
-// Both weight rows are loaded before the expert's rows are staged.  H % 256 == 0.
-template <typename T>
-__global__ void __launch_bounds__(256) moe_gateup_kernel(const T *__restrict__ m, int ldm, size_t lo, int k,
-                                                         const int *__restrict__ off, const int *__restrict__ list,
-                                                         const T *__restrict__ w_gate_up, int H, int Fe,
-                                                         T *__restrict__ h, size_t hlo) {
-    pdl_trigger();
-    pdl_wait();
-    extern __shared__ float xs[];  // [MOE_PC][H]
-    const int e = blockIdx.x;
-    const int p0 = off[e], np = off[e + 1] - p0;
-    if (np == 0) return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int f = blockIdx.y * 8 + warp;
-    const int cpl = H / 256;
-    uint4 wg[MOE_CPL], wu[MOE_CPL];
-    if (f < Fe) {
-        const uint4 *g = reinterpret_cast<const uint4 *>(w_gate_up + ((size_t)e * 2 * Fe + f) * H);
-        const uint4 *u = reinterpret_cast<const uint4 *>(w_gate_up + ((size_t)e * 2 * Fe + Fe + f) * H);
-#pragma unroll
-        for (int q = 0; q < MOE_CPL; ++q)
-            if (q < cpl) {
-                wg[q] = __ldg(g + q * 32 + lane);
-                wu[q] = __ldg(u + q * 32 + lane);
-            }
-    }
-    for (int c0 = 0; c0 < np; c0 += MOE_PC) {
-        const int nc = min(MOE_PC, np - c0);
-        __syncthreads();
-        moe_stage(m, ldm, lo, list, p0, c0, nc, k, H, xs);
-        __syncthreads();
-        if (f >= Fe) continue;
-        float gs[MOE_PC], us[MOE_PC];
-#pragma unroll
-        for (int j = 0; j < MOE_PC; ++j) gs[j] = us[j] = 0.f;
-        moe_dots(wg, cpl, xs, H, nc, gs);
-        moe_dots(wu, cpl, xs, H, nc, us);
-#pragma unroll
-        for (int j = 0; j < MOE_PC; ++j) {
-            const float a = warp_sum(gs[j]), b = warp_sum(us[j]);
-            if (lane == 0 && j < nc) st_act(h, (size_t)list[p0 + c0 + j] * Fe + f, hlo, silu_f(a) * b);
-        }
-    }
-}
-
-// down of expert blockIdx.x, one warp per output o = blockIdx.y * 8 + warp:
-// part[pair][o] = W_down[o] . h[pair].  Fe % 256 == 0.
-template <typename T>
-__global__ void __launch_bounds__(256) moe_down_kernel(const T *__restrict__ h, size_t hlo, const int *__restrict__ off,
-                                                       const int *__restrict__ list, const T *__restrict__ w_down,
-                                                       int H, int Fe, float *__restrict__ part) {
-    pdl_trigger();
-    pdl_wait();
-    extern __shared__ float hs[];  // [MOE_PC][Fe]
-    const int e = blockIdx.x;
-    const int p0 = off[e], np = off[e + 1] - p0;
-    if (np == 0) return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int o = blockIdx.y * 8 + warp;
-    const int cpl = Fe / 256;
-    uint4 wr[MOE_CPL];
-    if (o < H) {
-        const uint4 *w = reinterpret_cast<const uint4 *>(w_down + ((size_t)e * H + o) * Fe);
-#pragma unroll
-        for (int q = 0; q < MOE_CPL; ++q)
-            if (q < cpl) wr[q] = __ldg(w + q * 32 + lane);
-    }
-    for (int c0 = 0; c0 < np; c0 += MOE_PC) {
-        const int nc = min(MOE_PC, np - c0);
-        __syncthreads();
-        moe_stage(h, Fe, hlo, list, p0, c0, nc, 1, Fe, hs);
-        __syncthreads();
-        if (o >= H) continue;
-        float acc[MOE_PC];
-#pragma unroll
-        for (int j = 0; j < MOE_PC; ++j) acc[j] = 0.f;
-        moe_dots(wr, cpl, hs, Fe, nc, acc);
-#pragma unroll
-        for (int j = 0; j < MOE_PC; ++j) {
-            const float sum = warp_sum(acc[j]);
-            if (lane == 0 && j < nc) part[(size_t)list[p0 + c0 + j] * H + o] = sum;
-        }
-    }
-}
-
-bool moe_bucketed_supported(int H, int Fe, int E) {
-    return H % 256 == 0 && Fe % 256 == 0 && H <= 256 * MOE_CPL && Fe <= 256 * MOE_CPL && E <= 256;
-}
-
-void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k, const int *sel, int E,
-                                 const bf16 *w_gate_up, const bf16 *w_down, int H, int Fe, int *off, int *list,
-                                 bf16 *h, size_t hlo, float *part, cudaStream_t s) {
-    if (R <= 0) return;
-    launch_k(moe_bucket_kernel, dim3(1), dim3(1024), 0, s, 1, sel, R * k, E, off, list);
-    launch_k(moe_gateup_kernel<bf16>, dim3(E, (Fe + 7) / 8), dim3(256), sizeof(float) * MOE_PC * H, s, 1, m, ldm, lo,
-             k, (const int *)off, (const int *)list, w_gate_up, H, Fe, h, hlo);
-    launch_k(moe_down_kernel<bf16>, dim3(E, (H + 7) / 8), dim3(256), sizeof(float) * MOE_PC * Fe, s, 1,
-             (const bf16 *)h, hlo, (const int *)off, (const int *)list, w_down, H, Fe, part);
-}
-
 template <typename T>
 __global__ void moe_combine_kernel(float *__restrict__ x, const float *__restrict__ part,
                                    const float *__restrict__ wt, int H, int k, TapDst<T> taps, size_t lo,
