@@ -36,11 +36,12 @@ namespace dfl {
 
 namespace {
 
-constexpr int XR = 8;           // expert rows staged per pass
+constexpr int XR = 4;           // expert rows staged per pass
 constexpr int MAX_CPL = 12;     // 16-byte chunks per lane and weight row (rows of up to 3072 bf16)
 constexpr int MAX_STAGES = 8;
 constexpr int NTHREADS = 256;   // 8 warps
-constexpr size_t SMEM_BUDGET = 220 * 1024;
+constexpr int CTAS_PER_SM = 2;  // two independent item chains per SM
+constexpr size_t SMEM_BUDGET = 110 * 1024;
 
 struct MoeStream {
     const bf16 *x;      // activation rows: m[row] (gate/up; row = pair / k) or h[pair] (down)
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(256) moe_down_kernel(const T *__restrict__ h, 
 // Weight-streaming experts, for sparse routing (decode): see the file header.
 // ------------------------------------------------------------------------
 template <bool GU>
-__global__ void __launch_bounds__(NTHREADS, 1) moe_stream_kernel(const MoeStream a) {
+__global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) moe_stream_kernel(const MoeStream a) {
     pdl_trigger();
     extern __shared__ __align__(128) unsigned char sm[];
     constexpr int ROWS = GU ? 8 : 16;  // weight rows per item
@@ -472,7 +473,7 @@ void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k
     a.part = part;
     a.err = err;
     a.stages = stream_stages(H, 8, E);
-    launch_k(moe_stream_kernel<true>, dim3(num_sms), dim3(NTHREADS), stream_smem(H, 8, E, a.stages), s, 1, a);
+    launch_k(moe_stream_kernel<true>, dim3(CTAS_PER_SM * num_sms), dim3(NTHREADS), stream_smem(H, 8, E, a.stages), s, 1, a);
     MoeStream d = a;
     d.x = h;
     d.ldx = Fe;
@@ -480,7 +481,7 @@ void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k
     d.div = 1;
     d.w = w_down;
     d.stages = stream_stages(Fe, 16, E);
-    launch_k(moe_stream_kernel<false>, dim3(num_sms), dim3(NTHREADS), stream_smem(Fe, 16, E, d.stages), s, 1, d);
+    launch_k(moe_stream_kernel<false>, dim3(CTAS_PER_SM * num_sms), dim3(NTHREADS), stream_smem(Fe, 16, E, d.stages), s, 1, d);
 }
 
 }  // namespace dfl
