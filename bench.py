@@ -423,7 +423,16 @@ def workload_config(cfg, args, world):
             "parallelism": f"replicas x{world}",
             "activations": ("bf16 hi+lo planes, fp32 accumulate" if args.bf16_act == "split"
                             else "bf16 single plane, fp32 accumulate") if cfg.dtype == "bf16" else "fp32",
-            "l2": "inputs larger than L2 (18.5 GB of weights streamed per step)"}
+            "l2": l2_note(cfg, 2 if cfg.dtype == "bf16" and args.bf16_act == "split" else 1)}
+
+
+def l2_note(cfg, kv_planes: int = 1, l2_bytes: float = 126e6) -> str:
+    """How the timed steps relate to the 126 MB L2: the bytes one iteration
+    streams (weights + K/V at the prompt length) against its size."""
+    gb = iteration_bytes(cfg, cfg.batch, cfg.prompt_len, kv_planes) / 1e9
+    if gb * 1e9 > l2_bytes:
+        return f"inputs larger than L2 ({gb:.1f} GB streamed per step)"
+    return f"inputs fit in L2 ({gb * 1e3:.0f} MB per step, no flush)"
 
 
 def run_reference(args, cfg, world, rank):
