@@ -1,7 +1,8 @@
 // kernels_simt.cu -- CUDA-core kernels for fp32 models (the tiny correctness
 // configuration computes in fp32 end to end, where tensor-core bf16 inputs
-// would change the model): GEMM, attention and MoE experts.  bf16 models use
-// the tensor-core kernels in gemm_tc.cu and attn_mma.cu instead.
+// would change the model): GEMM, attention and MoE experts, plus the MoE
+// combine every dtype uses.  bf16 models use the tensor-core kernels in
+// gemm_tc.cu and attn_mma.cu and the expert kernels in moe_experts.cu instead.
 #include <math.h>
 
 #include "kernels.h"
