@@ -1,4 +1,5 @@
-"""ctypes front end of the fp64 CPU oracle (dflash_oracle.c).
+"""ctypes front end of the fp64 CPU oracle (dflash_oracle.c), plus the
+temperature-sampling rule and its counter-based random numbers (sampling.py).
 
 TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
 benchmark's CPU-baseline leg.  The product package never imports it, and this
