@@ -33,7 +33,7 @@ EXPORTS = [
     "dflash_draft_block", "dflash_verify_commit", "dflash_generate", "dflash_generate_ar",
     "dflash_set_draft_mode", "dflash_set_script", "dflash_debug_logits", "dflash_seq_state",
     "dflash_debug_kv", "dflash_decode_iters", "dflash_get_stats", "dflash_reset_stats",
-    "dflash_profile", "dflash_profile_read", "dflash_head_argmax_noalloc",
+    "dflash_profile", "dflash_profile_read", "dflash_head_argmax_noalloc", "dflash_set_sampling",
 ]
 
 
@@ -55,7 +55,7 @@ class Config(C.Structure):
                 ("n_taps", C.c_int32), ("tap_layers", C.c_int32 * MAX_TAPS),
                 ("mask_token_id", C.c_int32), ("max_batch", C.c_int32), ("max_len", C.c_int32),
                 ("prefill_chunk", C.c_int32), ("dtype", C.c_int32), ("keep_logits", C.c_int32),
-                ("timeout_ms", C.c_int32)]
+                ("timeout_ms", C.c_int32), ("sampling", C.c_int32)]
 
 
 class Stats(C.Structure):
@@ -110,6 +110,7 @@ def load_library(path: Optional[str] = None):
         "dflash_profile": (_i32, [_vp, _i32]),
         "dflash_profile_read": (_i32, [_vp, C.POINTER(KernelProf)]),
         "dflash_head_argmax_noalloc": (_i32, [_vp, _i32, _ip, _ip]),
+        "dflash_set_sampling": (_i32, [_vp, C.c_double, C.c_uint64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -125,7 +126,8 @@ def _model_cfg(d) -> ModelCfg:
 
 
 def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: int = 0,
-                keep_logits: bool = False, timeout_ms: int = 0, bf16_act: str = "split") -> Config:
+                keep_logits: bool = False, timeout_ms: int = 0, bf16_act: str = "split",
+                sampling: bool = False) -> Config:
     """dflash_config from any object with target/drafter dims, block_size, tap_layers,
     mask_id and dtype ("bf16" / "fp32") attributes.  bf16_act selects how a bf16
     model carries its activations: "split" (two bf16 planes, DFLASH_BF16) or
@@ -151,6 +153,7 @@ def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: in
     else:
         c.dtype = DFLASH_FP32
     c.keep_logits = 1 if keep_logits else 0
+    c.sampling = 1 if sampling else 0
     c.timeout_ms = timeout_ms
     return c
 
@@ -168,10 +171,12 @@ class DFlash:
 
     def __init__(self, spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: int = 0,
                  keep_logits: bool = False, device: Optional[torch.device] = None,
-                 stream: Optional[torch.cuda.Stream] = None, timeout_ms: int = 0, bf16_act: str = "split"):
+                 stream: Optional[torch.cuda.Stream] = None, timeout_ms: int = 0, bf16_act: str = "split",
+                 sampling: bool = False):
         self.lib = load_library()
         self.spec = spec
-        self.cfg = make_config(spec, max_batch, max_len, prefill_chunk, keep_logits, timeout_ms, bf16_act)
+        self.cfg = make_config(spec, max_batch, max_len, prefill_chunk, keep_logits, timeout_ms, bf16_act,
+                               sampling)
         self.device = torch.device(device or "cuda")
         wb, sb = _sz(), _sz()
         self._check(self.lib.dflash_workspace_size(C.byref(self.cfg), C.byref(wb), C.byref(sb)),
@@ -342,6 +347,11 @@ class DFlash:
 
     def set_draft_mode(self, mode: int, tau: int = 1):
         self._check(self.lib.dflash_set_draft_mode(self.h, mode, tau), "dflash_set_draft_mode")
+
+    def set_sampling(self, temperature: float, seed: int = 0):
+        """Temperature sampling (needs sampling=True at construction); 0 = greedy."""
+        self._check(self.lib.dflash_set_sampling(self.h, float(temperature), int(seed) & (2 ** 64 - 1)),
+                    "dflash_set_sampling")
 
     def set_script(self, seq: int, script: Sequence[int]):
         s = _ints(script)

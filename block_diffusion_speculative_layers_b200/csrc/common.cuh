@@ -83,6 +83,41 @@ __device__ __forceinline__ void argmax_merge(float &v, int &i, float v2, int i2)
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
 
+// Commit one block of sequence i (slot s): drafts d[0..a) were accepted and x
+// follows them.  Records the committed row (tokens, then -1), emits the tokens
+// up to max_new, makes x the next anchor and moves the length and the pending
+// drafter-context rows by a + 1; a finished sequence only gets its row.
+__device__ __forceinline__ void commit_block(SeqState &S, int s, int i, int a, const int *d, int x, int B,
+                                             int *committed, int *out_tok, int out_ld, DevStats *stats) {
+    if (committed)
+        for (int k = 0; k < B; ++k) committed[i * B + k] = (k < a) ? d[k] : (k == a ? x : -1);
+    if (S.done) return;
+    int emitted = 0;
+    for (int k = 0; k <= a; ++k) {
+        const int tok = (k < a) ? d[k] : x;
+        if (S.n_out < S.max_new) {
+            out_tok[(size_t)s * out_ld + S.n_out] = tok;
+            S.n_out++;
+            emitted++;
+        }
+    }
+    S.anchor = x;
+    if (S.n_out >= S.max_new) {
+        S.done = 1;
+        S.pend_n = 0;
+        if (stats) atomicAdd(&stats->n_done, 1);
+    } else {
+        S.pend_pos0 = S.len;
+        S.pend_n = a + 1;
+        S.len += a + 1;
+    }
+    if (stats) {
+        atomicAdd(&stats->iterations, 1ull);
+        atomicAdd(&stats->tokens, (unsigned long long)emitted);
+        atomicAdd(&stats->hist[a], 1ull);
+    }
+}
+
 }  // namespace dfl
 
 namespace dfl {

@@ -205,6 +205,17 @@ static Layout make_layout(const dflash_config &c) {
     L.Y = take(R * (size_t)ycols * 4);
     L.logits = take((size_t)L.R_dec * t.vocab * 4);
     L.plogits = take((size_t)t.vocab * 4);
+    {
+        // temperature sampling: drafter logits kept through the verify pass, per-row
+        // log-sum-exp, chunk partials of the sampling passes, target and residual draws
+        const size_t rs = c.sampling ? (size_t)L.R_dec : 0, nc = (size_t)sample_chunks(t.vocab);
+        L.qlogits = take(rs * t.vocab * 4);
+        L.lse_p = take(rs * 4);
+        L.lse_q = take(rs * 4);
+        L.samp_part = take(std::max(rs, (size_t)1) * nc * 16);
+        L.tok_p = take(rs * 4);
+        L.resid = take(rs * 4);
+    }
     L.g = take((size_t)L.R_dec * 4);
     L.drafts = take((size_t)nb * B * 4);
     L.accept = take((size_t)nb * 4);
@@ -294,6 +305,9 @@ class Engine : public EngineBase {
     std::vector<LayerW> tl, dl;
     // state
     float *x, *Y, *logits, *plogits, *moe_wt, *moe_part;
+    float *qlogits = nullptr, *lse_p = nullptr, *lse_q = nullptr;
+    float4 *samp_part = nullptr;
+    int *tok_p = nullptr, *resid = nullptr;
     T *xn, *dq_in, *q, *ao, *h, *taps_dec, *taps_gather, *taps_pre, *cbuf, *tk, *tv, *dk, *dv;
     int *g, *drafts, *accept, *committed, *new_len, *active, *script, *out_tok, *tokens, *first_tok, *moe_sel;
     int *moe_off = nullptr, *moe_list = nullptr;
@@ -373,6 +387,14 @@ class Engine : public EngineBase {
         Y = sp<float>(L.Y);
         logits = sp<float>(L.logits);
         plogits = sp<float>(L.plogits);
+        if (c.sampling) {
+            qlogits = sp<float>(L.qlogits);
+            lse_p = sp<float>(L.lse_p);
+            lse_q = sp<float>(L.lse_q);
+            tok_p = sp<int>(L.tok_p);
+            resid = sp<int>(L.resid);
+        }
+        samp_part = sp<float4>(L.samp_part);
         moe_wt = sp<float>(L.moe_wt);
         moe_part = sp<float>(L.moe_part);
         xn = sp<T>(L.xn);
@@ -484,7 +506,7 @@ class Engine : public EngineBase {
         tc.tune_ctas_per_sm = env_int("DFLASH_TC_CTAS_PER_SM");
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);
-        tc.keep_logits = c.keep_logits;
+        tc.keep_logits = c.keep_logits || c.sampling;
         return check("create");
     }
 
@@ -749,22 +771,95 @@ class Engine : public EngineBase {
     }
 
     // LM head on normalised rows xin[R][H] -> greedy ids (mode 0: idx[r];
-    // mode 1: drafter rows j >= 1 of each block -> idx[i*(B-1)+j-1]).
-    void head_argmax(const T *xin, int R, float *lg, int mode, int B, int *idx) {
+    // mode 1: drafter rows j >= 1 of each block -> idx[i*(B-1)+j-1]), or with
+    // smp the temperature-sampled ids of the same rows.
+    void head_argmax(const T *xin, int R, float *lg, int mode, int B, int *idx, const SampleRows *smp = nullptr) {
         const int H = c.target.hidden, V = c.target.vocab;
         Epi<T> e;
         e.kind = EPI_LOGITS;
         e.Y = lg;
         e.ldy = V;
         gemm(xin, H, R, lm_head, V, H, e);
-        if (tc.supports(R, V, H)) launch_lm_argmax(lm_part, (V + 127) / 128, R, mode, B, idx, stats, s);
+        if (smp) launch_sample_rows(*smp, s);
+        else if (tc.supports(R, V, H)) launch_lm_argmax(lm_part, (V + 127) / 128, R, mode, B, idx, stats, s);
         else launch_argmax_rows(lg, V, V, R, mode, B, idx, stats, s);
     }
 
-    void lm_head_rows(const float *final_norm, float eps, int R, float *lg, int mode, int B, int *idx) {
+    void lm_head_rows(const float *final_norm, float eps, int R, float *lg, int mode, int B, int *idx,
+                      const SampleRows *smp = nullptr) {
         const int H = c.target.hidden;
         launch_rmsnorm<T>(x, H, final_norm, H, eps, xn, H, lo_, R, s);
-        head_argmax(xn, R, lg, mode, B, idx);
+        head_argmax(xn, R, lg, mode, B, idx, smp);
+    }
+
+    // ---- temperature sampling ----
+    bool sampling_on() const { return temperature > 0.f; }
+    float *draft_logits() { return c.sampling ? qlogits : logits; }
+
+    // rows [R] of logits lg (block B, row k of sequence i drawn at st.len + k + pos_off)
+    SampleRows sample_desc(const float *lg, int R, int B, int mode, uint32_t purpose, int pos_off, int *tok,
+                           float *lse) {
+        SampleRows a;
+        a.logits = lg;
+        a.ldl = a.V = c.target.vocab;
+        a.R = R;
+        a.B = B;
+        a.mode = mode;
+        a.inv_T = 1.f / temperature;
+        a.key = sample_key(seed);
+        a.purpose = purpose;
+        a.pos_off = pos_off;
+        a.st = st;
+        a.active = active;
+        a.part = samp_part;
+        a.lse = lse;
+        a.tok = tok;
+        a.stats = stats;
+        return a;
+    }
+
+    // after the verify head's draws (tok_p, lse_p): residual draws and the acceptance
+    void accept_sampled(int nseq) {
+        const int B = c.block_size, V = c.target.vocab;
+        if (B > 1) {
+            ResidualRows r;
+            r.plog = logits;
+            r.qlog = qlogits;
+            r.ldl = r.V = V;
+            r.B = B;
+            r.rows = nseq * (B - 1);
+            r.inv_T = 1.f / temperature;
+            r.key = sample_key(seed);
+            r.lse_p = lse_p;
+            r.lse_q = lse_q;
+            r.st = st;
+            r.active = active;
+            r.part = reinterpret_cast<float2 *>(samp_part);
+            r.resid = resid;
+            launch_residual_rows(r, s);
+        }
+        AcceptSample a;
+        a.st = st;
+        a.active = active;
+        a.nseq = nseq;
+        a.B = B;
+        a.drafts = drafts;
+        a.plog = logits;
+        a.qlog = qlogits;
+        a.ldl = V;
+        a.lse_p = lse_p;
+        a.lse_q = lse_q;
+        a.inv_T = 1.f / temperature;
+        a.key = sample_key(seed);
+        a.resid = resid;
+        a.tok_p = tok_p;
+        a.accept = accept;
+        a.committed = committed;
+        a.new_len = new_len;
+        a.out_tok = out_tok;
+        a.out_ld = c.max_len;
+        a.stats = stats;
+        launch_accept_sample(a, s);
     }
 
     // ---- persistent projection chains (bf16 decode) ----
@@ -794,7 +889,7 @@ class Engine : public EngineBase {
             p.splits = 1;
             p.err = &stats->status;
             p.lm_part = lm_part;
-            p.keep_logits = c.keep_logits;
+            p.keep_logits = c.keep_logits || c.sampling;
             const long long total = (long long)p.n_tiles * p.k_steps;
             // ops with fewer tile-k-steps than SMs use only the first `total` CTAs, so
             // the CTAs covering a tile are always consecutive (slot = CTA - first CTA)
@@ -989,7 +1084,7 @@ class Engine : public EngineBase {
                 chain_add(pg, toff, EPI_RESID, dl[j].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, xg_t, d_final, ssq));
                 Epi<T> lg;
                 lg.kind = EPI_LOGITS;
-                lg.Y = logits;
+                lg.Y = draft_logits();
                 lg.ldy = c.target.vocab;
                 chain_add(pg, toff, EPI_LOGITS, lm_head, c.target.vocab, H, xg_t, H, R, epi_norm_in(lg, (float)m.rms_eps, H));
             }
@@ -1066,8 +1161,13 @@ class Engine : public EngineBase {
             pass_done(pv, ai, k);
             run_ops(pv, 1 + 4 * l, 5 + 4 * l);
         }
-        launch_lm_argmax(lm_part, (t.vocab + 127) / 128, R, 0, B, g, stats, s);
-        launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
+        if (sampling_on()) {
+            launch_sample_rows(sample_desc(logits, R, B, 0, SP_TARGET, 1, tok_p, lse_p), s);
+            accept_sampled(nseq);
+        } else {
+            launch_lm_argmax(lm_part, (t.vocab + 127) / 128, R, 0, B, g, stats, s);
+            launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
+        }
         chain_used[1] = true;
     }
 
@@ -1088,7 +1188,12 @@ class Engine : public EngineBase {
             pass_done(pd, ai, k);
             run_ops(pd, 2 + 4 * j, 6 + 4 * j);
         }
-        if (B > 1) launch_lm_argmax(lm_part, (c.target.vocab + 127) / 128, R, 1, B, drafts, stats, s);
+        if (B > 1) {
+            if (sampling_on())
+                launch_sample_rows(sample_desc(qlogits, R, B, 1, SP_DRAFT, 0, drafts, lse_q), s);
+            else
+                launch_lm_argmax(lm_part, (c.target.vocab + 127) / 128, R, 1, B, drafts, stats, s);
+        }
         if (draft_mode == DFLASH_DRAFT_SCRIPT)
             launch_script_drafts(st, active, nseq, B, tau, c.target.vocab, script, c.max_len, drafts, s);
         chain_used[0] = true;
@@ -1104,9 +1209,16 @@ class Engine : public EngineBase {
             launch_embed_tokens<T>(embed, H, tokens + c0, R, seq, c0, x, meta, s);
             for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, 16, meta, taps_pre, TK);
             if (c0 + R == n) {
-                // greedy first token from the last prompt row
+                // first token from the last prompt row: greedy, or the target's draw at position n
                 launch_rmsnorm<T>(x + (size_t)(R - 1) * H, H, t_final, H, (float)t.rms_eps, xn, H, lo_, 1, s);
-                head_argmax(xn, 1, plogits, 0, 1, first_tok);
+                if (sampling_on()) {
+                    SampleRows a = sample_desc(plogits, 1, 1, 0, SP_TARGET, 0, first_tok, nullptr);
+                    a.fixed_pos = n;
+                    a.fixed_slot = seq;
+                    head_argmax(xn, 1, plogits, 0, 1, first_tok, &a);
+                } else {
+                    head_argmax(xn, 1, plogits, 0, 1, first_tok);
+                }
             }
             // context vectors of the prompt rows -> drafter context K/V
             Epi<T> f;
@@ -1160,7 +1272,14 @@ class Engine : public EngineBase {
         gemm(tin, TK, R, w_fc, H, TK, f);
         launch_rmsnorm<T>(Y, H, fc_norm, H, (float)d.rms_eps, dq_in + (size_t)R * H, H, lo_, R, s);
         for (int j = 0; j < d.n_layers; ++j) drafter_layer(j, R, true);
-        if (B > 1) lm_head_rows(d_final, (float)d.rms_eps, R, logits, 1, B, drafts);
+        if (B > 1) {
+            if (sampling_on()) {
+                const SampleRows a = sample_desc(qlogits, R, B, 1, SP_DRAFT, 0, drafts, lse_q);
+                lm_head_rows(d_final, (float)d.rms_eps, R, qlogits, 1, B, drafts, &a);
+            } else {
+                lm_head_rows(d_final, (float)d.rms_eps, R, draft_logits(), 1, B, drafts);
+            }
+        }
         if (draft_mode == DFLASH_DRAFT_SCRIPT)
             launch_script_drafts(st, active, nseq, B, tau, t.vocab, script, c.max_len, drafts, s);
     }
@@ -1176,8 +1295,14 @@ class Engine : public EngineBase {
         const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
         launch_embed_block<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
         for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, B, meta, taps_dec, TK);
-        lm_head_rows(t_final, (float)t.rms_eps, R, logits, 0, B, g);
-        launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
+        if (sampling_on()) {
+            const SampleRows a = sample_desc(logits, R, B, 0, SP_TARGET, 1, tok_p, lse_p);
+            lm_head_rows(t_final, (float)t.rms_eps, R, logits, 0, B, tok_p, &a);
+            accept_sampled(nseq);
+        } else {
+            lm_head_rows(t_final, (float)t.rms_eps, R, logits, 0, B, g);
+            launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
+        }
     }
 
     void enqueue_ar_step(int nseq) {
@@ -1185,7 +1310,12 @@ class Engine : public EngineBase {
         const int H = t.hidden;
         launch_embed_block<T>(embed, H, st, active, nseq, 1, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
         for (int l = 0; l < t.n_layers; ++l) target_layer(l, nseq, 1, meta, nullptr, 0);
-        lm_head_rows(t_final, (float)t.rms_eps, nseq, logits, 0, 1, g);
+        if (sampling_on()) {
+            const SampleRows a = sample_desc(logits, nseq, 1, 0, SP_TARGET, 1, g, nullptr);
+            lm_head_rows(t_final, (float)t.rms_eps, nseq, logits, 0, 1, g, &a);
+        } else {
+            lm_head_rows(t_final, (float)t.rms_eps, nseq, logits, 0, 1, g);
+        }
         launch_ar_step(st, active, nseq, g, out_tok, c.max_len, stats, s);
     }
 
@@ -1444,7 +1574,7 @@ class Engine : public EngineBase {
         if (nr * V > cap) { err = "output buffer too small"; return DFLASH_EINVAL; }
         dflash_status r = sync("debug_logits");
         if (r) return r;
-        const float *src = which == 2 ? plogits : logits;
+        const float *src = which == 2 ? plogits : (which == 0 && c.sampling ? qlogits : logits);
         if (cudaMemcpy(out, src, sizeof(float) * nr * V, cudaMemcpyDeviceToHost) != cudaSuccess)
             return fail_cuda("logits copy");
         if (rows) *rows = nr;
@@ -1782,8 +1912,32 @@ dflash_status dflash_set_draft_mode(dflash_ctx *ctx, int32_t mode, int32_t tau) 
     if (!ctx) return DFLASH_EINVAL;
     if ((mode != DFLASH_DRAFT_MODEL && mode != DFLASH_DRAFT_SCRIPT) || tau < 1 || tau > ctx->cfg.block_size)
         return DFLASH_EINVAL;
+    if (mode == DFLASH_DRAFT_SCRIPT && ctx->eng->temperature > 0.f) {
+        ctx->err = "script drafts are for greedy decoding (temperature is above 0)";
+        return DFLASH_ESTATE;
+    }
     ctx->eng->draft_mode = mode;
     ctx->eng->tau = tau;
+    return DFLASH_OK;
+}
+
+dflash_status dflash_set_sampling(dflash_ctx *ctx, double temperature, uint64_t seed) {
+    if (!ctx) return DFLASH_EINVAL;
+    if (!(temperature >= 0.0) || temperature > 1e30) {
+        ctx->err = "temperature must be a finite number >= 0";
+        return DFLASH_EINVAL;
+    }
+    if (temperature > 0.0 && !ctx->cfg.sampling) {
+        ctx->err = "context created without sampling";
+        return DFLASH_ESTATE;
+    }
+    if (temperature > 0.0 && ctx->eng->draft_mode == DFLASH_DRAFT_SCRIPT) {
+        ctx->err = "script drafts are for greedy decoding";
+        return DFLASH_ESTATE;
+    }
+    ctx->eng->temperature = (float)temperature;
+    ctx->eng->seed = seed;
+    ctx->err.clear();
     return DFLASH_OK;
 }
 

@@ -31,6 +31,7 @@ struct Layout {
     size_t weight_bytes = 0;
     // state arena offsets
     size_t x, xn, dq_in, Y, q, ao, h, taps_dec, taps_gather, taps_pre, cbuf, logits, plogits;
+    size_t qlogits, lse_p, lse_q, samp_part, tok_p, resid;  // temperature sampling (config.sampling)
     size_t g, drafts, accept, committed, new_len, st, active, meta, ctx_meta, ctx_meta_pre;
     size_t rope_t, rope_d, tk, tv, dk, dv, script, out_tok, tokens, stats, first_tok;
     size_t moe_sel, moe_wt, moe_part, moe_off = 0, moe_list = 0, lm_part, att_o, att_ml, att_sem;
@@ -73,6 +74,8 @@ class EngineBase {
     virtual dflash_status head_argmax_noalloc(int which, int32_t *host_out, int32_t *rows_out, void *scratch) = 0;
     std::string err;
     int draft_mode = DFLASH_DRAFT_MODEL, tau = 1;
+    float temperature = 0.f;  // > 0: temperature sampling (config.sampling), else greedy
+    uint64_t seed = 0;
 };
 
 }  // namespace dfl

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "philox.cuh"
 
 namespace dfl {
 
@@ -97,6 +98,59 @@ void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k
 template <typename T>
 void launch_moe_combine(float *x, const float *part, const float *wt, int H, int R, int k,
                         const TapDst<T> &taps, size_t lo, const RowMeta *meta, cudaStream_t s);
+
+// ---- temperature sampling (sampling.cu) ----
+// Rows of fp32 logits -> per-row log-sum-exp of z/T and a Gumbel-max draw from
+// softmax(z/T); draw positions: fixed_pos (one row, slot fixed_slot, prefill)
+// or st[active[i]].len + k + pos_off for row k of sequence i.
+struct SampleRows {
+    const float *logits = nullptr;
+    int ldl = 0, V = 0, R = 0, B = 1;
+    int mode = 0;  // 0: every row -> tok[r]; 1: block rows k >= 1 -> tok[i*(B-1)+k-1] (drafts)
+    float inv_T = 1.f;
+    SampleKey key{0, 0};
+    uint32_t purpose = SP_TARGET;
+    int pos_off = 0, fixed_pos = -1, fixed_slot = -1;
+    const SeqState *st = nullptr;
+    const int *active = nullptr;
+    float4 *part = nullptr;  // [sample_chunks(V)][R] scratch
+    float *lse = nullptr;    // [R] or null
+    int *tok = nullptr;
+    DevStats *stats = nullptr;
+};
+// Residual draws from max(0, P_{k-1} - Q_k) for block positions k = 1..B-1 of
+// every sequence: plog/qlog rows i*B+k-1 / i*B+k, resid[i*(B-1)+k-1] (-1: none).
+struct ResidualRows {
+    const float *plog = nullptr, *qlog = nullptr;
+    int ldl = 0, V = 0, B = 1, rows = 0;
+    float inv_T = 1.f;
+    SampleKey key{0, 0};
+    const float *lse_p = nullptr, *lse_q = nullptr;
+    const SeqState *st = nullptr;
+    const int *active = nullptr;
+    float2 *part = nullptr;  // [sample_chunks(V)][rows] scratch
+    int *resid = nullptr;
+};
+// The speculative-sampling acceptance + commit, one thread per sequence.
+struct AcceptSample {
+    SeqState *st = nullptr;
+    const int *active = nullptr;
+    int nseq = 0, B = 1;
+    const int *drafts = nullptr;
+    const float *plog = nullptr, *qlog = nullptr;
+    int ldl = 0;
+    const float *lse_p = nullptr, *lse_q = nullptr;
+    float inv_T = 1.f;
+    SampleKey key{0, 0};
+    const int *resid = nullptr, *tok_p = nullptr;  // residual draws; target draws (row B-1: the bonus)
+    int *accept = nullptr, *committed = nullptr, *new_len = nullptr, *out_tok = nullptr;
+    int out_ld = 0;
+    DevStats *stats = nullptr;
+};
+int sample_chunks(int V);
+void launch_sample_rows(const SampleRows &a, cudaStream_t s);
+void launch_residual_rows(const ResidualRows &a, cudaStream_t s);
+void launch_accept_sample(const AcceptSample &a, cudaStream_t s);
 
 // ---- tables ----
 void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStream_t s);

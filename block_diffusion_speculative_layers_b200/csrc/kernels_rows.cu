@@ -445,35 +445,9 @@ __global__ void accept_kernel(SeqState *st, const int *__restrict__ active, int 
     int a = 0;
     if (!S.done)
         while (a < B - 1 && d[a] == gi[a]) ++a;
-    if (committed)
-        for (int k = 0; k < B; ++k) committed[i * B + k] = (k < a) ? d[k] : (k == a ? gi[a] : -1);
-    if (!S.done) {
-        int emitted = 0;
-        for (int k = 0; k <= a; ++k) {
-            const int tok = (k < a) ? d[k] : gi[a];
-            if (S.n_out < S.max_new) {
-                out_tok[(size_t)s * out_ld + S.n_out] = tok;
-                S.n_out++;
-                emitted++;
-            }
-        }
-        S.anchor = gi[a];
-        if (S.n_out >= S.max_new) {
-            S.done = 1;
-            S.pend_n = 0;
-            if (stats) atomicAdd(&stats->n_done, 1);
-        } else {
-            S.pend_pos0 = S.len;
-            S.pend_n = a + 1;
-            S.len += a + 1;
-        }
-        if (stats) {
-            atomicAdd(&stats->iterations, 1ull);
-            atomicAdd(&stats->tokens, (unsigned long long)emitted);
-            atomicAdd(&stats->hist[a], 1ull);
-        }
-        st[s] = S;
-    }
+    const bool live = !S.done;
+    commit_block(S, s, i, a, d, gi[a], B, committed, out_tok, out_ld, stats);
+    if (live) st[s] = S;
     if (accept) accept[i] = a;
     if (new_len) new_len[i] = S.len;
 }

@@ -95,6 +95,8 @@ typedef struct {
     int32_t dtype;                /* DFLASH_FP32, DFLASH_BF16 or DFLASH_BF16_FAST (see above) */
     int32_t keep_logits;          /* 1: keep fp32 logits of the last draft/verify for dflash_debug_logits */
     int32_t timeout_ms;           /* host wait bound for synchronising calls (0: 600000) */
+    int32_t sampling;             /* 1: hold the buffers temperature sampling needs (dflash_set_sampling);
+                                     the LM heads then always store their fp32 logits */
 } dflash_config;
 
 typedef struct {
@@ -213,6 +215,21 @@ dflash_status dflash_set_draft_mode(dflash_ctx *ctx, int32_t mode, int32_t tau);
 /* script[i] is the token expected at output index i of slot `seq` (index 0 =
  * first token after the prompt); n <= max_len. */
 dflash_status dflash_set_script(dflash_ctx *ctx, int32_t seq, const int32_t *script, int32_t n);
+
+/* Temperature sampling ([P2] iaemfoco.com, "DFlash: Decodificação Especulativa
+ * com Blocos em Paralelo ...", "Casos de uso": the method also runs when
+ * sampling; [P4] imasters.com.br, "Os três mecanismos por trás do DFlash": the
+ * target's distribution is kept).  temperature 0 (the default): greedy.
+ * temperature > 0 (needs config.sampling): drafts d_i ~ softmax(z_draft / T),
+ * d_i accepted while u * Q_i(d_i) < P_{i-1}(d_i), the first rejected one
+ * replaced by a draw from max(0, P_{i-1} - Q_i), a bonus drawn from P_{B-1}
+ * when all are accepted; the first token after a prompt and target-only
+ * decoding draw from P.  Every draw comes from Philox4x32-10 keyed by seed,
+ * with counter (draw index / 4, absolute position, sequence slot, purpose),
+ * so runs are reproducible per (seed, slot).  Applies to later calls.
+ * Errors: DFLASH_EINVAL for a negative or non-finite temperature;
+ * DFLASH_ESTATE without config.sampling or with script drafts. */
+dflash_status dflash_set_sampling(dflash_ctx *ctx, double temperature, uint64_t seed);
 
 /* fp32 logits of the last pass (needs keep_logits): which = 0 drafter rows
  * [n_seqs][B][V] (row 0 of each block is the anchor row), 1 verify rows
