@@ -134,6 +134,9 @@ def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: in
     "fast" (one plane, DFLASH_BF16_FAST)."""
     if bf16_act not in ("split", "fast"):
         raise ValueError("bf16_act must be 'split' or 'fast'")
+    for d in (spec.target, spec.drafter):
+        if getattr(d, "qk_norm", False) or float(getattr(d, "rope_scaling", (0.0,))[0]) > 1.0:
+            raise NotImplementedError("QK-norm and RoPE frequency rescaling are not in the kernels yet")
     c = Config()
     c.target = _model_cfg(spec.target)
     c.drafter = _model_cfg(spec.drafter)

@@ -18,13 +18,16 @@ class Dims(C.Structure):
     _fields_ = [("n_layers", C.c_int32), ("hidden", C.c_int32), ("n_q_heads", C.c_int32),
                 ("n_kv_heads", C.c_int32), ("head_dim", C.c_int32), ("ffn", C.c_int32),
                 ("vocab", C.c_int32), ("n_experts", C.c_int32), ("top_k", C.c_int32),
-                ("expert_ffn", C.c_int32), ("rms_eps", C.c_double), ("rope_theta", C.c_double)]
+                ("expert_ffn", C.c_int32), ("rms_eps", C.c_double), ("rope_theta", C.c_double),
+                ("qk_norm", C.c_int32), ("rope_factor", C.c_double), ("rope_low_freq_factor", C.c_double),
+                ("rope_high_freq_factor", C.c_double), ("rope_original_max_pos", C.c_double)]
 
 
 class Layer(C.Structure):
     _fields_ = [("attn_norm", C.c_void_p), ("wqkv", C.c_void_p), ("wo", C.c_void_p),
                 ("ffn_norm", C.c_void_p), ("w_gate_up", C.c_void_p), ("w_down", C.c_void_p),
-                ("w_router", C.c_void_p), ("we_gate_up", C.c_void_p), ("we_down", C.c_void_p)]
+                ("w_router", C.c_void_p), ("we_gate_up", C.c_void_p), ("we_down", C.c_void_p),
+                ("q_norm", C.c_void_p), ("k_norm", C.c_void_p)]
 
 
 class Model(C.Structure):
@@ -49,6 +52,9 @@ def load_lib():
     lib = C.CDLL(build_oracle())
     lib.orc_rmsnorm.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_double, C.c_void_p]
     lib.orc_rope.argtypes = [C.c_void_p, C.c_int32, C.c_int64, C.c_double]
+    lib.orc_rope_inv_freq.argtypes = [C.POINTER(Dims), C.c_int32]
+    lib.orc_rope_inv_freq.restype = C.c_double
+    lib.orc_rope_dims.argtypes = [C.c_void_p, C.POINTER(Dims), C.c_int64]
     lib.orc_matmul.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_int32, C.c_void_p]
     lib.orc_attend.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_void_p]
     lib.orc_argmax.argtypes = [C.c_void_p, C.c_int32, C.c_void_p]
@@ -102,6 +108,14 @@ def _wtensor(t: torch.Tensor) -> torch.Tensor:
     return t
 
 
+def dims(d) -> Dims:
+    """The oracle's view of one model's shape and settings."""
+    f, lo, hi, orig = (float(x) for x in d.rope_scaling)
+    return Dims(d.n_layers, d.hidden, d.n_q_heads, d.n_kv_heads, d.head_dim, d.ffn, d.vocab,
+                d.n_experts, d.top_k, d.expert_ffn, float(d.rms_eps), float(d.rope_theta),
+                1 if d.qk_norm else 0, f, lo, hi, orig)
+
+
 class OracleSpec:
     """A target + drafter + fuse weight set, viewed by the C oracle (no copies)."""
 
@@ -131,8 +145,7 @@ class OracleSpec:
 
     def _model(self, prefix, d, w, dtype) -> Model:
         m = Model()
-        m.d = Dims(d.n_layers, d.hidden, d.n_q_heads, d.n_kv_heads, d.head_dim, d.ffn, d.vocab,
-                   d.n_experts, d.top_k, d.expert_ffn, float(d.rms_eps), float(d.rope_theta))
+        m.d = dims(d)
         m.dtype = dtype
         m.embed = _ptr(w["embed"])
         m.lm_head = _ptr(w["lm_head"])
@@ -145,6 +158,9 @@ class OracleSpec:
             L.wqkv = _ptr(w[p + "wqkv"])
             L.wo = _ptr(w[p + "wo"])
             L.ffn_norm = _ptr(w[p + "ffn_norm"])
+            if d.qk_norm:
+                L.q_norm = _ptr(w[p + "q_norm"])
+                L.k_norm = _ptr(w[p + "k_norm"])
             if d.n_experts > 0:
                 L.w_router = _ptr(w[p + "w_router"])
                 L.we_gate_up = _ptr(w[p + "we_gate_up"])
@@ -269,6 +285,20 @@ def rmsnorm(x, g, eps: float) -> np.ndarray:
     y = np.zeros_like(xx)
     lib.orc_rmsnorm(xx.ctypes.data, gg.ctypes.data, len(xx), eps, y.ctypes.data)
     return y
+
+
+def rope_inv_freq(d, i: int) -> float:
+    """Inverse frequency of RoPE pair i of model shape d (with its rescaling, if any)."""
+    dd = dims(d)
+    return load_lib().orc_rope_inv_freq(C.byref(dd), i)
+
+
+def rope_dims(v, pos: int, d) -> np.ndarray:
+    """RoPE of one head vector at pos under model shape d's settings."""
+    out = _f64(v).copy()
+    dd = dims(d)
+    load_lib().orc_rope_dims(out.ctypes.data, C.byref(dd), pos)
+    return out
 
 
 def rope(v, pos: int, theta: float) -> np.ndarray:

@@ -170,6 +170,49 @@ void orc_rope(double *v, int32_t hd, int64_t pos, double theta) {
     }
 }
 
+/* Fidelity toggle, not on the pages: the frequency rescaling published with
+ * Llama 3.1 (its rope_scaling settings factor, low_freq_factor,
+ * high_freq_factor, original_max_position_embeddings).  A pair whose
+ * wavelength 2*pi/f is shorter than original_max / high_freq_factor keeps f;
+ * one longer than original_max / low_freq_factor gets f / factor; in between
+ * f / factor and f are mixed with weight
+ * s = (original_max / wavelength - low_freq_factor) / (high_freq_factor - low_freq_factor)
+ * on f, which is continuous at both band edges. */
+double orc_rope_inv_freq(const orc_dims *d, int32_t i) {
+    double f = pow(d->rope_theta, -2.0 * (double)i / (double)d->head_dim);
+    if (!(d->rope_factor > 1.0)) return f;
+    double wavelen = 2.0 * 3.14159265358979323846 / f;
+    double lo_edge = d->rope_original_max_pos / d->rope_high_freq_factor;  /* shortest rescaled wavelength */
+    double hi_edge = d->rope_original_max_pos / d->rope_low_freq_factor;   /* longest partly kept wavelength */
+    if (wavelen < lo_edge) return f;
+    if (wavelen > hi_edge) return f / d->rope_factor;
+    double s = (d->rope_original_max_pos / wavelen - d->rope_low_freq_factor) /
+               (d->rope_high_freq_factor - d->rope_low_freq_factor);
+    return (1.0 - s) * f / d->rope_factor + s * f;
+}
+
+void orc_rope_dims(double *v, const orc_dims *d, int64_t pos) {
+    int32_t hd = d->head_dim, half = hd / 2;
+    if (!(d->rope_factor > 1.0)) {
+        orc_rope(v, hd, pos, d->rope_theta);
+        return;
+    }
+    for (int32_t i = 0; i < half; ++i) {
+        double ang = (double)pos * orc_rope_inv_freq(d, i);
+        double c = cos(ang), s = sin(ang);
+        double x1 = v[i], x2 = v[i + half];
+        v[i] = x1 * c - x2 * s;
+        v[i + half] = x2 * c + x1 * s;
+    }
+}
+
+/* Fidelity toggle, not on the pages: Qwen3 layers normalise every q and k head
+ * (RMSNorm over head_dim with a per-dimension gain, the layer's rms_eps) before
+ * RoPE.  In place on n_heads consecutive vectors of hd. */
+static void qk_norm_heads(double *v, int32_t n_heads, int32_t hd, const float *g, double eps) {
+    for (int32_t h = 0; h < n_heads; ++h) orc_rmsnorm(v + (size_t)h * hd, g, hd, eps, v + (size_t)h * hd);
+}
+
 void orc_attend(const double *q, const double *keys, const double *vals, int64_t ld_kv,
                 int32_t n_keys, int32_t hd, double *out) {
     /* softmax_j(q . k_j / sqrt(hd)) weighted sum of v_j, keys in order 0..n-1 */
@@ -384,11 +427,13 @@ static void layer_rows(const orc_model *m, int32_t l, double *x, int32_t R, int3
         const double *row = qkv + (size_t)r * nqkv;
         int32_t pos = pos0 + r;
         memcpy(q + (size_t)r * qd, row, sizeof(double) * qd);
-        for (int32_t h = 0; h < nq; ++h) orc_rope(q + (size_t)r * qd + (size_t)h * hd, hd, pos, d->rope_theta);
+        if (d->qk_norm) qk_norm_heads(q + (size_t)r * qd, nq, hd, L->q_norm, d->rms_eps);
+        for (int32_t h = 0; h < nq; ++h) orc_rope_dims(q + (size_t)r * qd + (size_t)h * hd, d, pos);
         double *kp = kc + (size_t)pos * kd, *vp = vc + (size_t)pos * kd;
         memcpy(kp, row + qd, sizeof(double) * kd);
         memcpy(vp, row + qd + kd, sizeof(double) * kd);
-        for (int32_t g = 0; g < nkv; ++g) orc_rope(kp + (size_t)g * hd, hd, pos, d->rope_theta);
+        if (d->qk_norm) qk_norm_heads(kp, nkv, hd, L->k_norm, d->rms_eps);
+        for (int32_t g = 0; g < nkv; ++g) orc_rope_dims(kp + (size_t)g * hd, d, pos);
     }
     attn_rows(d, q, kc, vc, n_keys, R, att);
     orc_matmul(L->wo, m->dtype, H, qd, att, R, o);
@@ -452,7 +497,9 @@ static void inject_ctx(orc_session *ss, int32_t n_rows, int32_t pos0) {
             double *kp = tkv_at(ss->dk, d, ss->max_len, j, t), *vp = tkv_at(ss->dv, d, ss->max_len, j, t);
             memcpy(kp, kv + (size_t)r * 2 * kd, sizeof(double) * kd);
             memcpy(vp, kv + (size_t)r * 2 * kd + kd, sizeof(double) * kd);
-            for (int32_t g = 0; g < d->n_kv_heads; ++g) orc_rope(kp + (size_t)g * hd, hd, t, d->rope_theta);
+            /* the context keys pass the same k processing as the block's keys (R5) */
+            if (d->qk_norm) qk_norm_heads(kp, d->n_kv_heads, hd, m->layers[j].k_norm, d->rms_eps);
+            for (int32_t g = 0; g < d->n_kv_heads; ++g) orc_rope_dims(kp + (size_t)g * hd, d, t);
         }
     }
     free(c); free(kv);

@@ -38,6 +38,11 @@ typedef struct {
     int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
     int32_t n_experts, top_k, expert_ffn;   /* n_experts == 0: dense SwiGLU */
     double rms_eps, rope_theta;
+    /* fidelity toggles, off by default (not on the pages):
+     * qk_norm: per-head RMSNorm of q and k before RoPE (Qwen3 layers);
+     * rope_factor > 1: Llama 3.1 rescaling of the RoPE frequencies. */
+    int32_t qk_norm;
+    double rope_factor, rope_low_freq_factor, rope_high_freq_factor, rope_original_max_pos;
 } orc_dims;
 
 typedef struct {
@@ -50,6 +55,8 @@ typedef struct {
     const void *w_router;     /* MoE: [E, H] */
     const void *we_gate_up;   /* MoE: [E, 2Fe, H] */
     const void *we_down;      /* MoE: [E, H, Fe] */
+    const float *q_norm;      /* qk_norm: [hd] gain of every q head */
+    const float *k_norm;      /* qk_norm: [hd] gain of every k head */
 } orc_layer;
 
 typedef struct {
@@ -76,6 +83,10 @@ typedef struct orc_session orc_session;
 /* ---- building blocks (each pinned separately by the tests) ---- */
 void orc_rmsnorm(const double *x, const float *g, int32_t n, double eps, double *y);
 void orc_rope(double *v, int32_t head_dim, int64_t pos, double theta);
+/* Inverse frequency of RoPE pair i under the model's settings (theta^(-2i/hd),
+ * rescaled when rope_factor > 1), and the rotation with those frequencies. */
+double orc_rope_inv_freq(const orc_dims *d, int32_t i);
+void orc_rope_dims(double *v, const orc_dims *d, int64_t pos);
 /* Y[r][n] = sum_k W[n][k] X[r][k]; W in fp32/bf16 storage. */
 void orc_matmul(const void *W, int32_t dtype, int32_t N, int32_t K,
                 const double *X, int32_t R, double *Y);

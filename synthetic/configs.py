@@ -28,6 +28,12 @@ class ModelDims:
     n_experts: int = 0      # 0 = dense SwiGLU FFN
     top_k: int = 0
     expert_ffn: int = 0
+    # fidelity toggles (not on the pages; off by default): per-head RMSNorm of
+    # q and k before RoPE as in Qwen3 layers, and the Llama 3.1 RoPE frequency
+    # rescaling (factor, low_freq_factor, high_freq_factor, original max
+    # position; factor <= 1 leaves the frequencies as they are)
+    qk_norm: bool = False
+    rope_scaling: Tuple[float, float, float, float] = (0.0, 0.0, 0.0, 0.0)
 
     @property
     def q_dim(self) -> int:

@@ -101,6 +101,9 @@ def _layer_shapes(prefix: str, d: ModelDims) -> "OrderedDict[str, Tuple[Tuple[in
         s[p + "attn_norm"] = ((H,), "norm")
         s[p + "wqkv"] = ((d.qkv_dim, H), "matrix")      # rows: [Wq; Wk; Wv]
         s[p + "wo"] = ((H, d.q_dim), "matrix")
+        if d.qk_norm:
+            s[p + "q_norm"] = ((d.head_dim,), "norm")
+            s[p + "k_norm"] = ((d.head_dim,), "norm")
         s[p + "ffn_norm"] = ((H,), "norm")
         if d.is_moe:
             s[p + "w_router"] = ((d.n_experts, H), "matrix")

@@ -23,11 +23,25 @@ def rms(x, g, eps):
     return x / np.sqrt((x * x).mean(-1, keepdims=True) + eps) * g
 
 
-def rope(x, pos, theta):
-    """x [..., T, hd]; rotate-half pairing."""
+def inv_freq(d):
+    """RoPE inverse frequencies of model shape d; with d.rope_scaling's factor
+    above 1, bands by wavelength: short ones kept, long ones divided by the
+    factor, the ones between mixed linearly in original_max / wavelength."""
+    hd = d.head_dim
+    f = d.rope_theta ** (-np.arange(hd // 2, dtype=np.float64) * 2.0 / hd)
+    factor, low, high, orig = d.rope_scaling
+    if factor <= 1.0:
+        return f
+    ratio = orig / (2.0 * np.pi / f)                  # how many wavelengths fit the original window
+    w = np.clip((ratio - low) / (high - low), 0.0, 1.0)  # 1: keep f, 0: f / factor
+    return w * f + (1.0 - w) * f / factor
+
+
+def rope(x, pos, d):
+    """x [..., T, hd]; rotate-half pairing with the frequencies of model shape d."""
     hd = x.shape[-1]
     half = hd // 2
-    freq = theta ** (-np.arange(half, dtype=np.float64) * 2.0 / hd)
+    freq = inv_freq(d)
     ang = np.asarray(pos, np.float64)[:, None] * freq[None, :]
     c, s = np.cos(ang), np.sin(ang)
     x1, x2 = x[..., :half], x[..., half:]
@@ -76,8 +90,11 @@ def _layer(d, W, p, x, pos, keys_extra=None, mask=None):
     q = qkv[:, :qd].reshape(T, nq, hd).transpose(1, 0, 2)
     k = qkv[:, qd:qd + kd].reshape(T, nkv, hd).transpose(1, 0, 2)
     v = qkv[:, qd + kd:].reshape(T, nkv, hd).transpose(1, 0, 2)
-    q = rope(q, pos, d.rope_theta)
-    k = rope(k, pos, d.rope_theta)
+    if d.qk_norm:                           # per-head RMSNorm of q and k before RoPE
+        q = rms(q, _np(W[p + "q_norm"]), d.rms_eps)
+        k = rms(k, _np(W[p + "k_norm"]), d.rms_eps)
+    q = rope(q, pos, d)
+    k = rope(k, pos, d)
     if keys_extra is not None:
         k = np.concatenate([keys_extra[0], k], axis=1)
         v = np.concatenate([keys_extra[1], v], axis=1)
@@ -138,7 +155,9 @@ def drafter_block(cfg, W, committed, anchor):
         wqkv = _np(W[f"drafter.L{j}.wqkv"])
         kc = (c @ wqkv[qd:qd + kd].T).reshape(p, nkv, hd).transpose(1, 0, 2)
         vc = (c @ wqkv[qd + kd:].T).reshape(p, nkv, hd).transpose(1, 0, 2)
-        kc = rope(kc, np.arange(p), d.rope_theta)
+        if d.qk_norm:
+            kc = rms(kc, _np(W[f"drafter.L{j}.k_norm"]), d.rms_eps)
+        kc = rope(kc, np.arange(p), d)
         x = _layer(d, W, f"drafter.L{j}.", x, pos, keys_extra=(kc, vc), mask=mask)
     logits = rms(x, _np(W["drafter.final_norm"]), d.rms_eps) @ _np(W["lm_head"]).T
     return logits[1:]

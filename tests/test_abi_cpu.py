@@ -81,3 +81,13 @@ def test_create_rejects_missing_arenas(lib):
     assert lib.dflash_create(C.byref(c), None, 0, None, 0, None, C.byref(h)) == 1
     assert lib.dflash_create(C.byref(c), 256, 1 << 40, 256, 1, None, C.byref(h)) == 1  # too small state arena
     assert not h.value
+
+
+def test_fidelity_toggles_are_refused_until_the_kernels_have_them():
+    from dataclasses import replace
+    from synthetic import get_config
+    base = get_config("tiny")
+    for t in (replace(base.target, qk_norm=True), replace(base.target, rope_scaling=(8.0, 1.0, 4.0, 256.0))):
+        with pytest.raises(NotImplementedError):
+            dfl.make_config(base.with_(target=t))
+    dfl.make_config(base.with_(target=replace(base.target, rope_scaling=(1.0, 1.0, 4.0, 256.0))))

@@ -25,13 +25,21 @@ import dense_ref
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
+# Llama 3.1-style RoPE rescaling scaled to the tiny model (theta 1e4, head_dim 64):
+# pairs 0-8 keep their frequency, 9-12 are mixed, 13-31 are divided by 8
+TINY_ROPE_SCALING = (8.0, 1.0, 4.0, 256.0)
+
+
 def tiny(dtype="fp32", block=4, nq=4, nkv=2, moe=False, taps=(0, 1), t_layers=2, d_layers=1,
-         vocab=1024):
+         vocab=1024, qk_norm=False, rope_scaling=None):
     base = get_config("tiny")
-    t = replace(base.target, n_layers=t_layers, n_q_heads=nq, n_kv_heads=nkv, vocab=vocab)
+    fid = dict(qk_norm=qk_norm)
+    if rope_scaling:
+        fid["rope_scaling"] = rope_scaling
+    t = replace(base.target, n_layers=t_layers, n_q_heads=nq, n_kv_heads=nkv, vocab=vocab, **fid)
     if moe:
         t = replace(t, n_experts=8, top_k=2, expert_ffn=64)
-    d = replace(base.drafter, n_layers=d_layers, n_q_heads=nq, n_kv_heads=nkv, vocab=vocab)
+    d = replace(base.drafter, n_layers=d_layers, n_q_heads=nq, n_kv_heads=nkv, vocab=vocab, **fid)
     return base.with_(target=t, drafter=d, block_size=block, tap_layers=taps, dtype=dtype)
 
 
@@ -255,6 +263,8 @@ CASES = {
     "moe": dict(moe=True),
     "mha": dict(nq=4, nkv=4),
     "block16": dict(block=16),
+    "qk_norm": dict(qk_norm=True),
+    "rope_scaled": dict(rope_scaling=TINY_ROPE_SCALING),
 }
 
 
@@ -303,7 +313,7 @@ def test_gqa_equals_mha_with_repeated_kv_heads():
     np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("case", ["fp32", "bf16", "moe", "block16"])
+@pytest.mark.parametrize("case", ["fp32", "bf16", "moe", "block16", "qk_norm", "rope_scaled"])
 def test_drafter_matches_dense_reference_through_rejections(case):
     """Drafter logits after several draft/verify/commit rounds equal a drafter
     whose context is rebuilt from scratch from the committed prefix: pins the
