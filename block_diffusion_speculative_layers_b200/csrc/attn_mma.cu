@@ -434,8 +434,6 @@ bool attn_mma_supported<float>(int) {
     return false;
 }
 
-static int g_num_sms = 0;
-
 // key groups per CTA: two when the kv group has at most 4 q heads (8 warps)
 static int attn_groups(int grp) { return grp <= 4 ? 2 : 1; }
 
@@ -454,11 +452,7 @@ static void launch_hd(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, co
     const int grp = nq / nkv;
     const int G = attn_groups(grp);
     const size_t smem = attn_smem(HD, SPLIT, grp, n_splits);
-    static bool set = false;
-    if (!set) {
-        cudaFuncSetAttribute(at::attn_mma_kernel<HD, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        set = true;
-    }
+    ensure_smem_attr((const void *)at::attn_mma_kernel<HD, SPLIT>);
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
     launch_k(at::attn_mma_kernel<HD, SPLIT>, dim3(n_tiles, nkv, n_splits), dim3(32 * grp * G), smem, s, n_splits, q, ldq,
              kc, vc, meta, R, rows_per_tile, nq, nkv, max_len, n_splits, G, scale_log2, out, ldo, lo, sy.dep_ctr,
@@ -469,13 +463,8 @@ template <>
 int launch_attention_mma<bf16>(const bf16 *q, int ldq, const bf16 *kc, const bf16 *vc, const RowMeta *meta, int R,
                                int rows_per_tile, int nq, int nkv, int hd, int max_len, bf16 *out, int ldo, size_t lo,
                                const AttnScratch &ws, cudaStream_t s, const AttnSync &sy) {
-    (void)ws;
     if (R <= 0) return 0;
-    if (!g_num_sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int g_num_sms = ws.num_sms;
     const int n_tiles = (R + rows_per_tile - 1) / rows_per_tile;
     const int ctas = n_tiles * nkv;
     // splits of one (tile, kv head) form a cluster of at most 8 CTAs; no more

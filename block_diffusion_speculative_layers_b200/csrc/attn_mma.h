@@ -16,6 +16,7 @@ struct AttnScratch {
     int *sem = nullptr;
     size_t max_parts = 0;
     int n_sem = 0;
+    int num_sms = 148;  // SMs of the context's device
 };
 
 struct AttnWorkspace {

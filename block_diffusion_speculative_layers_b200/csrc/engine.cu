@@ -20,13 +20,14 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <thread>
 #include <type_traits>
 
 #include "engine.h"
 #include "gemm_tc.h"
 #include "attn_mma.h"
-#include "chain_tc.h"
+#include "pass_program.h"
 
 namespace dfl {
 
@@ -37,18 +38,27 @@ constexpr int kNoallocTiles = 2048;
 constexpr size_t kNoallocPartBytes = (size_t)kNoallocRows * kNoallocTiles * sizeof(float2);
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocPartBytes + kNoallocRows * sizeof(int)];
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the host-side symbol is not a device address).
-static void *noalloc_scratch_ptr(std::string &err) {
-    static void *ptrs[64] = {nullptr};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-        err = "no current CUDA device";
+// Device address of g_noalloc_scratch on device `dev` (the host-side symbol is
+// not a device address), looked up once per device with that device current,
+// under a lock so that host threads driving different contexts can share it.
+static void *noalloc_scratch_ptr(int dev, std::string &err) {
+    static std::mutex mu;
+    static void *ptrs[kMaxDevices] = {nullptr};
+    if (dev < 0 || dev >= kMaxDevices) {
+        err = "device index out of range";
         return nullptr;
     }
+    std::lock_guard<std::mutex> lock(mu);
     if (!ptrs[dev]) {
+        int prev = 0;
+        if (cudaGetDevice(&prev) != cudaSuccess) {
+            err = "no current CUDA device";
+            return nullptr;
+        }
         void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        cudaError_t e = cudaSetDevice(dev);
+        if (e == cudaSuccess) e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        cudaSetDevice(prev);
         if (e != cudaSuccess) {
             err = std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e);
             return nullptr;
@@ -252,30 +262,15 @@ static Layout make_layout(const dflash_config &c) {
         L.att_ml = take(L.att_parts * 2 * 4);
         L.att_sem = take((size_t)tiles * std::max(t.n_kv_heads, d.n_kv_heads) * 4);
     }
-    // persistent projection chains (bf16 decode): folded-norm activations,
-    // per-tile sums of squares, two programs (verify, draft) and split-K partials
+    // bf16 decode passes: folded-norm activations, per-tile sums of squares and
+    // the completion counters of the two pass programs (verify, draft)
     {
         L.ssq_ld = 2 * L.R_dec;
         L.ssq = take((size_t)(H / 128 + 1) * L.ssq_ld * 4);
-        const int F_d = d.ffn;
-        const int F_tmax = t.n_experts > 0 ? t.expert_ffn : t.ffn;
-        L.max_tiles = std::max({(t.vocab + 127) / 128, (qd_t + 2 * kd_t + 127) / 128, (qd_d + 2 * kd_d + 127) / 128,
-                                (F_tmax + 63) / 64, (F_d + 63) / 64, (H + 127) / 128});
         L.n_ops_v = 1 + 4 * t.n_layers;
         L.n_ops_d = 2 + 4 * d.n_layers;
-        auto prog_bytes = [&](int n_ops) {
-            return align_up((size_t)n_ops * sizeof(ChainOp), 256) + align_up((size_t)2 * n_ops * sizeof(CUtensorMap), 256) +
-                   align_up((size_t)n_ops * 4, 256) + align_up((size_t)n_ops * L.max_tiles * 4, 256) +
-                   align_up((size_t)n_ops * L.max_tiles * sizeof(int4), 256) + align_up((size_t)2 * n_ops * 4, 256);
-        };
-        L.chain_v_bytes = prog_bytes(L.n_ops_v);
-        L.chain_d_bytes = prog_bytes(L.n_ops_d);
-        L.chain_v = take(L.chain_v_bytes);
-        L.chain_d = take(L.chain_d_bytes);
-        int tm_max = 16;
-        while (tm_max < 2 * L.R_dec && tm_max < 256) tm_max *= 2;
-        L.chain_ws_floats = (size_t)2 * 160 * tm_max * 128;  // units per op stay near the SM count
-        L.chain_ws = take(2 * L.chain_ws_floats * 4);
+        L.dep_v = take((size_t)2 * L.n_ops_v * 4);
+        L.dep_d = take((size_t)2 * L.n_ops_d * 4);
     }
     // split-K workspace and tile semaphores of the tensor-core GEMM
     L.ws_floats = gemm_tc_workspace_floats(L.R_max, std::max(ycols, t.vocab > 0 ? H : H));
@@ -319,22 +314,31 @@ class Engine : public EngineBase {
     int *gemm_sem;
     float2 *lm_part;
     AttnScratch att;
-    // persistent projection chains (bf16 decode)
+    // folded-norm decode passes (bf16)
     T *xg_t = nullptr, *xg2 = nullptr;
     size_t lo_ = 0;  // low plane offset of two-plane activations (elements), 0: one plane
     float *ssq = nullptr;
-    ChainProgram pv, pd;
+    PassProgram pv, pd;
     // bf16 decode passes run as projection programs with folded RMSNorms
-    // (fold_*_ok), one kernel per projection or, with chain_on, as persistent chains
-    bool chain_verify_ok = false, chain_draft_ok = false, chain_on = false;
+    // (fold_*_ok), one kernel per projection
+    bool fold_verify_ok = false, fold_draft_ok = false;
     bool dep_on = false;  // completion counters between the kernels of a pass (per-kernel mode)
-    bool chain_used[3] = {false, false, false};
+    bool fold_used[3] = {false, false, false};
     int num_sms = 148;
     GemmTC<T> tc;
     // host mirrors
     std::vector<int> h_len, h_prefilled;
     std::vector<int> last_draft;
     int last_logits_rows[3] = {0, 0, 0};
+    // kind of the last pass that ran on this context: what the LM-head input
+    // buffers (xn / xg_t) hold now.  PASS_OTHER: generation loops, target-only steps.
+    enum { PASS_NONE = -1, PASS_DRAFT = 0, PASS_VERIFY = 1, PASS_PREFILL = 2, PASS_OTHER = 3 };
+    int last_pass = PASS_NONE;
+    struct OtherPass {  // marks a generation loop on every return path
+        int &r;
+        ~OtherPass() { r = PASS_OTHER; }
+    };
+    int device = 0;
     int *pinned = nullptr;  // small pinned host buffer for the done counter
     bool lens_stale = false;
     // per-launch timing (dflash_profile)
@@ -440,47 +444,29 @@ class Engine : public EngineBase {
         {
             int dev = 0;
             cudaGetDevice(&dev);
+            device = dev;
             cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
             const bool bf = std::is_same<T, bf16>::value;
             const int H = c.target.hidden;
             const bool shapes = H % 128 == 0 && num_sms <= 160 && 2 * L.R_dec <= 256;
-            // DFLASH_PROJECTION_CHAIN=1 runs the dependent projections of a pass as
-            // persistent chains instead of one kernel per projection (same arithmetic);
             // DFLASH_FOLDED_NORM=0 goes back to separate RMSNorm kernels
-            const char *ev = getenv("DFLASH_PROJECTION_CHAIN");
-            chain_on = ev && ev[0] == '1';
             // DFLASH_DEP_COUNTERS=1: device completion counters between the kernels of a
             // pass instead of griddepcontrol.wait (same results; measured 0.2 ms per step
             // slower on B200: the fences of every writer cost more than the grid release)
             const char *dv_env = getenv("DFLASH_DEP_COUNTERS");
-            dep_on = !chain_on && dv_env && dv_env[0] == '1';
+            dep_on = dv_env && dv_env[0] == '1';
             const char *fv = getenv("DFLASH_FOLDED_NORM");
             const bool allow = !(fv && fv[0] == '0');
-            chain_draft_ok = allow && bf && shapes;
-            chain_verify_ok = allow && bf && shapes && c.target.n_experts == 0;
-            auto carve = [&](ChainProgram &pg, size_t off, int n_ops) {
-                char *b = S + off;
-                pg.d_ops = reinterpret_cast<ChainOp *>(b);
-                b += align_up((size_t)n_ops * sizeof(ChainOp), 256);
-                pg.d_maps = reinterpret_cast<CUtensorMap *>(b);
-                b += align_up((size_t)2 * n_ops * sizeof(CUtensorMap), 256);
-                pg.d_op_done = reinterpret_cast<int *>(b);
-                b += align_up((size_t)n_ops * 4, 256);
-                pg.d_tile_cnt = reinterpret_cast<int *>(b);
-                b += align_up((size_t)n_ops * L.max_tiles * 4, 256);
-                pg.d_tinfo = reinterpret_cast<int4 *>(b);
-                b += align_up((size_t)n_ops * L.max_tiles * sizeof(int4), 256);
-                pg.d_dep = reinterpret_cast<int *>(b);
-                pg.d_ws = sp<float>(L.chain_ws);
-                pg.ws_floats = L.chain_ws_floats;
-            };
-            carve(pv, L.chain_v, L.n_ops_v);
-            carve(pd, L.chain_d, L.n_ops_d);
+            fold_draft_ok = allow && bf && shapes;
+            fold_verify_ok = allow && bf && shapes && c.target.n_experts == 0;
+            pv.d_dep = sp<int>(L.dep_v);
+            pd.d_dep = sp<int>(L.dep_d);
         }
         att.o_part = sp<float>(L.att_o);
         att.ml_part = sp<float>(L.att_ml);
         att.sem = sp<int>(L.att_sem);
         att.max_parts = L.att_parts;
+        att.num_sms = num_sms;
         att.n_sem = std::max(L.R_dec, (L.C + 15) / 16) * std::max(c.target.n_kv_heads, c.drafter.n_kv_heads);
         h_len.assign(c.max_batch, 0);
         h_prefilled.assign(c.max_batch, 0);
@@ -524,6 +510,10 @@ class Engine : public EngineBase {
     }
 
     dflash_status check(const char *what) {
+        if (tc.failed) {  // a projection could not be launched (tensor map encoding)
+            err = std::string(what) + ": " + tc.err;
+            return DFLASH_ECUDA;
+        }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) {
             err = std::string(what) + ": " + cudaGetErrorString(e);
@@ -862,80 +852,20 @@ class Engine : public EngineBase {
         launch_accept_sample(a, s);
     }
 
-    // ---- persistent projection chains (bf16 decode) ----
-    static int pow2_at_least(int x, int lo) {
-        int t = lo;
-        while (t < x) t *= 2;
-        return t;
-    }
-
-    // Append one projection to a chain program (host side; uploaded by finish_program).
-    void chain_add(ChainProgram &pg, int &tile_off, int kind, const void *W, int N, int K, const T *X, int ldx, int M,
-                   const Epi<T> &e) {
+    // ---- folded-norm decode passes (bf16) ----
+    // Append one projection to a pass program.
+    void prog_add(PassProgram &pg, int kind, const void *W, int N, int K, const T *X, int ldx, int M, const Epi<T> &e) {
         if constexpr (std::is_same<T, bf16>::value) {
-            ChainOp op{};
+            PassOp op;
             op.kind = kind;
-            TcParams &p = op.p;
-            const bool swiglu = kind == EPI_SWIGLU;
-            p.M = M;
-            p.N = N;
-            p.K = K;
-            p.swiglu_F = swiglu ? e.F : 0;
-            p.n_tiles = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
-            p.m_tiles = 1;
-            p.k_steps = (K + 63) / 64;
-            // stream-K: CTA b streams tile-k-steps [total*b/G, total*(b+1)/G); a tile
-            // covered by several CTAs gets consecutive partial slots in the workspace
-            p.splits = 1;
-            p.err = &stats->status;
-            p.lm_part = lm_part;
-            p.keep_logits = c.keep_logits || c.sampling;
-            const long long total = (long long)p.n_tiles * p.k_steps;
-            // ops with fewer tile-k-steps than SMs use only the first `total` CTAs, so
-            // the CTAs covering a tile are always consecutive (slot = CTA - first CTA)
-            const int G = (int)std::min<long long>(num_sms, total);
-            std::vector<int4> ti(p.n_tiles, make_int4(-1, 0, 0, 0));
-            for (int b = 0; b < G; ++b) {
-                const long long g0 = total * b / G, g1 = total * (b + 1) / G;
-                for (long long g = g0; g < g1;) {
-                    const int nt = (int)(g / p.k_steps);
-                    if (ti[nt].x < 0) ti[nt].x = b;
-                    ti[nt].y += 1;
-                    g = std::min(g1, (long long)(nt + 1) * p.k_steps);
-                }
-            }
-            int slots = 0;
-            for (int t = 0; t < p.n_tiles; ++t) {
-                ti[t].z = slots;
-                if (ti[t].y > 1) slots += ti[t].y;
-            }
-            if ((size_t)slots * pg.tm * 128 > pg.ws_floats) pg.valid = false;  // use the per-kernel path
-            const int idx = (int)pg.ops.size();
-            CUtensorMap mw = *tc.tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
-            CUtensorMap mx = *tc.tensor_map(X, M, K, ldx, pg.tm, lo_);
-            pg.maps.push_back(mw);
-            pg.maps.push_back(mx);
-            op.wmap = pg.d_maps + 2 * idx;
-            op.xmap = pg.d_maps + 2 * idx + 1;
             op.e = e;
             op.e.lo = lo_;
-            op.ws = pg.d_ws + (size_t)(idx & 1) * pg.ws_floats;
-            op.tile_cnt = pg.d_tile_cnt + tile_off;
-            op.tinfo = pg.d_tinfo + tile_off;
-            pg.tinfo.insert(pg.tinfo.end(), ti.begin(), ti.end());
-            tile_off += p.n_tiles;
             pg.ops.push_back(op);
             pg.hops.push_back(HostOp{W, N, K, X, ldx, M});
         }
     }
 
-    void finish_program(ChainProgram &pg) {
-        cudaMemcpyAsync(pg.d_ops, pg.ops.data(), sizeof(ChainOp) * pg.ops.size(), cudaMemcpyHostToDevice, s);
-        cudaMemcpyAsync(pg.d_tinfo, pg.tinfo.data(), sizeof(int4) * pg.tinfo.size(), cudaMemcpyHostToDevice, s);
-        cudaMemcpyAsync(pg.d_maps, pg.maps.data(), sizeof(CUtensorMap) * pg.maps.size(), cudaMemcpyHostToDevice, s);
-        cudaMemsetAsync(pg.d_op_done, 0, sizeof(int) * pg.ops.size(), s);
-        cudaMemsetAsync(pg.d_tile_cnt, 0, sizeof(int) * (size_t)pg.ops.size() * L.max_tiles, s);
-        pg.epoch = 0;
+    void finish_program(PassProgram &pg) {
         cudaMemsetAsync(pg.d_dep, 0, sizeof(int) * 2 * pg.ops.size(), s);
         pg.dep_run = 0;
         pg.dep_ctas.assign(2 * pg.ops.size(), 0);
@@ -965,16 +895,10 @@ class Engine : public EngineBase {
         const dflash_model_cfg &m = c.target;
         const int B = c.block_size, R = nseq * B, H = m.hidden, hd = m.head_dim;
         const int qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd, TK = c.n_taps * H;
-        ChainProgram &pg = pv;
+        PassProgram &pg = pv;
         pg.ops.clear();
         pg.hops.clear();
-        pg.maps.clear();
-        pg.tinfo.clear();
-        pg.valid = true;
-        pg.tm = pow2_at_least(R, 16);
-        pg.planes = lo_ ? 2 : 1;
         pg.key = nseq;
-        int toff = 0;
         auto qkv = [&](int l) {
             Epi<T> e;
             e.kind = EPI_QKV;
@@ -988,7 +912,7 @@ class Engine : public EngineBase {
             e.q_out = q;
             e.kc = tk + (size_t)l * kv_layer_elems(m);
             e.vc = tv + (size_t)l * kv_layer_elems(m);
-            chain_add(pg, toff, EPI_QKV, tl[l].wqkv, qd + 2 * kd, H, xg_t, H, R, epi_norm_in(e, (float)m.rms_eps, H));
+            prog_add(pg, EPI_QKV, tl[l].wqkv, qd + 2 * kd, H, xg_t, H, R, epi_norm_in(e, (float)m.rms_eps, H));
         };
         qkv(0);
         for (int l = 0; l < m.n_layers; ++l) {
@@ -996,12 +920,12 @@ class Engine : public EngineBase {
             o.kind = EPI_RESID;
             o.x = x;
             o.meta = meta;
-            chain_add(pg, toff, EPI_RESID, tl[l].wo, H, qd, ao, qd, R, epi_norm_out(o, xg2, tl[l].ffn_norm, ssq));
+            prog_add(pg, EPI_RESID, tl[l].wo, H, qd, ao, qd, R, epi_norm_out(o, xg2, tl[l].ffn_norm, ssq));
             Epi<T> gu;
             gu.kind = EPI_SWIGLU;
             gu.h = h;
             gu.F = m.ffn;
-            chain_add(pg, toff, EPI_SWIGLU, tl[l].w_gate_up, 2 * m.ffn, H, xg2, H, R, epi_norm_in(gu, (float)m.rms_eps, H));
+            prog_add(pg, EPI_SWIGLU, tl[l].w_gate_up, 2 * m.ffn, H, xg2, H, R, epi_norm_in(gu, (float)m.rms_eps, H));
             Epi<T> dn;
             dn.kind = EPI_RESID;
             dn.x = x;
@@ -1013,7 +937,7 @@ class Engine : public EngineBase {
                 if (c.tap_layers[i] == l) taps.col[taps.n++] = i * H;
             dn.taps = taps;
             const float *gn = l + 1 < m.n_layers ? tl[l + 1].attn_norm : t_final;
-            chain_add(pg, toff, EPI_RESID, tl[l].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, xg_t, gn, ssq));
+            prog_add(pg, EPI_RESID, tl[l].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, xg_t, gn, ssq));
             if (l + 1 < m.n_layers) {
                 qkv(l + 1);
             } else {
@@ -1021,7 +945,7 @@ class Engine : public EngineBase {
                 lg.kind = EPI_LOGITS;
                 lg.Y = logits;
                 lg.ldy = m.vocab;
-                chain_add(pg, toff, EPI_LOGITS, lm_head, m.vocab, H, xg_t, H, R, epi_norm_in(lg, (float)m.rms_eps, H));
+                prog_add(pg, EPI_LOGITS, lm_head, m.vocab, H, xg_t, H, R, epi_norm_in(lg, (float)m.rms_eps, H));
             }
         }
         finish_program(pg);
@@ -1032,19 +956,13 @@ class Engine : public EngineBase {
         const dflash_model_cfg &m = c.drafter;
         const int B = c.block_size, R = nseq * B, H = m.hidden, hd = m.head_dim;
         const int qd = m.n_q_heads * hd, kd = m.n_kv_heads * hd, TK = c.n_taps * c.target.hidden;
-        ChainProgram &pg = pd;
+        PassProgram &pg = pd;
         pg.ops.clear();
         pg.hops.clear();
-        pg.maps.clear();
-        pg.tinfo.clear();
-        pg.valid = true;
-        pg.tm = pow2_at_least(2 * R, 16);
-        pg.planes = lo_ ? 2 : 1;
         pg.key = nseq;
-        int toff = 0;
         Epi<T> f;
         f.kind = EPI_NORMOUT;
-        chain_add(pg, toff, EPI_NORMOUT, w_fc, H, TK, taps_dec, TK, R, epi_norm_out(f, dq_in + (size_t)R * H, fc_norm, ssq + R));
+        prog_add(pg, EPI_NORMOUT, w_fc, H, TK, taps_dec, TK, R, epi_norm_out(f, dq_in + (size_t)R * H, fc_norm, ssq + R));
         auto qkv = [&](int j) {
             Epi<T> e;
             e.kind = EPI_QKV;
@@ -1059,7 +977,7 @@ class Engine : public EngineBase {
             e.q_out = q;
             e.kc = dk + (size_t)j * kv_layer_elems(m);
             e.vc = dv + (size_t)j * kv_layer_elems(m);
-            chain_add(pg, toff, EPI_QKV, dl[j].wqkv, qd + 2 * kd, H, dq_in, H, 2 * R, epi_norm_in(e, (float)m.rms_eps, H));
+            prog_add(pg, EPI_QKV, dl[j].wqkv, qd + 2 * kd, H, dq_in, H, 2 * R, epi_norm_in(e, (float)m.rms_eps, H));
         };
         qkv(0);
         for (int j = 0; j < m.n_layers; ++j) {
@@ -1067,41 +985,34 @@ class Engine : public EngineBase {
             o.kind = EPI_RESID;
             o.x = x;
             o.meta = meta;
-            chain_add(pg, toff, EPI_RESID, dl[j].wo, H, qd, ao, qd, R, epi_norm_out(o, xg2, dl[j].ffn_norm, ssq));
+            prog_add(pg, EPI_RESID, dl[j].wo, H, qd, ao, qd, R, epi_norm_out(o, xg2, dl[j].ffn_norm, ssq));
             Epi<T> gu;
             gu.kind = EPI_SWIGLU;
             gu.h = h;
             gu.F = m.ffn;
-            chain_add(pg, toff, EPI_SWIGLU, dl[j].w_gate_up, 2 * m.ffn, H, xg2, H, R, epi_norm_in(gu, (float)m.rms_eps, H));
+            prog_add(pg, EPI_SWIGLU, dl[j].w_gate_up, 2 * m.ffn, H, xg2, H, R, epi_norm_in(gu, (float)m.rms_eps, H));
             Epi<T> dn;
             dn.kind = EPI_RESID;
             dn.x = x;
             dn.meta = meta;
             if (j + 1 < m.n_layers) {
-                chain_add(pg, toff, EPI_RESID, dl[j].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, dq_in, dl[j + 1].attn_norm, ssq));
+                prog_add(pg, EPI_RESID, dl[j].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, dq_in, dl[j + 1].attn_norm, ssq));
                 qkv(j + 1);
             } else {
-                chain_add(pg, toff, EPI_RESID, dl[j].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, xg_t, d_final, ssq));
+                prog_add(pg, EPI_RESID, dl[j].w_down, H, m.ffn, h, m.ffn, R, epi_norm_out(dn, xg_t, d_final, ssq));
                 Epi<T> lg;
                 lg.kind = EPI_LOGITS;
                 lg.Y = draft_logits();
                 lg.ldy = c.target.vocab;
-                chain_add(pg, toff, EPI_LOGITS, lm_head, c.target.vocab, H, xg_t, H, R, epi_norm_in(lg, (float)m.rms_eps, H));
+                prog_add(pg, EPI_LOGITS, lm_head, c.target.vocab, H, xg_t, H, R, epi_norm_in(lg, (float)m.rms_eps, H));
             }
         }
         finish_program(pg);
     }
 
-    // ops [b, e) of a program: one persistent chain launch, or one projection kernel each
-    void run_ops(ChainProgram &pg, int b, int e) {
+    // ops [b, e) of a program, one projection kernel each
+    void run_ops(PassProgram &pg, int b, int e) {
         if constexpr (std::is_same<T, bf16>::value) {
-            if (chain_on && pg.valid) {
-                double bytes = 0.0;
-                for (int i = b; i < e; ++i)
-                    bytes += gemm_bytes(pg.hops[i].M, pg.hops[i].N, pg.hops[i].K, pg.ops[i].e);
-                timed(0, bytes, [&] { launch_chain(pg, b, e, num_sms, &stats->status, s); });
-                return;
-            }
             for (int i = b; i < e; ++i) {
                 const HostOp &h = pg.hops[i];
                 int tgt = 0;
@@ -1117,11 +1028,11 @@ class Engine : public EngineBase {
     // projection and attention launch waits until every CTA of the launch before
     // it has signalled (instead of waiting for that grid to exit and flush), which
     // lets it start about as soon as the last epilogue store is visible.
-    void pass_begin(ChainProgram &pg) {
+    void pass_begin(PassProgram &pg) {
         pg.dep_run += 1;
         pg.dep_prev = -1;  // the first launch of a pass waits with griddepcontrol.wait
     }
-    const int *pass_dep(ChainProgram &pg, int &target) {
+    const int *pass_dep(PassProgram &pg, int &target) {
         if (!dep_on || pg.dep_prev < 0) {
             target = 0;
             return nullptr;
@@ -1129,12 +1040,12 @@ class Engine : public EngineBase {
         target = (int)pg.dep_run * pg.dep_ctas[pg.dep_prev];
         return pg.d_dep + pg.dep_prev;
     }
-    void pass_done(ChainProgram &pg, int idx, int ctas) {
+    void pass_done(PassProgram &pg, int idx, int ctas) {
         if (!dep_on) return;
         pg.dep_ctas[idx] = ctas;
         pg.dep_prev = ctas > 0 ? idx : -1;  // a launch that signals nothing cannot be waited on
     }
-    AttnSync pass_attn_sync(ChainProgram &pg, int layer, int &idx) {
+    AttnSync pass_attn_sync(PassProgram &pg, int layer, int &idx) {
         AttnSync sy;
         idx = (int)pg.ops.size() + layer;
         if (!dep_on) return sy;
@@ -1144,11 +1055,10 @@ class Engine : public EngineBase {
         return sy;
     }
 
-    void enqueue_verify_chain(int nseq) {
+    void enqueue_verify_folded(int nseq) {
         const dflash_model_cfg &t = c.target;
         const int B = c.block_size, R = nseq * B, H = t.hidden;
         if (pv.key != nseq) build_verify_program(nseq);
-        if (chain_on && pv.valid) pv.epoch++;
         pass_begin(pv);
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, tl[0].attn_norm,
                              xg_t, H, lo_, ssq, L.ssq_ld, s);
@@ -1168,14 +1078,13 @@ class Engine : public EngineBase {
             launch_lm_argmax(lm_part, (t.vocab + 127) / 128, R, 0, B, g, stats, s);
             launch_accept(st, active, nseq, B, drafts, g, accept, committed, new_len, out_tok, c.max_len, stats, s);
         }
-        chain_used[1] = true;
+        fold_used[1] = true;
     }
 
-    void enqueue_draft_chain(int nseq) {
+    void enqueue_draft_folded(int nseq) {
         const dflash_model_cfg &d = c.drafter;
         const int B = c.block_size, R = nseq * B, H = d.hidden;
         if (pd.key != nseq) build_draft_program(nseq);
-        if (chain_on && pd.valid) pd.epoch++;
         pass_begin(pd);
         launch_embed_norm<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, dl[0].attn_norm,
                              dq_in, H, lo_, ssq, L.ssq_ld, s);
@@ -1196,7 +1105,7 @@ class Engine : public EngineBase {
         }
         if (draft_mode == DFLASH_DRAFT_SCRIPT)
             launch_script_drafts(st, active, nseq, B, tau, c.target.vocab, script, c.max_len, drafts, s);
-        chain_used[0] = true;
+        fold_used[0] = true;
     }
 
     // ---- steps ----
@@ -1249,12 +1158,12 @@ class Engine : public EngineBase {
     }
 
     void enqueue_draft(int nseq, bool contiguous) {
-        if (chain_draft_ok && contiguous) {
+        if (fold_draft_ok && contiguous) {
             if (pd.key != nseq) build_draft_program(nseq);
-            enqueue_draft_chain(nseq);
+            enqueue_draft_folded(nseq);
             return;
         }
-        chain_used[0] = false;
+        fold_used[0] = false;
         const dflash_model_cfg &t = c.target, &d = c.drafter;
         const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
         launch_embed_block<T>(embed, H, st, active, nseq, B, 1, nullptr, c.mask_token_id, x, meta, ctx_meta, s);
@@ -1285,12 +1194,12 @@ class Engine : public EngineBase {
     }
 
     void enqueue_verify(int nseq) {
-        if (chain_verify_ok) {
+        if (fold_verify_ok) {
             if (pv.key != nseq) build_verify_program(nseq);
-            enqueue_verify_chain(nseq);
+            enqueue_verify_folded(nseq);
             return;
         }
-        chain_used[1] = false;
+        fold_used[1] = false;
         const dflash_model_cfg &t = c.target;
         const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
         launch_embed_block<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
@@ -1352,17 +1261,20 @@ class Engine : public EngineBase {
         if (n + c.block_size > c.max_len) { err = "prompt + block exceeds max_len"; return DFLASH_ECAPACITY; }
         for (int i = 0; i < n; ++i)
             if (prompt[i] < 0 || prompt[i] >= c.target.vocab) { err = "prompt id out of vocab"; return DFLASH_EINVAL; }
+        last_pass = PASS_NONE;
         if (cudaMemcpyAsync(tokens, prompt, sizeof(int32_t) * n, cudaMemcpyHostToDevice, s) != cudaSuccess)
             return fail_cuda("prompt copy");
         enqueue_prefill(seq, n, max_new);
         dflash_status r = check("prefill launch");
         if (r) return r;
+        last_pass = PASS_PREFILL;
         h_len[seq] = n;
         h_prefilled[seq] = 1;
         last_draft.clear();
         last_logits_rows[2] = 1;
         if (first) {
             if ((r = sync("prefill"))) return r;
+            if ((r = numeric_status())) return r;
             if (cudaMemcpy(first, first_tok, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return fail_cuda("first token");
         }
         return DFLASH_OK;
@@ -1383,12 +1295,15 @@ class Engine : public EngineBase {
         dflash_status r = check_seqs(seqs, n);
         if (r) return r;
         if ((r = set_active(seqs, n))) return r;
+        last_pass = PASS_NONE;
         enqueue_draft(n, is_iota(seqs, n));
         if ((r = check("draft launch"))) return r;
+        last_pass = PASS_DRAFT;
         last_draft.assign(seqs, seqs + n);
         last_logits_rows[0] = n * c.block_size;
         if (out && c.block_size > 1) {
             if ((r = sync("draft"))) return r;
+            if ((r = numeric_status())) return r;
             if (cudaMemcpy(out, drafts, sizeof(int32_t) * n * (c.block_size - 1), cudaMemcpyDeviceToHost) != cudaSuccess)
                 return fail_cuda("drafts copy");
         }
@@ -1410,8 +1325,10 @@ class Engine : public EngineBase {
             if (B > 1 && cudaMemcpyAsync(drafts, dr, sizeof(int32_t) * n * (B - 1), cudaMemcpyHostToDevice, s) != cudaSuccess)
                 return fail_cuda("drafts copy");
         }
+        last_pass = PASS_NONE;
         enqueue_verify(n);
         if ((r = check("verify launch"))) return r;
+        last_pass = PASS_VERIFY;
         last_draft.clear();
         last_logits_rows[1] = n * B;
         if ((r = sync("verify"))) return r;
@@ -1419,6 +1336,7 @@ class Engine : public EngineBase {
         if (cudaMemcpy(lens.data(), new_len, sizeof(int32_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
             return fail_cuda("new_len copy");
         for (int i = 0; i < n; ++i) h_len[seqs[i]] = lens[i];
+        if ((r = numeric_status())) return r;
         if (nl) std::copy(lens.begin(), lens.end(), nl);
         if (acc && cudaMemcpy(acc, accept, sizeof(int32_t) * n, cudaMemcpyDeviceToHost) != cudaSuccess)
             return fail_cuda("accept copy");
@@ -1427,11 +1345,19 @@ class Engine : public EngineBase {
         return DFLASH_OK;
     }
 
-    dflash_status numeric_status() {
-        DevStats hs;
-        if (cudaMemcpy(&hs, stats, sizeof hs, cudaMemcpyDeviceToHost) != cudaSuccess) return fail_cuda("stats copy");
-        if (hs.status) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
+    // The device status word (stream already synchronised): bit 0 a non-finite
+    // logit reached an argmax, bits 2-4 a bounded device wait expired.  Sticky
+    // until dflash_reset_stats or the next generation.
+    static dflash_status status_code(int st, std::string &err) {
+        if (st & 1) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
+        if (st & (4 | 8 | 16)) { err = "a bounded device wait expired"; return DFLASH_ETIMEOUT; }
         return DFLASH_OK;
+    }
+    dflash_status numeric_status() {
+        int32_t st = 0;
+        if (cudaMemcpy(&st, &stats->status, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return fail_cuda("status copy");
+        return status_code(st, err);
     }
 
     dflash_status start_run(const int32_t *const *prompts, const int32_t *lens, int n, int max_new) {
@@ -1502,6 +1428,7 @@ class Engine : public EngineBase {
     dflash_status generate(const int32_t *const *prompts, const int32_t *lens, int n, int max_new, int32_t *out,
                            dflash_stats *ost) override {
         ScopedEvents ev;
+        OtherPass mark{last_pass};
         cudaEvent_t t0 = ev.e[0], t1 = ev.e[1], t2 = ev.e[2];
         cudaEventRecord(t0, s);
         dflash_status r = start_run(prompts, lens, n, max_new);
@@ -1536,13 +1463,14 @@ class Engine : public EngineBase {
         }
         // generation leaves the slots in a finished state: refuse draft/verify on them
         for (int i = 0; i < n; ++i) h_prefilled[i] = 0;
-        if (hs.status) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
+        if ((r = status_code(hs.status, err))) return r;
         return check("generate");
     }
 
     dflash_status generate_ar(const int32_t *const *prompts, const int32_t *lens, int n, int max_new, int32_t *out,
                               double *ms) override {
         ScopedEvents ev;
+        OtherPass mark{last_pass};
         cudaEvent_t t1 = ev.e[0], t2 = ev.e[1];
         dflash_status r = start_run(prompts, lens, n, max_new);
         if (r) return r;
@@ -1649,6 +1577,7 @@ class Engine : public EngineBase {
         std::vector<int32_t> iota(n);
         for (int i = 0; i < n; ++i) iota[i] = i;
         if ((r = set_active(iota.data(), n))) return r;
+        OtherPass mark{last_pass};
         for (int it = 0; it < iters; ++it) {
             enqueue_draft(n, true);
             enqueue_verify(n);
@@ -1670,8 +1599,7 @@ class Engine : public EngineBase {
         for (int i = 0; i < DFLASH_MAX_BLOCK; ++i) o->accept_hist[i] = (int64_t)hs.hist[i];
         o->mean_tau = hs.iterations ? (double)hs.tokens / (double)hs.iterations : 0.0;
         o->kernel_launches = launch_count();
-        if (hs.status & 4) { err = "a bounded device wait expired"; return DFLASH_ETIMEOUT; }
-        return DFLASH_OK;
+        return status_code(hs.status, err);
     }
 
     dflash_status reset_stats() override {
@@ -1715,6 +1643,14 @@ class Engine : public EngineBase {
         if (!std::is_same<T, bf16>::value) { err = "dflash_head_argmax_noalloc needs a bf16 context"; return DFLASH_EUNSUPPORTED; }
         if (which < 0 || which > 2 || !host_out || !rows_out) { err = "bad dflash_head_argmax_noalloc arguments"; return DFLASH_EINVAL; }
         const int V = c.target.vocab, H = c.target.hidden, B = c.block_size;
+        if (last_pass != which) {
+            err = "the last pass on this context is not of the requested kind (call right after that pass)";
+            return DFLASH_ESTATE;
+        }
+        if (sampling_on() || (which == 0 && draft_mode == DFLASH_DRAFT_SCRIPT)) {
+            err = "dflash_head_argmax_noalloc returns greedy argmaxes: not with sampling or script drafts";
+            return DFLASH_ESTATE;
+        }
         const int rows = last_logits_rows[which];
         const int n_tiles = (V + 127) / 128;
         if (rows < 1) { err = "no pass of that kind has run on this context"; return DFLASH_ESTATE; }
@@ -1732,15 +1668,20 @@ class Engine : public EngineBase {
         const int saved_keep = tc.keep_logits;
         tc.lm_part = part;
         tc.keep_logits = 0;
-        if (which < 2 && chain_used[which]) {
-            // chain passes feed the head bf16(x * g_final) and scale each row by its RMSNorm factor
+        int ctas = 0;
+        if (which < 2 && fold_used[which]) {
+            // folded passes feed the head bf16(x * g_final) and scale each row by its RMSNorm factor
             const float eps = (float)(which == 0 ? c.drafter.rms_eps : c.target.rms_eps);
-            gemm_launch(xg_t, H, rows, lm_head, V, H, epi_norm_in(e, eps, H));
+            ctas = gemm_launch(xg_t, H, rows, lm_head, V, H, epi_norm_in(e, eps, H));
         } else {
-            gemm_launch(xn, H, rows, lm_head, V, H, e);
+            ctas = gemm_launch(xn, H, rows, lm_head, V, H, e);
         }
         tc.lm_part = saved_part;
         tc.keep_logits = saved_keep;
+        if (ctas < 1) {  // every partial the argmax reads must come from this call
+            err = "dflash_head_argmax_noalloc: LM-head projection not launched: " + tc.err;
+            return DFLASH_ECUDA;
+        }
         const int mode = which == 0 ? 1 : 0;
         launch_lm_argmax(part, n_tiles, rows, mode, B, idx, nullptr, s);
         const int n_out = which == 0 ? (rows / B) * (B - 1) : rows;
@@ -1770,6 +1711,21 @@ using namespace dfl;
 // C ABI
 // ------------------------------------------------------------------------
 
+// Every call runs with the context's device current (restored on return), so
+// one host thread can drive contexts on several devices.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+        else prev = -1;
+    }
+    ~DeviceGuard() {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
 extern "C" {
 
 dflash_status dflash_workspace_size(const dflash_config *cfg, size_t *wb, size_t *sb) {
@@ -1797,6 +1753,10 @@ dflash_status dflash_create(const dflash_config *cfg, void *warena, size_t wbyte
         return DFLASH_EINVAL;
     }
     for (size_t i = 0; i < ctx->lay.slots.size(); ++i) ctx->by_name[ctx->lay.slots[i].name] = (int)i;
+    if (cudaGetDevice(&ctx->device) != cudaSuccess) {
+        delete ctx;
+        return DFLASH_ECUDA;
+    }
     cudaStream_t s = (cudaStream_t)stream;
     if (cfg->dtype != DFLASH_FP32)
         ctx->eng.reset(new Engine<bf16>(*cfg, ctx->lay, (char *)warena, (char *)sarena, s));
@@ -1814,7 +1774,11 @@ dflash_status dflash_create(const dflash_config *cfg, void *warena, size_t wbyte
     return DFLASH_OK;
 }
 
-void dflash_destroy(dflash_ctx *ctx) { delete ctx; }
+void dflash_destroy(dflash_ctx *ctx) {
+    if (!ctx) return;
+    DeviceGuard g(ctx->device);
+    delete ctx;
+}
 
 const char *dflash_last_error(const dflash_ctx *ctx) {
     if (!ctx) return "null context";
@@ -1852,6 +1816,8 @@ dflash_status dflash_weight_slot(const dflash_ctx *ctx, const char *name, size_t
     do {                                                                      \
         if (!(ctx)) return DFLASH_EINVAL;                                     \
         if ((ctx)->broken) { (ctx)->err = "context unusable after a CUDA error"; return DFLASH_ECUDA; } \
+        DeviceGuard _dg((ctx)->device);                                       \
+        if (!_dg.ok) { (ctx)->err = "cannot make the context's device current"; return DFLASH_ECUDA; } \
         dflash_status _r = (expr);                                            \
         (ctx)->err = _r ? (ctx)->eng->err : std::string();                    \
         if (_r == DFLASH_ECUDA) (ctx)->broken = true;                         \
@@ -1899,8 +1865,12 @@ dflash_status dflash_profile_read(dflash_ctx *ctx, dflash_kernel_prof *out) {
 
 dflash_status dflash_head_argmax_noalloc(dflash_ctx *ctx, int32_t which, int32_t *host_out, int32_t *rows_out) {
     if (!ctx) return DFLASH_EINVAL;
+    if (ctx->broken) {
+        ctx->err = "context unusable after a CUDA error";
+        return DFLASH_ECUDA;
+    }
     std::string e;
-    void *scratch = noalloc_scratch_ptr(e);
+    void *scratch = noalloc_scratch_ptr(ctx->device, e);
     if (!scratch) {
         ctx->err = e;
         return DFLASH_ECUDA;

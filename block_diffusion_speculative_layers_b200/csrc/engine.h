@@ -11,6 +11,8 @@
 
 namespace dfl {
 
+constexpr int kMaxDevices = 64;
+
 struct WeightSlot {
     std::string name;
     size_t offset = 0, numel = 0;
@@ -36,10 +38,9 @@ struct Layout {
     size_t rope_t, rope_d, tk, tv, dk, dv, script, out_tok, tokens, stats, first_tok;
     size_t moe_sel, moe_wt, moe_part, moe_off = 0, moe_list = 0, lm_part, att_o, att_ml, att_sem;
     size_t att_parts = 0;
-    size_t xg_t, xg2, ssq, chain_v, chain_d, chain_ws;
+    size_t xg_t, xg2, ssq, dep_v, dep_d;
     size_t act_lo = 0;  // two-plane activations: low plane offset in elements (0: one plane)
-    size_t chain_v_bytes = 0, chain_d_bytes = 0, chain_ws_floats = 0;
-    int ssq_ld = 0, n_ops_v = 0, n_ops_d = 0, max_tiles = 0;
+    int ssq_ld = 0, n_ops_v = 0, n_ops_d = 0;
     size_t gemm_ws, gemm_sem;
     size_t state_bytes = 0;
     // dims
@@ -87,4 +88,5 @@ struct dflash_ctx {
     std::unique_ptr<dfl::EngineBase> eng;
     std::string err;
     bool broken = false;
+    int device = 0;  // CUDA device the context was created on
 };

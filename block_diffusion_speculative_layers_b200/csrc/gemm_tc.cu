@@ -443,11 +443,7 @@ template <int TM, int KIND>
 static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p, const Epi<bf16> &e,
                       int stages, size_t smem, cudaStream_t s, int grid_x) {
     auto kern = tc::gemm_tc_kernel<TM, KIND>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        attr_set = true;
-    }
+    ensure_smem_attr((const void *)kern);
     (void)grid_x;
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
     launch_k(kern, grid, dim3(tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
@@ -517,7 +513,10 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int K
     const int grid_x = p.n_tiles;  // one tile per CTA
     const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
     const CUtensorMap *mx = tensor_map(X, M, K, ldx, TM, e.lo);
-    if (!mw || !mx) return 0;
+    if (!mw || !mx) {
+        failed = true;
+        return 0;
+    }
     switch (TM) {
         case 16: launch_kind<16>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
         case 32: launch_kind<32>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;

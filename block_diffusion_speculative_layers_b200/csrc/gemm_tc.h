@@ -42,6 +42,7 @@ struct TcParams {
 template <typename T>
 struct GemmTC {
     std::string err;
+    bool failed = false;  // a launch was dropped (tensor map encoding failed); err says why
     bool supports(int M, int N, int K) const;
     int init(float *ws, int ws_floats, int *sem, int n_sem);
     // returns the number of CTAs launched (the count a completion counter reaches per run)

@@ -4,9 +4,29 @@
 
 #include <cuda_runtime.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "kernels.h"
 
 namespace dfl {
+
+// Raise a kernel's dynamic shared-memory limit to the B200 maximum (227 KB),
+// once per (kernel, device): the attribute is per device, so a process that
+// drives several devices sets it on each.  Thread-safe.
+inline cudaError_t ensure_smem_attr(const void *kern) {
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kern, dev})) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e == cudaSuccess) done.insert({kern, dev});
+    return e;
+}
 
 // Process-wide switch for programmatic dependent launch (on by default).
 bool &pdl_enabled();

@@ -438,12 +438,8 @@ void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k
                                  const bf16 *w_gate_up, const bf16 *w_down, int H, int Fe, int *off, int *list,
                                  bf16 *h, size_t hlo, float *part, int num_sms, int *err, cudaStream_t s) {
     if (R <= 0) return;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(moe_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        cudaFuncSetAttribute(moe_stream_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        attr = true;
-    }
+    ensure_smem_attr((const void *)moe_stream_kernel<true>);
+    ensure_smem_attr((const void *)moe_stream_kernel<false>);
     int *touched = off + E + 1;
     launch_k(moe_bucket_kernel, dim3(1), dim3(1024), 0, s, 1, sel, R * k, E, off, list, touched);
     // streaming for at most two pairs per expert on average; beyond that the

@@ -390,10 +390,12 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
     } else if (KIND == EPI_LOGITS) {
         const int n = nt * 128 + n_local;
         const bool ok = n < p.N;
+        bool bad = false;  // a non-finite logit anywhere in the row makes the argmax meaningless
 #pragma unroll
         for (int j = 0; j < W; ++j) {
             const int m = m0c + j;
             const bool col = j < nc && m < M;
+            bad |= ok && col && !isfinite(v[j]);
             if (p.keep_logits && ok && col) e.Y[(size_t)m * e.ldy + n] = v[j];
             float bv = (ok && col) ? v[j] : -INFINITY;
             int bi = (ok && col) ? n : 0x7fffffff;
@@ -405,6 +407,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
             }
             if (lane == 0) red[q * CH + j] = make_float2(bv, __int_as_float(bi));
         }
+        if (__any_sync(0xffffffffu, bad) && lane == 0 && p.err) atomicOr(p.err, 1);
         epi_bar();
         if (threadIdx.x >= 64 && threadIdx.x < 64 + W) {
             const int j = threadIdx.x - 64;

@@ -30,7 +30,9 @@
  *  - Device memory: the caller allocates two device arenas (weights, state) of
  *    the sizes dflash_workspace_size reports and keeps them alive until
  *    dflash_destroy.  The library allocates no device memory of its own.
- *  - All GPU work is enqueued on the CUDA stream given to dflash_create.
+ *  - All GPU work is enqueued on the CUDA stream given to dflash_create, on
+ *    the device that was current at dflash_create; every call makes that
+ *    device current for its duration and restores the caller's afterwards.
  *  - A context is not thread-safe; use one context per host thread.
  */
 #ifndef DFLASH_H
@@ -160,24 +162,42 @@ dflash_status dflash_weight_slot(const dflash_ctx *ctx, const char *name, size_t
  * the prompt (KV cache positions 0..n-1), taps fused into the drafter's
  * context K/V for the same positions, first greedy token returned (it is the
  * anchor of the first block).  Resets the slot.
+ * Pages: the prompt pass is not described; it builds what "O alvo sabe mais"
+ * (iaemfoco.com DFlash page) needs before the first block -- the target's KV
+ * cache and the hidden states of the tapped layers for every prompt position,
+ * fused into the context K/V of every drafter layer.
  * Errors: EINVAL (seq out of range, n < 1, ids out of vocab), ECAPACITY
- * (n + block_size > max_len). */
+ * (n + block_size > max_len); with first_token: ENUMERIC (non-finite logits,
+ * device status word), ETIMEOUT. */
 dflash_status dflash_prefill(dflash_ctx *ctx, int32_t seq, const int32_t *prompt, int32_t n,
                              int32_t *first_token);
 
 /* One drafter forward for the listed sequences (seqs[0..n), distinct, each
  * prefilled): block [anchor, mask x (B-1)] at positions p..p+B-1 attends
  * bidirectionally over the context K/V [0, p) and the block itself.
+ * Pages: iaemfoco.com DFlash page, "O que o DFlash faz de diferente" (the
+ * drafter fills the whole block in one parallel forward) and "O alvo sabe
+ * mais" (the context vector of the positions the last verify committed,
+ * RMSNorm(W_fc . concat(taps)), is injected into the K/V projections of every
+ * drafter layer first); ceviu.com.br page (16 tokens per drafter pass).
  * drafts: host [n*(B-1)] or NULL (then nothing is copied and the call does not
- * synchronise).  Errors: EINVAL, ESTATE, ECAPACITY. */
+ * synchronise).  Errors: EINVAL, ESTATE, ECAPACITY; with drafts: ENUMERIC,
+ * ETIMEOUT. */
 dflash_status dflash_draft_block(dflash_ctx *ctx, const int32_t *seqs, int32_t n, int32_t *drafts);
 
 /* Target verify of [anchor, d_1..d_{B-1}] for the same sequences as the last
  * dflash_draft_block (drafts == NULL: use the drafter's; else host [n*(B-1)]
  * supplied by the caller), greedy acceptance a = longest prefix with
  * d_i == g_{i-1}, commit of d_1..d_a and the bonus g_a, KV rollback by length.
+ * Pages: iaemfoco.com DFlash page, "O que o DFlash faz de diferente" (the
+ * target checks the whole block in one parallel pass) and "Decodificação
+ * especulativa tradicional" (accepted tokens are kept; the output equals
+ * target-only decoding); imasters.com.br page, "Os três mecanismos por trás do
+ * DFlash" (verification in parallel keeps the target's distribution).
  * accept [n], committed [n*B] (first a+1 valid), new_len [n]: host or NULL.
- * Errors: EINVAL, ESTATE (no preceding draft for these sequences). */
+ * Errors: EINVAL, ESTATE (no preceding draft for these sequences); ENUMERIC
+ * when a non-finite logit reached an argmax (device status word, sticky until
+ * dflash_reset_stats); ETIMEOUT (host wait, or a bounded device wait expired). */
 dflash_status dflash_verify_commit(dflash_ctx *ctx, const int32_t *seqs, int32_t n,
                                    const int32_t *drafts, int32_t *accept, int32_t *committed,
                                    int32_t *new_len);
@@ -254,12 +274,16 @@ dflash_status dflash_debug_kv(dflash_ctx *ctx, int32_t which, int32_t layer, int
  * process that reserved its whole device memory pool up front, or a runtime
  * that forbids cudaMalloc on its decode thread (cudaMalloc can synchronise
  * the device and may fail once the pool is carved up).
- * It recomputes the argmax over the vocabulary of the rows that the last
- * pass on this context fed to the LM head -- which = 0: the drafter rows of
- * the last dflash_draft_block (outputs: n*(B-1) draft ids, as that call
+ * It recomputes the greedy argmax over the vocabulary of the rows that the
+ * last pass on this context fed to the LM head -- which = 0: the drafter rows
+ * of the last dflash_draft_block (outputs: n*(B-1) draft ids, as that call
  * returns them); 1: the rows of the last dflash_verify_commit (n*B ids);
- * 2: the last row of the last dflash_prefill (1 id) -- and must be called
- * right after that pass, before any other call on the context.  The per-tile
+ * 2: the last row of the last dflash_prefill (1 id).  The pass named by
+ * `which` must be the last one that ran on the context: DFLASH_ESTATE after
+ * any other pass (a draft, verify or prefill of another kind, or
+ * dflash_generate / dflash_generate_ar / dflash_decode_iters), before any pass,
+ * with temperature sampling on, and for which = 0 with script drafts (the
+ * ids would not be what the pass returned).  The per-tile
  * partial maxima and the output ids live in one file-scope device array of
  * the library (about 1 MiB; every GPU that loads the library holds it until
  * exit) instead of in the state arena, so the call allocates nothing: no
@@ -273,7 +297,9 @@ dflash_status dflash_debug_kv(dflash_ctx *ctx, int32_t which, int32_t layer, int
  * the last call's contents; every element a call reads is written by the
  * same call first, so nothing needs clearing.
  * host_out: host buffer of at least *rows_out ids (n*(B-1), n*B or 1);
- * rows_out: receives the number of ids written.  Synchronises the stream. */
+ * rows_out: receives the number of ids written.  Synchronises the stream.
+ * DFLASH_ECUDA if the array's address cannot be looked up or the LM-head
+ * projection could not be launched. */
 dflash_status dflash_head_argmax_noalloc(dflash_ctx *ctx, int32_t which, int32_t *host_out, int32_t *rows_out);
 
 #ifdef __cplusplus

@@ -129,3 +129,83 @@ def check_lossless_generate(gpu, spec, cfg, prompt, max_new, tie):
         assert margins[k] < tie, (k, out[:k + 2], ar[:k + 2], margins[k])
         return k, st
     return None, st
+
+
+def replay_forced(gpu, spec, cfg, prompt, cuts, tol, tie, seq=0, check_kv=True, kv_tol=1e-2):
+    """Greedy acceptance at chosen lengths: the caller's drafts are the oracle's
+    own target-only continuation, made wrong at draft k+1 (none wrong for
+    k = B-1), so the verify must accept exactly k drafts and commit k+1 tokens
+    -- unless a counted near-tie of the oracle sits at an index <= k.  Each
+    iteration checks the drafter and verify logits against the oracle replaying
+    the same block, the accept length / committed tokens / new length bit for
+    bit against the rule on the GPU's own argmaxes, the committed tokens against
+    the oracle's continuation, and the target K/V of the committed positions
+    and the drafter context K/V injected for them against the oracle's."""
+    rep = Report()
+    B, V = cfg.block_size, cfg.target.vocab
+    n_ar = 1 + sum(k + 1 for k in cuts) + B
+    ar, ar_mg = spec.generate_ar(prompt, n_ar, with_margins=True)
+    ss = spec.session(len(prompt) + n_ar + 2 * B)
+    first = gpu.prefill(seq, prompt)
+    tok_o, mg, lg_o = ss.prefill(prompt, want_logits=True)
+    lg = gpu.debug_logits(2, 1)[0]
+    rep.max_dlogit = max(rep.max_dlogit, float(np.abs(lg - lg_o).max()))
+    assert first == tok_o or mg < tie
+    assert first == ar[0] or ar_mg[0] < tie
+    j = 0  # index of the anchor in the continuation
+    anchor = first
+    for k in cuts:
+        assert 0 <= k <= B - 1
+        d_gpu = gpu.draft_block([seq])[0]
+        if B > 1:
+            d_o, mg_d, dl_o = ss.draft(anchor, want_logits=True)
+            dl = gpu.debug_logits(0, B)[1:]
+            rep.max_dlogit = max(rep.max_dlogit, float(np.abs(dl - dl_o).max()))
+            _cmp_tokens(d_gpu, d_o, mg_d, tie, rep)
+        drafts = [int(t) for t in ar[j + 1:j + B]]
+        if k < B - 1:
+            drafts[k] = (drafts[k] + 1) % V
+        p0 = ss.len
+        acc, com, nl = gpu.verify_commit([seq], drafts=np.array(drafts, np.int32).reshape(1, -1))
+        vl = gpu.debug_logits(1, B)
+        g_o, mg_v, vl_o = ss.verify([anchor] + drafts, want_logits=True)
+        rep.max_dlogit = max(rep.max_dlogit, float(np.abs(vl - vl_o).max()))
+        g_gpu = np.argmax(vl, axis=-1)
+        ties = _cmp_tokens(g_gpu, g_o, mg_v, tie, rep)
+        a = int(acc[0])
+        assert a == accept_rule(drafts, list(g_gpu)), (k, a)
+        assert list(com[0][:a + 1]) == drafts[:a] + [int(g_gpu[a])]
+        assert int(nl[0]) == p0 + a + 1
+        if a != k:  # only an oracle near-tie at an index <= k may shorten the block
+            assert any(t <= k for t in ties), (k, a, ties)
+        else:
+            want = [int(t) for t in ar[j + 1:j + k + 2]]
+            got = [int(t) for t in com[0][:a + 1]]
+            if got != want:  # continuation and block verify may round a near-tie differently
+                bad = [i for i in range(a + 1) if got[i] != want[i]]
+                assert mg_v[bad[0]] < tie, (k, got, want)
+        ss.commit(a)
+        rep.accepts.append(a)
+        if check_kv:
+            for layer in sorted({0, cfg.target.n_layers - 1}):
+                kg, vg = gpu.debug_kv(0, layer, seq, p0, a + 1)
+                for t in range(a + 1):
+                    ko, vo = ss.target_kv(layer, p0 + t)
+                    assert np.abs(kg[t] - ko).max() <= kv_tol and np.abs(vg[t] - vo).max() <= kv_tol, (k, layer, t)
+        anchor = int(g_gpu[a])
+        if a != k or [int(t) for t in com[0][:a + 1]] != [int(t) for t in ar[j + 1:j + k + 2]]:
+            break  # the GPU left the oracle's continuation at a near-tie: stop forcing
+        j += a + 1
+    if check_kv and B > 1 and rep.accepts:
+        # the context rows of the last commit are injected by the next draft
+        a = rep.accepts[-1]
+        p0 = ss.len - (a + 1)
+        gpu.draft_block([seq])
+        ss.draft(anchor)
+        for layer in range(cfg.drafter.n_layers):
+            kg, vg = gpu.debug_kv(1, layer, seq, p0, a + 1)
+            for t in range(a + 1):
+                ko, vo = ss.ctx_kv(layer, p0 + t)
+                assert np.abs(kg[t] - ko).max() <= kv_tol and np.abs(vg[t] - vo).max() <= kv_tol, (layer, t)
+    rep.sessions = [ss]
+    return rep

@@ -20,7 +20,7 @@ from synthetic.configs import ModelDims
 import oracle
 from synthetic import make_weights
 from synthetic.fast import make_weights_host
-from parity import build_pair, replay, check_lossless_generate, accept_rule
+from parity import build_pair, replay, replay_forced, check_lossless_generate, accept_rule
 
 pytestmark = pytest.mark.gpu
 
@@ -188,18 +188,19 @@ def test_kv_rollback_matches_oracle(cuda_device):
             np.testing.assert_allclose(v[t], vo, rtol=0, atol=1e-4)
 
 
-@pytest.mark.parametrize("mode", ["fast", "chain", "counters"])
+@pytest.mark.parametrize("mode", ["fast", "unfolded", "counters"])
 def test_alternative_execution_modes(cuda_device, mode, monkeypatch):
     """The opt-in execution modes compute the same decode step: single-plane bf16
-    activations (DFLASH_BF16_FAST, looser logits), the persistent projection chain,
-    and device completion counters between the kernels of a pass."""
+    activations (DFLASH_BF16_FAST, looser logits), separate RMSNorm kernels
+    instead of norms folded into the projections, and device completion
+    counters between the kernels of a pass."""
     cfg = tiny_cfg(dtype="bf16", block=16, hidden=2048, nq=16, nkv=4, hd=128, vocab=8192)
     tol, tie = TOL["bf16"]
     act = "split"
     if mode == "fast":
         act, tol = "fast", 0.15   # one plane: plain bf16 rounding of GEMM inputs, q and K/V
-    if mode == "chain":
-        monkeypatch.setenv("DFLASH_PROJECTION_CHAIN", "1")
+    if mode == "unfolded":
+        monkeypatch.setenv("DFLASH_FOLDED_NORM", "0")
     if mode == "counters":
         monkeypatch.setenv("DFLASH_DEP_COUNTERS", "1")
     w_cpu = make_weights_host(cfg, random_gains=True)
@@ -252,3 +253,42 @@ def test_batch16_block16_uses_wide_row_tiles(cuda_device):
     prompts = [make_prompt("uniform", L, cfg.target.vocab, 40 + i) for i, L in enumerate(lens)]
     rep = replay(gpu, spec, cfg, prompts, 2, tol, tie)
     _finish(rep, tol)
+
+
+@pytest.mark.parametrize("dtype,block,cuts", [("fp32", 4, (3, 1, 0, 3)), ("bf16", 4, (3, 2, 0)),
+                                              ("bf16", 16, (15, 7, 3, 0))])
+def test_forced_accept_lengths_against_oracle(cuda_device, dtype, block, cuts):
+    """Caller drafts = the oracle's greedy continuation, wrong after k drafts:
+    the verify accepts exactly k (k = B-1: the whole block), commits the
+    oracle's tokens, and the target / drafter-context K/V of the committed
+    positions equal the oracle's."""
+    cfg = tiny_cfg(dtype, block=block)
+    tol, tie = TOL[dtype]
+    gpu, spec, _ = build_pair(cfg, max_len=128)
+    prompt = make_prompt("uniform", 14, cfg.target.vocab, 21)
+    rep = replay_forced(gpu, spec, cfg, prompt, cuts, tol, tie, kv_tol=1e-4 if dtype == "fp32" else 1e-2)
+    _finish(rep, tol)
+    assert rep.accepts[0] == cuts[0] or rep.near_ties > 0
+
+
+def test_nonfinite_logits_report_enumeric(cuda_device):
+    """One NaN in the LM head makes one logit of every row non-finite: the
+    synchronising calls return DFLASH_ENUMERIC from the device status word."""
+    cfg = tiny_cfg("bf16", block=4)
+    gpu, spec, _ = build_pair(cfg, max_len=96)
+    gpu.weight_view("lm_head")[7, 3] = float("nan")
+    torch.cuda.synchronize()
+    prompt = make_prompt("uniform", 10, cfg.target.vocab, 2)
+    with pytest.raises(dfl.DFlashError) as e:
+        gpu.generate([prompt], 12)
+    assert e.value.status == dfl.DFLASH_ENUMERIC
+    gpu.reset_stats()
+    with pytest.raises(dfl.DFlashError) as e:
+        gpu.prefill(0, prompt)
+    assert e.value.status == dfl.DFLASH_ENUMERIC
+    with pytest.raises(dfl.DFlashError) as e:
+        gpu.draft_block([0])
+    assert e.value.status == dfl.DFLASH_ENUMERIC
+    with pytest.raises(dfl.DFlashError) as e:
+        gpu.verify_commit([0])
+    assert e.value.status == dfl.DFLASH_ENUMERIC
