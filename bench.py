@@ -6,8 +6,11 @@ the batch: context fuse + K/V injection, the 5-layer block-bidirectional
 drafter pass and its LM-head argmax, the 36-layer causal verify pass, the
 target LM-head argmax and the accept/commit step.  Workload: Qwen3-8B-shaped
 target with a 5-layer block-16 drafter, bf16 random-init weights N(0, 0.02),
-batch 1 per GPU, 512-token Zipf(1.1) prompt.  Weights (18.5 GB) exceed the
-126 MB L2, so every step streams them from HBM.
+batch 1 per GPU, 512-token Zipf(1.1) prompt, 2048 generated tokens: by
+default the timed iterations are the rest of that generation after the
+warm-up (about 2038 iterations at the random drafter's one token per
+iteration, mean context about 1536).  Weights (18.5 GB) exceed the 126 MB L2,
+so every step streams them from HBM.
 
 --gpus N runs N independent replicas (one process per GPU; the decode step has
 no collective), and `value` sums their tokens over the slowest replica's time.
@@ -43,11 +46,6 @@ FALLBACK_HBM = 6650.0
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
-
-
-# DRAM bytes (read + write) of one gate/up projection launch, from an ncu
-# capture of the same kernel shape (see profiles/); None until measured
-GATE_UP_TRAFFIC = {"qwen3_8b": 205.26e6}
 
 
 def hbm_peak():
@@ -138,14 +136,18 @@ def iteration_bytes(cfg, batch: int, mean_ctx: float, kv_planes: int = 1) -> flo
         touched = t.n_experts * (1.0 - (1.0 - t.top_k / t.n_experts) ** rows)
         w += t.n_layers * touched * 3 * t.hidden * t.expert_ffn * es
     kv = batch * (mean_ctx + cfg.block_size) * 2 * es * kv_planes * (t.n_layers * t.n_kv_heads * t.head_dim
-                                                          + d.n_layers * d.n_kv_heads * d.head_dim)
+                                                                     + d.n_layers * d.n_kv_heads * d.head_dim)
     return float(w * (1 if batch else 0) + kv)
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
-def cpu_oracle_sample(cfg, prompt_len: int = 16, iters: int = 1, seed: int = 0):
+def cpu_oracle_sample(cfg, gpu_ctx=None, prompt_len: int = 16, iters: int = 1, seed: int = 0, tie: float = 0.05):
     """Time the fp64 CPU oracle on a bounded sample of the workload: one
-    draft + verify iteration of the full-size model after a short prompt."""
+    draft + verify iteration of the full-size model after a short prompt.
+    With gpu_ctx, the GPU context decodes the same prompt teacher-forced beside
+    it (slot 0, the oracle following the GPU's drafts): its drafts and target
+    argmaxes are compared with the oracle's and the near-ties (oracle top-1 /
+    top-2 margin below `tie`) counted."""
     import oracle
     from synthetic.fast import make_weights_host
     t0 = time.time()
@@ -154,39 +156,101 @@ def cpu_oracle_sample(cfg, prompt_len: int = 16, iters: int = 1, seed: int = 0):
     spec = oracle.OracleSpec(cfg, w)
     prompt = make_prompt(cfg.prompt_kind, prompt_len, cfg.target.vocab, cfg.seed + seed)
     ss = spec.session(prompt_len + (iters + 2) * cfg.block_size)
+    ties = {"checked": 0, "near_ties": 0, "mismatches_outside_ties": 0, "tie_margin": tie} if gpu_ctx else None
+
+    def count(gpu_tok, orc_tok, margins):
+        for a, o, m in zip(gpu_tok, orc_tok, margins):
+            ties["checked"] += 1
+            if m < tie:
+                ties["near_ties"] += 1
+            elif int(a) != int(o):
+                ties["mismatches_outside_ties"] += 1
+
     t0 = time.time()
-    anchor, _, _ = ss.prefill(prompt)
+    anchor, mg0, _ = ss.prefill(prompt)
     pre_s = time.time() - t0
+    if gpu_ctx is not None:
+        first = gpu_ctx.prefill(0, prompt)
+        count([first], [anchor], [mg0])
+        anchor = first
     tokens = 0
-    t0 = time.time()
+    it_s = 0.0
     for _ in range(iters):
-        d, _, _ = ss.draft(anchor)
-        g, _, _ = ss.verify([anchor] + list(d))
-        a = 0
-        while a < cfg.block_size - 1 and d[a] == g[a]:
-            a += 1
+        t0 = time.time()
+        d, mg_d, _ = ss.draft(anchor)
+        it_s += time.time() - t0
+        if gpu_ctx is not None:
+            d_gpu = gpu_ctx.draft_block([0])[0]
+            count(d_gpu, d, mg_d)
+            d = d_gpu
+        t0 = time.time()
+        g, mg_v, _ = ss.verify([anchor] + list(d))
+        it_s += time.time() - t0
+        if gpu_ctx is not None:
+            acc, com, _ = gpu_ctx.verify_commit([0])
+            a = int(acc[0])
+            count(list(d[:a]) + [com[0][a]], list(g[:a + 1]), mg_v[:a + 1])
+        else:
+            a = 0
+            while a < cfg.block_size - 1 and d[a] == g[a]:
+                a += 1
+        t0 = time.time()
         ss.commit(a)
-        anchor = int(g[a])
+        it_s += time.time() - t0
+        anchor = int(com[0][a]) if gpu_ctx is not None else int(g[a])
         tokens += a + 1
-    it_s = time.time() - t0
-    return {"tokens": tokens, "seconds": it_s, "iters": iters, "weight_gen_s": gen_s, "prefill_s": pre_s}
+    return ({"tokens": tokens, "seconds": it_s, "iters": iters, "weight_gen_s": gen_s, "prefill_s": pre_s},
+            ties)
 
 
 # ------------------------------------------------------------------ main
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum per launch) of each
+# kernel shape, from one ncu capture of the 2-layer model of the same widths;
+# the file under profiles/ gives the command.  A shape is absent until captured
+# for the kernel version in this tree.
+TRAFFIC = {}
+TRAFFIC_SOURCE = None
+
+SHAPES = ("qkv", "attention", "o", "gate_up", "down", "lm_head", "fuse")
+
+
+def per_shape(prof, peak, attn_bytes_per_launch):
+    """Per-shape launches, mean microseconds and achieved bandwidth of a profile
+    record (CUDA events around each launch); attention bytes are the visible
+    K/V (one bf16 plane) at the profiled context."""
+    out = {}
+    for name in SHAPES:
+        n, ms, by = prof[name]
+        if n == 0:
+            continue
+        if name == "attention":
+            by = attn_bytes_per_launch * n
+        us = 1000.0 * ms / n
+        gbs = by / (ms / 1000.0) / 1e9 if ms > 0 else 0.0
+        out[name] = {"launches": n, "us_per_launch": round(us, 2), "bytes_per_launch": by / n,
+                     "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "ms_total": round(ms, 4),
+                     "traffic": TRAFFIC.get(name)}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed draft+verify iterations (default: the rest of the workload's generation)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="qwen3_8b")
     ap.add_argument("--batch", type=int, default=None, help="sequences per GPU (default: the config's)")
     ap.add_argument("--prompt-len", type=int, default=None)
     ap.add_argument("--forced", default="1,4,8,16", help="forced accept lengths to time ('' = none)")
+    ap.add_argument("--forced-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sampling", action="store_true")
     ap.add_argument("--bf16-act", choices=["split", "fast"], default="split",
                     help="bf16 activations as two planes (parity-grade) or one plane")
     ap.add_argument("--e2e-tokens", type=int, default=128)
+    ap.add_argument("--profile-steps", type=int, default=50)
     ap.add_argument("--target-layers", type=int, default=None, help="layer-reduced copy (profiling small cases)")
     ap.add_argument("--drafter-layers", type=int, default=None)
     ap.add_argument("--ref-budget-s", type=float, default=150.0, help="reference arm: cap on timed CPU seconds")
@@ -206,6 +270,11 @@ def main():
         from synthetic.configs import shrink
         cfg = shrink(cfg, target_layers=args.target_layers or cfg.target.n_layers,
                      drafter_layers=args.drafter_layers or cfg.drafter.n_layers)
+    if args.steps is None:
+        # the workload generates max_new tokens per sequence; with the random
+        # drafter (about one token per iteration) the timed iterations cover the
+        # rest of that generation after the warm-up
+        args.steps = max(1, cfg.max_new - args.warmup)
 
     if args.impl == "reference":
         return run_reference(args, cfg, world, rank)
@@ -221,16 +290,21 @@ def main():
         pg = dist
 
     b, B = cfg.batch, cfg.block_size
-    max_new_cap = (args.warmup + args.steps + 8) * B
-    max_len = cfg.prompt_len + max(max_new_cap, args.e2e_tokens + 2 * B, 2048) + 2 * B
+    P = cfg.prompt_len
+    # decode_iters checks capacity for the worst case (B tokens per iteration)
+    max_len = P + (args.warmup + max(args.steps, args.profile_steps, args.forced_steps) + 4) * B + 2 * B
+    max_len = max(max_len, P + args.e2e_tokens + 2 * B)
     log(f"[rank {rank}] building context: {cfg.name} batch {b} max_len {max_len}")
-    ctx = dfl.DFlash(cfg, max_batch=b, max_len=max_len, device=dev, bf16_act=args.bf16_act)
+    sampling = not args.no_sampling
+    ctx = dfl.DFlash(cfg, max_batch=b, max_len=max_len, device=dev, bf16_act=args.bf16_act, sampling=sampling)
     t0 = time.time()
     ctx.load_weights_from(lambda n: make_weight(cfg, n, device=dev))
     log(f"[rank {rank}] weights generated + loaded in {time.time() - t0:.1f}s ({ctx.weight_bytes / 1e9:.2f} GB)")
-    prompts = [make_prompt(cfg.prompt_kind, cfg.prompt_len, cfg.target.vocab, sd)
+    prompts = [make_prompt(cfg.prompt_kind, P, cfg.target.vocab, sd)
                for sd in rank_prompt_seeds(cfg.seed, rank, b)]
     stream = torch.cuda.current_stream(dev)
+    kv_planes = 1  # algorithmic K/V bytes: one bf16 plane per element
+    peak, peak_kind = hbm_peak()
 
     def prefill_all():
         for i, p in enumerate(prompts):
@@ -252,13 +326,14 @@ def main():
         st = ctx.stats()
         return e0.elapsed_time(e1), st, st.kernel_launches - l0
 
-    # ---- natural acceptance (the drafter's own argmax) ----
+    # ---- headline: the workload's generation with the model drafter ----
     t0 = time.time()
     prefill_all()
     torch.cuda.synchronize(dev)
     prefill_s = time.time() - t0
     ctx.decode_iters(b, args.warmup)
     torch.cuda.synchronize(dev)
+    w_tau = ctx.stats().mean_tau
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -269,35 +344,57 @@ def main():
     ms_max, tok_sum = reduce_step(pg, ms, tokens, dev)
     value = tok_sum / (ms_max / 1000.0)
     mean_tau = st.mean_tau
-    ctx_len_mean = cfg.prompt_len + args.warmup * mean_tau + 0.5 * args.steps * mean_tau
-    it_bytes = iteration_bytes(cfg, b, ctx_len_mean, 2 if (cfg.dtype == "bf16" and args.bf16_act == "split") else 1)
+    ctx_start = P + 1 + args.warmup * w_tau
+    ctx_mean = ctx_start + 0.5 * args.steps * mean_tau
+    it_bytes = iteration_bytes(cfg, b, ctx_mean, kv_planes)
     us_iter = ms_max * 1000.0 / args.steps
     log(f"[rank {rank}] {args.steps} iters in {ms:.2f} ms: {us_iter:.1f} us/iter, tau {mean_tau:.3f}, "
-        f"{value:.1f} tok/s, launches {launches}")
+        f"{value:.1f} tok/s, mean context {ctx_mean:.0f}, launches {launches}")
 
-    # ---- per-kernel roofline: CUDA events around each projection / attention launch ----
-    ctx.profile(True)
-    ctx.decode_iters(b, min(args.steps, 50))
-    prof = ctx.profile_read()
-    ctx.profile(False)
-    pl, pms, pbytes = prof["projection"]
-    al, ams, _ = prof["attention"]
-    gl, gms, gbytes = prof["gate_up"]
-    peak, peak_kind = hbm_peak()
-    achieved = pbytes / (pms / 1000.0) / 1e9 if pms > 0 else 0.0
-    # dominant kernel: the gate/up projection (a third of the step); algorithmic
-    # bytes per launch / its mean launch time (events around each launch)
-    g_achieved = gbytes / (gms / 1000.0) / 1e9 if gms > 0 else 0.0
-    log(f"[rank {rank}] projections: {pl} launches, {pms:.2f} ms, {pbytes / 1e9:.2f} GB -> {achieved:.0f} GB/s; "
-        f"gate/up {gl} launches {gms:.2f} ms -> {g_achieved:.0f} GB/s; attention {al} launches {ams:.2f} ms")
+    # ---- split and per-kernel timing at the start and at the end of the generation ----
+    def profile_run(mode, k):
+        ctx.profile(mode)
+        ctx.decode_iters(b, k)
+        prof = ctx.profile_read()
+        ctx.profile(0)
+        return prof
+
+    def kv_bytes_per_launch(m, ctx_len):
+        # one attention launch of model m reads the visible K and V of every sequence
+        return b * (ctx_len + B) * 2 * 2 * kv_planes * m.n_kv_heads * m.head_dim
+
+    def passes(prof, k):
+        _, dms, _ = prof["draft_pass"]
+        _, vms, _ = prof["verify_pass"]
+        return round(1000.0 * dms / k, 2), round(1000.0 * vms / k, 2)
+
+    kp = args.profile_steps
+    end_ctx = ctx_start + args.steps * mean_tau
+    p_end = profile_run(2, kp)
+    end_split = passes(p_end, kp)
+    prefill_all()
+    ctx.decode_iters(b, args.warmup)
+    p_start = profile_run(2, kp)
+    start_split = passes(p_start, kp)
+    kprof = profile_run(1, kp)
+    start_ctx = P + 1 + args.warmup * w_tau + 0.5 * kp * mean_tau
+    t, d = cfg.target, cfg.drafter
+    attn_b = (t.n_layers * kv_bytes_per_launch(t, start_ctx) + d.n_layers * kv_bytes_per_launch(d, start_ctx)) / (
+        t.n_layers + d.n_layers)
+    shapes = per_shape(kprof, peak, attn_b)
+    # dominant kernel: the shape with the largest share of the kernel time
+    dom = max(shapes, key=lambda k: shapes[k]["ms_total"]) if shapes else None
+    log(f"[rank {rank}] split at ctx ~{start_ctx:.0f}: draft {start_split[0]} us, verify {start_split[1]} us; "
+        f"at ctx ~{end_ctx:.0f}: draft {end_split[0]} us, verify {end_split[1]} us")
+    log(f"[rank {rank}] per shape: " + ", ".join(f"{k}: {v['us_per_launch']} us {v['frac']}" for k, v in shapes.items()))
 
     # ---- forced acceptance lengths via a script = the GPU's own target-only continuation ----
     forced = {}
     taus = [int(x) for x in args.forced.split(",") if x.strip()] if args.forced else []
     ar_tps = None
     if taus:
-        need = (args.warmup + args.steps) * B + 2 * B
-        need = min(need, max_len - cfg.prompt_len - B)
+        need = (args.warmup + args.forced_steps) * B + 2 * B
+        need = min(need, max_len - P - B)
         ar_out, ar_ms = ctx.generate_ar(prompts, need)
         ar_tps = b * (need - 1) / (ar_ms / 1000.0) if ar_ms > 0 else None
         # The one-row greedy decode and the block verify round differently; at a
@@ -322,13 +419,27 @@ def main():
             ctx.set_draft_mode(dfl.DFLASH_DRAFT_SCRIPT, tau)
             prefill_all()
             ctx.decode_iters(b, args.warmup)
-            k = max(1, min(args.steps, (need - args.warmup * tau) // max(tau, 1) - 2))
+            k = max(1, min(args.forced_steps, (need - args.warmup * tau) // max(tau, 1) - 2))
             fms, fst, _ = timed_iters(k)
-            forced[str(tau)] = {"tokens_per_s": fst.tokens / (fms / 1000.0), "mean_tau": fst.mean_tau,
-                                "tokens_per_s_at_tau": b * tau * k / (fms / 1000.0),
-                                "us_per_iter": fms * 1000.0 / k, "iters": k}
+            forced[str(tau)] = {"tokens_per_s": round(fst.tokens / (fms / 1000.0), 2),
+                                "mean_tau": round(fst.mean_tau, 4),
+                                "tokens_per_s_at_tau": round(b * tau * k / (fms / 1000.0), 2),
+                                "us_per_iter": round(fms * 1000.0 / k, 2), "iters": k}
             log(f"[rank {rank}] forced tau={tau}: {forced[str(tau)]}")
         ctx.set_draft_mode(dfl.DFLASH_DRAFT_MODEL, 1)
+
+    # ---- temperature sampling (T = 0.8): the speculative-sampling acceptance ----
+    sampled = None
+    if sampling:
+        ctx.set_sampling(0.8, seed=1)
+        prefill_all()
+        ctx.decode_iters(b, args.warmup)
+        k = args.profile_steps
+        sms, sst, _ = timed_iters(k)
+        ctx.set_sampling(0.0)
+        sampled = {"temperature": 0.8, "tokens_per_s": round(sst.tokens / (sms / 1000.0), 2),
+                   "mean_tau": round(sst.mean_tau, 4), "us_per_iter": round(sms * 1000.0 / k, 2), "iters": k}
+        log(f"[rank {rank}] sampled: {sampled}")
 
     # ---- end to end through the public call, host buffers in and out ----
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -347,10 +458,11 @@ def main():
     d2h = out.nbytes + 4 * (iters_e2e + 2)
 
     cpu = None
+    ties = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         log("[rank 0] timing the CPU oracle on a bounded sample ...")
         try:
-            s = cpu_oracle_sample(cfg)
+            s, ties = cpu_oracle_sample(cfg, ctx)
             cpu = {"value": s["tokens"] / s["seconds"], "unit": "tokens/s", "cores": omp_threads(),
                    "kind": "oracle",
                    "sample": (f"{s['iters']} full-size fp64 draft+verify iteration(s) after a 16-token prompt "
@@ -364,6 +476,16 @@ def main():
         if pg:
             pg.destroy_process_group()
         return
+    roof = None
+    if dom:
+        sd = shapes[dom]
+        roof = {"bound": "hbm", "achieved": sd["achieved_gbs"], "peak": peak, "unit": "GB/s", "frac": sd["frac"],
+                "traffic": sd["traffic"], "kernel": dom, "bytes_per_launch": sd["bytes_per_launch"],
+                "us_per_launch": sd["us_per_launch"],
+                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s",
+                "traffic_source": TRAFFIC_SOURCE if sd["traffic"] is not None else None,
+                "context": round(start_ctx, 1), "per_shape": shapes}
     result = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -379,26 +501,25 @@ def main():
         "data": "synthetic (counter-based N(0,0.02)-like weights, Zipf(1.1) prompts)",
         "config": workload_config(cfg, args, world),
         "us_per_iter": round(us_iter, 2),
+        "us_per_draft": start_split[0],
+        "us_per_verify": start_split[1],
+        "split_by_context": {f"{start_ctx:.0f}": {"us_per_draft": start_split[0], "us_per_verify": start_split[1]},
+                             f"{end_ctx:.0f}": {"us_per_draft": end_split[0], "us_per_verify": end_split[1]}},
         "mean_tau": round(mean_tau, 4),
+        "context_mean": round(ctx_mean, 1),
         "iter_bytes": it_bytes,
         "iter_hbm_frac_8tbps": round(it_bytes / (us_iter * 1e-6) / 8e12, 4),
         "iter_hbm_frac_measured": round(it_bytes / (us_iter * 1e-6) / (peak * 1e9), 4),
         "forced_tau": forced,
+        "sampled": sampled,
         "ar_tokens_per_s": round(ar_tps, 2) if ar_tps else None,
         "prefill_s": round(prefill_s, 3),
         "gpu_launches": int(launches),
         "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s", "h2d_bytes_per_step": h2d / iters_e2e,
                 "d2h_bytes_per_step": d2h / iters_e2e,
                 "note": f"dflash_generate: prefill + {args.e2e_tokens} tokens, host prompt in, host tokens out"},
-        "roofline": {"bound": "hbm", "achieved": round(g_achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(g_achieved / peak, 4), "traffic": GATE_UP_TRAFFIC.get(cfg.name),
-                     "kernel": "gemm_tc_kernel<16, SWIGLU> (gate/up projection, tcgen05)",
-                     "bytes_per_launch": gbytes / max(gl, 1), "us_per_launch": 1000.0 * gms / max(gl, 1),
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback 6.65 TB/s",
-                     "all_projections": {"achieved": round(achieved, 1), "frac": round(achieved / peak, 4),
-                                         "launches": pl, "ms": round(pms, 3), "bytes": pbytes}},
-        "attention_ms_per_step": round(ams / max(1, min(args.steps, 50)), 4),
+        "roofline": roof,
+        "near_ties": ties,
         "cpu_baseline": cpu,
         "clocks": clk,
     }
@@ -413,17 +534,19 @@ def omp_threads() -> int:
     return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
 
 
-def workload_config(cfg, args, world):
-    """The `config` object of both arms' JSON lines."""
+def workload_config(cfg, args, world, prompt_len=None):
+    """The `config` object of both arms' JSON lines (prompt_len: the prompt the
+    arm actually decodes after, when it differs from the workload's)."""
     b, B = cfg.batch, cfg.block_size
+    plen = cfg.prompt_len if prompt_len is None else prompt_len
     return {"workload": f"{cfg.name}: {cfg.target.n_layers}-layer target (hidden {cfg.target.hidden}, "
                         f"vocab {cfg.target.vocab}) + {cfg.drafter.n_layers}-layer block-{B} drafter, "
-                        f"batch {b} per GPU, {cfg.prompt_len}-token prompt",
-            "global_batch": b * world, "seq_len": cfg.prompt_len, "block_size": B,
+                        f"batch {b} per GPU, {plen}-token prompt",
+            "global_batch": b * world, "seq_len": plen, "block_size": B,
             "parallelism": f"replicas x{world}",
             "activations": ("bf16 hi+lo planes, fp32 accumulate" if args.bf16_act == "split"
                             else "bf16 single plane, fp32 accumulate") if cfg.dtype == "bf16" else "fp32",
-            "l2": l2_note(cfg, 2 if cfg.dtype == "bf16" and args.bf16_act == "split" else 1)}
+            "l2": l2_note(cfg)}
 
 
 def l2_note(cfg, kv_planes: int = 1, l2_bytes: float = 126e6) -> str:
@@ -478,7 +601,8 @@ def run_reference(args, cfg, world, rank):
     res = {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "tokens/s", "n_gpus": world,
            "steps": n_steps, "warmup": args.warmup, "ms_per_step": round(1000 * sec / n_steps, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": dict(workload_config(cfg, args, world), activations="fp64 (oracle)"),
+           "data": "synthetic",
+           "config": dict(workload_config(cfg, args, world, prompt_len=plen), activations="fp64 (oracle)"),
            "cpu_baseline": {"value": round(v, 5), "unit": "tokens/s", "cores": omp_threads(), "kind": "oracle",
                             "sample": f"{n_steps} full-size draft+verify iterations after a 16-token prompt "
                                       f"(capped at {args.ref_budget_s:.0f} s of CPU time; {args.steps} requested)"},

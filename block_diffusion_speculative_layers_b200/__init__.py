@@ -22,6 +22,9 @@ DFLASH_ECUDA, DFLASH_ENUMERIC, DFLASH_ETIMEOUT, DFLASH_EUNSUPPORTED = 4, 5, 6, 7
 DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST = 0, 1, 2
 DFLASH_DRAFT_MODEL, DFLASH_DRAFT_SCRIPT = 0, 1
 MAX_TAPS, MAX_BLOCK = 8, 16
+# dflash_profile_read classes, in the order of the DFLASH_PROF_* values
+PROF_CLASSES = ("projection", "attention", "gate_up", "qkv", "o", "down", "lm_head", "fuse", "other_proj",
+                "draft_pass", "verify_pass")
 
 STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ESTATE", 3: "ECAPACITY", 4: "ECUDA", 5: "ENUMERIC",
                 6: "ETIMEOUT", 7: "EUNSUPPORTED"}
@@ -47,7 +50,10 @@ class ModelCfg(C.Structure):
     _fields_ = [("n_layers", C.c_int32), ("hidden", C.c_int32), ("n_q_heads", C.c_int32),
                 ("n_kv_heads", C.c_int32), ("head_dim", C.c_int32), ("ffn", C.c_int32),
                 ("vocab", C.c_int32), ("n_experts", C.c_int32), ("top_k", C.c_int32),
-                ("expert_ffn", C.c_int32), ("rms_eps", C.c_double), ("rope_theta", C.c_double)]
+                ("expert_ffn", C.c_int32), ("rms_eps", C.c_double), ("rope_theta", C.c_double),
+                ("qk_norm", C.c_int32), ("reserved", C.c_int32), ("rope_factor", C.c_double),
+                ("rope_low_freq_factor", C.c_double), ("rope_high_freq_factor", C.c_double),
+                ("rope_original_max_pos", C.c_double)]
 
 
 class Config(C.Structure):
@@ -121,8 +127,10 @@ def load_library(path: Optional[str] = None):
 
 
 def _model_cfg(d) -> ModelCfg:
+    f, lo, hi, orig = (float(x) for x in getattr(d, "rope_scaling", (0.0, 0.0, 0.0, 0.0)))
     return ModelCfg(d.n_layers, d.hidden, d.n_q_heads, d.n_kv_heads, d.head_dim, d.ffn, d.vocab,
-                    d.n_experts, d.top_k, d.expert_ffn, float(d.rms_eps), float(d.rope_theta))
+                    d.n_experts, d.top_k, d.expert_ffn, float(d.rms_eps), float(d.rope_theta),
+                    1 if getattr(d, "qk_norm", False) else 0, 0, f, lo, hi, orig)
 
 
 def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: int = 0,
@@ -134,9 +142,6 @@ def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: in
     "fast" (one plane, DFLASH_BF16_FAST)."""
     if bf16_act not in ("split", "fast"):
         raise ValueError("bf16_act must be 'split' or 'fast'")
-    for d in (spec.target, spec.drafter):
-        if getattr(d, "qk_norm", False) or float(getattr(d, "rope_scaling", (0.0,))[0]) > 1.0:
-            raise NotImplementedError("QK-norm and RoPE frequency rescaling are not in the kernels yet")
     c = Config()
     c.target = _model_cfg(spec.target)
     c.drafter = _model_cfg(spec.drafter)
@@ -313,15 +318,15 @@ class DFlash:
     def reset_stats(self):
         self._check(self.lib.dflash_reset_stats(self.h), "dflash_reset_stats")
 
-    def profile(self, enable: bool):
-        self._check(self.lib.dflash_profile(self.h, 1 if enable else 0), "dflash_profile")
+    def profile(self, mode):
+        """mode: False/0 off, True/1 events around every kernel launch, 2 around passes, 3 both."""
+        self._check(self.lib.dflash_profile(self.h, int(mode)), "dflash_profile")
 
     def profile_read(self):
-        out = (KernelProf * 3)()
+        """{class name: (launches, ms, algorithmic bytes)} of the current record."""
+        out = (KernelProf * len(PROF_CLASSES))()
         self._check(self.lib.dflash_profile_read(self.h, out), "dflash_profile_read")
-        return {"projection": (out[0].launches, out[0].ms, out[0].bytes),
-                "attention": (out[1].launches, out[1].ms, out[1].bytes),
-                "gate_up": (out[2].launches, out[2].ms, out[2].bytes)}
+        return {name: (out[i].launches, out[i].ms, out[i].bytes) for i, name in enumerate(PROF_CLASSES)}
 
     def load_weights_from(self, make_one, names=None):
         """Fill each weight slot from make_one(name) (one tensor alive at a time)."""

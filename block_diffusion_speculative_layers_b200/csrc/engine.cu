@@ -92,6 +92,13 @@ static bool check_model(const dflash_model_cfg &m, std::string &why) {
         return false;
     }
     if (!(m.rms_eps >= 0.0) || !(m.rope_theta > 1.0)) { why = "bad rms_eps / rope_theta"; return false; }
+    if (m.n_q_heads + m.n_kv_heads > 256) { why = "at most 256 q + kv heads"; return false; }
+    if (m.qk_norm != 0 && m.qk_norm != 1) { why = "qk_norm must be 0 or 1"; return false; }
+    if (m.rope_factor > 1.0 && !(m.rope_low_freq_factor > 0.0 && m.rope_high_freq_factor > m.rope_low_freq_factor &&
+                                 m.rope_original_max_pos > 0.0)) {
+        why = "RoPE rescaling needs 0 < low < high and original_max_pos > 0";
+        return false;
+    }
     return true;
 }
 
@@ -138,6 +145,10 @@ static void add_model_slots(Layout &L, const char *prefix, const dflash_model_cf
     for (int l = 0; l < m.n_layers; ++l) {
         std::string p = std::string(prefix) + ".L" + std::to_string(l) + ".";
         add_slot(L, p + "attn_norm", 1, H, 0, 0, DFLASH_FP32);
+        if (m.qk_norm) {
+            add_slot(L, p + "q_norm", 1, m.head_dim, 0, 0, DFLASH_FP32);
+            add_slot(L, p + "k_norm", 1, m.head_dim, 0, 0, DFLASH_FP32);
+        }
         add_slot(L, p + "wqkv", 2, qd + 2 * kd, H, 0, dt);
         add_slot(L, p + "wo", 2, H, qd, 0, dt);
         add_slot(L, p + "ffn_norm", 1, H, 0, 0, DFLASH_FP32);
@@ -342,8 +353,8 @@ class Engine : public EngineBase {
     int *pinned = nullptr;  // small pinned host buffer for the done counter
     bool lens_stale = false;
     // per-launch timing (dflash_profile)
-    struct ProfRec { int cls, sub; double bytes; cudaEvent_t a, b; };  // sub: second class or -1
-    bool profiling = false;
+    struct ProfRec { int cls[3]; double bytes; cudaEvent_t a, b; };  // classes (-1: none)
+    int profiling = 0;  // bit 0: events around every projection / attention launch; bit 1: around passes
     std::vector<ProfRec> prof;
     std::vector<cudaEvent_t> ev_pool;
     size_t ev_used = 0;
@@ -372,6 +383,10 @@ class Engine : public EngineBase {
                 std::string p = std::string(pre) + ".L" + std::to_string(l) + ".";
                 LayerW &w = v[l];
                 w.attn_norm = (const float *)wslot(by, p + "attn_norm");
+                if (m.qk_norm) {
+                    w.q_norm = (const float *)wslot(by, p + "q_norm");
+                    w.k_norm = (const float *)wslot(by, p + "k_norm");
+                }
                 w.ffn_norm = (const float *)wslot(by, p + "ffn_norm");
                 w.wqkv = wslot(by, p + "wqkv");
                 w.wo = wslot(by, p + "wo");
@@ -472,8 +487,12 @@ class Engine : public EngineBase {
         h_prefilled.assign(c.max_batch, 0);
         // zero the whole state arena once: stale taps / KV never hold NaN bit patterns
         if (cudaMemsetAsync(S, 0, L.state_bytes, s) != cudaSuccess) return fail_cuda("memset state");
-        launch_rope_table(rope_t, c.max_len, c.target.head_dim, c.target.rope_theta, s);
-        launch_rope_table(rope_d, c.max_len, c.drafter.head_dim, c.drafter.rope_theta, s);
+        auto rope_table = [&](float2 *tab, const dflash_model_cfg &m) {
+            launch_rope_table(tab, c.max_len, m.head_dim, m.rope_theta, m.rope_factor, m.rope_low_freq_factor,
+                              m.rope_high_freq_factor, m.rope_original_max_pos, s);
+        };
+        rope_table(rope_t, c.target);
+        rope_table(rope_d, c.drafter);
         if (cudaMallocHost((void **)&pinned, 64) != cudaSuccess) return fail_cuda("pinned host buffer");
         if (cudaEventCreateWithFlags(&ev_a, cudaEventDisableTiming) != cudaSuccess) return fail_cuda("event");
         if (cudaEventCreateWithFlags(&ev_b, cudaEventDisableTiming) != cudaSuccess) return fail_cuda("event");
@@ -492,7 +511,7 @@ class Engine : public EngineBase {
         tc.tune_ctas_per_sm = env_int("DFLASH_TC_CTAS_PER_SM");
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);
-        tc.keep_logits = c.keep_logits || c.sampling;
+        tc.keep_logits = c.keep_logits;  // plus while sampling (sampling_changed)
         return check("create");
     }
 
@@ -558,16 +577,36 @@ class Engine : public EngineBase {
     }
 
     template <typename F>
-    void timed(int cls, double bytes, F &&launch, int sub = -1) {
-        if (!profiling) {
+    void record(int mode_bit, int c0, int c1, double bytes, F &&launch) {
+        if (!(profiling & mode_bit)) {
             launch();
             return;
         }
-        ProfRec r{cls, sub, bytes, next_event(), next_event()};
+        ProfRec r{{c0, c1, -1}, bytes, next_event(), next_event()};
         cudaEventRecord(r.a, s);
         launch();
         cudaEventRecord(r.b, s);
         prof.push_back(r);
+    }
+    template <typename F>
+    void timed(int cls, double bytes, F &&launch, int sub = -1) { record(1, cls, sub, bytes, launch); }
+    template <typename F>
+    void timed_pass(int cls, F &&launch) { record(2, cls, -1, 0.0, launch); }
+
+    // profile class of a projection launch (reporting only)
+    int proj_class(int N, int K, int kind) const {
+        const int H = c.target.hidden;
+        switch (kind) {
+            case EPI_QKV: return DFLASH_PROF_QKV;
+            case EPI_SWIGLU: return DFLASH_PROF_GATE_UP;
+            case EPI_LOGITS: return DFLASH_PROF_LM_HEAD;
+            case EPI_NORMOUT: return DFLASH_PROF_FUSE;
+            case EPI_RESID: {
+                const int qt = c.target.n_q_heads * c.target.head_dim, qd = c.drafter.n_q_heads * c.drafter.head_dim;
+                return N == H && (K == qt || K == qd) ? DFLASH_PROF_O : DFLASH_PROF_DOWN;
+            }
+            default: return K == c.n_taps * H ? DFLASH_PROF_FUSE : DFLASH_PROF_OTHER_PROJ;
+        }
     }
 
     // algorithmic HBM bytes of one projection: the weight matrix once, the
@@ -594,8 +633,7 @@ class Engine : public EngineBase {
         if (M <= 0) return 0;
         int ctas = 0;
         timed(DFLASH_PROF_PROJECTION, gemm_bytes(M, N, K, e),
-              [&] { ctas = gemm_launch(X, ldx, M, Wt, N, K, e, dep, dep_target, done); },
-              e.kind == EPI_SWIGLU ? DFLASH_PROF_GATE_UP : -1);
+              [&] { ctas = gemm_launch(X, ldx, M, Wt, N, K, e, dep, dep_target, done); }, proj_class(N, K, e.kind));
         return ctas;
     }
 
@@ -611,7 +649,7 @@ class Engine : public EngineBase {
         switch (e.kind) {
             case EPI_QKV:
                 launch_qkv_epilogue<T>(Y, N, e.col0, e.R_blk, M, e.meta, e.ctx_meta, e.nq, e.nkv, e.hd, e.rope,
-                                       e.q_out, e.kc, e.vc, e.max_len, lo_, s);
+                                       e.q_out, e.kc, e.vc, e.max_len, lo_, e.qn_g, e.kn_g, e.qk_eps, s);
                 break;
             case EPI_RESID:
                 launch_residual<T>(e.x, Y, N, N, M, e.taps, lo_, e.meta, s);
@@ -630,7 +668,7 @@ class Engine : public EngineBase {
                   const dflash_model_cfg &m, T *out, const AttnSync &sy = AttnSync()) {
         const int qd = m.n_q_heads * m.head_dim;
         int ctas = 0;
-        timed(1, 0.0, [&] {
+        timed(DFLASH_PROF_ATTENTION, 0.0, [&] {
             if (attn_mma_supported<T>(m.head_dim))
                 ctas = launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads,
                                                m.head_dim, c.max_len, out, qd, lo_, att, s, sy);
@@ -639,6 +677,16 @@ class Engine : public EngineBase {
                                          qd, s);
         });
         return ctas;
+    }
+
+    // QK-norm gains of a layer (fidelity toggle) into a QKV epilogue
+    static Epi<T> with_qk_norm(Epi<T> e, const dflash_model_cfg &m, const LayerW &w) {
+        if (m.qk_norm) {
+            e.qn_g = w.q_norm;
+            e.kn_g = w.k_norm;
+            e.qk_eps = (float)m.rms_eps;
+        }
+        return e;
     }
 
     // one pre-norm decoder layer of the target over R rows in x (meta)
@@ -659,7 +707,7 @@ class Engine : public EngineBase {
         e.q_out = q;
         e.kc = tk + (size_t)l * kv_layer_elems(m);
         e.vc = tv + (size_t)l * kv_layer_elems(m);
-        gemm(xn, H, R, w.wqkv, qd + 2 * kd, H, e);
+        gemm(xn, H, R, w.wqkv, qd + 2 * kd, H, with_qk_norm(e, m, w));
         attention(q, e.kc, e.vc, mt, R, rpt, m, ao);
         Epi<T> r;
         r.kind = EPI_RESID;
@@ -740,7 +788,7 @@ class Engine : public EngineBase {
         e.kc = dk + (size_t)j * kv_layer_elems(m);
         e.vc = dv + (size_t)j * kv_layer_elems(m);
         // block rows and context rows share one pass over Wqkv (K/V injection)
-        gemm(dq_in, H, with_ctx ? 2 * R : R, w.wqkv, qd + 2 * kd, H, e);
+        gemm(dq_in, H, with_ctx ? 2 * R : R, w.wqkv, qd + 2 * kd, H, with_qk_norm(e, m, w));
         attention(q, e.kc, e.vc, meta, R, c.block_size, m, ao);
         Epi<T> r;
         r.kind = EPI_RESID;
@@ -784,6 +832,9 @@ class Engine : public EngineBase {
 
     // ---- temperature sampling ----
     bool sampling_on() const { return temperature > 0.f; }
+    // the sampling kernels read the fp32 logits rows the LM heads store; greedy
+    // passes store them only for dflash_debug_logits
+    void sampling_changed() override { tc.keep_logits = c.keep_logits || sampling_on(); }
     float *draft_logits() { return c.sampling ? qlogits : logits; }
 
     // rows [R] of logits lg (block B, row k of sequence i drawn at st.len + k + pos_off)
@@ -912,7 +963,8 @@ class Engine : public EngineBase {
             e.q_out = q;
             e.kc = tk + (size_t)l * kv_layer_elems(m);
             e.vc = tv + (size_t)l * kv_layer_elems(m);
-            prog_add(pg, EPI_QKV, tl[l].wqkv, qd + 2 * kd, H, xg_t, H, R, epi_norm_in(e, (float)m.rms_eps, H));
+            prog_add(pg, EPI_QKV, tl[l].wqkv, qd + 2 * kd, H, xg_t, H, R,
+                     epi_norm_in(with_qk_norm(e, m, tl[l]), (float)m.rms_eps, H));
         };
         qkv(0);
         for (int l = 0; l < m.n_layers; ++l) {
@@ -977,7 +1029,8 @@ class Engine : public EngineBase {
             e.q_out = q;
             e.kc = dk + (size_t)j * kv_layer_elems(m);
             e.vc = dv + (size_t)j * kv_layer_elems(m);
-            prog_add(pg, EPI_QKV, dl[j].wqkv, qd + 2 * kd, H, dq_in, H, 2 * R, epi_norm_in(e, (float)m.rms_eps, H));
+            prog_add(pg, EPI_QKV, dl[j].wqkv, qd + 2 * kd, H, dq_in, H, 2 * R,
+                     epi_norm_in(with_qk_norm(e, m, dl[j]), (float)m.rms_eps, H));
         };
         qkv(0);
         for (int j = 0; j < m.n_layers; ++j) {
@@ -1151,7 +1204,7 @@ class Engine : public EngineBase {
                 e.kc = dk + (size_t)j * kv_layer_elems(d);
                 e.vc = dv + (size_t)j * kv_layer_elems(d);
                 const T *wkv = (const T *)dl[j].wqkv + (size_t)qd * H;
-                gemm(cbuf, H, R, wkv, 2 * kd, H, e);
+                gemm(cbuf, H, R, wkv, 2 * kd, H, with_qk_norm(e, d, dl[j]));
             }
         }
         launch_prefill_finish(st, seq, n, first_tok, out_tok, c.max_len, max_new, s);
@@ -1296,7 +1349,7 @@ class Engine : public EngineBase {
         if (r) return r;
         if ((r = set_active(seqs, n))) return r;
         last_pass = PASS_NONE;
-        enqueue_draft(n, is_iota(seqs, n));
+        timed_pass(DFLASH_PROF_DRAFT_PASS, [&] { enqueue_draft(n, is_iota(seqs, n)); });
         if ((r = check("draft launch"))) return r;
         last_pass = PASS_DRAFT;
         last_draft.assign(seqs, seqs + n);
@@ -1326,7 +1379,7 @@ class Engine : public EngineBase {
                 return fail_cuda("drafts copy");
         }
         last_pass = PASS_NONE;
-        enqueue_verify(n);
+        timed_pass(DFLASH_PROF_VERIFY_PASS, [&] { enqueue_verify(n); });
         if ((r = check("verify launch"))) return r;
         last_pass = PASS_VERIFY;
         last_draft.clear();
@@ -1579,8 +1632,8 @@ class Engine : public EngineBase {
         if ((r = set_active(iota.data(), n))) return r;
         OtherPass mark{last_pass};
         for (int it = 0; it < iters; ++it) {
-            enqueue_draft(n, true);
-            enqueue_verify(n);
+            timed_pass(DFLASH_PROF_DRAFT_PASS, [&] { enqueue_draft(n, true); });
+            timed_pass(DFLASH_PROF_VERIFY_PASS, [&] { enqueue_verify(n); });
         }
         last_draft.clear();
         lens_stale = true;
@@ -1610,7 +1663,8 @@ class Engine : public EngineBase {
     dflash_status profile(int enable) override {
         dflash_status r = sync("profile");
         if (r) return r;
-        profiling = enable != 0;
+        if (enable < 0 || enable > 3) { err = "profile mode must be 0..3"; return DFLASH_EINVAL; }
+        profiling = enable;
         if (profiling) {
             prof.clear();
             ev_used = 0;
@@ -1626,9 +1680,8 @@ class Engine : public EngineBase {
         for (const ProfRec &p : prof) {
             float ms = 0.f;
             if (cudaEventElapsedTime(&ms, p.a, p.b) != cudaSuccess) return fail_cuda("event time");
-            const int cls2[2] = {p.cls, p.sub};
-            for (int k : cls2) {
-                if (k < 0) continue;
+            for (int k : p.cls) {
+                if (k < 0 || k >= DFLASH_PROF_CLASSES) continue;
                 o[k].launches += 1;
                 o[k].ms += ms;
                 o[k].bytes += p.bytes;
@@ -1907,6 +1960,7 @@ dflash_status dflash_set_sampling(dflash_ctx *ctx, double temperature, uint64_t 
     }
     ctx->eng->temperature = (float)temperature;
     ctx->eng->seed = seed;
+    ctx->eng->sampling_changed();
     ctx->err.clear();
     return DFLASH_OK;
 }

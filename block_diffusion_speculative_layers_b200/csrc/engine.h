@@ -23,6 +23,7 @@ struct WeightSlot {
 
 struct LayerW {
     const float *attn_norm = nullptr, *ffn_norm = nullptr;
+    const float *q_norm = nullptr, *k_norm = nullptr;  // QK-norm gains (fidelity toggle)
     const void *wqkv = nullptr, *wo = nullptr, *w_gate_up = nullptr, *w_down = nullptr;
     const void *w_router = nullptr, *we_gate_up = nullptr, *we_down = nullptr;
 };
@@ -73,6 +74,7 @@ class EngineBase {
     virtual dflash_status profile(int enable) = 0;
     virtual dflash_status profile_read(dflash_kernel_prof *out) = 0;
     virtual dflash_status head_argmax_noalloc(int which, int32_t *host_out, int32_t *rows_out, void *scratch) = 0;
+    virtual void sampling_changed() {}
     std::string err;
     int draft_mode = DFLASH_DRAFT_MODEL, tau = 1;
     float temperature = 0.f;  // > 0: temperature sampling (config.sampling), else greedy

@@ -53,7 +53,8 @@ void launch_swiglu(const float *Y, int ldy, int F, int R, T *h, int ldh, size_t 
 template <typename T>
 void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot,
                          const RowMeta *meta, const RowMeta *ctx_meta, int nq, int nkv, int hd,
-                         const float2 *rope, T *q_out, T *kc, T *vc, int max_len, size_t lo, cudaStream_t s);
+                         const float2 *rope, T *q_out, T *kc, T *vc, int max_len, size_t lo, const float *qn_g,
+                         const float *kn_g, float qk_eps, cudaStream_t s);
 
 // ---- GEMM (CUDA-core, fp32 accumulate): Y[M][N] = X[M][K] . W[N][K]^T ----
 template <typename T>
@@ -153,7 +154,11 @@ void launch_residual_rows(const ResidualRows &a, cudaStream_t s);
 void launch_accept_sample(const AcceptSample &a, cudaStream_t s);
 
 // ---- tables ----
-void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStream_t s);
+// (cos, sin) of position x frequency for every position and RoPE pair, in fp64;
+// factor > 1: the frequencies rescaled in the Llama 3.1 form (low / high
+// frequency factors, original maximum position).
+void launch_rope_table(float2 *tab, int max_len, int hd, double theta, double factor, double low, double high,
+                       double orig, cudaStream_t s);
 
 }  // namespace dfl
 
@@ -175,6 +180,10 @@ struct Epi {
     int nq = 0, nkv = 0, hd = 0, max_len = 0;
     const float2 *rope = nullptr;
     T *q_out = nullptr, *kc = nullptr, *vc = nullptr;
+    // QK-norm (qn_g != nullptr): q and k heads RMS-normalised over hd with these
+    // gains and qk_eps before RoPE
+    const float *qn_g = nullptr, *kn_g = nullptr;
+    float qk_eps = 0.f;
     // EPI_RESID: x[M][N] += Y, then tap copies of the new x
     float *x = nullptr;
     TapDst<T> taps{};

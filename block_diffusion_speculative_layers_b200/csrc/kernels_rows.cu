@@ -336,7 +336,8 @@ __global__ void qkv_epilogue_kernel(const float *__restrict__ Y, int ldy, int co
                                     const RowMeta *__restrict__ meta, const RowMeta *__restrict__ ctx_meta,
                                     int nq, int nkv, int hd, const float2 *__restrict__ rope,
                                     T *__restrict__ q_out, T *__restrict__ kc, T *__restrict__ vc,
-                                    int max_len, size_t lo) {
+                                    int max_len, size_t lo, const float *__restrict__ qn_g,
+                                    const float *__restrict__ kn_g, float qk_eps) {
     pdl_trigger();
     pdl_wait();
     const int r = blockIdx.x;
@@ -347,12 +348,30 @@ __global__ void qkv_epilogue_kernel(const float *__restrict__ Y, int ldy, int co
     const float *y = Y + (size_t)r * ldy - col0;   // y[c] for global Wqkv row c
     const float2 *tab = rope + (size_t)m.pos * half;
     const int c_begin = is_ctx ? qd : 0;
+    // QK-norm: 1 / rms of every q and k head of this row (one warp per head)
+    __shared__ float hs[256];  // nq + nkv <= 256 (checked at create)
+    if (qn_g) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        for (int head = warp; head < nq + nkv; head += blockDim.x >> 5) {
+            float a = 0.f;
+            if (!(head < nq && is_ctx))
+                for (int d = lane; d < hd; d += 32) a += y[head * hd + d] * y[head * hd + d];
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            if (lane == 0) hs[head] = 1.0f / sqrtf(a / (float)hd + qk_eps);
+        }
+        __syncthreads();
+    }
     // RoPE pairs over q and k heads
     for (int e = threadIdx.x; e < (nq + nkv) * half; e += blockDim.x) {
         const int head = e / half, i = e % half;
         if (head < nq && is_ctx) continue;
         const int base = head * hd;  // q heads then k heads (k starts at qd)
-        const float x1 = y[base + i], x2 = y[base + i + half];
+        float x1 = y[base + i], x2 = y[base + i + half];
+        if (qn_g) {
+            const float *g = head < nq ? qn_g : kn_g;
+            x1 *= hs[head] * g[i];
+            x2 *= hs[head] * g[i + half];
+        }
         const float2 cs = tab[i];
         const float o1 = x1 * cs.x - x2 * cs.y, o2 = x2 * cs.x + x1 * cs.y;
         if (head < nq) {
@@ -376,10 +395,11 @@ __global__ void qkv_epilogue_kernel(const float *__restrict__ Y, int ldy, int co
 template <typename T>
 void launch_qkv_epilogue(const float *Y, int ldy, int col0, int R_blk, int R_tot, const RowMeta *meta,
                          const RowMeta *ctx_meta, int nq, int nkv, int hd, const float2 *rope, T *q_out,
-                         T *kc, T *vc, int max_len, size_t lo, cudaStream_t s) {
+                         T *kc, T *vc, int max_len, size_t lo, const float *qn_g, const float *kn_g, float qk_eps,
+                         cudaStream_t s) {
     if (R_tot <= 0) return;
     launch_k(qkv_epilogue_kernel<T>, dim3(R_tot), dim3(128), 0, s, 1, Y, ldy, col0, R_blk, meta, ctx_meta, nq, nkv, hd, rope,
-                                                 q_out, kc, vc, max_len, lo);
+                                                 q_out, kc, vc, max_len, lo, qn_g, kn_g, qk_eps);
 }
 
 // ------------------------------------------------------------------------
@@ -536,22 +556,36 @@ void launch_ar_step(SeqState *st, const int *active, int nseq, const int *g, int
 // RoPE table: (cos, sin)(pos * theta^(-2i/hd)), angles in double precision
 // ------------------------------------------------------------------------
 
-__global__ void rope_table_kernel(float2 *tab, int max_len, int hd, double theta) {
+// RoPE frequency of pair i; factor > 1: Llama 3.1 rescaling by wavelength band
+__device__ double rope_freq(int i, int hd, double theta, double factor, double low, double high, double orig) {
+    const double f = pow(theta, -2.0 * (double)i / (double)hd);
+    if (!(factor > 1.0)) return f;
+    const double wavelen = 2.0 * 3.14159265358979323846 / f;
+    if (wavelen < orig / high) return f;        // short wavelengths: kept
+    if (wavelen > orig / low) return f / factor;  // long wavelengths: divided by the factor
+    const double sm = (orig / wavelen - low) / (high - low);
+    return (1.0 - sm) * f / factor + sm * f;
+}
+
+__global__ void rope_table_kernel(float2 *tab, int max_len, int hd, double theta, double factor, double low,
+                                  double high, double orig) {
     pdl_trigger();
     pdl_wait();
     const int half = hd / 2;
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= (int64_t)max_len * half) return;
     const int pos = (int)(e / half), i = (int)(e % half);
-    const double freq = pow(theta, -2.0 * (double)i / (double)hd);
+    const double freq = rope_freq(i, hd, theta, factor, low, high, orig);
     double sn, cs;
     sincos((double)pos * freq, &sn, &cs);
     tab[e] = make_float2((float)cs, (float)sn);
 }
 
-void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStream_t s) {
+void launch_rope_table(float2 *tab, int max_len, int hd, double theta, double factor, double low, double high,
+                       double orig, cudaStream_t s) {
     const int64_t n = (int64_t)max_len * (hd / 2);
-    launch_k(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, 1, tab, max_len, hd, theta);
+    launch_k(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, 1, tab, max_len, hd, theta,
+             factor, low, high, orig);
 }
 
 // ------------------------------------------------------------------------
@@ -572,7 +606,7 @@ void launch_rope_table(float2 *tab, int max_len, int hd, double theta, cudaStrea
     template void launch_swiglu<T>(const float *, int, int, int, T *, int, size_t, cudaStream_t);           \
     template void launch_qkv_epilogue<T>(const float *, int, int, int, int, const RowMeta *,                \
                                          const RowMeta *, int, int, int, const float2 *, T *, T *, T *,     \
-                                         int, size_t, cudaStream_t);
+                                         int, size_t, const float *, const float *, float, cudaStream_t);
 DFL_INST(float)
 DFL_INST(bf16)
 #undef DFL_INST

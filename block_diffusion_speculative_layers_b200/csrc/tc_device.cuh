@@ -436,13 +436,36 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
         }
         epi_bar();
     } else if (KIND == EPI_QKV) {
+        const int hd = e.hd, half = hd >> 1;
+        const int qd = e.nq * hd, kd = e.nkv * hd;
+        const int cg = e.col0 + nt * 128 + n_local;  // row of [Wq; Wk; Wv]
+        if (e.qn_g) {
+            // QK-norm: each q / k head (hd rows of this tile, tiles start on head
+            // boundaries) is RMS-normalised per column before RoPE; per-warp sums of
+            // squares over 32 rows, then over the head's warps in a fixed order
+            const bool normed = nt * 128 + n_local < p.N && cg < qd + kd;
+#pragma unroll
+            for (int j = 0; j < W; ++j) {
+                float sq = normed ? v[j] * v[j] : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                if (lane == 0) red[q * CH + j].x = sq;
+            }
+            epi_bar();
+            const int w0 = (n_local / hd) * hd / 32, nw = hd / 32;
+            const float g = normed ? (cg < qd ? e.qn_g[cg % hd] : e.kn_g[cg % hd]) : 0.f;
+#pragma unroll
+            for (int j = 0; j < W; ++j) {
+                float a = 0.f;
+                for (int w = 0; w < nw; ++w) a += red[(w0 + w) * CH + j].x;
+                if (normed) v[j] *= g / sqrtf(a / (float)hd + e.qk_eps);
+            }
+            epi_bar();  // red is reused below
+        }
 #pragma unroll
         for (int j = 0; j < W; ++j) stg[n_local * STG_LD + j] = v[j];
         if (pre) epi_bar();  // smeta is already filled; stg must be complete before partners are read
         else qkv_fill_meta(e, m0c, nc, M, smeta);
-        const int hd = e.hd, half = hd >> 1;
-        const int qd = e.nq * hd, kd = e.nkv * hd;
-        const int cg = e.col0 + nt * 128 + n_local;  // row of [Wq; Wk; Wv]
         if (nt * 128 + n_local < p.N) {
             const int head_base = (cg / hd) * hd;
             const int d = cg - head_base;

@@ -82,6 +82,18 @@ typedef struct {
     int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
     int32_t n_experts, top_k, expert_ffn;   /* n_experts == 0: dense SwiGLU FFN */
     double rms_eps, rope_theta;
+    /* Fidelity toggles of real checkpoints (not on the DFlash pages; 0 = off).
+     * qk_norm = 1: every q and k head is RMS-normalised over head_dim (gain
+     * slots q_norm / k_norm [head_dim] per layer, eps rms_eps) before RoPE, as
+     * in Qwen3 layers; the drafter's context keys too.  rope_factor > 1: the
+     * RoPE frequencies are rescaled as published with Llama 3.1 -- a pair whose
+     * wavelength 2*pi/f is below rope_original_max_pos / rope_high_freq_factor
+     * keeps f, one above rope_original_max_pos / rope_low_freq_factor gets
+     * f / rope_factor, and in between the two are mixed with weight
+     * (rope_original_max_pos / wavelength - low) / (high - low) on f. */
+    int32_t qk_norm;
+    int32_t reserved;             /* 0 */
+    double rope_factor, rope_low_freq_factor, rope_high_freq_factor, rope_original_max_pos;
 } dflash_model_cfg;
 
 typedef struct {
@@ -98,7 +110,7 @@ typedef struct {
     int32_t keep_logits;          /* 1: keep fp32 logits of the last draft/verify for dflash_debug_logits */
     int32_t timeout_ms;           /* host wait bound for synchronising calls (0: 600000) */
     int32_t sampling;             /* 1: hold the buffers temperature sampling needs (dflash_set_sampling);
-                                     the LM heads then always store their fp32 logits */
+                                     while the temperature is above 0 the LM heads store fp32 logits */
 } dflash_config;
 
 typedef struct {
@@ -121,8 +133,16 @@ typedef struct {
 } dflash_kernel_prof;
 
 /* PROJECTION: every projection launch; ATTENTION: every attention launch;
- * GATE_UP: the gate/up (SwiGLU) projections alone (also counted in PROJECTION). */
-enum { DFLASH_PROF_PROJECTION = 0, DFLASH_PROF_ATTENTION = 1, DFLASH_PROF_GATE_UP = 2, DFLASH_PROF_CLASSES = 3 };
+ * then every projection once more by its shape: GATE_UP (SwiGLU gate/up),
+ * QKV, O (attention output), DOWN, LM_HEAD, FUSE (context fuse W_fc),
+ * OTHER_PROJ (MoE router).  DRAFT_PASS / VERIFY_PASS: one record per drafter
+ * pass (context fuse, drafter layers, head) and per verify pass (target
+ * layers, head, accept/commit), events at the pass boundaries only. */
+enum {
+    DFLASH_PROF_PROJECTION = 0, DFLASH_PROF_ATTENTION = 1, DFLASH_PROF_GATE_UP = 2, DFLASH_PROF_QKV = 3,
+    DFLASH_PROF_O = 4, DFLASH_PROF_DOWN = 5, DFLASH_PROF_LM_HEAD = 6, DFLASH_PROF_FUSE = 7,
+    DFLASH_PROF_OTHER_PROJ = 8, DFLASH_PROF_DRAFT_PASS = 9, DFLASH_PROF_VERIFY_PASS = 10, DFLASH_PROF_CLASSES = 11
+};
 
 /* Bytes of the weight and state arenas for this configuration.
  * Errors: DFLASH_EINVAL on inconsistent configuration, DFLASH_EUNSUPPORTED on
@@ -149,7 +169,8 @@ const char *dflash_last_error(const dflash_ctx *ctx);
  *   {target|drafter}.L{l}.attn_norm [H], .wqkv [(nq+2nkv)*hd, H] (rows Wq;Wk;Wv),
  *   .wo [H, nq*hd], .ffn_norm [H], .w_gate_up [2F, H] (rows W_gate;W_up),
  *   .w_down [H, F]; MoE layers: .w_router [E,H], .we_gate_up [E,2Fe,H],
- *   .we_down [E,H,Fe]; {target|drafter}.final_norm [H];
+ *   .we_down [E,H,Fe]; with qk_norm: .q_norm [hd], .k_norm [hd] (fp32);
+ *   {target|drafter}.final_norm [H];
  *   fuse.w_fc [H, n_taps*H], fuse.norm [H]. */
 int32_t dflash_weight_count(const dflash_ctx *ctx);
 dflash_status dflash_weight_info(const dflash_ctx *ctx, int32_t index, const char **name,
@@ -224,9 +245,12 @@ dflash_status dflash_decode_iters(dflash_ctx *ctx, int32_t n_seqs, int32_t iters
 dflash_status dflash_get_stats(dflash_ctx *ctx, dflash_stats *out);
 dflash_status dflash_reset_stats(dflash_ctx *ctx);
 
-/* Per-launch CUDA-event timing of the projection and attention kernels
- * (enable = 1 starts a fresh record, 0 stops).  Adds two event records per
- * timed launch.  dflash_profile_read fills out[DFLASH_PROF_CLASSES]. */
+/* CUDA-event timing on the context's stream.  mode 0 stops; a nonzero mode
+ * starts a fresh record: bit 0 = two events around every projection and
+ * attention launch (these break the overlap of consecutive kernels, so the
+ * pass is slower while it runs), bit 1 = two events around every drafter and
+ * verify pass.  dflash_profile_read fills out[DFLASH_PROF_CLASSES].
+ * Errors: EINVAL for a mode outside 0..3. */
 dflash_status dflash_profile(dflash_ctx *ctx, int32_t enable);
 dflash_status dflash_profile_read(dflash_ctx *ctx, dflash_kernel_prof *out);
 

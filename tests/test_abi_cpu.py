@@ -83,11 +83,52 @@ def test_create_rejects_missing_arenas(lib):
     assert not h.value
 
 
-def test_fidelity_toggles_are_refused_until_the_kernels_have_them():
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of dflash_model_cfg / dflash_config / dflash_stats /
+    dflash_kernel_prof have the C header's size and field offsets (gcc)."""
+    import ctypes as C
+    import subprocess
+    structs = {"dflash_model_cfg": dfl.ModelCfg, "dflash_config": dfl.Config, "dflash_stats": dfl.Stats,
+               "dflash_kernel_prof": dfl.KernelProf}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "dflash.h"', 'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            lines.append(f'printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(ln.split()[:2]): int(ln.split()[2]) for ln in out if ln.strip()}
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == C.sizeof(py), cname
+        for f, _ in py._fields_:
+            assert got[(cname, f)] == getattr(py, f).offset, (cname, f)
+
+
+def test_fidelity_toggles_reach_the_library():
+    """QK-norm adds the q_norm / k_norm slots of every layer; RoPE rescaling
+    needs 0 < low < high and a positive original length (EINVAL otherwise)."""
+    import ctypes as C
     from dataclasses import replace
     from synthetic import get_config
+    lib = dfl.load_library()
     base = get_config("tiny")
-    for t in (replace(base.target, qk_norm=True), replace(base.target, rope_scaling=(8.0, 1.0, 4.0, 256.0))):
-        with pytest.raises(NotImplementedError):
-            dfl.make_config(base.with_(target=t))
-    dfl.make_config(base.with_(target=replace(base.target, rope_scaling=(1.0, 1.0, 4.0, 256.0))))
+
+    def sizes(cfg):
+        c = dfl.make_config(cfg)
+        wb, sb = C.c_size_t(), C.c_size_t()
+        return lib.dflash_workspace_size(C.byref(c), C.byref(wb), C.byref(sb)), wb.value
+
+    st0, w0 = sizes(base)
+    qk = base.with_(target=replace(base.target, qk_norm=True), drafter=replace(base.drafter, qk_norm=True))
+    st1, w1 = sizes(qk)
+    assert st0 == st1 == dfl.DFLASH_OK
+    n_layers = base.target.n_layers + base.drafter.n_layers
+    assert w0 < w1 <= w0 + n_layers * 2 * (base.target.head_dim * 4 + 256)
+    ok = base.with_(target=replace(base.target, rope_scaling=(8.0, 1.0, 4.0, 256.0)))
+    assert sizes(ok)[0] == dfl.DFLASH_OK
+    bad = base.with_(target=replace(base.target, rope_scaling=(8.0, 4.0, 1.0, 256.0)))
+    assert sizes(bad)[0] == dfl.DFLASH_EINVAL

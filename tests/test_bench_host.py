@@ -62,8 +62,8 @@ def test_workload_config_and_threads():
     assert c["global_batch"] == 2 * cfg.batch and c["parallelism"] == "replicas x2"
     assert "512-token prompt" in c["workload"] and "36-layer target" in c["workload"]
     assert c["activations"].startswith("bf16 hi+lo")
-    assert c["l2"] == "inputs larger than L2 (18.7 GB streamed per step)"
+    assert c["l2"] == "inputs larger than L2 (18.6 GB streamed per step)"
     moe = bench.workload_config(get_config("qwen3_coder_30b_a3b"), A, 1)
-    assert moe["l2"] == "inputs larger than L2 (41.8 GB streamed per step)"
+    assert moe["l2"] == "inputs larger than L2 (41.6 GB streamed per step)"
     assert bench.workload_config(get_config("tiny"), A, 1)["l2"].startswith("inputs fit in L2")
     assert bench.omp_threads() >= 1

@@ -28,15 +28,18 @@ TOL = {"fp32": (1e-4, 1e-3), "bf16": (3e-2, 0.05)}
 
 
 def tiny_cfg(dtype="fp32", block=4, moe=False, t_layers=2, d_layers=1, nq=4, nkv=2, hd=64, hidden=256,
-             vocab=1024, taps=(0, 1), expert_ffn=64):
+             vocab=1024, taps=(0, 1), expert_ffn=64, qk_norm=False, rope_scaling=None):
     base = get_config("tiny")
     ffn = 3 * hidden
+    fid = dict(qk_norm=qk_norm)
+    if rope_scaling is not None:
+        fid["rope_scaling"] = rope_scaling
     t = replace(base.target, n_layers=t_layers, n_q_heads=nq, n_kv_heads=nkv, head_dim=hd, hidden=hidden,
-                vocab=vocab, ffn=ffn)
+                vocab=vocab, ffn=ffn, **fid)
     if moe:
         t = replace(t, n_experts=8, top_k=2, expert_ffn=expert_ffn)
     d = replace(base.drafter, n_layers=d_layers, n_q_heads=nq, n_kv_heads=nkv, head_dim=hd, hidden=hidden,
-                vocab=vocab, ffn=ffn)
+                vocab=vocab, ffn=ffn, **fid)
     return base.with_(target=t, drafter=d, block_size=block, tap_layers=taps, dtype=dtype)
 
 
@@ -292,3 +295,28 @@ def test_nonfinite_logits_report_enumeric(cuda_device):
     with pytest.raises(dfl.DFlashError) as e:
         gpu.verify_commit([0])
     assert e.value.status == dfl.DFLASH_ENUMERIC
+
+
+@pytest.mark.parametrize("dtype,toggle", [("fp32", "qk_norm"), ("bf16", "qk_norm"), ("fp32", "rope_scaled"),
+                                          ("bf16", "rope_scaled"), ("bf16", "both_hd128")])
+def test_fidelity_toggles_replay(cuda_device, dtype, toggle):
+    """Fidelity toggles of real checkpoints (not on the pages): Qwen3 QK-norm
+    (per-head RMSNorm of q and k before RoPE, context keys included) and the
+    Llama 3.1 RoPE frequency rescaling, with prompts long enough that all three
+    wavelength bands rotate; bf16 cases take the tensor-core epilogue (head_dim
+    64: two heads per 128-row tile; 128: one), fp32 the CUDA-core one."""
+    from test_oracle_pins import TINY_ROPE_SCALING
+    kw = dict(block=8)
+    if toggle in ("qk_norm", "both_hd128"):
+        kw["qk_norm"] = True
+    if toggle in ("rope_scaled", "both_hd128"):
+        kw["rope_scaling"] = TINY_ROPE_SCALING
+    if toggle == "both_hd128":
+        kw.update(block=16, hidden=512, nq=4, nkv=2, hd=128)
+    cfg = tiny_cfg(dtype, **kw)
+    tol, tie = TOL[dtype]
+    gpu, spec, _ = build_pair(cfg, max_batch=2, max_len=400)
+    prompts = [make_prompt("uniform", 300, cfg.target.vocab, 31), make_prompt("uniform", 45, cfg.target.vocab, 32)]
+    rep = replay(gpu, spec, cfg, prompts, 4, tol, tie)
+    print(f"{toggle} {dtype}: max |dlogit| {rep.max_dlogit:.2e}, near ties {rep.near_ties}/{rep.checked_tokens}")
+    _finish(rep, tol)
