@@ -9,7 +9,7 @@ import torch
 
 from .build import build_oracle
 
-ORC_F32, ORC_BF16 = 0, 1
+ORC_F32, ORC_BF16, ORC_FP8 = 0, 1, 2
 
 _lib = None
 
@@ -32,7 +32,12 @@ class Layer(C.Structure):
 
 class Model(C.Structure):
     _fields_ = [("d", Dims), ("dtype", C.c_int32), ("embed", C.c_void_p), ("lm_head", C.c_void_p),
-                ("final_norm", C.c_void_p), ("layers", C.POINTER(Layer))]
+                ("final_norm", C.c_void_p), ("layers", C.POINTER(Layer)), ("mat_dtype", C.c_int32)]
+
+
+class Fp8(C.Structure):
+    """orc_fp8: E4M3 codes [rows][K] and one fp32 scale per row."""
+    _fields_ = [("codes", C.c_void_p), ("scale", C.c_void_p)]
 
 
 class Spec(C.Structure):
@@ -56,6 +61,10 @@ def load_lib():
     lib.orc_rope_inv_freq.restype = C.c_double
     lib.orc_rope_dims.argtypes = [C.c_void_p, C.POINTER(Dims), C.c_int64]
     lib.orc_matmul.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_int32, C.c_void_p]
+    lib.orc_matmul_rows.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
+                                    C.c_void_p]
+    lib.orc_e4m3_value.argtypes = [C.c_uint8]
+    lib.orc_e4m3_value.restype = C.c_double
     lib.orc_attend.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_void_p]
     lib.orc_argmax.argtypes = [C.c_void_p, C.c_int32, C.c_void_p]
     lib.orc_argmax.restype = C.c_int32
@@ -101,9 +110,9 @@ def _i32(a) -> np.ndarray:
 
 
 def _wtensor(t: torch.Tensor) -> torch.Tensor:
-    """Host tensor in a storage type the oracle reads (fp32 or bf16 bits)."""
+    """Host tensor in a storage type the oracle reads (fp32, bf16 bits or FP8 codes)."""
     t = t.detach().to("cpu").contiguous()
-    if t.dtype not in (torch.float32, torch.bfloat16):
+    if t.dtype not in (torch.float32, torch.bfloat16, torch.uint8):
         raise TypeError(t.dtype)
     return t
 
@@ -126,11 +135,16 @@ class OracleSpec:
         w = {k: _wtensor(v) for k, v in weights.items()}
         self._keep.append(w)
         dtype = ORC_BF16 if w["embed"].dtype == torch.bfloat16 else ORC_F32
+        self.mat_dtype = ORC_FP8 if w["lm_head"].dtype == torch.uint8 else dtype
         for k, v in w.items():
-            if v.dim() > 1 and (v.dtype == torch.bfloat16) != (dtype == ORC_BF16):
+            if k == "embed" or k.endswith(".scale"):
+                continue
+            if v.dim() > 1 and v.dtype != {ORC_BF16: torch.bfloat16, ORC_F32: torch.float32,
+                                           ORC_FP8: torch.uint8}[self.mat_dtype]:
                 raise TypeError(f"{k}: mixed storage types")
             if v.dim() == 1 and v.dtype != torch.float32:
                 raise TypeError(f"{k}: norm gains must be fp32")
+        self._w = w
         self.spec = Spec()
         self.spec.target = self._model("target", cfg.target, w, dtype)
         self.spec.drafter = self._model("drafter", cfg.drafter, w, dtype)
@@ -140,23 +154,35 @@ class OracleSpec:
         self.spec.n_taps = len(cfg.tap_layers)
         self.spec.tap_layers = taps.ctypes.data_as(_ip)
         self.spec.mask_token_id = cfg.mask_id
-        self.spec.w_fc = _ptr(w["fuse.w_fc"])
+        self.spec.w_fc = self._mat("fuse.w_fc")
         self.spec.fc_norm = _ptr(w["fuse.norm"])
+
+    def _mat(self, name):
+        """Address the oracle reads matrix `name` from: its storage, or for FP8
+        weights an orc_fp8 descriptor of its codes and per-row scales."""
+        if self.mat_dtype != ORC_FP8:
+            return _ptr(self._w[name])
+        q = Fp8(_ptr(self._w[name]), _ptr(self._w[name + ".scale"]))
+        self._keep.append(q)
+        return C.addressof(q)
 
     def _model(self, prefix, d, w, dtype) -> Model:
         m = Model()
         m.d = dims(d)
         m.dtype = dtype
+        m.mat_dtype = self.mat_dtype
+        if self.mat_dtype == ORC_FP8 and d.n_experts > 0:
+            raise ValueError("the oracle reads FP8 weights for dense models only")
         m.embed = _ptr(w["embed"])
-        m.lm_head = _ptr(w["lm_head"])
+        m.lm_head = self._mat("lm_head")
         m.final_norm = _ptr(w[f"{prefix}.final_norm"])
         layers = (Layer * max(1, d.n_layers))()
         for l in range(d.n_layers):
             p = f"{prefix}.L{l}."
             L = layers[l]
             L.attn_norm = _ptr(w[p + "attn_norm"])
-            L.wqkv = _ptr(w[p + "wqkv"])
-            L.wo = _ptr(w[p + "wo"])
+            L.wqkv = self._mat(p + "wqkv")
+            L.wo = self._mat(p + "wo")
             L.ffn_norm = _ptr(w[p + "ffn_norm"])
             if d.qk_norm:
                 L.q_norm = _ptr(w[p + "q_norm"])
@@ -166,8 +192,8 @@ class OracleSpec:
                 L.we_gate_up = _ptr(w[p + "we_gate_up"])
                 L.we_down = _ptr(w[p + "we_down"])
             else:
-                L.w_gate_up = _ptr(w[p + "w_gate_up"])
-                L.w_down = _ptr(w[p + "w_down"])
+                L.w_gate_up = self._mat(p + "w_gate_up")
+                L.w_down = self._mat(p + "w_down")
         self._keep.append(layers)
         m.layers = C.cast(layers, C.POINTER(Layer))
         return m
@@ -317,6 +343,23 @@ def matmul(W: torch.Tensor, X) -> np.ndarray:
     Y = np.zeros((XX.shape[0], N), np.float64)
     lib.orc_matmul(_ptr(W), dt, N, K, XX.ctypes.data, XX.shape[0], Y.ctypes.data)
     return Y
+
+
+def matmul_fp8(codes: torch.Tensor, scale: torch.Tensor, X, row0: int = 0, n_rows: Optional[int] = None) -> np.ndarray:
+    """Y[r][n] = sum_k scale[row0+n] * e4m3(codes[row0+n][k]) * X[r][k] through the oracle."""
+    lib = load_lib()
+    codes, scale = _wtensor(codes), _wtensor(scale)
+    N, K = codes.shape
+    n = N - row0 if n_rows is None else n_rows
+    q = Fp8(_ptr(codes), _ptr(scale))
+    XX = _f64(X).reshape(-1, K)
+    Y = np.zeros((XX.shape[0], n), np.float64)
+    lib.orc_matmul_rows(C.addressof(q), ORC_FP8, row0, n, K, XX.ctypes.data, XX.shape[0], Y.ctypes.data)
+    return Y
+
+
+def e4m3_value(code: int) -> float:
+    return load_lib().orc_e4m3_value(int(code) & 0xFF)
 
 
 def attend(q, keys, vals) -> np.ndarray:

@@ -71,6 +71,36 @@ static inline double wget(const void *w, int32_t dtype, size_t i) {
                              : (double)((const float *)w)[i];
 }
 
+/* E4M3 (OCP 8-bit float, 4 exponent bits with bias 7, 3 mantissa bits, no
+ * infinities): sign * 2^(e-7) * (1 + m/8) for e > 0, sign * 2^-6 * (m/8) for
+ * e = 0; codes 0x7F / 0xFF are NaN.  Written from that definition. */
+double orc_e4m3_value(uint8_t c) {
+    int32_t e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (c & 0x80) ? -mag : mag;
+}
+
+/* Dot product of one row of an FP8 matrix: the quantised weight of element k
+ * is scale * e4m3_value(code_k) (fp64), summed like the other dot products. */
+static double dot_fp8(const uint8_t *c, double scale, const double *x, int32_t K) {
+    double a0 = 0, a1 = 0, a2 = 0, a3 = 0, a4 = 0, a5 = 0, a6 = 0, a7 = 0;
+    int32_t k = 0;
+    for (; k + 8 <= K; k += 8) {
+        a0 += scale * orc_e4m3_value(c[k + 0]) * x[k + 0];
+        a1 += scale * orc_e4m3_value(c[k + 1]) * x[k + 1];
+        a2 += scale * orc_e4m3_value(c[k + 2]) * x[k + 2];
+        a3 += scale * orc_e4m3_value(c[k + 3]) * x[k + 3];
+        a4 += scale * orc_e4m3_value(c[k + 4]) * x[k + 4];
+        a5 += scale * orc_e4m3_value(c[k + 5]) * x[k + 5];
+        a6 += scale * orc_e4m3_value(c[k + 6]) * x[k + 6];
+        a7 += scale * orc_e4m3_value(c[k + 7]) * x[k + 7];
+    }
+    double s = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+    for (; k < K; ++k) s += scale * orc_e4m3_value(c[k]) * x[k];
+    return s;
+}
+
 static inline const void *wrow(const void *w, int32_t dtype, size_t elem_offset) {
     return dtype == ORC_BF16 ? (const void *)((const uint16_t *)w + elem_offset)
                              : (const void *)((const float *)w + elem_offset);
@@ -135,18 +165,30 @@ static double dot_f64(const double *a, const double *b, int32_t K) {
 /* building blocks                                                     */
 /* ------------------------------------------------------------------ */
 
-void orc_matmul(const void *W, int32_t dtype, int32_t N, int32_t K,
-                const double *X, int32_t R, double *Y) {
-    /* Y[r][n] = sum_k W[n][k] * X[r][k]; each (r, n) is one dot_* call. */
+void orc_matmul_rows(const void *W, int32_t dtype, int32_t row0, int32_t N, int32_t K,
+                     const double *X, int32_t R, double *Y) {
+    /* Y[r][n] = sum_k W[row0 + n][k] * X[r][k]; each (r, n) is one dot_* call. */
 #pragma omp parallel for schedule(static)
     for (int32_t n = 0; n < N; ++n) {
+        const size_t row = (size_t)row0 + (size_t)n;
         for (int32_t r = 0; r < R; ++r) {
-            double v = dtype == ORC_BF16
-                ? dot_bf16((const uint16_t *)W + (size_t)n * K, X + (size_t)r * K, K)
-                : dot_f32((const float *)W + (size_t)n * K, X + (size_t)r * K, K);
+            double v;
+            if (dtype == ORC_FP8) {
+                const orc_fp8 *q = (const orc_fp8 *)W;
+                v = dot_fp8(q->codes + row * K, (double)q->scale[row], X + (size_t)r * K, K);
+            } else if (dtype == ORC_BF16) {
+                v = dot_bf16((const uint16_t *)W + row * K, X + (size_t)r * K, K);
+            } else {
+                v = dot_f32((const float *)W + row * K, X + (size_t)r * K, K);
+            }
             Y[(size_t)r * N + n] = v;
         }
     }
+}
+
+void orc_matmul(const void *W, int32_t dtype, int32_t N, int32_t K,
+                const double *X, int32_t R, double *Y) {
+    orc_matmul_rows(W, dtype, 0, N, K, X, R, Y);
 }
 
 void orc_rmsnorm(const double *x, const float *g, int32_t n, double eps, double *y) {
@@ -276,7 +318,7 @@ static void moe_row(const orc_model *m, const orc_layer *L, const double *x, dou
     const orc_dims *d = &m->d;
     int32_t E = d->n_experts, H = d->hidden, Fe = d->expert_ffn, K = d->top_k;
     double *r = (double *)malloc(sizeof(double) * (size_t)E);
-    orc_matmul(L->w_router, m->dtype, E, H, x, 1, r);
+    orc_matmul(L->w_router, m->mat_dtype, E, H, x, 1, r);
     double mx = -INFINITY;
     for (int32_t e = 0; e < E; ++e) if (r[e] > mx) mx = r[e];
     double den = 0.0;
@@ -298,8 +340,8 @@ static void moe_row(const orc_model *m, const orc_layer *L, const double *x, dou
     for (int32_t k = 0; k < K; ++k) {
         int32_t e = sel[k];
         double w = r[e] / wsum;
-        swiglu_rows(wrow(L->we_gate_up, m->dtype, (size_t)e * 2 * Fe * H),
-                    wrow(L->we_down, m->dtype, (size_t)e * H * Fe), m->dtype, H, Fe, x, 1, y);
+        swiglu_rows(wrow(L->we_gate_up, m->mat_dtype, (size_t)e * 2 * Fe * H),
+                    wrow(L->we_down, m->mat_dtype, (size_t)e * H * Fe), m->mat_dtype, H, Fe, x, 1, y);
         for (int32_t i = 0; i < H; ++i) out[i] += w * y[i];
     }
     free(y); free(used); free(sel); free(r);
@@ -308,7 +350,7 @@ static void moe_row(const orc_model *m, const orc_layer *L, const double *x, dou
 void orc_ffn(const orc_model *m, int32_t layer, const double *x, double *out) {
     const orc_layer *L = &m->layers[layer];
     if (m->d.n_experts > 0) moe_row(m, L, x, out);
-    else swiglu_rows(L->w_gate_up, L->w_down, m->dtype, m->d.hidden, m->d.ffn, x, 1, out);
+    else swiglu_rows(L->w_gate_up, L->w_down, m->mat_dtype, m->d.hidden, m->d.ffn, x, 1, out);
 }
 
 static void ffn_rows(const orc_model *m, int32_t layer, const double *xn, int32_t R, double *out) {
@@ -318,14 +360,14 @@ static void ffn_rows(const orc_model *m, int32_t layer, const double *xn, int32_
 #pragma omp parallel for schedule(dynamic, 1) if (R > 1)
         for (int32_t r = 0; r < R; ++r) moe_row(m, L, xn + (size_t)r * H, out + (size_t)r * H);
     } else {
-        swiglu_rows(L->w_gate_up, L->w_down, m->dtype, H, m->d.ffn, xn, R, out);
+        swiglu_rows(L->w_gate_up, L->w_down, m->mat_dtype, H, m->d.ffn, xn, R, out);
     }
 }
 
 void orc_fuse(const orc_spec *s, const double *taps, double *c) {
     int32_t H = s->target.d.hidden, Hd = s->drafter.d.hidden;
     double *u = (double *)malloc(sizeof(double) * (size_t)Hd);
-    orc_matmul(s->w_fc, s->drafter.dtype, Hd, s->n_taps * H, taps, 1, u);
+    orc_matmul(s->w_fc, s->drafter.mat_dtype, Hd, s->n_taps * H, taps, 1, u);
     orc_rmsnorm(u, s->fc_norm, Hd, s->drafter.d.rms_eps, c);
     free(u);
 }
@@ -422,7 +464,7 @@ static void layer_rows(const orc_model *m, int32_t l, double *x, int32_t R, int3
     double *att = (double *)malloc(sizeof(double) * (size_t)R * qd);
     double *o = (double *)malloc(sizeof(double) * (size_t)R * H);
     for (int32_t r = 0; r < R; ++r) orc_rmsnorm(x + (size_t)r * H, L->attn_norm, H, d->rms_eps, n + (size_t)r * H);
-    orc_matmul(L->wqkv, m->dtype, nqkv, H, n, R, qkv);
+    orc_matmul(L->wqkv, m->mat_dtype, nqkv, H, n, R, qkv);
     for (int32_t r = 0; r < R; ++r) {
         const double *row = qkv + (size_t)r * nqkv;
         int32_t pos = pos0 + r;
@@ -436,7 +478,7 @@ static void layer_rows(const orc_model *m, int32_t l, double *x, int32_t R, int3
         for (int32_t g = 0; g < nkv; ++g) orc_rope_dims(kp + (size_t)g * hd, d, pos);
     }
     attn_rows(d, q, kc, vc, n_keys, R, att);
-    orc_matmul(L->wo, m->dtype, H, qd, att, R, o);
+    orc_matmul(L->wo, m->mat_dtype, H, qd, att, R, o);
     for (size_t i = 0; i < (size_t)R * H; ++i) x[i] += o[i];
     for (int32_t r = 0; r < R; ++r) orc_rmsnorm(x + (size_t)r * H, L->ffn_norm, H, d->rms_eps, n + (size_t)r * H);
     ffn_rows(m, l, n, R, o);
@@ -491,7 +533,7 @@ static void inject_ctx(orc_session *ss, int32_t n_rows, int32_t pos0) {
     for (int32_t r = 0; r < n_rows; ++r) orc_fuse(&ss->s, ss->taps + (size_t)r * nt * Ht, c + (size_t)r * Hd);
     for (int32_t j = 0; j < d->n_layers; ++j) {
         /* rows qd..qd+2kd of Wqkv_j are [Wk_j; Wv_j] */
-        orc_matmul(wrow(m->layers[j].wqkv, m->dtype, (size_t)qd * Hd), m->dtype, 2 * kd, Hd, c, n_rows, kv);
+        orc_matmul_rows(m->layers[j].wqkv, m->mat_dtype, qd, 2 * kd, Hd, c, n_rows, kv);
         for (int32_t r = 0; r < n_rows; ++r) {
             int32_t t = pos0 + r;
             double *kp = tkv_at(ss->dk, d, ss->max_len, j, t), *vp = tkv_at(ss->dv, d, ss->max_len, j, t);
@@ -513,7 +555,7 @@ static int32_t prefill_impl(orc_session *ss, const int32_t *prompt, int32_t n, d
     double *lg = (double *)malloc(sizeof(double) * (size_t)V);
     ss->len = 0;
     target_rows(ss, prompt, n, x);
-    head_rows(m, m->lm_head, m->dtype, V, x + (size_t)(n - 1) * H, 1, lg);
+    head_rows(m, m->lm_head, m->mat_dtype, V, x + (size_t)(n - 1) * H, 1, lg);
     int32_t tok = orc_argmax(lg, V, margin);
     if (last_logits) memcpy(last_logits, lg, sizeof(double) * V);
     if (with_ctx) inject_ctx(ss, n, 0);
@@ -543,7 +585,7 @@ void orc_draft(orc_session *ss, int32_t anchor, int32_t *drafts, double *logits,
         layer_rows(m, j, x, B, p, tkv_at(ss->dk, d, ss->max_len, j, 0),
                    tkv_at(ss->dv, d, ss->max_len, j, 0), nk);
     if (B > 1) {
-        head_rows(m, t->lm_head, t->dtype, V, x + H, B - 1, lg);
+        head_rows(m, t->lm_head, t->mat_dtype, V, x + H, B - 1, lg);
         for (int32_t r = 0; r < B - 1; ++r)
             drafts[r] = orc_argmax(lg + (size_t)r * V, V, margins ? margins + r : NULL);
         if (logits) memcpy(logits, lg, sizeof(double) * (size_t)(B - 1) * V);
@@ -557,7 +599,7 @@ void orc_verify(orc_session *ss, const int32_t *tokens, int32_t *g, double *logi
     double *x = (double *)malloc(sizeof(double) * (size_t)B * H);
     double *lg = (double *)malloc(sizeof(double) * (size_t)B * V);
     target_rows(ss, tokens, B, x);
-    head_rows(m, m->lm_head, m->dtype, V, x, B, lg);
+    head_rows(m, m->lm_head, m->mat_dtype, V, x, B, lg);
     for (int32_t r = 0; r < B; ++r) g[r] = orc_argmax(lg + (size_t)r * V, V, margins ? margins + r : NULL);
     if (logits) memcpy(logits, lg, sizeof(double) * (size_t)B * V);
     free(x); free(lg);
@@ -585,7 +627,7 @@ void orc_generate_ar(const orc_spec *s, const int32_t *prompt, int32_t n, int32_
     for (int32_t i = 1; i < max_new; ++i) {
         target_rows(ss, out + i - 1, 1, x);
         ss->len += 1;
-        head_rows(m, m->lm_head, m->dtype, V, x, 1, lg);
+        head_rows(m, m->lm_head, m->mat_dtype, V, x, 1, lg);
         out[i] = orc_argmax(lg, V, margins ? margins + i : NULL);
     }
     free(x); free(lg);

@@ -21,7 +21,8 @@
  *
  * Everything the pages leave open follows one stated reading (see the .c file).
  * All arithmetic is IEEE fp64.  Matrix weights are read from fp32 or bf16
- * storage and widened exactly to fp64.
+ * storage and widened exactly to fp64, or from FP8 codes with per-row scales
+ * (scale * E4M3 value, in fp64).
  */
 #ifndef DFLASH_ORACLE_H
 #define DFLASH_ORACLE_H
@@ -32,7 +33,15 @@
 extern "C" {
 #endif
 
-enum { ORC_F32 = 0, ORC_BF16 = 1 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8 = 2 };
+
+/* A matrix in FP8 storage: E4M3 codes [rows][K] and one fp32 scale per row;
+ * the quantised weight is scale[row] * e4m3_value(code).  Matrix pointers of
+ * an ORC_FP8 model point to one of these. */
+typedef struct {
+    const uint8_t *codes;
+    const float *scale;
+} orc_fp8;
 
 typedef struct {
     int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
@@ -61,11 +70,13 @@ typedef struct {
 
 typedef struct {
     orc_dims d;
-    int32_t dtype;            /* storage type of matrices: ORC_F32 / ORC_BF16 */
+    int32_t dtype;            /* storage type of the embedding: ORC_F32 / ORC_BF16 */
     const void *embed;        /* [V, H] (the drafter uses the target's) */
     const void *lm_head;      /* [V, H] (the drafter uses the target's) */
     const float *final_norm;  /* [H] */
     const orc_layer *layers;  /* [n_layers] */
+    int32_t mat_dtype;        /* storage of the projection matrices, the LM head and W_fc:
+                                 ORC_F32, ORC_BF16 or ORC_FP8 (pointers to orc_fp8) */
 } orc_model;
 
 typedef struct {
@@ -87,9 +98,14 @@ void orc_rope(double *v, int32_t head_dim, int64_t pos, double theta);
  * rescaled when rope_factor > 1), and the rotation with those frequencies. */
 double orc_rope_inv_freq(const orc_dims *d, int32_t i);
 void orc_rope_dims(double *v, const orc_dims *d, int64_t pos);
-/* Y[r][n] = sum_k W[n][k] X[r][k]; W in fp32/bf16 storage. */
+/* Y[r][n] = sum_k W[n][k] X[r][k]; W in fp32 / bf16 / FP8 storage. */
 void orc_matmul(const void *W, int32_t dtype, int32_t N, int32_t K,
                 const double *X, int32_t R, double *Y);
+/* The same over rows row0 .. row0+N-1 of W. */
+void orc_matmul_rows(const void *W, int32_t dtype, int32_t row0, int32_t N, int32_t K,
+                     const double *X, int32_t R, double *Y);
+/* Value of an E4M3 code (NaN for 0x7F / 0xFF). */
+double orc_e4m3_value(uint8_t code);
 /* One query row over keys[0..n_keys) (each hd doubles, stride ld_k); softmax scale 1/sqrt(hd). */
 void orc_attend(const double *q, const double *keys, const double *vals, int64_t ld_kv,
                 int32_t n_keys, int32_t head_dim, double *out);

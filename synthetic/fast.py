@@ -53,6 +53,20 @@ def make_weight_host(cfg: SpecConfig, name: str, random_gains: bool = False, see
         lib.fastgen_f32(t.data_ptr(), n, key, float(torch.tensor(0.1 / SIGMA_S, dtype=torch.float32)), 1.0, 1)
         return t
     scale = float(torch.tensor(cfg.weight_std / SIGMA_S, dtype=torch.float32))
+    if kind in ("fp8", "scale"):
+        from .weights import quantized
+        base = name[:-len(".scale")] if kind == "scale" else name
+        bshape = weight_shapes(cfg)[base][0]
+        bn = 1
+        for d in bshape:
+            bn *= d
+
+        def make_base():
+            t = torch.empty(bshape, dtype=torch.bfloat16)
+            lib.fastgen_bf16(t.data_ptr(), bn, tensor_key(base, seed), scale)
+            return t
+        codes, sc = quantized(base, (cfg.name, seed, "cpu", cfg.weight_std), make_base)
+        return sc if kind == "scale" else codes
     if storage_dtype(cfg) == torch.bfloat16:
         t = torch.empty(shape, dtype=torch.bfloat16)
         lib.fastgen_bf16(t.data_ptr(), n, key, scale)

@@ -117,7 +117,11 @@ def _layer_shapes(prefix: str, d: ModelDims) -> "OrderedDict[str, Tuple[Tuple[in
 
 
 def weight_shapes(cfg: SpecConfig) -> "OrderedDict[str, Tuple[Tuple[int, ...], str]]":
-    """Logical, row-major tensors of one workload, in a fixed order."""
+    """Logical, row-major tensors of one workload, in a fixed order.
+
+    With cfg.dtype == "fp8" every matrix but the embedding is stored as E4M3
+    codes (kind "fp8", uint8) plus "<name>.scale" (kind "scale", fp32, one
+    value per row); see synthetic.fp8."""
     t, dr = cfg.target, cfg.drafter
     s: "OrderedDict[str, Tuple[Tuple[int, ...], str]]" = OrderedDict()
     s["embed"] = ((t.vocab, t.hidden), "matrix")
@@ -126,7 +130,18 @@ def weight_shapes(cfg: SpecConfig) -> "OrderedDict[str, Tuple[Tuple[int, ...], s
     s.update(_layer_shapes("drafter", dr))
     s["fuse.w_fc"] = ((dr.hidden, cfg.n_taps * t.hidden), "matrix")
     s["fuse.norm"] = ((dr.hidden,), "norm")
-    return s
+    if cfg.dtype != "fp8":
+        return s
+    if t.is_moe:
+        raise ValueError("fp8 weights are built for dense targets only")
+    q: "OrderedDict[str, Tuple[Tuple[int, ...], str]]" = OrderedDict()
+    for name, (shape, kind) in s.items():
+        if kind == "matrix" and name != "embed":
+            q[name] = (shape, "fp8")
+            q[name + ".scale"] = (shape[:-1], "scale")
+        else:
+            q[name] = (shape, kind)
+    return q
 
 
 def weight_names(cfg: SpecConfig):
@@ -134,7 +149,21 @@ def weight_names(cfg: SpecConfig):
 
 
 def storage_dtype(cfg: SpecConfig) -> torch.dtype:
-    return torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    """Type of the generated matrices (fp8 models quantise bf16 ones)."""
+    return torch.bfloat16 if cfg.dtype in ("bf16", "fp8") else torch.float32
+
+
+_QCACHE: dict = {}
+
+
+def quantized(name: str, key, make_base):
+    """(codes, scale) of matrix `name`, cached for the codes / scale pair."""
+    from .fp8 import quantize_rows
+    k = (name, key)
+    if k not in _QCACHE:
+        _QCACHE.clear()
+        _QCACHE[k] = quantize_rows(make_base())
+    return _QCACHE[k]
 
 
 def make_weight(cfg: SpecConfig, name: str, device="cpu", random_gains: bool = False,
@@ -145,6 +174,13 @@ def make_weight(cfg: SpecConfig, name: str, device="cpu", random_gains: bool = F
         if not random_gains:
             return torch.ones(shape, dtype=torch.float32, device=device)
         return _fill(shape, name, seed, 0.1 / SIGMA_S, 1.0, torch.float32, device)
+    if kind in ("fp8", "scale"):
+        base = name[:-len(".scale")] if kind == "scale" else name
+        bshape = weight_shapes(cfg)[base][0]
+        codes, scale = quantized(base, (cfg.name, seed, str(device), cfg.weight_std),
+                                 lambda: _fill(bshape, base, seed, cfg.weight_std / SIGMA_S, 0.0, torch.bfloat16,
+                                               device))
+        return scale if kind == "scale" else codes
     return _fill(shape, name, seed, cfg.weight_std / SIGMA_S, 0.0, storage_dtype(cfg), device)
 
 
