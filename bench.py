@@ -118,16 +118,17 @@ def iteration_bytes(cfg, batch: int, mean_ctx: float, kv_planes: int = 1) -> flo
     """Algorithmic HBM bytes of one draft+verify iteration: every projection
     matrix once (the LM head twice: drafter and target), plus K/V reads of both
     models at the mean context length (kv_planes bf16 planes per element)."""
-    es = 2 if cfg.dtype == "bf16" else 4
+    es = 2 if cfg.dtype in ("bf16", "fp8") else 4   # activations / K/V (and bf16 weights)
     shapes = weight_shapes(cfg)
     w = 0
     for name, (shape, kind) in shapes.items():
-        if kind != "matrix" or name == "embed":
+        if kind not in ("matrix", "fp8", "scale") or name == "embed":
             continue
         n = int(np.prod(shape))
         if name.endswith("we_gate_up") or name.endswith("we_down"):
             continue  # MoE experts: only the touched ones are read (below)
-        w += n * es * (2 if name == "lm_head" else 1)
+        wes = {"matrix": es, "fp8": 1, "scale": 4}[kind]
+        w += n * wes * (2 if name.startswith("lm_head") else 1)
     t, d = cfg.target, cfg.drafter
     if t.is_moe:
         # expected experts a verify pass touches per layer when its batch*block rows
@@ -249,6 +250,8 @@ def main():
     ap.add_argument("--no-sampling", action="store_true")
     ap.add_argument("--bf16-act", choices=["split", "fast"], default="split",
                     help="bf16 activations as two planes (parity-grade) or one plane")
+    ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
+                    help="weight storage: bf16, or FP8 E4M3 codes with per-row scales (a quantised model)")
     ap.add_argument("--e2e-tokens", type=int, default=128)
     ap.add_argument("--profile-steps", type=int, default=50)
     ap.add_argument("--target-layers", type=int, default=None, help="layer-reduced copy (profiling small cases)")
@@ -266,6 +269,8 @@ def main():
         cfg = cfg.with_(batch=args.batch)
     if args.prompt_len:
         cfg = cfg.with_(prompt_len=args.prompt_len)
+    if args.weights == "fp8":
+        cfg = cfg.with_(dtype="fp8")
     if args.target_layers or args.drafter_layers:
         from synthetic.configs import shrink
         cfg = shrink(cfg, target_layers=args.target_layers or cfg.target.n_layers,
@@ -545,7 +550,9 @@ def workload_config(cfg, args, world, prompt_len=None):
             "global_batch": b * world, "seq_len": plen, "block_size": B,
             "parallelism": f"replicas x{world}",
             "activations": ("bf16 hi+lo planes, fp32 accumulate" if args.bf16_act == "split"
-                            else "bf16 single plane, fp32 accumulate") if cfg.dtype == "bf16" else "fp32",
+                            else "bf16 single plane, fp32 accumulate") if cfg.dtype in ("bf16", "fp8") else "fp32",
+            "weights": {"bf16": "bf16", "fp8": "FP8 E4M3 codes + per-row fp32 scales (quantised model)",
+                        "fp32": "fp32"}[cfg.dtype],
             "l2": l2_note(cfg)}
 
 

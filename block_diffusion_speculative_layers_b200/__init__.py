@@ -19,9 +19,10 @@ from .build import lib_path
 
 DFLASH_OK, DFLASH_EINVAL, DFLASH_ESTATE, DFLASH_ECAPACITY = 0, 1, 2, 3
 DFLASH_ECUDA, DFLASH_ENUMERIC, DFLASH_ETIMEOUT, DFLASH_EUNSUPPORTED = 4, 5, 6, 7
-DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST = 0, 1, 2
+DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST, DFLASH_FP8 = 0, 1, 2, 3
+_SLOT_TYPES = {DFLASH_FP32: (torch.float32, 4), DFLASH_BF16: (torch.bfloat16, 2), DFLASH_FP8: (torch.uint8, 1)}
 DFLASH_DRAFT_MODEL, DFLASH_DRAFT_SCRIPT = 0, 1
-MAX_TAPS, MAX_BLOCK = 8, 16
+MAX_TAPS, MAX_BLOCK = 8, 32
 # dflash_profile_read classes, in the order of the DFLASH_PROF_* values
 PROF_CLASSES = ("projection", "attention", "gate_up", "qkv", "o", "down", "lm_head", "fuse", "other_proj",
                 "draft_pass", "verify_pass")
@@ -158,6 +159,8 @@ def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: in
     c.prefill_chunk = prefill_chunk
     if spec.dtype == "bf16":
         c.dtype = DFLASH_BF16 if bf16_act == "split" else DFLASH_BF16_FAST
+    elif spec.dtype == "fp8":
+        c.dtype = DFLASH_FP8
     else:
         c.dtype = DFLASH_FP32
     c.keep_logits = 1 if keep_logits else 0
@@ -235,8 +238,7 @@ class DFlash:
 
     def weight_view(self, name: str) -> torch.Tensor:
         off, numel, dt, shape = self.weight_slots()[name]
-        tdt = torch.bfloat16 if dt == DFLASH_BF16 else torch.float32
-        es = 2 if dt == DFLASH_BF16 else 4
+        tdt, es = _SLOT_TYPES[dt]
         base = self._woff + off
         return self.warena[base:base + numel * es].view(tdt).view(shape)
 
@@ -247,10 +249,9 @@ class DFlash:
             raise KeyError(f"missing weights: {sorted(missing)[:5]}")
         for name, (off, numel, dt, shape) in slots.items():
             t = weights[name]
-            tdt = torch.bfloat16 if dt == DFLASH_BF16 else torch.float32
+            tdt, es = _SLOT_TYPES[dt]
             if tuple(t.shape) != shape or t.dtype != tdt:
                 raise ValueError(f"{name}: expected {shape} {tdt}, got {tuple(t.shape)} {t.dtype}")
-            es = 2 if dt == DFLASH_BF16 else 4
             base = self._woff + off
             self.warena[base:base + numel * es].view(tdt).view(shape).copy_(t, non_blocking=False)
         torch.cuda.synchronize(self.device)
@@ -334,10 +335,9 @@ class DFlash:
         for name in (names or slots):
             off, numel, dt, shape = slots[name]
             t = make_one(name)
-            tdt = torch.bfloat16 if dt == DFLASH_BF16 else torch.float32
+            tdt, es = _SLOT_TYPES[dt]
             if tuple(t.shape) != shape or t.dtype != tdt:
                 raise ValueError(f"{name}: expected {shape} {tdt}, got {tuple(t.shape)} {t.dtype}")
-            es = 2 if dt == DFLASH_BF16 else 4
             base = self._woff + off
             self.warena[base:base + numel * es].view(tdt).view(shape).copy_(t)
             del t
@@ -390,4 +390,5 @@ class DFlash:
 
 
 __all__ = ["DFlash", "DFlashError", "load_library", "make_config", "Config", "Stats", "EXPORTS",
-           "DFLASH_DRAFT_MODEL", "DFLASH_DRAFT_SCRIPT", "DFLASH_FP32", "DFLASH_BF16", "DFLASH_BF16_FAST"]
+           "DFLASH_DRAFT_MODEL", "DFLASH_DRAFT_SCRIPT", "DFLASH_FP32", "DFLASH_BF16", "DFLASH_BF16_FAST",
+           "DFLASH_FP8"]

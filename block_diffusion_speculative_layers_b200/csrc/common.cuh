@@ -35,7 +35,7 @@ struct SeqState {
 struct DevStats {
     unsigned long long iterations;          // sequence-iterations
     unsigned long long tokens;              // tokens emitted by verify/commit
-    unsigned long long hist[16];
+    unsigned long long hist[32];             // accept lengths a (block size <= 32)
     int32_t n_done;                         // sequences that reached max_new
     int32_t status;                         // nonzero: non-finite logits seen
 };

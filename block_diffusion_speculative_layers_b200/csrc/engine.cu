@@ -27,6 +27,7 @@
 #include "engine.h"
 #include "gemm_tc.h"
 #include "attn_mma.h"
+#include "attn_tma.h"
 #include "pass_program.h"
 
 namespace dfl {
@@ -70,7 +71,7 @@ static void *noalloc_scratch_ptr(int dev, std::string &err) {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-static int elem_size(int dtype) { return dtype == DFLASH_FP32 ? 4 : 2; }
+static int elem_size(int dtype) { return dtype == DFLASH_FP32 ? 4 : dtype == DFLASH_FP8 ? 1 : 2; }
 
 static bool check_model(const dflash_model_cfg &m, std::string &why) {
     if (m.n_layers < 1 || m.hidden < 32 || m.n_q_heads < 1 || m.n_kv_heads < 1 || m.vocab < 2) {
@@ -110,7 +111,7 @@ static bool check_config(const dflash_config &c, std::string &why) {
         why = "drafter hidden/vocab must equal the target's (shared embedding and head)";
         return false;
     }
-    if (c.block_size < 1 || c.block_size > DFLASH_MAX_BLOCK) { why = "block_size must be in [1, 16]"; return false; }
+    if (c.block_size < 1 || c.block_size > DFLASH_MAX_BLOCK) { why = "block_size must be in [1, 32]"; return false; }
     if (c.n_taps < 1 || c.n_taps > DFLASH_MAX_TAPS) { why = "n_taps must be in [1, 8]"; return false; }
     for (int i = 0; i < c.n_taps; ++i)
         if (c.tap_layers[i] < 0 || c.tap_layers[i] >= c.target.n_layers) { why = "tap layer out of range"; return false; }
@@ -118,11 +119,29 @@ static bool check_config(const dflash_config &c, std::string &why) {
     if (c.max_batch < 1 || c.max_batch > 64) { why = "max_batch must be in [1, 64]"; return false; }
     if (c.max_len < c.block_size + 1 || c.max_len > (1 << 20)) { why = "max_len out of range"; return false; }
     if (c.prefill_chunk < 0 || c.prefill_chunk > 8192) { why = "prefill_chunk must be in [0, 8192]"; return false; }
-    if (c.dtype != DFLASH_FP32 && c.dtype != DFLASH_BF16 && c.dtype != DFLASH_BF16_FAST) {
-        why = "dtype must be DFLASH_FP32, DFLASH_BF16 or DFLASH_BF16_FAST";
+    if (c.dtype != DFLASH_FP32 && c.dtype != DFLASH_BF16 && c.dtype != DFLASH_BF16_FAST && c.dtype != DFLASH_FP8) {
+        why = "dtype must be DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST or DFLASH_FP8";
         return false;
     }
+    if (c.dtype == DFLASH_FP8) {
+        const dflash_model_cfg *ms[2] = {&c.target, &c.drafter};
+        for (const dflash_model_cfg *m : ms) {
+            if (m->n_experts > 0) { why = "FP8 weights need dense models"; return false; }
+            if (m->hidden % 16 || m->ffn % 16 || (m->n_q_heads * m->head_dim) % 16) {
+                why = "FP8 weights need hidden, ffn and q width multiples of 16";
+                return false;
+            }
+        }
+    }
     return true;
+}
+
+static void add_slot(Layout &L, const std::string &name, int ndim, int64_t d0, int64_t d1, int64_t d2, int dtype);
+
+// A projection matrix [d0, d1]; FP8 storage adds "<name>.scale" [d0] (fp32, one per row).
+static void add_matrix(Layout &L, const std::string &name, int64_t d0, int64_t d1, int dtype) {
+    add_slot(L, name, 2, d0, d1, 0, dtype);
+    if (dtype == DFLASH_FP8) add_slot(L, name + ".scale", 1, d0, 0, 0, DFLASH_FP32);
 }
 
 static void add_slot(Layout &L, const std::string &name, int ndim, int64_t d0, int64_t d1, int64_t d2, int dtype) {
@@ -149,16 +168,16 @@ static void add_model_slots(Layout &L, const char *prefix, const dflash_model_cf
             add_slot(L, p + "q_norm", 1, m.head_dim, 0, 0, DFLASH_FP32);
             add_slot(L, p + "k_norm", 1, m.head_dim, 0, 0, DFLASH_FP32);
         }
-        add_slot(L, p + "wqkv", 2, qd + 2 * kd, H, 0, dt);
-        add_slot(L, p + "wo", 2, H, qd, 0, dt);
+        add_matrix(L, p + "wqkv", qd + 2 * kd, H, dt);
+        add_matrix(L, p + "wo", H, qd, dt);
         add_slot(L, p + "ffn_norm", 1, H, 0, 0, DFLASH_FP32);
         if (m.n_experts > 0) {
             add_slot(L, p + "w_router", 2, m.n_experts, H, 0, dt);
             add_slot(L, p + "we_gate_up", 3, m.n_experts, 2 * (int64_t)m.expert_ffn, H, dt);
             add_slot(L, p + "we_down", 3, m.n_experts, H, m.expert_ffn, dt);
         } else {
-            add_slot(L, p + "w_gate_up", 2, 2 * (int64_t)m.ffn, H, 0, dt);
-            add_slot(L, p + "w_down", 2, H, m.ffn, 0, dt);
+            add_matrix(L, p + "w_gate_up", 2 * (int64_t)m.ffn, H, dt);
+            add_matrix(L, p + "w_down", H, m.ffn, dt);
         }
     }
     add_slot(L, std::string(prefix) + ".final_norm", 1, H, 0, 0, DFLASH_FP32);
@@ -166,14 +185,16 @@ static void add_model_slots(Layout &L, const char *prefix, const dflash_model_cf
 
 static Layout make_layout(const dflash_config &c) {
     Layout L;
-    // weight storage: fp32 or bf16 (both bf16 activation modes store bf16 weights)
-    const int dt = c.dtype == DFLASH_FP32 ? DFLASH_FP32 : DFLASH_BF16, es = elem_size(dt);
+    // weight storage: fp32 or bf16 (both bf16 activation modes store bf16 weights);
+    // FP8: every projection matrix as E4M3 codes + row scales, the embedding in bf16
+    const int dt_emb = c.dtype == DFLASH_FP32 ? DFLASH_FP32 : DFLASH_BF16, es = elem_size(dt_emb);
+    const int dt = c.dtype == DFLASH_FP8 ? DFLASH_FP8 : dt_emb;
     const dflash_model_cfg &t = c.target, &d = c.drafter;
-    add_slot(L, "embed", 2, t.vocab, t.hidden, 0, dt);
-    add_slot(L, "lm_head", 2, t.vocab, t.hidden, 0, dt);
+    add_slot(L, "embed", 2, t.vocab, t.hidden, 0, dt_emb);
+    add_matrix(L, "lm_head", t.vocab, t.hidden, dt);
     add_model_slots(L, "target", t, dt);
     add_model_slots(L, "drafter", d, dt);
-    add_slot(L, "fuse.w_fc", 2, d.hidden, (int64_t)c.n_taps * t.hidden, 0, dt);
+    add_matrix(L, "fuse.w_fc", d.hidden, (int64_t)c.n_taps * t.hidden, dt);
     add_slot(L, "fuse.norm", 1, d.hidden, 0, 0, DFLASH_FP32);
     L.weight_bytes = align_up(L.weight_bytes, 256);
 
@@ -218,7 +239,7 @@ static Layout make_layout(const dflash_config &c) {
     L.xg_t = take((size_t)L.R_dec * H * es);
     L.xg2 = take((size_t)L.R_dec * H * es);
     const size_t act_bytes = align_up(o, 256) - act0;
-    if (c.dtype == DFLASH_BF16) {
+    if (c.dtype == DFLASH_BF16 || c.dtype == DFLASH_FP8) {
         take(act_bytes);
         L.act_lo = act_bytes / es;
     }
@@ -306,7 +327,11 @@ class Engine : public EngineBase {
     cudaStream_t s;
     char *W, *S;
     // weights
-    const T *embed, *lm_head, *w_fc;
+    const T *embed;
+    const void *lm_head, *w_fc;
+    // FP8 weights: the scale vector of every projection matrix, by its base address
+    bool f8_ = false;
+    std::unordered_map<const void *, const float *> wscales;
     const float *fc_norm, *t_final, *d_final;
     std::vector<LayerW> tl, dl;
     // state
@@ -325,6 +350,9 @@ class Engine : public EngineBase {
     int *gemm_sem;
     float2 *lm_part;
     AttnScratch att;
+    // TMA attention: K / V maps of the target (0) and the drafter (1) caches
+    CUtensorMap kv_map[2][2];
+    bool attn_tma_on = false;
     // folded-norm decode passes (bf16)
     T *xg_t = nullptr, *xg2 = nullptr;
     size_t lo_ = 0;  // low plane offset of two-plane activations (elements), 0: one plane
@@ -372,8 +400,14 @@ class Engine : public EngineBase {
 
     dflash_status init(const std::unordered_map<std::string, int> &by) {
         embed = (const T *)wslot(by, "embed");
-        lm_head = (const T *)wslot(by, "lm_head");
-        w_fc = (const T *)wslot(by, "fuse.w_fc");
+        lm_head = wslot(by, "lm_head");
+        w_fc = wslot(by, "fuse.w_fc");
+        f8_ = c.dtype == DFLASH_FP8;
+        if (f8_)
+            for (const WeightSlot &sl : L.slots)
+                if (sl.name.size() > 6 && sl.name.compare(sl.name.size() - 6, 6, ".scale") == 0)
+                    wscales[W + L.slots[by.at(sl.name.substr(0, sl.name.size() - 6))].offset] =
+                        (const float *)(W + sl.offset);
         fc_norm = (const float *)wslot(by, "fuse.norm");
         t_final = (const float *)wslot(by, "target.final_norm");
         d_final = (const float *)wslot(by, "drafter.final_norm");
@@ -482,6 +516,21 @@ class Engine : public EngineBase {
         att.sem = sp<int>(L.att_sem);
         att.max_parts = L.att_parts;
         att.num_sms = num_sms;
+        if constexpr (std::is_same<T, bf16>::value) {
+            // DFLASH_ATTN=mma: the cluster-of-kv-heads mma.sync attention instead
+            const char *av = getenv("DFLASH_ATTN");
+            const bool legacy = av && strcmp(av, "mma") == 0;
+            const dflash_model_cfg *ms[2] = {&c.target, &c.drafter};
+            T *caches[2][2] = {{tk, tv}, {dk, dv}};
+            attn_tma_on = !legacy;
+            for (int w = 0; w < 2 && attn_tma_on; ++w) {
+                const dflash_model_cfg &m = *ms[w];
+                attn_tma_on = attn_tma_supported(m.head_dim, m.n_q_heads / m.n_kv_heads);
+                for (int kv = 0; kv < 2 && attn_tma_on; ++kv)
+                    attn_tma_on = attn_tma_make_map(&kv_map[w][kv], (const bf16 *)caches[w][kv], m.head_dim, c.max_len,
+                                                    c.max_batch * m.n_kv_heads, m.n_layers, kv_layer_elems(m), lo_);
+            }
+        }
         att.n_sem = std::max(L.R_dec, (L.C + 15) / 16) * std::max(c.target.n_kv_heads, c.drafter.n_kv_heads);
         h_len.assign(c.max_batch, 0);
         h_prefilled.assign(c.max_batch, 0);
@@ -528,9 +577,14 @@ class Engine : public EngineBase {
         return DFLASH_ECUDA;
     }
 
+    bool attn_failed = false;  // an attention launch was refused
     dflash_status check(const char *what) {
         if (tc.failed) {  // a projection could not be launched (tensor map encoding)
             err = std::string(what) + ": " + tc.err;
+            return DFLASH_ECUDA;
+        }
+        if (attn_failed) {
+            err = std::string(what) + ": attention launch failed";
             return DFLASH_ECUDA;
         }
         cudaError_t e = cudaGetLastError();
@@ -613,7 +667,9 @@ class Engine : public EngineBase {
     // activation input (both planes of two-plane activations) and the outputs
     double gemm_bytes(int M, int N, int K, const Epi<T> &e) const {
         const double es = sizeof(T), ea = es * (lo_ ? 2 : 1);
-        double b = (double)N * K * es + (double)M * K * ea;
+        const int wrows = e.kind == EPI_SWIGLU ? 2 * e.F : N;
+        double b = f8_ ? (double)wrows * K + 4.0 * wrows : (double)N * K * es;
+        b += (double)M * K * ea;
         switch (e.kind) {
             case EPI_QKV: b += (double)M * N * ea; break;
             case EPI_RESID:
@@ -628,20 +684,38 @@ class Engine : public EngineBase {
 
     // One projection; returns the CTAs launched (tensor-core path).  dep/done:
     // completion counters of a decode pass (see PassSync), else griddepcontrol.wait.
+    // FP8 weights: the row scales of matrix Wt (its base address; rows from row0 on)
+    const float *scales_of(const void *Wt, int row0 = 0) const {
+        if (!f8_) return nullptr;
+        auto it = wscales.find(Wt);
+        return it == wscales.end() ? nullptr : it->second + row0;
+    }
+    // matrix Wt from row row0 on (FP8 codes are one byte per element)
+    const void *rows_of(const void *Wt, int row0, int K) const {
+        return (const char *)Wt + (size_t)row0 * K * (f8_ ? 1 : sizeof(T));
+    }
+
     int gemm(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e, const int *dep = nullptr,
-             int dep_target = 0, int *done = nullptr) {
+             int dep_target = 0, int *done = nullptr, const float *ws = nullptr) {
         if (M <= 0) return 0;
         int ctas = 0;
+        if (!ws) ws = scales_of(Wt);
         timed(DFLASH_PROF_PROJECTION, gemm_bytes(M, N, K, e),
-              [&] { ctas = gemm_launch(X, ldx, M, Wt, N, K, e, dep, dep_target, done); }, proj_class(N, K, e.kind));
+              [&] { ctas = gemm_launch(X, ldx, M, Wt, N, K, e, dep, dep_target, done, ws); }, proj_class(N, K, e.kind));
         return ctas;
     }
 
     int gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e_in,
-                    const int *dep = nullptr, int dep_target = 0, int *done = nullptr) {
+                    const int *dep = nullptr, int dep_target = 0, int *done = nullptr, const float *ws = nullptr) {
         Epi<T> e = e_in;
         e.lo = lo_;  // every input and output of the engine's projections lives in the activation span
-        if (tc.supports(M, N, K)) return tc.run(X, ldx, M, (const T *)Wt, N, K, e, s, dep, dep_target, done);
+        if (f8_ && !ws) ws = scales_of(Wt);
+        if (f8_ && !ws) {  // an FP8 matrix without its scales: refuse rather than read codes as bf16
+            tc.failed = true;
+            tc.err = "FP8 matrix without row scales";
+            return 0;
+        }
+        if (tc.supports(M, N, K)) return tc.run(X, ldx, M, Wt, N, K, e, s, dep, dep_target, done, ws);
         // CUDA-core path (fp32 models): GEMM into fp32 Y, then the epilogue.
         float *Yo = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.Y : Y;
         const int ldy = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.ldy : N;
@@ -664,12 +738,46 @@ class Engine : public EngineBase {
     }
 
     // returns the CTAs launched by the tensor-core attention (0 on the CUDA-core path)
-    int attention(const T *qq, const T *kc, const T *vc, const RowMeta *mt, int R, int rows_per_tile,
-                  const dflash_model_cfg &m, T *out, const AttnSync &sy = AttnSync()) {
+    // Query rows per attention tile for blocks of B rows: the attention kernels
+    // take at most 16 rows of one sequence per tile, so larger blocks split into
+    // equal tiles (the largest divisor of B that is at most 16).
+    static int block_tile_rows(int B) {
+        for (int t = std::min(B, 16); t > 1; --t)
+            if (B % t == 0) return t;
+        return 1;
+    }
+
+    // attention of layer `layer` of the target (which = 0) or the drafter (1)
+    int attention(int which, int layer, const T *qq, const RowMeta *mt, int R, int rows_per_tile, T *out,
+                  const AttnSync &sy = AttnSync()) {
+        const dflash_model_cfg &m = which ? c.drafter : c.target;
+        const T *kc = (which ? dk : tk) + (size_t)layer * kv_layer_elems(m);
+        const T *vc = (which ? dv : tv) + (size_t)layer * kv_layer_elems(m);
         const int qd = m.n_q_heads * m.head_dim;
         int ctas = 0;
         timed(DFLASH_PROF_ATTENTION, 0.0, [&] {
-            if (attn_mma_supported<T>(m.head_dim))
+            if (attn_tma_on && !sy.dep_ctr && !sy.done_ctr) {
+                if constexpr (std::is_same<T, bf16>::value) {
+                    AttnTmaArgs a;
+                    a.q = (const bf16 *)qq;
+                    a.ldq = qd;
+                    a.meta = mt;
+                    a.R = R;
+                    a.rows_per_tile = rows_per_tile;
+                    a.nq = m.n_q_heads;
+                    a.nkv = m.n_kv_heads;
+                    a.max_len = c.max_len;
+                    a.layer = layer;
+                    a.scale_log2 = 1.4426950408889634f / sqrtf((float)m.head_dim);
+                    a.out = (bf16 *)out;
+                    a.ldo = qd;
+                    a.lo = lo_;
+                    a.err = &stats->status;
+                    ctas = launch_attention_tma(kv_map[which][0], kv_map[which][1], a, m.head_dim, lo_ != 0, num_sms,
+                                                s);
+                    if (ctas < 0) attn_failed = true;
+                }
+            } else if (attn_mma_supported<T>(m.head_dim))
                 ctas = launch_attention_mma<T>(qq, qd, kc, vc, mt, R, rows_per_tile, m.n_q_heads, m.n_kv_heads,
                                                m.head_dim, c.max_len, out, qd, lo_, att, s, sy);
             else
@@ -708,7 +816,7 @@ class Engine : public EngineBase {
         e.kc = tk + (size_t)l * kv_layer_elems(m);
         e.vc = tv + (size_t)l * kv_layer_elems(m);
         gemm(xn, H, R, w.wqkv, qd + 2 * kd, H, with_qk_norm(e, m, w));
-        attention(q, e.kc, e.vc, mt, R, rpt, m, ao);
+        attention(0, l, q, mt, R, rpt, ao);
         Epi<T> r;
         r.kind = EPI_RESID;
         r.x = x;
@@ -789,7 +897,7 @@ class Engine : public EngineBase {
         e.vc = dv + (size_t)j * kv_layer_elems(m);
         // block rows and context rows share one pass over Wqkv (K/V injection)
         gemm(dq_in, H, with_ctx ? 2 * R : R, w.wqkv, qd + 2 * kd, H, with_qk_norm(e, m, w));
-        attention(q, e.kc, e.vc, meta, R, c.block_size, m, ao);
+        attention(1, j, q, meta, R, block_tile_rows(c.block_size), ao);
         Epi<T> r;
         r.kind = EPI_RESID;
         r.x = x;
@@ -1119,8 +1227,7 @@ class Engine : public EngineBase {
         for (int l = 0; l < t.n_layers; ++l) {
             int ai;
             const AttnSync sy = pass_attn_sync(pv, l, ai);
-            const int k = attention(q, tk + (size_t)l * kv_layer_elems(t), tv + (size_t)l * kv_layer_elems(t), meta, R,
-                                    B, t, ao, sy);
+            const int k = attention(0, l, q, meta, R, block_tile_rows(B), ao, sy);
             pass_done(pv, ai, k);
             run_ops(pv, 1 + 4 * l, 5 + 4 * l);
         }
@@ -1145,8 +1252,7 @@ class Engine : public EngineBase {
         for (int j = 0; j < d.n_layers; ++j) {
             int ai;
             const AttnSync sy = pass_attn_sync(pd, j, ai);
-            const int k = attention(q, dk + (size_t)j * kv_layer_elems(d), dv + (size_t)j * kv_layer_elems(d), meta, R,
-                                    B, d, ao, sy);
+            const int k = attention(1, j, q, meta, R, block_tile_rows(B), ao, sy);
             pass_done(pd, ai, k);
             run_ops(pd, 2 + 4 * j, 6 + 4 * j);
         }
@@ -1203,8 +1309,9 @@ class Engine : public EngineBase {
                 e.rope = rope_d;
                 e.kc = dk + (size_t)j * kv_layer_elems(d);
                 e.vc = dv + (size_t)j * kv_layer_elems(d);
-                const T *wkv = (const T *)dl[j].wqkv + (size_t)qd * H;
-                gemm(cbuf, H, R, wkv, 2 * kd, H, with_qk_norm(e, d, dl[j]));
+                // rows qd .. qd + 2kd of Wqkv are [Wk; Wv]
+                gemm(cbuf, H, R, rows_of(dl[j].wqkv, qd, H), 2 * kd, H, with_qk_norm(e, d, dl[j]), nullptr, 0, nullptr,
+                     scales_of(dl[j].wqkv, qd));
             }
         }
         launch_prefill_finish(st, seq, n, first_tok, out_tok, c.max_len, max_new, s);
@@ -1256,7 +1363,7 @@ class Engine : public EngineBase {
         const dflash_model_cfg &t = c.target;
         const int B = c.block_size, R = nseq * B, H = t.hidden, TK = c.n_taps * H;
         launch_embed_block<T>(embed, H, st, active, nseq, B, 0, drafts, c.mask_token_id, x, meta, nullptr, s);
-        for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, B, meta, taps_dec, TK);
+        for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, block_tile_rows(B), meta, taps_dec, TK);
         if (sampling_on()) {
             const SampleRows a = sample_desc(logits, R, B, 0, SP_TARGET, 1, tok_p, lse_p);
             lm_head_rows(t_final, (float)t.rms_eps, R, logits, 0, B, tok_p, &a);
@@ -1725,9 +1832,10 @@ class Engine : public EngineBase {
         if (which < 2 && fold_used[which]) {
             // folded passes feed the head bf16(x * g_final) and scale each row by its RMSNorm factor
             const float eps = (float)(which == 0 ? c.drafter.rms_eps : c.target.rms_eps);
-            ctas = gemm_launch(xg_t, H, rows, lm_head, V, H, epi_norm_in(e, eps, H));
+            ctas = gemm_launch(xg_t, H, rows, lm_head, V, H, epi_norm_in(e, eps, H), nullptr, 0, nullptr,
+                               scales_of(lm_head));
         } else {
-            ctas = gemm_launch(xn, H, rows, lm_head, V, H, e);
+            ctas = gemm_launch(xn, H, rows, lm_head, V, H, e, nullptr, 0, nullptr, scales_of(lm_head));
         }
         tc.lm_part = saved_part;
         tc.keep_logits = saved_keep;

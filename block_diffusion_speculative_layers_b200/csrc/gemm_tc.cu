@@ -44,21 +44,67 @@ namespace tc {
 // A 1-D grid smaller than the tile count makes CTAs loop over tiles with two
 // TMEM accumulators (the epilogue of one tile overlapping the MMAs of the
 // next); the host policy does not use that form at present.
-template <int TM, int KIND>
+// FP8 weights (F8): the weight tile arrives as E4M3 codes, 128 rows x 128 K
+// (16 KB, one TMA box per 64 rows), half the bytes of bf16.  During the main
+// loop the four epilogue warps convert it -- thread = weight row -- to bf16
+// (exact: every E4M3 value is a bf16 value) and write it into tensor memory
+// with tcgen05.st; tcgen05.mma then reads the A operand from tensor memory and
+// the activation rows from shared memory as before.  Each weight row's fp32
+// scale multiplies its accumulator before the epilogue.  Rings: raw stages in
+// shared memory (codes + the activation tiles of the same 128 K), released by
+// the converters and the MMA commit together; A stages in tensor memory,
+// released by the MMA commit.
+
+// Two E4M3 codes (low byte first) -> two bf16 values, exactly: the codes go to
+// f16 with the hardware conversion (exact), then each f16 half, always normal
+// or zero here, moves to bf16 by rebiasing the exponent (15 -> 127) and
+// dropping three mantissa bits that are zero.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t c) {
+    uint32_t f;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f) : "h"(c));
+    const uint32_t t = (f >> 3) & 0x0FFF0FFFu;       // exponent and 7 mantissa bits of each half
+    const uint32_t nz = __vcmpne2(t, 0u);            // 0xFFFF for nonzero halves
+    return ((t + 0x38003800u) & nz) | (f & 0x80008000u);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// bf16 x bf16 -> fp32 with the A operand (128 x 16) in tensor memory
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                                uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+template <int TM, int KIND, bool F8>
 __global__ void __launch_bounds__(NT, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcParams p,
                    Epi<bf16> e, int stages) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const int B_BYTES = TM * 128 * p.planes;  // activation tile(s) of one stage
+    const int B_BYTES = TM * 128 * p.planes;  // activation tile(s) of 64 K
+    // F8 stages cover 128 K: 16 KB of codes and two activation tiles
+    const int A_ST = F8 ? F8_A_BYTES : A_BYTES, B_ST = F8 ? 2 * B_BYTES : B_BYTES;
     // two planes and TM <= 128: one MMA with N = 2*TM covers the hi and lo rows
     // (they are contiguous in the stage), accumulating into 2*TM columns
     const bool wide = p.planes == 2 && TM <= 128;
     const int lo_col = wide ? TM : 0;
     const int NC1 = max(32, wide ? 2 * TM : TM);  // TMEM columns of one accumulator
     uint8_t *sA = smem;
-    uint8_t *sB = smem + (size_t)stages * A_BYTES;
-    float *stg = (float *)(sB + (size_t)stages * B_BYTES);
+    uint8_t *sB = smem + (size_t)stages * A_ST;
+    float *stg = (float *)(sB + (size_t)stages * B_ST);
     float2 *red = (float2 *)(stg + 128 * STG_LD);
     RowMeta *smeta = (RowMeta *)(red + 4 * CH);
     float *rsc = (float *)(smeta + CH);       // [RS_MAX] row scales of the folded norm
@@ -66,7 +112,9 @@ __global__ void __launch_bounds__(NT, 1)
     uint64_t *empty = full + stages;
     uint64_t *acc_full = empty + stages;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
-    uint32_t *tmem_slot = (uint32_t *)(acc_empty + 2);
+    uint64_t *a_conv = acc_empty + 2;      // [F8_ASTAGES] A stage converted into tensor memory
+    uint64_t *a_free = a_conv + F8_ASTAGES;  // [F8_ASTAGES] A stage read by the MMAs
+    uint32_t *tmem_slot = (uint32_t *)(a_free + F8_ASTAGES);
     // split-K receive buffer [S][128][cpr] (16-byte aligned, after the fixed area)
     float *recv = (float *)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
     EpiIn pre;
@@ -77,24 +125,29 @@ __global__ void __launch_bounds__(NT, 1)
     const int n_tiles_total = p.n_tiles * p.m_tiles;
     // one tile per CTA: (blockIdx.x, blockIdx.y); a persistent launch would pass
     // a 1-D grid smaller than the tile count and stride over the tiles
-    const bool persistent = !split && gridDim.y == 1 && (int)gridDim.x < n_tiles_total;
+    const bool persistent = !F8 && !split && gridDim.y == 1 && (int)gridDim.x < n_tiles_total;
     const int tile0 = persistent ? blockIdx.x : blockIdx.y * p.n_tiles + blockIdx.x;
     const int tstride = persistent ? gridDim.x : n_tiles_total;
     const int k_per = (p.k_steps + S - 1) / S;
     const int kb = split ? blockIdx.z * k_per : 0;
     const int ke = split ? min(p.k_steps, kb + k_per) : p.k_steps;
     const int nk = max(0, ke - kb);
-    const int ncols = persistent ? 2 * NC1 : NC1;  // persistent CTAs double-buffer the accumulator
+    const int a_cols = F8 ? F8_ASTAGES * 64 : 0;  // tensor-memory A stages (64 columns = 128 bf16 K each)
+    const int ncols = tmem_cols_for((persistent ? 2 * NC1 : NC1) + a_cols);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], F8 ? 5 : 1);  // F8: four converter warps + the MMA commit
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
         mbar_init(&acc_empty[0], 4);
         mbar_init(&acc_empty[1], 4);
+        for (int s = 0; s < F8_ASTAGES; ++s) {
+            mbar_init(&a_conv[s], 4);
+            mbar_init(&a_free[s], 1);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -107,6 +160,7 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_a = tmem + (uint32_t)(persistent ? 2 * NC1 : NC1);  // F8: A stages after the accumulator
     // K split: every CTA of the cluster has started before any pushes into another's
     // shared memory (arrive now; the epilogue warps wait before their first push)
     if (split) cluster_arrive_relaxed();
@@ -116,6 +170,14 @@ __global__ void __launch_bounds__(NT, 1)
         if (lane == 0) {
             // ---------------- TMA producer: one continuous ring over all tiles of this CTA ----------------
             const uint64_t wpol = l2_evict_first_policy();
+            const int kstep = F8 ? 2 * BK : BK;  // K elements per stage
+            auto load_x = [&](int s, int k, int m0) {
+                for (int h = 0; h < (F8 ? 2 : 1); ++h) {
+                    uint8_t *b = sB + (size_t)s * B_ST + h * B_BYTES;
+                    if (p.planes == 2) tma_load_3d(b, &tmX, k + h * BK, m0, 0, &full[s]);
+                    else tma_load_2d(b, &tmX, k + h * BK, m0, &full[s]);
+                }
+            };
             int it = 0;     // global stage counter
             bool first = true, abort = false;
             for (int t = tile0; t < n_tiles_total && !abort; t += tstride) {
@@ -128,16 +190,13 @@ __global__ void __launch_bounds__(NT, 1)
                     // weights do not depend on the previous kernel: start streaming them first
                     const int pre = min(nk, stages);
                     for (int i = 0; i < pre; ++i) {
-                        uint8_t *a = sA + (size_t)i * A_BYTES;
-                        mbar_expect_tx(&full[i], A_BYTES + B_BYTES);
-                        tma_load_2d_hint(a, &tmW, (kb + i) * BK, rowA0, &full[i], wpol);
-                        tma_load_2d_hint(a + A_BYTES / 2, &tmW, (kb + i) * BK, rowA1, &full[i], wpol);
+                        uint8_t *a = sA + (size_t)i * A_ST;
+                        mbar_expect_tx(&full[i], A_ST + B_ST);
+                        tma_load_2d_hint(a, &tmW, (kb + i) * kstep, rowA0, &full[i], wpol);
+                        tma_load_2d_hint(a + A_ST / 2, &tmW, (kb + i) * kstep, rowA1, &full[i], wpol);
                     }
                     dep_wait(p.dep_ctr, p.dep_target, p.err);
-                    for (int i = 0; i < pre; ++i) {
-                        if (p.planes == 2) tma_load_3d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, 0, &full[i]);
-                        else tma_load_2d(sB + (size_t)i * B_BYTES, &tmX, (kb + i) * BK, m0, &full[i]);
-                    }
+                    for (int i = 0; i < pre; ++i) load_x(i, (kb + i) * kstep, m0);
                     kk0 = pre;
                     it = pre;
                     first = false;
@@ -148,13 +207,12 @@ __global__ void __launch_bounds__(NT, 1)
                         abort = true;
                         break;
                     }
-                    const int k = (kb + kk) * BK;
-                    uint8_t *a = sA + (size_t)s * A_BYTES;
-                    mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
+                    const int k = (kb + kk) * kstep;
+                    uint8_t *a = sA + (size_t)s * A_ST;
+                    mbar_expect_tx(&full[s], A_ST + B_ST);
                     tma_load_2d_hint(a, &tmW, k, rowA0, &full[s], wpol);
-                    tma_load_2d_hint(a + A_BYTES / 2, &tmW, k, rowA1, &full[s], wpol);
-                    if (p.planes == 2) tma_load_3d(sB + (size_t)s * B_BYTES, &tmX, k, m0, 0, &full[s]);
-                    else tma_load_2d(sB + (size_t)s * B_BYTES, &tmX, k, m0, &full[s]);
+                    tma_load_2d_hint(a + A_ST / 2, &tmW, k, rowA1, &full[s], wpol);
+                    load_x(s, k, m0);
                 }
             }
         }
@@ -171,22 +229,43 @@ __global__ void __launch_bounds__(NT, 1)
                 const uint32_t acc = tmem + (uint32_t)(b * NC1);
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const int s = it % stages;
-                    if (!mbar_wait(&full[s], (it / stages) & 1, p.err)) {
-                        ok = false;
-                        break;
-                    }
-                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                    const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_BYTES));
-                    const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_BYTES));
+                    if constexpr (F8) {
+                        const int sa = it % F8_ASTAGES;
+                        if (!mbar_wait(&a_conv[sa], (it / F8_ASTAGES) & 1, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                        const uint32_t ta = tmem_a + (uint32_t)(sa * 64);
 #pragma unroll
-                    for (int k4 = 0; k4 < BK / 16; ++k4) {  // +32 bytes per K=16 step inside the swizzle row
-                        mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)(k4 * 2), idesc,
-                                 (kk > 0 || k4 > 0) ? 1u : 0u);
-                        if (p.planes == 2 && !wide)  // lo plane: TM rows (TM*128 bytes, a multiple of 1024) further on
-                            mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)((TM * 128) >> 4) + (uint64_t)(k4 * 2),
-                                     idesc, 1u);
+                        for (int k8 = 0; k8 < 8; ++k8) {  // 8 x K=16 over the stage's 128 K
+                            const uint64_t db =
+                                sw128_desc(smem_u32(sB + (size_t)s * B_ST + (k8 >> 2) * B_BYTES)) + (uint64_t)((k8 & 3) * 2);
+                            mma_bf16_tmem_a(acc, ta + (uint32_t)(k8 * 8), db, idesc, (kk > 0 || k8 > 0) ? 1u : 0u);
+                            if (p.planes == 2 && !wide)
+                                mma_bf16_tmem_a(acc, ta + (uint32_t)(k8 * 8), db + (uint64_t)((TM * 128) >> 4), idesc,
+                                                1u);
+                        }
+                        mma_commit(&empty[s]);
+                        mma_commit(&a_free[sa]);
+                    } else {
+                        if (!mbar_wait(&full[s], (it / stages) & 1, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                        const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_BYTES));
+                        const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_BYTES));
+#pragma unroll
+                        for (int k4 = 0; k4 < BK / 16; ++k4) {  // +32 bytes per K=16 step inside the swizzle row
+                            mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)(k4 * 2), idesc,
+                                     (kk > 0 || k4 > 0) ? 1u : 0u);
+                            if (p.planes == 2 && !wide)  // lo plane: TM rows (TM*128 bytes, a multiple of 1024) further on
+                                mma_bf16(acc, da + (uint64_t)(k4 * 2), db + (uint64_t)((TM * 128) >> 4) + (uint64_t)(k4 * 2),
+                                         idesc, 1u);
+                        }
+                        mma_commit(&empty[s]);
                     }
-                    mma_commit(&empty[s]);
                 }
                 mma_commit(&acc_full[b]);
             }
@@ -201,6 +280,15 @@ __global__ void __launch_bounds__(NT, 1)
         }
         const int q = warp & 3;
         const int n_local = q * 32 + lane;
+        // F8: this thread's weight row and its scale
+        float wsc = 1.f;
+        if constexpr (F8) {
+            const int nt0 = tile0 % p.n_tiles;
+            const int row = p.swiglu_F ? (n_local < 64 ? nt0 * 64 + n_local : p.swiglu_F + nt0 * 64 + n_local - 64)
+                                       : nt0 * 128 + n_local;
+            const int rows = p.swiglu_F ? 2 * p.swiglu_F : p.N;
+            wsc = row < rows ? p.w_scale[row] : 0.f;
+        }
         // K split: CTA `rank` of the cluster reduces and finishes columns [c_begin, c_end)
         const int rank = split ? (int)cluster_rank() : 0;
         const int cpr = split ? split_cols(TM, S) : TM;
@@ -216,6 +304,43 @@ __global__ void __launch_bounds__(NT, 1)
             }
             // inputs of this CTA's first epilogue chunk, while the mainloop streams
             if (c_end > c_begin) epi_prefetch<KIND, CH>(p, e, nt, n_local, mt * TM + c_begin, min(CH, c_end - c_begin), pre, smeta);
+            if constexpr (F8) {
+                // ---- convert the weight stages into tensor memory (thread = weight row n_local) ----
+                const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+                const int rr = n_local & 63;                       // row within its 64-row box
+                bool dead = false;
+                for (int kk = 0; kk < nk; ++kk) {
+                    const int s = kk % stages, sa = kk % F8_ASTAGES;
+                    if (!dead && !mbar_wait(&full[s], (kk / stages) & 1, p.err)) dead = true;
+                    if (!dead && kk >= F8_ASTAGES && !mbar_wait(&a_free[sa], ((kk / F8_ASTAGES) - 1) & 1, p.err))
+                        dead = true;
+                    const uint8_t *row = sA + (size_t)s * A_ST + (n_local >> 6) * (A_ST / 2) + rr * 128;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {  // 64 K per tcgen05.st of 32 columns
+                        uint32_t w[32];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int chunk = h * 4 + c;  // 16 codes = K 16*chunk .. +15, 128-byte swizzle
+                            const uint4 v = dead ? make_uint4(0, 0, 0, 0)
+                                                 : *reinterpret_cast<const uint4 *>(row + (((chunk ^ rr) & 7) << 4));
+                            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
+                                w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
+                            }
+                        }
+                        tmem_st32(tmem_a + lane_base + (uint32_t)(sa * 64 + h * 32), w);
+                    }
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&a_conv[sa]);
+                        mbar_arrive(&empty[s]);
+                    }
+                }
+            }
             const uint32_t trow = tmem + (uint32_t)(b * NC1) + ((uint32_t)(q * 32) << 16);
             const bool ok = mbar_wait(&acc_full[b], (lt >> 1) & 1, p.err) && nk > 0;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -226,6 +351,9 @@ __global__ void __launch_bounds__(NT, 1)
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
+                    if (F8)
+#pragma unroll
+                        for (int j = 0; j < CH; ++j) v[j] *= wsc;
                     if (c == TM - CH || TM == CH) {
                         // accumulator fully read: hand it back to the MMA warp
                         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -246,6 +374,9 @@ __global__ void __launch_bounds__(NT, 1)
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
+                    if (F8)
+#pragma unroll
+                        for (int j = 0; j < CH; ++j) v[j] *= wsc;
 #pragma unroll
                     for (int g = 0; g < CH / 4; ++g) {
                         const int col = c + 4 * g, owner = col / cpr;
@@ -412,24 +543,27 @@ int GemmTC<T>::init(float *w, int wf, int *sm, int ns) {
 
 template <typename T>
 const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows,
-                                         size_t plane_stride) {
+                                         size_t plane_stride, bool fp8) {
     char key[128];
-    snprintf(key, sizeof key, "%p/%d/%d/%d/%d/%zu", ptr, rows, cols, ld, box_rows, plane_stride);
+    snprintf(key, sizeof key, "%p/%d/%d/%d/%d/%zu/%d", ptr, rows, cols, ld, box_rows, plane_stride, fp8 ? 1 : 0);
     auto it = maps.find(key);
     if (it != maps.end()) return &it->second;
     if (maps.size() > 4096) maps.clear();
     CUtensorMap m;
     memset(&m, 0, sizeof m);
     const cuuint32_t rank = plane_stride ? 3 : 2;
+    const size_t es = fp8 ? 1 : sizeof(bf16);
     cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, 2};
-    cuuint64_t strides[2] = {(cuuint64_t)ld * sizeof(bf16), (cuuint64_t)plane_stride * sizeof(bf16)};
-    cuuint32_t box[3] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows, 2};
+    cuuint64_t strides[2] = {(cuuint64_t)ld * es, (cuuint64_t)plane_stride * es};
+    // one 128-byte swizzle row per box row: 64 bf16 or 128 FP8 codes
+    cuuint32_t box[3] = {(cuuint32_t)(fp8 ? 2 * tc::BK : tc::BK), (cuuint32_t)box_rows, 2};
     cuuint32_t estr[3] = {1, 1, 1};
     if (plane_stride && (plane_stride * sizeof(bf16)) % 16) {
         err = "lo-plane offset is not a multiple of 16 bytes";
         return nullptr;
     }
-    CUresult r = get_encode()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims, strides, box,
+    CUresult r = get_encode()(&m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                              const_cast<void *>(ptr), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -439,34 +573,36 @@ const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, in
     return &(maps[key] = m);
 }
 
-template <int TM, int KIND>
+template <int TM, int KIND, bool F8>
 static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p, const Epi<bf16> &e,
                       int stages, size_t smem, cudaStream_t s, int grid_x) {
-    auto kern = tc::gemm_tc_kernel<TM, KIND>;
+    auto kern = tc::gemm_tc_kernel<TM, KIND, F8>;
     ensure_smem_attr((const void *)kern);
     (void)grid_x;
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
     launch_k(kern, grid, dim3(tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
 }
 
-template <int TM>
+template <int TM, bool F8>
 static void launch_kind(int kind, const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p,
                         const Epi<bf16> &e, int stages, size_t smem, cudaStream_t s, int gx) {
     switch (kind) {
-        case EPI_STORE: launch_tm<TM, EPI_STORE>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_QKV: launch_tm<TM, EPI_QKV>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_RESID: launch_tm<TM, EPI_RESID>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_SWIGLU: launch_tm<TM, EPI_SWIGLU>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_NORMOUT: launch_tm<TM, EPI_NORMOUT>(mw, mx, p, e, stages, smem, s, gx); break;
-        default: launch_tm<TM, EPI_LOGITS>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_STORE: launch_tm<TM, EPI_STORE, F8>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_QKV: launch_tm<TM, EPI_QKV, F8>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_RESID: launch_tm<TM, EPI_RESID, F8>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_SWIGLU: launch_tm<TM, EPI_SWIGLU, F8>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_NORMOUT: launch_tm<TM, EPI_NORMOUT, F8>(mw, mx, p, e, stages, smem, s, gx); break;
+        default: launch_tm<TM, EPI_LOGITS, F8>(mw, mx, p, e, stages, smem, s, gx); break;
     }
 }
 
 template <>
-int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int K, const Epi<bf16> &e,
-                      cudaStream_t s, const int *dep_ctr, int dep_target, int *done_ctr) {
+int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K, const Epi<bf16> &e,
+                      cudaStream_t s, const int *dep_ctr, int dep_target, int *done_ctr, const float *w_scale) {
     const bool swiglu = e.kind == EPI_SWIGLU;
+    const bool f8 = w_scale != nullptr;
     int TM = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    if (f8) TM = std::min(TM, 64);  // FP8: tensor memory holds the A stages too; larger M takes several row tiles
     TcParams p;
     memset(&p, 0, sizeof p);
     p.M = M;
@@ -475,11 +611,14 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int K
     p.swiglu_F = swiglu ? e.F : 0;
     p.n_tiles = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
     p.m_tiles = (M + TM - 1) / TM;
-    p.k_steps = (K + tc::BK - 1) / tc::BK;
+    const int kstep = f8 ? 2 * tc::BK : tc::BK;  // K per stage: 128 FP8 codes or 64 bf16 values per weight row
+    p.k_steps = (K + kstep - 1) / kstep;
     const int tiles = p.n_tiles * p.m_tiles;
     p.planes = e.lo ? 2 : 1;
-    const int stage_bytes = tc::A_BYTES + TM * 128 * p.planes;
-    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64;
+    p.w_scale = w_scale;
+    const int stage_bytes = f8 ? tc::F8_A_BYTES + 2 * TM * 128 * p.planes : tc::A_BYTES + TM * 128 * p.planes;
+    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
+                      2 * tc::F8_ASTAGES * 8;
     // Measured on B200 (decode shapes, M = 16, whole decode iteration): every
     // projection streams best with ~110 KB CTAs, two of which fit on an SM;
     // projections with fewer tiles than that split K over a cluster (up to 8
@@ -511,25 +650,33 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const bf16 *W, int N, int K
     p.dep_target = dep_target;
     p.done_ctr = done_ctr;
     const int grid_x = p.n_tiles;  // one tile per CTA
-    const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64);
+    const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64, 0, f8);
     const CUtensorMap *mx = tensor_map(X, M, K, ldx, TM, e.lo);
     if (!mw || !mx) {
         failed = true;
         return 0;
     }
-    switch (TM) {
-        case 16: launch_kind<16>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-        case 32: launch_kind<32>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-        case 64: launch_kind<64>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-        case 128: launch_kind<128>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-        default: launch_kind<256>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+    if (f8) {
+        switch (TM) {
+            case 16: launch_kind<16, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            case 32: launch_kind<32, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            default: launch_kind<64, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+        }
+    } else {
+        switch (TM) {
+            case 16: launch_kind<16, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            case 32: launch_kind<32, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            case 64: launch_kind<64, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            case 128: launch_kind<128, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            default: launch_kind<256, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+        }
     }
     return p.n_tiles * p.m_tiles * p.splits;
 }
 
 template <>
-int GemmTC<float>::run(const float *, int, int, const float *, int, int, const Epi<float> &, cudaStream_t,
-                       const int *, int, int *) {
+int GemmTC<float>::run(const float *, int, int, const void *, int, int, const Epi<float> &, cudaStream_t,
+                       const int *, int, int *, const float *) {
     return 0;
 }
 

@@ -37,6 +37,7 @@ struct TcParams {
     const int *dep_ctr;
     int dep_target;
     int *done_ctr;
+    const float *w_scale;   // FP8 weights: fp32 scale of every weight row (the codes' row of W)
 };
 
 template <typename T>
@@ -45,9 +46,12 @@ struct GemmTC {
     bool failed = false;  // a launch was dropped (tensor map encoding failed); err says why
     bool supports(int M, int N, int K) const;
     int init(float *ws, int ws_floats, int *sem, int n_sem);
-    // returns the number of CTAs launched (the count a completion counter reaches per run)
-    int run(const T *X, int ldx, int M, const T *W, int N, int K, const Epi<T> &e, cudaStream_t s,
-            const int *dep_ctr = nullptr, int dep_target = 0, int *done_ctr = nullptr);
+    // returns the number of CTAs launched (the count a completion counter reaches per run).
+    // W: bf16 [N][K], or with w_scale != nullptr FP8 E4M3 codes [N][K] (one byte each)
+    // whose row n stands for w_scale[n] * code value.
+    int run(const T *X, int ldx, int M, const void *W, int N, int K, const Epi<T> &e, cudaStream_t s,
+            const int *dep_ctr = nullptr, int dep_target = 0, int *done_ctr = nullptr,
+            const float *w_scale = nullptr);
     // LM-head partial argmax buffer (value, index as float bits), [n_tiles][rows]
     void set_lm_part(float2 *p, int cap) { lm_part = p; lm_cap = cap; }
     void set_err(int *e) { err_word = e; }
@@ -67,7 +71,8 @@ struct GemmTC {
     // 2-D map of a [rows][cols] bf16 matrix (leading dimension ld), box {64, box_rows};
     // plane_stride > 0: 3-D map over the hi plane and the lo plane plane_stride
     // elements after it, box {64, box_rows, 2}
-    const CUtensorMap *tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows, size_t plane_stride = 0);
+    const CUtensorMap *tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows, size_t plane_stride = 0,
+                                  bool fp8 = false);
 };
 
 // Row-wise argmax over the LM-head partials: mode 0 idx[r]; mode 1 drafter rows.

@@ -12,6 +12,11 @@ namespace tc {
 
 constexpr int BK = 64;                 // bf16 K elements per stage = one 128-byte swizzle row
 constexpr int A_BYTES = 128 * BK * 2;  // 16 KB weight tile per stage
+constexpr int F8_A_BYTES = 128 * 128;  // FP8 weights: 128 rows x 128 codes per stage
+constexpr int F8_ASTAGES = 2;          // FP8 weights: bf16 A stages in tensor memory (64 columns each)
+
+// tensor-memory columns to allocate for n used columns: a power of two >= 32
+__host__ __device__ constexpr int tmem_cols_for(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 constexpr int NT = 192;
 constexpr int CH = 16;                 // accumulator columns per epilogue chunk
 constexpr int STG_LD = CH + 1;

@@ -64,8 +64,15 @@ typedef enum {
  * two (attention: three) MMAs and the result keeps ~16 significant bits --
  * weight bytes are unchanged, activation and K/V bytes double.  BF16_FAST:
  * bf16 weights and single-plane bf16 activations (half the K/V bytes and MMAs,
- * with the rounding error of plain bf16 inference). */
-enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1, DFLASH_BF16_FAST = 2 };
+ * with the rounding error of plain bf16 inference).  FP8: every projection
+ * matrix (Wqkv, Wo, gate/up, down, the LM head, the fuse W_fc) stored as E4M3
+ * codes (1 byte; OCP 8-bit float, exponent bias 7, no infinities) with one fp32
+ * scale per output row in the slot "<name>.scale", the embedding in bf16,
+ * activations as for BF16; the model computed is the quantised one,
+ * W[r][k] = scale[r] * e4m3_value(code[r][k]), so the greedy output equals the
+ * quantised target's own greedy decoding.  Weight bytes per step halve.
+ * Dense models only (MoE targets: EINVAL). */
+enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1, DFLASH_BF16_FAST = 2, DFLASH_FP8 = 3 };
 
 /* Draft modes.  MODEL: drafts are the drafter's argmax.  SCRIPT: the drafter
  * still runs in full, then its drafts are replaced from a per-sequence token
@@ -76,7 +83,7 @@ enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1, DFLASH_BF16_FAST = 2 };
 enum { DFLASH_DRAFT_MODEL = 0, DFLASH_DRAFT_SCRIPT = 1 };
 
 #define DFLASH_MAX_TAPS 8
-#define DFLASH_MAX_BLOCK 16
+#define DFLASH_MAX_BLOCK 32
 
 typedef struct {
     int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
@@ -99,14 +106,14 @@ typedef struct {
 typedef struct {
     dflash_model_cfg target;      /* the model whose greedy output is reproduced */
     dflash_model_cfg drafter;     /* dense; drafter.vocab == target.vocab, same hidden */
-    int32_t block_size;           /* B in [1, 16]: anchor + (B-1) drafted tokens */
+    int32_t block_size;           /* B in [1, 32]: anchor + (B-1) drafted tokens */
     int32_t n_taps;               /* target layers whose outputs feed the context vector */
     int32_t tap_layers[DFLASH_MAX_TAPS];
     int32_t mask_token_id;        /* id embedded at block positions 1..B-1 */
     int32_t max_batch;            /* sequences held at once */
     int32_t max_len;              /* positions per sequence (prompt + generated + B) */
     int32_t prefill_chunk;        /* prompt rows per prefill pass (0: default 1024) */
-    int32_t dtype;                /* DFLASH_FP32, DFLASH_BF16 or DFLASH_BF16_FAST (see above) */
+    int32_t dtype;                /* DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST or DFLASH_FP8 (see above) */
     int32_t keep_logits;          /* 1: keep fp32 logits of the last draft/verify for dflash_debug_logits */
     int32_t timeout_ms;           /* host wait bound for synchronising calls (0: 600000) */
     int32_t sampling;             /* 1: hold the buffers temperature sampling needs (dflash_set_sampling);
@@ -163,8 +170,9 @@ void dflash_destroy(dflash_ctx *ctx);
 const char *dflash_last_error(const dflash_ctx *ctx);
 
 /* Weight tensors: names, shapes, storage.  Tensors are row-major and live at
- * byte `offset` of the weight arena.  Matrices use cfg.dtype storage, RMSNorm
- * gains are always fp32.  Names:
+ * byte `offset` of the weight arena.  Matrices use cfg.dtype storage (FP8:
+ * uint8 codes plus "<name>.scale" [rows] fp32; the embedding stays bf16),
+ * RMSNorm gains are always fp32.  Names:
  *   embed [V,H], lm_head [V,H] (both shared by the drafter),
  *   {target|drafter}.L{l}.attn_norm [H], .wqkv [(nq+2nkv)*hd, H] (rows Wq;Wk;Wv),
  *   .wo [H, nq*hd], .ffn_norm [H], .w_gate_up [2F, H] (rows W_gate;W_up),

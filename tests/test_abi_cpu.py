@@ -63,7 +63,7 @@ def test_workspace_size_matches_weight_count(lib):
 
 @pytest.mark.parametrize("mutate", [
     lambda c: c.with_(block_size=0),
-    lambda c: c.with_(block_size=17),
+    lambda c: c.with_(block_size=33),
     lambda c: c.with_(tap_layers=(0, 5)),
     lambda c: c.with_(mask_token_id=5000),
     lambda c: c.with_(target=replace(c.target, head_dim=96)),

@@ -1,0 +1,74 @@
+"""FP8 weight streaming on the GPU against the fp64 oracle of the quantised model.
+
+Every projection matrix (and the LM head and the fuse W_fc) is stored as E4M3
+codes with one fp32 scale per row (synthetic.fp8); the kernels stream the
+codes, widen them to bf16 in tensor memory and apply the row scales in the
+epilogue.  The oracle computes the same quantised model in fp64, so the same
+bars hold as for bf16 weights: logits within 3e-2, token ids equal outside
+oracle near-ties (margin < 0.05), integer results bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_diffusion_speculative_layers_b200 as dfl
+import oracle
+from synthetic import get_config, make_prompt, make_weight
+from synthetic.configs import shrink
+from synthetic.fast import make_weights_host
+
+from parity import build_pair, check_lossless_generate, replay, replay_forced
+from test_parity_gpu import tiny_cfg
+
+pytestmark = pytest.mark.gpu
+
+TOL, TIE = 3e-2, 0.05
+
+
+@pytest.mark.parametrize("case", ["block4", "block16", "wide", "batch3", "chunked"])
+def test_fp8_tiny_replay(cuda_device, case):
+    kw = dict(dtype="fp8")
+    lens, chunk = [30], 0
+    if case in ("block16", "wide", "chunked"):
+        kw["block"] = 16
+    if case == "wide":  # K split across a cluster, several tiles per projection
+        kw.update(hidden=2048, nq=16, nkv=4, hd=128, vocab=8192)
+    if case == "batch3":
+        kw["block"] = 8
+        lens = [17, 40, 33]
+    if case == "chunked":
+        chunk, lens = 16, [45]
+    cfg = tiny_cfg(**kw)
+    gpu, spec, _ = build_pair(cfg, max_batch=len(lens), max_len=256, prefill_chunk=chunk)
+    prompts = [make_prompt("uniform", L, cfg.target.vocab, 60 + i) for i, L in enumerate(lens)]
+    rep = replay(gpu, spec, cfg, prompts, 5, TOL, TIE)
+    print(f"fp8 {case}: max |dlogit| {rep.max_dlogit:.2e}, near ties {rep.near_ties}/{rep.checked_tokens}")
+    assert rep.mismatches_outside_ties == 0, rep
+    assert rep.max_dlogit <= TOL
+
+
+def test_fp8_forced_acceptance_and_lossless_generation(cuda_device):
+    cfg = tiny_cfg("fp8", block=16)
+    gpu, spec, _ = build_pair(cfg, max_len=160)
+    prompt = make_prompt("uniform", 20, cfg.target.vocab, 70)
+    rep = replay_forced(gpu, spec, cfg, prompt, (15, 6, 0), TOL, TIE)
+    assert rep.mismatches_outside_ties == 0 and rep.max_dlogit <= TOL
+    k, st = check_lossless_generate(gpu, spec, cfg, make_prompt("uniform", 25, cfg.target.vocab, 71), 60, TIE)
+    assert st.tokens == 59
+
+
+def test_fp8_qwen3_8b_widths(cuda_device):
+    """The Qwen3-8B widths (hidden 4096, FFN 12288, vocab 151936) with FP8 weights:
+    two target layers and one drafter layer, two iterations."""
+    cfg = shrink(get_config("qwen3_8b"), target_layers=2, drafter_layers=1).with_(dtype="fp8")
+    gpu = dfl.DFlash(cfg, max_batch=1, max_len=128, keep_logits=True)
+    try:
+        gpu.load_weights_from(lambda n: make_weight(cfg, n, device="cuda"))
+        spec = oracle.OracleSpec(cfg, make_weights_host(cfg))
+        rep = replay(gpu, spec, cfg, [make_prompt("zipf", 24, cfg.target.vocab, cfg.seed)], 2, TOL, TIE)
+        print(f"fp8 qwen widths: max |dlogit| {rep.max_dlogit:.2e}, near ties {rep.near_ties}/{rep.checked_tokens}")
+        assert rep.mismatches_outside_ties == 0, rep
+        assert rep.max_dlogit <= TOL
+    finally:
+        gpu.close()
+        torch.cuda.empty_cache()

@@ -320,3 +320,21 @@ def test_fidelity_toggles_replay(cuda_device, dtype, toggle):
     rep = replay(gpu, spec, cfg, prompts, 4, tol, tie)
     print(f"{toggle} {dtype}: max |dlogit| {rep.max_dlogit:.2e}, near ties {rep.near_ties}/{rep.checked_tokens}")
     _finish(rep, tol)
+
+
+@pytest.mark.parametrize("block", [32, 24])
+def test_blocks_above_16_rows(cuda_device, block):
+    """Blocks of 32 and 24 positions (31 / 23 drafts): the attention tiles split
+    each block into 16- (or 12-) row tiles of one sequence; replay, forced full
+    and partial acceptance, and lossless generation against the oracle."""
+    cfg = tiny_cfg("bf16", block=block)
+    tol, tie = TOL["bf16"]
+    gpu, spec, _ = build_pair(cfg, max_batch=2, max_len=256)
+    prompts = [make_prompt("uniform", 20, cfg.target.vocab, 50), make_prompt("uniform", 33, cfg.target.vocab, 51)]
+    rep = replay(gpu, spec, cfg, prompts, 3, tol, tie)
+    _finish(rep, tol)
+    rep2 = replay_forced(gpu, spec, cfg, make_prompt("uniform", 17, cfg.target.vocab, 52), (block - 1, 9, 0), tol, tie,
+                         seq=1)
+    _finish(rep2, tol)
+    k, st = check_lossless_generate(gpu, spec, cfg, prompts[0], 60, tie)
+    assert st.tokens == 59
