@@ -40,7 +40,6 @@
 namespace dfl {
 namespace atm {
 
-constexpr int KT = 32;                   // keys per TMA tile
 constexpr int NCW = 4;                   // consumer warps
 constexpr int NTH = 32 * (NCW + 1);      // + one producer warp
 constexpr unsigned long long WAIT_NS = 2000000000ull;
@@ -81,13 +80,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, int *err
         for (int i = 0; i < 32; ++i)
             if (mbar_try(b, parity)) return true;
         if (gtimer() - t0 > WAIT_NS) {
-            if (err) atomicOr(err, 32);
+            if (err) atomicOr(err, 32);  // bit 5: an attention wait gave up
             return false;
         }
     }
 }
 
 // one box {64, KT, 1, 1, planes} of a 5-D (or {64, KT, 1, 1} of a 4-D) K/V map
+// (KT, the keys per tile, is the map's box height)
 __device__ __forceinline__ void tma_box(void *dst, const CUtensorMap *map, int d0, int key, int sh, int layer,
                                         bool five, uint64_t *bar) {
     if (five)
@@ -165,15 +165,18 @@ __device__ __forceinline__ void st_cluster_v4(float *local, uint32_t rank, float
                  : "memory");
 }
 
-// byte offset of (key, dim) in one swizzled box region [KT keys][64 dims] (128-byte
+// byte offset of (key, dim) in one swizzled box region [keys][64 dims] (128-byte
 // rows; 16-byte chunk c of row k stored at chunk c ^ (k & 7))
 __device__ __forceinline__ uint32_t swz(int key, int dim64) {
     return (uint32_t)(key * 128 + ((((dim64 >> 3) ^ key) & 7) << 4) + (dim64 & 7) * 2);
 }
 
 // Stage layout: [K box 0][K box 1][V box 0][V box 1], each box [planes][KT][128 B]
-// (dims 64*box .. 64*box+63), so one stage is 4 * planes * 4 KB.
-template <int HD, bool SPLIT, int HPC>
+// (dims 64*box .. 64*box+63).  Key group g consumes tiles g, g+G, ... so the
+// stage count is a multiple of G: each stage then always serves the same group,
+// which waits for every fill of it in order (an mbarrier tells two successive
+// phases apart only).
+template <int HD, bool SPLIT, int HPC, int KT>
 __global__ void __launch_bounds__(NTH, 2) attn_tma_kernel(const __grid_constant__ CUtensorMap tmK,
                                                        const __grid_constant__ CUtensorMap tmV, AttnTmaArgs a) {
     constexpr int PL = SPLIT ? 2 : 1;
@@ -523,7 +526,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool attn_tma_supported(int hd, int grp) { return (hd == 64 || hd == 128) && grp >= 1 && grp <= 8; }
 
 bool attn_tma_make_map(CUtensorMap *map, const bf16 *cache, int hd, int max_len, int n_seq_heads, int n_layers,
-                       size_t layer_elems, size_t lo) {
+                       size_t layer_elems, size_t lo, int kt) {
     auto enc = encode_fn();
     if (!enc || !cache) return false;
     memset(map, 0, sizeof *map);
@@ -531,7 +534,7 @@ bool attn_tma_make_map(CUtensorMap *map, const bf16 *cache, int hd, int max_len,
     cuuint64_t dims[5] = {(cuuint64_t)hd, (cuuint64_t)max_len, (cuuint64_t)n_seq_heads, (cuuint64_t)n_layers, 2};
     cuuint64_t strides[4] = {(cuuint64_t)hd * 2, (cuuint64_t)max_len * hd * 2, (cuuint64_t)layer_elems * 2,
                              (cuuint64_t)lo * 2};
-    cuuint32_t box[5] = {64, (cuuint32_t)atm::KT, 1, 1, 2};
+    cuuint32_t box[5] = {64, (cuuint32_t)kt, 1, 1, 2};
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     if ((lo * 2) % 16 || (layer_elems * 2) % 16) return false;
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<bf16 *>(cache), dims, strides, box, estr,
@@ -539,17 +542,31 @@ bool attn_tma_make_map(CUtensorMap *map, const bf16 *cache, int hd, int max_len,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static int attn_tma_hpc(int grp, int max_len) {
-    // one q head per CTA spreads short contexts over every SM (each q head's CTAs
-    // read the kv head's K/V, mostly from L2); long contexts share one K/V tile
-    // between the q heads of a kv head
-    if (max_len <= 4096) return 1;
+// q heads per CTA: one while the launch has fewer query tiles x kv heads than
+// SMs (decode of a few sequences: each q head's CTAs stream the kv head's K/V,
+// the copies after the first mostly from L2); the whole GQA group of a kv head
+// (up to 4 heads) once the tiles alone fill the GPU (prefill chunks, large
+// batches), so each K/V tile is read once for all of them
+int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms) {
+    if (n_tiles * nkv < num_sms) return 1;
     return grp % 4 == 0 ? 4 : grp % 2 == 0 ? 2 : 1;
+}
+// keys per tile: 16 when four key groups share the ring (its stages stay small),
+// 32 for one group
+int attn_tma_kt(int hpc) { return hpc == 4 ? 32 : 16; }
+
+static size_t attn_tma_stage(int hd, bool split, int kt) { return (size_t)2 * (hd / 64) * (split ? 2 : 1) * kt * 128; }
+
+// stages: a multiple of the key groups, as many as fit in ~100 KB (two CTAs per SM)
+static int attn_tma_stages(int hd, bool split, int hpc) {
+    const int G = atm::NCW / hpc;
+    const size_t st = attn_tma_stage(hd, split, attn_tma_kt(hpc));
+    const int k = std::max(1, (int)((100u << 10) / (st * G)));
+    return G * std::min(k, std::max(1, 4 / G));
 }
 
 static size_t attn_tma_smem(int hd, bool split, int hpc, int S, int stages) {
-    const int pl = split ? 2 : 1;
-    const size_t stage = (size_t)2 * (hd / 64) * pl * atm::KT * 128;
+    const size_t stage = attn_tma_stage(hd, split, attn_tma_kt(hpc));
     const int G = atm::NCW / hpc;
     const size_t combine = (size_t)G * hpc * 16 * (hd + 2) * 4;
     const size_t ring = std::max((size_t)stages * stage, combine);
@@ -560,23 +577,25 @@ static size_t attn_tma_smem(int hd, bool split, int hpc, int S, int stages) {
 template <int HD, bool SPLIT, int HPC>
 static cudaError_t launch_one(const CUtensorMap &mk, const CUtensorMap &mv, const AttnTmaArgs &a, int n_tiles,
                               cudaStream_t s) {
-    auto kern = atm::attn_tma_kernel<HD, SPLIT, HPC>;
+    constexpr int KT = HPC == 4 ? 32 : 16;
+    auto kern = atm::attn_tma_kernel<HD, SPLIT, HPC, KT>;
     ensure_smem_attr((const void *)kern);
     const size_t smem = attn_tma_smem(HD, SPLIT, HPC, a.n_splits, a.stages);
     return launch_k(kern, dim3(n_tiles, a.nq / HPC, a.n_splits), dim3(atm::NTH), smem, s, a.n_splits, mk, mv, a);
 }
 
-int launch_attention_tma(const CUtensorMap &mk, const CUtensorMap &mv, AttnTmaArgs a, int hd, bool split,
-                         int num_sms, cudaStream_t s) {
+int launch_attention_tma(const AttnTmaMaps &maps, AttnTmaArgs a, int hd, bool split, int num_sms, cudaStream_t s) {
     if (a.R <= 0) return 0;
     const int grp = a.nq / a.nkv;
-    const int hpc = attn_tma_hpc(grp, a.max_len);
     const int n_tiles = (a.R + a.rows_per_tile - 1) / a.rows_per_tile;
+    const int hpc = attn_tma_hpc(grp, n_tiles, a.nkv, num_sms);
+    const int kt = attn_tma_kt(hpc);
+    const CUtensorMap &mk = kt == 32 ? maps.k32 : maps.k16, &mv = kt == 32 ? maps.v32 : maps.v16;
     const int units = n_tiles * (a.nq / hpc);
     // splits of one (tile, head group) form a cluster of at most 8 CTAs; enough
-    // CTAs for two per SM, no more splits than 32-key tiles the longest context has
-    a.n_splits = std::max(1, std::min({8, (2 * num_sms + units - 1) / units, (a.max_len + atm::KT - 1) / atm::KT}));
-    a.stages = split ? 3 : 4;
+    // CTAs for two per SM, no more splits than key tiles the longest context has
+    a.n_splits = std::max(1, std::min({8, (2 * num_sms + units - 1) / units, (a.max_len + kt - 1) / kt}));
+    a.stages = attn_tma_stages(hd, split, hpc);
     cudaError_t e = cudaErrorInvalidValue;
 #define ATM_CASE(HD_, SP_, HPC_)                                                  \
     if (hd == HD_ && split == SP_ && hpc == HPC_) e = launch_one<HD_, SP_, HPC_>(mk, mv, a, n_tiles, s);

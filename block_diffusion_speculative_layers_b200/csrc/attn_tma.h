@@ -29,13 +29,21 @@ bool attn_tma_supported(int hd, int grp);
 
 // Tensor map of one model's K (or V) cache [layer][seq][kv head][max_len][hd]
 // viewed as (hd, position, seq * kv head, layer[, plane]): 4-D for one plane,
-// 5-D with the low plane `lo` elements on; box {64, 32, 1, 1[, 2]}, 128-byte
+// 5-D with the low plane `lo` elements on; box {64, kt, 1, 1[, 2]}, 128-byte
 // swizzle.  false if the driver cannot encode it.
 bool attn_tma_make_map(CUtensorMap *map, const bf16 *cache, int hd, int max_len, int n_seq_heads, int n_layers,
-                       size_t layer_elems, size_t lo);
+                       size_t layer_elems, size_t lo, int kt);
+
+// The K and V maps of one model's caches, with 16- and 32-key boxes.
+struct AttnTmaMaps {
+    CUtensorMap k16, v16, k32, v32;
+};
+
+// q heads per CTA and keys per tile the launcher picks (exposed for tests of the policy)
+int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms);
+int attn_tma_kt(int hpc);
 
 // Launch on stream s; returns the CTAs launched, -1 if the launch failed.
-int launch_attention_tma(const CUtensorMap &mk, const CUtensorMap &mv, AttnTmaArgs a, int hd, bool split,
-                         int num_sms, cudaStream_t s);
+int launch_attention_tma(const AttnTmaMaps &maps, AttnTmaArgs a, int hd, bool split, int num_sms, cudaStream_t s);
 
 }  // namespace dfl

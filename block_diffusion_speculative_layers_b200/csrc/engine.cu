@@ -351,7 +351,7 @@ class Engine : public EngineBase {
     float2 *lm_part;
     AttnScratch att;
     // TMA attention: K / V maps of the target (0) and the drafter (1) caches
-    CUtensorMap kv_map[2][2];
+    AttnTmaMaps kv_map[2];
     bool attn_tma_on = false;
     // folded-norm decode passes (bf16)
     T *xg_t = nullptr, *xg2 = nullptr;
@@ -526,9 +526,16 @@ class Engine : public EngineBase {
             for (int w = 0; w < 2 && attn_tma_on; ++w) {
                 const dflash_model_cfg &m = *ms[w];
                 attn_tma_on = attn_tma_supported(m.head_dim, m.n_q_heads / m.n_kv_heads);
-                for (int kv = 0; kv < 2 && attn_tma_on; ++kv)
-                    attn_tma_on = attn_tma_make_map(&kv_map[w][kv], (const bf16 *)caches[w][kv], m.head_dim, c.max_len,
-                                                    c.max_batch * m.n_kv_heads, m.n_layers, kv_layer_elems(m), lo_);
+                CUtensorMap *dst[2][2] = {{&kv_map[w].k16, &kv_map[w].v16}, {&kv_map[w].k32, &kv_map[w].v32}};
+                for (int kt = 0; kt < 2; ++kt)
+                    for (int kv = 0; kv < 2 && attn_tma_on; ++kv)
+                        attn_tma_on = attn_tma_make_map(dst[kt][kv], (const bf16 *)caches[w][kv], m.head_dim, c.max_len,
+                                                        c.max_batch * m.n_kv_heads, m.n_layers, kv_layer_elems(m), lo_,
+                                                        kt ? 32 : 16);
+            }
+            if (!legacy && !attn_tma_on) {
+                err = "attention: K/V tensor maps could not be encoded";
+                return DFLASH_ECUDA;
             }
         }
         att.n_sem = std::max(L.R_dec, (L.C + 15) / 16) * std::max(c.target.n_kv_heads, c.drafter.n_kv_heads);
@@ -558,6 +565,9 @@ class Engine : public EngineBase {
         tc.tune_smem_kb = env_int("DFLASH_TC_SMEM_KB");
         tc.tune_split_smem_kb = env_int("DFLASH_TC_SPLIT_SMEM_KB");
         tc.tune_ctas_per_sm = env_int("DFLASH_TC_CTAS_PER_SM");
+        // weight stages a projection prefetches into L2 beyond its shared-memory ring
+        tc.l2_ahead = env_int("DFLASH_TC_L2_AHEAD");
+        tc.tune_tm_max = env_int("DFLASH_TC_TM_MAX");
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);
         tc.keep_logits = c.keep_logits;  // plus while sampling (sampling_changed)
@@ -773,8 +783,7 @@ class Engine : public EngineBase {
                     a.ldo = qd;
                     a.lo = lo_;
                     a.err = &stats->status;
-                    ctas = launch_attention_tma(kv_map[which][0], kv_map[which][1], a, m.head_dim, lo_ != 0, num_sms,
-                                                s);
+                    ctas = launch_attention_tma(kv_map[which], a, m.head_dim, lo_ != 0, num_sms, s);
                     if (ctas < 0) attn_failed = true;
                 }
             } else if (attn_mma_supported<T>(m.head_dim))
@@ -1506,11 +1515,11 @@ class Engine : public EngineBase {
     }
 
     // The device status word (stream already synchronised): bit 0 a non-finite
-    // logit reached an argmax, bits 2-4 a bounded device wait expired.  Sticky
+    // logit reached an argmax, bits 2-5 a bounded device wait expired.  Sticky
     // until dflash_reset_stats or the next generation.
     static dflash_status status_code(int st, std::string &err) {
         if (st & 1) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
-        if (st & (4 | 8 | 16)) { err = "a bounded device wait expired"; return DFLASH_ETIMEOUT; }
+        if (st & (4 | 8 | 16 | 32)) { err = "a bounded device wait expired"; return DFLASH_ETIMEOUT; }
         return DFLASH_OK;
     }
     dflash_status numeric_status() {

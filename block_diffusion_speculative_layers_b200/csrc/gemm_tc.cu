@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(NT, 1)
     uint64_t *acc_empty = acc_full + 2;    // [2]
     uint64_t *a_conv = acc_empty + 2;      // [F8_ASTAGES] A stage converted into tensor memory
     uint64_t *a_free = a_conv + F8_ASTAGES;  // [F8_ASTAGES] A stage read by the MMAs
-    uint32_t *tmem_slot = (uint32_t *)(a_free + F8_ASTAGES);
+    // F8: the activation tiles of a stage complete on their own barrier, so the
+    // weight codes (full[]) can be converted before the previous kernel is done
+    uint64_t *full_b = a_free + F8_ASTAGES;  // [stages]
+    uint32_t *tmem_slot = (uint32_t *)(full_b + (F8 ? stages : 0));
     // split-K receive buffer [S][128][cpr] (16-byte aligned, after the fixed area)
     float *recv = (float *)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
     EpiIn pre;
@@ -148,6 +151,8 @@ __global__ void __launch_bounds__(NT, 1)
             mbar_init(&a_conv[s], 4);
             mbar_init(&a_free[s], 1);
         }
+        if (F8)
+            for (int s = 0; s < stages; ++s) mbar_init(&full_b[s], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -172,12 +177,15 @@ __global__ void __launch_bounds__(NT, 1)
             const uint64_t wpol = l2_evict_first_policy();
             const int kstep = F8 ? 2 * BK : BK;  // K elements per stage
             auto load_x = [&](int s, int k, int m0) {
+                uint64_t *bar = F8 ? &full_b[s] : &full[s];
+                if (F8) mbar_expect_tx(bar, B_ST);
                 for (int h = 0; h < (F8 ? 2 : 1); ++h) {
                     uint8_t *b = sB + (size_t)s * B_ST + h * B_BYTES;
-                    if (p.planes == 2) tma_load_3d(b, &tmX, k + h * BK, m0, 0, &full[s]);
-                    else tma_load_2d(b, &tmX, k + h * BK, m0, &full[s]);
+                    if (p.planes == 2) tma_load_3d(b, &tmX, k + h * BK, m0, 0, bar);
+                    else tma_load_2d(b, &tmX, k + h * BK, m0, bar);
                 }
             };
+            const int a_tx = F8 ? A_ST : A_ST + B_ST;  // bytes completing full[]
             int it = 0;     // global stage counter
             bool first = true, abort = false;
             for (int t = tile0; t < n_tiles_total && !abort; t += tstride) {
@@ -191,7 +199,7 @@ __global__ void __launch_bounds__(NT, 1)
                     const int pre = min(nk, stages);
                     for (int i = 0; i < pre; ++i) {
                         uint8_t *a = sA + (size_t)i * A_ST;
-                        mbar_expect_tx(&full[i], A_ST + B_ST);
+                        mbar_expect_tx(&full[i], a_tx);
                         tma_load_2d_hint(a, &tmW, (kb + i) * kstep, rowA0, &full[i], wpol);
                         tma_load_2d_hint(a + A_ST / 2, &tmW, (kb + i) * kstep, rowA1, &full[i], wpol);
                     }
@@ -201,15 +209,26 @@ __global__ void __launch_bounds__(NT, 1)
                     it = pre;
                     first = false;
                 }
+                // L2 prefetch: keep the stages l2_ahead beyond the ring in flight from HBM
+                int pf = kk0;
+                auto prefetch_to = [&](int upto) {
+                    for (; pf < min(nk, upto); ++pf) {
+                        const int kp = (kb + pf) * kstep;
+                        tma_prefetch_2d(&tmW, kp, rowA0);
+                        tma_prefetch_2d(&tmW, kp, rowA1);
+                    }
+                };
+                if (p.l2_ahead > 0) prefetch_to(kk0 + p.l2_ahead);
                 for (int kk = kk0; kk < nk; ++kk, ++it) {
                     const int s = it % stages;
                     if (it >= stages && !mbar_wait(&empty[s], ((it / stages) & 1) ^ 1, p.err)) {
                         abort = true;
                         break;
                     }
+                    if (p.l2_ahead > 0) prefetch_to(kk + 1 + p.l2_ahead);
                     const int k = (kb + kk) * kstep;
                     uint8_t *a = sA + (size_t)s * A_ST;
-                    mbar_expect_tx(&full[s], A_ST + B_ST);
+                    mbar_expect_tx(&full[s], a_tx);
                     tma_load_2d_hint(a, &tmW, k, rowA0, &full[s], wpol);
                     tma_load_2d_hint(a + A_ST / 2, &tmW, k, rowA1, &full[s], wpol);
                     load_x(s, k, m0);
@@ -231,7 +250,8 @@ __global__ void __launch_bounds__(NT, 1)
                     const int s = it % stages;
                     if constexpr (F8) {
                         const int sa = it % F8_ASTAGES;
-                        if (!mbar_wait(&a_conv[sa], (it / F8_ASTAGES) & 1, p.err)) {
+                        if (!mbar_wait(&full_b[s], (it / stages) & 1, p.err) ||
+                            !mbar_wait(&a_conv[sa], (it / F8_ASTAGES) & 1, p.err)) {
                             ok = false;
                             break;
                         }
@@ -272,14 +292,52 @@ __global__ void __launch_bounds__(NT, 1)
         }
     } else {
         // ---------------- epilogue warps 2..5 ----------------
+        const int q = warp & 3;
+        const int n_local = q * 32 + lane;
+        if constexpr (F8) {
+            // ---- convert the weight stages into tensor memory (thread = weight row n_local) ----
+            // The codes do not depend on the previous kernel: this runs before the wait for it.
+            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+            const int rr = n_local & 63;  // row within its 64-row box
+            bool dead = false;
+            for (int kk = 0; kk < nk; ++kk) {
+                const int s = kk % stages, sa = kk % F8_ASTAGES;
+                if (!dead && !mbar_wait(&full[s], (kk / stages) & 1, p.err)) dead = true;
+                if (!dead && kk >= F8_ASTAGES && !mbar_wait(&a_free[sa], ((kk / F8_ASTAGES) - 1) & 1, p.err))
+                    dead = true;
+                const uint8_t *row = sA + (size_t)s * A_ST + (n_local >> 6) * (A_ST / 2) + rr * 128;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // 64 K per tcgen05.st of 32 columns
+                    uint32_t w[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int chunk = h * 4 + c;  // 16 codes = K 16*chunk .. +15, 128-byte swizzle
+                        const uint4 v = dead ? make_uint4(0, 0, 0, 0)
+                                             : *reinterpret_cast<const uint4 *>(row + (((chunk ^ rr) & 7) << 4));
+                        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
+                            w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
+                        }
+                    }
+                    tmem_st32(tmem_a + lane_base + (uint32_t)(sa * 64 + h * 32), w);
+                }
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&a_conv[sa]);
+                    mbar_arrive(&empty[s]);
+                }
+            }
+        }
         if (p.dep_ctr) {
             if (threadIdx.x == 64) dep_wait(p.dep_ctr, p.dep_target, p.err);
             epi_bar();
         } else {
             pdl_wait();
         }
-        const int q = warp & 3;
-        const int n_local = q * 32 + lane;
         // F8: this thread's weight row and its scale
         float wsc = 1.f;
         if constexpr (F8) {
@@ -304,43 +362,6 @@ __global__ void __launch_bounds__(NT, 1)
             }
             // inputs of this CTA's first epilogue chunk, while the mainloop streams
             if (c_end > c_begin) epi_prefetch<KIND, CH>(p, e, nt, n_local, mt * TM + c_begin, min(CH, c_end - c_begin), pre, smeta);
-            if constexpr (F8) {
-                // ---- convert the weight stages into tensor memory (thread = weight row n_local) ----
-                const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-                const int rr = n_local & 63;                       // row within its 64-row box
-                bool dead = false;
-                for (int kk = 0; kk < nk; ++kk) {
-                    const int s = kk % stages, sa = kk % F8_ASTAGES;
-                    if (!dead && !mbar_wait(&full[s], (kk / stages) & 1, p.err)) dead = true;
-                    if (!dead && kk >= F8_ASTAGES && !mbar_wait(&a_free[sa], ((kk / F8_ASTAGES) - 1) & 1, p.err))
-                        dead = true;
-                    const uint8_t *row = sA + (size_t)s * A_ST + (n_local >> 6) * (A_ST / 2) + rr * 128;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {  // 64 K per tcgen05.st of 32 columns
-                        uint32_t w[32];
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int chunk = h * 4 + c;  // 16 codes = K 16*chunk .. +15, 128-byte swizzle
-                            const uint4 v = dead ? make_uint4(0, 0, 0, 0)
-                                                 : *reinterpret_cast<const uint4 *>(row + (((chunk ^ rr) & 7) << 4));
-                            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
-                                w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
-                            }
-                        }
-                        tmem_st32(tmem_a + lane_base + (uint32_t)(sa * 64 + h * 32), w);
-                    }
-                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&a_conv[sa]);
-                        mbar_arrive(&empty[s]);
-                    }
-                }
-            }
             const uint32_t trow = tmem + (uint32_t)(b * NC1) + ((uint32_t)(q * 32) << 16);
             const bool ok = mbar_wait(&acc_full[b], (lt >> 1) & 1, p.err) && nk > 0;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -602,6 +623,15 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     const bool swiglu = e.kind == EPI_SWIGLU;
     const bool f8 = w_scale != nullptr;
     int TM = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    if (tune_tm_max >= 16) {
+        TM = std::min(TM, tune_tm_max);
+    } else if (TM > 64) {
+        // many activation rows (batched decode, prefill chunks): the largest row tile
+        // that still gives every SM a tile; the weight tile is then re-read per row
+        // tile, from L2 (measured: one CTA per weight tile left most SMs idle)
+        const int nt = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
+        while (TM > 64 && nt * ((M + TM - 1) / TM) < num_sms) TM /= 2;
+    }
     if (f8) TM = std::min(TM, 64);  // FP8: tensor memory holds the A stages too; larger M takes several row tiles
     TcParams p;
     memset(&p, 0, sizeof p);
@@ -616,9 +646,10 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     const int tiles = p.n_tiles * p.m_tiles;
     p.planes = e.lo ? 2 : 1;
     p.w_scale = w_scale;
+    p.l2_ahead = l2_ahead;
     const int stage_bytes = f8 ? tc::F8_A_BYTES + 2 * TM * 128 * p.planes : tc::A_BYTES + TM * 128 * p.planes;
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
-                      2 * tc::F8_ASTAGES * 8;
+                      2 * tc::F8_ASTAGES * 8 + 16 * 8;
     // Measured on B200 (decode shapes, M = 16, whole decode iteration): every
     // projection streams best with ~110 KB CTAs, two of which fit on an SM;
     // projections with fewer tiles than that split K over a cluster (up to 8

@@ -38,6 +38,7 @@ struct TcParams {
     int dep_target;
     int *done_ctr;
     const float *w_scale;   // FP8 weights: fp32 scale of every weight row (the codes' row of W)
+    int l2_ahead;           // weight stages prefetched into L2 beyond the shared-memory ring (0: none)
 };
 
 template <typename T>
@@ -66,7 +67,8 @@ struct GemmTC {
     int num_sms = 148;
     // tuning overrides (0 = automatic): K splits per tile, shared-memory budget in KB
     // of unsplit / K-split launches, CTAs per SM the K split aims to fill
-    int tune_splits = 0, tune_smem_kb = 0, tune_split_smem_kb = 0, tune_ctas_per_sm = 0;
+    int tune_splits = 0, tune_smem_kb = 0, tune_split_smem_kb = 0, tune_ctas_per_sm = 0, l2_ahead = 0;
+    int tune_tm_max = 0;  // cap on the activation rows of one tile (more row tiles, weights re-read from L2)
     std::unordered_map<std::string, CUtensorMap> maps;
     // 2-D map of a [rows][cols] bf16 matrix (leading dimension ld), box {64, box_rows};
     // plane_stride > 0: 3-D map over the hi plane and the lo plane plane_stride
