@@ -568,6 +568,7 @@ class Engine : public EngineBase {
         // weight stages a projection prefetches into L2 beyond its shared-memory ring
         tc.l2_ahead = env_int("DFLASH_TC_L2_AHEAD");
         tc.tune_tm_max = env_int("DFLASH_TC_TM_MAX");
+        tc.f8_int_conv = env_int("DFLASH_F8_INT_CONV");
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);
         tc.keep_logits = c.keep_logits;  // plus while sampling (sampling_changed)

@@ -67,6 +67,42 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t c) {
     return ((t + 0x38003800u) & nz) | (f & 0x80008000u);
 }
 
+// Four E4M3 codes (byte j of w) -> bf16 pairs (codes 0,1) and (codes 2,3) with
+// integer operations only.  Normal codes: the sign moves to bit 15 and the
+// 7 exponent/mantissa bits shift by 4 with the exponent rebiased by 120
+// (7 -> 127), exactly.  Codes with a zero exponent field (zero, subnormals
+// m * 2^-9) -- rare in scaled weights -- take an exact per-byte path.
+__device__ __noinline__ uint32_t e4m3x2_small_to_bf16x2(uint32_t pair) {
+    // pair = b1 << 16 | b0
+    uint32_t out = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t b = (pair >> (16 * h)) & 0xFFu;
+        uint32_t v;
+        if (b & 0x78u) {
+            v = ((b & 0x7Fu) << 4) + 0x3C00u;
+        } else {
+            const uint32_t m = b & 7u;
+            // m = 0: 0; 1: 0x3B00; 2: 0x3B80; 3: 0x3BC0; 4..7: 0x3C00 + 0x20 * (m - 4)
+            v = m == 0 ? 0u : m == 1 ? 0x3B00u : m == 2 ? 0x3B80u : m == 3 ? 0x3BC0u : 0x3C00u + 0x20u * (m - 4);
+        }
+        out |= (v | ((b & 0x80u) << 8)) << (16 * h);
+    }
+    return out;
+}
+
+__device__ __forceinline__ void e4m3x4_to_bf16_int(uint32_t w, uint32_t &r0, uint32_t &r1) {
+    const uint32_t p0 = __byte_perm(w, 0u, 0x4140u);  // b1 << 16 | b0
+    const uint32_t p1 = __byte_perm(w, 0u, 0x4342u);  // b3 << 16 | b2
+    r0 = ((p0 & 0x007F007Fu) * 16u + 0x3C003C00u) | ((p0 << 8) & 0x80008000u);
+    r1 = ((p1 & 0x007F007Fu) * 16u + 0x3C003C00u) | ((p1 << 8) & 0x80008000u);
+    const uint32_t t = w & 0x78787878u;  // exponent fields: a zero byte marks zero / subnormal codes
+    if ((t - 0x01010101u) & ~t & 0x80808080u) {
+        r0 = e4m3x2_small_to_bf16x2(p0);
+        r1 = e4m3x2_small_to_bf16x2(p1);
+    }
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
@@ -315,10 +351,15 @@ __global__ void __launch_bounds__(NT, 1)
                         const uint4 v = dead ? make_uint4(0, 0, 0, 0)
                                              : *reinterpret_cast<const uint4 *>(row + (((chunk ^ rr) & 7) << 4));
                         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+                        if (p.f8_int_conv) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
-                            w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
+                            for (int j = 0; j < 4; ++j) e4m3x4_to_bf16_int(u[j], w[c * 8 + 2 * j], w[c * 8 + 2 * j + 1]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
+                                w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
+                            }
                         }
                     }
                     tmem_st32(tmem_a + lane_base + (uint32_t)(sa * 64 + h * 32), w);
@@ -647,6 +688,7 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     p.planes = e.lo ? 2 : 1;
     p.w_scale = w_scale;
     p.l2_ahead = l2_ahead;
+    p.f8_int_conv = f8_int_conv;
     const int stage_bytes = f8 ? tc::F8_A_BYTES + 2 * TM * 128 * p.planes : tc::A_BYTES + TM * 128 * p.planes;
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
                       2 * tc::F8_ASTAGES * 8 + 16 * 8;

@@ -72,3 +72,13 @@ def test_fp8_qwen3_8b_widths(cuda_device):
     finally:
         gpu.close()
         torch.cuda.empty_cache()
+
+
+def test_fp8_integer_widening_variant(cuda_device, monkeypatch):
+    """The integer widening of the codes (DFLASH_F8_INT_CONV=1) gives the same model."""
+    monkeypatch.setenv("DFLASH_F8_INT_CONV", "1")
+    cfg = tiny_cfg(dtype="fp8", block=16, hidden=2048, nq=16, nkv=4, hd=128, vocab=8192)
+    gpu, spec, _ = build_pair(cfg, max_len=128)
+    rep = replay(gpu, spec, cfg, [make_prompt("uniform", 30, cfg.target.vocab, 80)], 4, TOL, TIE)
+    assert rep.mismatches_outside_ties == 0, rep
+    assert rep.max_dlogit <= TOL
