@@ -238,6 +238,8 @@ static Layout make_layout(const dflash_config &c) {
     L.dv = take(kv_d);
     L.xg_t = take((size_t)L.R_dec * H * es);
     L.xg2 = take((size_t)L.R_dec * H * es);
+    // MoE decode: the pairs' activation rows in expert-grouped order
+    L.moe_xg = take(t.n_experts > 0 ? (size_t)L.R_dec * t.top_k * H * es : 16);
     const size_t act_bytes = align_up(o, 256) - act0;
     if (c.dtype == DFLASH_BF16 || c.dtype == DFLASH_FP8) {
         take(act_bytes);
@@ -340,6 +342,8 @@ class Engine : public EngineBase {
     float4 *samp_part = nullptr;
     int *tok_p = nullptr, *resid = nullptr;
     T *xn, *dq_in, *q, *ao, *h, *taps_dec, *taps_gather, *taps_pre, *cbuf, *tk, *tv, *dk, *dv;
+    T *moe_xg = nullptr;
+    bool moe_grouped_on = false;  // MoE decode experts as grouped tensor-core projections
     int *g, *drafts, *accept, *committed, *new_len, *active, *script, *out_tok, *tokens, *first_tok, *moe_sel;
     int *moe_off = nullptr, *moe_list = nullptr;
     SeqState *st;
@@ -487,6 +491,13 @@ class Engine : public EngineBase {
         gemm_sem = sp<int>(L.gemm_sem);
         lm_part = sp<float2>(L.lm_part);
         xg_t = sp<T>(L.xg_t);
+        moe_xg = sp<T>(L.moe_xg);
+        {
+            // DFLASH_MOE_STREAM=1: the CUDA-core weight-streaming expert kernels instead
+            const char *mv = getenv("DFLASH_MOE_STREAM");
+            moe_grouped_on = std::is_same<T, bf16>::value && c.target.n_experts > 0 && !(mv && mv[0] == '1') &&
+                             c.target.hidden % 64 == 0 && c.target.expert_ffn % 64 == 0;
+        }
         lo_ = L.act_lo;
         xg2 = sp<T>(L.xg2);
         ssq = sp<float>(L.ssq);
@@ -868,6 +879,33 @@ class Engine : public EngineBase {
         gemm(xn, H, R, w.w_router, E, H, e);
         launch_moe_topk(Y, E, R, k, moe_sel, moe_wt, s);
         if constexpr (std::is_same<T, bf16>::value) {
+            if (moe_grouped_on && R <= L.R_dec) {
+                // decode: each touched expert's gate/up and down as one grouped tcgen05
+                // projection over its pairs (rows gathered in expert order)
+                int *touched = moe_off + E + 1;
+                launch_moe_bucket(moe_sel, R * k, E, moe_off, moe_list, s);
+                launch_moe_gather(xn, H, lo_, moe_list, k, R * k, H, moe_xg, s);
+                Epi<T> gu;
+                gu.kind = EPI_SWIGLU;
+                gu.h = h;
+                gu.F = Fe;
+                gu.lo = lo_;
+                timed(DFLASH_PROF_PROJECTION, (double)R * k * H * 2, [&] {
+                    tc.run_grouped(moe_xg, H, R * k, (const T *)w.we_gate_up, 2 * Fe, 2 * Fe, H, gu, moe_off, touched,
+                                   moe_list, E, R, s);
+                }, DFLASH_PROF_OTHER_PROJ);
+                Epi<T> dn;
+                dn.kind = EPI_STORE;
+                dn.Y = moe_part;
+                dn.ldy = H;
+                dn.lo = lo_;
+                timed(DFLASH_PROF_PROJECTION, (double)R * k * Fe * 2, [&] {
+                    tc.run_grouped(h, Fe, R * k, (const T *)w.we_down, H, H, Fe, dn, moe_off, touched, moe_list, E, R,
+                                   s);
+                }, DFLASH_PROF_OTHER_PROJ);
+                launch_moe_combine<T>(x, moe_part, moe_wt, H, R, k, taps, lo_, mt, s);
+                return;
+            }
             if (moe_bucketed_supported(H, Fe, E)) {
                 // touched experts only, each expert's weights streamed once per layer
                 launch_moe_experts_bucketed(xn, H, lo_, R, k, moe_sel, E, (const bf16 *)w.we_gate_up,

@@ -37,7 +37,7 @@ struct Layout {
     size_t qlogits, lse_p, lse_q, samp_part, tok_p, resid;  // temperature sampling (config.sampling)
     size_t g, drafts, accept, committed, new_len, st, active, meta, ctx_meta, ctx_meta_pre;
     size_t rope_t, rope_d, tk, tv, dk, dv, script, out_tok, tokens, stats, first_tok;
-    size_t moe_sel, moe_wt, moe_part, moe_off = 0, moe_list = 0, lm_part, att_o, att_ml, att_sem;
+    size_t moe_sel, moe_wt, moe_part, moe_off = 0, moe_list = 0, moe_xg = 0, lm_part, att_o, att_ml, att_sem;
     size_t att_parts = 0;
     size_t xg_t, xg2, ssq, dep_v, dep_d;
     size_t act_lo = 0;  // two-plane activations: low plane offset in elements (0: one plane)

@@ -126,8 +126,26 @@ __device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a
 
 template <int TM, int KIND, bool F8>
 __global__ void __launch_bounds__(NT, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcParams p,
-                   Epi<bf16> e, int stages) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcParams p_in,
+                   Epi<bf16> e_in, int stages) {
+    TcParams p = p_in;
+    Epi<bf16> e = e_in;
+    // grouped (MoE experts): this CTA's expert, rows and weight rows
+    const bool grouped = p.g_off != nullptr;
+    int g_row0 = 0, g_wrow0 = 0;
+    if (grouped) {
+        pdl_wait();  // the expert lists come from the bucketing kernel
+        const int ex = p.g_touched[blockIdx.y];
+        if (ex < 0) return;
+        const int r0 = p.g_off[ex], m0 = (int)blockIdx.z * TM;
+        const int nr = p.g_off[ex + 1] - r0;
+        if (m0 >= nr) return;
+        p.M = min(TM, nr - m0);
+        g_row0 = r0 + m0;
+        g_wrow0 = ex * p.g_wrows;
+        if (KIND == EPI_SWIGLU) e.h += (size_t)g_row0 * p.swiglu_F;
+        if (KIND == EPI_STORE && p.g_list) e.row_map = p.g_list + g_row0;
+    }
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int B_BYTES = TM * 128 * p.planes;  // activation tile(s) of 64 K
@@ -161,11 +179,12 @@ __global__ void __launch_bounds__(NT, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.splits;
     const bool split = S > 1;
-    const int n_tiles_total = p.n_tiles * p.m_tiles;
+    const int n_tiles_total = grouped ? p.n_tiles : p.n_tiles * p.m_tiles;
     // one tile per CTA: (blockIdx.x, blockIdx.y); a persistent launch would pass
-    // a 1-D grid smaller than the tile count and stride over the tiles
-    const bool persistent = !F8 && !split && gridDim.y == 1 && (int)gridDim.x < n_tiles_total;
-    const int tile0 = persistent ? blockIdx.x : blockIdx.y * p.n_tiles + blockIdx.x;
+    // a 1-D grid smaller than the tile count and stride over the tiles; a grouped
+    // launch has one weight tile (blockIdx.x) of one expert's rows per CTA
+    const bool persistent = !F8 && !split && !grouped && gridDim.y == 1 && (int)gridDim.x < n_tiles_total;
+    const int tile0 = persistent || grouped ? blockIdx.x : blockIdx.y * p.n_tiles + blockIdx.x;
     const int tstride = persistent ? gridDim.x : n_tiles_total;
     const int k_per = (p.k_steps + S - 1) / S;
     const int kb = split ? blockIdx.z * k_per : 0;
@@ -226,9 +245,9 @@ __global__ void __launch_bounds__(NT, 1)
             bool first = true, abort = false;
             for (int t = tile0; t < n_tiles_total && !abort; t += tstride) {
                 const int nt = t % p.n_tiles, mt = t / p.n_tiles;
-                const int rowA0 = p.swiglu_F ? nt * 64 : nt * 128;
-                const int rowA1 = p.swiglu_F ? p.swiglu_F + nt * 64 : nt * 128 + 64;
-                const int m0 = mt * TM;
+                const int rowA0 = g_wrow0 + (p.swiglu_F ? nt * 64 : nt * 128);
+                const int rowA1 = g_wrow0 + (p.swiglu_F ? p.swiglu_F + nt * 64 : nt * 128 + 64);
+                const int m0 = grouped ? g_row0 : mt * TM;
                 int kk0 = 0;
                 if (first) {
                     // weights do not depend on the previous kernel: start streaming them first
@@ -239,7 +258,7 @@ __global__ void __launch_bounds__(NT, 1)
                         tma_load_2d_hint(a, &tmW, (kb + i) * kstep, rowA0, &full[i], wpol);
                         tma_load_2d_hint(a + A_ST / 2, &tmW, (kb + i) * kstep, rowA1, &full[i], wpol);
                     }
-                    dep_wait(p.dep_ctr, p.dep_target, p.err);
+                    if (!grouped) dep_wait(p.dep_ctr, p.dep_target, p.err);
                     for (int i = 0; i < pre; ++i) load_x(i, (kb + i) * kstep, m0);
                     kk0 = pre;
                     it = pre;
@@ -376,7 +395,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (p.dep_ctr) {
             if (threadIdx.x == 64) dep_wait(p.dep_ctr, p.dep_target, p.err);
             epi_bar();
-        } else {
+        } else if (!grouped) {
             pdl_wait();
         }
         // F8: this thread's weight row and its scale
@@ -750,6 +769,57 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
 template <>
 int GemmTC<float>::run(const float *, int, int, const void *, int, int, const Epi<float> &, cudaStream_t,
                        const int *, int, int *, const float *) {
+    return 0;
+}
+
+template <>
+int GemmTC<bf16>::run_grouped(const bf16 *X, int ldx, int n_pairs, const bf16 *W, int wrows, int N, int K,
+                              const Epi<bf16> &e, const int *off, const int *touched, const int *list, int E,
+                              int max_rows, cudaStream_t s) {
+    const bool swiglu = e.kind == EPI_SWIGLU;
+    const int TM = max_rows <= 16 ? 16 : max_rows <= 32 ? 32 : 64;
+    TcParams p;
+    memset(&p, 0, sizeof p);
+    p.M = n_pairs;
+    p.N = N;
+    p.K = K;
+    p.swiglu_F = swiglu ? e.F : 0;
+    p.n_tiles = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
+    p.m_tiles = (max_rows + TM - 1) / TM;
+    p.k_steps = (K + tc::BK - 1) / tc::BK;
+    p.planes = e.lo ? 2 : 1;
+    p.splits = 1;
+    p.err = err_word;
+    p.g_off = off;
+    p.g_touched = touched;
+    p.g_list = list;
+    p.g_wrows = wrows;
+    const int stage_bytes = tc::A_BYTES + TM * 128 * p.planes;
+    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
+                      2 * tc::F8_ASTAGES * 8 + 16 * 8;
+    const int stages = std::max(2, std::min(16, (112 * 1024 - fixed) / stage_bytes));
+    const size_t smem = (size_t)fixed + (size_t)stages * stage_bytes;
+    const CUtensorMap *mw = tensor_map(W, E * wrows, K, K, 64);
+    const CUtensorMap *mx = tensor_map(X, n_pairs, K, ldx, TM, e.lo);
+    if (!mw || !mx) {
+        failed = true;
+        return 0;
+    }
+    auto go = [&](auto tm_c) {
+        constexpr int T_ = decltype(tm_c)::value;
+        auto kern = swiglu ? tc::gemm_tc_kernel<T_, EPI_SWIGLU, false> : tc::gemm_tc_kernel<T_, EPI_STORE, false>;
+        ensure_smem_attr((const void *)kern);
+        launch_k(kern, dim3(p.n_tiles, E, p.m_tiles), dim3(tc::NT), smem, s, 1, *mw, *mx, p, e, stages);
+    };
+    if (TM == 16) go(std::integral_constant<int, 16>{});
+    else if (TM == 32) go(std::integral_constant<int, 32>{});
+    else go(std::integral_constant<int, 64>{});
+    return p.n_tiles * E * p.m_tiles;
+}
+
+template <>
+int GemmTC<float>::run_grouped(const float *, int, int, const float *, int, int, int, const Epi<float> &, const int *,
+                               const int *, const int *, int, int, cudaStream_t) {
     return 0;
 }
 

@@ -40,6 +40,11 @@ struct TcParams {
     const float *w_scale;   // FP8 weights: fp32 scale of every weight row (the codes' row of W)
     int l2_ahead;           // weight stages prefetched into L2 beyond the shared-memory ring (0: none)
     int f8_int_conv;        // FP8: widen codes with integer operations instead of the f16 conversion
+    // grouped (MoE experts): blockIdx.y = touched-expert slot, blockIdx.z = row tile of
+    // that expert; its rows are g_off[e] .. g_off[e+1]-1 of X (expert-grouped order) and
+    // its weights rows e*g_wrows .. of W; nullptr g_off = an ordinary projection
+    const int *g_off, *g_touched, *g_list;
+    int g_wrows;
 };
 
 template <typename T>
@@ -54,6 +59,12 @@ struct GemmTC {
     int run(const T *X, int ldx, int M, const void *W, int N, int K, const Epi<T> &e, cudaStream_t s,
             const int *dep_ctr = nullptr, int dep_target = 0, int *done_ctr = nullptr,
             const float *w_scale = nullptr);
+    // Grouped projection over the touched experts of a MoE layer: W is [E][wrows][K],
+    // X the pair rows in expert-grouped order (off[E+1], touched[E] as bucketed),
+    // at most max_rows rows per expert.  EPI_SWIGLU writes h in grouped order;
+    // EPI_STORE writes row list[pos] of Y.  Returns the CTAs launched.
+    int run_grouped(const T *X, int ldx, int n_pairs, const T *W, int wrows, int N, int K, const Epi<T> &e,
+                    const int *off, const int *touched, const int *list, int E, int max_rows, cudaStream_t s);
     // LM-head partial argmax buffer (value, index as float bits), [n_tiles][rows]
     void set_lm_part(float2 *p, int cap) { lm_part = p; lm_cap = cap; }
     void set_err(int *e) { err_word = e; }

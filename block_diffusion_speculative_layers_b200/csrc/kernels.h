@@ -93,6 +93,13 @@ void launch_moe_experts_simt(const T *m, int ldm, size_t lo, int R, int k, const
 // h[pair][Fe] (two planes when hlo != 0) and down -> part[pair][H], each a
 // persistent weight-streaming kernel of num_sms CTAs; timed-out waits set bit 4 of *err.
 bool moe_bucketed_supported(int H, int Fe, int E);
+// Rows of the pairs in expert-grouped order: xg[pos] = m[list[pos] / k] (both
+// planes), for the grouped tensor-core expert projections.
+void launch_moe_gather(const bf16 *m, int ldm, size_t lo, const int *list, int k, int n_pairs, int H, bf16 *xg,
+                       cudaStream_t s);
+// Bucketing alone: off[E+1] pair ranges, list[n_pairs] pairs by expert, off[E+1 ..
+// 2E+1] touched experts (ascending, -1 after them), off[2E+1] their count.
+void launch_moe_bucket(const int *sel, int n_pairs, int E, int *off, int *list, cudaStream_t s);
 void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k, const int *sel, int E,
                                  const bf16 *w_gate_up, const bf16 *w_down, int H, int Fe, int *off, int *list,
                                  bf16 *h, size_t hlo, float *part, int num_sms, int *err, cudaStream_t s);
@@ -173,6 +180,8 @@ struct Epi {
     // EPI_STORE / EPI_LOGITS: fp32 output Y[M][ldy]
     float *Y = nullptr;
     int ldy = 0;
+    // EPI_STORE: output row of activation row m is row_map[m] (nullptr: m)
+    const int *row_map = nullptr;
     // EPI_QKV: columns are rows col0.. of [Wq; Wk; Wv]; rows < R_blk are block rows
     // (q, k, v at meta.pos), rows >= R_blk context rows (k, v at ctx_meta.pos if aux)
     int col0 = 0, R_blk = 0;

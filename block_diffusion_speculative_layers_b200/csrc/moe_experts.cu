@@ -430,8 +430,33 @@ int stream_stages(int n, int rows, int E) {
 
 }  // namespace
 
+// xg[pos] = m[list[pos] / k], both planes: one CTA per pair, 16-byte copies
+__global__ void moe_gather_kernel(const bf16 *__restrict__ m, int ldm, size_t lo, const int *__restrict__ list, int k,
+                                  int H, bf16 *__restrict__ xg) {
+    pdl_trigger();
+    pdl_wait();
+    const int pos = blockIdx.x;
+    const int row = list[pos] / k;
+    const uint4 *src = reinterpret_cast<const uint4 *>(m + (size_t)row * ldm);
+    uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)pos * H);
+    for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+        dst[c] = src[c];
+        if (lo) reinterpret_cast<uint4 *>(xg + lo + (size_t)pos * H)[c] = reinterpret_cast<const uint4 *>(m + lo + (size_t)row * ldm)[c];
+    }
+}
+
+void launch_moe_gather(const bf16 *m, int ldm, size_t lo, const int *list, int k, int n_pairs, int H, bf16 *xg,
+                       cudaStream_t s) {
+    if (n_pairs <= 0) return;
+    launch_k(moe_gather_kernel, dim3(n_pairs), dim3(128), 0, s, 1, m, ldm, lo, list, k, H, xg);
+}
+
 bool moe_bucketed_supported(int H, int Fe, int E) {
     return H % 256 == 0 && Fe % 256 == 0 && H <= 256 * MAX_CPL && Fe <= 256 * MAX_CPL && E <= 256;
+}
+
+void launch_moe_bucket(const int *sel, int n_pairs, int E, int *off, int *list, cudaStream_t s) {
+    launch_k(moe_bucket_kernel, dim3(1), dim3(1024), 0, s, 1, sel, n_pairs, E, off, list, off + E + 1);
 }
 
 void launch_moe_experts_bucketed(const bf16 *m, int ldm, size_t lo, int R, int k, const int *sel, int E,

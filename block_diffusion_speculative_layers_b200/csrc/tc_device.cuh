@@ -367,7 +367,8 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams &p, const Epi<bf16
         if (n < p.N) {
 #pragma unroll
             for (int j = 0; j < W; ++j)
-                if (j < nc && m0c + j < M) e.Y[(size_t)(m0c + j) * e.ldy + n] = v[j];
+                if (j < nc && m0c + j < M)
+                    e.Y[(size_t)(e.row_map ? e.row_map[m0c + j] : m0c + j) * e.ldy + n] = v[j];
         }
     } else if (KIND == EPI_RESID) {
         const int n = nt * 128 + n_local;

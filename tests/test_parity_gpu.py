@@ -69,16 +69,18 @@ def test_config1_generate_is_lossless(cuda_device):
     assert 1.0 <= st.mean_tau <= cfg.block_size
 
 
-@pytest.mark.parametrize("case", ["block16", "moe", "moe_bucketed", "mha_hd128", "chunked_prefill", "batch3", "wide",
-                                  "wide_batch2"])
-def test_bf16_variants_replay(cuda_device, case):
+@pytest.mark.parametrize("case", ["block16", "moe", "moe_bucketed", "moe_stream", "mha_hd128", "chunked_prefill",
+                                  "batch3", "wide", "wide_batch2"])
+def test_bf16_variants_replay(cuda_device, case, monkeypatch):
     kw = dict(dtype="bf16")
+    if case == "moe_stream":  # the CUDA-core weight-streaming expert kernels instead of the grouped projections
+        monkeypatch.setenv("DFLASH_MOE_STREAM", "1")
     prompts_n, lens, chunk = 1, [40], 0
     if case == "block16":
         kw.update(block=16)
     if case == "moe":
         kw.update(moe=True)                   # expert FFN 64: CUDA-core expert kernel
-    if case == "moe_bucketed":
+    if case in ("moe_bucketed", "moe_stream"):
         kw.update(moe=True, expert_ffn=256)   # bucketed experts (hidden and expert FFN multiples of 256)
     if case == "mha_hd128":
         kw.update(nq=2, nkv=2, hd=128)
