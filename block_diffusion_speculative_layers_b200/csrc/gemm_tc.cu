@@ -125,7 +125,7 @@ __device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a
 }
 
 template <int TM, int KIND, bool F8>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcParams p_in,
                    Epi<bf16> e_in, int stages) {
     TcParams p = p_in;
@@ -196,14 +196,14 @@ __global__ void __launch_bounds__(NT, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], F8 ? 5 : 1);  // F8: four converter warps + the MMA commit
+            mbar_init(&empty[s], F8 ? F8_CONV_WARPS + 1 : 1);  // F8: the converter warps + the MMA commit
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
         mbar_init(&acc_empty[0], 4);
         mbar_init(&acc_empty[1], 4);
         for (int s = 0; s < F8_ASTAGES; ++s) {
-            mbar_init(&a_conv[s], 4);
+            mbar_init(&a_conv[s], F8_CONV_WARPS);
             mbar_init(&a_free[s], 1);
         }
         if (F8)
@@ -225,6 +225,50 @@ __global__ void __launch_bounds__(NT, 1)
     // shared memory (arrive now; the epilogue warps wait before their first push)
     if (split) cluster_arrive_relaxed();
     pdl_trigger();
+
+    // F8: widen the weight stages into tensor memory.  Converter warps 2..5 take
+    // K 0..63 of every stage, warps 6..9 K 64..127; thread = weight row (the
+    // TMEM lane quarter of warp w is w % 4).  The codes do not depend on the
+    // previous kernel: this runs before the wait for it.
+    auto convert_f8 = [&](int half) {
+        const int q = warp & 3;
+        const int n_local = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const int rr = n_local & 63;  // row within its 64-row box
+        bool dead = false;
+        for (int kk = 0; kk < nk; ++kk) {
+            const int s = kk % stages, sa = kk % F8_ASTAGES;
+            if (!dead && !mbar_wait(&full[s], (kk / stages) & 1, p.err)) dead = true;
+            if (!dead && kk >= F8_ASTAGES && !mbar_wait(&a_free[sa], ((kk / F8_ASTAGES) - 1) & 1, p.err)) dead = true;
+            const uint8_t *row = sA + (size_t)s * A_ST + (n_local >> 6) * (A_ST / 2) + rr * 128;
+            uint32_t w[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int chunk = half * 4 + c;  // 16 codes = K 16*chunk .. +15, 128-byte swizzle
+                const uint4 v = dead ? make_uint4(0, 0, 0, 0)
+                                     : *reinterpret_cast<const uint4 *>(row + (((chunk ^ rr) & 7) << 4));
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+                if (p.f8_int_conv) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) e4m3x4_to_bf16_int(u[j], w[c * 8 + 2 * j], w[c * 8 + 2 * j + 1]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
+                        w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
+                    }
+                }
+            }
+            tmem_st32(tmem_a + lane_base + (uint32_t)(sa * 64 + half * 32), w);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&a_conv[sa]);
+                mbar_arrive(&empty[s]);
+            }
+        }
+    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -345,53 +389,14 @@ __global__ void __launch_bounds__(NT, 1)
                 mma_commit(&acc_full[b]);
             }
         }
+    } else if (warp >= 6) {
+        // ---------------- F8: the second half of the converter warps ----------------
+        if constexpr (F8) convert_f8(1);
     } else {
         // ---------------- epilogue warps 2..5 ----------------
         const int q = warp & 3;
         const int n_local = q * 32 + lane;
-        if constexpr (F8) {
-            // ---- convert the weight stages into tensor memory (thread = weight row n_local) ----
-            // The codes do not depend on the previous kernel: this runs before the wait for it.
-            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-            const int rr = n_local & 63;  // row within its 64-row box
-            bool dead = false;
-            for (int kk = 0; kk < nk; ++kk) {
-                const int s = kk % stages, sa = kk % F8_ASTAGES;
-                if (!dead && !mbar_wait(&full[s], (kk / stages) & 1, p.err)) dead = true;
-                if (!dead && kk >= F8_ASTAGES && !mbar_wait(&a_free[sa], ((kk / F8_ASTAGES) - 1) & 1, p.err))
-                    dead = true;
-                const uint8_t *row = sA + (size_t)s * A_ST + (n_local >> 6) * (A_ST / 2) + rr * 128;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {  // 64 K per tcgen05.st of 32 columns
-                    uint32_t w[32];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int chunk = h * 4 + c;  // 16 codes = K 16*chunk .. +15, 128-byte swizzle
-                        const uint4 v = dead ? make_uint4(0, 0, 0, 0)
-                                             : *reinterpret_cast<const uint4 *>(row + (((chunk ^ rr) & 7) << 4));
-                        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-                        if (p.f8_int_conv) {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) e4m3x4_to_bf16_int(u[j], w[c * 8 + 2 * j], w[c * 8 + 2 * j + 1]);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
-                                w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
-                            }
-                        }
-                    }
-                    tmem_st32(tmem_a + lane_base + (uint32_t)(sa * 64 + h * 32), w);
-                }
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&a_conv[sa]);
-                    mbar_arrive(&empty[s]);
-                }
-            }
-        }
+        if constexpr (F8) convert_f8(0);
         if (p.dep_ctr) {
             if (threadIdx.x == 64) dep_wait(p.dep_ctr, p.dep_target, p.err);
             epi_bar();
@@ -472,9 +477,9 @@ __global__ void __launch_bounds__(NT, 1)
         // the pushes of every CTA are visible after the barrier (release / acquire);
         // afterwards no CTA touches another's shared memory, so one barrier suffices
         __syncwarp();
-        if (warp < 2) cluster_wait();  // the epilogue warps waited before pushing
+        if (warp < 2 || warp >= 6) cluster_wait();  // the epilogue warps waited before pushing
         cluster_sync_all();
-        if (warp >= 2) {
+        if (warp >= 2 && warp < 6) {
             const int q = warp & 3;
             const int n_local = q * 32 + lane;
             const int nt = blockIdx.x, mt = blockIdx.y;
@@ -661,7 +666,7 @@ static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcPara
     ensure_smem_attr((const void *)kern);
     (void)grid_x;
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-    launch_k(kern, grid, dim3(tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
+    launch_k(kern, grid, dim3(F8 ? tc::NT_F8 : tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
 }
 
 template <int TM, bool F8>

@@ -18,6 +18,8 @@ constexpr int F8_ASTAGES = 2;          // FP8 weights: bf16 A stages in tensor m
 // tensor-memory columns to allocate for n used columns: a power of two >= 32
 __host__ __device__ constexpr int tmem_cols_for(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 constexpr int NT = 192;
+constexpr int F8_CONV_WARPS = 8;         // FP8: warps 2..9 widen the codes (two per TMEM lane quarter)
+constexpr int NT_F8 = 32 * (2 + F8_CONV_WARPS);
 constexpr int CH = 16;                 // accumulator columns per epilogue chunk
 constexpr int STG_LD = CH + 1;
 constexpr unsigned long long WAIT_NS = 2000000000ull;
