@@ -104,6 +104,28 @@ __device__ __forceinline__ void tma_box(void *dst, const CUtensorMap *map, int d
             : "memory");
 }
 
+// L2 prefetch of the same box (no shared memory written, no barrier)
+__device__ __forceinline__ void tma_box_prefetch(const CUtensorMap *map, int d0, int key, int sh, int layer, bool five) {
+    if (five)
+        asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];" ::"l"(
+                         reinterpret_cast<uint64_t>(map)),
+                     "r"(d0), "r"(key), "r"(sh), "r"(layer), "r"(0)
+                     : "memory");
+    else
+        asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                         reinterpret_cast<uint64_t>(map)),
+                     "r"(d0), "r"(key), "r"(sh), "r"(layer)
+                     : "memory");
+}
+
+// this CTA's key tiles [t0, t1) of a query tile whose longest row sees nk_max keys
+__device__ __forceinline__ void split_range(int nk_max, int KT, int S, int split, int &t0, int &t1) {
+    const int ntk = (nk_max + KT - 1) / KT;
+    const int per = (ntk + S - 1) / S;
+    t0 = min(ntk, split * per);
+    t1 = min(ntk, t0 + per);
+}
+
 __device__ __forceinline__ void ldm_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3, uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -208,8 +230,6 @@ __global__ void __launch_bounds__(NTH, 2) attn_tma_kernel(const __grid_constant_
     // every CTA of the cluster has started before any pushes into another's shared memory
     if (S > 1) cluster_arrive_relaxed();
     pdl_trigger();
-    __syncthreads();
-    pdl_wait();  // q, K and V come from the projection before this kernel
 
     const int tile = blockIdx.x, hgrp = blockIdx.y, split = blockIdx.z;
     const int grp = a.nq / a.nkv;
@@ -217,14 +237,38 @@ __global__ void __launch_bounds__(NTH, 2) attn_tma_kernel(const __grid_constant_
     const int kvh = h0 / grp;
     const int r0 = tile * a.rows_per_tile;
     const int nrows = min(a.rows_per_tile, a.R - r0);
+    if (warp == NCW) {
+        // While the projection before this kernel finishes: pull this CTA's K/V
+        // tiles and the row metadata into L2.  The metadata read here (through
+        // L2, no L1 line) may predate this pass; it only steers the prefetch.
+        // The K/V rows the projection is still writing reach L2 after their
+        // prefetch and replace it there, so the loads below see them.
+        int nk_s = lane < nrows ? __ldcg(&a.meta[r0 + lane].nk) : 0;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) nk_s = max(nk_s, __shfl_xor_sync(0xffffffffu, nk_s, o2));
+        const int seq_s = __ldcg(&a.meta[r0].seq);
+        nk_s = min(max(nk_s, 0), a.max_len);
+        if (seq_s >= 0 && seq_s < a.n_seq) {
+            int p0, p1;
+            split_range(nk_s, KT, S, split, p0, p1);
+            const int sh = seq_s * a.nkv + kvh;
+            // lane j: tile p0 + j / (2 * NBOX), box (j / 2) % NBOX, K (even j) or V (odd j)
+            for (int j = lane; j < (p1 - p0) * 2 * NBOX; j += 32) {
+                const int t = p0 + j / (2 * NBOX), b = (j / 2) % NBOX;
+                tma_box_prefetch((j & 1) ? &tmV : &tmK, 64 * b, t * KT, sh, a.layer, SPLIT);
+            }
+        }
+    }
+    __syncthreads();
+    pdl_wait();  // q, K and V come from the projection before this kernel
+
     // longest visible key range of the tile's rows (<= 16 rows), the same in every lane
     int nk_max = lane < nrows ? a.meta[r0 + lane].nk : 0;
 #pragma unroll
     for (int o2 = 16; o2 > 0; o2 >>= 1) nk_max = max(nk_max, __shfl_xor_sync(0xffffffffu, nk_max, o2));
     const int seq = a.meta[r0].seq;
-    const int ntk = (nk_max + KT - 1) / KT;
-    const int per = (ntk + S - 1) / S;
-    const int t0 = min(ntk, split * per), t1 = min(ntk, t0 + per);
+    int t0, t1;
+    split_range(nk_max, KT, S, split, t0, t1);
     const int nt = t1 - t0;
 
     if (warp == NCW) {

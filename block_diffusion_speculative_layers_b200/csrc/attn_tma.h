@@ -16,6 +16,7 @@ struct AttnTmaArgs {
     int ldq = 0;
     const RowMeta *meta = nullptr;  // per row: sequence slot, position, visible keys nk
     int R = 0, rows_per_tile = 16, nq = 0, nkv = 0, max_len = 0;
+    int n_seq = 0;                  // sequence slots of the K/V caches
     int layer = 0;                  // layer of the K/V maps
     float scale_log2 = 0.f;         // log2(e) / sqrt(hd)
     bf16 *out = nullptr;            // [R][ldo] (low plane lo elements on)

@@ -579,7 +579,6 @@ class Engine : public EngineBase {
         // weight stages a projection prefetches into L2 beyond its shared-memory ring
         tc.l2_ahead = env_int("DFLASH_TC_L2_AHEAD");
         tc.tune_tm_max = env_int("DFLASH_TC_TM_MAX");
-        tc.f8_int_conv = env_int("DFLASH_F8_INT_CONV");
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);
         tc.keep_logits = c.keep_logits;  // plus while sampling (sampling_changed)
@@ -789,6 +788,7 @@ class Engine : public EngineBase {
                     a.nq = m.n_q_heads;
                     a.nkv = m.n_kv_heads;
                     a.max_len = c.max_len;
+                    a.n_seq = c.max_batch;
                     a.layer = layer;
                     a.scale_log2 = 1.4426950408889634f / sqrtf((float)m.head_dim);
                     a.out = (bf16 *)out;

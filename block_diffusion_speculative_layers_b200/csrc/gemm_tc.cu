@@ -18,6 +18,7 @@
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
 // records an error bit and drains.
 #include <cudaTypedefs.h>
+#include <cuda_fp8.h>
 
 #include <algorithm>
 #include <type_traits>
@@ -45,107 +46,91 @@ namespace tc {
 // TMEM accumulators (the epilogue of one tile overlapping the MMAs of the
 // next); the host policy does not use that form at present.
 // FP8 weights (F8): the weight tile arrives as E4M3 codes, 128 rows x 128 K
-// (16 KB, one TMA box per 64 rows), half the bytes of bf16.  During the main
-// loop the four epilogue warps convert it -- thread = weight row -- to bf16
-// (exact: every E4M3 value is a bf16 value) and write it into tensor memory
-// with tcgen05.st; tcgen05.mma then reads the A operand from tensor memory and
-// the activation rows from shared memory as before.  Each weight row's fp32
-// scale multiplies its accumulator before the epilogue.  Rings: raw stages in
-// shared memory (codes + the activation tiles of the same 128 K), released by
-// the converters and the MMA commit together; A stages in tensor memory,
-// released by the MMA commit.
+// (16 KB, one TMA box per 64 rows), half the bytes of bf16, and goes to the
+// tensor cores as it is: tcgen05.mma kind::mxf8f6f4 with block scales.  The
+// activation tile of the same 128 K arrives as bf16 (both planes) and the four
+// epilogue warps, during the main loop, rewrite it as F8_PLANES E4M3 planes
+// with one power-of-two (UE8M0) scale per 32 values of a row and plane, the
+// MX block-scaled form: plane p holds what planes 0..p-1 left over, so the
+// planes sum to the value up to 2^-16 of its block's largest magnitude.  The
+// planes are the N operand (N = F8_PLANES * TM), their scales go to tensor
+// memory (tcgen05.st), the weight rows' block scales are all 1 and each weight
+// row's fp32 scale multiplies the plane-summed accumulator in the epilogue.
+// Rings: stages in shared memory (codes + the bf16 activation tiles), released
+// by the quantiser warps and the MMA commit together; quantised slots (planes
+// in shared memory, scales in tensor memory), released by the MMA commit.
 
-// Two E4M3 codes (low byte first) -> two bf16 values, exactly: the codes go to
-// f16 with the hardware conversion (exact), then each f16 half, always normal
-// or zero here, moves to bf16 by rebiasing the exponent (15 -> 127) and
-// dropping three mantissa bits that are zero.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t c) {
-    uint32_t f;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f) : "h"(c));
-    const uint32_t t = (f >> 3) & 0x0FFF0FFFu;       // exponent and 7 mantissa bits of each half
-    const uint32_t nz = __vcmpne2(t, 0u);            // 0xFFFF for nonzero halves
-    return ((t + 0x38003800u) & nz) | (f & 0x80008000u);
+// Smallest E with m * 2^-E <= 448 (the largest E4M3 magnitude) for m > 0,
+// kept inside [-126, 126]; 0 for m == 0.  m = 1.f * 2^x: E = x - 8 unless the
+// fraction is above 0.75 (then m / 2^(x-8) would pass 448).
+__device__ __forceinline__ int mx_exp(float m) {
+    const uint32_t b = __float_as_uint(m);
+    const int e = (int)(b >> 23) - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    return m > 0.f ? min(126, max(-126, e)) : 0;
 }
 
-// Four E4M3 codes (byte j of w) -> bf16 pairs (codes 0,1) and (codes 2,3) with
-// integer operations only.  Normal codes: the sign moves to bit 15 and the
-// 7 exponent/mantissa bits shift by 4 with the exponent rebiased by 120
-// (7 -> 127), exactly.  Codes with a zero exponent field (zero, subnormals
-// m * 2^-9) -- rare in scaled weights -- take an exact per-byte path.
-__device__ __noinline__ uint32_t e4m3x2_small_to_bf16x2(uint32_t pair) {
-    // pair = b1 << 16 | b0
-    uint32_t out = 0;
+// MX planes of 16 values, half of a 32-value block whose other half sits in
+// lane ^ 1.  Plane p: E = mx_exp(block max of what is left), codes of
+// left * 2^-E rounded to nearest E4M3 (never saturating: |left * 2^-E| <= 448),
+// then left -= code * 2^E, which is exact.  code[p] holds the 16 codes in
+// order (two per 16-bit half, the first in the low byte), ex[p] the exponent.
+template <int P>
+__device__ __forceinline__ void mx_planes16(float (&r)[16], uint4 (&code)[P], int (&ex)[P]) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const uint32_t b = (pair >> (16 * h)) & 0xFFu;
-        uint32_t v;
-        if (b & 0x78u) {
-            v = ((b & 0x7Fu) << 4) + 0x3C00u;
-        } else {
-            const uint32_t m = b & 7u;
-            // m = 0: 0; 1: 0x3B00; 2: 0x3B80; 3: 0x3BC0; 4..7: 0x3C00 + 0x20 * (m - 4)
-            v = m == 0 ? 0u : m == 1 ? 0x3B00u : m == 2 ? 0x3B80u : m == 3 ? 0x3BC0u : 0x3C00u + 0x20u * (m - 4);
+    for (int p = 0; p < P; ++p) {
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(r[i]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        const int E = mx_exp(m);
+        ex[p] = E;
+        const float inv = __uint_as_float((uint32_t)(127 - E) << 23), sc = __uint_as_float((uint32_t)(127 + E) << 23);
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const __nv_fp8x2_storage_t c2 =
+                __nv_cvt_float2_to_fp8x2(make_float2(r[2 * q] * inv, r[2 * q + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+            const float2 d = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(c2, __NV_E4M3)));
+            r[2 * q] -= d.x * sc;
+            r[2 * q + 1] -= d.y * sc;
+            if (q & 1) w[q >> 1] |= (uint32_t)c2 << 16;
+            else w[q >> 1] = (uint32_t)c2;
         }
-        out |= (v | ((b & 0x80u) << 8)) << (16 * h);
-    }
-    return out;
-}
-
-__device__ __forceinline__ void e4m3x4_to_bf16_int(uint32_t w, uint32_t &r0, uint32_t &r1) {
-    const uint32_t p0 = __byte_perm(w, 0u, 0x4140u);  // b1 << 16 | b0
-    const uint32_t p1 = __byte_perm(w, 0u, 0x4342u);  // b3 << 16 | b2
-    r0 = ((p0 & 0x007F007Fu) * 16u + 0x3C003C00u) | ((p0 << 8) & 0x80008000u);
-    r1 = ((p1 & 0x007F007Fu) * 16u + 0x3C003C00u) | ((p1 << 8) & 0x80008000u);
-    const uint32_t t = w & 0x78787878u;  // exponent fields: a zero byte marks zero / subnormal codes
-    if ((t - 0x01010101u) & ~t & 0x80808080u) {
-        r0 = e4m3x2_small_to_bf16x2(p0);
-        r1 = e4m3x2_small_to_bf16x2(p1);
+        code[p] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
-// bf16 x bf16 -> fp32 with the A operand (128 x 16) in tensor memory
-__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
-                                                uint32_t acc) {
+// E4M3 x E4M3 -> fp32 with UE8M0 block scales from tensor memory (one per 32 K
+// of each A row and B column), M = 128, K = 32
+__device__ __forceinline__ void mma_mx(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc));
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
 }
 
-template <int TM, int KIND, bool F8>
-__global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcParams p_in,
-                   Epi<bf16> e_in, int stages) {
-    TcParams p = p_in;
-    Epi<bf16> e = e_in;
-    // grouped (MoE experts): this CTA's expert, rows and weight rows
-    const bool grouped = p.g_off != nullptr;
-    int g_row0 = 0, g_wrow0 = 0;
-    if (grouped) {
-        pdl_wait();  // the expert lists come from the bucketing kernel
-        const int ex = p.g_touched[blockIdx.y];
-        if (ex < 0) return;
-        const int r0 = p.g_off[ex], m0 = (int)blockIdx.z * TM;
-        const int nr = p.g_off[ex + 1] - r0;
-        if (m0 >= nr) return;
-        p.M = min(TM, nr - m0);
-        g_row0 = r0 + m0;
-        g_wrow0 = ex * p.g_wrows;
-        if (KIND == EPI_SWIGLU) e.h += (size_t)g_row0 * p.swiglu_F;
-        if (KIND == EPI_STORE && p.g_list) e.row_map = p.g_list + g_row0;
-    }
+// Instruction descriptor of mma_mx: E4M3 A and B, both K-major, UE8M0 scales,
+// M = 128, N = n; scale byte `kb` of the A and B scale words (the 32-K block
+// within a 128-K stage).
+__host__ __device__ constexpr uint32_t idesc_mx(int n, int kb) {
+    return ((uint32_t)kb << 4) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(128 >> 4) << 24) |
+           ((uint32_t)kb << 29);
+}
+
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+// The kernel body.  p and e are the launch's parameters (ungrouped launches
+// read them in place, without a copy) or a grouped CTA's adjusted copies.
+template <int TM, int KIND, bool F8, bool GR>
+__device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUtensorMap &tmX, const TcParams &p,
+                                             const Epi<bf16> &e, int stages, int g_row0, int g_wrow0) {
+    constexpr bool grouped = GR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int B_BYTES = TM * 128 * p.planes;  // activation tile(s) of 64 K
@@ -153,12 +138,15 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
     const int A_ST = F8 ? F8_A_BYTES : A_BYTES, B_ST = F8 ? 2 * B_BYTES : B_BYTES;
     // two planes and TM <= 128: one MMA with N = 2*TM covers the hi and lo rows
     // (they are contiguous in the stage), accumulating into 2*TM columns
-    const bool wide = p.planes == 2 && TM <= 128;
+    const bool wide = !F8 && p.planes == 2 && TM <= 128;
     const int lo_col = wide ? TM : 0;
-    const int NC1 = max(32, wide ? 2 * TM : TM);  // TMEM columns of one accumulator
+    // F8: N = F8_PLANES * TM quantised rows (plane-major)
+    const int NC1 = max(32, F8 ? F8_PLANES * TM : wide ? 2 * TM : TM);  // TMEM columns of one accumulator
+    constexpr int QB = F8 ? F8_PLANES * TM * 128 : 0;  // one quantised slot: planes x TM rows x 128 K codes
     uint8_t *sA = smem;
     uint8_t *sB = smem + (size_t)stages * A_ST;
-    float *stg = (float *)(sB + (size_t)stages * B_ST);
+    uint8_t *sQ = sB + (size_t)stages * B_ST;  // F8: [F8_QSTAGES] quantised slots (1024-byte multiples)
+    float *stg = (float *)(sQ + (F8 ? F8_QSTAGES * QB : 0));
     float2 *red = (float2 *)(stg + 128 * STG_LD);
     RowMeta *smeta = (RowMeta *)(red + 4 * CH);
     float *rsc = (float *)(smeta + CH);       // [RS_MAX] row scales of the folded norm
@@ -166,12 +154,14 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
     uint64_t *empty = full + stages;
     uint64_t *acc_full = empty + stages;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
-    uint64_t *a_conv = acc_empty + 2;      // [F8_ASTAGES] A stage converted into tensor memory
-    uint64_t *a_free = a_conv + F8_ASTAGES;  // [F8_ASTAGES] A stage read by the MMAs
-    // F8: the activation tiles of a stage complete on their own barrier, so the
-    // weight codes (full[]) can be converted before the previous kernel is done
-    uint64_t *full_b = a_free + F8_ASTAGES;  // [stages]
-    uint32_t *tmem_slot = (uint32_t *)(full_b + (F8 ? stages : 0));
+    uint64_t *q_full = acc_empty + 2;       // [F8_QSTAGES] quantised slot written
+    uint64_t *q_free = q_full + F8_QSTAGES;  // [F8_QSTAGES] quantised slot read by the MMAs
+    // F8: the activation tiles of a stage complete on their own barrier (the
+    // quantiser waits for them only; the MMA for the codes and the slot)
+    uint64_t *full_b = q_free + F8_QSTAGES;  // [stages]
+    // F8: scale bytes of a quantised slot, [F8_QSTAGES][F8_PLANES * TM][4 blocks of 32 K]
+    uint8_t *sSF = (uint8_t *)(full_b + (F8 ? stages : 0));
+    uint32_t *tmem_slot = (uint32_t *)(sSF + (F8 ? F8_QSTAGES * F8_PLANES * TM * 4 : 0));
     // split-K receive buffer [S][128][cpr] (16-byte aligned, after the fixed area)
     float *recv = (float *)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
     EpiIn pre;
@@ -190,21 +180,25 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
     const int kb = split ? blockIdx.z * k_per : 0;
     const int ke = split ? min(p.k_steps, kb + k_per) : p.k_steps;
     const int nk = max(0, ke - kb);
-    const int a_cols = F8 ? F8_ASTAGES * 64 : 0;  // tensor-memory A stages (64 columns = 128 bf16 K each)
-    const int ncols = tmem_cols_for((persistent ? 2 * NC1 : NC1) + a_cols);
+    // F8: after the accumulator, the weights' scale words (4 columns: row m at
+    // lane m, column m / 32) and one 4-column group per quantised slot (plane row
+    // n at lane n % 32 of every lane quarter, column n / 32; byte b of a word =
+    // the scale of 32-K block b of the stage)
+    const int sf_cols = F8 ? 4 + 4 * F8_QSTAGES : 0;
+    const int ncols = tmem_cols_for((persistent ? 2 * NC1 : NC1) + sf_cols);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], F8 ? F8_CONV_WARPS + 1 : 1);  // F8: the converter warps + the MMA commit
+            mbar_init(&empty[s], F8 ? 5 : 1);  // F8: the four quantiser warps + the MMA commit
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
         mbar_init(&acc_empty[0], 4);
         mbar_init(&acc_empty[1], 4);
-        for (int s = 0; s < F8_ASTAGES; ++s) {
-            mbar_init(&a_conv[s], F8_CONV_WARPS);
-            mbar_init(&a_free[s], 1);
+        for (int s = 0; s < F8_QSTAGES; ++s) {
+            mbar_init(&q_full[s], 4);
+            mbar_init(&q_free[s], 1);
         }
         if (F8)
             for (int s = 0; s < stages; ++s) mbar_init(&full_b[s], 1);
@@ -220,51 +214,80 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_a = tmem + (uint32_t)(persistent ? 2 * NC1 : NC1);  // F8: A stages after the accumulator
+    const uint32_t tmem_sfa = tmem + (uint32_t)NC1, tmem_sfb = tmem_sfa + 4u;  // F8 scale columns
     // K split: every CTA of the cluster has started before any pushes into another's
     // shared memory (arrive now; the epilogue warps wait before their first push)
     if (split) cluster_arrive_relaxed();
     pdl_trigger();
 
-    // F8: widen the weight stages into tensor memory.  Converter warps 2..5 take
-    // K 0..63 of every stage, warps 6..9 K 64..127; thread = weight row (the
-    // TMEM lane quarter of warp w is w % 4).  The codes do not depend on the
-    // previous kernel: this runs before the wait for it.
-    auto convert_f8 = [&](int half) {
+    // F8: quantise the activation tile of every stage into MX planes (warps
+    // 2..5, 128 threads).  Thread = (row j, 32-K block, half): 16 values, the
+    // block's other half in lane ^ 1.  Codes go to the slot in the 128-byte
+    // swizzled layout of the MMA's N operand; scale bytes go to sSF and then,
+    // as one word per plane row, into tensor memory, copied into every lane
+    // quarter (each quarter of the MMA reads its own copy).
+    auto quantise = [&] {
+        const int t = threadIdx.x - 64;  // 0..127
         const int q = warp & 3;
-        const int n_local = q * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const int rr = n_local & 63;  // row within its 64-row box
+        // the weights' block scales: 1.0 (UE8M0 127) in every byte
+        tmem_st4(tmem_sfa + ((uint32_t)(q * 32) << 16), 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
         bool dead = false;
         for (int kk = 0; kk < nk; ++kk) {
-            const int s = kk % stages, sa = kk % F8_ASTAGES;
-            if (!dead && !mbar_wait(&full[s], (kk / stages) & 1, p.err)) dead = true;
-            if (!dead && kk >= F8_ASTAGES && !mbar_wait(&a_free[sa], ((kk / F8_ASTAGES) - 1) & 1, p.err)) dead = true;
-            const uint8_t *row = sA + (size_t)s * A_ST + (n_local >> 6) * (A_ST / 2) + rr * 128;
-            uint32_t w[32];
+            const int s = kk % stages, sq = kk % F8_QSTAGES;
+            if (!dead && !mbar_wait(&full_b[s], (kk / stages) & 1, p.err)) dead = true;
+            if (!dead && kk >= F8_QSTAGES && !mbar_wait(&q_free[sq], ((kk / F8_QSTAGES) - 1) & 1, p.err)) dead = true;
+            const uint8_t *xb = sB + (size_t)s * B_ST;
+            uint8_t *qs = sQ + (size_t)sq * QB;
+            uint8_t *sf = sSF + sq * (F8_PLANES * TM * 4);
+#pragma unroll 1
+            for (int u = t; u < TM * 8; u += 128) {
+                const int j = u >> 3, blk = (u >> 1) & 3, h2 = u & 1;
+                const int k0 = blk * 32 + h2 * 16;                 // first K of the 16 values in the stage
+                const uint8_t *row = xb + (k0 >> 6) * (TM * 128 * p.planes) + j * 128;
+                const int c0 = (k0 & 63) >> 3;                     // first 16-byte chunk of 8 values
+                float r[16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int chunk = half * 4 + c;  // 16 codes = K 16*chunk .. +15, 128-byte swizzle
-                const uint4 v = dead ? make_uint4(0, 0, 0, 0)
-                                     : *reinterpret_cast<const uint4 *>(row + (((chunk ^ rr) & 7) << 4));
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-                if (p.f8_int_conv) {
+                for (int h = 0; h < 2; ++h) {
+                    const int off = (((c0 + h) ^ j) & 7) << 4;
+                    const uint4 hv = dead ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4 *>(row + off);
+                    uint4 lv = make_uint4(0, 0, 0, 0);
+                    if (p.planes == 2 && !dead) lv = *reinterpret_cast<const uint4 *>(row + TM * 128 + off);
+                    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) e4m3x4_to_bf16_int(u[j], w[c * 8 + 2 * j], w[c * 8 + 2 * j + 1]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        w[c * 8 + 2 * j] = e4m3x2_to_bf16x2((uint16_t)(u[j] & 0xFFFFu));
-                        w[c * 8 + 2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(u[j] >> 16));
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hw[i]));
+                        const float2 lf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&lw[i]));
+                        r[h * 8 + 2 * i] = hf.x + lf.x;
+                        r[h * 8 + 2 * i + 1] = hf.y + lf.y;
                     }
                 }
+                uint4 code[F8_PLANES];
+                int ex[F8_PLANES];
+                mx_planes16<F8_PLANES>(r, code, ex);
+#pragma unroll
+                for (int pl = 0; pl < F8_PLANES; ++pl) {
+                    const int rq = pl * TM + j;  // row of the N operand
+                    *reinterpret_cast<uint4 *>(qs + rq * 128 + ((((blk * 2 + h2) ^ rq) & 7) << 4)) = code[pl];
+                    if (h2 == 0) sf[rq * 4 + blk] = (uint8_t)(ex[pl] + 127);
+                }
             }
-            tmem_st32(tmem_a + lane_base + (uint32_t)(sa * 64 + half * 32), w);
+            // codes written by the generic proxy, read by the tensor cores
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            epi_bar();  // every scale byte of the slot is in sSF
+            {
+                // plane row n = 32 c + lane: word c of this lane (up to 4 words; TM <= 32)
+                uint32_t w4[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    w4[c] = 32 * c < F8_PLANES * TM ? *reinterpret_cast<const uint32_t *>(sf + (32 * c + lane) * 4)
+                                                    : 0x7F7F7F7Fu;
+                tmem_st4(tmem_sfb + (uint32_t)(sq * 4) + ((uint32_t)(q * 32) << 16), w4[0], w4[1], w4[2], w4[3]);
+            }
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&a_conv[sa]);
+                mbar_arrive(&q_full[sq]);
                 mbar_arrive(&empty[s]);
             }
         }
@@ -348,25 +371,23 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const int s = it % stages;
                     if constexpr (F8) {
-                        const int sa = it % F8_ASTAGES;
-                        if (!mbar_wait(&full_b[s], (it / stages) & 1, p.err) ||
-                            !mbar_wait(&a_conv[sa], (it / F8_ASTAGES) & 1, p.err)) {
+                        const int sq = it % F8_QSTAGES;
+                        if (!mbar_wait(&full[s], (it / stages) & 1, p.err) ||
+                            !mbar_wait(&q_full[sq], (it / F8_QSTAGES) & 1, p.err)) {
                             ok = false;
                             break;
                         }
                         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                        const uint32_t ta = tmem_a + (uint32_t)(sa * 64);
+                        const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_ST));
+                        const uint64_t db = sw128_desc(smem_u32(sQ + (size_t)sq * QB));
+                        const uint32_t sfb = tmem_sfb + (uint32_t)(sq * 4);
 #pragma unroll
-                        for (int k8 = 0; k8 < 8; ++k8) {  // 8 x K=16 over the stage's 128 K
-                            const uint64_t db =
-                                sw128_desc(smem_u32(sB + (size_t)s * B_ST + (k8 >> 2) * B_BYTES)) + (uint64_t)((k8 & 3) * 2);
-                            mma_bf16_tmem_a(acc, ta + (uint32_t)(k8 * 8), db, idesc, (kk > 0 || k8 > 0) ? 1u : 0u);
-                            if (p.planes == 2 && !wide)
-                                mma_bf16_tmem_a(acc, ta + (uint32_t)(k8 * 8), db + (uint64_t)((TM * 128) >> 4), idesc,
-                                                1u);
-                        }
+                        for (int k32 = 0; k32 < 4; ++k32)  // 4 x K=32 over the stage's 128 K (+32 bytes each)
+                            mma_mx(acc, da + (uint64_t)(k32 * 2), db + (uint64_t)(k32 * 2),
+                                   idesc_mx(F8_PLANES * TM, k32), tmem_sfa | ((uint32_t)k32 << 30),
+                                   sfb | ((uint32_t)k32 << 30), (kk > 0 || k32 > 0) ? 1u : 0u);
                         mma_commit(&empty[s]);
-                        mma_commit(&a_free[sa]);
+                        mma_commit(&q_free[sq]);
                     } else {
                         if (!mbar_wait(&full[s], (it / stages) & 1, p.err)) {
                             ok = false;
@@ -389,14 +410,11 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
                 mma_commit(&acc_full[b]);
             }
         }
-    } else if (warp >= 6) {
-        // ---------------- F8: the second half of the converter warps ----------------
-        if constexpr (F8) convert_f8(1);
     } else {
         // ---------------- epilogue warps 2..5 ----------------
         const int q = warp & 3;
         const int n_local = q * 32 + lane;
-        if constexpr (F8) convert_f8(0);
+        if constexpr (F8) quantise();
         if (p.dep_ctr) {
             if (threadIdx.x == 64) dep_wait(p.dep_ctr, p.dep_target, p.err);
             epi_bar();
@@ -412,6 +430,21 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
             const int rows = p.swiglu_F ? 2 * p.swiglu_F : p.N;
             wsc = row < rows ? p.w_scale[row] : 0.f;
         }
+        // accumulator columns c..c+15 of a tile (F8: summed over the planes)
+        auto load_acc = [&](uint32_t trow, int c, float *v) {
+            if constexpr (F8) {
+                tmem_ld16(trow + (uint32_t)c, v);
+#pragma unroll
+                for (int pl = 1; pl < F8_PLANES; ++pl) {
+                    float t2[16];
+                    tmem_ld16(trow + (uint32_t)(pl * TM + c), t2);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] += t2[j];
+                }
+            } else {
+                acc_ld16(trow, c, lo_col, v);
+            }
+        };
         // K split: CTA `rank` of the cluster reduces and finishes columns [c_begin, c_end)
         const int rank = split ? (int)cluster_rank() : 0;
         const int cpr = split ? split_cols(TM, S) : TM;
@@ -433,7 +466,7 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
             float v[CH];
             if (!split) {
                 for (int c = 0; c < TM; c += CH) {
-                    if (ok) acc_ld16(trow, c, lo_col, v);
+                    if (ok) load_acc(trow, c, v);
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
@@ -456,7 +489,7 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
                 // four columns (one owner, cpr being a multiple of 4) per store
                 cluster_wait();
                 for (int c = 0; c < TM; c += CH) {
-                    if (ok) acc_ld16(trow, c, lo_col, v);
+                    if (ok) load_acc(trow, c, v);
                     else
 #pragma unroll
                         for (int j = 0; j < CH; ++j) v[j] = 0.f;
@@ -477,9 +510,9 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
         // the pushes of every CTA are visible after the barrier (release / acquire);
         // afterwards no CTA touches another's shared memory, so one barrier suffices
         __syncwarp();
-        if (warp < 2 || warp >= 6) cluster_wait();  // the epilogue warps waited before pushing
+        if (warp < 2) cluster_wait();  // the epilogue warps waited before pushing
         cluster_sync_all();
-        if (warp >= 2 && warp < 6) {
+        if (warp >= 2) {
             const int q = warp & 3;
             const int n_local = q * 32 + lane;
             const int nt = blockIdx.x, mt = blockIdx.y;
@@ -522,6 +555,29 @@ __global__ void __launch_bounds__(F8 ? NT_F8 : NT, F8 ? 2 : 1)
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
+    }
+}
+
+template <int TM, int KIND, bool F8, bool GR>
+__global__ void __launch_bounds__(NT, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   const __grid_constant__ TcParams p, const __grid_constant__ Epi<bf16> e, int stages) {
+    if constexpr (GR) {
+        // grouped (MoE experts): this CTA's expert, its rows and weight rows
+        pdl_wait();  // the expert lists come from the bucketing kernel
+        const int ex = p.g_touched[blockIdx.y];
+        if (ex < 0) return;
+        const int r0 = p.g_off[ex], m0 = (int)blockIdx.z * TM;
+        const int nr = p.g_off[ex + 1] - r0;
+        if (m0 >= nr) return;
+        TcParams pg = p;
+        Epi<bf16> eg = e;
+        pg.M = min(TM, nr - m0);
+        if (KIND == EPI_SWIGLU) eg.h += (size_t)(r0 + m0) * p.swiglu_F;
+        if (KIND == EPI_STORE && p.g_list) eg.row_map = p.g_list + r0 + m0;
+        gemm_tc_body<TM, KIND, F8, true>(tmW, tmX, pg, eg, stages, r0 + m0, ex * p.g_wrows);
+    } else {
+        gemm_tc_body<TM, KIND, F8, false>(tmW, tmX, p, e, stages, 0, 0);
     }
 }
 
@@ -662,11 +718,11 @@ const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, in
 template <int TM, int KIND, bool F8>
 static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p, const Epi<bf16> &e,
                       int stages, size_t smem, cudaStream_t s, int grid_x) {
-    auto kern = tc::gemm_tc_kernel<TM, KIND, F8>;
+    auto kern = tc::gemm_tc_kernel<TM, KIND, F8, false>;
     ensure_smem_attr((const void *)kern);
     (void)grid_x;
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-    launch_k(kern, grid, dim3(F8 ? tc::NT_F8 : tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
+    launch_k(kern, grid, dim3(tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
 }
 
 template <int TM, bool F8>
@@ -697,7 +753,9 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
         const int nt = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
         while (TM > 64 && nt * ((M + TM - 1) / TM) < num_sms) TM /= 2;
     }
-    if (f8) TM = std::min(TM, 64);  // FP8: tensor memory holds the A stages too; larger M takes several row tiles
+    // FP8: N = 4 planes x TM <= 128 keeps the accumulator and the scale columns in
+    // 256 TMEM columns (two CTAs per SM); larger M takes several row tiles
+    if (f8) TM = std::min(TM, 32);
     TcParams p;
     memset(&p, 0, sizeof p);
     p.M = M;
@@ -712,10 +770,12 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     p.planes = e.lo ? 2 : 1;
     p.w_scale = w_scale;
     p.l2_ahead = l2_ahead;
-    p.f8_int_conv = f8_int_conv;
     const int stage_bytes = f8 ? tc::F8_A_BYTES + 2 * TM * 128 * p.planes : tc::A_BYTES + TM * 128 * p.planes;
+    // fixed area: alignment, epilogue staging, barriers; FP8 adds the quantised
+    // slots (codes + scale bytes)
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
-                      2 * tc::F8_ASTAGES * 8 + 16 * 8;
+                      2 * tc::F8_QSTAGES * 8 + 16 * 8 +
+                      (f8 ? tc::F8_QSTAGES * tc::F8_PLANES * TM * (128 + 4) : 0);
     // Measured on B200 (decode shapes, M = 16, whole decode iteration): every
     // projection streams best with ~110 KB CTAs, two of which fit on an SM;
     // projections with fewer tiles than that split K over a cluster (up to 8
@@ -723,8 +783,11 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     // rings were faster for a projection timed alone but 0.5 ms per iteration
     // slower in the pipeline; filling one slot per SM was 0.2 ms slower.
     int splits = 1;
-    // the K split aims to fill two ~110 KB CTAs per SM (measured best in the decode pipeline)
-    const int slots = num_sms * (tune_ctas_per_sm > 0 ? tune_ctas_per_sm : 2);
+    // the K split aims to fill two ~110 KB CTAs per SM (measured best in the decode
+    // pipeline), as far as clusters allow: a cluster is placed whole inside one GPC,
+    // and on B200 one wave of these CTAs held 43 clusters of 6 or 32 clusters of 8
+    // (about 256 CTAs, not the 296 slots on paper); 48 clusters of 6 ran as 43 + 5
+    const int slots = tune_ctas_per_sm > 0 ? num_sms * tune_ctas_per_sm : std::min(2 * num_sms, 256);
     if (e.kind != EPI_LOGITS && tiles < slots && p.k_steps >= 4) {
         splits = std::max(1, std::min({8, p.k_steps / 2, slots / std::max(1, tiles)}));
         if (tune_splits > 0) splits = std::min(8, tune_splits);
@@ -756,8 +819,7 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     if (f8) {
         switch (TM) {
             case 16: launch_kind<16, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-            case 32: launch_kind<32, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-            default: launch_kind<64, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            default: launch_kind<32, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
         }
     } else {
         switch (TM) {
@@ -801,7 +863,7 @@ int GemmTC<bf16>::run_grouped(const bf16 *X, int ldx, int n_pairs, const bf16 *W
     p.g_wrows = wrows;
     const int stage_bytes = tc::A_BYTES + TM * 128 * p.planes;
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
-                      2 * tc::F8_ASTAGES * 8 + 16 * 8;
+                      2 * tc::F8_QSTAGES * 8 + 16 * 8;
     const int stages = std::max(2, std::min(16, (112 * 1024 - fixed) / stage_bytes));
     const size_t smem = (size_t)fixed + (size_t)stages * stage_bytes;
     const CUtensorMap *mw = tensor_map(W, E * wrows, K, K, 64);
@@ -812,7 +874,7 @@ int GemmTC<bf16>::run_grouped(const bf16 *X, int ldx, int n_pairs, const bf16 *W
     }
     auto go = [&](auto tm_c) {
         constexpr int T_ = decltype(tm_c)::value;
-        auto kern = swiglu ? tc::gemm_tc_kernel<T_, EPI_SWIGLU, false> : tc::gemm_tc_kernel<T_, EPI_STORE, false>;
+        auto kern = swiglu ? tc::gemm_tc_kernel<T_, EPI_SWIGLU, false, true> : tc::gemm_tc_kernel<T_, EPI_STORE, false, true>;
         ensure_smem_attr((const void *)kern);
         launch_k(kern, dim3(p.n_tiles, E, p.m_tiles), dim3(tc::NT), smem, s, 1, *mw, *mx, p, e, stages);
     };

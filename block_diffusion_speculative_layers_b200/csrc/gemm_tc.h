@@ -39,7 +39,6 @@ struct TcParams {
     int *done_ctr;
     const float *w_scale;   // FP8 weights: fp32 scale of every weight row (the codes' row of W)
     int l2_ahead;           // weight stages prefetched into L2 beyond the shared-memory ring (0: none)
-    int f8_int_conv;        // FP8: widen codes with integer operations instead of the f16 conversion
     // grouped (MoE experts): blockIdx.y = touched-expert slot, blockIdx.z = row tile of
     // that expert; its rows are g_off[e] .. g_off[e+1]-1 of X (expert-grouped order) and
     // its weights rows e*g_wrows .. of W; nullptr g_off = an ordinary projection
@@ -81,7 +80,6 @@ struct GemmTC {
     // of unsplit / K-split launches, CTAs per SM the K split aims to fill
     int tune_splits = 0, tune_smem_kb = 0, tune_split_smem_kb = 0, tune_ctas_per_sm = 0, l2_ahead = 0;
     int tune_tm_max = 0;  // cap on the activation rows of one tile (more row tiles, weights re-read from L2)
-    int f8_int_conv = 0;  // FP8 code widening: 0 hardware f16 conversion + rebias, 1 integer operations
     std::unordered_map<std::string, CUtensorMap> maps;
     // 2-D map of a [rows][cols] bf16 matrix (leading dimension ld), box {64, box_rows};
     // plane_stride > 0: 3-D map over the hi plane and the lo plane plane_stride

@@ -13,13 +13,12 @@ namespace tc {
 constexpr int BK = 64;                 // bf16 K elements per stage = one 128-byte swizzle row
 constexpr int A_BYTES = 128 * BK * 2;  // 16 KB weight tile per stage
 constexpr int F8_A_BYTES = 128 * 128;  // FP8 weights: 128 rows x 128 codes per stage
-constexpr int F8_ASTAGES = 2;          // FP8 weights: bf16 A stages in tensor memory (64 columns each)
+constexpr int F8_QSTAGES = 2;          // FP8 weights: quantised activation slots (shared memory + scale columns)
+constexpr int F8_PLANES = 4;           // FP8 weights: E4M3 planes per activation value (MX block scales)
 
 // tensor-memory columns to allocate for n used columns: a power of two >= 32
 __host__ __device__ constexpr int tmem_cols_for(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 constexpr int NT = 192;
-constexpr int F8_CONV_WARPS = 8;         // FP8: warps 2..9 widen the codes (two per TMEM lane quarter)
-constexpr int NT_F8 = 32 * (2 + F8_CONV_WARPS);
 constexpr int CH = 16;                 // accumulator columns per epilogue chunk
 constexpr int STG_LD = CH + 1;
 constexpr unsigned long long WAIT_NS = 2000000000ull;
