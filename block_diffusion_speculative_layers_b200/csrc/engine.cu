@@ -576,8 +576,6 @@ class Engine : public EngineBase {
         tc.tune_smem_kb = env_int("DFLASH_TC_SMEM_KB");
         tc.tune_split_smem_kb = env_int("DFLASH_TC_SPLIT_SMEM_KB");
         tc.tune_ctas_per_sm = env_int("DFLASH_TC_CTAS_PER_SM");
-        // weight stages a projection prefetches into L2 beyond its shared-memory ring
-        tc.l2_ahead = env_int("DFLASH_TC_L2_AHEAD");
         tc.tune_tm_max = env_int("DFLASH_TC_TM_MAX");
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);

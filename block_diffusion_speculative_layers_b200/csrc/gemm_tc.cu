@@ -331,23 +331,12 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
                     it = pre;
                     first = false;
                 }
-                // L2 prefetch: keep the stages l2_ahead beyond the ring in flight from HBM
-                int pf = kk0;
-                auto prefetch_to = [&](int upto) {
-                    for (; pf < min(nk, upto); ++pf) {
-                        const int kp = (kb + pf) * kstep;
-                        tma_prefetch_2d(&tmW, kp, rowA0);
-                        tma_prefetch_2d(&tmW, kp, rowA1);
-                    }
-                };
-                if (p.l2_ahead > 0) prefetch_to(kk0 + p.l2_ahead);
                 for (int kk = kk0; kk < nk; ++kk, ++it) {
                     const int s = it % stages;
                     if (it >= stages && !mbar_wait(&empty[s], ((it / stages) & 1) ^ 1, p.err)) {
                         abort = true;
                         break;
                     }
-                    if (p.l2_ahead > 0) prefetch_to(kk + 1 + p.l2_ahead);
                     const int k = (kb + kk) * kstep;
                     uint8_t *a = sA + (size_t)s * A_ST;
                     mbar_expect_tx(&full[s], a_tx);
@@ -716,8 +705,8 @@ const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, in
 }
 
 template <int TM, int KIND, bool F8>
-static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p, const Epi<bf16> &e,
-                      int stages, size_t smem, cudaStream_t s, int grid_x) {
+static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p,
+                      const Epi<bf16> &e, int stages, size_t smem, cudaStream_t s, int grid_x) {
     auto kern = tc::gemm_tc_kernel<TM, KIND, F8, false>;
     ensure_smem_attr((const void *)kern);
     (void)grid_x;
@@ -738,11 +727,10 @@ static void launch_kind(int kind, const CUtensorMap *mw, const CUtensorMap *mx, 
     }
 }
 
-template <>
-int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K, const Epi<bf16> &e,
-                      cudaStream_t s, const int *dep_ctr, int dep_target, int *done_ctr, const float *w_scale) {
-    const bool swiglu = e.kind == EPI_SWIGLU;
-    const bool f8 = w_scale != nullptr;
+template <typename T>
+TcPlan GemmTC<T>::plan(int M, int N, int K, int kind, int F, bool f8, int planes) const {
+    const bool swiglu = kind == EPI_SWIGLU;
+    TcPlan pl;
     int TM = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
     if (tune_tm_max >= 16) {
         TM = std::min(TM, tune_tm_max);
@@ -750,27 +738,19 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
         // many activation rows (batched decode, prefill chunks): the largest row tile
         // that still gives every SM a tile; the weight tile is then re-read per row
         // tile, from L2 (measured: one CTA per weight tile left most SMs idle)
-        const int nt = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
+        const int nt = swiglu ? (F + 63) / 64 : (N + 127) / 128;
         while (TM > 64 && nt * ((M + TM - 1) / TM) < num_sms) TM /= 2;
     }
     // FP8: N = 4 planes x TM <= 128 keeps the accumulator and the scale columns in
     // 256 TMEM columns (two CTAs per SM); larger M takes several row tiles
     if (f8) TM = std::min(TM, 32);
-    TcParams p;
-    memset(&p, 0, sizeof p);
-    p.M = M;
-    p.N = N;
-    p.K = K;
-    p.swiglu_F = swiglu ? e.F : 0;
-    p.n_tiles = swiglu ? (e.F + 63) / 64 : (N + 127) / 128;
-    p.m_tiles = (M + TM - 1) / TM;
-    const int kstep = f8 ? 2 * tc::BK : tc::BK;  // K per stage: 128 FP8 codes or 64 bf16 values per weight row
-    p.k_steps = (K + kstep - 1) / kstep;
-    const int tiles = p.n_tiles * p.m_tiles;
-    p.planes = e.lo ? 2 : 1;
-    p.w_scale = w_scale;
-    p.l2_ahead = l2_ahead;
-    const int stage_bytes = f8 ? tc::F8_A_BYTES + 2 * TM * 128 * p.planes : tc::A_BYTES + TM * 128 * p.planes;
+    pl.TM = TM;
+    pl.n_tiles = swiglu ? (F + 63) / 64 : (N + 127) / 128;
+    pl.m_tiles = (M + TM - 1) / TM;
+    pl.kstep = f8 ? 2 * tc::BK : tc::BK;  // K per stage: 128 FP8 codes or 64 bf16 values per weight row
+    pl.k_steps = (K + pl.kstep - 1) / pl.kstep;
+    const int tiles = pl.n_tiles * pl.m_tiles;
+    const int stage_bytes = f8 ? tc::F8_A_BYTES + 2 * TM * 128 * planes : tc::A_BYTES + TM * 128 * planes;
     // fixed area: alignment, epilogue staging, barriers; FP8 adds the quantised
     // slots (codes + scale bytes)
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
@@ -788,20 +768,43 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     // and on B200 one wave of these CTAs held 43 clusters of 6 or 32 clusters of 8
     // (about 256 CTAs, not the 296 slots on paper); 48 clusters of 6 ran as 43 + 5
     const int slots = tune_ctas_per_sm > 0 ? num_sms * tune_ctas_per_sm : std::min(2 * num_sms, 256);
-    if (e.kind != EPI_LOGITS && tiles < slots && p.k_steps >= 4) {
-        splits = std::max(1, std::min({8, p.k_steps / 2, slots / std::max(1, tiles)}));
+    if (kind != EPI_LOGITS && tiles < slots && pl.k_steps >= 4) {
+        splits = std::max(1, std::min({8, pl.k_steps / 2, slots / std::max(1, tiles)}));
         if (tune_splits > 0) splits = std::min(8, tune_splits);
-        const int k_per = (p.k_steps + splits - 1) / splits;
-        splits = (p.k_steps + k_per - 1) / k_per;
+        const int k_per = (pl.k_steps + splits - 1) / splits;
+        splits = (pl.k_steps + k_per - 1) / k_per;
     }
     if (TM > 64) splits = 1;  // keeps the split-K receive buffer (S x 128 x TM/S floats) small
+    pl.splits = splits;
     // split-K receive buffer [S][128][ceil(TM/S)] floats, placed after the fixed area
     const int recv_bytes = splits > 1 ? splits * 128 * tc::split_cols(TM, splits) * 4 + 64 : 0;
     int budget = splits > 1 ? 110 * 1024 : (TM <= 64 ? 112 * 1024 : 200 * 1024);
     if (splits > 1 && tune_split_smem_kb > 0) budget = tune_split_smem_kb * 1024;
     if (splits == 1 && tune_smem_kb > 0) budget = tune_smem_kb * 1024;
-    const int stages = std::max(2, std::min(16, (budget - fixed - recv_bytes) / stage_bytes));
-    const size_t smem = (size_t)fixed + (size_t)recv_bytes + (size_t)stages * stage_bytes;
+    pl.stages = std::max(2, std::min(16, (budget - fixed - recv_bytes) / stage_bytes));
+    pl.smem = (size_t)fixed + (size_t)recv_bytes + (size_t)pl.stages * stage_bytes;
+    return pl;
+}
+
+template <>
+int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K, const Epi<bf16> &e,
+                      cudaStream_t s, const int *dep_ctr, int dep_target, int *done_ctr, const float *w_scale) {
+    const bool swiglu = e.kind == EPI_SWIGLU;
+    const bool f8 = w_scale != nullptr;
+    const TcPlan pl = plan(M, N, K, e.kind, e.F, f8, e.lo ? 2 : 1);
+    const int TM = pl.TM, splits = pl.splits, stages = pl.stages;
+    const size_t smem = pl.smem;
+    TcParams p;
+    memset(&p, 0, sizeof p);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.swiglu_F = swiglu ? e.F : 0;
+    p.n_tiles = pl.n_tiles;
+    p.m_tiles = pl.m_tiles;
+    p.k_steps = pl.k_steps;
+    p.planes = e.lo ? 2 : 1;
+    p.w_scale = w_scale;
     p.splits = splits;
     p.err = err_word;
     p.lm_part = lm_part;

@@ -38,12 +38,17 @@ struct TcParams {
     int dep_target;
     int *done_ctr;
     const float *w_scale;   // FP8 weights: fp32 scale of every weight row (the codes' row of W)
-    int l2_ahead;           // weight stages prefetched into L2 beyond the shared-memory ring (0: none)
     // grouped (MoE experts): blockIdx.y = touched-expert slot, blockIdx.z = row tile of
     // that expert; its rows are g_off[e] .. g_off[e+1]-1 of X (expert-grouped order) and
     // its weights rows e*g_wrows .. of W; nullptr g_off = an ordinary projection
     const int *g_off, *g_touched, *g_list;
     int g_wrows;
+};
+
+// Tiling of one projection launch (GemmTC::plan).
+struct TcPlan {
+    int TM, n_tiles, m_tiles, k_steps, kstep, splits, stages;
+    size_t smem;
 };
 
 template <typename T>
@@ -64,6 +69,9 @@ struct GemmTC {
     // EPI_STORE writes row list[pos] of Y.  Returns the CTAs launched.
     int run_grouped(const T *X, int ldx, int n_pairs, const T *W, int wrows, int N, int K, const Epi<T> &e,
                     const int *off, const int *touched, const int *list, int E, int max_rows, cudaStream_t s);
+    // tiling of a launch of M activation rows (planes 1 or 2) against an N x K weight
+    // matrix (SwiGLU: F output columns, N = 2F), bf16 or FP8
+    TcPlan plan(int M, int N, int K, int kind, int F, bool f8, int planes) const;
     // LM-head partial argmax buffer (value, index as float bits), [n_tiles][rows]
     void set_lm_part(float2 *p, int cap) { lm_part = p; lm_cap = cap; }
     void set_err(int *e) { err_word = e; }
@@ -78,7 +86,7 @@ struct GemmTC {
     int num_sms = 148;
     // tuning overrides (0 = automatic): K splits per tile, shared-memory budget in KB
     // of unsplit / K-split launches, CTAs per SM the K split aims to fill
-    int tune_splits = 0, tune_smem_kb = 0, tune_split_smem_kb = 0, tune_ctas_per_sm = 0, l2_ahead = 0;
+    int tune_splits = 0, tune_smem_kb = 0, tune_split_smem_kb = 0, tune_ctas_per_sm = 0;
     int tune_tm_max = 0;  // cap on the activation rows of one tile (more row tiles, weights re-read from L2)
     std::unordered_map<std::string, CUtensorMap> maps;
     // 2-D map of a [rows][cols] bf16 matrix (leading dimension ld), box {64, box_rows};
