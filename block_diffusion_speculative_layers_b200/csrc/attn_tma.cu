@@ -52,6 +52,12 @@ __device__ __forceinline__ unsigned long long gtimer() {
     return t;
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
 }
@@ -259,8 +265,27 @@ __global__ void __launch_bounds__(NTH, 2) attn_tma_kernel(const __grid_constant_
             }
         }
     }
-    __syncthreads();
-    pdl_wait();  // q, K and V come from the projection before this kernel
+    if (a.dep_ctr) {
+        // q, K and V come from the projection before this kernel: wait until each of
+        // its CTAs has signalled (acquire), then make its writes visible to TMA
+        if (threadIdx.x == 0) {
+            bool ok = true;
+            const unsigned long long t0 = gtimer();
+            while (ld_acquire_gpu(a.dep_ctr) < a.dep_target) {
+                if (gtimer() - t0 > WAIT_NS) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(32);
+            }
+            if (!ok && a.err) atomicOr(a.err, 32);
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        __syncthreads();
+    } else {
+        __syncthreads();
+        pdl_wait();  // q, K and V come from the projection before this kernel
+    }
 
     // longest visible key range of the tile's rows (<= 16 rows), the same in every lane
     int nk_max = lane < nrows ? a.meta[r0 + lane].nk : 0;
@@ -546,6 +571,12 @@ __global__ void __launch_bounds__(NTH, 2) attn_tma_kernel(const __grid_constant_
         bf16 *dst = a.out + (size_t)(r0 + row) * a.ldo + (h0 + hh) * HD + d0;
         store_pair(dst, a.lo, acc.x * inv, acc.y * inv);
         store_pair(dst + 2, a.lo, acc.z * inv, acc.w * inv);
+    }
+    if (a.done_ctr) {  // every writer fences (generic and async proxy) before the signal
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncthreads();
+        if (threadIdx.x == 0) atomicAdd(a.done_ctr, 1);
     }
 }
 

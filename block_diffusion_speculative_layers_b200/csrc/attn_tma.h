@@ -24,6 +24,12 @@ struct AttnTmaArgs {
     size_t lo = 0;                  // two-plane activations: low plane offset (elements), 0: one plane
     int *err = nullptr;             // device error word (bit 32: a bounded wait expired)
     int n_splits = 1, stages = 3;   // set by the launcher
+    // completion counters (decode passes): wait until *dep_ctr >= dep_target instead
+    // of griddepcontrol.wait (nullptr: griddepcontrol.wait); each CTA adds 1 to
+    // *done_ctr after its last store (nullptr: no signal)
+    const int *dep_ctr = nullptr;
+    int dep_target = 0;
+    int *done_ctr = nullptr;
 };
 
 bool attn_tma_supported(int hd, int grp);

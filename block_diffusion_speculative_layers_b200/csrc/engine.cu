@@ -306,6 +306,15 @@ static Layout make_layout(const dflash_config &c) {
         L.dep_v = take((size_t)2 * L.n_ops_v * 4);
         L.dep_d = take((size_t)2 * L.n_ops_d * 4);
     }
+    // FP8 projections: the activation rows as MX planes (codes + scale words), sized
+    // for the most rows and the widest K of any projection
+    if (c.dtype == DFLASH_FP8) {
+        const int kmax = std::max({t.hidden, d.hidden, qmax, fmax, TK});
+        L.mx_mpad = (int)align_up((size_t)L.R_max, 32);
+        L.mx_kpad = (int)align_up((size_t)kmax, 128);
+        L.mx_codes = take((size_t)4 * L.mx_mpad * L.mx_kpad);
+        L.mx_words = take((size_t)(L.mx_kpad / 128) * 4 * L.mx_mpad * 4);
+    }
     // split-K workspace and tile semaphores of the tensor-core GEMM
     L.ws_floats = gemm_tc_workspace_floats(L.R_max, std::max(ycols, t.vocab > 0 ? H : H));
     L.gemm_ws = take((size_t)L.ws_floats * 4);
@@ -514,7 +523,7 @@ class Engine : public EngineBase {
             // pass instead of griddepcontrol.wait (same results; measured 0.2 ms per step
             // slower on B200: the fences of every writer cost more than the grid release)
             const char *dv_env = getenv("DFLASH_DEP_COUNTERS");
-            dep_on = dv_env && dv_env[0] == '1';
+            dep_on = dv_env && dv_env[0] == '1' && !f8_;  // FP8 projections run a quantiser launch first
             const char *fv = getenv("DFLASH_FOLDED_NORM");
             const bool allow = !(fv && fv[0] == '0');
             fold_draft_ok = allow && bf && shapes;
@@ -577,6 +586,15 @@ class Engine : public EngineBase {
         tc.tune_split_smem_kb = env_int("DFLASH_TC_SPLIT_SMEM_KB");
         tc.tune_ctas_per_sm = env_int("DFLASH_TC_CTAS_PER_SM");
         tc.tune_tm_max = env_int("DFLASH_TC_TM_MAX");
+        if (f8_) {
+            // every scale byte starts as 1.0 (127): bytes past a projection's K are never NaN
+            tc.mx_codes = (uint8_t *)(S + L.mx_codes);
+            tc.mx_words = (uint8_t *)(S + L.mx_words);
+            tc.mx_mpad = L.mx_mpad;
+            tc.mx_kpad = L.mx_kpad;
+            if (cudaMemsetAsync(tc.mx_words, 0x7F, (size_t)(L.mx_kpad / 128) * 4 * L.mx_mpad * 4, s) != cudaSuccess)
+                return fail_cuda("MX scale buffer");
+        }
         tc.set_lm_part(lm_part, (c.target.vocab + 127) / 128 * L.R_dec);
         tc.set_err(&stats->status);
         tc.keep_logits = c.keep_logits;  // plus while sampling (sampling_changed)
@@ -775,7 +793,7 @@ class Engine : public EngineBase {
         const int qd = m.n_q_heads * m.head_dim;
         int ctas = 0;
         timed(DFLASH_PROF_ATTENTION, 0.0, [&] {
-            if (attn_tma_on && !sy.dep_ctr && !sy.done_ctr) {
+            if (attn_tma_on) {
                 if constexpr (std::is_same<T, bf16>::value) {
                     AttnTmaArgs a;
                     a.q = (const bf16 *)qq;
@@ -793,6 +811,9 @@ class Engine : public EngineBase {
                     a.ldo = qd;
                     a.lo = lo_;
                     a.err = &stats->status;
+                    a.dep_ctr = sy.dep_ctr;
+                    a.dep_target = sy.dep_target;
+                    a.done_ctr = sy.done_ctr;
                     ctas = launch_attention_tma(kv_map[which], a, m.head_dim, lo_ != 0, num_sms, s);
                     if (ctas < 0) attn_failed = true;
                 }

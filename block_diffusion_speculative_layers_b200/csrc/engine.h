@@ -40,6 +40,8 @@ struct Layout {
     size_t moe_sel, moe_wt, moe_part, moe_off = 0, moe_list = 0, moe_xg = 0, lm_part, att_o, att_ml, att_sem;
     size_t att_parts = 0;
     size_t xg_t, xg2, ssq, dep_v, dep_d;
+    size_t mx_codes = 0, mx_words = 0;  // FP8: MX planes of a projection's activation rows
+    int mx_mpad = 0, mx_kpad = 0;
     size_t act_lo = 0;  // two-plane activations: low plane offset in elements (0: one plane)
     int ssq_ld = 0, n_ops_v = 0, n_ops_d = 0;
     size_t gemm_ws, gemm_sem;

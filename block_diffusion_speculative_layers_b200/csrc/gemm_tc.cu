@@ -48,17 +48,16 @@ namespace tc {
 // FP8 weights (F8): the weight tile arrives as E4M3 codes, 128 rows x 128 K
 // (16 KB, one TMA box per 64 rows), half the bytes of bf16, and goes to the
 // tensor cores as it is: tcgen05.mma kind::mxf8f6f4 with block scales.  The
-// activation tile of the same 128 K arrives as bf16 (both planes) and the four
-// epilogue warps, during the main loop, rewrite it as F8_PLANES E4M3 planes
-// with one power-of-two (UE8M0) scale per 32 values of a row and plane, the
-// MX block-scaled form: plane p holds what planes 0..p-1 left over, so the
-// planes sum to the value up to 2^-16 of its block's largest magnitude.  The
-// planes are the N operand (N = F8_PLANES * TM), their scales go to tensor
-// memory (tcgen05.st), the weight rows' block scales are all 1 and each weight
-// row's fp32 scale multiplies the plane-summed accumulator in the epilogue.
-// Rings: stages in shared memory (codes + the bf16 activation tiles), released
-// by the quantiser warps and the MMA commit together; quantised slots (planes
-// in shared memory, scales in tensor memory), released by the MMA commit.
+// activations reach the kernel already in the MX block-scaled form: a small
+// kernel before each FP8 projection (mx_quantize_kernel) rewrites the bf16
+// rows (both planes) as F8_PLANES E4M3 planes with one power-of-two (UE8M0)
+// scale per 32 values of a row and plane; plane p holds what planes 0..p-1
+// left over, so the planes sum to the value within 2^-16 of its block's
+// largest magnitude.  Each stage loads the planes of its 128 K by TMA (the N
+// operand, N = F8_PLANES * TM) and their scale words; the epilogue warps copy
+// the words into tensor memory (tcgen05.st) during the main loop.  The weight
+// rows' block scales are all 1; each weight row's fp32 scale multiplies the
+// plane-summed accumulator in the epilogue.
 
 // Smallest E with m * 2^-E <= 448 (the largest E4M3 magnitude) for m > 0,
 // kept inside [-126, 126]; 0 for m == 0.  m = 1.f * 2^x: E = x - 8 unless the
@@ -128,25 +127,26 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b,
 // The kernel body.  p and e are the launch's parameters (ungrouped launches
 // read them in place, without a copy) or a grouped CTA's adjusted copies.
 template <int TM, int KIND, bool F8, bool GR>
-__device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUtensorMap &tmX, const TcParams &p,
-                                             const Epi<bf16> &e, int stages, int g_row0, int g_wrow0) {
+__device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmS,
+                                             const TcParams &p, const Epi<bf16> &e, int stages, int g_row0,
+                                             int g_wrow0) {
     constexpr bool grouped = GR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const int B_BYTES = TM * 128 * p.planes;  // activation tile(s) of 64 K
-    // F8 stages cover 128 K: 16 KB of codes and two activation tiles
-    const int A_ST = F8 ? F8_A_BYTES : A_BYTES, B_ST = F8 ? 2 * B_BYTES : B_BYTES;
+    // bf16: the activation tile(s) of 64 K; F8: the activation planes of 128 K
+    const int B_BYTES = F8 ? F8_PLANES * TM * 128 : TM * 128 * p.planes;
+    const int A_ST = F8 ? F8_A_BYTES : A_BYTES, B_ST = B_BYTES;
+    constexpr int SW_ST = F8 ? F8_PLANES * TM * 4 : 0;  // F8: scale words of a stage, [plane][row]
     // two planes and TM <= 128: one MMA with N = 2*TM covers the hi and lo rows
     // (they are contiguous in the stage), accumulating into 2*TM columns
     const bool wide = !F8 && p.planes == 2 && TM <= 128;
     const int lo_col = wide ? TM : 0;
     // F8: N = F8_PLANES * TM quantised rows (plane-major)
     const int NC1 = max(32, F8 ? F8_PLANES * TM : wide ? 2 * TM : TM);  // TMEM columns of one accumulator
-    constexpr int QB = F8 ? F8_PLANES * TM * 128 : 0;  // one quantised slot: planes x TM rows x 128 K codes
     uint8_t *sA = smem;
     uint8_t *sB = smem + (size_t)stages * A_ST;
-    uint8_t *sQ = sB + (size_t)stages * B_ST;  // F8: [F8_QSTAGES] quantised slots (1024-byte multiples)
-    float *stg = (float *)(sQ + (F8 ? F8_QSTAGES * QB : 0));
+    uint32_t *sW = (uint32_t *)(sB + (size_t)stages * B_ST);  // F8: [stages] scale words
+    float *stg = (float *)((uint8_t *)sW + (size_t)stages * SW_ST);
     float2 *red = (float2 *)(stg + 128 * STG_LD);
     RowMeta *smeta = (RowMeta *)(red + 4 * CH);
     float *rsc = (float *)(smeta + CH);       // [RS_MAX] row scales of the folded norm
@@ -154,14 +154,8 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
     uint64_t *empty = full + stages;
     uint64_t *acc_full = empty + stages;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
-    uint64_t *q_full = acc_empty + 2;       // [F8_QSTAGES] quantised slot written
-    uint64_t *q_free = q_full + F8_QSTAGES;  // [F8_QSTAGES] quantised slot read by the MMAs
-    // F8: the activation tiles of a stage complete on their own barrier (the
-    // quantiser waits for them only; the MMA for the codes and the slot)
-    uint64_t *full_b = q_free + F8_QSTAGES;  // [stages]
-    // F8: scale bytes of a quantised slot, [F8_QSTAGES][F8_PLANES * TM][4 blocks of 32 K]
-    uint8_t *sSF = (uint8_t *)(full_b + (F8 ? stages : 0));
-    uint32_t *tmem_slot = (uint32_t *)(sSF + (F8 ? F8_QSTAGES * F8_PLANES * TM * 4 : 0));
+    uint64_t *sf_full = acc_empty + 2;  // F8: [stages] a stage's scale words are in tensor memory
+    uint32_t *tmem_slot = (uint32_t *)(sf_full + (F8 ? stages : 0));
     // split-K receive buffer [S][128][cpr] (16-byte aligned, after the fixed area)
     float *recv = (float *)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
     EpiIn pre;
@@ -181,27 +175,23 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
     const int ke = split ? min(p.k_steps, kb + k_per) : p.k_steps;
     const int nk = max(0, ke - kb);
     // F8: after the accumulator, the weights' scale words (4 columns: row m at
-    // lane m, column m / 32) and one 4-column group per quantised slot (plane row
-    // n at lane n % 32 of every lane quarter, column n / 32; byte b of a word =
-    // the scale of 32-K block b of the stage)
-    const int sf_cols = F8 ? 4 + 4 * F8_QSTAGES : 0;
+    // lane m, column m / 32) and one 4-column group per stage (plane row n at
+    // lane n % 32 of every lane quarter, column n / 32; byte b of a word = the
+    // scale of 32-K block b of the stage), as measured on the device
+    const int sf_cols = F8 ? 4 + 4 * stages : 0;
     const int ncols = tmem_cols_for((persistent ? 2 * NC1 : NC1) + sf_cols);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], F8 ? 5 : 1);  // F8: the four quantiser warps + the MMA commit
+            mbar_init(&empty[s], F8 ? 5 : 1);  // F8: the four scale-copy warps + the MMA commit
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(&acc_full[1], 1);
         mbar_init(&acc_empty[0], 4);
         mbar_init(&acc_empty[1], 4);
-        for (int s = 0; s < F8_QSTAGES; ++s) {
-            mbar_init(&q_full[s], 4);
-            mbar_init(&q_free[s], 1);
-        }
         if (F8)
-            for (int s = 0; s < stages; ++s) mbar_init(&full_b[s], 1);
+            for (int s = 0; s < stages; ++s) mbar_init(&sf_full[s], 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -220,74 +210,27 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
     if (split) cluster_arrive_relaxed();
     pdl_trigger();
 
-    // F8: quantise the activation tile of every stage into MX planes (warps
-    // 2..5, 128 threads).  Thread = (row j, 32-K block, half): 16 values, the
-    // block's other half in lane ^ 1.  Codes go to the slot in the 128-byte
-    // swizzled layout of the MMA's N operand; scale bytes go to sSF and then,
-    // as one word per plane row, into tensor memory, copied into every lane
-    // quarter (each quarter of the MMA reads its own copy).
-    auto quantise = [&] {
-        const int t = threadIdx.x - 64;  // 0..127
+    // F8: copy every stage's activation scale words into tensor memory (warps
+    // 2..5; lane i of warp w writes plane rows i, 32 + i, ... of lane quarter
+    // w % 4, each quarter of the MMA reading its own copy)
+    auto copy_scales = [&] {
         const int q = warp & 3;
         // the weights' block scales: 1.0 (UE8M0 127) in every byte
         tmem_st4(tmem_sfa + ((uint32_t)(q * 32) << 16), 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
         bool dead = false;
         for (int kk = 0; kk < nk; ++kk) {
-            const int s = kk % stages, sq = kk % F8_QSTAGES;
-            if (!dead && !mbar_wait(&full_b[s], (kk / stages) & 1, p.err)) dead = true;
-            if (!dead && kk >= F8_QSTAGES && !mbar_wait(&q_free[sq], ((kk / F8_QSTAGES) - 1) & 1, p.err)) dead = true;
-            const uint8_t *xb = sB + (size_t)s * B_ST;
-            uint8_t *qs = sQ + (size_t)sq * QB;
-            uint8_t *sf = sSF + sq * (F8_PLANES * TM * 4);
-#pragma unroll 1
-            for (int u = t; u < TM * 8; u += 128) {
-                const int j = u >> 3, blk = (u >> 1) & 3, h2 = u & 1;
-                const int k0 = blk * 32 + h2 * 16;                 // first K of the 16 values in the stage
-                const uint8_t *row = xb + (k0 >> 6) * (TM * 128 * p.planes) + j * 128;
-                const int c0 = (k0 & 63) >> 3;                     // first 16-byte chunk of 8 values
-                float r[16];
+            const int s = kk % stages;
+            if (!dead && !mbar_wait(&full[s], (kk / stages) & 1, p.err)) dead = true;
+            const uint32_t *w = sW + (size_t)s * (F8_PLANES * TM);
+            uint32_t w4[4];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int off = (((c0 + h) ^ j) & 7) << 4;
-                    const uint4 hv = dead ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4 *>(row + off);
-                    uint4 lv = make_uint4(0, 0, 0, 0);
-                    if (p.planes == 2 && !dead) lv = *reinterpret_cast<const uint4 *>(row + TM * 128 + off);
-                    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hw[i]));
-                        const float2 lf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&lw[i]));
-                        r[h * 8 + 2 * i] = hf.x + lf.x;
-                        r[h * 8 + 2 * i + 1] = hf.y + lf.y;
-                    }
-                }
-                uint4 code[F8_PLANES];
-                int ex[F8_PLANES];
-                mx_planes16<F8_PLANES>(r, code, ex);
-#pragma unroll
-                for (int pl = 0; pl < F8_PLANES; ++pl) {
-                    const int rq = pl * TM + j;  // row of the N operand
-                    *reinterpret_cast<uint4 *>(qs + rq * 128 + ((((blk * 2 + h2) ^ rq) & 7) << 4)) = code[pl];
-                    if (h2 == 0) sf[rq * 4 + blk] = (uint8_t)(ex[pl] + 127);
-                }
-            }
-            // codes written by the generic proxy, read by the tensor cores
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            epi_bar();  // every scale byte of the slot is in sSF
-            {
-                // plane row n = 32 c + lane: word c of this lane (up to 4 words; TM <= 32)
-                uint32_t w4[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    w4[c] = 32 * c < F8_PLANES * TM ? *reinterpret_cast<const uint32_t *>(sf + (32 * c + lane) * 4)
-                                                    : 0x7F7F7F7Fu;
-                tmem_st4(tmem_sfb + (uint32_t)(sq * 4) + ((uint32_t)(q * 32) << 16), w4[0], w4[1], w4[2], w4[3]);
-            }
+            for (int c = 0; c < 4; ++c) w4[c] = (!dead && 32 * c + lane < F8_PLANES * TM) ? w[32 * c + lane] : 0x7F7F7F7Fu;
+            tmem_st4(tmem_sfb + (uint32_t)(s * 4) + ((uint32_t)(q * 32) << 16), w4[0], w4[1], w4[2], w4[3]);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&q_full[sq]);
+                mbar_arrive(&sf_full[s]);
                 mbar_arrive(&empty[s]);
             }
         }
@@ -299,15 +242,18 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
             const uint64_t wpol = l2_evict_first_policy();
             const int kstep = F8 ? 2 * BK : BK;  // K elements per stage
             auto load_x = [&](int s, int k, int m0) {
-                uint64_t *bar = F8 ? &full_b[s] : &full[s];
-                if (F8) mbar_expect_tx(bar, B_ST);
-                for (int h = 0; h < (F8 ? 2 : 1); ++h) {
-                    uint8_t *b = sB + (size_t)s * B_ST + h * B_BYTES;
-                    if (p.planes == 2) tma_load_3d(b, &tmX, k + h * BK, m0, 0, bar);
-                    else tma_load_2d(b, &tmX, k + h * BK, m0, bar);
+                uint8_t *b = sB + (size_t)s * B_ST;
+                if constexpr (F8) {
+                    // the stage's planes {128 K, TM rows, planes} and scale words {TM rows, planes}
+                    tma_load_3d(b, &tmX, k, m0, 0, &full[s]);
+                    tma_load_2d(sW + (size_t)s * (F8_PLANES * TM), &tmS, m0, (k / (2 * BK)) * F8_PLANES, &full[s]);
+                } else if (p.planes == 2) {
+                    tma_load_3d(b, &tmX, k, m0, 0, &full[s]);
+                } else {
+                    tma_load_2d(b, &tmX, k, m0, &full[s]);
                 }
             };
-            const int a_tx = F8 ? A_ST : A_ST + B_ST;  // bytes completing full[]
+            const int a_tx = A_ST + B_ST + SW_ST;  // bytes completing full[]
             int it = 0;     // global stage counter
             bool first = true, abort = false;
             for (int t = tile0; t < n_tiles_total && !abort; t += tstride) {
@@ -360,23 +306,21 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const int s = it % stages;
                     if constexpr (F8) {
-                        const int sq = it % F8_QSTAGES;
                         if (!mbar_wait(&full[s], (it / stages) & 1, p.err) ||
-                            !mbar_wait(&q_full[sq], (it / F8_QSTAGES) & 1, p.err)) {
+                            !mbar_wait(&sf_full[s], (it / stages) & 1, p.err)) {
                             ok = false;
                             break;
                         }
                         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                         const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_ST));
-                        const uint64_t db = sw128_desc(smem_u32(sQ + (size_t)sq * QB));
-                        const uint32_t sfb = tmem_sfb + (uint32_t)(sq * 4);
+                        const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_ST));
+                        const uint32_t sfb = tmem_sfb + (uint32_t)(s * 4);
 #pragma unroll
                         for (int k32 = 0; k32 < 4; ++k32)  // 4 x K=32 over the stage's 128 K (+32 bytes each)
                             mma_mx(acc, da + (uint64_t)(k32 * 2), db + (uint64_t)(k32 * 2),
                                    idesc_mx(F8_PLANES * TM, k32), tmem_sfa | ((uint32_t)k32 << 30),
                                    sfb | ((uint32_t)k32 << 30), (kk > 0 || k32 > 0) ? 1u : 0u);
                         mma_commit(&empty[s]);
-                        mma_commit(&q_free[sq]);
                     } else {
                         if (!mbar_wait(&full[s], (it / stages) & 1, p.err)) {
                             ok = false;
@@ -403,7 +347,7 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
         // ---------------- epilogue warps 2..5 ----------------
         const int q = warp & 3;
         const int n_local = q * 32 + lane;
-        if constexpr (F8) quantise();
+        if constexpr (F8) copy_scales();
         if (p.dep_ctr) {
             if (threadIdx.x == 64) dep_wait(p.dep_ctr, p.dep_target, p.err);
             epi_bar();
@@ -550,7 +494,8 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
 template <int TM, int KIND, bool F8, bool GR>
 __global__ void __launch_bounds__(NT, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   const __grid_constant__ TcParams p, const __grid_constant__ Epi<bf16> e, int stages) {
+                   const __grid_constant__ CUtensorMap tmS, const __grid_constant__ TcParams p,
+                   const __grid_constant__ Epi<bf16> e, int stages) {
     if constexpr (GR) {
         // grouped (MoE experts): this CTA's expert, its rows and weight rows
         pdl_wait();  // the expert lists come from the bucketing kernel
@@ -564,9 +509,52 @@ __global__ void __launch_bounds__(NT, 1)
         pg.M = min(TM, nr - m0);
         if (KIND == EPI_SWIGLU) eg.h += (size_t)(r0 + m0) * p.swiglu_F;
         if (KIND == EPI_STORE && p.g_list) eg.row_map = p.g_list + r0 + m0;
-        gemm_tc_body<TM, KIND, F8, true>(tmW, tmX, pg, eg, stages, r0 + m0, ex * p.g_wrows);
+        gemm_tc_body<TM, KIND, F8, true>(tmW, tmX, tmS, pg, eg, stages, r0 + m0, ex * p.g_wrows);
     } else {
-        gemm_tc_body<TM, KIND, F8, false>(tmW, tmX, p, e, stages, 0, 0);
+        gemm_tc_body<TM, KIND, F8, false>(tmW, tmX, tmS, p, e, stages, 0, 0);
+    }
+}
+
+// MX planes of the activation rows of an FP8 projection: X [M][ld] bf16 (its
+// low plane lo elements on when lo != 0), K columns.  Thread = 16 columns of a
+// row (half a 32-column block; the other half in lane ^ 1).  Codes of plane p,
+// row m, column k at codes[(p * mpad + m) * kpad + k]; the scale byte of
+// (p, m, 32-column block b) is byte b % 4 of word ((b / 4) * F8_PLANES + p) *
+// mpad + m of `words` (UE8M0: exponent + 127).
+__global__ void __launch_bounds__(256) mx_quantize_kernel(const bf16 *__restrict__ X, int ld, size_t lo, int M, int K,
+                                                          int mpad, int kpad, uint8_t *__restrict__ codes,
+                                                          uint8_t *__restrict__ words) {
+    pdl_trigger();
+    pdl_wait();  // X comes from the kernel before this one
+    const int halves = K >> 4;
+    const long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool in = u < (long long)M * halves;  // pairs of halves are both in or both out (halves is even)
+    const int m = in ? (int)(u / halves) : 0, hb = in ? (int)(u % halves) : 0;
+    const int k0 = hb * 16;
+    float r[16];
+    const bf16 *xr = X + (size_t)m * ld + k0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 hv = in ? *reinterpret_cast<const uint4 *>(xr + 8 * h) : make_uint4(0, 0, 0, 0);
+        const uint4 lv = (in && lo) ? *reinterpret_cast<const uint4 *>(xr + lo + 8 * h) : make_uint4(0, 0, 0, 0);
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hw[i]));
+            const float2 lf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&lw[i]));
+            r[h * 8 + 2 * i] = hf.x + lf.x;
+            r[h * 8 + 2 * i + 1] = hf.y + lf.y;
+        }
+    }
+    uint4 code[F8_PLANES];
+    int ex[F8_PLANES];
+    mx_planes16<F8_PLANES>(r, code, ex);
+    if (!in) return;
+    const int blk = k0 >> 5;
+#pragma unroll
+    for (int pl = 0; pl < F8_PLANES; ++pl) {
+        *reinterpret_cast<uint4 *>(codes + ((size_t)pl * mpad + m) * kpad + k0) = code[pl];
+        if ((hb & 1) == 0) words[(((size_t)(blk >> 2) * F8_PLANES + pl) * mpad + m) * 4 + (blk & 3)] = (uint8_t)(ex[pl] + 127);
     }
 }
 
@@ -704,26 +692,74 @@ const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, in
     return &(maps[key] = m);
 }
 
+// Tensor map of the MX activation planes of an M x K projection input:
+// (K bytes, M rows, planes), box {128 K, tm rows, planes}, 128-byte swizzle.
+// Rows >= M and columns >= K read as zero codes.
+template <typename T>
+const CUtensorMap *GemmTC<T>::mx_map_codes(int M, int K, int tm) {
+    char key[96];
+    snprintf(key, sizeof key, "mxc/%p/%d/%d/%d", (void *)mx_codes, M, K, tm);
+    auto it = maps.find(key);
+    if (it != maps.end()) return &it->second;
+    CUtensorMap m;
+    memset(&m, 0, sizeof m);
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)M, (cuuint64_t)tc::F8_PLANES};
+    cuuint64_t strides[2] = {(cuuint64_t)mx_kpad, (cuuint64_t)mx_kpad * mx_mpad};
+    cuuint32_t box[3] = {128, (cuuint32_t)tm, (cuuint32_t)tc::F8_PLANES};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (get_encode()(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, mx_codes, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        err = "cuTensorMapEncodeTiled failed (MX planes)";
+        return nullptr;
+    }
+    return &(maps[key] = m);
+}
+
+// Tensor map of the MX scale words: (M words, stages x planes rows), box
+// {tm words, planes}: a stage's words land as [plane][row].
+template <typename T>
+const CUtensorMap *GemmTC<T>::mx_map_words(int M, int K, int tm) {
+    char key[96];
+    snprintf(key, sizeof key, "mxw/%p/%d/%d/%d", (void *)mx_words, M, K, tm);
+    auto it = maps.find(key);
+    if (it != maps.end()) return &it->second;
+    CUtensorMap m;
+    memset(&m, 0, sizeof m);
+    const int ks = (K + 127) / 128;
+    cuuint64_t dims[2] = {(cuuint64_t)M, (cuuint64_t)ks * tc::F8_PLANES};
+    cuuint64_t strides[1] = {(cuuint64_t)mx_mpad * 4};
+    cuuint32_t box[2] = {(cuuint32_t)tm, (cuuint32_t)tc::F8_PLANES};
+    cuuint32_t estr[2] = {1, 1};
+    if (get_encode()(&m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, mx_words, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        err = "cuTensorMapEncodeTiled failed (MX scales)";
+        return nullptr;
+    }
+    return &(maps[key] = m);
+}
+
 template <int TM, int KIND, bool F8>
-static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p,
+static void launch_tm(const CUtensorMap *mw, const CUtensorMap *mx, const CUtensorMap *ms, const TcParams &p,
                       const Epi<bf16> &e, int stages, size_t smem, cudaStream_t s, int grid_x) {
     auto kern = tc::gemm_tc_kernel<TM, KIND, F8, false>;
     ensure_smem_attr((const void *)kern);
     (void)grid_x;
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-    launch_k(kern, grid, dim3(tc::NT), smem, s, p.splits, *mw, *mx, p, e, stages);
+    launch_k(kern, grid, dim3(tc::NT), smem, s, p.splits, *mw, *mx, *ms, p, e, stages);
 }
 
 template <int TM, bool F8>
-static void launch_kind(int kind, const CUtensorMap *mw, const CUtensorMap *mx, const TcParams &p,
+static void launch_kind(int kind, const CUtensorMap *mw, const CUtensorMap *mx, const CUtensorMap *ms, const TcParams &p,
                         const Epi<bf16> &e, int stages, size_t smem, cudaStream_t s, int gx) {
     switch (kind) {
-        case EPI_STORE: launch_tm<TM, EPI_STORE, F8>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_QKV: launch_tm<TM, EPI_QKV, F8>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_RESID: launch_tm<TM, EPI_RESID, F8>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_SWIGLU: launch_tm<TM, EPI_SWIGLU, F8>(mw, mx, p, e, stages, smem, s, gx); break;
-        case EPI_NORMOUT: launch_tm<TM, EPI_NORMOUT, F8>(mw, mx, p, e, stages, smem, s, gx); break;
-        default: launch_tm<TM, EPI_LOGITS, F8>(mw, mx, p, e, stages, smem, s, gx); break;
+        case EPI_STORE: launch_tm<TM, EPI_STORE, F8>(mw, mx, ms, p, e, stages, smem, s, gx); break;
+        case EPI_QKV: launch_tm<TM, EPI_QKV, F8>(mw, mx, ms, p, e, stages, smem, s, gx); break;
+        case EPI_RESID: launch_tm<TM, EPI_RESID, F8>(mw, mx, ms, p, e, stages, smem, s, gx); break;
+        case EPI_SWIGLU: launch_tm<TM, EPI_SWIGLU, F8>(mw, mx, ms, p, e, stages, smem, s, gx); break;
+        case EPI_NORMOUT: launch_tm<TM, EPI_NORMOUT, F8>(mw, mx, ms, p, e, stages, smem, s, gx); break;
+        default: launch_tm<TM, EPI_LOGITS, F8>(mw, mx, ms, p, e, stages, smem, s, gx); break;
     }
 }
 
@@ -750,12 +786,10 @@ TcPlan GemmTC<T>::plan(int M, int N, int K, int kind, int F, bool f8, int planes
     pl.kstep = f8 ? 2 * tc::BK : tc::BK;  // K per stage: 128 FP8 codes or 64 bf16 values per weight row
     pl.k_steps = (K + pl.kstep - 1) / pl.kstep;
     const int tiles = pl.n_tiles * pl.m_tiles;
-    const int stage_bytes = f8 ? tc::F8_A_BYTES + 2 * TM * 128 * planes : tc::A_BYTES + TM * 128 * planes;
-    // fixed area: alignment, epilogue staging, barriers; FP8 adds the quantised
-    // slots (codes + scale bytes)
-    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
-                      2 * tc::F8_QSTAGES * 8 + 16 * 8 +
-                      (f8 ? tc::F8_QSTAGES * tc::F8_PLANES * TM * (128 + 4) : 0);
+    // a stage: the weight tile + the activation tile(s) (FP8: codes + activation planes + scale words)
+    const int stage_bytes = f8 ? tc::F8_A_BYTES + tc::F8_PLANES * TM * (128 + 4) : tc::A_BYTES + TM * 128 * planes;
+    // fixed area: alignment, epilogue staging, barriers
+    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 + 16 * 8;
     // Measured on B200 (decode shapes, M = 16, whole decode iteration): every
     // projection streams best with ~110 KB CTAs, two of which fit on an SM;
     // projections with fewer tiles than that split K over a cluster (up to 8
@@ -814,23 +848,39 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     p.done_ctr = done_ctr;
     const int grid_x = p.n_tiles;  // one tile per CTA
     const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64, 0, f8);
-    const CUtensorMap *mx = tensor_map(X, M, K, ldx, TM, e.lo);
-    if (!mw || !mx) {
+    const CUtensorMap *mx = nullptr, *ms = nullptr;
+    if (f8) {
+        // the activation rows as MX planes (a kernel of their own, before the projection)
+        if (!mx_codes || M > mx_mpad || K > mx_kpad || K % 32 || ldx % 8) {
+            failed = true;
+            err = "FP8 projection: activation rows do not fit the MX buffers";
+            return 0;
+        }
+        const int threads = M * (K / 16);
+        launch_k(tc::mx_quantize_kernel, dim3((threads + 255) / 256), dim3(256), 0, s, 1, X, ldx, e.lo, M, K,
+                 mx_mpad, mx_kpad, mx_codes, mx_words);
+        mx = mx_map_codes(M, K, TM);
+        ms = mx_map_words(M, K, TM);
+    } else {
+        mx = tensor_map(X, M, K, ldx, TM, e.lo);
+        ms = mx;
+    }
+    if (!mw || !mx || !ms) {
         failed = true;
         return 0;
     }
     if (f8) {
         switch (TM) {
-            case 16: launch_kind<16, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-            default: launch_kind<32, true>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            case 16: launch_kind<16, true>(e.kind, mw, mx, ms, p, e, stages, smem, s, grid_x); break;
+            default: launch_kind<32, true>(e.kind, mw, mx, ms, p, e, stages, smem, s, grid_x); break;
         }
     } else {
         switch (TM) {
-            case 16: launch_kind<16, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-            case 32: launch_kind<32, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-            case 64: launch_kind<64, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-            case 128: launch_kind<128, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
-            default: launch_kind<256, false>(e.kind, mw, mx, p, e, stages, smem, s, grid_x); break;
+            case 16: launch_kind<16, false>(e.kind, mw, mx, ms, p, e, stages, smem, s, grid_x); break;
+            case 32: launch_kind<32, false>(e.kind, mw, mx, ms, p, e, stages, smem, s, grid_x); break;
+            case 64: launch_kind<64, false>(e.kind, mw, mx, ms, p, e, stages, smem, s, grid_x); break;
+            case 128: launch_kind<128, false>(e.kind, mw, mx, ms, p, e, stages, smem, s, grid_x); break;
+            default: launch_kind<256, false>(e.kind, mw, mx, ms, p, e, stages, smem, s, grid_x); break;
         }
     }
     return p.n_tiles * p.m_tiles * p.splits;
@@ -865,8 +915,7 @@ int GemmTC<bf16>::run_grouped(const bf16 *X, int ldx, int n_pairs, const bf16 *W
     p.g_list = list;
     p.g_wrows = wrows;
     const int stage_bytes = tc::A_BYTES + TM * 128 * p.planes;
-    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 +
-                      2 * tc::F8_QSTAGES * 8 + 16 * 8;
+    const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 + 16 * 8;
     const int stages = std::max(2, std::min(16, (112 * 1024 - fixed) / stage_bytes));
     const size_t smem = (size_t)fixed + (size_t)stages * stage_bytes;
     const CUtensorMap *mw = tensor_map(W, E * wrows, K, K, 64);
@@ -879,7 +928,7 @@ int GemmTC<bf16>::run_grouped(const bf16 *X, int ldx, int n_pairs, const bf16 *W
         constexpr int T_ = decltype(tm_c)::value;
         auto kern = swiglu ? tc::gemm_tc_kernel<T_, EPI_SWIGLU, false, true> : tc::gemm_tc_kernel<T_, EPI_STORE, false, true>;
         ensure_smem_attr((const void *)kern);
-        launch_k(kern, dim3(p.n_tiles, E, p.m_tiles), dim3(tc::NT), smem, s, 1, *mw, *mx, p, e, stages);
+        launch_k(kern, dim3(p.n_tiles, E, p.m_tiles), dim3(tc::NT), smem, s, 1, *mw, *mx, *mx, p, e, stages);
     };
     if (TM == 16) go(std::integral_constant<int, 16>{});
     else if (TM == 32) go(std::integral_constant<int, 32>{});

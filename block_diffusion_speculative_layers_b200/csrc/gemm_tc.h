@@ -88,6 +88,12 @@ struct GemmTC {
     // of unsplit / K-split launches, CTAs per SM the K split aims to fill
     int tune_splits = 0, tune_smem_kb = 0, tune_split_smem_kb = 0, tune_ctas_per_sm = 0;
     int tune_tm_max = 0;  // cap on the activation rows of one tile (more row tiles, weights re-read from L2)
+    // FP8 projections: MX planes of the activation rows (codes [planes][mx_mpad][mx_kpad],
+    // scale words [K/128][planes][mx_mpad]; every scale byte starts as 127), owned by the caller
+    uint8_t *mx_codes = nullptr, *mx_words = nullptr;
+    int mx_mpad = 0, mx_kpad = 0;
+    const CUtensorMap *mx_map_codes(int M, int K, int tm);
+    const CUtensorMap *mx_map_words(int M, int K, int tm);
     std::unordered_map<std::string, CUtensorMap> maps;
     // 2-D map of a [rows][cols] bf16 matrix (leading dimension ld), box {64, box_rows};
     // plane_stride > 0: 3-D map over the hi plane and the lo plane plane_stride

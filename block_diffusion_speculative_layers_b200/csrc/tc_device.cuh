@@ -13,7 +13,6 @@ namespace tc {
 constexpr int BK = 64;                 // bf16 K elements per stage = one 128-byte swizzle row
 constexpr int A_BYTES = 128 * BK * 2;  // 16 KB weight tile per stage
 constexpr int F8_A_BYTES = 128 * 128;  // FP8 weights: 128 rows x 128 codes per stage
-constexpr int F8_QSTAGES = 2;          // FP8 weights: quantised activation slots (shared memory + scale columns)
 constexpr int F8_PLANES = 4;           // FP8 weights: E4M3 planes per activation value (MX block scales)
 
 // tensor-memory columns to allocate for n used columns: a power of two >= 32
