@@ -209,16 +209,25 @@ def cpu_oracle_sample(cfg, gpu_ctx=None, prompt_len: int = 16, iters: int = 1, s
 # kernel shape, from one ncu capture of the 2-layer model of the same widths;
 # the file under profiles/ gives the command.  A shape is absent until captured
 # for the kernel version in this tree.
-TRAFFIC = {}
-TRAFFIC_SOURCE = None
+# Keyed by (config, weights): the Qwen3-8B shape at batch 1, block 16 only.
+TRAFFIC = {
+    ("qwen3_8b", "bf16"): {"qkv": 50.77e6, "attention": 4.76e6, "o": 34.18e6, "gate_up": 201.94e6,
+                           "down": 93.56e6, "lm_head": 1245.40e6, "fuse": 169.45e6},
+    ("qwen3_8b", "fp8"): {"qkv": 25.66e6, "attention": 4.76e6, "o": 17.44e6, "gate_up": 101.51e6,
+                          "down": 51.55e6, "lm_head": 623.53e6, "fuse": 85.49e6},
+}
+TRAFFIC_SOURCE = ("profiles/traffic_per_shape_qwen3_8b_2layer.md (2-layer model, one cold launch each; "
+                  "FP8: the projection launch, without its mx_quantize_kernel)")
 
 SHAPES = ("qkv", "attention", "o", "gate_up", "down", "lm_head", "fuse")
 
 
-def per_shape(prof, peak, attn_bytes_per_launch):
+def per_shape(prof, peak, attn_bytes_per_launch, traffic=None):
     """Per-shape launches, mean microseconds and achieved bandwidth of a profile
     record (CUDA events around each launch); attention bytes are the visible
-    K/V (one bf16 plane) at the profiled context."""
+    K/V (one bf16 plane) at the profiled context; traffic: the captured DRAM
+    bytes per launch of each shape (None: not captured for this workload)."""
+    traffic = traffic or {}
     out = {}
     for name in SHAPES:
         n, ms, by = prof[name]
@@ -230,7 +239,7 @@ def per_shape(prof, peak, attn_bytes_per_launch):
         gbs = by / (ms / 1000.0) / 1e9 if ms > 0 else 0.0
         out[name] = {"launches": n, "us_per_launch": round(us, 2), "bytes_per_launch": by / n,
                      "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "ms_total": round(ms, 4),
-                     "traffic": TRAFFIC.get(name)}
+                     "traffic": traffic.get(name)}
     return out
 
 
@@ -244,6 +253,8 @@ def main():
     ap.add_argument("--config", default="qwen3_8b")
     ap.add_argument("--batch", type=int, default=None, help="sequences per GPU (default: the config's)")
     ap.add_argument("--prompt-len", type=int, default=None)
+    ap.add_argument("--block-size", type=int, default=None,
+                    help="positions per drafted block (default: the config's; 1..32)")
     ap.add_argument("--forced", default="1,4,8,16", help="forced accept lengths to time ('' = none)")
     ap.add_argument("--forced-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -269,6 +280,8 @@ def main():
         cfg = cfg.with_(batch=args.batch)
     if args.prompt_len:
         cfg = cfg.with_(prompt_len=args.prompt_len)
+    if args.block_size:
+        cfg = cfg.with_(block_size=args.block_size)
     if args.weights == "fp8":
         cfg = cfg.with_(dtype="fp8")
     if args.target_layers or args.drafter_layers:
@@ -386,7 +399,10 @@ def main():
     t, d = cfg.target, cfg.drafter
     attn_b = (t.n_layers * kv_bytes_per_launch(t, start_ctx) + d.n_layers * kv_bytes_per_launch(d, start_ctx)) / (
         t.n_layers + d.n_layers)
-    shapes = per_shape(kprof, peak, attn_b)
+    # captured traffic holds for the configuration it was captured on (batch 1, block 16, 512-token prompt)
+    cap = (TRAFFIC.get((cfg.name, cfg.dtype))
+           if cfg.batch == 1 and cfg.block_size == 16 and args.target_layers is None else None)
+    shapes = per_shape(kprof, peak, attn_b, cap)
     # dominant kernel: the shape with the largest share of the kernel time
     dom = max(shapes, key=lambda k: shapes[k]["ms_total"]) if shapes else None
     log(f"[rank {rank}] split at ctx ~{start_ctx:.0f}: draft {start_split[0]} us, verify {start_split[1]} us; "
