@@ -1577,7 +1577,14 @@ class Engine : public EngineBase {
     // until dflash_reset_stats or the next generation.
     static dflash_status status_code(int st, std::string &err) {
         if (st & 1) { err = "non-finite logits reached an argmax"; return DFLASH_ENUMERIC; }
-        if (st & (4 | 8 | 16 | 32)) { err = "a bounded device wait expired"; return DFLASH_ETIMEOUT; }
+        if (st & (4 | 8 | 16 | 32)) {
+            // which waits gave up: 4 an mbarrier, 8 a completion counter, 16 an
+            // attention split counter, 32 an attention input wait
+            char buf[96];
+            snprintf(buf, sizeof buf, "a bounded device wait expired (status bits 0x%x)", st & 60);
+            err = buf;
+            return DFLASH_ETIMEOUT;
+        }
         return DFLASH_OK;
     }
     dflash_status numeric_status() {
