@@ -34,6 +34,9 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <algorithm>
+#include <cstdlib>
+
 #include "attn_tma.h"
 #include "launch.h"
 
@@ -632,12 +635,34 @@ int attn_tma_kt(int hpc) { return hpc == 4 ? 32 : 16; }
 
 static size_t attn_tma_stage(int hd, bool split, int kt) { return (size_t)2 * (hd / 64) * (split ? 2 : 1) * kt * 128; }
 
-// stages: a multiple of the key groups, as many as fit in ~100 KB (two CTAs per SM)
-static int attn_tma_stages(int hd, bool split, int hpc) {
+// stages: a multiple of the key groups, as many as fit in ~100 KB (two CTAs per SM);
+// rounds > 0: rounds x the key groups
+static int attn_tma_stages(int hd, bool split, int hpc, int rounds) {
     const int G = atm::NCW / hpc;
+    if (rounds > 0) return G * rounds;
     const size_t st = attn_tma_stage(hd, split, attn_tma_kt(hpc));
     const int k = std::max(1, (int)((100u << 10) / (st * G)));
     return G * std::min(k, std::max(1, 4 / G));
+}
+
+// Decomposition overrides for measurement sweeps (unset or 0 = the built-in
+// policy): DFLASH_ATTN_HPC (q heads per CTA: 1, 2 or 4), DFLASH_ATTN_SPLITS (key
+// splits, at most 8), DFLASH_ATTN_ROUNDS (ring stages per key group)
+struct AttnTune {
+    int hpc = 0, splits = 0, rounds = 0;
+    AttnTune() {
+        auto env_int = [](const char *name) {
+            const char *v = getenv(name);
+            return v ? atoi(v) : 0;
+        };
+        hpc = env_int("DFLASH_ATTN_HPC");
+        splits = env_int("DFLASH_ATTN_SPLITS");
+        rounds = std::max(0, std::min(16, env_int("DFLASH_ATTN_ROUNDS")));
+    }
+};
+static const AttnTune &attn_tune() {
+    static const AttnTune t;
+    return t;
 }
 
 static size_t attn_tma_smem(int hd, bool split, int hpc, int S, int stages) {
@@ -663,14 +688,17 @@ int launch_attention_tma(const AttnTmaMaps &maps, AttnTmaArgs a, int hd, bool sp
     if (a.R <= 0) return 0;
     const int grp = a.nq / a.nkv;
     const int n_tiles = (a.R + a.rows_per_tile - 1) / a.rows_per_tile;
-    const int hpc = attn_tma_hpc(grp, n_tiles, a.nkv, num_sms);
+    const AttnTune &tune = attn_tune();
+    int hpc = attn_tma_hpc(grp, n_tiles, a.nkv, num_sms);
+    if ((tune.hpc == 1 || tune.hpc == 2 || tune.hpc == 4) && grp % tune.hpc == 0) hpc = tune.hpc;
     const int kt = attn_tma_kt(hpc);
     const CUtensorMap &mk = kt == 32 ? maps.k32 : maps.k16, &mv = kt == 32 ? maps.v32 : maps.v16;
     const int units = n_tiles * (a.nq / hpc);
     // splits of one (tile, head group) form a cluster of at most 8 CTAs; enough
     // CTAs for two per SM, no more splits than key tiles the longest context has
     a.n_splits = std::max(1, std::min({8, (2 * num_sms + units - 1) / units, (a.max_len + kt - 1) / kt}));
-    a.stages = attn_tma_stages(hd, split, hpc);
+    if (tune.splits > 0) a.n_splits = std::min({8, tune.splits, (a.max_len + kt - 1) / kt});
+    a.stages = attn_tma_stages(hd, split, hpc, tune.rounds);
     cudaError_t e = cudaErrorInvalidValue;
 #define ATM_CASE(HD_, SP_, HPC_)                                                  \
     if (hd == HD_ && split == SP_ && hpc == HPC_) e = launch_one<HD_, SP_, HPC_>(mk, mv, a, n_tiles, s);
