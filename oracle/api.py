@@ -9,7 +9,7 @@ import torch
 
 from .build import build_oracle
 
-ORC_F32, ORC_BF16, ORC_FP8 = 0, 1, 2
+ORC_F32, ORC_BF16, ORC_FP8, ORC_MXFP4 = 0, 1, 2, 3
 
 _lib = None
 
@@ -40,6 +40,12 @@ class Fp8(C.Structure):
     _fields_ = [("codes", C.c_void_p), ("scale", C.c_void_p)]
 
 
+class Mx4(C.Structure):
+    """orc_mxfp4: packed E2M1 codes [rows][K/2], block exponents [K/128][rows][4],
+    one fp32 scale per row, and the matrix's row count."""
+    _fields_ = [("codes", C.c_void_p), ("bscale", C.c_void_p), ("scale", C.c_void_p), ("rows", C.c_int64)]
+
+
 class Spec(C.Structure):
     _fields_ = [("target", Model), ("drafter", Model), ("block_size", C.c_int32),
                 ("n_taps", C.c_int32), ("tap_layers", C.POINTER(C.c_int32)),
@@ -65,6 +71,8 @@ def load_lib():
                                     C.c_void_p]
     lib.orc_e4m3_value.argtypes = [C.c_uint8]
     lib.orc_e4m3_value.restype = C.c_double
+    lib.orc_e2m1_value.argtypes = [C.c_uint8]
+    lib.orc_e2m1_value.restype = C.c_double
     lib.orc_attend.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_void_p]
     lib.orc_argmax.argtypes = [C.c_void_p, C.c_int32, C.c_void_p]
     lib.orc_argmax.restype = C.c_int32
@@ -135,12 +143,15 @@ class OracleSpec:
         w = {k: _wtensor(v) for k, v in weights.items()}
         self._keep.append(w)
         dtype = ORC_BF16 if w["embed"].dtype == torch.bfloat16 else ORC_F32
-        self.mat_dtype = ORC_FP8 if w["lm_head"].dtype == torch.uint8 else dtype
+        if w["lm_head"].dtype == torch.uint8:
+            self.mat_dtype = ORC_MXFP4 if "lm_head.bscale" in w else ORC_FP8
+        else:
+            self.mat_dtype = dtype
         for k, v in w.items():
-            if k == "embed" or k.endswith(".scale"):
+            if k == "embed" or k.endswith(".scale") or k.endswith(".bscale"):
                 continue
             if v.dim() > 1 and v.dtype != {ORC_BF16: torch.bfloat16, ORC_F32: torch.float32,
-                                           ORC_FP8: torch.uint8}[self.mat_dtype]:
+                                           ORC_FP8: torch.uint8, ORC_MXFP4: torch.uint8}[self.mat_dtype]:
                 raise TypeError(f"{k}: mixed storage types")
             if v.dim() == 1 and v.dtype != torch.float32:
                 raise TypeError(f"{k}: norm gains must be fp32")
@@ -158,11 +169,15 @@ class OracleSpec:
         self.spec.fc_norm = _ptr(w["fuse.norm"])
 
     def _mat(self, name):
-        """Address the oracle reads matrix `name` from: its storage, or for FP8
-        weights an orc_fp8 descriptor of its codes and per-row scales."""
-        if self.mat_dtype != ORC_FP8:
+        """Address the oracle reads matrix `name` from: its storage, or for FP8 /
+        MXFP4 weights a descriptor of its codes and scales."""
+        if self.mat_dtype == ORC_FP8:
+            q = Fp8(_ptr(self._w[name]), _ptr(self._w[name + ".scale"]))
+        elif self.mat_dtype == ORC_MXFP4:
+            q = Mx4(_ptr(self._w[name]), _ptr(self._w[name + ".bscale"]), _ptr(self._w[name + ".scale"]),
+                    self._w[name].shape[0])
+        else:
             return _ptr(self._w[name])
-        q = Fp8(_ptr(self._w[name]), _ptr(self._w[name + ".scale"]))
         self._keep.append(q)
         return C.addressof(q)
 
@@ -171,8 +186,8 @@ class OracleSpec:
         m.d = dims(d)
         m.dtype = dtype
         m.mat_dtype = self.mat_dtype
-        if self.mat_dtype == ORC_FP8 and d.n_experts > 0:
-            raise ValueError("the oracle reads FP8 weights for dense models only")
+        if self.mat_dtype in (ORC_FP8, ORC_MXFP4) and d.n_experts > 0:
+            raise ValueError("the oracle reads FP8 / MXFP4 weights for dense models only")
         m.embed = _ptr(w["embed"])
         m.lm_head = self._mat("lm_head")
         m.final_norm = _ptr(w[f"{prefix}.final_norm"])
@@ -360,6 +375,26 @@ def matmul_fp8(codes: torch.Tensor, scale: torch.Tensor, X, row0: int = 0, n_row
 
 def e4m3_value(code: int) -> float:
     return load_lib().orc_e4m3_value(int(code) & 0xFF)
+
+
+def e2m1_value(code: int) -> float:
+    return load_lib().orc_e2m1_value(int(code) & 0xF)
+
+
+def matmul_mxfp4(codes: torch.Tensor, bscale: torch.Tensor, scale: torch.Tensor, X, row0: int = 0,
+                 n_rows: Optional[int] = None) -> np.ndarray:
+    """Y[r][n] = sum_k W_q[row0+n][k] * X[r][k] through the oracle (W_q the MXFP4
+    matrix's quantised weights)."""
+    lib = load_lib()
+    codes, bscale, scale = _wtensor(codes), _wtensor(bscale), _wtensor(scale)
+    N, K2 = codes.shape
+    K = 2 * K2
+    n = N - row0 if n_rows is None else n_rows
+    q = Mx4(_ptr(codes), _ptr(bscale), _ptr(scale), N)
+    XX = _f64(X).reshape(-1, K)
+    Y = np.zeros((XX.shape[0], n), np.float64)
+    lib.orc_matmul_rows(C.addressof(q), ORC_MXFP4, row0, n, K, XX.ctypes.data, XX.shape[0], Y.ctypes.data)
+    return Y
 
 
 def attend(q, keys, vals) -> np.ndarray:

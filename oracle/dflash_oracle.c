@@ -81,6 +81,30 @@ double orc_e4m3_value(uint8_t c) {
     return (c & 0x80) ? -mag : mag;
 }
 
+/* E2M1 (OCP 4-bit float: sign bit, 2 exponent bits with bias 1, 1 mantissa
+ * bit, no infinities or NaN): sign * 2^(e-1) * (1 + m/2) for e > 0, sign * m/2
+ * for e = 0.  Written from that definition. */
+double orc_e2m1_value(uint8_t c) {
+    int32_t e = (c >> 1) & 3, m = c & 1;
+    double mag = e == 0 ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, e - 1);
+    return (c & 8) ? -mag : mag;
+}
+
+/* Dot product of row `row` of an MXFP4 matrix: the quantised weight of element
+ * k is scale[row] * 2^(E - 127) * e2m1_value(code_k), with E the block scale
+ * byte of k's 32-value block (fp64), summed like the other dot products. */
+static double dot_mxfp4(const orc_mxfp4 *q, size_t row, const double *x, int32_t K) {
+    const uint8_t *c = q->codes + row * (size_t)(K / 2);
+    const double sc = (double)q->scale[row];
+    double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int32_t k = 0; k < K; ++k) {
+        const uint8_t code = (k & 1) ? (uint8_t)(c[k / 2] >> 4) : (uint8_t)(c[k / 2] & 15);
+        const uint8_t e = q->bscale[(((size_t)(k / 128) * (size_t)q->rows + row) * 4) + (size_t)((k / 32) % 4)];
+        acc[k % 8] += sc * ldexp(orc_e2m1_value(code), (int)e - 127) * x[k];
+    }
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
 /* Dot product of one row of an FP8 matrix: the quantised weight of element k
  * is scale * e4m3_value(code_k) (fp64), summed like the other dot products. */
 static double dot_fp8(const uint8_t *c, double scale, const double *x, int32_t K) {
@@ -176,6 +200,8 @@ void orc_matmul_rows(const void *W, int32_t dtype, int32_t row0, int32_t N, int3
             if (dtype == ORC_FP8) {
                 const orc_fp8 *q = (const orc_fp8 *)W;
                 v = dot_fp8(q->codes + row * K, (double)q->scale[row], X + (size_t)r * K, K);
+            } else if (dtype == ORC_MXFP4) {
+                v = dot_mxfp4((const orc_mxfp4 *)W, row, X + (size_t)r * K, K);
             } else if (dtype == ORC_BF16) {
                 v = dot_bf16((const uint16_t *)W + row * K, X + (size_t)r * K, K);
             } else {

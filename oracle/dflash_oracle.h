@@ -33,7 +33,7 @@
 extern "C" {
 #endif
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8 = 2, ORC_MXFP4 = 3 };
 
 /* A matrix in FP8 storage: E4M3 codes [rows][K] and one fp32 scale per row;
  * the quantised weight is scale[row] * e4m3_value(code).  Matrix pointers of
@@ -42,6 +42,20 @@ typedef struct {
     const uint8_t *codes;
     const float *scale;
 } orc_fp8;
+
+/* A matrix in MXFP4 storage (OCP Microscaling: FP4 E2M1 elements sharing a
+ * power-of-two scale per 32 values along K) with one fp32 scale per row:
+ * codes [rows][K/2] (element k in byte k/2, low nibble for even k), bscale
+ * [K/128][rows][4] (byte (k/128, row, (k/32) % 4) = the block's exponent + 127),
+ * scale [rows].  The quantised weight of element (row, k) is
+ * scale[row] * 2^(bscale byte - 127) * e2m1_value(code).  Matrix pointers of an
+ * ORC_MXFP4 model point to one of these. */
+typedef struct {
+    const uint8_t *codes;
+    const uint8_t *bscale;
+    const float *scale;
+    int64_t rows;             /* rows of the whole matrix (the bscale row stride) */
+} orc_mxfp4;
 
 typedef struct {
     int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
@@ -76,7 +90,8 @@ typedef struct {
     const float *final_norm;  /* [H] */
     const orc_layer *layers;  /* [n_layers] */
     int32_t mat_dtype;        /* storage of the projection matrices, the LM head and W_fc:
-                                 ORC_F32, ORC_BF16 or ORC_FP8 (pointers to orc_fp8) */
+                                 ORC_F32, ORC_BF16, ORC_FP8 (pointers to orc_fp8) or
+                                 ORC_MXFP4 (pointers to orc_mxfp4) */
 } orc_model;
 
 typedef struct {
@@ -106,6 +121,8 @@ void orc_matmul_rows(const void *W, int32_t dtype, int32_t row0, int32_t N, int3
                      const double *X, int32_t R, double *Y);
 /* Value of an E4M3 code (NaN for 0x7F / 0xFF). */
 double orc_e4m3_value(uint8_t code);
+/* Value of a 4-bit E2M1 code (0..15). */
+double orc_e2m1_value(uint8_t code);
 /* One query row over keys[0..n_keys) (each hd doubles, stride ld_k); softmax scale 1/sqrt(hd). */
 void orc_attend(const double *q, const double *keys, const double *vals, int64_t ld_kv,
                 int32_t n_keys, int32_t head_dim, double *out);

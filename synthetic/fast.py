@@ -13,7 +13,8 @@ from typing import Optional
 import torch
 
 from .configs import SpecConfig
-from .weights import SIGMA_S, tensor_key, weight_shapes, storage_dtype
+from .weights import (QUANT_KINDS, SIGMA_S, _layer_base_shape, quantized, split_part, storage_dtype, tensor_key,
+                      weight_shapes)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -53,10 +54,9 @@ def make_weight_host(cfg: SpecConfig, name: str, random_gains: bool = False, see
         lib.fastgen_f32(t.data_ptr(), n, key, float(torch.tensor(0.1 / SIGMA_S, dtype=torch.float32)), 1.0, 1)
         return t
     scale = float(torch.tensor(cfg.weight_std / SIGMA_S, dtype=torch.float32))
-    if kind in ("fp8", "scale"):
-        from .weights import quantized
-        base = name[:-len(".scale")] if kind == "scale" else name
-        bshape = weight_shapes(cfg)[base][0]
+    if kind in QUANT_KINDS:
+        base, part = split_part(name, kind)
+        bshape = _layer_base_shape(cfg, base)
         bn = 1
         for d in bshape:
             bn *= d
@@ -65,8 +65,7 @@ def make_weight_host(cfg: SpecConfig, name: str, random_gains: bool = False, see
             t = torch.empty(bshape, dtype=torch.bfloat16)
             lib.fastgen_bf16(t.data_ptr(), bn, tensor_key(base, seed), scale)
             return t
-        codes, sc = quantized(base, (cfg.name, seed, "cpu", cfg.weight_std), make_base)
-        return sc if kind == "scale" else codes
+        return quantized(base, (cfg.name, seed, "cpu", cfg.weight_std), make_base, cfg.dtype)[part]
     if storage_dtype(cfg) == torch.bfloat16:
         t = torch.empty(shape, dtype=torch.bfloat16)
         lib.fastgen_bf16(t.data_ptr(), n, key, scale)

@@ -121,7 +121,10 @@ def weight_shapes(cfg: SpecConfig) -> "OrderedDict[str, Tuple[Tuple[int, ...], s
 
     With cfg.dtype == "fp8" every matrix but the embedding is stored as E4M3
     codes (kind "fp8", uint8) plus "<name>.scale" (kind "scale", fp32, one
-    value per row); see synthetic.fp8."""
+    value per row); see synthetic.fp8.  With cfg.dtype == "fp4" the same
+    matrices are MXFP4: packed E2M1 codes (kind "fp4", uint8 [rows, K/2]),
+    "<name>.bscale" (kind "bscale", uint8 [K/128, rows, 4]) and "<name>.scale";
+    see synthetic.fp4."""
     t, dr = cfg.target, cfg.drafter
     s: "OrderedDict[str, Tuple[Tuple[int, ...], str]]" = OrderedDict()
     s["embed"] = ((t.vocab, t.hidden), "matrix")
@@ -130,18 +133,29 @@ def weight_shapes(cfg: SpecConfig) -> "OrderedDict[str, Tuple[Tuple[int, ...], s
     s.update(_layer_shapes("drafter", dr))
     s["fuse.w_fc"] = ((dr.hidden, cfg.n_taps * t.hidden), "matrix")
     s["fuse.norm"] = ((dr.hidden,), "norm")
-    if cfg.dtype != "fp8":
+    if cfg.dtype not in ("fp8", "fp4"):
         return s
     if t.is_moe:
-        raise ValueError("fp8 weights are built for dense targets only")
+        raise ValueError(f"{cfg.dtype} weights are built for dense targets only")
     q: "OrderedDict[str, Tuple[Tuple[int, ...], str]]" = OrderedDict()
     for name, (shape, kind) in s.items():
         if kind == "matrix" and name != "embed":
-            q[name] = (shape, "fp8")
+            if cfg.dtype == "fp8":
+                q[name] = (shape, "fp8")
+            else:
+                rows, K = shape
+                q[name] = ((rows, K // 2), "fp4")
+                q[name + ".bscale"] = ((K // 128, rows, 4), "bscale")
             q[name + ".scale"] = (shape[:-1], "scale")
         else:
             q[name] = (shape, kind)
     return q
+
+
+def _layer_base_shape(cfg: SpecConfig, base: str) -> Tuple[int, ...]:
+    """Logical shape [rows, K] of a quantised matrix (its codes' shape for fp8)."""
+    shape, kind = weight_shapes(cfg)[base]
+    return (shape[0], shape[1] * 2) if kind == "fp4" else shape
 
 
 def weight_names(cfg: SpecConfig):
@@ -149,21 +163,39 @@ def weight_names(cfg: SpecConfig):
 
 
 def storage_dtype(cfg: SpecConfig) -> torch.dtype:
-    """Type of the generated matrices (fp8 models quantise bf16 ones)."""
-    return torch.bfloat16 if cfg.dtype in ("bf16", "fp8") else torch.float32
+    """Type of the generated matrices (fp8 and fp4 models quantise bf16 ones)."""
+    return torch.bfloat16 if cfg.dtype in ("bf16", "fp8", "fp4") else torch.float32
 
 
 _QCACHE: dict = {}
 
 
-def quantized(name: str, key, make_base):
-    """(codes, scale) of matrix `name`, cached for the codes / scale pair."""
-    from .fp8 import quantize_rows
-    k = (name, key)
+QUANT_KINDS = ("fp8", "fp4", "bscale", "scale")
+
+
+def quantized(name: str, key, make_base, fmt: str = "fp8"):
+    """The stored parts of matrix `name` quantised to `fmt`: {"": codes, ".scale":
+    row scales} (+ ".bscale" for fp4), cached while the parts are fetched."""
+    k = (name, key, fmt)
     if k not in _QCACHE:
         _QCACHE.clear()
-        _QCACHE[k] = quantize_rows(make_base())
+        if fmt == "fp8":
+            from .fp8 import quantize_rows
+            codes, scale = quantize_rows(make_base())
+            _QCACHE[k] = {"": codes, ".scale": scale}
+        else:
+            from .fp4 import quantize_mx
+            codes, bscale, scale = quantize_mx(make_base())
+            _QCACHE[k] = {"": codes, ".bscale": bscale, ".scale": scale}
     return _QCACHE[k]
+
+
+def split_part(name: str, kind: str) -> Tuple[str, str]:
+    """(matrix name, part suffix) of a stored tensor of a quantised matrix."""
+    for suf in (".scale", ".bscale"):
+        if kind in ("scale", "bscale") and name.endswith(suf):
+            return name[:-len(suf)], suf
+    return name, ""
 
 
 def make_weight(cfg: SpecConfig, name: str, device="cpu", random_gains: bool = False,
@@ -174,13 +206,13 @@ def make_weight(cfg: SpecConfig, name: str, device="cpu", random_gains: bool = F
         if not random_gains:
             return torch.ones(shape, dtype=torch.float32, device=device)
         return _fill(shape, name, seed, 0.1 / SIGMA_S, 1.0, torch.float32, device)
-    if kind in ("fp8", "scale"):
-        base = name[:-len(".scale")] if kind == "scale" else name
-        bshape = weight_shapes(cfg)[base][0]
-        codes, scale = quantized(base, (cfg.name, seed, str(device), cfg.weight_std),
-                                 lambda: _fill(bshape, base, seed, cfg.weight_std / SIGMA_S, 0.0, torch.bfloat16,
-                                               device))
-        return scale if kind == "scale" else codes
+    if kind in QUANT_KINDS:
+        base, part = split_part(name, kind)
+        bshape = _layer_base_shape(cfg, base)
+        parts = quantized(base, (cfg.name, seed, str(device), cfg.weight_std),
+                          lambda: _fill(bshape, base, seed, cfg.weight_std / SIGMA_S, 0.0, torch.bfloat16, device),
+                          cfg.dtype)
+        return parts[part]
     return _fill(shape, name, seed, cfg.weight_std / SIGMA_S, 0.0, storage_dtype(cfg), device)
 
 
