@@ -118,16 +118,18 @@ def iteration_bytes(cfg, batch: int, mean_ctx: float, kv_planes: int = 1) -> flo
     """Algorithmic HBM bytes of one draft+verify iteration: every projection
     matrix once (the LM head twice: drafter and target), plus K/V reads of both
     models at the mean context length (kv_planes bf16 planes per element)."""
-    es = 2 if cfg.dtype in ("bf16", "fp8") else 4   # activations / K/V (and bf16 weights)
+    es = 2 if cfg.dtype in ("bf16", "fp8", "fp4") else 4   # activations / K/V (and bf16 weights)
     shapes = weight_shapes(cfg)
     w = 0
     for name, (shape, kind) in shapes.items():
-        if kind not in ("matrix", "fp8", "scale") or name == "embed":
+        if kind not in ("matrix", "fp8", "fp4", "bscale", "scale") or name == "embed":
             continue
         n = int(np.prod(shape))
         if name.endswith("we_gate_up") or name.endswith("we_down"):
             continue  # MoE experts: only the touched ones are read (below)
-        wes = {"matrix": es, "fp8": 1, "scale": 4}[kind]
+        # stored bytes per element of each kind (fp4 codes are stored two a byte,
+        # so their stored shape already counts bytes)
+        wes = {"matrix": es, "fp8": 1, "fp4": 1, "bscale": 1, "scale": 4}[kind]
         w += n * wes * (2 if name.startswith("lm_head") else 1)
     t, d = cfg.target, cfg.drafter
     if t.is_moe:
@@ -261,8 +263,8 @@ def main():
     ap.add_argument("--no-sampling", action="store_true")
     ap.add_argument("--bf16-act", choices=["split", "fast"], default="split",
                     help="bf16 activations as two planes (parity-grade) or one plane")
-    ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
-                    help="weight storage: bf16, or FP8 E4M3 codes with per-row scales (a quantised model)")
+    ap.add_argument("--weights", choices=["bf16", "fp8", "fp4"], default="bf16",
+                    help="weight storage: bf16, FP8 E4M3 codes with per-row scales, or MXFP4 (quantised models)")
     ap.add_argument("--e2e-tokens", type=int, default=128)
     ap.add_argument("--profile-steps", type=int, default=50)
     ap.add_argument("--target-layers", type=int, default=None, help="layer-reduced copy (profiling small cases)")
@@ -282,8 +284,8 @@ def main():
         cfg = cfg.with_(prompt_len=args.prompt_len)
     if args.block_size:
         cfg = cfg.with_(block_size=args.block_size)
-    if args.weights == "fp8":
-        cfg = cfg.with_(dtype="fp8")
+    if args.weights in ("fp8", "fp4"):
+        cfg = cfg.with_(dtype=args.weights)
     if args.target_layers or args.drafter_layers:
         from synthetic.configs import shrink
         cfg = shrink(cfg, target_layers=args.target_layers or cfg.target.n_layers,
@@ -566,8 +568,11 @@ def workload_config(cfg, args, world, prompt_len=None):
             "global_batch": b * world, "seq_len": plen, "block_size": B,
             "parallelism": f"replicas x{world}",
             "activations": ("bf16 hi+lo planes, fp32 accumulate" if args.bf16_act == "split"
-                            else "bf16 single plane, fp32 accumulate") if cfg.dtype in ("bf16", "fp8") else "fp32",
+                            else "bf16 single plane, fp32 accumulate") if cfg.dtype in ("bf16", "fp8", "fp4")
+            else "fp32",
             "weights": {"bf16": "bf16", "fp8": "FP8 E4M3 codes + per-row fp32 scales (quantised model)",
+                        "fp4": "MXFP4: E2M1 codes + a power-of-two scale per 32 values + per-row fp32 scales "
+                               "(quantised model)",
                         "fp32": "fp32"}[cfg.dtype],
             "l2": l2_note(cfg)}
 

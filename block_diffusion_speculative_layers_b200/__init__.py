@@ -19,8 +19,9 @@ from .build import lib_path
 
 DFLASH_OK, DFLASH_EINVAL, DFLASH_ESTATE, DFLASH_ECAPACITY = 0, 1, 2, 3
 DFLASH_ECUDA, DFLASH_ENUMERIC, DFLASH_ETIMEOUT, DFLASH_EUNSUPPORTED = 4, 5, 6, 7
-DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST, DFLASH_FP8 = 0, 1, 2, 3
-_SLOT_TYPES = {DFLASH_FP32: (torch.float32, 4), DFLASH_BF16: (torch.bfloat16, 2), DFLASH_FP8: (torch.uint8, 1)}
+DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST, DFLASH_FP8, DFLASH_FP4, DFLASH_UE8M0 = 0, 1, 2, 3, 4, 5
+_SLOT_TYPES = {DFLASH_FP32: (torch.float32, 4), DFLASH_BF16: (torch.bfloat16, 2), DFLASH_FP8: (torch.uint8, 1),
+               DFLASH_FP4: (torch.uint8, 1), DFLASH_UE8M0: (torch.uint8, 1)}
 DFLASH_DRAFT_MODEL, DFLASH_DRAFT_SCRIPT = 0, 1
 MAX_TAPS, MAX_BLOCK = 8, 32
 # dflash_profile_read classes, in the order of the DFLASH_PROF_* values
@@ -161,6 +162,8 @@ def make_config(spec, max_batch: int = 1, max_len: int = 4096, prefill_chunk: in
         c.dtype = DFLASH_BF16 if bf16_act == "split" else DFLASH_BF16_FAST
     elif spec.dtype == "fp8":
         c.dtype = DFLASH_FP8
+    elif spec.dtype == "fp4":
+        c.dtype = DFLASH_FP4
     else:
         c.dtype = DFLASH_FP32
     c.keep_logits = 1 if keep_logits else 0
@@ -391,4 +394,4 @@ class DFlash:
 
 __all__ = ["DFlash", "DFlashError", "load_library", "make_config", "Config", "Stats", "EXPORTS",
            "DFLASH_DRAFT_MODEL", "DFLASH_DRAFT_SCRIPT", "DFLASH_FP32", "DFLASH_BF16", "DFLASH_BF16_FAST",
-           "DFLASH_FP8"]
+           "DFLASH_FP8", "DFLASH_FP4"]

@@ -71,7 +71,9 @@ static void *noalloc_scratch_ptr(int dev, std::string &err) {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-static int elem_size(int dtype) { return dtype == DFLASH_FP32 ? 4 : dtype == DFLASH_FP8 ? 1 : 2; }
+static int elem_size(int dtype) {
+    return dtype == DFLASH_FP32 ? 4 : (dtype == DFLASH_FP8 || dtype == DFLASH_FP4 || dtype == DFLASH_UE8M0) ? 1 : 2;
+}
 
 static bool check_model(const dflash_model_cfg &m, std::string &why) {
     if (m.n_layers < 1 || m.hidden < 32 || m.n_q_heads < 1 || m.n_kv_heads < 1 || m.vocab < 2) {
@@ -119,9 +121,21 @@ static bool check_config(const dflash_config &c, std::string &why) {
     if (c.max_batch < 1 || c.max_batch > 64) { why = "max_batch must be in [1, 64]"; return false; }
     if (c.max_len < c.block_size + 1 || c.max_len > (1 << 20)) { why = "max_len out of range"; return false; }
     if (c.prefill_chunk < 0 || c.prefill_chunk > 8192) { why = "prefill_chunk must be in [0, 8192]"; return false; }
-    if (c.dtype != DFLASH_FP32 && c.dtype != DFLASH_BF16 && c.dtype != DFLASH_BF16_FAST && c.dtype != DFLASH_FP8) {
-        why = "dtype must be DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST or DFLASH_FP8";
+    if (c.dtype != DFLASH_FP32 && c.dtype != DFLASH_BF16 && c.dtype != DFLASH_BF16_FAST && c.dtype != DFLASH_FP8 &&
+        c.dtype != DFLASH_FP4) {
+        why = "dtype must be DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST, DFLASH_FP8 or DFLASH_FP4";
         return false;
+    }
+    if (c.dtype == DFLASH_FP4) {
+        // MXFP4 rows: K (hidden, ffn, q width, n_taps * hidden) in whole 128-value groups
+        const dflash_model_cfg *ms[2] = {&c.target, &c.drafter};
+        for (const dflash_model_cfg *m : ms) {
+            if (m->n_experts > 0) { why = "FP4 weights need dense models"; return false; }
+            if (m->hidden % 128 || m->ffn % 128 || (m->n_q_heads * m->head_dim) % 128) {
+                why = "FP4 weights need hidden, ffn and q width multiples of 128";
+                return false;
+            }
+        }
     }
     if (c.dtype == DFLASH_FP8) {
         const dflash_model_cfg *ms[2] = {&c.target, &c.drafter};
@@ -138,10 +152,17 @@ static bool check_config(const dflash_config &c, std::string &why) {
 
 static void add_slot(Layout &L, const std::string &name, int ndim, int64_t d0, int64_t d1, int64_t d2, int dtype);
 
-// A projection matrix [d0, d1]; FP8 storage adds "<name>.scale" [d0] (fp32, one per row).
+// A projection matrix [d0, d1]; FP8 storage adds "<name>.scale" [d0] (fp32, one per
+// row); FP4 (MXFP4) stores the codes two per byte [d0, d1/2] and adds
+// "<name>.bscale" [d1/128, d0, 4] (UE8M0 block exponents) and "<name>.scale".
 static void add_matrix(Layout &L, const std::string &name, int64_t d0, int64_t d1, int dtype) {
-    add_slot(L, name, 2, d0, d1, 0, dtype);
-    if (dtype == DFLASH_FP8) add_slot(L, name + ".scale", 1, d0, 0, 0, DFLASH_FP32);
+    if (dtype == DFLASH_FP4) {
+        add_slot(L, name, 2, d0, d1 / 2, 0, DFLASH_FP4);
+        add_slot(L, name + ".bscale", 3, d1 / 128, d0, 4, DFLASH_UE8M0);
+    } else {
+        add_slot(L, name, 2, d0, d1, 0, dtype);
+    }
+    if (dtype == DFLASH_FP8 || dtype == DFLASH_FP4) add_slot(L, name + ".scale", 1, d0, 0, 0, DFLASH_FP32);
 }
 
 static void add_slot(Layout &L, const std::string &name, int ndim, int64_t d0, int64_t d1, int64_t d2, int dtype) {
@@ -188,7 +209,7 @@ static Layout make_layout(const dflash_config &c) {
     // weight storage: fp32 or bf16 (both bf16 activation modes store bf16 weights);
     // FP8: every projection matrix as E4M3 codes + row scales, the embedding in bf16
     const int dt_emb = c.dtype == DFLASH_FP32 ? DFLASH_FP32 : DFLASH_BF16, es = elem_size(dt_emb);
-    const int dt = c.dtype == DFLASH_FP8 ? DFLASH_FP8 : dt_emb;
+    const int dt = (c.dtype == DFLASH_FP8 || c.dtype == DFLASH_FP4) ? c.dtype : dt_emb;
     const dflash_model_cfg &t = c.target, &d = c.drafter;
     add_slot(L, "embed", 2, t.vocab, t.hidden, 0, dt_emb);
     add_matrix(L, "lm_head", t.vocab, t.hidden, dt);
@@ -241,7 +262,7 @@ static Layout make_layout(const dflash_config &c) {
     // MoE decode: the pairs' activation rows in expert-grouped order
     L.moe_xg = take(t.n_experts > 0 ? (size_t)L.R_dec * t.top_k * H * es : 16);
     const size_t act_bytes = align_up(o, 256) - act0;
-    if (c.dtype == DFLASH_BF16 || c.dtype == DFLASH_FP8) {
+    if (c.dtype == DFLASH_BF16 || c.dtype == DFLASH_FP8 || c.dtype == DFLASH_FP4) {
         take(act_bytes);
         L.act_lo = act_bytes / es;
     }
@@ -306,9 +327,9 @@ static Layout make_layout(const dflash_config &c) {
         L.dep_v = take((size_t)2 * L.n_ops_v * 4);
         L.dep_d = take((size_t)2 * L.n_ops_d * 4);
     }
-    // FP8 projections: the activation rows as MX planes (codes + scale words), sized
-    // for the most rows and the widest K of any projection
-    if (c.dtype == DFLASH_FP8) {
+    // FP8 / FP4 projections: the activation rows as MX planes (codes + scale words),
+    // sized for the most rows and the widest K of any projection
+    if (c.dtype == DFLASH_FP8 || c.dtype == DFLASH_FP4) {
         const int kmax = std::max({t.hidden, d.hidden, qmax, fmax, TK});
         L.mx_mpad = (int)align_up((size_t)L.R_max, 32);
         L.mx_kpad = (int)align_up((size_t)kmax, 128);
@@ -340,9 +361,12 @@ class Engine : public EngineBase {
     // weights
     const T *embed;
     const void *lm_head, *w_fc;
-    // FP8 weights: the scale vector of every projection matrix, by its base address
-    bool f8_ = false;
+    // FP8 / FP4 weights (f8_: either; f4_: MXFP4): the scale vector of every
+    // projection matrix and, for FP4, its block exponents and row count, by the
+    // matrix's base address
+    bool f8_ = false, f4_ = false;
     std::unordered_map<const void *, const float *> wscales;
+    std::unordered_map<const void *, std::pair<const uint8_t *, int>> wbscales;
     const float *fc_norm, *t_final, *d_final;
     std::vector<LayerW> tl, dl;
     // state
@@ -415,12 +439,21 @@ class Engine : public EngineBase {
         embed = (const T *)wslot(by, "embed");
         lm_head = wslot(by, "lm_head");
         w_fc = wslot(by, "fuse.w_fc");
-        f8_ = c.dtype == DFLASH_FP8;
+        f8_ = c.dtype == DFLASH_FP8 || c.dtype == DFLASH_FP4;
+        f4_ = c.dtype == DFLASH_FP4;
+        auto ends = [](const std::string &s, const char *suf) {
+            const size_t n = strlen(suf);
+            return s.size() > n && s.compare(s.size() - n, n, suf) == 0;
+        };
         if (f8_)
-            for (const WeightSlot &sl : L.slots)
-                if (sl.name.size() > 6 && sl.name.compare(sl.name.size() - 6, 6, ".scale") == 0)
+            for (const WeightSlot &sl : L.slots) {
+                if (ends(sl.name, ".scale"))
                     wscales[W + L.slots[by.at(sl.name.substr(0, sl.name.size() - 6))].offset] =
                         (const float *)(W + sl.offset);
+                if (ends(sl.name, ".bscale"))
+                    wbscales[W + L.slots[by.at(sl.name.substr(0, sl.name.size() - 7))].offset] = {
+                        (const uint8_t *)(W + sl.offset), (int)sl.shape[1]};
+            }
         fc_norm = (const float *)wslot(by, "fuse.norm");
         t_final = (const float *)wslot(by, "target.final_norm");
         d_final = (const float *)wslot(by, "drafter.final_norm");
@@ -523,7 +556,7 @@ class Engine : public EngineBase {
             // pass instead of griddepcontrol.wait (same results; measured 0.2 ms per step
             // slower on B200: the fences of every writer cost more than the grid release)
             const char *dv_env = getenv("DFLASH_DEP_COUNTERS");
-            dep_on = dv_env && dv_env[0] == '1' && !f8_;  // FP8 projections run a quantiser launch first
+            dep_on = dv_env && dv_env[0] == '1' && !f8_;  // FP8 / FP4 projections run a quantiser launch first
             const char *fv = getenv("DFLASH_FOLDED_NORM");
             const bool allow = !(fv && fv[0] == '0');
             fold_draft_ok = allow && bf && shapes;
@@ -705,7 +738,10 @@ class Engine : public EngineBase {
     double gemm_bytes(int M, int N, int K, const Epi<T> &e) const {
         const double es = sizeof(T), ea = es * (lo_ ? 2 : 1);
         const int wrows = e.kind == EPI_SWIGLU ? 2 * e.F : N;
-        double b = f8_ ? (double)wrows * K + 4.0 * wrows : (double)N * K * es;
+        // weights: FP4 half a byte per value + one exponent byte per 32 + the row
+        // scales; FP8 one byte per value + the row scales
+        double b = f4_ ? (double)wrows * K / 2 + (double)wrows * K / 32 + 4.0 * wrows
+                       : f8_ ? (double)wrows * K + 4.0 * wrows : (double)N * K * es;
         b += (double)M * K * ea;
         switch (e.kind) {
             case EPI_QKV: b += (double)M * N * ea; break;
@@ -722,37 +758,49 @@ class Engine : public EngineBase {
     // One projection; returns the CTAs launched (tensor-core path).  dep/done:
     // completion counters of a decode pass (see PassSync), else griddepcontrol.wait.
     // FP8 weights: the row scales of matrix Wt (its base address; rows from row0 on)
-    const float *scales_of(const void *Wt, int row0 = 0) const {
-        if (!f8_) return nullptr;
+    WScales scales_of(const void *Wt, int row0 = 0) const {
+        WScales w;
+        if (!f8_) return w;
         auto it = wscales.find(Wt);
-        return it == wscales.end() ? nullptr : it->second + row0;
+        if (it != wscales.end()) w.row = it->second + row0;
+        if (f4_) {
+            auto ib = wbscales.find(Wt);
+            if (ib != wbscales.end()) {
+                w.blk = ib->second.first;
+                w.blk_rows = ib->second.second;
+                w.blk_row0 = row0;
+            }
+        }
+        return w;
     }
-    // matrix Wt from row row0 on (FP8 codes are one byte per element)
+    // matrix Wt from row row0 on (FP8 codes are one byte per element, FP4 half a byte)
     const void *rows_of(const void *Wt, int row0, int K) const {
-        return (const char *)Wt + (size_t)row0 * K * (f8_ ? 1 : sizeof(T));
+        const size_t row_bytes = f4_ ? (size_t)K / 2 : f8_ ? (size_t)K : (size_t)K * sizeof(T);
+        return (const char *)Wt + (size_t)row0 * row_bytes;
     }
 
     int gemm(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e, const int *dep = nullptr,
-             int dep_target = 0, int *done = nullptr, const float *ws = nullptr) {
+             int dep_target = 0, int *done = nullptr, WScales ws = WScales()) {
         if (M <= 0) return 0;
         int ctas = 0;
-        if (!ws) ws = scales_of(Wt);
+        if (!ws.row) ws = scales_of(Wt);
         timed(DFLASH_PROF_PROJECTION, gemm_bytes(M, N, K, e),
               [&] { ctas = gemm_launch(X, ldx, M, Wt, N, K, e, dep, dep_target, done, ws); }, proj_class(N, K, e.kind));
         return ctas;
     }
 
     int gemm_launch(const T *X, int ldx, int M, const void *Wt, int N, int K, const Epi<T> &e_in,
-                    const int *dep = nullptr, int dep_target = 0, int *done = nullptr, const float *ws = nullptr) {
+                    const int *dep = nullptr, int dep_target = 0, int *done = nullptr, WScales ws = WScales()) {
         Epi<T> e = e_in;
         e.lo = lo_;  // every input and output of the engine's projections lives in the activation span
-        if (f8_ && !ws) ws = scales_of(Wt);
-        if (f8_ && !ws) {  // an FP8 matrix without its scales: refuse rather than read codes as bf16
+        if (f8_ && !ws.row) ws = scales_of(Wt);
+        if (f8_ && (!ws.row || (f4_ && !ws.blk))) {  // a quantised matrix without its scales: refuse
             tc.failed = true;
-            tc.err = "FP8 matrix without row scales";
+            tc.err = "FP8 / FP4 matrix without its scales";
             return 0;
         }
-        if (tc.supports(M, N, K)) return tc.run(X, ldx, M, Wt, N, K, e, s, dep, dep_target, done, ws);
+        if (tc.supports(M, N, K))
+            return tc.run(X, ldx, M, Wt, N, K, e, s, dep, dep_target, done, ws.row, ws.blk, ws.blk_rows, ws.blk_row0);
         // CUDA-core path (fp32 models): GEMM into fp32 Y, then the epilogue.
         float *Yo = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.Y : Y;
         const int ldy = (e.kind == EPI_STORE || e.kind == EPI_LOGITS) ? e.ldy : N;

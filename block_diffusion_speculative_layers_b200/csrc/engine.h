@@ -16,9 +16,17 @@ constexpr int kMaxDevices = 64;
 struct WeightSlot {
     std::string name;
     size_t offset = 0, numel = 0;
-    int dtype = 0;  // DFLASH_FP32 / DFLASH_BF16
+    int dtype = 0;  // DFLASH_FP32 / DFLASH_BF16 / DFLASH_FP8 / DFLASH_FP4 / DFLASH_UE8M0
     int ndim = 0;
     int64_t shape[3] = {0, 0, 0};
+};
+
+// Scales of a quantised projection matrix (from row blk_row0 on): FP8 / FP4 row
+// scales; FP4 block exponents [K/128][blk_rows][4] of the whole matrix
+struct WScales {
+    const float *row = nullptr;
+    const uint8_t *blk = nullptr;
+    int blk_rows = 0, blk_row0 = 0;
 };
 
 struct LayerW {

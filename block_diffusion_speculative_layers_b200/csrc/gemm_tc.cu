@@ -118,6 +118,19 @@ __host__ __device__ constexpr uint32_t idesc_mx(int n, int kb) {
            ((uint32_t)kb << 29);
 }
 
+// Plain (untiled) bulk copy global -> shared of `bytes` (a multiple of 16; both
+// addresses 16-byte aligned), completing on mbarrier `bar`
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t a) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
+}
+
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
@@ -146,7 +159,10 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
     uint8_t *sA = smem;
     uint8_t *sB = smem + (size_t)stages * A_ST;
     uint32_t *sW = (uint32_t *)(sB + (size_t)stages * B_ST);  // F8: [stages] scale words
-    float *stg = (float *)((uint8_t *)sW + (size_t)stages * SW_ST);
+    // FP4 weights: [stages][128] exponent words of the stage's weight rows
+    const bool f4 = F8 && p.w_bexp != nullptr;
+    uint32_t *sE = (uint32_t *)((uint8_t *)sW + (size_t)stages * SW_ST);
+    float *stg = (float *)((uint8_t *)sE + (f4 ? (size_t)stages * 512 : 0));
     float2 *red = (float2 *)(stg + 128 * STG_LD);
     RowMeta *smeta = (RowMeta *)(red + 4 * CH);
     float *rsc = (float *)(smeta + CH);       // [RS_MAX] row scales of the folded norm
@@ -178,7 +194,8 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
     // lane m, column m / 32) and one 4-column group per stage (plane row n at
     // lane n % 32 of every lane quarter, column n / 32; byte b of a word = the
     // scale of 32-K block b of the stage), as measured on the device
-    const int sf_cols = F8 ? 4 + 4 * stages : 0;
+    // FP4 weights: one 4-column group per stage for the weights' block scales too
+    const int sf_cols = F8 ? (f4 ? 8 * stages : 4 + 4 * stages) : 0;
     const int ncols = tmem_cols_for((persistent ? 2 * NC1 : NC1) + sf_cols);
 
     if (threadIdx.x == 0) {
@@ -204,7 +221,9 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_sfa = tmem + (uint32_t)NC1, tmem_sfb = tmem_sfa + 4u;  // F8 scale columns
+    // F8 scale columns: the weights' (FP8: one group of constant 1.0 bytes; FP4: one
+    // group per stage), then one group per stage for the activation planes
+    const uint32_t tmem_sfa = tmem + (uint32_t)NC1, tmem_sfb = tmem_sfa + (f4 ? 4u * (uint32_t)stages : 4u);
     // K split: every CTA of the cluster has started before any pushes into another's
     // shared memory (arrive now; the epilogue warps wait before their first push)
     if (split) cluster_arrive_relaxed();
@@ -215,8 +234,11 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
     // w % 4, each quarter of the MMA reading its own copy)
     auto copy_scales = [&] {
         const int q = warp & 3;
-        // the weights' block scales: 1.0 (UE8M0 127) in every byte
-        tmem_st4(tmem_sfa + ((uint32_t)(q * 32) << 16), 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        const uint32_t quarter = (uint32_t)(q * 32) << 16;
+        // FP8: the weights' block scales are 1.0 (UE8M0 127) in every byte.  FP4:
+        // A row 32q + lane of the stage takes its exponent word (loaded with the
+        // stage) at lane 32q + lane, column q of the stage's group
+        if (!f4) tmem_st4(tmem_sfa + quarter, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
         bool dead = false;
         for (int kk = 0; kk < nk; ++kk) {
             const int s = kk % stages;
@@ -225,7 +247,8 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
             uint32_t w4[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) w4[c] = (!dead && 32 * c + lane < F8_PLANES * TM) ? w[32 * c + lane] : 0x7F7F7F7Fu;
-            tmem_st4(tmem_sfb + (uint32_t)(s * 4) + ((uint32_t)(q * 32) << 16), w4[0], w4[1], w4[2], w4[3]);
+            if (f4) tmem_st1(tmem_sfa + (uint32_t)(s * 4 + q) + quarter, dead ? 0x7F7F7F7Fu : sE[s * 128 + q * 32 + lane]);
+            tmem_st4(tmem_sfb + (uint32_t)(s * 4) + quarter, w4[0], w4[1], w4[2], w4[3]);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             __syncwarp();
@@ -253,7 +276,22 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
                     tma_load_2d(b, &tmX, k, m0, &full[s]);
                 }
             };
-            const int a_tx = A_ST + B_ST + SW_ST;  // bytes completing full[]
+            // FP4: the exponent words of the tile's two 64-row halves (rows past the
+            // matrix are not copied; the host keeps the row count a multiple of 4)
+            int e_bytes0 = 0, e_bytes1 = 0;
+            if (f4) {
+                const int nt0 = tile0 % p.n_tiles, rows = p.swiglu_F ? 2 * p.swiglu_F : p.N;
+                const int r0 = p.swiglu_F ? nt0 * 64 : nt0 * 128, r1 = p.swiglu_F ? p.swiglu_F + nt0 * 64 : nt0 * 128 + 64;
+                e_bytes0 = 4 * max(0, min(64, rows - r0));
+                e_bytes1 = 4 * max(0, min(64, rows - r1));
+            }
+            // bytes completing full[] (FP4 codes: the packed bytes the copy reads)
+            const int a_tx = (f4 ? p.a_tx + e_bytes0 + e_bytes1 : A_ST) + B_ST + SW_ST;
+            auto load_e = [&](int s, int kblk, int rowA0, int rowA1) {
+                const uint32_t *src = p.w_bexp + (size_t)kblk * p.bs_rows + p.bs_row0;
+                if (e_bytes0) bulk_load(sE + s * 128, src + rowA0, (uint32_t)e_bytes0, &full[s]);
+                if (e_bytes1) bulk_load(sE + s * 128 + 64, src + rowA1, (uint32_t)e_bytes1, &full[s]);
+            };
             int it = 0;     // global stage counter
             bool first = true, abort = false;
             for (int t = tile0; t < n_tiles_total && !abort; t += tstride) {
@@ -270,6 +308,7 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
                         mbar_expect_tx(&full[i], a_tx);
                         tma_load_2d_hint(a, &tmW, (kb + i) * kstep, rowA0, &full[i], wpol);
                         tma_load_2d_hint(a + A_ST / 2, &tmW, (kb + i) * kstep, rowA1, &full[i], wpol);
+                        if (f4) load_e(i, kb + i, rowA0, rowA1);
                     }
                     if (!grouped) dep_wait(p.dep_ctr, p.dep_target, p.err);
                     for (int i = 0; i < pre; ++i) load_x(i, (kb + i) * kstep, m0);
@@ -288,6 +327,7 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
                     mbar_expect_tx(&full[s], a_tx);
                     tma_load_2d_hint(a, &tmW, k, rowA0, &full[s], wpol);
                     tma_load_2d_hint(a + A_ST / 2, &tmW, k, rowA1, &full[s], wpol);
+                    if (f4) load_e(s, kb + kk, rowA0, rowA1);
                     load_x(s, k, m0);
                 }
             }
@@ -315,10 +355,13 @@ __device__ __forceinline__ void gemm_tc_body(const CUtensorMap &tmW, const CUten
                         const uint64_t da = sw128_desc(smem_u32(sA + (size_t)s * A_ST));
                         const uint64_t db = sw128_desc(smem_u32(sB + (size_t)s * B_ST));
                         const uint32_t sfb = tmem_sfb + (uint32_t)(s * 4);
+                        const uint32_t sfa = f4 ? tmem_sfa + (uint32_t)(s * 4) : tmem_sfa;
+                        // A format: E4M3 (0) or, for FP4 weights, E2M1 (5), bits 7-9
+                        const uint32_t afmt = f4 ? (5u << 7) : 0u;
 #pragma unroll
                         for (int k32 = 0; k32 < 4; ++k32)  // 4 x K=32 over the stage's 128 K (+32 bytes each)
                             mma_mx(acc, da + (uint64_t)(k32 * 2), db + (uint64_t)(k32 * 2),
-                                   idesc_mx(F8_PLANES * TM, k32), tmem_sfa | ((uint32_t)k32 << 30),
+                                   idesc_mx(F8_PLANES * TM, k32) | afmt, sfa | ((uint32_t)k32 << 30),
                                    sfb | ((uint32_t)k32 << 30), (kk > 0 || k32 > 0) ? 1u : 0u);
                         mma_commit(&empty[s]);
                     } else {
@@ -692,6 +735,30 @@ const CUtensorMap *GemmTC<T>::tensor_map(const void *ptr, int rows, int cols, in
     return &(maps[key] = m);
 }
 
+template <typename T>
+const CUtensorMap *GemmTC<T>::fp4_map(const void *ptr, int rows, int cols, int box_rows) {
+    char key[96];
+    snprintf(key, sizeof key, "fp4/%p/%d/%d/%d", ptr, rows, cols, box_rows);
+    auto it = maps.find(key);
+    if (it != maps.end()) return &it->second;
+    if (maps.size() > 4096) maps.clear();
+    CUtensorMap m;
+    memset(&m, 0, sizeof m);
+    // dims count 4-bit elements; the row stride is in bytes (cols / 2)
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols / 2};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = get_encode()(&m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(ptr), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        err = "cuTensorMapEncodeTiled failed (FP4 weights)";
+        return nullptr;
+    }
+    return &(maps[key] = m);
+}
+
 // Tensor map of the MX activation planes of an M x K projection input:
 // (K bytes, M rows, planes), box {128 K, tm rows, planes}, 128-byte swizzle.
 // Rows >= M and columns >= K read as zero codes.
@@ -764,7 +831,7 @@ static void launch_kind(int kind, const CUtensorMap *mw, const CUtensorMap *mx, 
 }
 
 template <typename T>
-TcPlan GemmTC<T>::plan(int M, int N, int K, int kind, int F, bool f8, int planes) const {
+TcPlan GemmTC<T>::plan(int M, int N, int K, int kind, int F, bool f8, int planes, bool f4) const {
     const bool swiglu = kind == EPI_SWIGLU;
     TcPlan pl;
     int TM = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
@@ -787,7 +854,9 @@ TcPlan GemmTC<T>::plan(int M, int N, int K, int kind, int F, bool f8, int planes
     pl.k_steps = (K + pl.kstep - 1) / pl.kstep;
     const int tiles = pl.n_tiles * pl.m_tiles;
     // a stage: the weight tile + the activation tile(s) (FP8: codes + activation planes + scale words)
-    const int stage_bytes = f8 ? tc::F8_A_BYTES + tc::F8_PLANES * TM * (128 + 4) : tc::A_BYTES + TM * 128 * planes;
+    // (FP4: the same 16 KB of weight codes in shared memory, plus the 128 rows' exponent words)
+    const int stage_bytes = f8 ? tc::F8_A_BYTES + tc::F8_PLANES * TM * (128 + 4) + (f4 ? 512 : 0)
+                               : tc::A_BYTES + TM * 128 * planes;
     // fixed area: alignment, epilogue staging, barriers
     const int fixed = 1024 + 128 * tc::STG_LD * 4 + 4 * tc::CH * 8 + tc::CH * 16 + tc::RS_MAX * 4 + 64 * 8 + 64 + 16 * 8;
     // Measured on B200 (decode shapes, M = 16, whole decode iteration): every
@@ -822,10 +891,11 @@ TcPlan GemmTC<T>::plan(int M, int N, int K, int kind, int F, bool f8, int planes
 
 template <>
 int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K, const Epi<bf16> &e,
-                      cudaStream_t s, const int *dep_ctr, int dep_target, int *done_ctr, const float *w_scale) {
+                      cudaStream_t s, const int *dep_ctr, int dep_target, int *done_ctr, const float *w_scale,
+                      const uint8_t *w_bexp, int bs_rows, int bs_row0) {
     const bool swiglu = e.kind == EPI_SWIGLU;
     const bool f8 = w_scale != nullptr;
-    const TcPlan pl = plan(M, N, K, e.kind, e.F, f8, e.lo ? 2 : 1);
+    const TcPlan pl = plan(M, N, K, e.kind, e.F, f8, e.lo ? 2 : 1, f8 && w_bexp != nullptr);
     const int TM = pl.TM, splits = pl.splits, stages = pl.stages;
     const size_t smem = pl.smem;
     TcParams p;
@@ -839,6 +909,16 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     p.k_steps = pl.k_steps;
     p.planes = e.lo ? 2 : 1;
     p.w_scale = w_scale;
+    const bool f4 = f8 && w_bexp != nullptr;
+    if (f4) {
+        p.w_bexp = reinterpret_cast<const uint32_t *>(w_bexp);
+        p.bs_rows = bs_rows;
+        p.bs_row0 = bs_row0;
+        // a stage's codes complete the barrier with the bytes the copy reads (8 KB
+        // packed), not the 16 KB they fill in shared memory (measured on B200: with
+        // 16 KB the barrier never completed)
+        p.a_tx = tc::F8_A_BYTES / 2;
+    }
     p.splits = splits;
     p.err = err_word;
     p.lm_part = lm_part;
@@ -847,7 +927,13 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
     p.dep_target = dep_target;
     p.done_ctr = done_ctr;
     const int grid_x = p.n_tiles;  // one tile per CTA
-    const CUtensorMap *mw = tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64, 0, f8);
+    if (f4 && (K % 128 || ((swiglu ? 2 * e.F : N) % 4) || bs_rows % 4 || bs_row0 % 4 ||
+               (reinterpret_cast<uintptr_t>(W) & 31) || (reinterpret_cast<uintptr_t>(w_bexp) & 15))) {
+        failed = true;
+        err = "FP4 projection: K must be a multiple of 128, the row counts of 4, the codes 32-byte aligned";
+        return 0;
+    }
+    const CUtensorMap *mw = f4 ? fp4_map(W, swiglu ? 2 * e.F : N, K, 64) : tensor_map(W, swiglu ? 2 * e.F : N, K, K, 64, 0, f8);
     const CUtensorMap *mx = nullptr, *ms = nullptr;
     if (f8) {
         // the activation rows as MX planes (a kernel of their own, before the projection)
@@ -888,7 +974,7 @@ int GemmTC<bf16>::run(const bf16 *X, int ldx, int M, const void *W, int N, int K
 
 template <>
 int GemmTC<float>::run(const float *, int, int, const void *, int, int, const Epi<float> &, cudaStream_t,
-                       const int *, int, int *, const float *) {
+                       const int *, int, int *, const float *, const uint8_t *, int, int) {
     return 0;
 }
 

@@ -38,6 +38,12 @@ struct TcParams {
     int dep_target;
     int *done_ctr;
     const float *w_scale;   // FP8 weights: fp32 scale of every weight row (the codes' row of W)
+    // FP4 (MXFP4) weights (w_bexp != nullptr): W holds packed E2M1 codes; the
+    // exponent bytes of row r's 32-value blocks k/32 = 4j .. 4j+3 are the word
+    // w_bexp[j * bs_rows + bs_row0 + r] (UE8M0, byte b = block 4j + b)
+    const uint32_t *w_bexp;
+    int bs_rows, bs_row0;
+    int a_tx;               // FP4: bytes a weight stage's TMA completes (its shared-memory footprint)
     // grouped (MoE experts): blockIdx.y = touched-expert slot, blockIdx.z = row tile of
     // that expert; its rows are g_off[e] .. g_off[e+1]-1 of X (expert-grouped order) and
     // its weights rows e*g_wrows .. of W; nullptr g_off = an ordinary projection
@@ -59,10 +65,13 @@ struct GemmTC {
     int init(float *ws, int ws_floats, int *sem, int n_sem);
     // returns the number of CTAs launched (the count a completion counter reaches per run).
     // W: bf16 [N][K], or with w_scale != nullptr FP8 E4M3 codes [N][K] (one byte each)
-    // whose row n stands for w_scale[n] * code value.
+    // whose row n stands for w_scale[n] * code value, or with w_bexp != nullptr as
+    // well MXFP4 codes [N][K/2] (two E2M1 codes a byte, the low nibble first) whose
+    // element (n, k) stands for w_scale[n] * 2^(e - 127) * code value, e the byte
+    // (k / 32) % 4 of word (k / 128) * bs_rows + bs_row0 + n of w_bexp.
     int run(const T *X, int ldx, int M, const void *W, int N, int K, const Epi<T> &e, cudaStream_t s,
             const int *dep_ctr = nullptr, int dep_target = 0, int *done_ctr = nullptr,
-            const float *w_scale = nullptr);
+            const float *w_scale = nullptr, const uint8_t *w_bexp = nullptr, int bs_rows = 0, int bs_row0 = 0);
     // Grouped projection over the touched experts of a MoE layer: W is [E][wrows][K],
     // X the pair rows in expert-grouped order (off[E+1], touched[E] as bucketed),
     // at most max_rows rows per expert.  EPI_SWIGLU writes h in grouped order;
@@ -71,7 +80,7 @@ struct GemmTC {
                     const int *off, const int *touched, const int *list, int E, int max_rows, cudaStream_t s);
     // tiling of a launch of M activation rows (planes 1 or 2) against an N x K weight
     // matrix (SwiGLU: F output columns, N = 2F), bf16 or FP8
-    TcPlan plan(int M, int N, int K, int kind, int F, bool f8, int planes) const;
+    TcPlan plan(int M, int N, int K, int kind, int F, bool f8, int planes, bool f4 = false) const;
     // LM-head partial argmax buffer (value, index as float bits), [n_tiles][rows]
     void set_lm_part(float2 *p, int cap) { lm_part = p; lm_cap = cap; }
     void set_err(int *e) { err_word = e; }
@@ -100,6 +109,10 @@ struct GemmTC {
     // elements after it, box {64, box_rows, 2}
     const CUtensorMap *tensor_map(const void *ptr, int rows, int cols, int ld, int box_rows, size_t plane_stride = 0,
                                   bool fp8 = false);
+    // 2-D map of [rows][cols] packed E2M1 codes (cols / 2 bytes a row), box {128, box_rows}:
+    // each 16 codes (8 bytes) land in 16 bytes of shared memory, the layout the
+    // block-scaled MMA reads 4-bit elements in
+    const CUtensorMap *fp4_map(const void *ptr, int rows, int cols, int box_rows);
 };
 
 // Row-wise argmax over the LM-head partials: mode 0 idx[r]; mode 1 drafter rows.

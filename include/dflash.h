@@ -71,8 +71,18 @@ typedef enum {
  * activations as for BF16; the model computed is the quantised one,
  * W[r][k] = scale[r] * e4m3_value(code[r][k]), so the greedy output equals the
  * quantised target's own greedy decoding.  Weight bytes per step halve.
- * Dense models only (MoE targets: EINVAL). */
-enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1, DFLASH_BF16_FAST = 2, DFLASH_FP8 = 3 };
+ * FP4: the same matrices in MXFP4 (OCP Microscaling): 4-bit E2M1 codes, two per
+ * byte (element k of a row in byte k/2, the low nibble for even k; 1 sign, 2
+ * exponent bits with bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6), one power-of-two exponent per 32 values of a row in "<name>.bscale"
+ * [K/128][rows][4] (byte (k/128, r, (k/32) % 4) = exponent + 127, UE8M0) and
+ * one fp32 scale per row in "<name>.scale"; W[r][k] = scale[r] *
+ * 2^(bscale - 127) * e2m1_value(code[r][k]).  Weight bytes per step ~quarter.
+ * Every K (hidden, ffn, q width, n_taps * hidden) a multiple of 128.
+ * FP8 and FP4: dense models only (MoE targets: EINVAL). */
+enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1, DFLASH_BF16_FAST = 2, DFLASH_FP8 = 3, DFLASH_FP4 = 4 };
+/* Storage type of the "<name>.bscale" weight slots (dflash_weight_info): bytes. */
+enum { DFLASH_UE8M0 = 5 };
 
 /* Draft modes.  MODEL: drafts are the drafter's argmax.  SCRIPT: the drafter
  * still runs in full, then its drafts are replaced from a per-sequence token
@@ -113,7 +123,7 @@ typedef struct {
     int32_t max_batch;            /* sequences held at once */
     int32_t max_len;              /* positions per sequence (prompt + generated + B) */
     int32_t prefill_chunk;        /* prompt rows per prefill pass (0: default 1024) */
-    int32_t dtype;                /* DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST or DFLASH_FP8 (see above) */
+    int32_t dtype;                /* DFLASH_FP32, DFLASH_BF16, DFLASH_BF16_FAST, DFLASH_FP8 or DFLASH_FP4 (see above) */
     int32_t keep_logits;          /* 1: keep fp32 logits of the last draft/verify for dflash_debug_logits */
     int32_t timeout_ms;           /* host wait bound for synchronising calls (0: 600000) */
     int32_t sampling;             /* 1: hold the buffers temperature sampling needs (dflash_set_sampling);
@@ -171,7 +181,9 @@ const char *dflash_last_error(const dflash_ctx *ctx);
 
 /* Weight tensors: names, shapes, storage.  Tensors are row-major and live at
  * byte `offset` of the weight arena.  Matrices use cfg.dtype storage (FP8:
- * uint8 codes plus "<name>.scale" [rows] fp32; the embedding stays bf16),
+ * uint8 codes plus "<name>.scale" [rows] fp32; FP4: packed codes [rows][K/2]
+ * (slot type DFLASH_FP4), "<name>.bscale" [K/128][rows][4] (DFLASH_UE8M0) and
+ * "<name>.scale"; the embedding stays bf16),
  * RMSNorm gains are always fp32.  Names:
  *   embed [V,H], lm_head [V,H] (both shared by the drafter),
  *   {target|drafter}.L{l}.attn_norm [H], .wqkv [(nq+2nkv)*hd, H] (rows Wq;Wk;Wv),
