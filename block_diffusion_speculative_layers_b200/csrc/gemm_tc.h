@@ -43,7 +43,7 @@ struct TcParams {
     // w_bexp[j * bs_rows + bs_row0 + r] (UE8M0, byte b = block 4j + b)
     const uint32_t *w_bexp;
     int bs_rows, bs_row0;
-    int a_tx;               // FP4: bytes a weight stage's TMA completes (its shared-memory footprint)
+    int a_tx;               // FP4: bytes a weight stage's TMA completes (the packed bytes it reads)
     // grouped (MoE experts): blockIdx.y = touched-expert slot, blockIdx.z = row tile of
     // that expert; its rows are g_off[e] .. g_off[e+1]-1 of X (expert-grouped order) and
     // its weights rows e*g_wrows .. of W; nullptr g_off = an ordinary projection
