@@ -217,9 +217,11 @@ TRAFFIC = {
                            "down": 93.56e6, "lm_head": 1245.40e6, "fuse": 169.45e6},
     ("qwen3_8b", "fp8"): {"qkv": 25.66e6, "attention": 4.76e6, "o": 17.44e6, "gate_up": 101.51e6,
                           "down": 51.55e6, "lm_head": 623.53e6, "fuse": 85.49e6},
+    ("qwen3_8b", "fp4"): {"qkv": 13.86e6, "attention": 4.76e6, "o": 9.57e6, "gate_up": 53.94e6,
+                          "down": 27.96e6, "lm_head": 331.90e6, "fuse": 46.07e6},
 }
 TRAFFIC_SOURCE = ("profiles/traffic_per_shape_qwen3_8b_2layer.md (2-layer model, one cold launch each; "
-                  "FP8: the projection launch, without its mx_quantize_kernel)")
+                  "FP8 / FP4: the projection launch, without its mx_quantize_kernel)")
 
 SHAPES = ("qkv", "attention", "o", "gate_up", "down", "lm_head", "fuse")
 
