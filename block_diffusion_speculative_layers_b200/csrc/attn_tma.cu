@@ -620,14 +620,26 @@ bool attn_tma_make_map(CUtensorMap *map, const bf16 *cache, int hd, int max_len,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// q heads per CTA: one while the launch has fewer query tiles x kv heads than
-// SMs (decode of a few sequences: each q head's CTAs stream the kv head's K/V,
-// the copies after the first mostly from L2); the whole GQA group of a kv head
-// (up to 4 heads) once the tiles alone fill the GPU (prefill chunks, large
-// batches), so each K/V tile is read once for all of them
-int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms) {
-    if (n_tiles * nkv < num_sms) return 1;
-    return grp % 4 == 0 ? 4 : grp % 2 == 0 ? 2 : 1;
+// q heads per CTA.  Measured on B200 (Qwen3-8B shape: 32 q heads, 8 kv heads,
+// 16-row query tiles, ~530-key contexts; attention us per launch):
+//  - one query tile (batch 1): one q head per CTA, 8 key splits (16.8; the GQA
+//    group per CTA 18.8);
+//  - up to 64 (tile, kv head) pairs (batch 4, 8): the GQA group of 4 heads per
+//    CTA with the keys split to ~128 CTAs (batch 4: 37.3 -> 25.0, batch 8: 45.4
+//    -> 35.2 against one head per CTA);
+//  - more (batch 16, 32): 2 heads per CTA, no split (batch 16: 68.5 -> 51.3,
+//    batch 32 with 4 heads per CTA: 133.6 -> 104.4).
+// A prefill chunk (the tiles of one sequence, causal) keeps the GQA group per
+// CTA once its tiles fill the GPU (512-token prompt: 0.073 s against 0.105 s
+// with 2 heads per CTA).
+int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms, bool one_seq) {
+    if (n_tiles <= 1) return 1;
+    if (one_seq) {
+        if (n_tiles * nkv < num_sms) return 1;
+        return grp % 4 == 0 ? 4 : grp % 2 == 0 ? 2 : 1;
+    }
+    if (n_tiles * nkv <= 64 && grp % 4 == 0) return 4;
+    return grp % 2 == 0 ? 2 : 1;
 }
 // keys per tile: 16 when four key groups share the ring (its stages stay small),
 // 32 for one group
@@ -689,14 +701,19 @@ int launch_attention_tma(const AttnTmaMaps &maps, AttnTmaArgs a, int hd, bool sp
     const int grp = a.nq / a.nkv;
     const int n_tiles = (a.R + a.rows_per_tile - 1) / a.rows_per_tile;
     const AttnTune &tune = attn_tune();
-    int hpc = attn_tma_hpc(grp, n_tiles, a.nkv, num_sms);
+    int hpc = attn_tma_hpc(grp, n_tiles, a.nkv, num_sms, a.one_seq != 0);
     if ((tune.hpc == 1 || tune.hpc == 2 || tune.hpc == 4) && grp % tune.hpc == 0) hpc = tune.hpc;
     const int kt = attn_tma_kt(hpc);
     const CUtensorMap &mk = kt == 32 ? maps.k32 : maps.k16, &mv = kt == 32 ? maps.v32 : maps.v16;
     const int units = n_tiles * (a.nq / hpc);
-    // splits of one (tile, head group) form a cluster of at most 8 CTAs; enough
-    // CTAs for two per SM, no more splits than key tiles the longest context has
-    a.n_splits = std::max(1, std::min({8, (2 * num_sms + units - 1) / units, (a.max_len + kt - 1) / kt}));
+    // splits of one (tile, head group) form a cluster of at most 8 CTAs; no more
+    // splits than key tiles the longest context has.  One head per CTA: enough
+    // CTAs for two per SM; several query tiles: ~128 CTAs for the 4-head form,
+    // none for 2 heads (the measurements above)
+    const int want = (n_tiles <= 1 || hpc == 1 || a.one_seq) ? (2 * num_sms + units - 1) / units
+                     : hpc == 4                               ? 128 / units
+                                                              : 1;
+    a.n_splits = std::max(1, std::min({8, want, (a.max_len + kt - 1) / kt}));
     if (tune.splits > 0) a.n_splits = std::min({8, tune.splits, (a.max_len + kt - 1) / kt});
     a.stages = attn_tma_stages(hd, split, hpc, tune.rounds);
     cudaError_t e = cudaErrorInvalidValue;

@@ -17,6 +17,7 @@ struct AttnTmaArgs {
     const RowMeta *meta = nullptr;  // per row: sequence slot, position, visible keys nk
     int R = 0, rows_per_tile = 16, nq = 0, nkv = 0, max_len = 0;
     int n_seq = 0;                  // sequence slots of the K/V caches
+    int one_seq = 0;                // 1: every row is of one sequence (a prefill chunk)
     int layer = 0;                  // layer of the K/V maps
     float scale_log2 = 0.f;         // log2(e) / sqrt(hd)
     bf16 *out = nullptr;            // [R][ldo] (low plane lo elements on)
@@ -47,7 +48,7 @@ struct AttnTmaMaps {
 };
 
 // q heads per CTA and keys per tile the launcher picks (exposed for tests of the policy)
-int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms);
+int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms, bool one_seq);
 int attn_tma_kt(int hpc);
 
 // Launch on stream s; returns the CTAs launched, -1 if the launch failed.

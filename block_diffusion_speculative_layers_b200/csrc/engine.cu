@@ -648,6 +648,7 @@ class Engine : public EngineBase {
     }
 
     bool attn_failed = false;  // an attention launch was refused
+    bool attn_one_seq = false;  // the attention launches under way are one sequence's prefill chunk
     dflash_status check(const char *what) {
         if (tc.failed) {  // a projection could not be launched (tensor map encoding)
             err = std::string(what) + ": " + tc.err;
@@ -853,6 +854,7 @@ class Engine : public EngineBase {
                     a.nkv = m.n_kv_heads;
                     a.max_len = c.max_len;
                     a.n_seq = c.max_batch;
+                    a.one_seq = attn_one_seq ? 1 : 0;
                     a.layer = layer;
                     a.scale_log2 = 1.4426950408889634f / sqrtf((float)m.head_dim);
                     a.out = (bf16 *)out;
@@ -1390,7 +1392,9 @@ class Engine : public EngineBase {
         for (int c0 = 0; c0 < n; c0 += L.C) {
             const int R = std::min(L.C, n - c0);
             launch_embed_tokens<T>(embed, H, tokens + c0, R, seq, c0, x, meta, s);
+            attn_one_seq = true;
             for (int l = 0; l < t.n_layers; ++l) target_layer(l, R, 16, meta, taps_pre, TK);
+            attn_one_seq = false;
             if (c0 + R == n) {
                 // first token from the last prompt row: greedy, or the target's draw at position n
                 launch_rmsnorm<T>(x + (size_t)(R - 1) * H, H, t_final, H, (float)t.rms_eps, xn, H, lo_, 1, s);
