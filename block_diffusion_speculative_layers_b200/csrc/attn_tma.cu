@@ -629,12 +629,14 @@ bool attn_tma_make_map(CUtensorMap *map, const bf16 *cache, int hd, int max_len,
 //    -> 35.2 against one head per CTA);
 //  - more (batch 16, 32): 2 heads per CTA, no split (batch 16: 68.5 -> 51.3,
 //    batch 32 with 4 heads per CTA: 133.6 -> 104.4).
-// A prefill chunk (the tiles of one sequence, causal) keeps the GQA group per
-// CTA once its tiles fill the GPU (512-token prompt: 0.073 s against 0.105 s
-// with 2 heads per CTA).
+// Fewer than 4 query tiles (one or two sequences, blocks up to 32 rows) and
+// prefill chunks (the tiles of one sequence, causal) keep one q head per CTA
+// while the (tile, kv head) pairs do not fill the GPU, the GQA group per CTA
+// once they do (block 32 at batch 1: 30.8 us against 33.2 us with the group).
+static bool attn_tma_batched(int n_tiles, bool one_seq) { return !one_seq && n_tiles >= 4; }
+
 int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms, bool one_seq) {
-    if (n_tiles <= 1) return 1;
-    if (one_seq) {
+    if (!attn_tma_batched(n_tiles, one_seq)) {
         if (n_tiles * nkv < num_sms) return 1;
         return grp % 4 == 0 ? 4 : grp % 2 == 0 ? 2 : 1;
     }
@@ -707,12 +709,11 @@ int launch_attention_tma(const AttnTmaMaps &maps, AttnTmaArgs a, int hd, bool sp
     const CUtensorMap &mk = kt == 32 ? maps.k32 : maps.k16, &mv = kt == 32 ? maps.v32 : maps.v16;
     const int units = n_tiles * (a.nq / hpc);
     // splits of one (tile, head group) form a cluster of at most 8 CTAs; no more
-    // splits than key tiles the longest context has.  One head per CTA: enough
-    // CTAs for two per SM; several query tiles: ~128 CTAs for the 4-head form,
-    // none for 2 heads (the measurements above)
-    const int want = (n_tiles <= 1 || hpc == 1 || a.one_seq) ? (2 * num_sms + units - 1) / units
-                     : hpc == 4                               ? 128 / units
-                                                              : 1;
+    // splits than key tiles the longest context has.  Batched decode (the
+    // measurements above): ~128 CTAs for the 4-head form, no split for 2 heads;
+    // otherwise enough CTAs for two per SM
+    const bool batched = attn_tma_batched(n_tiles, a.one_seq != 0) && hpc != 1;
+    const int want = !batched ? (2 * num_sms + units - 1) / units : hpc == 4 ? 128 / units : 1;
     a.n_splits = std::max(1, std::min({8, want, (a.max_len + kt - 1) / kt}));
     if (tune.splits > 0) a.n_splits = std::min({8, tune.splits, (a.max_len + kt - 1) / kt});
     a.stages = attn_tma_stages(hd, split, hpc, tune.rounds);
