@@ -213,8 +213,8 @@ def cpu_oracle_sample(cfg, gpu_ctx=None, prompt_len: int = 16, iters: int = 1, s
 # for the kernel version in this tree.
 # Keyed by (config, weights): the Qwen3-8B shape at batch 1, block 16 only.
 TRAFFIC = {
-    ("qwen3_8b", "bf16"): {"qkv": 50.77e6, "attention": 4.76e6, "o": 34.18e6, "gate_up": 201.94e6,
-                           "down": 93.56e6, "lm_head": 1245.40e6, "fuse": 169.45e6},
+    ("qwen3_8b", "bf16"): {"qkv": 50.77e6, "attention": 4.76e6, "o": 34.18e6, "gate_up": 201.88e6,
+                           "down": 93.52e6, "lm_head": 1245.35e6, "fuse": 169.25e6},
     ("qwen3_8b", "fp8"): {"qkv": 25.66e6, "attention": 4.76e6, "o": 17.44e6, "gate_up": 101.51e6,
                           "down": 51.55e6, "lm_head": 623.53e6, "fuse": 85.49e6},
     ("qwen3_8b", "fp4"): {"qkv": 13.86e6, "attention": 4.76e6, "o": 9.57e6, "gate_up": 53.94e6,
