@@ -47,7 +47,8 @@ struct AttnTmaMaps {
     CUtensorMap k16, v16, k32, v32;
 };
 
-// q heads per CTA and keys per tile the launcher picks (exposed for tests of the policy)
+// q heads per CTA and keys per tile the launcher picks for n_tiles query tiles of
+// a GQA group size grp (one_seq: the tiles are one sequence's prefill chunk)
 int attn_tma_hpc(int grp, int n_tiles, int nkv, int num_sms, bool one_seq);
 int attn_tma_kt(int hpc);
 
