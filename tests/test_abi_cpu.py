@@ -132,3 +132,37 @@ def test_fidelity_toggles_reach_the_library():
     assert sizes(ok)[0] == dfl.DFLASH_OK
     bad = base.with_(target=replace(base.target, rope_scaling=(8.0, 4.0, 1.0, 256.0)))
     assert sizes(bad)[0] == dfl.DFLASH_EINVAL
+
+
+def test_quantised_weight_storage_sizes():
+    """FP8 and FP4 weight arenas hold what the header describes: the stored bytes
+    of every slot synthetic.weights lays out (FP4: codes two per byte, a block
+    exponent byte per 32 values, an fp32 scale per row), each slot 256-byte
+    aligned; at the Qwen3-8B shape the quantised arenas shrink accordingly; FP4
+    refuses widths off the 128 grid and MoE targets."""
+    import numpy as np
+    from synthetic.weights import weight_shapes
+    tiny = get_config("tiny")
+    sizes = {}
+    for dt in ("bf16", "fp8", "fp4"):
+        cfg = tiny.with_(dtype=dt)
+        st, wb, _ = _sizes(cfg, max_batch=1, max_len=128)
+        assert st == dfl.DFLASH_OK, dt
+        stored = 0
+        for shape, kind in weight_shapes(cfg).values():
+            es = {"norm": 4, "scale": 4, "matrix": 2, "fp8": 1, "fp4": 1, "bscale": 1}[kind]
+            stored += int(np.prod(shape)) * es
+        n_slots = len(weight_shapes(cfg))
+        assert stored <= wb <= stored + 256 * n_slots, dt
+        sizes[dt] = wb
+    assert sizes["fp4"] < sizes["fp8"] < sizes["bf16"]
+    q = {dt: _sizes(get_config("qwen3_8b").with_(dtype=dt), max_batch=1, max_len=3000)[1] for dt in ("fp8", "fp4")}
+    # every matrix but the embedding: 1 byte (FP8) or 0.5 + 1/32 byte (FP4) per weight; the embedding stays bf16
+    emb = 151936 * 4096 * 2
+    assert 8.5e9 < q["fp8"] - emb < 8.8e9  # LM head 0.62 GB + 41 layers x 0.19 GB + fuse
+    assert 0.5 * (q["fp8"] - emb) < q["fp4"] - emb < 0.56 * (q["fp8"] - emb)
+    off_grid = tiny.with_(dtype="fp4", target=replace(tiny.target, hidden=192, ffn=576),
+                          drafter=replace(tiny.drafter, hidden=192, ffn=576))
+    assert _sizes(off_grid, max_batch=1, max_len=128)[0] == dfl.DFLASH_EINVAL
+    moe = tiny.with_(dtype="fp4", target=replace(tiny.target, n_experts=8, top_k=2, expert_ffn=128))
+    assert _sizes(moe, max_batch=1, max_len=128)[0] == dfl.DFLASH_EINVAL
